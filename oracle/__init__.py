@@ -1,0 +1,261 @@
+"""CPU oracle for the int8-frozen-kernel LoRA Dense layer.
+
+TEST INFRASTRUCTURE ONLY.  This package is imported by ``tests/``, by
+``__graft_entry__.smoke()`` and by the CPU-baseline leg of ``bench.py``; the
+product path (``lora_fine_tuning_qlora_b200``) never imports, links or calls
+it, and it never imports the product.  The arithmetic lives in the plain C
+file ``qlora_oracle.c`` next to this module (scalar loops, fp64 sums, fp32
+quantization); this module only marshals numpy arrays into it, plus the
+composition of layers into the MLP stack workload (a plain ReLU between
+layers).
+
+What each routine follows (page title, section):
+  * quantize_weight / quantize_rows -- "Introduce QLoRA-like technique"
+    (Keras PR 19356), Highlights: frozen int8 kernel; the quantizer itself
+    (symmetric abs-max, scale amax/127, round half to even, fp32) is the
+    reading stated in the C file's header, since the pages give no formula.
+  * int8_matmul / forward -- same page, Results (int8 Dense); "Parameter-
+    efficient fine-tuning of GPT-2 with LoRA", "LoRA equation" and "Create
+    LoRA layer" (scale alpha / rank).
+  * backward -- gradients reach only the LoRA factors, the int8 kernel is
+    frozen ("How to fine-tune the 4-bit model?" thread); straight-through
+    through the input quantizer.
+  * merge -- Keras PR 19356 Results footnote (lossy merge) and the 4-bit
+    thread (de-quantize, add the LoRA, re-quantize).
+
+Pins: every routine here is checked by ``tests/test_oracle_pins.py`` against
+closed forms, brute force, finite differences and printed values (see
+``tests/golden/``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "qlora_oracle.c")
+_SO = os.path.join(_HERE, "liboracle.so")
+_LOCK = threading.Lock()
+_LIB = None
+
+_CFLAGS = ["-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
+           "-shared", "-std=c11"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle into ``liboracle.so`` (gcc).  Returns its path."""
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        tmp = _SO + ".tmp.%d" % os.getpid()
+        subprocess.check_call(["gcc", *_CFLAGS, _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _SO)
+    return _SO
+
+
+def _lib():
+    global _LIB
+    with _LOCK:
+        if _LIB is None:
+            build()
+            lib = ctypes.CDLL(_SO)
+            P = ctypes.c_void_p
+            L = ctypes.c_long
+            D = ctypes.c_double
+            F = ctypes.c_float
+            lib.orc_set_threads.argtypes = [ctypes.c_int]
+            lib.orc_get_threads.restype = ctypes.c_int
+            lib.orc_quantize_weight.argtypes = [P, L, L, P, P]
+            lib.orc_quantize_rows.argtypes = [P, L, L, P, P]
+            lib.orc_int8_matmul.argtypes = [P, P, L, L, L, P]
+            lib.orc_int8_matmul.restype = L
+            lib.orc_lora_down.argtypes = [P, P, L, L, L, P]
+            lib.orc_forward.argtypes = [L, L, L, D, P, P, P, P, P, P, P]
+            lib.orc_backward.argtypes = [L, L, L, L, D, P, P, P, P, P, P,
+                                         P, P, P, P, P]
+            lib.orc_merge.argtypes = [P, P, P, P, L, L, L, F, P, P]
+            lib.orc_round_bf16.argtypes = [D]
+            lib.orc_round_bf16.restype = D
+            lib.orc_round_bf16_array.argtypes = [P, L, P]
+            _LIB = lib
+    return _LIB
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def set_threads(n: int) -> None:
+    _lib().orc_set_threads(int(n))
+
+
+def get_threads() -> int:
+    return int(_lib().orc_get_threads())
+
+
+# --------------------------------------------------------------------------
+# quantizers
+# --------------------------------------------------------------------------
+def quantize_weight(W):
+    """W [K,N] float32 -> (Wq [N,K] int8, sw [N] float32), per output channel."""
+    W = _c(W, np.float32)
+    K, N = W.shape
+    Wq = np.empty((N, K), np.int8)
+    sw = np.empty((N,), np.float32)
+    _lib().orc_quantize_weight(_p(W), K, N, _p(Wq), _p(sw))
+    return Wq, sw
+
+
+def quantize_rows(X):
+    """X [M,K] float32 -> (Xq [M,K] int8, sx [M] float32), per row."""
+    X = _c(X, np.float32)
+    M, K = X.shape
+    Xq = np.empty((M, K), np.int8)
+    sx = np.empty((M,), np.float32)
+    _lib().orc_quantize_rows(_p(X), M, K, _p(Xq), _p(sx))
+    return Xq, sx
+
+
+def int8_matmul(Xq, Wq):
+    """acc[m,n] = sum_k Xq[m,k] Wq[n,k] in int64; raises if it leaves int32."""
+    Xq = _c(Xq, np.int8)
+    Wq = _c(Wq, np.int8)
+    M, K = Xq.shape
+    N, K2 = Wq.shape
+    if K != K2:
+        raise ValueError("inner sizes differ")
+    acc = np.empty((M, N), np.int32)
+    bad = _lib().orc_int8_matmul(_p(Xq), _p(Wq), M, N, K, _p(acc))
+    if bad:
+        raise OverflowError("%d accumulator entries leave the int32 range" % bad)
+    return acc
+
+
+# --------------------------------------------------------------------------
+# layer
+# --------------------------------------------------------------------------
+def lora_down(X, A):
+    X = _c(X, np.float64)
+    A = _c(A, np.float64)
+    M, K = X.shape
+    r = A.shape[1]
+    xA = np.empty((M, r), np.float64)
+    _lib().orc_lora_down(_p(X), _p(A), M, K, r, _p(xA))
+    return xA
+
+
+def forward(X, Wq, sw, bias, A, B, alpha):
+    """One int8-LoRA Dense forward.
+
+    X holds exactly the values the layer sees (fp32, or bf16 widened).
+    Returns a dict with the quantized input ``xq``/``sx``, the int32
+    accumulator ``acc``, the LoRA down-projection ``xA`` and the fp64
+    output ``y``.
+    """
+    X32 = _c(X, np.float32)
+    M, K = X32.shape
+    N = Wq.shape[0]
+    r = A.shape[1]
+    c = float(alpha) / float(r)
+    Xq, sx = quantize_rows(X32)
+    acc = int8_matmul(Xq, Wq)
+    xA = lora_down(X32, A)
+    Bd = _c(B, np.float64)
+    bd = None if bias is None else _c(bias, np.float64)
+    sw = _c(sw, np.float32)
+    Y = np.empty((M, N), np.float64)
+    _lib().orc_forward(M, N, r, c, _p(acc), _p(sx), _p(sw), _p(bd), _p(xA),
+                       _p(Bd), _p(Y))
+    return {"xq": Xq, "sx": sx, "acc": acc, "xA": xA, "y": Y}
+
+
+def backward(X, dY, Wq, sw, A, B, alpha, want_dx=True):
+    """One int8-LoRA Dense backward; returns dict G, dX, dA, dB, dbias (fp64)."""
+    Xd = _c(X, np.float64)
+    dYd = _c(dY, np.float64)
+    M, K = Xd.shape
+    N = dYd.shape[1]
+    r = A.shape[1]
+    c = float(alpha) / float(r)
+    Ad = _c(A, np.float64)
+    Bd = _c(B, np.float64)
+    Wq = _c(Wq, np.int8)
+    sw = _c(sw, np.float32)
+    G = np.empty((M, r), np.float64)
+    dX = np.empty((M, K), np.float64) if want_dx else None
+    dA = np.empty((K, r), np.float64)
+    dB = np.empty((r, N), np.float64)
+    db = np.empty((N,), np.float64)
+    _lib().orc_backward(M, K, N, r, c, _p(Xd), _p(dYd), _p(Wq), _p(sw), _p(Ad),
+                        _p(Bd), _p(G), _p(dX), _p(dA), _p(dB), _p(db))
+    return {"G": G, "dX": dX, "dA": dA, "dB": dB, "dbias": db}
+
+
+def merge(Wq, sw, A, B, alpha):
+    """Lossy merge (fp32, fixed order) -> (Wq' [N,K] int8, sw' [N] float32)."""
+    Wq = _c(Wq, np.int8)
+    sw = _c(sw, np.float32)
+    A = _c(A, np.float32)
+    B = _c(B, np.float32)
+    N, K = Wq.shape
+    r = A.shape[1]
+    c = np.float32(np.float32(alpha) / np.float32(r))
+    Wq2 = np.empty_like(Wq)
+    sw2 = np.empty_like(sw)
+    _lib().orc_merge(_p(Wq), _p(sw), _p(A), _p(B), K, N, r, float(c), _p(Wq2), _p(sw2))
+    return Wq2, sw2
+
+
+def round_bf16(x):
+    """Round fp64 values to the nearest bfloat16 (ties to even), as fp64."""
+    x = _c(x, np.float64)
+    y = np.empty_like(x)
+    _lib().orc_round_bf16_array(_p(x), x.size, _p(y))
+    return y
+
+
+def to_act(y, act_dtype):
+    """Store an fp64 result in the activation dtype ("f32" or "bf16"), as fp64."""
+    if act_dtype == "bf16":
+        return round_bf16(y)
+    return np.asarray(y, np.float32).astype(np.float64)
+
+
+# --------------------------------------------------------------------------
+# the MLP stack workload: Dense layers with a plain ReLU between them
+# --------------------------------------------------------------------------
+def mlp_stack(X, layers, dY, act_dtype):
+    """Forward and backward through a stack of int8-LoRA Dense layers.
+
+    ``layers`` is a list of dicts with Wq, sw, bias, A, B, alpha.  Every
+    layer output is stored in ``act_dtype``; a ReLU follows every layer but
+    the last.  ``dY`` is the gradient of the last layer's output.  Returns
+    the final output, the gradient of the stack input, and per-layer dA/dB.
+    """
+    h = to_act(np.asarray(X, np.float64), act_dtype)
+    inputs, pre = [], []
+    n = len(layers)
+    for i, L in enumerate(layers):
+        inputs.append(h)
+        out = forward(h, L["Wq"], L["sw"], L["bias"], L["A"], L["B"], L["alpha"])
+        y = to_act(out["y"], act_dtype)
+        pre.append(y)
+        h = np.maximum(y, 0.0) if i < n - 1 else y
+    y_final = h
+    g = to_act(np.asarray(dY, np.float64), act_dtype)
+    grads = [None] * n
+    for i in range(n - 1, -1, -1):
+        L = layers[i]
+        if i < n - 1:
+            g = np.where(pre[i] > 0.0, g, 0.0)
+        b = backward(inputs[i], g, L["Wq"], L["sw"], L["A"], L["B"], L["alpha"],
+                     want_dx=True)
+        grads[i] = {"dA": b["dA"], "dB": b["dB"], "dbias": b["dbias"]}
+        g = to_act(b["dX"], act_dtype)
+    return {"y": y_final, "dX": g, "grads": grads, "inputs": inputs, "pre": pre}
