@@ -1,0 +1,225 @@
+/*
+ * qlora.h -- C ABI of the int8-frozen-kernel LoRA Dense layer library
+ * (libqlora.so), sm_100a.
+ *
+ * The layer: a Dense layer whose kernel is frozen int8 with one fp32 scale
+ * per output channel, fine-tuned through a floating-point LoRA adapter
+ * ("Introduce QLoRA-like technique", Keras PR 19356, Highlights: training
+ * with frozen int8 weights for Dense; "Parameter-efficient fine-tuning of
+ * GPT-2 with LoRA", section "LoRA equation": output = W0 x + b0 + B A x,
+ * scaled by alpha / rank as in section "Create LoRA layer").
+ *
+ * Shapes and names (all buffers row-major and contiguous):
+ *   M tokens, K in_features, N out_features, r LoRA rank, c = alpha / r
+ *   W  [K,N]  fp32 float kernel (input of qlora_quantize_weight only)
+ *   Wq [N,K]  int8 frozen kernel, one row per output channel (K-major)
+ *   sw [N]    fp32 per-output-channel scale
+ *   X  [M,K]  activations in act_dtype          Y  [M,N] act_dtype
+ *   dY [M,N]  act_dtype                          dX [M,K] act_dtype
+ *   A  [K,r]  fp32    B [r,N] fp32    bias [N] fp32
+ *   xA [M,r]  fp32 (x . A of the unquantized input, kept for the backward)
+ *   dA [K,r], dB [r,N], dbias [N]  fp32
+ *
+ * Quantization (the pages give no formula; this is the library's reading):
+ * symmetric abs-max, s = amax / 127, q = clamp(rne(v * (127 / amax)), -127,
+ * 127), IEEE fp32, one rounding per operation; amax == 0 gives q = 0, s = 0.
+ *
+ * Memory and ownership: every pointer argument is a DEVICE pointer owned by
+ * the caller, except `d` and `dbg`, which are host pointers read during the
+ * call.  The library allocates no device memory.  Scratch space is the
+ * caller's `workspace` of at least qlora_workspace_bytes(d, M) bytes, 256-byte
+ * aligned; its contents on entry do not matter.
+ *
+ * Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
+ * Every call only enqueues work on `stream` and returns; QLORA_OK means the
+ * launches were enqueued.  Device-side failures surface at the caller's next
+ * synchronisation (cudaGetLastError) or through qlora_device_status().
+ * Calls on the same stream are ordered; calls that share an output or a
+ * workspace must not run concurrently on different streams.
+ *
+ * Errors: every call validates its arguments before launching anything and
+ * then returns a negative qlora_status without touching any output.  The
+ * checks are: non-NULL required pointers (EINVAL), M, K, N >= 1 and
+ * 1 <= r <= 64 (ESHAPE), K a multiple of 16 (EUNSUPPORTED: the int8 rows are
+ * moved by the Tensor Memory Accelerator, whose row pitch must be a multiple
+ * of 16 bytes), 16-byte aligned pointers for X, Y, dY, dX, Wq, Wq_out and
+ * the workspace, and 4-byte aligned fp32 vectors (EALIGN).  A CUDA error while
+ * enqueuing returns ECUDA.  qlora_last_error() gives a message for the last
+ * non-OK status of the calling thread.
+ */
+#ifndef QLORA_H
+#define QLORA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QLORA_F32 = 0,
+    QLORA_BF16 = 1
+} qlora_dtype;
+
+typedef enum {
+    QLORA_OK = 0,
+    QLORA_EINVAL = -1,
+    QLORA_EALIGN = -2,
+    QLORA_ESHAPE = -3,
+    QLORA_ECUDA = -4,
+    QLORA_EUNSUPPORTED = -5,
+    QLORA_ETIMEOUT = -6
+} qlora_status;
+
+/* One layer: in_features K, out_features N, rank r (1..64), LoRA alpha and
+ * the activation dtype of X, Y, dY and dX. */
+typedef struct {
+    int K;
+    int N;
+    int r;
+    float alpha;
+    qlora_dtype act_dtype;
+} qlora_layer_desc;
+
+/* Optional debug outputs of qlora_forward (any member may be NULL): the
+ * quantized input Xq [M,K] int8, its row scales sx [M] fp32 and the int32
+ * accumulator acc [M,N] of the int8 GEMM. */
+typedef struct {
+    int8_t* xq;
+    float* sx;
+    int32_t* acc;
+} qlora_debug;
+
+/*
+ * Frozen-kernel quantization, once per layer ("Introduce QLoRA-like
+ * technique", Highlights and the model.quantize("int8") call of its
+ * benchmark script): W [K,N] fp32 -> Wq [N,K] int8 (transposed so that
+ * each output channel's K values are contiguous) and sw [N] fp32, abs-max
+ * per output channel n.  Wq and sw are bit-exact with the reading above.
+ */
+int qlora_quantize_weight(const float* W, int K, int N, int8_t* Wq, float* sw,
+                          void* stream);
+
+/* Bytes of scratch that qlora_forward and qlora_backward need for M tokens
+ * (the same workspace serves both).  Returns 0 for an invalid descriptor. */
+size_t qlora_workspace_bytes(const qlora_layer_desc* d, int M);
+
+/*
+ * Forward: Y = (Xq Wq^T) * sx[m] * sw[n] + bias[n] + c * (X A) B.
+ * The int8 GEMM (int32 accumulate) follows "Introduce QLoRA-like technique"
+ * (Results table, int8 Dense); the LoRA term follows "Parameter-efficient
+ * fine-tuning of GPT-2 with LoRA", section "LoRA equation".  Each input row
+ * is quantized by abs-max (Xq, sx); the LoRA branch uses the unquantized X.
+ * bias may be NULL.  xA [M,r] receives X . A (needed by qlora_backward).
+ * dbg may be NULL; its non-NULL members receive Xq, sx and the int32
+ * accumulator.  Y must not alias X.
+ */
+int qlora_forward(const qlora_layer_desc* d, int M, const void* X, const int8_t* Wq,
+                  const float* sw, const float* bias, const float* A, const float* B,
+                  void* Y, float* xA, void* workspace, size_t workspace_bytes,
+                  const qlora_debug* dbg, void* stream);
+
+/*
+ * Backward of L with upstream gradient dY: the frozen int8 kernel receives
+ * no gradient ("How to fine-tune the 4-bit model?" thread: the integer
+ * weights are not changed during gradient descent), the input quantizer is
+ * passed straight through:
+ *   G  = dY B^T                                  [M,r]
+ *   dX = dY (Wq * sw)^T + c * G A^T              [M,K]  (may be NULL)
+ *   dA = c * X^T G                               [K,r]
+ *   dB = c * xA^T dY                             [r,N]
+ *   dbias = sum over rows of dY                  [N]    (may be NULL)
+ * xA must be the one qlora_forward returned for this X.  In bf16 the
+ * dequantized kernel Wq * sw is rounded to bf16 before the tensor-core
+ * product; accumulation is fp32.  dA, dB and dbias are deterministic
+ * (fixed reduction order, no atomics).
+ */
+int qlora_backward(const qlora_layer_desc* d, int M, const void* X, const void* dY,
+                   const int8_t* Wq, const float* sw, const float* A, const float* B,
+                   const float* xA, void* dX, float* dA, float* dB, float* dbias,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Step-level entry points.  qlora_forward is qlora_quantize_input followed
+ * by qlora_gemm_forward; qlora_backward is qlora_lora_grad_dy, then
+ * qlora_gemm_dx, then qlora_lora_grad_x.  They are exported so that a caller
+ * can schedule, overlap or time the steps one by one.  Same conventions as
+ * above; M == 0 is a no-op (the gradient steps then write zeros).
+ * ------------------------------------------------------------------------ */
+
+/* a1: per-row abs-max quantization of X into Xq [M,K] int8 and sx [M] fp32
+ * (bit-exact with the reading above), and xA = X . A [M,r] fp32 from the
+ * same read of X ("LoRA equation": the adapter sees the layer input). */
+int qlora_quantize_input(const qlora_layer_desc* d, int M, const void* X, const float* A,
+                         int8_t* Xq, float* sx, float* xA, void* stream);
+
+/* a2: Y = (Xq Wq^T) * sx[m] * sw[n] + bias[n] + c * xA B on the int8 tensor
+ * cores (int32 accumulate).  bias and acc may be NULL; a non-NULL acc
+ * [M,N] int32 receives the raw accumulator. */
+int qlora_gemm_forward(const qlora_layer_desc* d, int M, const int8_t* Xq, const float* sx,
+                       const int8_t* Wq, const float* sw, const float* bias, const float* xA,
+                       const float* B, void* Y, int32_t* acc, void* stream);
+
+/* a3: one pass over dY: G = dY B^T [M,r], dB = c * xA^T dY [r,N] and, if
+ * dbias is not NULL, dbias = column sums of dY [N].  Deterministic.  Needs
+ * the workspace (qlora_workspace_bytes) for its partial sums. */
+int qlora_lora_grad_dy(const qlora_layer_desc* d, int M, const void* dY, const float* B,
+                       const float* xA, float* G, float* dB, float* dbias, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* a4: dX = dY (Wq * sw)^T + c * G A^T [M,K]; the int8 kernel is de-quantized
+ * tile by tile in shared memory ("How to fine-tune the 4-bit model?":
+ * de-quantize in place before the matrix unit). */
+int qlora_gemm_dx(const qlora_layer_desc* d, int M, const void* dY, const int8_t* Wq,
+                  const float* sw, const float* G, const float* A, void* dX, void* stream);
+
+/* a5: one pass over X: dA = c * X^T G [K,r].  Deterministic.  Needs the
+ * workspace for its partial sums. */
+int qlora_lora_grad_x(const qlora_layer_desc* d, int M, const void* X, const float* G, float* dA,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Lossy merge ("Introduce QLoRA-like technique", Results footnote: merging
+ * LoRA weights into int8 kernels is lossy; "How to fine-tune the 4-bit
+ * model?" thread: de-quantize, add the LoRA, re-quantize; the float merge
+ * adds einsum(A, B) * alpha / rank, "Merge weights and generate text!"):
+ *   W'[k,n] = fl(fl(Wq[n,k] * sw[n]) + fl(c * d)),
+ *   d = A[k,0]*B[0,n] + ... + A[k,r-1]*B[r-1,n] summed in ascending j,
+ * every operation a single fp32 rounding, then the per-output-channel
+ * quantization of W' into Wq_out [N,K] and sw_out [N].  Bit-exact with that
+ * order.  Wq_out and sw_out must not alias Wq and sw.
+ */
+int qlora_merge(const qlora_layer_desc* d, const int8_t* Wq, const float* sw,
+                const float* A, const float* B, int8_t* Wq_out, float* sw_out,
+                void* stream);
+
+/*
+ * The plain elementwise ReLU between the Dense layers of the MNIST MLP
+ * ("Introduce QLoRA-like technique", benchmark.py: Dense + ReLU blocks).
+ * Not part of the layer.  qlora_relu: Y[i] = max(Y[i], 0) in place, n
+ * elements of `dtype`.  qlora_relu_backward: dY[i] = 0 where Y[i] <= 0 (Y is
+ * the ReLU output), in place.  Device pointers; n == 0 is a no-op.
+ */
+int qlora_relu(void* Y, size_t n, qlora_dtype dtype, void* stream);
+int qlora_relu_backward(void* dY, const void* Y, size_t n, qlora_dtype dtype, void* stream);
+
+/* Message for the last non-OK status returned on the calling thread. */
+const char* qlora_last_error(void);
+
+/*
+ * Synchronises `stream`, then reads and clears the library's device status
+ * word on the current device: QLORA_OK, or QLORA_ETIMEOUT if a kernel gave up
+ * a bounded wait (its outputs are then unspecified), or QLORA_ECUDA if the
+ * synchronisation itself failed.
+ */
+int qlora_device_status(void* stream);
+
+/* Library version, e.g. "qlora-b200 0.1 sm_100a". */
+const char* qlora_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_H */

@@ -1,0 +1,87 @@
+// internal.h -- launchers shared between the kernel files and the C ABI
+// (qlora_api.cu).  Nothing here is exported from libqlora.so.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace qlora {
+
+enum Act { kF32 = 0, kBF16 = 1 };
+
+// ---------------------------------------------------------------- K1 / a0
+// Xq, sx (bit-exact quantization) and xA = X . A, one pass over X.
+cudaError_t launch_quantize_rows(Act act, const void* X, const float* A, int M, int K, int r,
+                                 int8_t* Xq, float* sx, float* xA, cudaStream_t s);
+// W [K,N] fp32 -> Wq [N,K], sw [N].
+cudaError_t launch_quantize_weight(const float* W, int K, int N, int8_t* Wq, float* sw,
+                                   cudaStream_t s);
+
+// ---------------------------------------------------------------- K2
+struct FwdEpilogue {
+    const float* sx;    // [M]
+    const float* sw;    // [N]
+    const float* bias;  // [N] or null
+    const float* xA;    // [M,r]
+    const float* B;     // [r,N]
+    int r;
+    float c;
+    void* Y;            // [M,N] act
+    int32_t* acc;       // [M,N] debug copy or null
+};
+// Y = (Xq Wq^T) sx sw + bias + c xA B with the tcgen05 int8 GEMM.
+cudaError_t launch_gemm_i8_fwd(Act act, const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
+                               const FwdEpilogue& ep, int* status, cudaStream_t s);
+
+// ---------------------------------------------------------------- K3
+struct DxEpilogue {
+    const float* G;   // [M,r]
+    const float* A;   // [K,r]
+    int r;
+    float c;
+    void* dX;         // [M,K] act
+};
+// dX = dY (Wq sw)^T + c G A^T.  tcgen05 bf16 path when possible, else SIMT.
+cudaError_t launch_gemm_dx(Act act, const void* dY, const int8_t* Wq, const float* sw, int M,
+                           int N, int K, const DxEpilogue& ep, int* status, cudaStream_t s);
+
+// ---------------------------------------------------------------- K4
+struct RankPlan {
+    int rows_per_chunk;  // RM
+    int n_chunks;        // ceil(M / RM)
+    int n_col_blocks;    // ceil(N / 256), G partial slices
+    int k_chunks;        // chunks for the pass over X
+    int rows_per_kchunk;
+};
+RankPlan plan_rank(int M, int K, int N, int r);
+size_t rank_workspace_floats(const RankPlan& p, int M, int K, int N, int r);
+
+// Pass over dY: G, dB, dbias (with its deterministic reductions) and the
+// pass over X: dA.  `wsf` is fp32 scratch of rank_workspace_floats() floats.
+cudaError_t launch_rank_dy(Act act, const void* dY, const float* B, const float* xA, int M, int N,
+                           int r, float c, const RankPlan& p, float* G, float* dB, float* dbias,
+                           float* wsf, cudaStream_t s);
+cudaError_t launch_rank_x(Act act, const void* X, const float* G, int M, int K, int r, float c,
+                          const RankPlan& p, float* dA, float* wsf, cudaStream_t s);
+
+// ---------------------------------------------------------------- KM
+cudaError_t launch_merge(const int8_t* Wq, const float* sw, const float* A, const float* B, int K,
+                         int N, int r, float c, int8_t* Wq_out, float* sw_out, cudaStream_t s);
+
+// ---------------------------------------------------------------- ReLU
+cudaError_t launch_relu(Act act, void* y, size_t n, cudaStream_t s);
+cudaError_t launch_relu_backward(Act act, void* g, const void* h, size_t n, cudaStream_t s);
+
+// ---------------------------------------------------------------- TMA maps
+// Encodes a 2D row-major tensor map: `rows` x `cols` elements of `elem`
+// bytes, row pitch `pitch_bytes`, box `box_rows` x `box_cols`.
+bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem_bytes,
+                  uint64_t rows, uint64_t cols, uint64_t pitch_bytes, uint32_t box_rows,
+                  uint32_t box_cols, CUtensorMapSwizzle swizzle);
+
+// Sets the dynamic shared memory limit of `func` once per device.
+cudaError_t ensure_smem_attr(const void* func, int bytes);
+
+}  // namespace qlora

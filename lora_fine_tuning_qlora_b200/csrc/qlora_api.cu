@@ -1,0 +1,404 @@
+// qlora_api.cu -- the C ABI of libqlora.so (declared in include/qlora.h):
+// argument validation, workspace layout, tensor-map encoding and the launch
+// sequence of each call.  No device memory is allocated here.
+#include <mutex>
+#include <set>
+#include <string>
+#include <utility>
+
+#include "../../include/qlora.h"
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace qlora {
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const std::string& msg) {
+    g_last_error = msg;
+    return code;
+}
+
+// Device status word (one per device context): kernels record a timed-out
+// bounded wait here; qlora_device_status() reads and clears it.
+__device__ int g_device_status;
+
+std::mutex g_mu;
+int* g_status_ptr[64] = {nullptr};
+
+int* status_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_status_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+        g_status_ptr[dev] = static_cast<int*>(p);
+    }
+    return g_status_ptr[dev];
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct WsLayout {
+    size_t xq, sx, fwd_total;
+    size_t g, part, bwd_total;
+    size_t total;
+    RankPlan plan;
+};
+
+WsLayout layout_for(const qlora_layer_desc& d, int M) {
+    WsLayout w{};
+    w.xq = 0;
+    w.sx = align256(static_cast<size_t>(M) * d.K);
+    w.fwd_total = w.sx + align256(static_cast<size_t>(M) * 4);
+    w.plan = plan_rank(M, d.K, d.N, d.r);
+    w.g = 0;
+    w.part = align256(static_cast<size_t>(M) * d.r * 4);
+    w.bwd_total = w.part + align256(rank_workspace_floats(w.plan, M, d.K, d.N, d.r) * 4);
+    w.total = w.fwd_total > w.bwd_total ? w.fwd_total : w.bwd_total;
+    return w;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_desc(const qlora_layer_desc* d) {
+    if (!d) return fail(QLORA_EINVAL, "layer descriptor is NULL");
+    if (d->K < 1 || d->N < 1) return fail(QLORA_ESHAPE, "K and N must be >= 1");
+    if (d->r < 1 || d->r > 64) return fail(QLORA_ESHAPE, "rank r must be in [1, 64]");
+    if (d->K % 16 != 0)
+        return fail(QLORA_EUNSUPPORTED, "K must be a multiple of 16 (16-byte int8 row pitch)");
+    if (d->K > 131072)
+        return fail(QLORA_EUNSUPPORTED, "K > 131072 would overflow the int32 accumulator");
+    if (d->act_dtype != QLORA_F32 && d->act_dtype != QLORA_BF16)
+        return fail(QLORA_EINVAL, "unknown activation dtype");
+    return QLORA_OK;
+}
+
+int cuda_status(cudaError_t e, const char* what) {
+    if (e == cudaSuccess) return QLORA_OK;
+    return fail(QLORA_ECUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+}  // namespace
+
+bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem_bytes,
+                  uint64_t rows, uint64_t cols, uint64_t pitch_bytes, uint32_t box_rows,
+                  uint32_t box_cols, CUtensorMapSwizzle swizzle) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    (void)elem_bytes;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {pitch_bytes};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+cudaError_t ensure_smem_attr(const void* func, int bytes) {
+    static std::mutex mu;
+    static std::set<std::pair<int, const void*>> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lk(mu);
+    if (done.count({dev, func})) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.insert({dev, func});
+    return e;
+}
+
+}  // namespace qlora
+
+using namespace qlora;
+
+extern "C" {
+
+const char* qlora_version(void) { return "qlora-b200 0.1 sm_100a"; }
+
+const char* qlora_last_error(void) { return g_last_error.c_str(); }
+
+int qlora_device_status(void* stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_status(e, "stream synchronisation failed");
+    int* p = status_ptr();
+    if (!p) return fail(QLORA_ECUDA, "device status word unavailable");
+    int v = 0;
+    e = cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_status(e, "reading the device status word");
+    if (v != 0) {
+        int zero = 0;
+        cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice);
+        return fail(QLORA_ETIMEOUT, "a kernel gave up a bounded wait");
+    }
+    return QLORA_OK;
+}
+
+size_t qlora_workspace_bytes(const qlora_layer_desc* d, int M) {
+    if (check_desc(d) != QLORA_OK || M < 0) return 0;
+    if (M == 0) return 256;
+    return layout_for(*d, M).total;
+}
+
+int qlora_quantize_weight(const float* W, int K, int N, int8_t* Wq, float* sw, void* stream) {
+    if (!W || !Wq || !sw) return fail(QLORA_EINVAL, "NULL pointer argument");
+    if (K < 1 || N < 1) return fail(QLORA_ESHAPE, "K and N must be >= 1");
+    if (K % 16 != 0) return fail(QLORA_EUNSUPPORTED, "K must be a multiple of 16");
+    if (!aligned(W, 4) || !aligned(sw, 4) || !aligned(Wq, 16))
+        return fail(QLORA_EALIGN, "misaligned pointer (W, sw 4 B; Wq 16 B)");
+    return cuda_status(launch_quantize_weight(W, K, N, Wq, sw, static_cast<cudaStream_t>(stream)),
+                       "quantize_weight launch");
+}
+
+// ---------------------------------------------------------------------------
+// step-level entry points (a1 .. a5) and their compositions
+// ---------------------------------------------------------------------------
+#define QL_REQUIRE(cond, code, msg) \
+    do {                            \
+        if (!(cond)) return fail((code), (msg)); \
+    } while (0)
+
+static int check_layer(const qlora_layer_desc* d, int M) {
+    int rc = check_desc(d);
+    if (rc != QLORA_OK) return rc;
+    QL_REQUIRE(M >= 0, QLORA_ESHAPE, "M must be >= 0");
+    return QLORA_OK;
+}
+
+static Act act_of(const qlora_layer_desc* d) { return d->act_dtype == QLORA_BF16 ? kBF16 : kF32; }
+static float lora_scale(const qlora_layer_desc* d) { return d->alpha / static_cast<float>(d->r); }
+
+int qlora_quantize_input(const qlora_layer_desc* d, int M, const void* X, const float* A,
+                         int8_t* Xq, float* sx, float* xA, void* stream) {
+    int rc = check_layer(d, M);
+    if (rc != QLORA_OK) return rc;
+    QL_REQUIRE(X && A && Xq && sx && xA, QLORA_EINVAL, "NULL pointer argument");
+    QL_REQUIRE(aligned(X, 16) && aligned(Xq, 16), QLORA_EALIGN, "X and Xq must be 16-byte aligned");
+    QL_REQUIRE(aligned(A, 4) && aligned(sx, 4) && aligned(xA, 4), QLORA_EALIGN,
+               "fp32 vectors must be 4-byte aligned");
+    if (M == 0) return QLORA_OK;
+    return cuda_status(launch_quantize_rows(act_of(d), X, A, M, d->K, d->r, Xq, sx, xA,
+                                            static_cast<cudaStream_t>(stream)),
+                       "input quantizer launch");
+}
+
+int qlora_gemm_forward(const qlora_layer_desc* d, int M, const int8_t* Xq, const float* sx,
+                       const int8_t* Wq, const float* sw, const float* bias, const float* xA,
+                       const float* B, void* Y, int32_t* acc, void* stream) {
+    int rc = check_layer(d, M);
+    if (rc != QLORA_OK) return rc;
+    QL_REQUIRE(Xq && sx && Wq && sw && xA && B && Y, QLORA_EINVAL, "NULL pointer argument");
+    QL_REQUIRE(aligned(Xq, 16) && aligned(Wq, 16) && aligned(Y, 16), QLORA_EALIGN,
+               "Xq, Wq and Y must be 16-byte aligned");
+    QL_REQUIRE(aligned(sx, 4) && aligned(sw, 4) && aligned(xA, 4) && aligned(B, 4) &&
+                   (!bias || aligned(bias, 4)) && (!acc || aligned(acc, 4)),
+               QLORA_EALIGN, "fp32/int32 vectors must be 4-byte aligned");
+    if (M == 0) return QLORA_OK;
+    int* status = status_ptr();
+    QL_REQUIRE(status, QLORA_ECUDA, "no CUDA device");
+    FwdEpilogue ep;
+    ep.sx = sx;
+    ep.sw = sw;
+    ep.bias = bias;
+    ep.xA = xA;
+    ep.B = B;
+    ep.r = d->r;
+    ep.c = lora_scale(d);
+    ep.Y = Y;
+    ep.acc = acc;
+    return cuda_status(launch_gemm_i8_fwd(act_of(d), Xq, Wq, M, d->N, d->K, ep, status,
+                                          static_cast<cudaStream_t>(stream)),
+                       "int8 GEMM launch");
+}
+
+int qlora_lora_grad_dy(const qlora_layer_desc* d, int M, const void* dY, const float* B,
+                       const float* xA, float* G, float* dB, float* dbias, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    int rc = check_layer(d, M);
+    if (rc != QLORA_OK) return rc;
+    QL_REQUIRE(dY && B && xA && G && dB && workspace, QLORA_EINVAL, "NULL pointer argument");
+    QL_REQUIRE(aligned(dY, 16) && aligned(workspace, 256), QLORA_EALIGN,
+               "dY must be 16-byte aligned, workspace 256-byte aligned");
+    QL_REQUIRE(aligned(B, 4) && aligned(xA, 4) && aligned(G, 4) && aligned(dB, 4) &&
+                   (!dbias || aligned(dbias, 4)),
+               QLORA_EALIGN, "fp32 vectors must be 4-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M == 0) {
+        rc = cuda_status(cudaMemsetAsync(dB, 0, sizeof(float) * d->r * d->N, s), "memset dB");
+        if (rc == QLORA_OK && dbias)
+            rc = cuda_status(cudaMemsetAsync(dbias, 0, sizeof(float) * d->N, s), "memset dbias");
+        return rc;
+    }
+    const WsLayout w = layout_for(*d, M);
+    QL_REQUIRE(workspace_bytes >= w.total, QLORA_EINVAL, "workspace too small");
+    float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.part);
+    return cuda_status(launch_rank_dy(act_of(d), dY, B, xA, M, d->N, d->r, lora_scale(d), w.plan,
+                                      G, dB, dbias, part, s),
+                       "dY pass launch");
+}
+
+int qlora_gemm_dx(const qlora_layer_desc* d, int M, const void* dY, const int8_t* Wq,
+                  const float* sw, const float* G, const float* A, void* dX, void* stream) {
+    int rc = check_layer(d, M);
+    if (rc != QLORA_OK) return rc;
+    QL_REQUIRE(dY && Wq && sw && G && A && dX, QLORA_EINVAL, "NULL pointer argument");
+    QL_REQUIRE(aligned(dY, 16) && aligned(Wq, 16) && aligned(dX, 16), QLORA_EALIGN,
+               "dY, Wq and dX must be 16-byte aligned");
+    QL_REQUIRE(aligned(sw, 4) && aligned(G, 4) && aligned(A, 4), QLORA_EALIGN,
+               "fp32 vectors must be 4-byte aligned");
+    if (M == 0) return QLORA_OK;
+    int* status = status_ptr();
+    QL_REQUIRE(status, QLORA_ECUDA, "no CUDA device");
+    DxEpilogue ep;
+    ep.G = G;
+    ep.A = A;
+    ep.r = d->r;
+    ep.c = lora_scale(d);
+    ep.dX = dX;
+    return cuda_status(launch_gemm_dx(act_of(d), dY, Wq, sw, M, d->N, d->K, ep, status,
+                                      static_cast<cudaStream_t>(stream)),
+                       "dX GEMM launch");
+}
+
+int qlora_lora_grad_x(const qlora_layer_desc* d, int M, const void* X, const float* G, float* dA,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_layer(d, M);
+    if (rc != QLORA_OK) return rc;
+    QL_REQUIRE(X && G && dA && workspace, QLORA_EINVAL, "NULL pointer argument");
+    QL_REQUIRE(aligned(X, 16) && aligned(workspace, 256), QLORA_EALIGN,
+               "X must be 16-byte aligned, workspace 256-byte aligned");
+    QL_REQUIRE(aligned(G, 4) && aligned(dA, 4), QLORA_EALIGN, "fp32 vectors must be 4-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M == 0) return cuda_status(cudaMemsetAsync(dA, 0, sizeof(float) * d->K * d->r, s), "memset dA");
+    const WsLayout w = layout_for(*d, M);
+    QL_REQUIRE(workspace_bytes >= w.total, QLORA_EINVAL, "workspace too small");
+    float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.part);
+    return cuda_status(launch_rank_x(act_of(d), X, G, M, d->K, d->r, lora_scale(d), w.plan, dA,
+                                     part, s),
+                       "X pass launch");
+}
+
+int qlora_forward(const qlora_layer_desc* d, int M, const void* X, const int8_t* Wq,
+                  const float* sw, const float* bias, const float* A, const float* B, void* Y,
+                  float* xA, void* workspace, size_t workspace_bytes, const qlora_debug* dbg,
+                  void* stream) {
+    int rc = check_layer(d, M);
+    if (rc != QLORA_OK) return rc;
+    QL_REQUIRE(X && Wq && sw && A && B && Y && xA && workspace, QLORA_EINVAL,
+               "NULL pointer argument");
+    QL_REQUIRE(aligned(X, 16) && aligned(Y, 16) && aligned(Wq, 16) && aligned(workspace, 256),
+               QLORA_EALIGN, "X, Y, Wq must be 16-byte aligned, workspace 256-byte aligned");
+    QL_REQUIRE(aligned(sw, 4) && aligned(A, 4) && aligned(B, 4) && aligned(xA, 4) &&
+                   (!bias || aligned(bias, 4)),
+               QLORA_EALIGN, "fp32 vectors must be 4-byte aligned");
+    QL_REQUIRE(!dbg || ((!dbg->xq || aligned(dbg->xq, 16)) && (!dbg->sx || aligned(dbg->sx, 4)) &&
+                        (!dbg->acc || aligned(dbg->acc, 4))),
+               QLORA_EALIGN, "misaligned debug output");
+    if (M == 0) return QLORA_OK;
+    const WsLayout w = layout_for(*d, M);
+    QL_REQUIRE(workspace_bytes >= w.total, QLORA_EINVAL, "workspace too small");
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int8_t* Xq = (dbg && dbg->xq) ? dbg->xq : reinterpret_cast<int8_t*>(ws + w.xq);
+    float* sx = (dbg && dbg->sx) ? dbg->sx : reinterpret_cast<float*>(ws + w.sx);
+    rc = qlora_quantize_input(d, M, X, A, Xq, sx, xA, stream);
+    if (rc != QLORA_OK) return rc;
+    return qlora_gemm_forward(d, M, Xq, sx, Wq, sw, bias, xA, B, Y, dbg ? dbg->acc : nullptr,
+                              stream);
+}
+
+int qlora_backward(const qlora_layer_desc* d, int M, const void* X, const void* dY,
+                   const int8_t* Wq, const float* sw, const float* A, const float* B,
+                   const float* xA, void* dX, float* dA, float* dB, float* dbias, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+    int rc = check_layer(d, M);
+    if (rc != QLORA_OK) return rc;
+    QL_REQUIRE(X && dY && Wq && sw && A && B && xA && dA && dB && workspace, QLORA_EINVAL,
+               "NULL pointer argument");
+    QL_REQUIRE(aligned(X, 16) && aligned(dY, 16) && aligned(Wq, 16) && (!dX || aligned(dX, 16)) &&
+                   aligned(workspace, 256),
+               QLORA_EALIGN, "X, dY, dX, Wq must be 16-byte aligned, workspace 256-byte aligned");
+    QL_REQUIRE(aligned(sw, 4) && aligned(A, 4) && aligned(B, 4) && aligned(xA, 4) &&
+                   aligned(dA, 4) && aligned(dB, 4) && (!dbias || aligned(dbias, 4)),
+               QLORA_EALIGN, "fp32 vectors must be 4-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M == 0) {
+        // empty batch: the gradients of the LoRA factors and bias are zero
+        rc = cuda_status(cudaMemsetAsync(dA, 0, sizeof(float) * d->K * d->r, s), "memset dA");
+        if (rc == QLORA_OK)
+            rc = cuda_status(cudaMemsetAsync(dB, 0, sizeof(float) * d->r * d->N, s), "memset dB");
+        if (rc == QLORA_OK && dbias)
+            rc = cuda_status(cudaMemsetAsync(dbias, 0, sizeof(float) * d->N, s), "memset dbias");
+        return rc;
+    }
+    const WsLayout w = layout_for(*d, M);
+    QL_REQUIRE(workspace_bytes >= w.total, QLORA_EINVAL, "workspace too small");
+    float* G = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.g);
+    rc = qlora_lora_grad_dy(d, M, dY, B, xA, G, dB, dbias, workspace, workspace_bytes, stream);
+    if (rc != QLORA_OK) return rc;
+    if (dX) {
+        rc = qlora_gemm_dx(d, M, dY, Wq, sw, G, A, dX, stream);
+        if (rc != QLORA_OK) return rc;
+    }
+    return qlora_lora_grad_x(d, M, X, G, dA, workspace, workspace_bytes, stream);
+}
+
+int qlora_merge(const qlora_layer_desc* d, const int8_t* Wq, const float* sw, const float* A,
+                const float* B, int8_t* Wq_out, float* sw_out, void* stream) {
+    int rc = check_desc(d);
+    if (rc != QLORA_OK) return rc;
+    if (!Wq || !sw || !A || !B || !Wq_out || !sw_out)
+        return fail(QLORA_EINVAL, "NULL pointer argument");
+    if (!aligned(Wq, 16) || !aligned(Wq_out, 16))
+        return fail(QLORA_EALIGN, "Wq and Wq_out must be 16-byte aligned");
+    if (!aligned(sw, 4) || !aligned(A, 4) || !aligned(B, 4) || !aligned(sw_out, 4))
+        return fail(QLORA_EALIGN, "fp32 vectors must be 4-byte aligned");
+    if (Wq_out == Wq || sw_out == sw) return fail(QLORA_EINVAL, "merge outputs alias its inputs");
+    const float c = d->alpha / static_cast<float>(d->r);
+    return cuda_status(launch_merge(Wq, sw, A, B, d->K, d->N, d->r, c, Wq_out, sw_out,
+                                    static_cast<cudaStream_t>(stream)),
+                       "merge launch");
+}
+
+int qlora_relu(void* Y, size_t n, qlora_dtype dtype, void* stream) {
+    if (!Y) return fail(QLORA_EINVAL, "NULL pointer argument");
+    if (dtype != QLORA_F32 && dtype != QLORA_BF16) return fail(QLORA_EINVAL, "unknown dtype");
+    if (n == 0) return QLORA_OK;
+    return cuda_status(launch_relu(dtype == QLORA_BF16 ? kBF16 : kF32, Y, n,
+                                   static_cast<cudaStream_t>(stream)),
+                       "relu launch");
+}
+
+int qlora_relu_backward(void* dY, const void* Y, size_t n, qlora_dtype dtype, void* stream) {
+    if (!dY || !Y) return fail(QLORA_EINVAL, "NULL pointer argument");
+    if (dtype != QLORA_F32 && dtype != QLORA_BF16) return fail(QLORA_EINVAL, "unknown dtype");
+    if (n == 0) return QLORA_OK;
+    return cuda_status(launch_relu_backward(dtype == QLORA_BF16 ? kBF16 : kF32, dY, Y, n,
+                                            static_cast<cudaStream_t>(stream)),
+                       "relu backward launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,282 @@
+"""Python binding of libqlora.so: the C ABI of include/qlora.h, same names.
+
+Argument marshalling only: every function checks dtypes/shapes of the torch
+tensors it is given, passes their device pointers and the current CUDA stream
+to the library, and raises ``QLoraError`` on a non-OK status.  All arithmetic
+runs in the library's kernels; there is no fallback of any kind.  If the
+library has not been built, importing this module raises.
+
+PyTorch only provides device memory and streams here.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqlora.so")
+
+QLORA_F32 = 0
+QLORA_BF16 = 1
+
+STATUS = {0: "QLORA_OK", -1: "QLORA_EINVAL", -2: "QLORA_EALIGN", -3: "QLORA_ESHAPE",
+          -4: "QLORA_ECUDA", -5: "QLORA_EUNSUPPORTED", -6: "QLORA_ETIMEOUT"}
+
+EXPORTED = ("qlora_quantize_weight", "qlora_workspace_bytes", "qlora_forward",
+            "qlora_backward", "qlora_merge", "qlora_last_error", "qlora_device_status",
+            "qlora_version", "qlora_relu", "qlora_relu_backward", "qlora_quantize_input",
+            "qlora_gemm_forward", "qlora_lora_grad_dy", "qlora_gemm_dx", "qlora_lora_grad_x")
+
+
+class QLoraError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__("%s (%d): %s" % (STATUS.get(code, "?"), code, msg))
+        self.code = code
+
+
+class LayerDesc(ctypes.Structure):
+    _fields_ = [("K", ctypes.c_int), ("N", ctypes.c_int), ("r", ctypes.c_int),
+                ("alpha", ctypes.c_float), ("act_dtype", ctypes.c_int)]
+
+
+class Debug(ctypes.Structure):
+    _fields_ = [("xq", ctypes.c_void_p), ("sx", ctypes.c_void_p), ("acc", ctypes.c_void_p)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libqlora.so is not built (run python -m lora_fine_tuning_qlora_b200.build)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    lib.qlora_quantize_weight.argtypes = [P, I, I, P, P, P]
+    lib.qlora_quantize_weight.restype = I
+    lib.qlora_workspace_bytes.argtypes = [ctypes.POINTER(LayerDesc), I]
+    lib.qlora_workspace_bytes.restype = ctypes.c_size_t
+    lib.qlora_forward.argtypes = [ctypes.POINTER(LayerDesc), I, P, P, P, P, P, P, P, P, P,
+                                  ctypes.c_size_t, ctypes.POINTER(Debug), P]
+    lib.qlora_forward.restype = I
+    lib.qlora_backward.argtypes = [ctypes.POINTER(LayerDesc), I, P, P, P, P, P, P, P, P, P, P,
+                                   P, P, ctypes.c_size_t, P]
+    lib.qlora_backward.restype = I
+    lib.qlora_merge.argtypes = [ctypes.POINTER(LayerDesc), P, P, P, P, P, P, P]
+    lib.qlora_merge.restype = I
+    lib.qlora_last_error.restype = ctypes.c_char_p
+    lib.qlora_device_status.argtypes = [P]
+    lib.qlora_device_status.restype = I
+    lib.qlora_version.restype = ctypes.c_char_p
+    lib.qlora_relu.argtypes = [P, ctypes.c_size_t, I, P]
+    lib.qlora_relu.restype = I
+    lib.qlora_relu_backward.argtypes = [P, P, ctypes.c_size_t, I, P]
+    lib.qlora_relu_backward.restype = I
+    D = ctypes.POINTER(LayerDesc)
+    Z = ctypes.c_size_t
+    lib.qlora_quantize_input.argtypes = [D, I, P, P, P, P, P, P]
+    lib.qlora_gemm_forward.argtypes = [D, I, P, P, P, P, P, P, P, P, P, P]
+    lib.qlora_lora_grad_dy.argtypes = [D, I, P, P, P, P, P, P, P, Z, P]
+    lib.qlora_gemm_dx.argtypes = [D, I, P, P, P, P, P, P, P]
+    lib.qlora_lora_grad_x.argtypes = [D, I, P, P, P, P, Z, P]
+    for f in (lib.qlora_quantize_input, lib.qlora_gemm_forward, lib.qlora_lora_grad_dy,
+              lib.qlora_gemm_dx, lib.qlora_lora_grad_x):
+        f.restype = I
+    return lib
+
+
+_lib = _load()
+
+
+def lib():
+    return _lib
+
+
+def _check(code: int):
+    if code != 0:
+        raise QLoraError(code, _lib.qlora_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def act_code(dtype: torch.dtype) -> int:
+    if dtype == torch.bfloat16:
+        return QLORA_BF16
+    if dtype == torch.float32:
+        return QLORA_F32
+    raise ValueError("activations must be float32 or bfloat16")
+
+
+def desc(K: int, N: int, r: int, alpha: float, act: torch.dtype) -> LayerDesc:
+    return LayerDesc(int(K), int(N), int(r), float(alpha), act_code(act))
+
+
+def version() -> str:
+    return _lib.qlora_version().decode()
+
+
+def qlora_workspace_bytes(d: LayerDesc, M: int) -> int:
+    return int(_lib.qlora_workspace_bytes(ctypes.byref(d), int(M)))
+
+
+def workspace(d: LayerDesc, M: int, device=None) -> torch.Tensor:
+    """A uint8 device buffer big enough for forward and backward at M tokens."""
+    n = qlora_workspace_bytes(d, M)
+    if n == 0:
+        raise QLoraError(-1, "invalid layer descriptor")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def qlora_quantize_weight(W: torch.Tensor, Wq: torch.Tensor, sw: torch.Tensor, stream=None):
+    K, N = W.shape
+    assert W.dtype == torch.float32 and Wq.dtype == torch.int8 and sw.dtype == torch.float32
+    assert tuple(Wq.shape) == (N, K) and tuple(sw.shape) == (N,)
+    _check(_lib.qlora_quantize_weight(_ptr(W), K, N, _ptr(Wq), _ptr(sw), _stream(stream)))
+
+
+def quantize_weight(W: torch.Tensor, stream=None):
+    K, N = W.shape
+    Wq = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    sw = torch.empty((N,), dtype=torch.float32, device=W.device)
+    qlora_quantize_weight(W, Wq, sw, stream)
+    return Wq, sw
+
+
+def qlora_forward(d: LayerDesc, M: int, X, Wq, sw, bias, A, B, Y, xA, ws, dbg: Optional[Debug] = None,
+                  stream=None):
+    _check(_lib.qlora_forward(ctypes.byref(d), int(M), _ptr(X), _ptr(Wq), _ptr(sw), _ptr(bias),
+                              _ptr(A), _ptr(B), _ptr(Y), _ptr(xA), _ptr(ws), ws.numel(),
+                              ctypes.byref(dbg) if dbg is not None else None, _stream(stream)))
+
+
+def qlora_backward(d: LayerDesc, M: int, X, dY, Wq, sw, A, B, xA, dX, dA, dB, dbias, ws,
+                   stream=None):
+    _check(_lib.qlora_backward(ctypes.byref(d), int(M), _ptr(X), _ptr(dY), _ptr(Wq), _ptr(sw),
+                               _ptr(A), _ptr(B), _ptr(xA), _ptr(dX), _ptr(dA), _ptr(dB),
+                               _ptr(dbias), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def qlora_merge(d: LayerDesc, Wq, sw, A, B, Wq_out, sw_out, stream=None):
+    _check(_lib.qlora_merge(ctypes.byref(d), _ptr(Wq), _ptr(sw), _ptr(A), _ptr(B), _ptr(Wq_out),
+                            _ptr(sw_out), _stream(stream)))
+
+
+def qlora_quantize_input(d: LayerDesc, M: int, X, A, Xq, sx, xA, stream=None):
+    _check(_lib.qlora_quantize_input(ctypes.byref(d), int(M), _ptr(X), _ptr(A), _ptr(Xq), _ptr(sx),
+                                     _ptr(xA), _stream(stream)))
+
+
+def qlora_gemm_forward(d: LayerDesc, M: int, Xq, sx, Wq, sw, bias, xA, B, Y, acc=None, stream=None):
+    _check(_lib.qlora_gemm_forward(ctypes.byref(d), int(M), _ptr(Xq), _ptr(sx), _ptr(Wq), _ptr(sw),
+                                   _ptr(bias), _ptr(xA), _ptr(B), _ptr(Y), _ptr(acc), _stream(stream)))
+
+
+def qlora_lora_grad_dy(d: LayerDesc, M: int, dY, B, xA, G, dB, dbias, ws, stream=None):
+    _check(_lib.qlora_lora_grad_dy(ctypes.byref(d), int(M), _ptr(dY), _ptr(B), _ptr(xA), _ptr(G),
+                                   _ptr(dB), _ptr(dbias), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def qlora_gemm_dx(d: LayerDesc, M: int, dY, Wq, sw, G, A, dX, stream=None):
+    _check(_lib.qlora_gemm_dx(ctypes.byref(d), int(M), _ptr(dY), _ptr(Wq), _ptr(sw), _ptr(G),
+                              _ptr(A), _ptr(dX), _stream(stream)))
+
+
+def qlora_lora_grad_x(d: LayerDesc, M: int, X, G, dA, ws, stream=None):
+    _check(_lib.qlora_lora_grad_x(ctypes.byref(d), int(M), _ptr(X), _ptr(G), _ptr(dA), _ptr(ws),
+                                  ws.numel(), _stream(stream)))
+
+
+def qlora_relu(Y: torch.Tensor, stream=None):
+    _check(_lib.qlora_relu(_ptr(Y), Y.numel(), act_code(Y.dtype), _stream(stream)))
+
+
+def qlora_relu_backward(dY: torch.Tensor, Y: torch.Tensor, stream=None):
+    assert dY.shape == Y.shape and dY.dtype == Y.dtype
+    _check(_lib.qlora_relu_backward(_ptr(dY), _ptr(Y), Y.numel(), act_code(Y.dtype), _stream(stream)))
+
+
+def qlora_device_status(stream=None) -> int:
+    return int(_lib.qlora_device_status(_stream(stream)))
+
+
+@dataclass
+class Layer:
+    """Device buffers of one int8-LoRA Dense layer (frozen Wq/sw, trainable A/B)."""
+
+    Wq: torch.Tensor
+    sw: torch.Tensor
+    bias: Optional[torch.Tensor]
+    A: torch.Tensor
+    B: torch.Tensor
+    alpha: float
+    act: torch.dtype
+
+    @property
+    def K(self):
+        return self.Wq.shape[1]
+
+    @property
+    def N(self):
+        return self.Wq.shape[0]
+
+    @property
+    def r(self):
+        return self.A.shape[1]
+
+    def desc(self) -> LayerDesc:
+        return desc(self.K, self.N, self.r, self.alpha, self.act)
+
+
+def forward(layer: Layer, X: torch.Tensor, ws: torch.Tensor, Y=None, xA=None, debug: bool = False,
+            stream=None):
+    """Returns (Y, xA[, (Xq, sx, acc)])."""
+    M = X.shape[0]
+    dev = X.device
+    Y = Y if Y is not None else torch.empty((M, layer.N), dtype=layer.act, device=dev)
+    xA = xA if xA is not None else torch.empty((M, layer.r), dtype=torch.float32, device=dev)
+    dbg = None
+    if debug:
+        xq = torch.empty((M, layer.K), dtype=torch.int8, device=dev)
+        sx = torch.empty((M,), dtype=torch.float32, device=dev)
+        acc = torch.empty((M, layer.N), dtype=torch.int32, device=dev)
+        dbg = Debug(xq.data_ptr(), sx.data_ptr(), acc.data_ptr())
+    qlora_forward(layer.desc(), M, X, layer.Wq, layer.sw, layer.bias, layer.A, layer.B, Y, xA, ws,
+                  dbg, stream)
+    if debug:
+        return Y, xA, (xq, sx, acc)
+    return Y, xA
+
+
+def backward(layer: Layer, X, dY, xA, ws, dX=None, want_dx=True, want_dbias=True, stream=None):
+    """Returns (dX or None, dA, dB, dbias or None)."""
+    M = X.shape[0]
+    dev = X.device
+    if want_dx and dX is None:
+        dX = torch.empty((M, layer.K), dtype=layer.act, device=dev)
+    dA = torch.empty((layer.K, layer.r), dtype=torch.float32, device=dev)
+    dB = torch.empty((layer.r, layer.N), dtype=torch.float32, device=dev)
+    dbias = torch.empty((layer.N,), dtype=torch.float32, device=dev) if want_dbias else None
+    qlora_backward(layer.desc(), M, X, dY, layer.Wq, layer.sw, layer.A, layer.B, xA,
+                   dX if want_dx else None, dA, dB, dbias, ws, stream)
+    return (dX if want_dx else None), dA, dB, dbias
+
+
+def merge(layer: Layer, stream=None):
+    Wq2 = torch.empty_like(layer.Wq)
+    sw2 = torch.empty_like(layer.sw)
+    qlora_merge(layer.desc(), layer.Wq, layer.sw, layer.A, layer.B, Wq2, sw2, stream)
+    return Wq2, sw2

@@ -1,0 +1,169 @@
+"""The MNIST MLP workload as a stack of int8-LoRA Dense layers on one GPU.
+
+784 -> 1024, 31 x (1024 -> 1024), 1024 -> 10 with a plain ReLU between
+layers ("Introduce QLoRA-like technique", benchmark.py and its Results
+table), batch 1024, bf16 activations, rank-8 adapters.  One ``step`` is the
+forward through every layer and the backward through every layer (dX, dA,
+dB of each), all through the C ABI into preallocated device buffers, so a
+step can be captured into a CUDA graph and replayed.
+"""
+from __future__ import annotations
+
+from typing import Dict, List, Optional
+
+import torch
+
+from . import inputs as _inputs
+from . import qlora
+
+
+class MLPStack:
+    def __init__(self, layers: List[qlora.Layer], batch: int, device="cuda"):
+        self.layers = layers
+        self.M = batch
+        self.act = layers[0].act
+        dev = torch.device(device)
+        # the largest workspace over the layers serves all of them
+        need = max(qlora.qlora_workspace_bytes(L.desc(), batch) for L in layers)
+        self.ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        self.X = torch.zeros((batch, layers[0].K), dtype=self.act, device=dev)
+        self.dY = torch.zeros((batch, layers[-1].N), dtype=self.act, device=dev)
+        self.H = [torch.empty((batch, L.N), dtype=self.act, device=dev) for L in layers]
+        self.xA = [torch.empty((batch, L.r), dtype=torch.float32, device=dev) for L in layers]
+        self.G = [torch.empty((batch, L.N), dtype=self.act, device=dev) for L in layers]
+        self.dX = torch.empty((batch, layers[0].K), dtype=self.act, device=dev)
+        self.dbias = [torch.empty((L.N,), dtype=torch.float32, device=dev) for L in layers]
+        Kmax = max(L.K for L in layers)
+        rmax = max(L.r for L in layers)
+        self.Xq = torch.empty((batch, Kmax), dtype=torch.int8, device=dev)
+        self.sx = torch.empty((batch,), dtype=torch.float32, device=dev)
+        self.Gr = torch.empty((batch, rmax), dtype=torch.float32, device=dev)
+        # the LoRA gradients live in one flat buffer (one all-reduce in data
+        # parallel runs); dA[i], dB[i] are views into it
+        sizes = [L.K * L.r + L.r * L.N for L in layers]
+        self.grad_flat = torch.empty((sum(sizes),), dtype=torch.float32, device=dev)
+        off = 0
+        self.dA, self.dB = [], []
+        for L in layers:
+            self.dA.append(self.grad_flat[off:off + L.K * L.r].view(L.K, L.r))
+            off += L.K * L.r
+            self.dB.append(self.grad_flat[off:off + L.r * L.N].view(L.r, L.N))
+            off += L.r * L.N
+        self.descs = [L.desc() for L in layers]
+        self.graph: Optional[torch.cuda.CUDAGraph] = None
+        self.events = None
+
+    @classmethod
+    def from_inputs(cls, specs: List[_inputs.LayerSpec], data: Dict[str, object], device="cuda"):
+        layers = []
+        act = torch.bfloat16 if specs[0].act == "bf16" else torch.float32
+        for s, L in zip(specs, data["layers"]):
+            Wq, sw = qlora.quantize_weight(torch.from_numpy(L["W"]).to(device))
+            bias = torch.from_numpy(L["bias"]).to(device) if L["bias"] is not None else None
+            layers.append(qlora.Layer(Wq=Wq, sw=sw, bias=bias,
+                                      A=torch.from_numpy(L["A"]).to(device),
+                                      B=torch.from_numpy(L["B"]).to(device),
+                                      alpha=s.alpha, act=act))
+        return cls(layers, specs[0].M, device)
+
+    # ------------------------------------------------------------------
+    def launches_per_step(self) -> int:
+        """Kernels this library launches in one step (for the benchmark)."""
+        n = 0
+        for i, L in enumerate(self.layers):
+            n += 2                                   # quantize+xA, int8 GEMM
+            n += 1 if i < len(self.layers) - 1 else 0  # ReLU
+            rj = (L.r + 7) // 8
+            n += rj + 1                              # dY pass(es) + reduction
+            n += 1                                   # dX GEMM
+            n += rj + 1                              # X pass(es) + reduction
+            n += 1 if i < len(self.layers) - 1 else 0  # ReLU backward
+        return n
+
+    def _run(self, stream=None, events=None):
+        """One step.  ``events`` optionally maps a step name ("gemm_forward"
+        or "gemm_dx") to a list of (start, end) CUDA events per layer that
+        are recorded around that step's launch."""
+        L_ = self.layers
+        n = len(L_)
+        D = self.descs
+        M = self.M
+        ev_f = events.get("gemm_forward") if events else None
+        ev_d = events.get("gemm_dx") if events else None
+        h = self.X
+        for i, L in enumerate(L_):
+            qlora.qlora_quantize_input(D[i], M, h, L.A, self.Xq, self.sx, self.xA[i], stream)
+            if ev_f:
+                ev_f[i][0].record()
+            qlora.qlora_gemm_forward(D[i], M, self.Xq, self.sx, L.Wq, L.sw, L.bias, self.xA[i],
+                                     L.B, self.H[i], None, stream)
+            if ev_f:
+                ev_f[i][1].record()
+            if i < n - 1:
+                qlora.qlora_relu(self.H[i], stream)
+            h = self.H[i]
+        g = self.dY
+        for i in range(n - 1, -1, -1):
+            L = L_[i]
+            if i < n - 1:
+                qlora.qlora_relu_backward(g, self.H[i], stream)
+            x_in = self.X if i == 0 else self.H[i - 1]
+            dX = self.dX if i == 0 else self.G[i - 1]
+            qlora.qlora_lora_grad_dy(D[i], M, g, L.B, self.xA[i], self.Gr, self.dB[i],
+                                     self.dbias[i], self.ws, stream)
+            if ev_d:
+                ev_d[i][0].record()
+            qlora.qlora_gemm_dx(D[i], M, g, L.Wq, L.sw, self.Gr, L.A, dX, stream)
+            if ev_d:
+                ev_d[i][1].record()
+            qlora.qlora_lora_grad_x(D[i], M, x_in, self.Gr, self.dA[i], self.ws, stream)
+            g = dX
+
+    def make_events(self, kinds=("gemm_dx",)):
+        """Timing events (graph-capturable) around the given steps, per layer."""
+        return {k: [(torch.cuda.Event(enable_timing=True, external=True),
+                     torch.cuda.Event(enable_timing=True, external=True))
+                    for _ in self.layers] for k in kinds}
+
+    def capture(self, warmup: int = 1, events=None):
+        """Records one step into a CUDA graph (after `warmup` eager steps)."""
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for _ in range(warmup):
+                self._run()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self._run(events=events)
+        self.graph = g
+        self.events = events
+        return g
+
+    def replay(self):
+        assert self.graph is not None
+        self.graph.replay()
+
+    def step(self, X: Optional[torch.Tensor] = None, dY: Optional[torch.Tensor] = None,
+             use_graph: bool = False):
+        if X is not None:
+            self.X.copy_(X)
+        if dY is not None:
+            self.dY.copy_(dY)
+        if use_graph:
+            self.replay()
+        else:
+            self._run()
+        return {"y": self.H[-1], "dX": self.dX, "dA": self.dA, "dB": self.dB, "dbias": self.dbias}
+
+    # ------------------------------------------------------------------
+    def flops_per_step(self) -> float:
+        """Algorithmic work of one step: int8 2MNK + bf16 2MNK per layer plus
+        the rank-r terms (x.A, (xA).B, G, G.A^T, dA, dB)."""
+        tot = 0.0
+        M = self.M
+        for L in self.layers:
+            tot += 2.0 * M * L.N * L.K * 2
+            tot += 2.0 * M * L.r * (2 * L.K + 2 * L.N) + 2.0 * M * L.r * (L.K + L.N)
+        return tot

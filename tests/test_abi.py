@@ -1,0 +1,115 @@
+"""The C-ABI library: it loads without a GPU, exports every function that
+include/qlora.h declares, and rejects bad arguments before launching anything
+(these calls return before the library touches the CUDA runtime)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    with open(os.path.join(ROOT, "include", "qlora.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qlora_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def q():
+    from lora_fine_tuning_qlora_b200 import build
+    build.build()
+    from lora_fine_tuning_qlora_b200 import qlora
+    return qlora
+
+
+def test_header_declares_the_boundary():
+    fns = _header_functions()
+    for name in ("qlora_quantize_weight", "qlora_workspace_bytes", "qlora_forward",
+                 "qlora_backward", "qlora_merge", "qlora_last_error"):
+        assert name in fns
+
+
+def test_library_exports_every_declared_symbol(q):
+    lib = ctypes.CDLL(q.LIB_PATH)
+    for name in _header_functions():
+        assert hasattr(lib, name), name
+    assert set(q.EXPORTED) == set(_header_functions())
+
+
+def test_library_has_no_libcuda_or_torch_dependency(q):
+    import subprocess
+    out = subprocess.run(["ldd", q.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out
+    assert "torch" not in out and "libc10" not in out
+
+
+def test_version(q):
+    assert "sm_100a" in q.version()
+
+
+def test_workspace_bytes(q):
+    d = q.desc(1024, 1024, 8, 8.0, __import__("torch").bfloat16)
+    n = q.qlora_workspace_bytes(d, 1024)
+    # at least the int8 copy of X and its scales
+    assert n >= 1024 * 1024 + 4 * 1024
+    assert n % 256 == 0
+    bad = q.desc(1000, 1024, 8, 8.0, __import__("torch").bfloat16)  # K % 16 != 0
+    assert q.qlora_workspace_bytes(bad, 1024) == 0
+
+
+def _fwd(q, d, M, X=0x1000, Wq=0x2000, sw=0x3000, bias=None, A=0x4000, B=0x5000, Y=0x6000,
+         xA=0x7000, ws=0x8000, wsb=1 << 30):
+    P = ctypes.c_void_p
+    return q.lib().qlora_forward(ctypes.byref(d) if d is not None else None, M, P(X), P(Wq), P(sw),
+                                 P(bias) if bias else None, P(A), P(B), P(Y), P(xA), P(ws), wsb,
+                                 None, None)
+
+
+def test_forward_rejects_bad_arguments_without_launching(q):
+    import torch
+    d = q.desc(784, 128, 4, 4.0, torch.float32)
+    assert _fwd(q, None, 64) == -1                       # NULL descriptor
+    assert _fwd(q, d, -1) == -3                          # negative M
+    assert _fwd(q, q.desc(784, 128, 0, 4.0, torch.float32), 64) == -3   # r = 0
+    assert _fwd(q, q.desc(784, 128, 65, 4.0, torch.float32), 64) == -3  # r > 64
+    assert _fwd(q, q.desc(780, 128, 4, 4.0, torch.float32), 64) == -5   # K % 16
+    assert _fwd(q, q.desc(784, 0, 4, 4.0, torch.float32), 64) == -3     # N = 0
+    assert _fwd(q, d, 64, X=0) == -1                     # NULL X
+    assert _fwd(q, d, 64, X=0x1008) == -2                # X not 16-byte aligned
+    assert _fwd(q, d, 64, ws=0x8010) == -2               # workspace not 256-byte aligned
+    assert _fwd(q, d, 64, sw=0x3002) == -2               # fp32 vector misaligned
+    assert b"aligned" in q.lib().qlora_last_error()
+    assert _fwd(q, d, 64, wsb=16) == -1                  # workspace too small
+    assert b"workspace" in q.lib().qlora_last_error()
+
+
+def test_backward_and_merge_reject_bad_arguments(q):
+    import torch
+    P = ctypes.c_void_p
+    d = q.desc(784, 128, 4, 4.0, torch.bfloat16)
+    rc = q.lib().qlora_backward(ctypes.byref(d), 64, P(0x1000), None, P(0x2000), P(0x3000),
+                                P(0x4000), P(0x5000), P(0x6000), None, P(0x7000), P(0x8000),
+                                None, P(0x9000), 1 << 30, None)
+    assert rc == -1  # NULL dY
+    rc = q.lib().qlora_backward(ctypes.byref(d), 64, P(0x1000), P(0x1804), P(0x2000), P(0x3000),
+                                P(0x4000), P(0x5000), P(0x6000), None, P(0x7000), P(0x8000),
+                                None, P(0x9000), 1 << 30, None)
+    assert rc == -2  # dY misaligned
+    rc = q.lib().qlora_merge(ctypes.byref(d), P(0x1000), P(0x2000), P(0x3000), P(0x4000),
+                             P(0x1000), P(0x5000), None)
+    assert rc == -1  # output aliases input
+    rc = q.lib().qlora_merge(ctypes.byref(d), P(0x1000), P(0x2000), P(0x3000), P(0x4000),
+                             P(0x6008), P(0x5000), None)
+    assert rc == -2  # Wq_out misaligned
+    rc = q.lib().qlora_quantize_weight(P(0x1000), 784, 0, P(0x2000), P(0x3000), None)
+    assert rc == -3
+
+
+def test_binding_refuses_host_tensors(q):
+    import torch
+    W = torch.zeros((32, 16))
+    with pytest.raises(ValueError):
+        q.quantize_weight(W)

@@ -1,0 +1,201 @@
+"""GPU parity: the C-ABI path against the CPU oracle, element by element, on
+seeded inputs shaped like the pages' workloads.  Needs a B200."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from lora_fine_tuning_qlora_b200 import inputs
+
+from parity import assert_close, run_and_compare, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def q():
+    if not torch.cuda.is_available():
+        pytest.fail("these tests need a CUDA device")
+    from lora_fine_tuning_qlora_b200 import build
+    build.build()
+    from lora_fine_tuning_qlora_b200 import qlora
+    oracle.set_threads(max(1, min(32, __import__("os").cpu_count() or 1)))
+    return qlora
+
+
+# ---------------------------------------------------------------- a0
+@pytest.mark.parametrize("K,N", [(784, 128), (1024, 10), (768, 2304), (64, 48), (16, 1)])
+def test_quantize_weight_bit_exact(q, K, N):
+    rng = np.random.Generator(np.random.PCG64(K * 7 + N))
+    W = rng.normal(0, 0.02, (K, N)).astype(np.float32)
+    W[:, 0] = 0.0                      # an all-zero output channel
+    if N > 1:
+        W[3, 1] = 127.0 / 64           # exact .5 ties in that channel
+        W[5, 1] = 2.5 / 64
+        W[7, 1] = -3.5 / 64
+    Wq, sw = q.quantize_weight(torch.from_numpy(W).cuda())
+    Wq_o, sw_o = oracle.quantize_weight(W)
+    np.testing.assert_array_equal(to_np(Wq), Wq_o)
+    np.testing.assert_array_equal(to_np(sw).view(np.uint32), sw_o.view(np.uint32))
+
+
+# ---------------------------------------------------------------- full layers
+def test_single_fp32_layer(q):
+    """The fp32 single-layer workload, every output compared."""
+    run_and_compare(inputs.single_fp32(), q)
+
+
+@pytest.mark.parametrize("M,K,N,r", [(300, 784, 520, 8), (129, 256, 136, 4), (1, 64, 16, 1),
+                                     (200, 1040, 264, 16), (70, 128, 24, 64)])
+def test_bf16_layer_tiles_and_ragged_tails(q, M, K, N, r):
+    spec = inputs.LayerSpec("ragged", M=M, K=K, N=N, r=r, alpha=2.0 * r, act="bf16",
+                            x_dist="normal", w_dist="glorot", a_dist="he_uniform", b_std=0.01,
+                            bias_dist="normal001", seed=M + K + N + r)
+    run_and_compare(spec, q)
+
+
+@pytest.mark.parametrize("M,K,N,r", [(96, 784, 128, 4), (33, 1040, 10, 8)])
+def test_fp32_layer_shapes(q, M, K, N, r):
+    spec = inputs.LayerSpec("f32", M=M, K=K, N=N, r=r, alpha=r, act="f32", x_dist="normal",
+                            w_dist="glorot", a_dist="he_uniform", b_std=0.01,
+                            bias_dist="normal001", seed=M + N)
+    run_and_compare(spec, q)
+
+
+@pytest.mark.parametrize("i", [0, 1, 32])
+def test_mlp_stack_layer_shapes(q, i):
+    """784->1024, 1024->1024 and 1024->10 at batch 1024, every row."""
+    run_and_compare(inputs.mlp_stack()[i], q)
+
+
+@pytest.mark.parametrize("i", range(4))
+def test_gpt2_base_projections(q, i):
+    run_and_compare(inputs.gpt2_base()[i], q, sample_rows=192, seed=i)
+
+
+@pytest.mark.parametrize("M", [512, 4096])
+@pytest.mark.parametrize("i", range(7))
+def test_gemma_2b_projections(q, M, i):
+    spec = inputs.gemma_2b(M)[i]
+    run_and_compare(spec, q, sample_rows=96, seed=i, check_merge=(M == 512))
+
+
+@pytest.mark.parametrize("M", inputs.DENSE4096_M)
+def test_dense4096_sweep(q, M):
+    run_and_compare(inputs.dense4096(M), q, sample_rows=128, seed=M, check_merge=(M == 16))
+
+
+# ---------------------------------------------------------------- edge cases
+def _edge_spec(M, K, N, r, act="bf16", seed=5):
+    return inputs.LayerSpec("edge", M=M, K=K, N=N, r=r, alpha=float(r), act=act, x_dist="normal",
+                            w_dist="glorot", a_dist="he_uniform", b_std=0.01,
+                            bias_dist="normal001", seed=seed)
+
+
+def test_zero_rows_and_exact_ties(q):
+    """All-zero input rows (scale 0), a row whose abs-max element is the only
+    non-zero, and exact .5 ties in the input quantizer."""
+    spec = _edge_spec(40, 256, 64, 4)
+    d = inputs.layer_inputs(spec)
+    X = d["X"]
+    X[3, :] = 0.0
+    X[7, :] = 0.0
+    X[7, 11] = -1.5
+    X[9, :] = 0.0
+    X[9, 0] = 127.0 / 32.0                                     # 127/amax = 32 exactly
+    X[9, 1:6] = np.array([2.5, 3.5, -0.5, 0.5, -1.5], np.float32) / 32.0
+    from lora_fine_tuning_qlora_b200 import qlora
+    layer_d = dict(d)
+    layer_d["X"] = X
+    W = torch.from_numpy(d["W"]).cuda()
+    Wq, sw = q.quantize_weight(W)
+    layer = q.Layer(Wq, sw, torch.from_numpy(d["bias"]).cuda(), torch.from_numpy(d["A"]).cuda(),
+                    torch.from_numpy(d["B"]).cuda(), spec.alpha, torch.bfloat16)
+    Xt = torch.from_numpy(X).to(torch.bfloat16).cuda()
+    ws = q.workspace(layer.desc(), spec.M)
+    Y, xA, (xq, sx, acc) = q.forward(layer, Xt, ws, debug=True)
+    Wq_o, sw_o = oracle.quantize_weight(d["W"])
+    f = oracle.forward(X, Wq_o, sw_o, d["bias"], d["A"], d["B"], spec.alpha)
+    np.testing.assert_array_equal(to_np(xq), f["xq"])
+    np.testing.assert_array_equal(to_np(sx).view(np.uint32), f["sx"].view(np.uint32))
+    np.testing.assert_array_equal(to_np(acc), f["acc"])
+    assert to_np(sx)[3] == 0 and np.all(to_np(xq)[3] == 0)
+    np.testing.assert_array_equal(to_np(xq)[9, :6], [127, 2, 4, 0, 0, -2])
+    assert to_np(xq)[7, 11] == -127
+    assert_close(to_np(Y), f["y"], "bf16", "Y")
+
+
+def test_empty_batch(q):
+    spec = _edge_spec(1, 64, 32, 4)
+    d = inputs.layer_inputs(spec)
+    from parity import device_layer
+    layer = device_layer(spec, d, q)
+    ws = q.workspace(layer.desc(), 1)
+    X = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    Y = torch.empty((0, 32), dtype=torch.bfloat16, device="cuda")
+    xA = torch.empty((0, 4), dtype=torch.float32, device="cuda")
+    # M = 0: nothing to compute; forward is a no-op, backward gives zero gradients
+    q.qlora_forward(layer.desc(), 0, torch.empty(16, dtype=torch.bfloat16, device="cuda"),
+                    layer.Wq, layer.sw, layer.bias, layer.A, layer.B,
+                    torch.empty(16, dtype=torch.bfloat16, device="cuda"),
+                    torch.empty(4, device="cuda"), ws)
+    dA = torch.full((64, 4), 7.0, device="cuda")
+    dB = torch.full((4, 32), 7.0, device="cuda")
+    db = torch.full((32,), 7.0, device="cuda")
+    q.qlora_backward(layer.desc(), 0, torch.empty(16, dtype=torch.bfloat16, device="cuda"),
+                     torch.empty(16, dtype=torch.bfloat16, device="cuda"), layer.Wq, layer.sw,
+                     layer.A, layer.B, torch.empty(4, device="cuda"), None, dA, dB, db, ws)
+    torch.cuda.synchronize()
+    assert torch.all(dA == 0) and torch.all(dB == 0) and torch.all(db == 0)
+    del X, Y, xA
+
+
+def test_B_zero_gives_base_layer(q):
+    """With the LoRA initialisation B = 0 the forward is the base layer and
+    dA is exactly zero."""
+    spec = inputs.scaled(_edge_spec(256, 512, 384, 4), b_std=0.0)
+    out = run_and_compare(spec, q)
+    assert torch.all(out["dA"] == 0)
+
+
+def test_backward_is_deterministic(q):
+    spec = inputs.gpt2_base(1024)[3]
+    d = inputs.layer_inputs(spec)
+    from parity import device_layer
+    layer = device_layer(spec, d, q)
+    X = torch.from_numpy(d["X"]).to(torch.bfloat16).cuda()
+    dY = torch.from_numpy(d["dY"]).to(torch.bfloat16).cuda()
+    ws = q.workspace(layer.desc(), spec.M)
+    Y, xA = q.forward(layer, X, ws)
+    r1 = q.backward(layer, X, dY, xA, ws)
+    r2 = q.backward(layer, X, dY, xA, ws)
+    for a, b in zip(r1, r2):
+        assert torch.equal(a, b)
+
+
+def test_device_status_is_clean(q):
+    assert q.qlora_device_status() == 0
+
+
+# ---------------------------------------------------------------- the MLP stack
+@pytest.mark.slow
+def test_mlp_stack_full(q):
+    """The whole 33-layer MLP stack at batch 1024, forward and backward,
+    against the oracle's stack (bf16 activations between layers)."""
+    from lora_fine_tuning_qlora_b200 import stack
+    specs = inputs.mlp_stack()
+    data = inputs.mlp_stack_inputs(specs)
+    net = stack.MLPStack.from_inputs(specs, data)
+    out = net.step(torch.from_numpy(data["X"]).to(torch.bfloat16).cuda(),
+                   torch.from_numpy(data["dY"]).to(torch.bfloat16).cuda())
+    torch.cuda.synchronize()
+    layers = []
+    for s, L in zip(specs, data["layers"]):
+        Wq, sw = oracle.quantize_weight(L["W"])
+        layers.append({"Wq": Wq, "sw": sw, "bias": L["bias"], "A": L["A"], "B": L["B"], "alpha": s.alpha})
+    ref = oracle.mlp_stack(data["X"], layers, data["dY"], "bf16")
+    assert_close(to_np(out["y"]), ref["y"], "bf16", "stack Y")
+    assert_close(to_np(out["dX"]), ref["dX"], "bf16", "stack dX")
+    for i in range(len(specs)):
+        assert_close(to_np(out["dA"][i]), ref["grads"][i]["dA"], "bf16", "dA[%d]" % i)
+        assert_close(to_np(out["dB"][i]), ref["grads"][i]["dB"], "bf16", "dB[%d]" % i)
