@@ -74,7 +74,7 @@ def _lib():
             lib.orc_lora_down.argtypes = [P, P, L, L, L, P]
             lib.orc_forward.argtypes = [L, L, L, D, P, P, P, P, P, P, P]
             lib.orc_backward.argtypes = [L, L, L, L, D, P, P, P, P, P, P,
-                                         P, P, P, P, P]
+                                         ctypes.c_int, P, P, P, P, P]
             lib.orc_merge.argtypes = [P, P, P, P, L, L, L, F, P, P]
             lib.orc_round_bf16.argtypes = [D]
             lib.orc_round_bf16.restype = D
@@ -175,8 +175,11 @@ def forward(X, Wq, sw, bias, A, B, alpha):
     return {"xq": Xq, "sx": sx, "acc": acc, "xA": xA, "y": Y}
 
 
-def backward(X, dY, Wq, sw, A, B, alpha, want_dx=True):
-    """One int8-LoRA Dense backward; returns dict G, dX, dA, dB, dbias (fp64)."""
+def backward(X, dY, Wq, sw, A, B, alpha, want_dx=True, act="f32"):
+    """One int8-LoRA Dense backward; returns dict G, dX, dA, dB, dbias (fp64).
+
+    ``act`` is the activation dtype: the de-quantized kernel that enters dX is
+    fl32(Wq * sw), rounded once more to bf16 when act == "bf16"."""
     Xd = _c(X, np.float64)
     dYd = _c(dY, np.float64)
     M, K = Xd.shape
@@ -192,8 +195,11 @@ def backward(X, dY, Wq, sw, A, B, alpha, want_dx=True):
     dA = np.empty((K, r), np.float64)
     dB = np.empty((r, N), np.float64)
     db = np.empty((N,), np.float64)
+    if act not in ("f32", "bf16"):
+        raise ValueError(act)
     _lib().orc_backward(M, K, N, r, c, _p(Xd), _p(dYd), _p(Wq), _p(sw), _p(Ad),
-                        _p(Bd), _p(G), _p(dX), _p(dA), _p(dB), _p(db))
+                        _p(Bd), 1 if act == "bf16" else 0, _p(G), _p(dX), _p(dA), _p(dB),
+                        _p(db))
     return {"G": G, "dX": dX, "dA": dA, "dB": dB, "dbias": db}
 
 
@@ -255,7 +261,7 @@ def mlp_stack(X, layers, dY, act_dtype):
         if i < n - 1:
             g = np.where(pre[i] > 0.0, g, 0.0)
         b = backward(inputs[i], g, L["Wq"], L["sw"], L["A"], L["B"], L["alpha"],
-                     want_dx=True)
+                     want_dx=True, act=act_dtype)
         grads[i] = {"dA": b["dA"], "dB": b["dB"], "dbias": b["dbias"]}
         g = to_act(b["dX"], act_dtype)
     return {"y": y_final, "dX": g, "grads": grads, "inputs": inputs, "pre": pre}

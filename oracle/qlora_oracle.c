@@ -30,7 +30,10 @@
  *   - amax == 0 gives inv = 0, hence q = 0 and s = 0;
  *   - the LoRA branch sees the unquantized input x;
  *   - the backward treats the input quantizer as the identity
- *     (straight-through): dX uses the dequantized kernel Wq * s_w;
+ *     (straight-through): dX uses the dequantized kernel Wq * s_w, formed
+ *     in fp32 and, for bf16 activations, stored as bf16 like every other
+ *     operand of that layer's products (the de-quantized tile is a bf16
+ *     operand of the input-gradient product);
  *   - floating-point sums are taken in fp64, integer sums in int64.
  *
  * Layouts (row-major, contiguous):
@@ -176,16 +179,22 @@ void orc_forward(long M, long N, long r, double c, const int32_t* acc,
 /*
  * a3..a5 -- the backward pass (fp64), gradients of L = sum(Y * dY):
  *   G[m,j]  = sum_n dY[m,n] * B[j,n]
- *   dX[m,k] = sum_n dY[m,n] * Wq[n,k] * sw[n] + c * sum_j G[m,j] * A[k,j]
+ *   dX[m,k] = sum_n dY[m,n] * Wd[n,k] + c * sum_j G[m,j] * A[k,j]
+ * where Wd is the de-quantized kernel as the activation dtype stores it:
+ * Wd = fl32(Wq * sw) (one fp32 rounding), further rounded to bfloat16 when
+ * wdq_bf16 is set (bf16 activations: the de-quantized kernel tile is a bf16
+ * operand of the input-gradient product).
  *   dA[k,j] = c * sum_m X[m,k] * G[m,j]
  *   dB[j,n] = c * sum_m xA[m,j] * dY[m,n]     (xA recomputed from X)
  *   dbias[n] = sum_m dY[m,n]
  * Any output pointer may be NULL to skip it.
  */
+double orc_round_bf16(double x);
+
 void orc_backward(long M, long K, long N, long r, double c, const double* X,
                   const double* dY, const int8_t* Wq, const float* sw,
-                  const double* A, const double* B, double* G, double* dX,
-                  double* dA, double* dB, double* dbias) {
+                  const double* A, const double* B, int wdq_bf16, double* G,
+                  double* dX, double* dA, double* dB, double* dbias) {
     double* g = (double*)malloc(sizeof(double) * (size_t)(M * r));
     double* xa = (double*)malloc(sizeof(double) * (size_t)(M * r));
     orc_lora_down(X, A, M, K, r, xa);
@@ -201,15 +210,23 @@ void orc_backward(long M, long K, long N, long r, double c, const double* X,
     if (G) memcpy(G, g, sizeof(double) * (size_t)(M * r));
 
     if (dX) {
+        /* the de-quantized kernel, one row per output channel n */
+        double* wd = (double*)malloc(sizeof(double) * (size_t)(N * K));
+        #pragma omp parallel for schedule(static)
+        for (long n = 0; n < N; ++n) {
+            for (long k = 0; k < K; ++k) {
+                float w = (float)Wq[n * K + k] * sw[n];   /* one fp32 rounding */
+                wd[n * K + k] = wdq_bf16 ? orc_round_bf16((double)w) : (double)w;
+            }
+        }
         #pragma omp parallel for schedule(static)
         for (long m = 0; m < M; ++m) {
             double* row = dX + m * K;
             for (long k = 0; k < K; ++k) row[k] = 0.0;
             for (long n = 0; n < N; ++n) {
                 double d = dY[m * N + n];
-                double s = (double)sw[n];
-                const int8_t* q = Wq + n * K;
-                for (long k = 0; k < K; ++k) row[k] += d * ((double)q[k] * s);
+                const double* w = wd + n * K;
+                for (long k = 0; k < K; ++k) row[k] += d * w[k];
             }
             for (long k = 0; k < K; ++k) {
                 double l = 0.0;
@@ -217,6 +234,7 @@ void orc_backward(long M, long K, long N, long r, double c, const double* X,
                 row[k] += c * l;
             }
         }
+        free(wd);
     }
 
     if (dA) {

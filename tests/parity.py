@@ -97,12 +97,14 @@ def run_and_compare(spec: inputs.LayerSpec, q, sample_rows=None, check_merge=Tru
     assert_close(to_np(xA)[rows], f["xA"], act, "xA")
     assert_close(to_np(Y)[rows], f["y"], act, "Y")
 
-    b_rows = oracle.backward(Xs, d["dY"][rows], Wq_o, sw_o, d["A"], d["B"], spec.alpha, want_dx=True)
+    b_rows = oracle.backward(Xs, d["dY"][rows], Wq_o, sw_o, d["A"], d["B"], spec.alpha,
+                             want_dx=True, act=act)
     assert_close(to_np(dX)[rows], b_rows["dX"], act, "dX")
     if sample_rows is None:
         b_full = b_rows
     else:
-        b_full = oracle.backward(d["X"], d["dY"], Wq_o, sw_o, d["A"], d["B"], spec.alpha, want_dx=False)
+        b_full = oracle.backward(d["X"], d["dY"], Wq_o, sw_o, d["A"], d["B"], spec.alpha,
+                                 want_dx=False, act=act)
     assert_close(to_np(dA), b_full["dA"], act, "dA")
     assert_close(to_np(dB), b_full["dB"], act, "dB")
     assert_close(to_np(dbias), b_full["dbias"], act, "dbias")

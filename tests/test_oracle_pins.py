@@ -328,6 +328,39 @@ def test_backward_dx_exact_grid_equals_float_layer_gradient():
     np.testing.assert_allclose(g["dX"], ref, rtol=1e-12, atol=1e-12)
 
 
+def test_backward_dx_bf16_dequant_is_float_product_with_rounded_kernel():
+    """For bf16 activations dX uses the de-quantized kernel rounded to bf16:
+    it equals the float product dY Wb^T + c dY B^T A^T where Wb is fp32
+    (q * s) rounded to bf16 by torch (library routine); on an exact grid
+    the rounding is the identity and the two activation dtypes agree."""
+    import torch
+    rng = _rng(14)
+    M, K, N, r = 7, 96, 40, 4
+    W = rng.normal(0, 0.05, (K, N)).astype(np.float32)
+    Wq, sw = oracle.quantize_weight(W)
+    X = rng.normal(0, 1, (M, K))
+    A = rng.normal(0, 0.2, (K, r))
+    B = rng.normal(0, 0.2, (r, N))
+    dY = rng.normal(0, 1, (M, N))
+    g = oracle.backward(X, dY, Wq, sw, A, B, 8.0, act="bf16")
+    w32 = Wq.T.astype(np.float32) * sw[None, :]
+    wb = torch.from_numpy(np.ascontiguousarray(w32)).to(torch.bfloat16).double().numpy()
+    ref = dY @ wb.T + 2.0 * (dY @ B.T) @ A.T
+    np.testing.assert_allclose(g["dX"], ref, rtol=1e-12, atol=1e-12)
+    # bf16 rounding really changed the kernel here (the pin is not vacuous)
+    assert np.abs(wb - w32).max() > 0
+    g32 = oracle.backward(X, dY, Wq, sw, A, B, 8.0, act="f32")
+    assert np.abs(g32["dX"] - g["dX"]).max() > 0
+    # exact grid: q * s is a short binary fraction, identical in both dtypes
+    Wg = rng.integers(-127, 128, (K, N)).astype(np.float32)
+    Wg[0, :] = 127.0
+    Wg *= np.float32(2.0 ** -6)
+    Wqg, swg = oracle.quantize_weight(Wg)
+    gb = oracle.backward(X, dY, Wqg, swg, A, B, 8.0, act="bf16")
+    gf = oracle.backward(X, dY, Wqg, swg, A, B, 8.0, act="f32")
+    np.testing.assert_array_equal(gb["dX"], gf["dX"])
+
+
 # --------------------------------------------------------------------------
 # merge
 # --------------------------------------------------------------------------
