@@ -215,6 +215,16 @@ const char* qlora_last_error(void);
  */
 int qlora_device_status(void* stream);
 
+/*
+ * Failure-path self test (no counterpart on the pages).  Enqueues one tiny
+ * kernel whose bounded wait on a barrier that nothing signals gives up after
+ * limit_us microseconds (1 .. 2e6) and records QLORA_ETIMEOUT in the device
+ * status word, exactly as a stalled pipeline in the GEMM kernels would; the
+ * kernel then exits normally and the context stays usable.  The following
+ * qlora_device_status() returns QLORA_ETIMEOUT and clears the word.
+ */
+int qlora_selftest_wait_timeout(unsigned int limit_us, void* stream);
+
 /* Library version, e.g. "qlora-b200 0.1 sm_100a". */
 const char* qlora_version(void);
 

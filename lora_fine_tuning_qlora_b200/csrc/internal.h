@@ -74,6 +74,10 @@ cudaError_t launch_merge(const int8_t* Wq, const float* sw, const float* A, cons
 cudaError_t launch_relu(Act act, void* y, size_t n, cudaStream_t s);
 cudaError_t launch_relu_backward(Act act, void* g, const void* h, size_t n, cudaStream_t s);
 
+// ---------------------------------------------------------------- self test
+// A kernel whose bounded wait runs out after limit_ns (records a timeout).
+cudaError_t launch_selftest_wait(int* status, unsigned long long limit_ns, cudaStream_t s);
+
 // ---------------------------------------------------------------- TMA maps
 // Encodes a 2D row-major tensor map: `rows` x `cols` elements of `elem`
 // bytes, row pitch `pitch_bytes`, box `box_rows` x `box_cols`.

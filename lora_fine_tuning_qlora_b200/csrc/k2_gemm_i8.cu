@@ -119,6 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_load_2d(sb, &tmB, &full[s], kb * kBK, n0);
             }
         }
+        __syncwarp();  // reconverge the warp before the teardown barrier
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_i8(kBM, BN);
@@ -140,6 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (ok) mma_commit(tfull);
         }
+        __syncwarp();  // reconverge the warp before the teardown barrier
     } else {
         // epilogue: warps 2..5 -> TMEM lane quarters 2,3,0,1
         const int q = warp & 3;
@@ -151,7 +153,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < RMAX; ++j)
             xa[j] = (row_ok && j < ep.r) ? ep.xA[static_cast<size_t>(row) * ep.r + j] * ep.c : 0.f;
         if (row_ok) sxm = ep.sx[row];
-        const bool ok = mbar_wait(tfull, 0, status);
+        // warp-uniform, so that the .sync.aligned TMEM loads below stay converged
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(tfull, 0, status));
         tc_fence_after();
         if (ok) {
             OutT* yrow = static_cast<OutT*>(ep.Y) + static_cast<size_t>(row_ok ? row : 0) * N;

@@ -122,6 +122,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_load_2d(sq, &tmQ, &full[s], k0, kb * kBKn);
             }
         }
+        __syncwarp();  // reconverge the warp before the teardown barrier
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16(kBM, BN, false, true);
@@ -146,6 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (ok) mma_commit(tfull);
         }
+        __syncwarp();  // reconverge the warp before the teardown barrier
     } else {
         const int dq = threadIdx.x - 64;  // 0 .. 255
         // ---- de-quantize every stage into the MN-major swizzled bf16 tile ----
@@ -155,7 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < nkb && ok; ++kb) {
             const int s = kb % STAGES;
             const int it = kb / STAGES;
-            ok = mbar_wait(&full[s], it & 1, status);
+            ok = __all_sync(0xffffffffu, mbar_wait(&full[s], it & 1, status));
             if (!ok) break;
             const uint8_t* sq = smem + s * L::kStageBytes + L::kABytes;
             uint8_t* sw_tile = smem + s * L::kStageBytes + L::kABytes + L::kQBytes;
@@ -197,7 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < RMAX; ++j)
             g[j] = (row_ok && j < ep.r) ? ep.G[static_cast<size_t>(row) * ep.r + j] * ep.c : 0.f;
-        ok = ok && mbar_wait(tfull, 0, status);
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(tfull, 0, status));
         tc_fence_after();
         if (ok) {
             __nv_bfloat16* drow =

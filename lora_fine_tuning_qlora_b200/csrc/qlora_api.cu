@@ -383,6 +383,15 @@ int qlora_merge(const qlora_layer_desc* d, const int8_t* Wq, const float* sw, co
                        "merge launch");
 }
 
+int qlora_selftest_wait_timeout(unsigned int limit_us, void* stream) {
+    QL_REQUIRE(limit_us >= 1 && limit_us <= 2000000, QLORA_EINVAL, "limit_us must be in [1, 2e6]");
+    int* status = status_ptr();
+    QL_REQUIRE(status, QLORA_ECUDA, "no CUDA device");
+    return cuda_status(launch_selftest_wait(status, 1000ull * limit_us,
+                                            static_cast<cudaStream_t>(stream)),
+                       "self-test launch");
+}
+
 int qlora_relu(void* Y, size_t n, qlora_dtype dtype, void* stream) {
     if (!Y) return fail(QLORA_EINVAL, "NULL pointer argument");
     if (dtype != QLORA_F32 && dtype != QLORA_BF16) return fail(QLORA_EINVAL, "unknown dtype");

@@ -29,7 +29,8 @@ STATUS = {0: "QLORA_OK", -1: "QLORA_EINVAL", -2: "QLORA_EALIGN", -3: "QLORA_ESHA
 EXPORTED = ("qlora_quantize_weight", "qlora_workspace_bytes", "qlora_forward",
             "qlora_backward", "qlora_merge", "qlora_last_error", "qlora_device_status",
             "qlora_version", "qlora_relu", "qlora_relu_backward", "qlora_quantize_input",
-            "qlora_gemm_forward", "qlora_lora_grad_dy", "qlora_gemm_dx", "qlora_lora_grad_x")
+            "qlora_gemm_forward", "qlora_lora_grad_dy", "qlora_gemm_dx", "qlora_lora_grad_x",
+            "qlora_selftest_wait_timeout")
 
 
 class QLoraError(RuntimeError):
@@ -83,6 +84,8 @@ def _load():
     for f in (lib.qlora_quantize_input, lib.qlora_gemm_forward, lib.qlora_lora_grad_dy,
               lib.qlora_gemm_dx, lib.qlora_lora_grad_x):
         f.restype = I
+    lib.qlora_selftest_wait_timeout.argtypes = [ctypes.c_uint, P]
+    lib.qlora_selftest_wait_timeout.restype = I
     return lib
 
 
@@ -207,6 +210,10 @@ def qlora_relu(Y: torch.Tensor, stream=None):
 def qlora_relu_backward(dY: torch.Tensor, Y: torch.Tensor, stream=None):
     assert dY.shape == Y.shape and dY.dtype == Y.dtype
     _check(_lib.qlora_relu_backward(_ptr(dY), _ptr(Y), Y.numel(), act_code(Y.dtype), _stream(stream)))
+
+
+def qlora_selftest_wait_timeout(limit_us: int, stream=None):
+    _check(_lib.qlora_selftest_wait_timeout(int(limit_us), _stream(stream)))
 
 
 def qlora_device_status(stream=None) -> int:
