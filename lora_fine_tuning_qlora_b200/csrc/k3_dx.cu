@@ -9,37 +9,55 @@
 // input quantizer is passed straight through, so only the de-quantized
 // kernel and the LoRA factors enter dX.
 //
-// tcgen05 path (bf16 activations, N a multiple of 8), one 128 x BN tile of dX
-// per CTA, 10 warps:
-//   warp 0      TMA producer: dY tile [128 x 64 bf16] (128B swizzle, K-major)
-//               and the int8 kernel tile Wq[n0:n0+64, k0:k0+BN] (row-major)
-//   warp 1      TMEM allocation; tcgen05.mma.kind::f16 (bf16 in, fp32 accum),
-//               M=128, N=BN, K=16 per instruction, from one thread
-//   warps 2..9  de-quantize each int8 stage into a bf16 tile laid out as the
-//               MN-major 128B-swizzled B operand, then run the epilogue
+// tcgen05 path (bf16 activations, N a multiple of 8): persistent, one CTA
+// per SM, a tile is (128 * MSUB) rows x BN columns of dX, 18 warps:
+//   warp 0       TMA producer: MSUB dY tiles [128 x 64 bf16] (128B swizzle,
+//                K-major) and the int8 kernel tile Wq[n0:n0+64, k0:k0+BN]
+//   warp 1       TMEM owner and MMA issuer: MSUB x tcgen05.mma.kind::f16
+//                (bf16 in, fp32 accumulate), M=128, N=BN, K=16, all sharing
+//                one de-quantized B tile; two TMEM accumulators per
+//                sub-tile so tile i+1's main loop overlaps tile i's epilogue
+//   warps 2..9   de-quantize every int8 stage into a bf16 tile laid out as
+//                the MN-major 128B-swizzled B operand
+//   warps 10..17 epilogue: + c G A^T, staged coalesced stores of dX
 // SIMT path: fp32 activations, or rows of dY that the Tensor Memory
 // Accelerator cannot describe (N*2 bytes not a multiple of 16).
 #include "internal.h"
 #include "ptx.cuh"
+#include "tile_epilogue.cuh"
 
 namespace qlora {
 
 namespace {
 
-constexpr int kBM = 128;
 constexpr int kBKn = 64;  // contraction (n) per stage: one 128-byte row of bf16
 constexpr int kDqWarps = 8;
-constexpr int kThreads = 64 + 32 * kDqWarps;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * (kDqWarps + kEpiWarps);
+constexpr int kSmemLimit = 232448;
 
-template <int BN, int STAGES>
-struct K3Layout {
-    static constexpr int kABytes = kBM * kBKn * 2;     // dY tile, bf16
+template <int MSUB, int BN, int RMAX>
+struct K3Cfg {
+    static constexpr int kBM = 128 * MSUB;
+    static constexpr int kRPad = RMAX <= 16 ? ((RMAX + 3) / 4) * 4 : 0;
+    static constexpr int kASub = 128 * kBKn * 2;       // one dY sub-tile, bf16
+    static constexpr int kABytes = MSUB * kASub;
     static constexpr int kQBytes = kBKn * BN;          // int8 kernel tile
     static constexpr int kWBytes = kBKn * BN * 2;      // de-quantized bf16 tile
     static constexpr int kStageBytes = kABytes + kQBytes + kWBytes;
-    static constexpr int kBarOff = STAGES * kStageBytes;
-    static constexpr int kLoraOff = kBarOff + 256;     // A tile [BN][16]
-    static constexpr int kTotal = kLoraOff + BN * 16 * 4 + 1024;
+    static constexpr int kStgBytes = kEpiWarps * 32 * stage_pitch<__nv_bfloat16>();
+    static constexpr int kParamBytes = BN * kRPad * 4;
+    static constexpr int kFixed = kStgBytes + kParamBytes + 256 + 1024;
+    static constexpr int kStagesFit = (kSmemLimit - kFixed) / kStageBytes;
+    static constexpr int STAGES = kStagesFit > 8 ? 8 : kStagesFit;
+    static_assert(STAGES >= 2, "shared memory budget");
+    static constexpr int kStgOff = STAGES * kStageBytes;
+    static constexpr int kTabOff = kStgOff + kStgBytes;
+    static constexpr int kBarOff = kTabOff + kParamBytes;
+    static constexpr int kTotal = kBarOff + 256 + 1024;
+    static constexpr uint32_t kAccCols = MSUB * BN;     // one accumulator buffer
+    static constexpr uint32_t kTmemCols = 2 * kAccCols;
+    static_assert(kTmemCols <= 512, "TMEM");
 };
 
 // byte offset of the 16-byte chunk holding bf16 elements (mn .. mn+7, kr) in
@@ -58,49 +76,46 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-template <int BN, int STAGES, int RMAX>
+template <int MSUB, int BN, int RMAX>
 __global__ void __launch_bounds__(kThreads, 1)
     k3_dx_dequant_kernel(const __grid_constant__ CUtensorMap tmDY,
                          const __grid_constant__ CUtensorMap tmQ, const float* __restrict__ sw,
                          int M, int N, int K, DxEpilogue ep, int* status) {
-    using L = K3Layout<BN, STAGES>;
+    using C = K3Cfg<MSUB, BN, RMAX>;
+    constexpr int S = C::STAGES;
+    constexpr uint32_t kLbo = (kBKn / 8) * 1024;  // MN-block stride of the bf16 tile
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-    uint64_t* wready = full + STAGES;
-    uint64_t* empty = wready + STAGES;
-    uint64_t* tfull = empty + STAGES;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tfull + 1);
-    float* s_a = reinterpret_cast<float*>(smem + L::kLoraOff);
-    constexpr bool kStageA = RMAX <= 16;
-    constexpr uint32_t kLbo = (kBKn / 8) * 1024;  // MN-block stride of the bf16 tile
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+    uint64_t* wready = full + S;
+    uint64_t* empty = wready + S;
+    uint64_t* tfull = empty + S;   // [2]
+    uint64_t* tempty = tfull + 2;  // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+    float* s_tab = reinterpret_cast<float*>(smem + C::kTabOff);
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const int m0 = blockIdx.y * kBM;
-    const int k0 = blockIdx.x * BN;
+    const int num_k = (K + BN - 1) / BN;
+    const int tiles = ((M + C::kBM - 1) / C::kBM) * num_k;
     const int nkb = (N + kBKn - 1) / kBKn;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&wready[s], kDqWarps);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(tfull, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], kEpiWarps);
+        }
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, BN);
+        tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
-    }
-    if constexpr (kStageA) {
-        for (int i = threadIdx.x; i < BN * RMAX; i += kThreads) {
-            const int kk = i / RMAX, j = i % RMAX;
-            const int k = k0 + kk;
-            s_a[i] = (k < K && j < ep.r) ? ep.A[static_cast<size_t>(k) * ep.r + j] : 0.f;
-        }
     }
     tc_fence_before();
     __syncthreads();
@@ -108,171 +123,221 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
+        // ------------------------------------------------------ producer
         if (lane == 0) {
             tma_prefetch_desc(&tmDY);
             tma_prefetch_desc(&tmQ);
-            for (int kb = 0; kb < nkb; ++kb) {
-                const int s = kb % STAGES;
-                const int it = kb / STAGES;
-                if (kb >= STAGES && !mbar_wait(&empty[s], (it - 1) & 1, status)) break;
-                uint8_t* sa = smem + s * L::kStageBytes;
-                uint8_t* sq = sa + L::kABytes;
-                mbar_arrive_expect_tx(&full[s], L::kABytes + L::kQBytes);
-                tma_load_2d(sa, &tmDY, &full[s], kb * kBKn, m0);
-                tma_load_2d(sq, &tmQ, &full[s], k0, kb * kBKn);
-            }
-        }
-        __syncwarp();  // reconverge the warp before the teardown barrier
-    } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16(kBM, BN, false, true);
+            int g = 0;
             bool ok = true;
-            for (int kb = 0; kb < nkb; ++kb) {
-                const int s = kb % STAGES;
-                const int it = kb / STAGES;
-                if (!mbar_wait(&full[s], it & 1, status) || !mbar_wait(&wready[s], it & 1, status)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t a_base = smem_u32(smem + s * L::kStageBytes);
-                const uint32_t w_base = a_base + L::kABytes + L::kQBytes;
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                const int m0 = (t / num_k) * C::kBM;
+                const int k0 = (t % num_k) * BN;
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s = g % S;
+                    if (g >= S && !mbar_wait(&empty[s], ((g / S) - 1) & 1, status)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + s * C::kStageBytes;
+                    mbar_arrive_expect_tx(&full[s], C::kABytes + C::kQBytes);
 #pragma unroll
-                for (int kk = 0; kk < kBKn / 16; ++kk) {
-                    const uint64_t ad = smem_desc(a_base + kk * 32, 16, 1024, kLayoutSw128);
-                    const uint64_t bd = smem_desc(w_base + kk * 2048, kLbo, 1024, kLayoutSw128);
-                    mma_bf16(tmem, ad, bd, idesc, (kb | kk) != 0);
+                    for (int ms = 0; ms < MSUB; ++ms)
+                        tma_load_2d(sa + ms * C::kASub, &tmDY, &full[s], kb * kBKn, m0 + 128 * ms);
+                    tma_load_2d(sa + C::kABytes, &tmQ, &full[s], k0, kb * kBKn);
                 }
-                mma_commit(&empty[s]);
             }
-            if (ok) mma_commit(tfull);
         }
-        __syncwarp();  // reconverge the warp before the teardown barrier
-    } else {
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16(128, BN, false, true);
+            int g = 0, i = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++i) {
+                const int ab = i & 1;
+                const int use = i >> 1;
+                if (use > 0 && !mbar_wait(&tempty[ab], (use - 1) & 1, status)) break;
+                tc_fence_after();
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s = g % S;
+                    if (!mbar_wait(&full[s], (g / S) & 1, status) ||
+                        !mbar_wait(&wready[s], (g / S) & 1, status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(smem + s * C::kStageBytes);
+                    const uint32_t w_base = a_base + C::kABytes + C::kQBytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBKn / 16; ++kk) {
+                        const uint64_t bd = smem_desc(w_base + kk * 2048, kLbo, 1024, kLayoutSw128);
+#pragma unroll
+                        for (int ms = 0; ms < MSUB; ++ms) {
+                            const uint64_t ad = smem_desc(a_base + ms * C::kASub + kk * 32, 16, 1024,
+                                                          kLayoutSw128);
+                            mma_bf16(tmem + ab * C::kAccCols + ms * BN, ad, bd, idesc, (kb | kk) != 0);
+                        }
+                    }
+                    mma_commit(&empty[s]);
+                }
+                if (ok) mma_commit(&tfull[ab]);
+            }
+        }
+        __syncwarp();
+    } else if (warp < 2 + kDqWarps) {
+        // ------------------------------------------------------ de-quantize
         const int dq = threadIdx.x - 64;  // 0 .. 255
-        // ---- de-quantize every stage into the MN-major swizzled bf16 tile ----
         constexpr int kChunksPerRow = BN / 16;
         constexpr int kChunks = kBKn * kChunksPerRow;
+        int g = 0;
         bool ok = true;
-        for (int kb = 0; kb < nkb && ok; ++kb) {
-            const int s = kb % STAGES;
-            const int it = kb / STAGES;
-            ok = __all_sync(0xffffffffu, mbar_wait(&full[s], it & 1, status));
-            if (!ok) break;
-            const uint8_t* sq = smem + s * L::kStageBytes + L::kABytes;
-            uint8_t* sw_tile = smem + s * L::kStageBytes + L::kABytes + L::kQBytes;
+        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            for (int kb = 0; kb < nkb; ++kb, ++g) {
+                const int s = g % S;
+                ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (g / S) & 1, status));
+                if (!ok) break;
+                const uint8_t* sq = smem + s * C::kStageBytes + C::kABytes;
+                uint8_t* wt = smem + s * C::kStageBytes + C::kABytes + C::kQBytes;
 #pragma unroll
-            for (int c = dq; c < kChunks; c += 32 * kDqWarps) {
-                const int nr = c / kChunksPerRow;   // contraction row within the stage
-                const int kc = c % kChunksPerRow;   // 16 output columns
-                const int n = kb * kBKn + nr;
-                const float scale = n < N ? __ldg(sw + n) : 0.f;
-                const uint4 raw = *reinterpret_cast<const uint4*>(sq + nr * BN + kc * 16);
-                const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-                uint32_t o[8];
+                for (int c = dq; c < kChunks; c += 32 * kDqWarps) {
+                    const int nr = c / kChunksPerRow;   // contraction row within the stage
+                    const int kc = c % kChunksPerRow;   // 16 output columns
+                    const int n = kb * kBKn + nr;
+                    const float scale = n < N ? __ldg(sw + n) : 0.f;
+                    const uint4 raw = *reinterpret_cast<const uint4*>(sq + nr * BN + kc * 16);
+                    const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+                    uint32_t o[8];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int32_t b = static_cast<int32_t>(w4[i]);
-                    const float f0 = __fmul_rn(static_cast<float>((b << 24) >> 24), scale);
-                    const float f1 = __fmul_rn(static_cast<float>((b << 16) >> 24), scale);
-                    const float f2 = __fmul_rn(static_cast<float>((b << 8) >> 24), scale);
-                    const float f3 = __fmul_rn(static_cast<float>(b >> 24), scale);
-                    o[2 * i] = pack_bf16x2(f0, f1);
-                    o[2 * i + 1] = pack_bf16x2(f2, f3);
+                    for (int i = 0; i < 4; ++i) {
+                        const int32_t b = static_cast<int32_t>(w4[i]);
+                        const float f0 = __fmul_rn(static_cast<float>((b << 24) >> 24), scale);
+                        const float f1 = __fmul_rn(static_cast<float>((b << 16) >> 24), scale);
+                        const float f2 = __fmul_rn(static_cast<float>((b << 8) >> 24), scale);
+                        const float f3 = __fmul_rn(static_cast<float>(b >> 24), scale);
+                        o[2 * i] = pack_bf16x2(f0, f1);
+                        o[2 * i + 1] = pack_bf16x2(f2, f3);
+                    }
+                    const int mn = kc * 16;
+                    *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn, nr, kLbo)) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn + 8, nr, kLbo)) =
+                        make_uint4(o[4], o[5], o[6], o[7]);
                 }
-                const int mn = kc * 16;
-                *reinterpret_cast<uint4*>(sw_tile + mn_sw128_offset(mn, nr, kLbo)) =
-                    make_uint4(o[0], o[1], o[2], o[3]);
-                *reinterpret_cast<uint4*>(sw_tile + mn_sw128_offset(mn + 8, nr, kLbo)) =
-                    make_uint4(o[4], o[5], o[6], o[7]);
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&wready[s]);
-        }
-        // ---- epilogue ----
-        const int q = warp & 3;
-        const int half = (warp - 2) / 4;
-        const int row = m0 + q * 32 + lane;
-        const bool row_ok = row < M;
-        float g[RMAX];
-#pragma unroll
-        for (int j = 0; j < RMAX; ++j)
-            g[j] = (row_ok && j < ep.r) ? ep.G[static_cast<size_t>(row) * ep.r + j] * ep.c : 0.f;
-        ok = __all_sync(0xffffffffu, ok && mbar_wait(tfull, 0, status));
-        tc_fence_after();
-        if (ok) {
-            __nv_bfloat16* drow =
-                static_cast<__nv_bfloat16*>(ep.dX) + static_cast<size_t>(row_ok ? row : 0) * K;
-#pragma unroll 1
-            for (int col = half * (BN / 2); col < (half + 1) * (BN / 2); col += 16) {
-                uint32_t v[16];
+                fence_proxy_async_smem();
                 __syncwarp();
-                tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + col, v);
-                tmem_ld_wait();
-                if (row_ok) {
-                    float outv[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int kl = col + i;
-                        const int k = k0 + kl;
-                        float l = 0.f;
-#pragma unroll
-                        for (int j = 0; j < RMAX; ++j) {
-                            if (j < ep.r) {
-                                const float a = kStageA ? s_a[kl * RMAX + j]
-                                                        : (k < K ? __ldg(ep.A + static_cast<size_t>(k) * ep.r + j) : 0.f);
-                                l = fmaf(g[j], a, l);
-                            }
-                        }
-                        outv[i] = __uint_as_float(v[i]) + l;
-                    }
-                    const int kbase = k0 + col;
-                    if (kbase + 16 <= K) {
-                        uint4 p0 = make_uint4(pack_bf16x2(outv[0], outv[1]), pack_bf16x2(outv[2], outv[3]),
-                                              pack_bf16x2(outv[4], outv[5]), pack_bf16x2(outv[6], outv[7]));
-                        uint4 p1 = make_uint4(pack_bf16x2(outv[8], outv[9]), pack_bf16x2(outv[10], outv[11]),
-                                              pack_bf16x2(outv[12], outv[13]), pack_bf16x2(outv[14], outv[15]));
-                        *reinterpret_cast<uint4*>(drow + kbase) = p0;
-                        *reinterpret_cast<uint4*>(drow + kbase + 8) = p1;
-                    } else {
-                        for (int i = 0; i < 16; ++i)
-                            if (kbase + i < K) drow[kbase + i] = __float2bfloat16_rn(outv[i]);
-                    }
-                }
+                if (lane == 0) mbar_arrive(&wready[s]);
             }
         }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------ epilogue
+        const int ew = warp - 2 - kDqWarps;  // 0 .. 7
+        const int q = warp & 3;              // TMEM lane quarter of this warp
+        const int sub = ew >> 2;             // MSUB == 2: row sub-tile, else column half
+        const int et = threadIdx.x - 64 - 32 * kDqWarps;
+        uint8_t* stg = smem + C::kStgOff + ew * 32 * stage_pitch<__nv_bfloat16>();
+        __nv_bfloat16* dX = static_cast<__nv_bfloat16*>(ep.dX);
+        int i = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+            const int ab = i & 1;
+            const int use = i >> 1;
+            const int m0 = (t / num_k) * C::kBM;
+            const int k0 = (t % num_k) * BN;
+            if constexpr (C::kRPad > 0) {
+                named_bar_sync(1, 32 * kEpiWarps);
+                for (int e = et; e < BN * C::kRPad; e += 32 * kEpiWarps) {
+                    const int c = e / C::kRPad, j = e % C::kRPad;
+                    const int k = k0 + c;
+                    s_tab[e] = (k < K && j < ep.r) ? ep.A[static_cast<size_t>(k) * ep.r + j] : 0.f;
+                }
+                named_bar_sync(1, 32 * kEpiWarps);
+            }
+            const int msub = MSUB == 2 ? sub : 0;
+            const int row0 = m0 + msub * 128 + q * 32;
+            const int row = row0 + lane;
+            const bool row_ok = row < M;
+            float gr[RMAX];
+#pragma unroll
+            for (int j = 0; j < RMAX; ++j)
+                gr[j] = (row_ok && j < ep.r) ? ep.G[static_cast<size_t>(row) * ep.r + j] * ep.c : 0.f;
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[ab], use & 1, status));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * C::kAccCols +
+                                   msub * BN;
+            const int cbeg = MSUB == 2 ? 0 : sub * (BN / 2);
+            const int cend = MSUB == 2 ? BN : (sub + 1) * (BN / 2);
+#pragma unroll 1
+            for (int col = cbeg; col < cend; col += kEpiCols) {
+                uint32_t v[kEpiCols];
+                tmem_ld16(tbase + col, v);
+                tmem_ld_wait();
+                float y[kEpiCols];
+#pragma unroll
+                for (int e = 0; e < kEpiCols; ++e) {
+                    const int c = col + e;
+                    float acc = __uint_as_float(v[e]);
+                    if constexpr (C::kRPad > 0) {
+                        const float4* tb = reinterpret_cast<const float4*>(s_tab + c * C::kRPad);
+#pragma unroll
+                        for (int j4 = 0; j4 < C::kRPad / 4; ++j4) {
+                            const float4 a4 = tb[j4];
+                            acc = fmaf(gr[4 * j4], a4.x, acc);
+                            if (4 * j4 + 1 < RMAX) acc = fmaf(gr[4 * j4 + 1], a4.y, acc);
+                            if (4 * j4 + 2 < RMAX) acc = fmaf(gr[4 * j4 + 2], a4.z, acc);
+                            if (4 * j4 + 3 < RMAX) acc = fmaf(gr[4 * j4 + 3], a4.w, acc);
+                        }
+                    } else {
+                        const int k = k0 + c;
+                        if (k < K)
+                            for (int j = 0; j < ep.r; ++j)
+                                acc = fmaf(gr[j], __ldg(ep.A + static_cast<size_t>(k) * ep.r + j), acc);
+                    }
+                    y[e] = acc;
+                }
+                store_block<__nv_bfloat16>(stg, y, lane, dX, static_cast<size_t>(K), row0, M, k0 + col,
+                                           K, true);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[ab]);
+        }
+        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, BN);
+        tmem_dealloc(tmem, C::kTmemCols);
     }
 }
 
-template <int BN, int STAGES, int RMAX>
+template <int MSUB, int BN, int RMAX>
 cudaError_t launch_tc(const CUtensorMap& tdy, const CUtensorMap& tq, const float* sw, int M, int N,
                       int K, const DxEpilogue& ep, int* status, cudaStream_t s) {
-    using L = K3Layout<BN, STAGES>;
-    auto kern = k3_dx_dequant_kernel<BN, STAGES, RMAX>;
-    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), L::kTotal);
+    using C = K3Cfg<MSUB, BN, RMAX>;
+    auto kern = k3_dx_dequant_kernel<MSUB, BN, RMAX>;
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), C::kTotal);
     if (e != cudaSuccess) return e;
-    dim3 grid((K + BN - 1) / BN, (M + kBM - 1) / kBM);
-    kern<<<grid, kThreads, L::kTotal, s>>>(tdy, tq, sw, M, N, K, ep, status);
+    const int tiles = ((M + C::kBM - 1) / C::kBM) * ((K + BN - 1) / BN);
+    const int grid = tiles < sm_count() ? tiles : sm_count();
+    kern<<<grid, kThreads, C::kTotal, s>>>(tdy, tq, sw, M, N, K, ep, status);
     return cudaGetLastError();
 }
 
 template <int RMAX>
-cudaError_t launch_tc_bn(int bn, const CUtensorMap& tdy, const CUtensorMap& tq, const float* sw,
-                         int M, int N, int K, const DxEpilogue& ep, int* status, cudaStream_t s) {
-    if (bn == 256) return launch_tc<256, 3, RMAX>(tdy, tq, sw, M, N, K, ep, status, s);
-    return launch_tc<128, 5, RMAX>(tdy, tq, sw, M, N, K, ep, status, s);
+cudaError_t launch_tc_cfg(int cfg, const CUtensorMap& tdy, const CUtensorMap& tq, const float* sw,
+                          int M, int N, int K, const DxEpilogue& ep, int* status, cudaStream_t s) {
+    if (cfg == 0) return launch_tc<2, 128, RMAX>(tdy, tq, sw, M, N, K, ep, status, s);
+    if (cfg == 1) return launch_tc<1, 128, RMAX>(tdy, tq, sw, M, N, K, ep, status, s);
+    return launch_tc<1, 64, RMAX>(tdy, tq, sw, M, N, K, ep, status, s);
 }
 
 // ---------------------------------------------------------------- SIMT path
 // 64 x 64 tile of dX per CTA, 256 threads (4 x 4 outputs each), n in steps of
-// 16 through shared memory; the kernel tile is de-quantized to fp32 on load.
+// 16 through shared memory; the kernel tile is de-quantized on load, to fp32
+// (fp32 activations) or rounded on to bf16 (bf16 activations).
 constexpr int kSB = 64;
 constexpr int kSN = 16;
 
@@ -295,9 +360,12 @@ __global__ void __launch_bounds__(256) k3_dx_simt_kernel(const T* __restrict__ d
         for (int i = threadIdx.x; i < kSN * kSB; i += 256) {
             const int nn = i / kSB, kk = i % kSB;
             const int n = n0 + nn, k = k0 + kk;
-            sW[nn][kk] = (n < N && k < K)
-                             ? __fmul_rn(static_cast<float>(Wq[static_cast<size_t>(n) * K + k]), __ldg(sw + n))
-                             : 0.f;
+            float w = 0.f;
+            if (n < N && k < K) {
+                w = __fmul_rn(static_cast<float>(Wq[static_cast<size_t>(n) * K + k]), __ldg(sw + n));
+                if constexpr (sizeof(T) == 2) w = __bfloat162float(__float2bfloat16_rn(w));
+            }
+            sW[nn][kk] = w;
         }
         __syncthreads();
 #pragma unroll
@@ -346,19 +414,24 @@ cudaError_t launch_gemm_dx(Act act, const void* dY, const int8_t* Wq, const floa
                                                           K, ep);
         return cudaGetLastError();
     }
-    const int mt = (M + kBM - 1) / kBM;
-    const int bn = (mt * ((K + 255) / 256) >= 148) ? 256 : 128;
+    // tile shape: the largest that still gives every SM a tile
+    const int sms = sm_count();
+    auto ntiles = [&](int bm, int bn) { return ((M + bm - 1) / bm) * ((K + bn - 1) / bn); };
+    int cfg = 2;
+    if (ntiles(256, 128) >= sms) cfg = 0;
+    else if (ntiles(128, 128) >= sms) cfg = 1;
+    const int bn = cfg == 2 ? 64 : 128;
     CUtensorMap tdy, tq;
     if (!make_tmap_2d(&tdy, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N,
-                      static_cast<uint64_t>(N) * 2, kBM, kBKn, CU_TENSOR_MAP_SWIZZLE_128B))
+                      static_cast<uint64_t>(N) * 2, 128, kBKn, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     if (!make_tmap_2d(&tq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, kBKn, bn,
                       CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    if (ep.r <= 4) return launch_tc_bn<4>(bn, tdy, tq, sw, M, N, K, ep, status, s);
-    if (ep.r <= 8) return launch_tc_bn<8>(bn, tdy, tq, sw, M, N, K, ep, status, s);
-    if (ep.r <= 16) return launch_tc_bn<16>(bn, tdy, tq, sw, M, N, K, ep, status, s);
-    return launch_tc_bn<64>(bn, tdy, tq, sw, M, N, K, ep, status, s);
+    if (ep.r <= 4) return launch_tc_cfg<4>(cfg, tdy, tq, sw, M, N, K, ep, status, s);
+    if (ep.r <= 8) return launch_tc_cfg<8>(cfg, tdy, tq, sw, M, N, K, ep, status, s);
+    if (ep.r <= 16) return launch_tc_cfg<16>(cfg, tdy, tq, sw, M, N, K, ep, status, s);
+    return launch_tc_cfg<64>(cfg, tdy, tq, sw, M, N, K, ep, status, s);
 }
 
 }  // namespace qlora
