@@ -161,23 +161,27 @@ int qlora_gemm_forward(const qlora_layer_desc* d, int M, const int8_t* Xq, const
                        const int8_t* Wq, const float* sw, const float* bias, const float* xA,
                        const float* B, void* Y, int32_t* acc, void* stream);
 
-/* a3: one pass over dY: G = dY B^T [M,r], dB = c * xA^T dY [r,N] and, if
- * dbias is not NULL, dbias = column sums of dY [N].  Deterministic.  Needs
- * the workspace (qlora_workspace_bytes) for its partial sums. */
+/* a3: one pass over dY: dB = c * xA^T dY [r,N] and, if dbias is not NULL,
+ * dbias = column sums of dY [N]; G = dY B^T is left in the workspace (as
+ * per-column-block slices) for the a4 and a5 calls that follow on the same
+ * workspace, with no forward call on that workspace in between.  If G is
+ * not NULL, the summed G [M,r] is also written there.  Deterministic. */
 int qlora_lora_grad_dy(const qlora_layer_desc* d, int M, const void* dY, const float* B,
-                       const float* xA, float* G, float* dB, float* dbias, void* workspace,
+                       const float* xA, float* dB, float* dbias, float* G, void* workspace,
                        size_t workspace_bytes, void* stream);
 
-/* a4: dX = dY (Wq * sw)^T + c * G A^T [M,K]; the int8 kernel is de-quantized
- * tile by tile in shared memory ("How to fine-tune the 4-bit model?":
- * de-quantize in place before the matrix unit). */
+/* a4: dX = dY (Wq * sw)^T + c * G A^T [M,K], G from the workspace that a3
+ * filled; the int8 kernel is de-quantized tile by tile in shared memory
+ * ("How to fine-tune the 4-bit model?": de-quantize in place before the
+ * matrix unit). */
 int qlora_gemm_dx(const qlora_layer_desc* d, int M, const void* dY, const int8_t* Wq,
-                  const float* sw, const float* G, const float* A, void* dX, void* stream);
+                  const float* sw, const float* A, void* dX, const void* workspace,
+                  size_t workspace_bytes, void* stream);
 
-/* a5: one pass over X: dA = c * X^T G [K,r].  Deterministic.  Needs the
- * workspace for its partial sums. */
-int qlora_lora_grad_x(const qlora_layer_desc* d, int M, const void* X, const float* G, float* dA,
-                      void* workspace, size_t workspace_bytes, void* stream);
+/* a5: one pass over X: dA = c * X^T G [K,r], G from the workspace that a3
+ * filled.  Deterministic. */
+int qlora_lora_grad_x(const qlora_layer_desc* d, int M, const void* X, float* dA,
+                      const void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Lossy merge ("Introduce QLoRA-like technique", Results footnote: merging

@@ -37,7 +37,8 @@ cudaError_t launch_gemm_i8_fwd(Act act, const int8_t* Xq, const int8_t* Wq, int 
 
 // ---------------------------------------------------------------- K3
 struct DxEpilogue {
-    const float* G;   // [M,r]
+    const float* Gp;  // [ncb][M,r] slices of G = dY B^T (G = sum of the slices)
+    int ncb;
     const float* A;   // [K,r]
     int r;
     float c;
@@ -48,23 +49,19 @@ cudaError_t launch_gemm_dx(Act act, const void* dY, const int8_t* Wq, const floa
                            int N, int K, const DxEpilogue& ep, int* status, cudaStream_t s);
 
 // ---------------------------------------------------------------- K4
-struct RankPlan {
-    int rows_per_chunk;  // RM
-    int n_chunks;        // ceil(M / RM)
-    int n_col_blocks;    // ceil(N / 256), G partial slices
-    int k_chunks;        // chunks for the pass over X
-    int rows_per_kchunk;
-};
-RankPlan plan_rank(int M, int K, int N, int r);
-size_t rank_workspace_floats(const RankPlan& p, int M, int K, int N, int r);
+// Column blocks of the passes (= number of G slices for N columns).
+int rank_col_blocks(int N);
+// fp32 workspace of the G slices: rank_col_blocks(N) * M * r.
+size_t rank_workspace_floats(int M, int N, int r);
 
-// Pass over dY: G, dB, dbias (with its deterministic reductions) and the
-// pass over X: dA.  `wsf` is fp32 scratch of rank_workspace_floats() floats.
+// Pass over dY: G slices into Gp, final dB and dbias (dbias may be null),
+// and, when G is not null, the summed G [M,r] as well.
 cudaError_t launch_rank_dy(Act act, const void* dY, const float* B, const float* xA, int M, int N,
-                           int r, float c, const RankPlan& p, float* G, float* dB, float* dbias,
-                           float* wsf, cudaStream_t s);
-cudaError_t launch_rank_x(Act act, const void* X, const float* G, int M, int K, int r, float c,
-                          const RankPlan& p, float* dA, float* wsf, cudaStream_t s);
+                           int r, float c, float* Gp, float* dB, float* dbias, float* G,
+                           cudaStream_t s);
+// Pass over X: final dA from X and the ncb G slices.
+cudaError_t launch_rank_x(Act act, const void* X, const float* Gp, int ncb, int M, int K, int r,
+                          float c, float* dA, cudaStream_t s);
 
 // ---------------------------------------------------------------- KM
 cudaError_t launch_merge(const int8_t* Wq, const float* sw, const float* A, const float* B, int K,
@@ -84,6 +81,13 @@ cudaError_t launch_selftest_wait(int* status, unsigned long long limit_ns, cudaS
 bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem_bytes,
                   uint64_t rows, uint64_t cols, uint64_t pitch_bytes, uint32_t box_rows,
                   uint32_t box_cols, CUtensorMapSwizzle swizzle);
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+// Tile-shape override for tuning sweeps: the integer value of environment
+// variable `name`, read once, or -1 when it is unset.
+int tile_override(const char* name);
 
 // Sets the dynamic shared memory limit of `func` once per device.
 cudaError_t ensure_smem_attr(const void* func, int bytes);

@@ -9,7 +9,10 @@
 // ("Parameter-efficient fine-tuning of GPT-2 with LoRA", "LoRA equation").
 //
 // K1 is HBM-bound: it reads M*K*e bytes of X once (128-bit loads held in
-// registers), writes M*K int8 codes, M scales and M*r floats of xA.
+// registers), writes M*K int8 codes, M scales and M*r floats of xA.  The
+// LoRA factor A [K,r] is staged in shared memory once per CTA (padded so that
+// the 8-row slices the lanes read are bank-conflict free) and the CTA then
+// walks over many row groups, so A is read from L2 once per CTA, not per row.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -18,9 +21,9 @@ namespace qlora {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kChunk = 8;   // elements per 128-bit (bf16) / 2x128-bit (f32) load
-constexpr int kMaxCPT = 8;  // chunks per thread held in registers
-constexpr int kRJ = 8;      // xA columns accumulated per sweep
+constexpr int kChunk = 8;    // elements per 128-bit (bf16) / 2x128-bit (f32) load
+constexpr int kMaxCPT = 8;   // chunks per thread held in registers
+constexpr int kSmemCap = 200 * 1024;
 
 template <typename T>
 struct Chunk8;
@@ -58,7 +61,66 @@ __device__ __forceinline__ uint2 pack8(const float (&v)[8], float inv) {
     return make_uint2(lo, hi);
 }
 
-// Reduction over the TPR threads that share a row (TPR in {32,64,128,256}).
+// Floats of the staged A slice for `chunks` 8-row chunks: each chunk holds
+// 8 rows of RP floats followed by 4 floats of padding.
+template <int RP>
+__host__ __device__ constexpr int a_chunk_floats() { return 8 * RP + 4; }
+
+// Stages A rows [k0, k0 + 8*chunks) into shared memory (zero outside K / r).
+template <int RP>
+__device__ __forceinline__ void stage_a(float* sA, const float* __restrict__ A, int K, int r,
+                                        int k0, int chunks) {
+    if (r == RP && (reinterpret_cast<uintptr_t>(A) & 15) == 0) {
+        // rows of A are RP floats: copy 16-byte vectors, four in flight per thread
+        constexpr int V = 2 * RP;  // float4 per 8-row chunk
+        const int n4 = chunks * V;
+        const int kmax4 = (K - k0) * RP / 4;  // float4 that lie inside A
+        const float4* src = reinterpret_cast<const float4*>(A + static_cast<size_t>(k0) * RP);
+        float4* dst = reinterpret_cast<float4*>(sA);
+        for (int base = threadIdx.x; base < n4; base += 4 * blockDim.x) {
+            float4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int idx = base + u * blockDim.x;
+                v[u] = (idx < n4 && idx < kmax4) ? __ldg(src + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int idx = base + u * blockDim.x;
+                if (idx < n4) dst[(idx / V) * (V + 1) + idx % V] = v[u];
+            }
+        }
+        return;
+    }
+    const int n = chunks * 8 * RP;
+    for (int idx = threadIdx.x; idx < n; idx += blockDim.x) {
+        const int kl = idx / RP, j = idx % RP;
+        const int k = k0 + kl;
+        sA[(kl >> 3) * a_chunk_floats<RP>() + (kl & 7) * RP + j] =
+            (k < K && j < r) ? __ldg(A + static_cast<size_t>(k) * r + j) : 0.f;
+    }
+}
+
+// acc[j] += sum_e v[e] * A[chunk row e, j] with the chunk's rows in shared memory.
+template <int RP>
+__device__ __forceinline__ void chunk_fma(const float* sA_chunk, const float (&v)[8],
+                                          float (&acc)[RP]) {
+    const float4* a4 = reinterpret_cast<const float4*>(sA_chunk);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+#pragma unroll
+        for (int j4 = 0; j4 < RP / 4; ++j4) {
+            const float4 a = a4[e * (RP / 4) + j4];
+            acc[4 * j4 + 0] = fmaf(v[e], a.x, acc[4 * j4 + 0]);
+            acc[4 * j4 + 1] = fmaf(v[e], a.y, acc[4 * j4 + 1]);
+            acc[4 * j4 + 2] = fmaf(v[e], a.z, acc[4 * j4 + 2]);
+            acc[4 * j4 + 3] = fmaf(v[e], a.w, acc[4 * j4 + 3]);
+        }
+    }
+}
+
+// Sum (or max) over the TPR threads that share a row (TPR in {32,64,128,256}).
+// `red` holds kThreads/32 floats per call site.
 template <int TPR, bool IS_MAX>
 __device__ __forceinline__ float row_reduce(float v, float* red, int row_in_block, int t) {
 #pragma unroll
@@ -68,7 +130,6 @@ __device__ __forceinline__ float row_reduce(float v, float* red, int row_in_bloc
     }
     if constexpr (TPR > 32) {
         constexpr int W = TPR / 32;
-        __syncwarp();
         if ((t & 31) == 0) red[row_in_block * W + (t >> 5)] = v;
         __syncthreads();
         float s = red[row_in_block * W];
@@ -83,78 +144,102 @@ __device__ __forceinline__ float row_reduce(float v, float* red, int row_in_bloc
     return v;
 }
 
-// One row per TPR threads; the row is read once into registers (K <= TPR*64).
-template <typename T, int TPR>
+// TPR threads per row, 256/TPR rows per group; the CTA walks row groups
+// blockIdx.x, blockIdx.x + gridDim.x, ...  A is staged once if it fits
+// (a_chunks >= number of chunks of a row), else in slices of a_chunks.
+template <typename T, int TPR, int RP>
 __global__ void __launch_bounds__(kThreads) k1_quantize_rows_kernel(
-    const T* __restrict__ X, const float* __restrict__ A, int M, int K, int r,
+    const T* __restrict__ X, const float* __restrict__ A, int M, int K, int r, int a_chunks,
     int8_t* __restrict__ Xq, float* __restrict__ sx, float* __restrict__ xA) {
     constexpr int RPB = kThreads / TPR;
-    __shared__ float red[RPB * (TPR / 32 > 0 ? TPR / 32 : 1)];
+    extern __shared__ float4 smem_f4[];
+    float* sA = reinterpret_cast<float*>(smem_f4);
+    __shared__ float red[kThreads / 32];
     const int row_in_block = threadIdx.x / TPR;
     const int t = threadIdx.x % TPR;
-    const int m = blockIdx.x * RPB + row_in_block;
-    const bool live = m < M;
     const int nchunks = K / kChunk;
-    const T* xr = X + static_cast<size_t>(live ? m : 0) * K;
+    const int groups = (M + RPB - 1) / RPB;
+    const bool whole_a = a_chunks >= nchunks;
+    bool staged = false;
 
-    float v[kMaxCPT][8];
-    float amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < kMaxCPT; ++i) {
-        const int ch = t + i * TPR;
-        if (live && ch < nchunks) {
-            Chunk8<T>::load(xr + ch * kChunk, v[i]);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[i][e]));
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[i][e] = 0.f;
-        }
-    }
-    amax = row_reduce<TPR, true>(amax, red, row_in_block, t);
-    const float inv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
+    for (int grp = blockIdx.x; grp < groups; grp += gridDim.x) {
+        const int m = grp * RPB + row_in_block;
+        const bool live = m < M;
+        const T* xr = X + static_cast<size_t>(live ? m : 0) * K;
 
-    if (live) {
-        int8_t* qr = Xq + static_cast<size_t>(m) * K;
-#pragma unroll
-        for (int i = 0; i < kMaxCPT; ++i) {
-            const int ch = t + i * TPR;
-            if (ch < nchunks) *reinterpret_cast<uint2*>(qr + ch * kChunk) = pack8(v[i], inv);
-        }
-        if (t == 0) sx[m] = __fdiv_rn(amax, 127.0f);
-    }
-
-    // xA[m, j] = sum_k X[m,k] A[k,j], kRJ columns per sweep over the registers.
-    for (int j0 = 0; j0 < r; j0 += kRJ) {
-        float acc[kRJ];
-#pragma unroll
-        for (int j = 0; j < kRJ; ++j) acc[j] = 0.f;
+        // the row's loads go out first; A is staged while they are in flight
+        float v[kMaxCPT][8];
 #pragma unroll
         for (int i = 0; i < kMaxCPT; ++i) {
             const int ch = t + i * TPR;
             if (live && ch < nchunks) {
+                Chunk8<T>::load(xr + ch * kChunk, v[i]);
+            } else {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float* ar = A + static_cast<size_t>(ch * kChunk + e) * r + j0;
+                for (int e = 0; e < 8; ++e) v[i][e] = 0.f;
+            }
+        }
+        if (whole_a && !staged) {
+            stage_a<RP>(sA, A, K, r, 0, nchunks);
+            __syncthreads();
+            staged = true;
+        }
+        float amax = 0.f;
 #pragma unroll
-                    for (int j = 0; j < kRJ; ++j)
-                        if (j0 + j < r) acc[j] = fmaf(v[i][e], __ldg(ar + j), acc[j]);
+        for (int i = 0; i < kMaxCPT; ++i)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[i][e]));
+        amax = row_reduce<TPR, true>(amax, red, row_in_block, t);
+        const float inv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
+        if (live) {
+            int8_t* qr = Xq + static_cast<size_t>(m) * K;
+#pragma unroll
+            for (int i = 0; i < kMaxCPT; ++i) {
+                const int ch = t + i * TPR;
+                if (ch < nchunks) *reinterpret_cast<uint2*>(qr + ch * kChunk) = pack8(v[i], inv);
+            }
+            if (t == 0) sx[m] = __fdiv_rn(amax, 127.0f);
+        }
+
+        // xA[m, :] = X[m, :] . A
+        float acc[RP];
+#pragma unroll
+        for (int j = 0; j < RP; ++j) acc[j] = 0.f;
+        if (whole_a) {
+#pragma unroll
+            for (int i = 0; i < kMaxCPT; ++i) {
+                const int ch = t + i * TPR;
+                if (live && ch < nchunks) chunk_fma<RP>(sA + ch * a_chunk_floats<RP>(), v[i], acc);
+            }
+        } else {
+            for (int c0 = 0; c0 < nchunks; c0 += a_chunks) {
+                __syncthreads();
+                stage_a<RP>(sA, A, K, r, c0 * kChunk, a_chunks);
+                __syncthreads();
+#pragma unroll
+                for (int i = 0; i < kMaxCPT; ++i) {
+                    const int ch = t + i * TPR;
+                    if (live && ch < nchunks && ch >= c0 && ch < c0 + a_chunks)
+                        chunk_fma<RP>(sA + (ch - c0) * a_chunk_floats<RP>(), v[i], acc);
                 }
             }
         }
 #pragma unroll
-        for (int j = 0; j < kRJ; ++j) {
-            float s = row_reduce<TPR, false>(acc[j], red, row_in_block, t);
-            if (live && t == 0 && j0 + j < r) xA[static_cast<size_t>(m) * r + j0 + j] = s;
+        for (int j = 0; j < RP; ++j) {
+            const float s = row_reduce<TPR, false>(acc[j], red, row_in_block, t);
+            if (live && t == 0 && j < r) xA[static_cast<size_t>(m) * r + j] = s;
         }
     }
 }
 
-// Rows longer than 256*64 elements: two sweeps over global memory.
-template <typename T>
+// Rows longer than 256*64 elements: one CTA per row, two sweeps over global
+// memory (abs-max, then quantize + x.A), A staged in slices.
+template <typename T, int RP>
 __global__ void __launch_bounds__(kThreads) k1_quantize_rows_long_kernel(
-    const T* __restrict__ X, const float* __restrict__ A, int M, int K, int r,
+    const T* __restrict__ X, const float* __restrict__ A, int M, int K, int r, int a_chunks,
     int8_t* __restrict__ Xq, float* __restrict__ sx, float* __restrict__ xA) {
+    extern __shared__ float4 smem_f4[];
+    float* sA = reinterpret_cast<float*>(smem_f4);
     __shared__ float red[kThreads / 32];
     const int m = blockIdx.x;
     const int t = threadIdx.x;
@@ -170,57 +255,79 @@ __global__ void __launch_bounds__(kThreads) k1_quantize_rows_long_kernel(
     amax = row_reduce<kThreads, true>(amax, red, 0, t);
     const float inv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
     int8_t* qr = Xq + static_cast<size_t>(m) * K;
-    for (int ch = t; ch < nchunks; ch += kThreads) {
-        float v[8];
-        Chunk8<T>::load(xr + ch * kChunk, v);
-        *reinterpret_cast<uint2*>(qr + ch * kChunk) = pack8(v, inv);
-    }
-    if (t == 0) sx[m] = __fdiv_rn(amax, 127.0f);
-    for (int j0 = 0; j0 < r; j0 += kRJ) {
-        float acc[kRJ];
+    float acc[RP];
 #pragma unroll
-        for (int j = 0; j < kRJ; ++j) acc[j] = 0.f;
-        for (int ch = t; ch < nchunks; ch += kThreads) {
+    for (int j = 0; j < RP; ++j) acc[j] = 0.f;
+    for (int c0 = 0; c0 < nchunks; c0 += a_chunks) {
+        __syncthreads();
+        stage_a<RP>(sA, A, K, r, c0 * kChunk, a_chunks);
+        __syncthreads();
+        for (int ch = c0 + t; ch < c0 + a_chunks && ch < nchunks; ch += kThreads) {
             float v[8];
             Chunk8<T>::load(xr + ch * kChunk, v);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float* ar = A + static_cast<size_t>(ch * kChunk + e) * r + j0;
-#pragma unroll
-                for (int j = 0; j < kRJ; ++j)
-                    if (j0 + j < r) acc[j] = fmaf(v[e], __ldg(ar + j), acc[j]);
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < kRJ; ++j) {
-            float s = row_reduce<kThreads, false>(acc[j], red, 0, t);
-            if (t == 0 && j0 + j < r) xA[static_cast<size_t>(m) * r + j0 + j] = s;
+            *reinterpret_cast<uint2*>(qr + ch * kChunk) = pack8(v, inv);
+            chunk_fma<RP>(sA + (ch - c0) * a_chunk_floats<RP>(), v, acc);
         }
     }
+    if (t == 0) sx[m] = __fdiv_rn(amax, 127.0f);
+#pragma unroll
+    for (int j = 0; j < RP; ++j) {
+        const float s = row_reduce<kThreads, false>(acc[j], red, 0, t);
+        if (t == 0 && j < r) xA[static_cast<size_t>(m) * r + j] = s;
+    }
+}
+
+template <typename T, int TPR, int RP>
+cudaError_t launch_tpr(const T* X, const float* A, int M, int K, int r, int8_t* Xq, float* sx,
+                       float* xA, cudaStream_t s) {
+    const int nchunks = K / kChunk;
+    const int cap_chunks = kSmemCap / (a_chunk_floats<RP>() * 4);
+    const int a_chunks = nchunks <= cap_chunks ? nchunks : cap_chunks;
+    const int smem = a_chunks * a_chunk_floats<RP>() * 4;
+    auto kern = k1_quantize_rows_kernel<T, TPR, RP>;
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), kSmemCap);
+    if (e != cudaSuccess) return e;
+    constexpr int RPB = kThreads / TPR;
+    const int groups = (M + RPB - 1) / RPB;
+    // whole A staged once: persistent over row groups; else one group per CTA
+    const int per_sm = smem <= 48 * 1024 ? 4 : (smem <= 100 * 1024 ? 2 : 1);
+    int grid = groups;
+    if (a_chunks >= nchunks && grid > per_sm * sm_count()) grid = per_sm * sm_count();
+    kern<<<grid, kThreads, smem, s>>>(X, A, M, K, r, a_chunks, Xq, sx, xA);
+    return cudaGetLastError();
+}
+
+template <typename T, int RP>
+cudaError_t launch_rows_rp(const T* X, const float* A, int M, int K, int r, int8_t* Xq, float* sx,
+                           float* xA, cudaStream_t s) {
+    const int nchunks = K / kChunk;
+    if (nchunks <= 32 * kMaxCPT) return launch_tpr<T, 32, RP>(X, A, M, K, r, Xq, sx, xA, s);
+    if (nchunks <= 64 * kMaxCPT) return launch_tpr<T, 64, RP>(X, A, M, K, r, Xq, sx, xA, s);
+    if (nchunks <= 128 * kMaxCPT) return launch_tpr<T, 128, RP>(X, A, M, K, r, Xq, sx, xA, s);
+    if (nchunks <= 256 * kMaxCPT) return launch_tpr<T, 256, RP>(X, A, M, K, r, Xq, sx, xA, s);
+    const int cap_chunks = kSmemCap / (a_chunk_floats<RP>() * 4);
+    const int a_chunks = nchunks <= cap_chunks ? nchunks : cap_chunks;
+    auto kern = k1_quantize_rows_long_kernel<T, RP>;
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), kSmemCap);
+    if (e != cudaSuccess) return e;
+    kern<<<M, kThreads, a_chunks * a_chunk_floats<RP>() * 4, s>>>(X, A, M, K, r, a_chunks, Xq, sx,
+                                                                  xA);
+    return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t launch_rows_t(const T* X, const float* A, int M, int K, int r, int8_t* Xq, float* sx,
                           float* xA, cudaStream_t s) {
-    const int nchunks = K / kChunk;
-    auto grid = [&](int tpr) { return dim3((M + kThreads / tpr - 1) / (kThreads / tpr)); };
-    if (nchunks <= 32 * kMaxCPT)
-        k1_quantize_rows_kernel<T, 32><<<grid(32), kThreads, 0, s>>>(X, A, M, K, r, Xq, sx, xA);
-    else if (nchunks <= 64 * kMaxCPT)
-        k1_quantize_rows_kernel<T, 64><<<grid(64), kThreads, 0, s>>>(X, A, M, K, r, Xq, sx, xA);
-    else if (nchunks <= 128 * kMaxCPT)
-        k1_quantize_rows_kernel<T, 128><<<grid(128), kThreads, 0, s>>>(X, A, M, K, r, Xq, sx, xA);
-    else if (nchunks <= 256 * kMaxCPT)
-        k1_quantize_rows_kernel<T, 256><<<grid(256), kThreads, 0, s>>>(X, A, M, K, r, Xq, sx, xA);
-    else
-        k1_quantize_rows_long_kernel<T><<<M, kThreads, 0, s>>>(X, A, M, K, r, Xq, sx, xA);
-    return cudaGetLastError();
+    if (r <= 4) return launch_rows_rp<T, 4>(X, A, M, K, r, Xq, sx, xA, s);
+    if (r <= 8) return launch_rows_rp<T, 8>(X, A, M, K, r, Xq, sx, xA, s);
+    if (r <= 16) return launch_rows_rp<T, 16>(X, A, M, K, r, Xq, sx, xA, s);
+    return launch_rows_rp<T, 64>(X, A, M, K, r, Xq, sx, xA, s);
 }
 
 // ------------------------------------------------------------------ a0
 // One CTA per 32 output channels.  Pass 1: column abs-max (coalesced rows of
-// 32 floats).  Pass 2: 32 x 128 tiles transposed through shared memory so that
-// Wq [N,K] rows are written contiguously.
+// 32 floats).  Pass 2: 128 x 32 tiles transposed through shared memory so
+// that Wq [N,K] rows are written contiguously.
 constexpr int kQwCols = 32;
 constexpr int kQwK = 128;
 
@@ -252,10 +359,9 @@ __global__ void __launch_bounds__(256) k_quantize_weight_kernel(const float* __r
             tile[kk][tx] = (n < N && k < K) ? __ldg(W + static_cast<size_t>(k) * N + n) : 0.f;
         }
         __syncthreads();
-        // thread writes 4 consecutive k of one output channel: 8 channels x 32 threads...
-        // 256 threads cover 32 channels x 8 groups of 16 k.
-        const int c = threadIdx.x / 8;       // channel within the tile
-        const int g = threadIdx.x % 8;       // 16 consecutive k per thread
+        // 256 threads cover 32 channels x 8 groups of 16 consecutive k
+        const int c = threadIdx.x / 8;
+        const int g = threadIdx.x % 8;
         const int nn = n0 + c;
         if (nn < N) {
             const float inv = inv_s[c];

@@ -1,23 +1,27 @@
 // k2_gemm_i8.cu -- forward int8 GEMM of the int8-LoRA Dense layer on the
 // 5th-generation tensor cores, with the whole layer epilogue fused:
 //
-//   acc[m,n] = sum_k Xq[m,k] Wq[n,k]                    (int32, in TMEM)
-//   Y[m,n]   = acc * sx[m] * sw[n] + bias[n] + c * sum_j xA[m,j] B[j,n]
+//   acc[m,n]  = sum_k Xq[m,k] Wq[n,k]                          (int32, TMEM)
+//   lora[m,n] = sum_j (c xA[m,j]) B[j,n] + 1 * bias[n]          (fp32, TMEM)
+//   Y[m,n]    = acc * sx[m] * sw[n] + lora[m,n]
 //
 // ("Introduce QLoRA-like technique", Results: int8 Dense needs a hardware
 // int8 matmul; "Parameter-efficient fine-tuning of GPT-2 with LoRA", "LoRA
 // equation" for the added low-rank term, with xA = x . A from the input pass.)
+// The rank-r term and the bias are one more small product, [c xA | 1] x
+// [B ; bias], issued as tf32 MMAs into a second TMEM accumulator (split into
+// tf32 head and remainder for fp32 outputs, which keeps fp32 accuracy).
 //
 // Persistent kernel, one CTA per SM, 10 warps:
 //   warp 0      TMA producer: Xq [128 x 128] and Wq [BN x 128] int8 tiles
 //               (128B swizzle, K-major) into a STAGES-deep ring
 //   warp 1      TMEM owner and MMA issuer: tcgen05.mma.kind::i8, M=128,
-//               N=BN, K=32, into one of two TMEM accumulators (2 x BN
-//               columns), so that tile i+1's main loop overlaps tile i's
+//               N=BN, K=32, then the tf32 rank-r MMAs; two accumulator
+//               buffers so that tile i+1's main loop overlaps tile i's
 //               epilogue
-//   warps 2..9  epilogue: two warps per TMEM lane quarter, each one half of
-//               the columns; scale, bias and the rank-r term per element,
-//               then a staged, coalesced 16-byte store of the output block
+//   warps 2..9  epilogue: write the tile's rank-r operand tables, then two
+//               warps per TMEM lane quarter, each one half of the columns:
+//               y = acc * (sx sw) + lora, staged coalesced 16-byte stores
 // Ragged M, N, K: the tensor maps zero-fill, the stores are predicated.
 #include "internal.h"
 #include "ptx.cuh"
@@ -35,23 +39,28 @@ constexpr int kSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory
 
 template <int BN, typename OutT, int RMAX>
 struct K2Cfg {
-    static constexpr int kRPad = RMAX <= 16 ? ((RMAX + 3) / 4) * 4 : 0;  // B table width
+    static constexpr bool kLoraMMA = RMAX <= 16;
+    static constexpr bool kSplit = sizeof(OutT) == 4;      // 3 x tf32 for fp32 outputs
+    static constexpr int kKL = ((RMAX + 1 + 7) / 8) * 8;   // [c xA | 1] width
+    static constexpr int kTerms = kSplit ? 2 : 1;          // head (+ remainder) tables
+    static constexpr int kXtBytes = kLoraMMA ? kBM * kKL * 4 : 0;
+    static constexpr int kBtBytes = kLoraMMA ? BN * kKL * 4 : 0;
+    static constexpr int kBufBytes = kTerms * (kXtBytes + kBtBytes) + BN * 4 * 2;  // + sw, bias
     static constexpr int kABytes = kBM * kBK;
     static constexpr int kBBytes = BN * kBK;
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kStgBytes = kEpiWarps * 32 * stage_pitch<OutT>();
-    static constexpr int kParamBytes = BN * 4 * 2 + BN * kRPad * 4;
-    static constexpr int kFixed = kStgBytes + kParamBytes + 256 + 1024;
+    static constexpr int kFixed = kStgBytes + 2 * kBufBytes + 512 + 1024;
     static constexpr int kStagesFit = (kSmemLimit - kFixed) / kStageBytes;
     static constexpr int STAGES = kStagesFit > 8 ? 8 : kStagesFit;
     static_assert(STAGES >= 2, "shared memory budget");
     static constexpr int kStgOff = STAGES * kStageBytes;
-    static constexpr int kSwOff = kStgOff + kStgBytes;
-    static constexpr int kBiasOff = kSwOff + BN * 4;
-    static constexpr int kTabOff = kBiasOff + BN * 4;
-    static constexpr int kBarOff = kTabOff + BN * kRPad * 4;
-    static constexpr int kTotal = kBarOff + 256 + 1024;
-    static constexpr uint32_t kTmemCols = 2 * BN;
+    static constexpr int kBufOff = kStgOff + kStgBytes;
+    static constexpr int kBarOff = kBufOff + 2 * kBufBytes;
+    static constexpr int kTotal = kBarOff + 512 + 1024;
+    static constexpr uint32_t kAccCols = 2 * BN;             // int32 acc + fp32 rank-r acc
+    static constexpr uint32_t kTmemCols = 2 * kAccCols;
+    static_assert(kTmemCols <= 512, "TMEM");
 };
 
 template <int BN, typename OutT, int RMAX>
@@ -66,12 +75,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
     uint64_t* empty = full + S;
-    uint64_t* tfull = empty + S;   // [2]
-    uint64_t* tempty = tfull + 2;  // [2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
-    float* s_sw = reinterpret_cast<float*>(smem + C::kSwOff);
-    float* s_bias = reinterpret_cast<float*>(smem + C::kBiasOff);
-    float* s_tab = reinterpret_cast<float*>(smem + C::kTabOff);
+    uint64_t* tfull = empty + S;    // [2]
+    uint64_t* tempty = tfull + 2;   // [2]
+    uint64_t* lready = tempty + 2;  // [2] rank-r operand tables written
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lready + 2);
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
@@ -87,6 +94,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], kEpiWarps);
+            mbar_init(&lready[b], 1);
         }
         fence_mbar_init();
     }
@@ -134,7 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int use = i >> 1;
                 if (use > 0 && !mbar_wait(&tempty[ab], (use - 1) & 1, status)) break;
                 tc_fence_after();
-                const uint32_t dacc = tmem + ab * BN;
+                const uint32_t dacc = tmem + ab * C::kAccCols;
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
                     const int s = g % S;
                     if (!mbar_wait(&full[s], (g / S) & 1, status)) {
@@ -151,6 +159,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_i8(dacc, ad, bd, idesc, (kb | kk) != 0);
                     }
                     mma_commit(&empty[s]);
+                }
+                if constexpr (C::kLoraMMA) {
+                    // [c xA | 1] x [B ; bias] into the fp32 accumulator
+                    if (ok && !mbar_wait(&lready[ab], use & 1, status)) ok = false;
+                    if (ok) {
+                        tc_fence_after();
+                        constexpr uint32_t tdesc = idesc_tf32(kBM, BN);
+                        constexpr uint32_t kSbo = (C::kKL / 4) * 128;
+                        const uint32_t buf = smem_u32(smem + C::kBufOff + ab * C::kBufBytes);
+                        const uint32_t xt_hi = buf;
+                        const uint32_t bt_hi = buf + C::kXtBytes;
+                        const uint32_t xt_lo = buf + C::kXtBytes + C::kBtBytes;
+                        const uint32_t bt_lo = xt_lo + C::kXtBytes;
+                        const uint32_t dl = dacc + BN;
+#pragma unroll
+                        for (int ks = 0; ks < C::kKL / 8; ++ks) {
+                            const uint32_t o = ks * 256;
+                            mma_tf32(dl, smem_desc(xt_hi + o, 128, kSbo, kLayoutNone),
+                                     smem_desc(bt_hi + o, 128, kSbo, kLayoutNone), tdesc, ks != 0);
+                            if constexpr (C::kSplit) {
+                                mma_tf32(dl, smem_desc(xt_hi + o, 128, kSbo, kLayoutNone),
+                                         smem_desc(bt_lo + o, 128, kSbo, kLayoutNone), tdesc, 1);
+                                mma_tf32(dl, smem_desc(xt_lo + o, 128, kSbo, kLayoutNone),
+                                         smem_desc(bt_hi + o, 128, kSbo, kLayoutNone), tdesc, 1);
+                            }
+                        }
+                    }
                 }
                 if (ok) mma_commit(&tfull[ab]);
             }
@@ -171,63 +206,95 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int use = i >> 1;
             const int m0 = (t / num_n) * kBM;
             const int n0 = (t % num_n) * BN;
-            // per-column tables of this tile (after every warp is done with the last ones)
-            named_bar_sync(1, 32 * kEpiWarps);
+            uint8_t* buf = smem + C::kBufOff + ab * C::kBufBytes;
+            float* s_sw = reinterpret_cast<float*>(buf + C::kTerms * (C::kXtBytes + C::kBtBytes));
+            float* s_bias = s_sw + BN;
+            // ---- this tile's tables (buffer ab was last read two tiles ago) ----
             for (int c = et; c < BN; c += 32 * kEpiWarps) {
                 const int n = n0 + c;
                 s_sw[c] = n < N ? ep.sw[n] : 0.f;
                 s_bias[c] = (n < N && ep.bias) ? ep.bias[n] : 0.f;
             }
-            if constexpr (C::kRPad > 0) {
-                for (int e = et; e < BN * C::kRPad; e += 32 * kEpiWarps) {
-                    const int c = e / C::kRPad, j = e % C::kRPad;
-                    const int n = n0 + c;
-                    s_tab[e] = (n < N && j < ep.r) ? ep.B[static_cast<size_t>(j) * N + n] : 0.f;
+            if constexpr (C::kLoraMMA) {
+                uint8_t* xt = buf;
+                uint8_t* bt = buf + C::kXtBytes;
+                uint8_t* xt_lo = buf + C::kXtBytes + C::kBtBytes;
+                uint8_t* bt_lo = xt_lo + C::kXtBytes;
+                for (int e = et; e < kBM * C::kKL; e += 32 * kEpiWarps) {
+                    const int rr = e / C::kKL, j = e % C::kKL;
+                    const int m = m0 + rr;
+                    float x = 0.f;
+                    if (m < M) x = j < ep.r ? ep.xA[static_cast<size_t>(m) * ep.r + j] * ep.c
+                                            : (j == ep.r ? 1.f : 0.f);
+                    float hi, lo;
+                    tf32_split(x, hi, lo);
+                    const uint32_t off = kmajor_tf32_offset(rr, j, C::kKL);
+                    *reinterpret_cast<float*>(xt + off) = hi;
+                    if constexpr (C::kSplit) *reinterpret_cast<float*>(xt_lo + off) = lo;
                 }
+                for (int e = et; e < BN * C::kKL; e += 32 * kEpiWarps) {
+                    const int cc = e / C::kKL, j = e % C::kKL;
+                    const int n = n0 + cc;
+                    float b = 0.f;
+                    if (n < N) b = j < ep.r ? ep.B[static_cast<size_t>(j) * N + n]
+                                            : ((j == ep.r && ep.bias) ? ep.bias[n] : 0.f);
+                    float hi, lo;
+                    tf32_split(b, hi, lo);
+                    const uint32_t off = kmajor_tf32_offset(cc, j, C::kKL);
+                    *reinterpret_cast<float*>(bt + off) = hi;
+                    if constexpr (C::kSplit) *reinterpret_cast<float*>(bt_lo + off) = lo;
+                }
+                fence_proxy_async_smem();
             }
             named_bar_sync(1, 32 * kEpiWarps);
+            if constexpr (C::kLoraMMA) {
+                if (et == 0) mbar_arrive(&lready[ab]);
+            }
 
             const int row0 = m0 + q * 32;
             const int row = row0 + lane;
             const bool row_ok = row < M;
             const float sxm = row_ok ? ep.sx[row] : 0.f;
-            float xa[RMAX];
+            float xa[C::kLoraMMA ? 1 : RMAX];
+            if constexpr (!C::kLoraMMA) {
 #pragma unroll
-            for (int j = 0; j < RMAX; ++j)
-                xa[j] = (row_ok && j < ep.r) ? ep.xA[static_cast<size_t>(row) * ep.r + j] * ep.c : 0.f;
+                for (int j = 0; j < RMAX; ++j)
+                    xa[j] = (row_ok && j < ep.r) ? ep.xA[static_cast<size_t>(row) * ep.r + j] * ep.c : 0.f;
+            }
 
             const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[ab], use & 1, status));
             if (!ok) break;
             tc_fence_after();
-            const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * BN;
+            const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * C::kAccCols;
 #pragma unroll 1
             for (int col = half * (BN / 2); col < (half + 1) * (BN / 2); col += kEpiCols) {
                 uint32_t v[kEpiCols];
+                uint32_t l[kEpiCols];
                 tmem_ld16(tbase + col, v);
+                if constexpr (C::kLoraMMA) tmem_ld16(tbase + BN + col, l);
                 tmem_ld_wait();
                 float y[kEpiCols];
+                const float4* sw4 = reinterpret_cast<const float4*>(s_sw + col);
 #pragma unroll
-                for (int e = 0; e < kEpiCols; ++e) {
-                    const int c = col + e;
-                    const float a = static_cast<float>(static_cast<int32_t>(v[e]));
-                    float acc = fmaf(a * sxm, s_sw[c], s_bias[c]);
-                    if constexpr (C::kRPad > 0) {
-                        const float4* tb = reinterpret_cast<const float4*>(s_tab + c * C::kRPad);
+                for (int e4 = 0; e4 < kEpiCols / 4; ++e4) {
+                    const float4 w4 = sw4[e4];
+                    const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-                        for (int j4 = 0; j4 < C::kRPad / 4; ++j4) {
-                            const float4 b4 = tb[j4];
-                            acc = fmaf(xa[4 * j4], b4.x, acc);
-                            if (4 * j4 + 1 < RMAX) acc = fmaf(xa[4 * j4 + 1], b4.y, acc);
-                            if (4 * j4 + 2 < RMAX) acc = fmaf(xa[4 * j4 + 2], b4.z, acc);
-                            if (4 * j4 + 3 < RMAX) acc = fmaf(xa[4 * j4 + 3], b4.w, acc);
+                    for (int u = 0; u < 4; ++u) {
+                        const int e = 4 * e4 + u;
+                        const float a = static_cast<float>(static_cast<int32_t>(v[e]));
+                        if constexpr (C::kLoraMMA) {
+                            y[e] = fmaf(a * sxm, wv[u], __uint_as_float(l[e]));
+                        } else {
+                            const int c = col + e;
+                            const int n = n0 + c;
+                            float acc = fmaf(a * sxm, wv[u], s_bias[c]);
+                            if (n < N)
+                                for (int j = 0; j < ep.r; ++j)
+                                    acc = fmaf(xa[j], __ldg(ep.B + static_cast<size_t>(j) * N + n), acc);
+                            y[e] = acc;
                         }
-                    } else {
-                        const int n = n0 + c;
-                        if (n < N)
-                            for (int j = 0; j < ep.r; ++j)
-                                acc = fmaf(xa[j], __ldg(ep.B + static_cast<size_t>(j) * N + n), acc);
                     }
-                    y[e] = acc;
                 }
                 if (ep.acc && row_ok) {
                     for (int e = 0; e < kEpiCols; ++e)
@@ -266,7 +333,6 @@ cudaError_t launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, int M, int 
 template <typename OutT, int RMAX>
 cudaError_t launch_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K,
                       const FwdEpilogue& ep, int* status, cudaStream_t s) {
-    if (bn == 256) return launch_cfg<256, OutT, RMAX>(ta, tb, M, N, K, ep, status, s);
     if (bn == 128) return launch_cfg<128, OutT, RMAX>(ta, tb, M, N, K, ep, status, s);
     return launch_cfg<64, OutT, RMAX>(ta, tb, M, N, K, ep, status, s);
 }
@@ -284,11 +350,11 @@ cudaError_t launch_r(int bn, const CUtensorMap& ta, const CUtensorMap& tb, int M
 
 cudaError_t launch_gemm_i8_fwd(Act act, const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
                                const FwdEpilogue& ep, int* status, cudaStream_t s) {
-    // Tile width: the widest BN that still gives every SM a tile.
+    // Tile width: 128 columns unless that leaves SMs without a tile.
     const int mt = (M + kBM - 1) / kBM;
-    const int sms = sm_count();
-    int bn = 256;
-    while (bn > 64 && mt * ((N + bn - 1) / bn) < sms) bn /= 2;
+    int bn = mt * ((N + 127) / 128) >= sm_count() ? 128 : 64;
+    const int forced = tile_override("QLORA_FWD_BN");  // tuning: 64 or 128
+    if (forced == 64 || forced == 128) bn = forced;
     CUtensorMap ta, tb;
     if (!make_tmap_2d(&ta, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, K, kBM, kBK,
                       CU_TENSOR_MAP_SWIZZLE_128B))

@@ -39,22 +39,31 @@ constexpr int kSmemLimit = 232448;
 template <int MSUB, int BN, int RMAX>
 struct K3Cfg {
     static constexpr int kBM = 128 * MSUB;
-    static constexpr int kRPad = RMAX <= 16 ? ((RMAX + 3) / 4) * 4 : 0;
+    // rank <= 16: c G A^T runs on the tensor cores as tf32 MMAs into the same
+    // fp32 accumulator (operand tables c*G [kBM x kKL] and A [BN x kKL] per
+    // accumulator buffer); larger ranks fall back to CUDA-core FMAs.
+    static constexpr bool kLoraMMA = RMAX <= 16;
+    static constexpr int kKL = RMAX <= 8 ? 8 : 16;
+    static constexpr int kGtBytes = kLoraMMA ? kBM * kKL * 4 : 0;
+    static constexpr int kAtBytes = kLoraMMA ? BN * kKL * 4 : 0;
     static constexpr int kASub = 128 * kBKn * 2;       // one dY sub-tile, bf16
     static constexpr int kABytes = MSUB * kASub;
     static constexpr int kQBytes = kBKn * BN;          // int8 kernel tile
     static constexpr int kWBytes = kBKn * BN * 2;      // de-quantized bf16 tile
     static constexpr int kStageBytes = kABytes + kQBytes + kWBytes;
     static constexpr int kStgBytes = kEpiWarps * 32 * stage_pitch<__nv_bfloat16>();
-    static constexpr int kParamBytes = BN * kRPad * 4;
-    static constexpr int kFixed = kStgBytes + kParamBytes + 256 + 1024;
+    static constexpr int kParamBytes = 2 * (kGtBytes + kAtBytes);
+    static constexpr int kFixed = kStgBytes + kParamBytes + 512 + 1024;
     static constexpr int kStagesFit = (kSmemLimit - kFixed) / kStageBytes;
     static constexpr int STAGES = kStagesFit > 8 ? 8 : kStagesFit;
     static_assert(STAGES >= 2, "shared memory budget");
+    // de-quantize warps per ring stage (warps beyond STAGES * kDqPerStage idle)
+    static constexpr int kDqPerStage = kDqWarps / STAGES > 0 ? kDqWarps / STAGES : 1;
+    static_assert(STAGES <= kDqWarps, "one de-quantize warp per stage at least");
     static constexpr int kStgOff = STAGES * kStageBytes;
     static constexpr int kTabOff = kStgOff + kStgBytes;
     static constexpr int kBarOff = kTabOff + kParamBytes;
-    static constexpr int kTotal = kBarOff + 256 + 1024;
+    static constexpr int kTotal = kBarOff + 512 + 1024;
     static constexpr uint32_t kAccCols = MSUB * BN;     // one accumulator buffer
     static constexpr uint32_t kTmemCols = 2 * kAccCols;
     static_assert(kTmemCols <= 512, "TMEM");
@@ -69,6 +78,15 @@ __device__ __forceinline__ uint32_t mn_sw128_offset(int mn, int kr, uint32_t lbo
     const int kg = kr >> 3;
     const int row = kr & 7;
     return mb * lbo + kg * 1024 + row * 128 + ((chunk ^ row) << 4);
+}
+
+// G[m,j] = sum over the column-block slices of G (fixed order).
+__device__ __forceinline__ float g_row(const DxEpilogue& ep, int M, int m, int j) {
+    const float* p = ep.Gp + static_cast<size_t>(m) * ep.r + j;
+    const size_t slice = static_cast<size_t>(M) * ep.r;
+    float s = __ldg(p);
+    for (int b = 1; b < ep.ncb; ++b) s += __ldg(p + b * slice);
+    return s;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -92,8 +110,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* empty = wready + S;
     uint64_t* tfull = empty + S;   // [2]
     uint64_t* tempty = tfull + 2;  // [2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
-    float* s_tab = reinterpret_cast<float*>(smem + C::kTabOff);
+    uint64_t* lready = tempty + 2; // [2] rank-r operand tables written
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lready + 2);
+    uint8_t* tabs = smem + C::kTabOff;  // [2] x (c*G table, A table)
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
@@ -104,12 +123,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&wready[s], kDqWarps);
+            mbar_init(&wready[s], C::kDqPerStage);  // the stage's de-quantize warps
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], kEpiWarps);
+            mbar_init(&lready[b], kEpiWarps);
         }
         fence_mbar_init();
     }
@@ -181,30 +201,63 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     mma_commit(&empty[s]);
                 }
+                if constexpr (C::kLoraMMA) {
+                    // + (c G) A^T: tf32 MMAs from the tables the epilogue warps wrote
+                    if (ok && !mbar_wait(&lready[ab], use & 1, status)) ok = false;
+                    if (ok) {
+                        tc_fence_after();
+                        constexpr uint32_t tdesc = idesc_tf32(128, BN);
+                        constexpr uint32_t kSbo = (C::kKL / 4) * 128;
+                        const uint32_t gt = smem_u32(tabs + ab * (C::kGtBytes + C::kAtBytes));
+                        const uint32_t at = gt + C::kGtBytes;
+#pragma unroll
+                        for (int ks = 0; ks < C::kKL / 8; ++ks) {
+                            const uint64_t bd = smem_desc(at + ks * 256, 128, kSbo, kLayoutNone);
+#pragma unroll
+                            for (int ms = 0; ms < MSUB; ++ms) {
+                                const uint64_t ad =
+                                    smem_desc(gt + ms * 16 * kSbo + ks * 256, 128, kSbo, kLayoutNone);
+                                mma_tf32(tmem + ab * C::kAccCols + ms * BN, ad, bd, tdesc, 1);
+                            }
+                        }
+                    }
+                }
                 if (ok) mma_commit(&tfull[ab]);
             }
         }
         __syncwarp();
     } else if (warp < 2 + kDqWarps) {
         // ------------------------------------------------------ de-quantize
-        const int dq = threadIdx.x - 64;  // 0 .. 255
+        // Each warp owns one ring stage (C::kDqPerStage warps share a stage
+        // when the ring is short) and converts every fill of that stage, in
+        // order, so its barrier phases are awaited one after the other and
+        // the stages are converted concurrently.
+        const int dw = warp - 2;  // 0 .. 7
         constexpr int kChunksPerRow = BN / 16;
         constexpr int kChunks = kBKn * kChunksPerRow;
-        int g = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-            for (int kb = 0; kb < nkb; ++kb, ++g) {
-                const int s = g % S;
-                ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (g / S) & 1, status));
-                if (!ok) break;
+        constexpr int kPer = C::kDqPerStage;
+        const int my_stage = dw / kPer;
+        const int part = dw % kPer;
+        const int my_tiles = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+        const int total_kb = my_tiles * nkb;
+        for (int g = my_stage; my_stage < S && g < total_kb; g += S) {
+            const int s = my_stage;
+            const int kb = g % nkb;
+            // the 64 row scales of this stage: lane l holds rows l and l + 32
+            const int nbase = kb * kBKn;
+            const float sc0 = nbase + lane < N ? __ldg(sw + nbase + lane) : 0.f;
+            const float sc1 = nbase + 32 + lane < N ? __ldg(sw + nbase + 32 + lane) : 0.f;
+            if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (g / S) & 1, status))) break;
+            {
                 const uint8_t* sq = smem + s * C::kStageBytes + C::kABytes;
                 uint8_t* wt = smem + s * C::kStageBytes + C::kABytes + C::kQBytes;
 #pragma unroll
-                for (int c = dq; c < kChunks; c += 32 * kDqWarps) {
+                for (int c = part * 32 + lane; c < kChunks; c += 32 * kPer) {
                     const int nr = c / kChunksPerRow;   // contraction row within the stage
                     const int kc = c % kChunksPerRow;   // 16 output columns
-                    const int n = kb * kBKn + nr;
-                    const float scale = n < N ? __ldg(sw + n) : 0.f;
+                    const float s0 = __shfl_sync(0xffffffffu, sc0, nr & 31);
+                    const float s1 = __shfl_sync(0xffffffffu, sc1, nr & 31);
+                    const float scale = nr < 32 ? s0 : s1;
                     const uint4 raw = *reinterpret_cast<const uint4*>(sq + nr * BN + kc * 16);
                     const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
                     uint32_t o[8];
@@ -224,10 +277,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn + 8, nr, kLbo)) =
                         make_uint4(o[4], o[5], o[6], o[7]);
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&wready[s]);
             }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&wready[s]);
         }
         __syncwarp();
     } else {
@@ -244,23 +297,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int use = i >> 1;
             const int m0 = (t / num_k) * C::kBM;
             const int k0 = (t % num_k) * BN;
-            if constexpr (C::kRPad > 0) {
-                named_bar_sync(1, 32 * kEpiWarps);
-                for (int e = et; e < BN * C::kRPad; e += 32 * kEpiWarps) {
-                    const int c = e / C::kRPad, j = e % C::kRPad;
-                    const int k = k0 + c;
-                    s_tab[e] = (k < K && j < ep.r) ? ep.A[static_cast<size_t>(k) * ep.r + j] : 0.f;
+            if constexpr (C::kLoraMMA) {
+                // operand tables of this tile's rank-r product, tf32-rounded:
+                // c*G rows m0.. and A rows k0.. (zero outside the matrices)
+                uint8_t* gt = tabs + ab * (C::kGtBytes + C::kAtBytes);
+                uint8_t* at = gt + C::kGtBytes;
+                for (int e = et; e < C::kBM * C::kKL; e += 32 * kEpiWarps) {
+                    const int rr = e / C::kKL, j = e % C::kKL;
+                    const int m = m0 + rr;
+                    const float g = (m < M && j < ep.r) ? g_row(ep, M, m, j) * ep.c : 0.f;
+                    float hi, lo;
+                    tf32_split(g, hi, lo);
+                    *reinterpret_cast<float*>(gt + kmajor_tf32_offset(rr, j, C::kKL)) = hi;
                 }
-                named_bar_sync(1, 32 * kEpiWarps);
+                for (int e = et; e < BN * C::kKL; e += 32 * kEpiWarps) {
+                    const int cc = e / C::kKL, j = e % C::kKL;
+                    const int k = k0 + cc;
+                    const float a = (k < K && j < ep.r) ? ep.A[static_cast<size_t>(k) * ep.r + j] : 0.f;
+                    float hi, lo;
+                    tf32_split(a, hi, lo);
+                    *reinterpret_cast<float*>(at + kmajor_tf32_offset(cc, j, C::kKL)) = hi;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&lready[ab]);
             }
             const int msub = MSUB == 2 ? sub : 0;
             const int row0 = m0 + msub * 128 + q * 32;
             const int row = row0 + lane;
             const bool row_ok = row < M;
-            float gr[RMAX];
+            float gr[C::kLoraMMA ? 1 : RMAX];
+            if constexpr (!C::kLoraMMA) {
 #pragma unroll
-            for (int j = 0; j < RMAX; ++j)
-                gr[j] = (row_ok && j < ep.r) ? ep.G[static_cast<size_t>(row) * ep.r + j] * ep.c : 0.f;
+                for (int j = 0; j < RMAX; ++j)
+                    gr[j] = (row_ok && j < ep.r) ? g_row(ep, M, row, j) * ep.c : 0.f;
+            }
             const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[ab], use & 1, status));
             if (!ok) break;
             tc_fence_after();
@@ -278,17 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int e = 0; e < kEpiCols; ++e) {
                     const int c = col + e;
                     float acc = __uint_as_float(v[e]);
-                    if constexpr (C::kRPad > 0) {
-                        const float4* tb = reinterpret_cast<const float4*>(s_tab + c * C::kRPad);
-#pragma unroll
-                        for (int j4 = 0; j4 < C::kRPad / 4; ++j4) {
-                            const float4 a4 = tb[j4];
-                            acc = fmaf(gr[4 * j4], a4.x, acc);
-                            if (4 * j4 + 1 < RMAX) acc = fmaf(gr[4 * j4 + 1], a4.y, acc);
-                            if (4 * j4 + 2 < RMAX) acc = fmaf(gr[4 * j4 + 2], a4.z, acc);
-                            if (4 * j4 + 3 < RMAX) acc = fmaf(gr[4 * j4 + 3], a4.w, acc);
-                        }
-                    } else {
+                    if constexpr (!C::kLoraMMA) {
                         const int k = k0 + c;
                         if (k < K)
                             for (int j = 0; j < ep.r; ++j)
@@ -382,6 +443,13 @@ __global__ void __launch_bounds__(256) k3_dx_simt_kernel(const T* __restrict__ d
         }
         __syncthreads();
     }
+    // G rows of this tile, summed from the column-block slices
+    __shared__ float sG[kSB][65];
+    for (int i = threadIdx.x; i < kSB * ep.r; i += 256) {
+        const int mm = i / ep.r, jj = i % ep.r;
+        sG[mm][jj] = (m0 + mm < M) ? g_row(ep, M, m0 + mm, jj) : 0.f;
+    }
+    __syncthreads();
     T* dX = static_cast<T*>(ep.dX);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -393,7 +461,7 @@ __global__ void __launch_bounds__(256) k3_dx_simt_kernel(const T* __restrict__ d
             if (k >= K) continue;
             float l = 0.f;
             for (int jj = 0; jj < ep.r; ++jj)
-                l = fmaf(ep.G[static_cast<size_t>(m) * ep.r + jj], ep.A[static_cast<size_t>(k) * ep.r + jj], l);
+                l = fmaf(sG[ty + 16 * i][jj], ep.A[static_cast<size_t>(k) * ep.r + jj], l);
             dX[static_cast<size_t>(m) * K + k] = ActIO<T>::from_f(acc[i][j] + ep.c * l);
         }
     }
@@ -420,6 +488,8 @@ cudaError_t launch_gemm_dx(Act act, const void* dY, const int8_t* Wq, const floa
     int cfg = 2;
     if (ntiles(256, 128) >= sms) cfg = 0;
     else if (ntiles(128, 128) >= sms) cfg = 1;
+    const int forced = tile_override("QLORA_DX_TILE");  // tuning: 0, 1 or 2
+    if (forced >= 0 && forced <= 2) cfg = forced;
     const int bn = cfg == 2 ? 64 : 128;
     CUtensorMap tdy, tq;
     if (!make_tmap_2d(&tdy, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N,

@@ -1,9 +1,9 @@
 // k4_rank.cu -- the skinny rank-r contractions of the LoRA backward:
 //
-//   G[m,j]   = sum_n dY[m,n] B[j,n]          (pass over dY)
-//   dB[j,n]  = c * sum_m xA[m,j] dY[m,n]     (same pass over dY)
-//   dbias[n] = sum_m dY[m,n]                 (same pass over dY)
-//   dA[k,j]  = c * sum_m X[m,k] G[m,j]       (pass over X)
+//   Gp[b][m,j] = sum_{n in column block b} dY[m,n] B[j,n]   (G = sum_b Gp[b])
+//   dB[j,n]    = c * sum_m xA[m,j] dY[m,n]                  (same pass over dY)
+//   dbias[n]   = sum_m dY[m,n]                              (same pass over dY)
+//   dA[k,j]    = c * sum_m X[m,k] G[m,j]                    (pass over X)
 //
 // ("How to fine-tune the 4-bit model?" thread: the LoRA factors are the
 // trainable fp32 weights and the backward needs the A @ B.T-style adapter
@@ -12,22 +12,34 @@
 // pass streams its matrix once from HBM with 128-bit loads and does 2r FMAs
 // per element on CUDA cores.
 //
-// Determinism: every sum has a fixed order.  A CTA owns a 256-column block
-// and a chunk of rows; its lanes own 8 columns each and sweep the chunk's rows
-// in a fixed order; per-row G partials are reduced inside the warp with a
-// fixed butterfly, per-chunk dB/dbias/dA partials go to the workspace, and a
-// second kernel sums the partials in chunk order.
+// Layout of the work: a CTA owns 128 columns (16 lanes x 8) and a chunk of
+// rows; the CL <= 8 CTAs that own the chunks of one column block form a
+// thread-block cluster along the rows.  Each CTA reduces its rows in
+// registers and shared memory, then the cluster sums the CL partial results
+// through distributed shared memory, rank by rank, so dB, dbias and dA leave
+// the kernel final, with a fixed summation order (deterministic) and no
+// second launch.  G's per-row sums over the column blocks stay as partial
+// slices Gp in the workspace; the two consumers (the dX GEMM and the X pass)
+// add the slices up themselves.
+#include <cooperative_groups.h>
+
 #include "internal.h"
 #include "ptx.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace qlora {
 
 namespace {
 
-constexpr int kWarps = 4;
-constexpr int kThreads = 32 * kWarps;
-constexpr int kCols = 256;  // columns per CTA: 32 lanes x 8
-constexpr int kRJ = 8;      // rank columns per sweep
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kCols = 128;         // columns per CTA: 16 lanes x 8
+constexpr int kRJ = 8;             // rank columns per sweep
+constexpr int kMaxCluster = 8;
+constexpr int kRowsPerPass = 2 * kWarps;  // a half-warp per row
+constexpr int kPassesInFlight = 4;
+constexpr int kXRowBlock = 128;    // rows whose G is staged at a time (X pass)
 
 template <typename T>
 __device__ __forceinline__ void load8(const T* row, int c0, int ncols, bool vec, float (&v)[8]) {
@@ -53,47 +65,51 @@ __device__ __forceinline__ void load8(const T* row, int c0, int ncols, bool vec,
     }
 }
 
-// Sum of an 8-vector over the 32 lanes of a warp.  On return, lane l holds the
-// total of component (l >> 2) & 7 when (l & 3) == 0.  Fixed order.
-__device__ __forceinline__ float warp_reduce8(float (&v)[8], int lane) {
-    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+// Sum of an 8-vector over the 16 lanes of a half-warp (xor offsets 8..1).  On
+// return, lane l holds the total of component (l >> 1) & 7 when (l & 1) == 0.
+__device__ __forceinline__ float half_reduce8(float (&v)[8], int lane) {
+    const bool b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const float send = b4 ? v[i] : v[i + 4];
-        const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
-        v[i] = (b4 ? v[i + 4] : v[i]) + recv;
+        const float send = b3 ? v[i] : v[i + 4];
+        const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
+        v[i] = (b3 ? v[i + 4] : v[i]) + recv;
     }
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-        const float send = b3 ? v[i] : v[i + 2];
-        const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
-        v[i] = (b3 ? v[i + 2] : v[i]) + recv;
+        const float send = b2 ? v[i] : v[i + 2];
+        const float recv = __shfl_xor_sync(0xffffffffu, send, 4);
+        v[i] = (b2 ? v[i + 2] : v[i]) + recv;
     }
     {
-        const float send = b2 ? v[0] : v[1];
-        const float recv = __shfl_xor_sync(0xffffffffu, send, 4);
-        v[0] = (b2 ? v[1] : v[0]) + recv;
+        const float send = b1 ? v[0] : v[1];
+        const float recv = __shfl_xor_sync(0xffffffffu, send, 2);
+        v[0] = (b1 ? v[1] : v[0]) + recv;
     }
-    float s = v[0];
-    s += __shfl_xor_sync(0xffffffffu, s, 2);
-    s += __shfl_xor_sync(0xffffffffu, s, 1);
-    return s;
+    return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
 }
 
-// Pass over dY for rank columns [j0, j0 + 8).
+// ---------------------------------------------------------------- dY pass
+// Shared memory: red[kWarps][(kRJ + 1) * kCols] (per-warp partials) and
+// part[(kRJ + 1) * kCols] (this CTA's partial, read by the cluster).
 template <typename T>
-__global__ void __launch_bounds__(kThreads) k4_dy_pass_kernel(
+__global__ void __launch_bounds__(kThreads) k4_dy_kernel(
     const T* __restrict__ dY, const float* __restrict__ B, const float* __restrict__ xA, int M,
-    int N, int r, int j0, int RM, float* __restrict__ Gp, float* __restrict__ dBp,
-    float* __restrict__ dbp) {
-    __shared__ float red[kWarps][kRJ + 1][kCols];
+    int N, int r, int j0, int RM, float cscale, float* __restrict__ Gp, float* __restrict__ dB,
+    float* __restrict__ dbias) {
+    constexpr int kW = (kRJ + 1) * kCols;
+    __shared__ float red[kWarps][kW];
+    __shared__ float part[kW];
+    cg::cluster_group cluster = cg::this_cluster();
+    const int CL = static_cast<int>(cluster.num_blocks());
+    const int crank = static_cast<int>(cluster.block_rank());
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int cb = blockIdx.x, rc = blockIdx.y;
-    const int c0 = cb * kCols + lane * 8;
-    const int mbeg = rc * RM;
+    const int half = lane >> 4, cl = lane & 15;
+    const int cb = blockIdx.x;
+    const int c0 = cb * kCols + cl * 8;
+    const int mbeg = blockIdx.y * RM;
     const int mend = min(M, mbeg + RM);
     const bool vec = (N % 8) == 0;
-    const bool with_bias = (j0 == 0) && dbp != nullptr;
 
     float bv[kRJ][8];
 #pragma unroll
@@ -102,222 +118,283 @@ __global__ void __launch_bounds__(kThreads) k4_dy_pass_kernel(
         for (int e = 0; e < 8; ++e)
             bv[j][e] = (j0 + j < r && c0 + e < N) ? __ldg(B + static_cast<size_t>(j0 + j) * N + c0 + e) : 0.f;
     float db[kRJ][8];
-    float dbias[8];
+    float dbi[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-        dbias[e] = 0.f;
+        dbi[e] = 0.f;
 #pragma unroll
         for (int j = 0; j < kRJ; ++j) db[j][e] = 0.f;
     }
 
-    for (int m = mbeg + warp; m < mend; m += kWarps) {
-        float v[8];
-        load8<T>(dY + static_cast<size_t>(m) * N, c0, N, vec, v);
-        float xa[kRJ];
+    const int rowoff = 2 * warp + half;
+    for (int pb = mbeg; pb < mend; pb += kRowsPerPass * kPassesInFlight) {
+        float v[kPassesInFlight][8];
+        float xr[kPassesInFlight][kRJ];
 #pragma unroll
-        for (int j = 0; j < kRJ; ++j) xa[j] = (j0 + j < r) ? __ldg(xA + static_cast<size_t>(m) * r + j0 + j) : 0.f;
-        float g[kRJ];
+        for (int u = 0; u < kPassesInFlight; ++u) {
+            const int m = pb + u * kRowsPerPass + rowoff;
+            const bool ok = m < mend;
+            if (ok) load8<T>(dY + static_cast<size_t>(m) * N, c0, N, vec, v[u]);
+            else
 #pragma unroll
-        for (int j = 0; j < kRJ; ++j) {
-            float s = 0.f;
+                for (int e = 0; e < 8; ++e) v[u][e] = 0.f;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) s = fmaf(v[e], bv[j][e], s);
-            g[j] = s;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) db[j][e] = fmaf(xa[j], v[e], db[j][e]);
+            for (int j = 0; j < kRJ; ++j)
+                xr[u][j] = (ok && j0 + j < r) ? __ldg(xA + static_cast<size_t>(m) * r + j0 + j) : 0.f;
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) dbias[e] += v[e];
-        const float gs = warp_reduce8(g, lane);
-        const int jj = (lane >> 2) & 7;
-        if ((lane & 3) == 0 && j0 + jj < r)
-            Gp[(static_cast<size_t>(cb) * M + m) * r + j0 + jj] = gs;
+        for (int u = 0; u < kPassesInFlight; ++u) {
+            const int m = pb + u * kRowsPerPass + rowoff;
+            float g[kRJ];
+#pragma unroll
+            for (int j = 0; j < kRJ; ++j) {
+                float s = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) s = fmaf(v[u][e], bv[j][e], s);
+                g[j] = s;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) db[j][e] = fmaf(xr[u][j], v[u][e], db[j][e]);
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dbi[e] += v[u][e];
+            const float gs = half_reduce8(g, lane);  // all lanes take part
+            const int jj = (cl >> 1) & 7;
+            if (m < mend && (cl & 1) == 0 && j0 + jj < r)
+                Gp[(static_cast<size_t>(cb) * M + m) * r + j0 + jj] = gs;
+        }
     }
 
-    // combine the warps of this CTA (fixed order), write the chunk's partials
+    // the two rows of a warp -> one partial per warp, then the warps in order
 #pragma unroll
     for (int j = 0; j < kRJ; ++j)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) red[warp][j][lane * 8 + e] = db[j][e];
+        for (int e = 0; e < 8; ++e) db[j][e] += __shfl_xor_sync(0xffffffffu, db[j][e], 16);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) red[warp][kRJ][lane * 8 + e] = dbias[e];
-    __syncthreads();
-    for (int i = threadIdx.x; i < (kRJ + 1) * kCols; i += kThreads) {
-        const int j = i / kCols, cl = i % kCols;
-        const int n = cb * kCols + cl;
-        if (n >= N) continue;
-        float s = red[0][j][cl];
+    for (int e = 0; e < 8; ++e) dbi[e] += __shfl_xor_sync(0xffffffffu, dbi[e], 16);
+    if (half == 0) {
 #pragma unroll
-        for (int w = 1; w < kWarps; ++w) s += red[w][j][cl];
-        if (j < kRJ) {
-            if (j0 + j < r) dBp[(static_cast<size_t>(rc) * r + j0 + j) * N + n] = s;
-        } else if (with_bias) {
-            dbp[static_cast<size_t>(rc) * N + n] = s;
-        }
+        for (int j = 0; j < kRJ; ++j)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) red[warp][j * kCols + cl * 8 + e] = db[j][e];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) red[warp][kRJ * kCols + cl * 8 + e] = dbi[e];
     }
+    __syncthreads();
+    for (int i = threadIdx.x; i < kW; i += kThreads) {
+        float s = red[0][i];
+#pragma unroll
+        for (int w = 1; w < kWarps; ++w) s += red[w][i];
+        part[i] = s;
+    }
+    cluster.sync();
+    // rank q finalises its slice of the columns, summing the ranks in order
+    const int per = (kCols + CL - 1) / CL;
+    const int cbeg = crank * per;
+    const int cend = min(kCols, cbeg + per);
+    const bool with_bias = (j0 == 0) && dbias != nullptr;
+    for (int i = threadIdx.x; i < (kRJ + 1) * (cend - cbeg); i += kThreads) {
+        const int j = i / (cend - cbeg);
+        const int cc = cbeg + i % (cend - cbeg);
+        const int n = cb * kCols + cc;
+        if (n >= N) continue;
+        if (j < kRJ && j0 + j >= r) continue;
+        if (j == kRJ && !with_bias) continue;
+        float s = 0.f;
+        for (int q = 0; q < CL; ++q) {
+            const float* rp = cluster.map_shared_rank(part, q);
+            s = q == 0 ? rp[j * kCols + cc] : s + rp[j * kCols + cc];
+        }
+        if (j < kRJ) dB[static_cast<size_t>(j0 + j) * N + n] = cscale * s;
+        else dbias[n] = s;
+    }
+    cluster.sync();
 }
 
-// Pass over X for rank columns [j0, j0 + 8): dA partials [chunk][K][r].
+// ---------------------------------------------------------------- X pass
+// G for a block of rows is staged in shared memory from the Gp slices.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) k4_x_pass_kernel(const T* __restrict__ X,
-                                                             const float* __restrict__ G, int M,
-                                                             int K, int r, int j0, int RM,
-                                                             float* __restrict__ dAp) {
-    __shared__ float red[kWarps][kCols][kRJ + 1];
+__global__ void __launch_bounds__(kThreads) k4_x_kernel(
+    const T* __restrict__ X, const float* __restrict__ Gp, int ncb, int M, int K, int r, int j0,
+    int RM, float cscale, float* __restrict__ dA) {
+    constexpr int kW = kCols * kRJ;
+    __shared__ float red[kWarps][kW];
+    __shared__ float part[kW];
+    __shared__ float sG[kXRowBlock][kRJ];
+    cg::cluster_group cluster = cg::this_cluster();
+    const int CL = static_cast<int>(cluster.num_blocks());
+    const int crank = static_cast<int>(cluster.block_rank());
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int cb = blockIdx.x, rc = blockIdx.y;
-    const int c0 = cb * kCols + lane * 8;
-    const int mbeg = rc * RM;
+    const int half = lane >> 4, cl = lane & 15;
+    const int cb = blockIdx.x;
+    const int c0 = cb * kCols + cl * 8;
+    const int mbeg = blockIdx.y * RM;
     const int mend = min(M, mbeg + RM);
     const bool vec = (K % 8) == 0;
+    const size_t gslice = static_cast<size_t>(M) * r;
+
     float acc[8][kRJ];
 #pragma unroll
     for (int e = 0; e < 8; ++e)
 #pragma unroll
         for (int j = 0; j < kRJ; ++j) acc[e][j] = 0.f;
-    for (int m = mbeg + warp; m < mend; m += kWarps) {
-        float v[8];
-        load8<T>(X + static_cast<size_t>(m) * K, c0, K, vec, v);
-        float g[kRJ];
+
+    const int rowoff = 2 * warp + half;
+    for (int rb = mbeg; rb < mend; rb += kXRowBlock) {
+        const int rbe = min(mend, rb + kXRowBlock);
+        __syncthreads();  // the previous block's G is no longer read
+        for (int i = threadIdx.x; i < kXRowBlock * kRJ; i += kThreads) {
+            const int rr = i / kRJ, j = i % kRJ;
+            const int m = rb + rr;
+            float s = 0.f;
+            if (m < rbe && j0 + j < r) {
+                const float* p = Gp + static_cast<size_t>(m) * r + j0 + j;
+                s = __ldg(p);
+                for (int b = 1; b < ncb; ++b) s += __ldg(p + b * gslice);
+            }
+            sG[rr][j] = s;
+        }
+        __syncthreads();
+        for (int pb = rb; pb < rbe; pb += kRowsPerPass * kPassesInFlight) {
+            float v[kPassesInFlight][8];
 #pragma unroll
-        for (int j = 0; j < kRJ; ++j) g[j] = (j0 + j < r) ? __ldg(G + static_cast<size_t>(m) * r + j0 + j) : 0.f;
+            for (int u = 0; u < kPassesInFlight; ++u) {
+                const int m = pb + u * kRowsPerPass + rowoff;
+                if (m < rbe) load8<T>(X + static_cast<size_t>(m) * K, c0, K, vec, v[u]);
+                else
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
+                    for (int e = 0; e < 8; ++e) v[u][e] = 0.f;
+            }
 #pragma unroll
-            for (int j = 0; j < kRJ; ++j) acc[e][j] = fmaf(v[e], g[j], acc[e][j]);
+            for (int u = 0; u < kPassesInFlight; ++u) {
+                const int rr = pb - rb + u * kRowsPerPass + rowoff;
+                if (rr >= kXRowBlock) break;
+                const float4 g0 = *reinterpret_cast<const float4*>(&sG[rr][0]);
+                const float4 g1 = *reinterpret_cast<const float4*>(&sG[rr][4]);
+                const float g[kRJ] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+#pragma unroll
+                    for (int j = 0; j < kRJ; ++j) acc[e][j] = fmaf(v[u][e], g[j], acc[e][j]);
+            }
+        }
     }
+
 #pragma unroll
     for (int e = 0; e < 8; ++e)
 #pragma unroll
-        for (int j = 0; j < kRJ; ++j) red[warp][lane * 8 + e][j] = acc[e][j];
-    __syncthreads();
-    for (int i = threadIdx.x; i < kCols * kRJ; i += kThreads) {
-        const int cl = i / kRJ, j = i % kRJ;
-        const int k = cb * kCols + cl;
-        if (k >= K || j0 + j >= r) continue;
-        float s = red[0][cl][j];
+        for (int j = 0; j < kRJ; ++j) acc[e][j] += __shfl_xor_sync(0xffffffffu, acc[e][j], 16);
+    if (half == 0) {
 #pragma unroll
-        for (int w = 1; w < kWarps; ++w) s += red[w][cl][j];
-        dAp[(static_cast<size_t>(rc) * K + k) * r + j0 + j] = s;
+        for (int e = 0; e < 8; ++e)
+#pragma unroll
+            for (int j = 0; j < kRJ; ++j) red[warp][(cl * 8 + e) * kRJ + j] = acc[e][j];
     }
-}
-
-// G = sum over column blocks, dB = c * sum over row chunks, dbias likewise.
-__global__ void k4_reduce_dy_kernel(const float* __restrict__ Gp, const float* __restrict__ dBp,
-                                    const float* __restrict__ dbp, int M, int N, int r, int ncb,
-                                    int nrc, float c, float* __restrict__ G, float* __restrict__ dB,
-                                    float* __restrict__ dbias) {
-    const size_t nG = static_cast<size_t>(M) * r;
-    const size_t nB = static_cast<size_t>(r) * N;
-    const size_t nb = dbias ? static_cast<size_t>(N) : 0;
-    const size_t total = nG + nB + nb;
-    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
-         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-        if (i < nG) {
-            float s = Gp[i];
-            for (int b = 1; b < ncb; ++b) s += Gp[static_cast<size_t>(b) * nG + i];
-            G[i] = s;
-        } else if (i < nG + nB) {
-            const size_t o = i - nG;
-            float s = dBp[o];
-            for (int b = 1; b < nrc; ++b) s += dBp[static_cast<size_t>(b) * nB + o];
-            dB[o] = c * s;
-        } else {
-            const size_t o = i - nG - nB;
-            float s = dbp[o];
-            for (int b = 1; b < nrc; ++b) s += dbp[static_cast<size_t>(b) * N + o];
-            dbias[o] = s;
+    __syncthreads();
+    for (int i = threadIdx.x; i < kW; i += kThreads) {
+        float s = red[0][i];
+#pragma unroll
+        for (int w = 1; w < kWarps; ++w) s += red[w][i];
+        part[i] = s;
+    }
+    cluster.sync();
+    const int per = (kCols + CL - 1) / CL;
+    const int cbeg = crank * per;
+    const int cend = min(kCols, cbeg + per);
+    for (int i = threadIdx.x; i < (cend - cbeg) * kRJ; i += kThreads) {
+        const int cc = cbeg + i / kRJ, j = i % kRJ;
+        const int k = cb * kCols + cc;
+        if (k >= K || j0 + j >= r) continue;
+        float s = 0.f;
+        for (int q = 0; q < CL; ++q) {
+            const float* rp = cluster.map_shared_rank(part, q);
+            s = q == 0 ? rp[cc * kRJ + j] : s + rp[cc * kRJ + j];
         }
+        dA[static_cast<size_t>(k) * r + j0 + j] = cscale * s;
     }
+    cluster.sync();
 }
 
-__global__ void k4_reduce_x_kernel(const float* __restrict__ dAp, int K, int r, int nrc, float c,
-                                   float* __restrict__ dA) {
-    const size_t n = static_cast<size_t>(K) * r;
+// G[m,j] = sum_b Gp[b][m,j] (only when a caller asks for G itself).
+__global__ void k4_g_reduce_kernel(const float* __restrict__ Gp, int ncb, size_t n,
+                                   float* __restrict__ G) {
     for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
          i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-        float s = dAp[i];
-        for (int b = 1; b < nrc; ++b) s += dAp[static_cast<size_t>(b) * n + i];
-        dA[i] = c * s;
+        float s = Gp[i];
+        for (int b = 1; b < ncb; ++b) s += Gp[static_cast<size_t>(b) * n + i];
+        G[i] = s;
     }
 }
 
-int chunks_for(int M, int col_blocks) {
-    // about two CTAs per SM, at least 8 rows per chunk
-    int want = (2 * 148 + col_blocks - 1) / col_blocks;
-    int maxc = (M + 7) / 8;
-    if (want > maxc) want = maxc;
-    if (want < 1) want = 1;
-    return want;
+int cluster_for(int M) {
+    int cl = (M + 63) / 64;
+    return cl > kMaxCluster ? kMaxCluster : (cl < 1 ? 1 : cl);
+}
+
+template <typename Kern, typename... Args>
+cudaError_t launch_clustered(Kern kern, dim3 grid, int cl, cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = cl;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
 }  // namespace
 
-RankPlan plan_rank(int M, int K, int N, int r) {
-    (void)r;
-    RankPlan p;
-    p.n_col_blocks = (N + kCols - 1) / kCols;
-    int nc = chunks_for(M, p.n_col_blocks);
-    p.rows_per_chunk = (M + nc - 1) / nc;
-    p.n_chunks = (M + p.rows_per_chunk - 1) / p.rows_per_chunk;
-    const int kcb = (K + kCols - 1) / kCols;
-    int kc = chunks_for(M, kcb);
-    p.rows_per_kchunk = (M + kc - 1) / kc;
-    p.k_chunks = (M + p.rows_per_kchunk - 1) / p.rows_per_kchunk;
-    return p;
-}
+int rank_col_blocks(int N) { return (N + kCols - 1) / kCols; }
 
-size_t rank_workspace_floats(const RankPlan& p, int M, int K, int N, int r) {
-    const size_t gp = static_cast<size_t>(p.n_col_blocks) * M * r;
-    const size_t dbp = static_cast<size_t>(p.n_chunks) * r * N;
-    const size_t dbias = static_cast<size_t>(p.n_chunks) * N;
-    const size_t dap = static_cast<size_t>(p.k_chunks) * K * r;
-    // the dY-pass partials and the X-pass partials are live at different times
-    const size_t dy = gp + dbp + dbias;
-    return dy > dap ? dy : dap;
+size_t rank_workspace_floats(int M, int N, int r) {
+    return static_cast<size_t>(rank_col_blocks(N)) * M * r;
 }
 
 cudaError_t launch_rank_dy(Act act, const void* dY, const float* B, const float* xA, int M, int N,
-                           int r, float c, const RankPlan& p, float* G, float* dB, float* dbias,
-                           float* wsf, cudaStream_t s) {
-    float* Gp = wsf;
-    float* dBp = Gp + static_cast<size_t>(p.n_col_blocks) * M * r;
-    float* dbp = dBp + static_cast<size_t>(p.n_chunks) * r * N;
-    dim3 grid(p.n_col_blocks, p.n_chunks);
+                           int r, float c, float* Gp, float* dB, float* dbias, float* G,
+                           cudaStream_t s) {
+    const int cl = cluster_for(M);
+    const int RM = (M + cl - 1) / cl;
+    const dim3 grid(rank_col_blocks(N), cl);
     for (int j0 = 0; j0 < r; j0 += kRJ) {
+        cudaError_t e;
         if (act == kBF16)
-            k4_dy_pass_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(
-                static_cast<const __nv_bfloat16*>(dY), B, xA, M, N, r, j0, p.rows_per_chunk, Gp,
-                dBp, dbias ? dbp : nullptr);
+            e = launch_clustered(k4_dy_kernel<__nv_bfloat16>, grid, cl, s,
+                                 static_cast<const __nv_bfloat16*>(dY), B, xA, M, N, r, j0, RM, c,
+                                 Gp, dB, dbias);
         else
-            k4_dy_pass_kernel<float><<<grid, kThreads, 0, s>>>(static_cast<const float*>(dY), B, xA,
-                                                               M, N, r, j0, p.rows_per_chunk, Gp,
-                                                               dBp, dbias ? dbp : nullptr);
+            e = launch_clustered(k4_dy_kernel<float>, grid, cl, s, static_cast<const float*>(dY), B,
+                                 xA, M, N, r, j0, RM, c, Gp, dB, dbias);
+        if (e != cudaSuccess) return e;
     }
-    const size_t total = static_cast<size_t>(M) * r + static_cast<size_t>(r) * N + (dbias ? N : 0);
-    int blocks = static_cast<int>((total + 255) / 256);
-    if (blocks > 4 * 148) blocks = 4 * 148;
-    k4_reduce_dy_kernel<<<blocks, 256, 0, s>>>(Gp, dBp, dbp, M, N, r, p.n_col_blocks, p.n_chunks, c,
-                                                G, dB, dbias);
+    if (G) {
+        const size_t n = static_cast<size_t>(M) * r;
+        const int blocks = static_cast<int>((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
+        k4_g_reduce_kernel<<<blocks, 256, 0, s>>>(Gp, rank_col_blocks(N), n, G);
+    }
     return cudaGetLastError();
 }
 
-cudaError_t launch_rank_x(Act act, const void* X, const float* G, int M, int K, int r, float c,
-                          const RankPlan& p, float* dA, float* wsf, cudaStream_t s) {
-    float* dAp = wsf;
-    dim3 grid((K + kCols - 1) / kCols, p.k_chunks);
+cudaError_t launch_rank_x(Act act, const void* X, const float* Gp, int ncb, int M, int K, int r,
+                          float c, float* dA, cudaStream_t s) {
+    const int cl = cluster_for(M);
+    const int RM = (M + cl - 1) / cl;
+    const dim3 grid(rank_col_blocks(K), cl);
     for (int j0 = 0; j0 < r; j0 += kRJ) {
+        cudaError_t e;
         if (act == kBF16)
-            k4_x_pass_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(
-                static_cast<const __nv_bfloat16*>(X), G, M, K, r, j0, p.rows_per_kchunk, dAp);
+            e = launch_clustered(k4_x_kernel<__nv_bfloat16>, grid, cl, s,
+                                 static_cast<const __nv_bfloat16*>(X), Gp, ncb, M, K, r, j0, RM, c, dA);
         else
-            k4_x_pass_kernel<float><<<grid, kThreads, 0, s>>>(static_cast<const float*>(X), G, M, K,
-                                                              r, j0, p.rows_per_kchunk, dAp);
+            e = launch_clustered(k4_x_kernel<float>, grid, cl, s, static_cast<const float*>(X), Gp,
+                                 ncb, M, K, r, j0, RM, c, dA);
+        if (e != cudaSuccess) return e;
     }
-    const size_t total = static_cast<size_t>(K) * r;
-    int blocks = static_cast<int>((total + 255) / 256);
-    if (blocks > 4 * 148) blocks = 4 * 148;
-    k4_reduce_x_kernel<<<blocks, 256, 0, s>>>(dAp, K, r, p.k_chunks, c, dA);
     return cudaGetLastError();
 }
 

@@ -158,6 +158,18 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
         : "memory");
 }
 
+// D[tmem] (+)= A x B, tf32 x tf32 -> fp32 (operands are fp32 words in smem;
+// the tensor core uses their tf32 part).
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrives (once) on `bar` when all previously issued MMAs of this thread finish.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile(
@@ -216,6 +228,32 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n, bool a_mn_major,
     return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
            ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(n >> 3) << 17) |
            (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// kind::tf32, fp32 accumulate, both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_tf32(int m, int n) {
+    return (1u << 4) | (2u << 7) | (2u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+constexpr uint32_t kLayoutNone = 0;
+
+// Byte offset of element (row, k) of a K-major fp32 operand table with `kl`
+// columns in the no-swizzle canonical layout: 8-row x 16-byte core matrices,
+// core matrices adjacent in K 128 bytes apart (leading byte offset) and 8-row
+// groups kl/4 * 128 bytes apart (stride byte offset).
+__host__ __device__ constexpr uint32_t kmajor_tf32_offset(int row, int k, int kl) {
+    return static_cast<uint32_t>((row >> 3) * (kl / 4) * 128 + (k >> 2) * 128 + (row & 7) * 16 +
+                                 (k & 3) * 4);
+}
+
+// Splits x into a tf32 head (round to nearest, ties away) and the fp32
+// remainder, so that hi*hi' + hi*lo' + lo*hi' reproduces fp32 products.
+__device__ __forceinline__ void tf32_split(float x, float& hi, float& lo) {
+    uint32_t h;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(x));
+    hi = __uint_as_float(h);
+    lo = x - hi;
 }
 
 // ---------------------------------------------------------------------------

@@ -1,6 +1,8 @@
 // qlora_api.cu -- the C ABI of libqlora.so (declared in include/qlora.h):
 // argument validation, workspace layout, tensor-map encoding and the launch
 // sequence of each call.  No device memory is allocated here.
+#include <cstdlib>
+#include <map>
 #include <mutex>
 #include <set>
 #include <string>
@@ -62,11 +64,14 @@ EncodeTiledFn encode_fn() {
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Forward: Xq [M,K] int8 and sx [M] fp32.  Backward: the G slices
+// Gp [ncb][M,r] fp32 (written by the dY pass, read by the dX GEMM and the X
+// pass).  The two uses do not overlap in time.
 struct WsLayout {
     size_t xq, sx, fwd_total;
-    size_t g, part, bwd_total;
+    size_t gp, bwd_total;
+    int ncb;
     size_t total;
-    RankPlan plan;
 };
 
 WsLayout layout_for(const qlora_layer_desc& d, int M) {
@@ -74,10 +79,9 @@ WsLayout layout_for(const qlora_layer_desc& d, int M) {
     w.xq = 0;
     w.sx = align256(static_cast<size_t>(M) * d.K);
     w.fwd_total = w.sx + align256(static_cast<size_t>(M) * 4);
-    w.plan = plan_rank(M, d.K, d.N, d.r);
-    w.g = 0;
-    w.part = align256(static_cast<size_t>(M) * d.r * 4);
-    w.bwd_total = w.part + align256(rank_workspace_floats(w.plan, M, d.K, d.N, d.r) * 4);
+    w.gp = 0;
+    w.ncb = rank_col_blocks(d.N);
+    w.bwd_total = align256(rank_workspace_floats(M, d.N, d.r) * 4);
     w.total = w.fwd_total > w.bwd_total ? w.fwd_total : w.bwd_total;
     return w;
 }
@@ -118,6 +122,18 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+int tile_override(const char* name) {
+    static std::mutex mu;
+    static std::map<std::string, int> cache;
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = cache.find(name);
+    if (it != cache.end()) return it->second;
+    const char* v = std::getenv(name);
+    const int val = (v && *v) ? std::atoi(v) : -1;
+    cache[name] = val;
+    return val;
 }
 
 int sm_count() {
@@ -250,14 +266,14 @@ int qlora_gemm_forward(const qlora_layer_desc* d, int M, const int8_t* Xq, const
 }
 
 int qlora_lora_grad_dy(const qlora_layer_desc* d, int M, const void* dY, const float* B,
-                       const float* xA, float* G, float* dB, float* dbias, void* workspace,
+                       const float* xA, float* dB, float* dbias, float* G, void* workspace,
                        size_t workspace_bytes, void* stream) {
     int rc = check_layer(d, M);
     if (rc != QLORA_OK) return rc;
-    QL_REQUIRE(dY && B && xA && G && dB && workspace, QLORA_EINVAL, "NULL pointer argument");
+    QL_REQUIRE(dY && B && xA && dB && workspace, QLORA_EINVAL, "NULL pointer argument");
     QL_REQUIRE(aligned(dY, 16) && aligned(workspace, 256), QLORA_EALIGN,
                "dY must be 16-byte aligned, workspace 256-byte aligned");
-    QL_REQUIRE(aligned(B, 4) && aligned(xA, 4) && aligned(G, 4) && aligned(dB, 4) &&
+    QL_REQUIRE(aligned(B, 4) && aligned(xA, 4) && (!G || aligned(G, 4)) && aligned(dB, 4) &&
                    (!dbias || aligned(dbias, 4)),
                QLORA_EALIGN, "fp32 vectors must be 4-byte aligned");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -269,26 +285,29 @@ int qlora_lora_grad_dy(const qlora_layer_desc* d, int M, const void* dY, const f
     }
     const WsLayout w = layout_for(*d, M);
     QL_REQUIRE(workspace_bytes >= w.total, QLORA_EINVAL, "workspace too small");
-    float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.part);
-    return cuda_status(launch_rank_dy(act_of(d), dY, B, xA, M, d->N, d->r, lora_scale(d), w.plan,
-                                      G, dB, dbias, part, s),
+    float* gp = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.gp);
+    return cuda_status(launch_rank_dy(act_of(d), dY, B, xA, M, d->N, d->r, lora_scale(d), gp, dB,
+                                      dbias, G, s),
                        "dY pass launch");
 }
 
 int qlora_gemm_dx(const qlora_layer_desc* d, int M, const void* dY, const int8_t* Wq,
-                  const float* sw, const float* G, const float* A, void* dX, void* stream) {
+                  const float* sw, const float* A, void* dX, const void* workspace,
+                  size_t workspace_bytes, void* stream) {
     int rc = check_layer(d, M);
     if (rc != QLORA_OK) return rc;
-    QL_REQUIRE(dY && Wq && sw && G && A && dX, QLORA_EINVAL, "NULL pointer argument");
-    QL_REQUIRE(aligned(dY, 16) && aligned(Wq, 16) && aligned(dX, 16), QLORA_EALIGN,
-               "dY, Wq and dX must be 16-byte aligned");
-    QL_REQUIRE(aligned(sw, 4) && aligned(G, 4) && aligned(A, 4), QLORA_EALIGN,
-               "fp32 vectors must be 4-byte aligned");
+    QL_REQUIRE(dY && Wq && sw && A && dX && workspace, QLORA_EINVAL, "NULL pointer argument");
+    QL_REQUIRE(aligned(dY, 16) && aligned(Wq, 16) && aligned(dX, 16) && aligned(workspace, 256),
+               QLORA_EALIGN, "dY, Wq and dX must be 16-byte aligned, workspace 256-byte aligned");
+    QL_REQUIRE(aligned(sw, 4) && aligned(A, 4), QLORA_EALIGN, "fp32 vectors must be 4-byte aligned");
     if (M == 0) return QLORA_OK;
+    const WsLayout w = layout_for(*d, M);
+    QL_REQUIRE(workspace_bytes >= w.total, QLORA_EINVAL, "workspace too small");
     int* status = status_ptr();
     QL_REQUIRE(status, QLORA_ECUDA, "no CUDA device");
     DxEpilogue ep;
-    ep.G = G;
+    ep.Gp = reinterpret_cast<const float*>(static_cast<const uint8_t*>(workspace) + w.gp);
+    ep.ncb = w.ncb;
     ep.A = A;
     ep.r = d->r;
     ep.c = lora_scale(d);
@@ -298,21 +317,20 @@ int qlora_gemm_dx(const qlora_layer_desc* d, int M, const void* dY, const int8_t
                        "dX GEMM launch");
 }
 
-int qlora_lora_grad_x(const qlora_layer_desc* d, int M, const void* X, const float* G, float* dA,
-                      void* workspace, size_t workspace_bytes, void* stream) {
+int qlora_lora_grad_x(const qlora_layer_desc* d, int M, const void* X, float* dA,
+                      const void* workspace, size_t workspace_bytes, void* stream) {
     int rc = check_layer(d, M);
     if (rc != QLORA_OK) return rc;
-    QL_REQUIRE(X && G && dA && workspace, QLORA_EINVAL, "NULL pointer argument");
+    QL_REQUIRE(X && dA && workspace, QLORA_EINVAL, "NULL pointer argument");
     QL_REQUIRE(aligned(X, 16) && aligned(workspace, 256), QLORA_EALIGN,
                "X must be 16-byte aligned, workspace 256-byte aligned");
-    QL_REQUIRE(aligned(G, 4) && aligned(dA, 4), QLORA_EALIGN, "fp32 vectors must be 4-byte aligned");
+    QL_REQUIRE(aligned(dA, 4), QLORA_EALIGN, "fp32 vectors must be 4-byte aligned");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (M == 0) return cuda_status(cudaMemsetAsync(dA, 0, sizeof(float) * d->K * d->r, s), "memset dA");
     const WsLayout w = layout_for(*d, M);
     QL_REQUIRE(workspace_bytes >= w.total, QLORA_EINVAL, "workspace too small");
-    float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.part);
-    return cuda_status(launch_rank_x(act_of(d), X, G, M, d->K, d->r, lora_scale(d), w.plan, dA,
-                                     part, s),
+    const float* gp = reinterpret_cast<const float*>(static_cast<const uint8_t*>(workspace) + w.gp);
+    return cuda_status(launch_rank_x(act_of(d), X, gp, w.ncb, M, d->K, d->r, lora_scale(d), dA, s),
                        "X pass launch");
 }
 
@@ -370,14 +388,13 @@ int qlora_backward(const qlora_layer_desc* d, int M, const void* X, const void* 
     }
     const WsLayout w = layout_for(*d, M);
     QL_REQUIRE(workspace_bytes >= w.total, QLORA_EINVAL, "workspace too small");
-    float* G = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.g);
-    rc = qlora_lora_grad_dy(d, M, dY, B, xA, G, dB, dbias, workspace, workspace_bytes, stream);
+    rc = qlora_lora_grad_dy(d, M, dY, B, xA, dB, dbias, nullptr, workspace, workspace_bytes, stream);
     if (rc != QLORA_OK) return rc;
     if (dX) {
-        rc = qlora_gemm_dx(d, M, dY, Wq, sw, G, A, dX, stream);
+        rc = qlora_gemm_dx(d, M, dY, Wq, sw, A, dX, workspace, workspace_bytes, stream);
         if (rc != QLORA_OK) return rc;
     }
-    return qlora_lora_grad_x(d, M, X, G, dA, workspace, workspace_bytes, stream);
+    return qlora_lora_grad_x(d, M, X, dA, workspace, workspace_bytes, stream);
 }
 
 int qlora_merge(const qlora_layer_desc* d, const int8_t* Wq, const float* sw, const float* A,

@@ -79,8 +79,8 @@ def _load():
     lib.qlora_quantize_input.argtypes = [D, I, P, P, P, P, P, P]
     lib.qlora_gemm_forward.argtypes = [D, I, P, P, P, P, P, P, P, P, P, P]
     lib.qlora_lora_grad_dy.argtypes = [D, I, P, P, P, P, P, P, P, Z, P]
-    lib.qlora_gemm_dx.argtypes = [D, I, P, P, P, P, P, P, P]
-    lib.qlora_lora_grad_x.argtypes = [D, I, P, P, P, P, Z, P]
+    lib.qlora_gemm_dx.argtypes = [D, I, P, P, P, P, P, P, Z, P]
+    lib.qlora_lora_grad_x.argtypes = [D, I, P, P, P, Z, P]
     for f in (lib.qlora_quantize_input, lib.qlora_gemm_forward, lib.qlora_lora_grad_dy,
               lib.qlora_gemm_dx, lib.qlora_lora_grad_x):
         f.restype = I
@@ -188,19 +188,21 @@ def qlora_gemm_forward(d: LayerDesc, M: int, Xq, sx, Wq, sw, bias, xA, B, Y, acc
                                    _ptr(bias), _ptr(xA), _ptr(B), _ptr(Y), _ptr(acc), _stream(stream)))
 
 
-def qlora_lora_grad_dy(d: LayerDesc, M: int, dY, B, xA, G, dB, dbias, ws, stream=None):
-    _check(_lib.qlora_lora_grad_dy(ctypes.byref(d), int(M), _ptr(dY), _ptr(B), _ptr(xA), _ptr(G),
-                                   _ptr(dB), _ptr(dbias), _ptr(ws), ws.numel(), _stream(stream)))
+def qlora_lora_grad_dy(d: LayerDesc, M: int, dY, B, xA, dB, dbias, ws, G=None, stream=None):
+    """dB, dbias; leaves G in `ws` for qlora_gemm_dx / qlora_lora_grad_x (and
+    writes the summed G too when a tensor is given)."""
+    _check(_lib.qlora_lora_grad_dy(ctypes.byref(d), int(M), _ptr(dY), _ptr(B), _ptr(xA), _ptr(dB),
+                                   _ptr(dbias), _ptr(G), _ptr(ws), ws.numel(), _stream(stream)))
 
 
-def qlora_gemm_dx(d: LayerDesc, M: int, dY, Wq, sw, G, A, dX, stream=None):
-    _check(_lib.qlora_gemm_dx(ctypes.byref(d), int(M), _ptr(dY), _ptr(Wq), _ptr(sw), _ptr(G),
-                              _ptr(A), _ptr(dX), _stream(stream)))
+def qlora_gemm_dx(d: LayerDesc, M: int, dY, Wq, sw, A, dX, ws, stream=None):
+    _check(_lib.qlora_gemm_dx(ctypes.byref(d), int(M), _ptr(dY), _ptr(Wq), _ptr(sw), _ptr(A),
+                              _ptr(dX), _ptr(ws), ws.numel(), _stream(stream)))
 
 
-def qlora_lora_grad_x(d: LayerDesc, M: int, X, G, dA, ws, stream=None):
-    _check(_lib.qlora_lora_grad_x(ctypes.byref(d), int(M), _ptr(X), _ptr(G), _ptr(dA), _ptr(ws),
-                                  ws.numel(), _stream(stream)))
+def qlora_lora_grad_x(d: LayerDesc, M: int, X, dA, ws, stream=None):
+    _check(_lib.qlora_lora_grad_x(ctypes.byref(d), int(M), _ptr(X), _ptr(dA), _ptr(ws), ws.numel(),
+                                  _stream(stream)))
 
 
 def qlora_relu(Y: torch.Tensor, stream=None):

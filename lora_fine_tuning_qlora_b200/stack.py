@@ -74,9 +74,9 @@ class MLPStack:
             n += 2                                   # quantize+xA, int8 GEMM
             n += 1 if i < len(self.layers) - 1 else 0  # ReLU
             rj = (L.r + 7) // 8
-            n += rj + 1                              # dY pass(es) + reduction
+            n += rj                                  # dY pass(es), cluster-reduced
             n += 1                                   # dX GEMM
-            n += rj + 1                              # X pass(es) + reduction
+            n += rj                                  # X pass(es), cluster-reduced
             n += 1 if i < len(self.layers) - 1 else 0  # ReLU backward
         return n
 
@@ -109,14 +109,14 @@ class MLPStack:
                 qlora.qlora_relu_backward(g, self.H[i], stream)
             x_in = self.X if i == 0 else self.H[i - 1]
             dX = self.dX if i == 0 else self.G[i - 1]
-            qlora.qlora_lora_grad_dy(D[i], M, g, L.B, self.xA[i], self.Gr, self.dB[i],
-                                     self.dbias[i], self.ws, stream)
+            qlora.qlora_lora_grad_dy(D[i], M, g, L.B, self.xA[i], self.dB[i], self.dbias[i],
+                                     self.ws, None, stream)
             if ev_d:
                 ev_d[i][0].record()
-            qlora.qlora_gemm_dx(D[i], M, g, L.Wq, L.sw, self.Gr, L.A, dX, stream)
+            qlora.qlora_gemm_dx(D[i], M, g, L.Wq, L.sw, L.A, dX, self.ws, stream)
             if ev_d:
                 ev_d[i][1].record()
-            qlora.qlora_lora_grad_x(D[i], M, x_in, self.Gr, self.dA[i], self.ws, stream)
+            qlora.qlora_lora_grad_x(D[i], M, x_in, self.dA[i], self.ws, stream)
             g = dX
 
     def make_events(self, kinds=("gemm_dx",)):

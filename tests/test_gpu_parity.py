@@ -199,3 +199,55 @@ def test_mlp_stack_full(q):
     for i in range(len(specs)):
         assert_close(to_np(out["dA"][i]), ref["grads"][i]["dA"], "bf16", "dA[%d]" % i)
         assert_close(to_np(out["dB"][i]), ref["grads"][i]["dB"], "bf16", "dB[%d]" % i)
+
+
+def test_step_level_calls_match_composite(q):
+    """a1..a5 called one by one (G left in the workspace by a3, also
+    materialised on request) give the composite forward/backward results."""
+    spec = _edge_spec(200, 384, 264, 8, seed=11)
+    d = inputs.layer_inputs(spec)
+    from parity import device_layer
+    layer = device_layer(spec, d, q)
+    X = torch.from_numpy(d["X"]).to(torch.bfloat16).cuda()
+    dY = torch.from_numpy(d["dY"]).to(torch.bfloat16).cuda()
+    ws = q.workspace(layer.desc(), spec.M)
+    Y, xA = q.forward(layer, X, ws)
+    dX, dA, dB, db = q.backward(layer, X, dY, xA, ws)
+    D = layer.desc()
+    M = spec.M
+    Xq = torch.empty((M, spec.K), dtype=torch.int8, device="cuda")
+    sx = torch.empty((M,), device="cuda")
+    xA2 = torch.empty_like(xA)
+    Y2 = torch.empty_like(Y)
+    q.qlora_quantize_input(D, M, X, layer.A, Xq, sx, xA2)
+    q.qlora_gemm_forward(D, M, Xq, sx, layer.Wq, layer.sw, layer.bias, xA2, layer.B, Y2)
+    dB2 = torch.empty_like(dB)
+    db2 = torch.empty_like(db)
+    G = torch.empty((M, spec.r), device="cuda")
+    q.qlora_lora_grad_dy(D, M, dY, layer.B, xA2, dB2, db2, ws, G)
+    dX2 = torch.empty_like(dX)
+    q.qlora_gemm_dx(D, M, dY, layer.Wq, layer.sw, layer.A, dX2, ws)
+    dA2 = torch.empty_like(dA)
+    q.qlora_lora_grad_x(D, M, X, dA2, ws)
+    torch.cuda.synchronize()
+    for a, b in ((Y, Y2), (dX, dX2), (dA, dA2), (dB, dB2), (db, db2)):
+        assert torch.equal(a, b)
+    G_ref = oracle.backward(d["X"], d["dY"], *oracle.quantize_weight(d["W"]), d["A"], d["B"],
+                            spec.alpha, want_dx=False)["G"]
+    assert_close(to_np(G), G_ref, "bf16", "G")
+
+
+def test_relu_kernels(q):
+    """The stack's elementwise ReLU and its backward, aligned and unaligned."""
+    rng = np.random.Generator(np.random.PCG64(21))
+    for dtype in (torch.bfloat16, torch.float32):
+        x = torch.from_numpy(rng.normal(0, 1, 1003).astype(np.float32)).to(dtype).cuda()
+        for off in (0, 1):
+            y = x[off:].clone() if off == 0 else x.clone()[off:]
+            ref = torch.clamp(y.float(), min=0)
+            q.qlora_relu(y)
+            g = torch.ones_like(y)
+            q.qlora_relu_backward(g, y)
+            torch.cuda.synchronize()
+            assert torch.equal(y.float(), ref)
+            assert torch.equal(g.float(), (ref > 0).float())
