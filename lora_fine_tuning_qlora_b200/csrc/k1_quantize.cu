@@ -152,6 +152,8 @@ __global__ void __launch_bounds__(kThreads) k1_quantize_rows_kernel(
     const T* __restrict__ X, const float* __restrict__ A, int M, int K, int r, int a_chunks,
     int8_t* __restrict__ Xq, float* __restrict__ sx, float* __restrict__ xA) {
     constexpr int RPB = kThreads / TPR;
+    pdl_trigger();
+    pdl_wait();
     extern __shared__ float4 smem_f4[];
     float* sA = reinterpret_cast<float*>(smem_f4);
     __shared__ float red[kThreads / 32];
@@ -238,6 +240,8 @@ template <typename T, int RP>
 __global__ void __launch_bounds__(kThreads) k1_quantize_rows_long_kernel(
     const T* __restrict__ X, const float* __restrict__ A, int M, int K, int r, int a_chunks,
     int8_t* __restrict__ Xq, float* __restrict__ sx, float* __restrict__ xA) {
+    pdl_trigger();
+    pdl_wait();
     extern __shared__ float4 smem_f4[];
     float* sA = reinterpret_cast<float*>(smem_f4);
     __shared__ float red[kThreads / 32];
@@ -293,8 +297,7 @@ cudaError_t launch_tpr(const T* X, const float* A, int M, int K, int r, int8_t* 
     const int per_sm = smem <= 48 * 1024 ? 4 : (smem <= 100 * 1024 ? 2 : 1);
     int grid = groups;
     if (a_chunks >= nchunks && grid > per_sm * sm_count()) grid = per_sm * sm_count();
-    kern<<<grid, kThreads, smem, s>>>(X, A, M, K, r, a_chunks, Xq, sx, xA);
-    return cudaGetLastError();
+    return launch_k(kern, dim3(grid), dim3(kThreads), smem, s, 1, X, A, M, K, r, a_chunks, Xq, sx, xA);
 }
 
 template <typename T, int RP>
@@ -310,9 +313,8 @@ cudaError_t launch_rows_rp(const T* X, const float* A, int M, int K, int r, int8
     auto kern = k1_quantize_rows_long_kernel<T, RP>;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), kSmemCap);
     if (e != cudaSuccess) return e;
-    kern<<<M, kThreads, a_chunks * a_chunk_floats<RP>() * 4, s>>>(X, A, M, K, r, a_chunks, Xq, sx,
-                                                                  xA);
-    return cudaGetLastError();
+    return launch_k(kern, dim3(M), dim3(kThreads), a_chunks * a_chunk_floats<RP>() * 4, s, 1, X, A, M,
+                    K, r, a_chunks, Xq, sx, xA);
 }
 
 template <typename T>

@@ -85,6 +85,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int num_n = (N + BN - 1) / BN;
     const int tiles = ((M + kBM - 1) / kBM) * num_n;
     const int nkb = (K + kBK - 1) / kBK;
+    pdl_trigger();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -106,6 +107,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();  // the prologue above touched no global memory
 
     if (warp == 0) {
         // ------------------------------------------------------ producer
@@ -326,8 +328,7 @@ cudaError_t launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, int M, int 
     if (e != cudaSuccess) return e;
     const int tiles = ((M + kBM - 1) / kBM) * ((N + BN - 1) / BN);
     const int grid = tiles < sm_count() ? tiles : sm_count();
-    kern<<<grid, kThreads, C::kTotal, s>>>(ta, tb, M, N, K, ep, status);
-    return cudaGetLastError();
+    return launch_k(kern, dim3(grid), dim3(kThreads), C::kTotal, s, 1, ta, tb, M, N, K, ep, status);
 }
 
 template <typename OutT, int RMAX>

@@ -82,16 +82,48 @@ __device__ __forceinline__ uint32_t mn_sw128_offset(int mn, int kr, uint32_t lbo
 
 // G[m,j] = sum over the column-block slices of G (fixed order).
 __device__ __forceinline__ float g_row(const DxEpilogue& ep, int M, int m, int j) {
-    const float* p = ep.Gp + static_cast<size_t>(m) * ep.r + j;
-    const size_t slice = static_cast<size_t>(M) * ep.r;
-    float s = __ldg(p);
-    for (int b = 1; b < ep.ncb; ++b) s += __ldg(p + b * slice);
-    return s;
+    return sum_slices(ep.Gp + static_cast<size_t>(m) * ep.r + j, static_cast<size_t>(M) * ep.r,
+                      ep.ncb);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ unsigned long long f2(float a, float b) {
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+// 16 int8 codes (one 16-byte chunk, element i in byte i) -> 8 words of packed
+// bf16 pairs holding bf16(fl32(q * scale)).  Each code becomes the exact
+// float 2^23 + (q + 128) by a byte permute into 0x4B000000, an exact add of
+// -(2^23 + 128) recovers q, then one fp32 multiply by the scale (pairs of
+// lanes in f32x2 instructions) and a round-to-nearest-even to bf16: the same
+// value as converting q to float and multiplying, at full ALU rate.
+__device__ __forceinline__ void dequant16(const uint4 raw, float scale, uint32_t (&o)[8]) {
+    const uint32_t w[4] = {raw.x ^ 0x80808080u, raw.y ^ 0x80808080u, raw.z ^ 0x80808080u,
+                           raw.w ^ 0x80808080u};
+    const unsigned long long bias2 = f2(-8388736.0f, -8388736.0f);
+    const unsigned long long sc2 = f2(scale, scale);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        unsigned long long lo = f2(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7540)),
+                                   __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7541)));
+        unsigned long long hi = f2(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7542)),
+                                   __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7543)));
+        asm("add.rn.f32x2 %0, %0, %1;" : "+l"(lo) : "l"(bias2));
+        asm("add.rn.f32x2 %0, %0, %1;" : "+l"(hi) : "l"(bias2));
+        asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(lo) : "l"(sc2));
+        asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(hi) : "l"(sc2));
+        float a, b, c, d;
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(lo));
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(c), "=f"(d) : "l"(hi));
+        o[2 * i] = pack_bf16x2(a, b);
+        o[2 * i + 1] = pack_bf16x2(c, d);
+    }
 }
 
 template <int MSUB, int BN, int RMAX>
@@ -119,11 +151,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int num_k = (K + BN - 1) / BN;
     const int tiles = ((M + C::kBM - 1) / C::kBM) * num_k;
     const int nkb = (N + kBKn - 1) / kBKn;
+    pdl_trigger();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&wready[s], C::kDqPerStage);  // the stage's de-quantize warps
+            mbar_init(&wready[s], kDqWarps);  // every de-quantize warp, once per fill
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -141,6 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();  // the prologue above touched no global memory
 
     if (warp == 0) {
         // ------------------------------------------------------ producer
@@ -228,49 +262,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp < 2 + kDqWarps) {
         // ------------------------------------------------------ de-quantize
-        // Each warp owns one ring stage (C::kDqPerStage warps share a stage
-        // when the ring is short) and converts every fill of that stage, in
-        // order, so its barrier phases are awaited one after the other and
-        // the stages are converted concurrently.
+        // All eight warps convert every stage, each its own slice of the
+        // chunks, walking the stages in order (so every barrier phase is
+        // awaited in turn); a warp's row scales are loaded before it waits
+        // for the stage, so no global load sits on the conversion path.
         const int dw = warp - 2;  // 0 .. 7
         constexpr int kChunksPerRow = BN / 16;
         constexpr int kChunks = kBKn * kChunksPerRow;
-        constexpr int kPer = C::kDqPerStage;
-        const int my_stage = dw / kPer;
-        const int part = dw % kPer;
+        constexpr int kPerLane = kChunks / (32 * kDqWarps);
+        static_assert(kChunks % (32 * kDqWarps) == 0, "chunks per stage");
         const int my_tiles = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
         const int total_kb = my_tiles * nkb;
-        for (int g = my_stage; my_stage < S && g < total_kb; g += S) {
-            const int s = my_stage;
+        for (int g = 0; g < total_kb; ++g) {
+            const int s = g % S;
             const int kb = g % nkb;
-            // the 64 row scales of this stage: lane l holds rows l and l + 32
-            const int nbase = kb * kBKn;
-            const float sc0 = nbase + lane < N ? __ldg(sw + nbase + lane) : 0.f;
-            const float sc1 = nbase + 32 + lane < N ? __ldg(sw + nbase + 32 + lane) : 0.f;
+            float scl[kPerLane];
+#pragma unroll
+            for (int i = 0; i < kPerLane; ++i) {
+                const int n = kb * kBKn + (dw * 32 + lane + i * 32 * kDqWarps) / kChunksPerRow;
+                scl[i] = n < N ? __ldg(sw + n) : 0.f;
+            }
             if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (g / S) & 1, status))) break;
             {
                 const uint8_t* sq = smem + s * C::kStageBytes + C::kABytes;
                 uint8_t* wt = smem + s * C::kStageBytes + C::kABytes + C::kQBytes;
 #pragma unroll
-                for (int c = part * 32 + lane; c < kChunks; c += 32 * kPer) {
+                for (int i = 0; i < kPerLane; ++i) {
+                    const int c = dw * 32 + lane + i * 32 * kDqWarps;
                     const int nr = c / kChunksPerRow;   // contraction row within the stage
                     const int kc = c % kChunksPerRow;   // 16 output columns
-                    const float s0 = __shfl_sync(0xffffffffu, sc0, nr & 31);
-                    const float s1 = __shfl_sync(0xffffffffu, sc1, nr & 31);
-                    const float scale = nr < 32 ? s0 : s1;
+                    const float scale = scl[i];
                     const uint4 raw = *reinterpret_cast<const uint4*>(sq + nr * BN + kc * 16);
-                    const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
                     uint32_t o[8];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int32_t b = static_cast<int32_t>(w4[i]);
-                        const float f0 = __fmul_rn(static_cast<float>((b << 24) >> 24), scale);
-                        const float f1 = __fmul_rn(static_cast<float>((b << 16) >> 24), scale);
-                        const float f2 = __fmul_rn(static_cast<float>((b << 8) >> 24), scale);
-                        const float f3 = __fmul_rn(static_cast<float>(b >> 24), scale);
-                        o[2 * i] = pack_bf16x2(f0, f1);
-                        o[2 * i + 1] = pack_bf16x2(f2, f3);
-                    }
+                    dequant16(raw, scale, o);
                     const int mn = kc * 16;
                     *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn, nr, kLbo)) =
                         make_uint4(o[0], o[1], o[2], o[3]);
@@ -383,8 +407,8 @@ cudaError_t launch_tc(const CUtensorMap& tdy, const CUtensorMap& tq, const float
     if (e != cudaSuccess) return e;
     const int tiles = ((M + C::kBM - 1) / C::kBM) * ((K + BN - 1) / BN);
     const int grid = tiles < sm_count() ? tiles : sm_count();
-    kern<<<grid, kThreads, C::kTotal, s>>>(tdy, tq, sw, M, N, K, ep, status);
-    return cudaGetLastError();
+    return launch_k(kern, dim3(grid), dim3(kThreads), C::kTotal, s, 1, tdy, tq, sw, M, N, K, ep,
+                    status);
 }
 
 template <int RMAX>
@@ -409,6 +433,8 @@ __global__ void __launch_bounds__(256) k3_dx_simt_kernel(const T* __restrict__ d
                                                          int N, int K, DxEpilogue ep) {
     __shared__ float sD[kSN][kSB + 1];  // [n][m]
     __shared__ float sW[kSN][kSB + 1];  // [n][k]
+    pdl_trigger();
+    pdl_wait();
     const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
     const int m0 = blockIdx.y * kSB, k0 = blockIdx.x * kSB;
     float acc[4][4] = {};
@@ -475,12 +501,10 @@ cudaError_t launch_gemm_dx(Act act, const void* dY, const int8_t* Wq, const floa
     if (!tc) {
         dim3 grid((K + kSB - 1) / kSB, (M + kSB - 1) / kSB);
         if (act == kBF16)
-            k3_dx_simt_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-                static_cast<const __nv_bfloat16*>(dY), Wq, sw, M, N, K, ep);
-        else
-            k3_dx_simt_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(dY), Wq, sw, M, N,
-                                                          K, ep);
-        return cudaGetLastError();
+            return launch_k(k3_dx_simt_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, 1,
+                            static_cast<const __nv_bfloat16*>(dY), Wq, sw, M, N, K, ep);
+        return launch_k(k3_dx_simt_kernel<float>, grid, dim3(256), 0, s, 1,
+                        static_cast<const float*>(dY), Wq, sw, M, N, K, ep);
     }
     // tile shape: the largest that still gives every SM a tile
     const int sms = sm_count();

@@ -12,15 +12,15 @@
 // pass streams its matrix once from HBM with 128-bit loads and does 2r FMAs
 // per element on CUDA cores.
 //
-// Layout of the work: a CTA owns 128 columns (16 lanes x 8) and a chunk of
-// rows; the CL <= 8 CTAs that own the chunks of one column block form a
-// thread-block cluster along the rows.  Each CTA reduces its rows in
-// registers and shared memory, then the cluster sums the CL partial results
-// through distributed shared memory, rank by rank, so dB, dbias and dA leave
-// the kernel final, with a fixed summation order (deterministic) and no
-// second launch.  G's per-row sums over the column blocks stay as partial
-// slices Gp in the workspace; the two consumers (the dX GEMM and the X pass)
-// add the slices up themselves.
+// Layout of the work: a CTA owns 64 columns (8 lanes x 8, so a warp covers
+// four rows per load) and a chunk of rows; the CL <= 8 CTAs that own the
+// chunks of one column block form a thread-block cluster along the rows.
+// Each CTA reduces its rows in registers and shared memory, then the cluster
+// sums the CL partial results through distributed shared memory, rank by
+// rank, so dB, dbias and dA leave the kernel final, with a fixed summation
+// order (deterministic) and no second launch.  G's per-row sums over the
+// column blocks stay as partial slices Gp in the workspace; the two
+// consumers (the dX GEMM and the X pass) add the slices up themselves.
 #include <cooperative_groups.h>
 
 #include "internal.h"
@@ -34,12 +34,14 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kCols = 128;         // columns per CTA: 16 lanes x 8
-constexpr int kRJ = 8;             // rank columns per sweep
+constexpr int kLanesPerRow = 8;
+constexpr int kCols = 8 * kLanesPerRow;             // 64 columns per CTA
+constexpr int kRowsPerWarp = 32 / kLanesPerRow;     // 4 rows per warp-wide load
+constexpr int kRowsPerPass = kRowsPerWarp * kWarps; // 32 rows per pass of the CTA
+constexpr int kRJ = 8;                              // rank columns per sweep
 constexpr int kMaxCluster = 8;
-constexpr int kRowsPerPass = 2 * kWarps;  // a half-warp per row
 constexpr int kPassesInFlight = 4;
-constexpr int kXRowBlock = 128;    // rows whose G is staged at a time (X pass)
+constexpr int kXRowBlock = 128;                     // rows whose G is staged at a time
 
 template <typename T>
 __device__ __forceinline__ void load8(const T* row, int c0, int ncols, bool vec, float (&v)[8]) {
@@ -65,33 +67,48 @@ __device__ __forceinline__ void load8(const T* row, int c0, int ncols, bool vec,
     }
 }
 
-// Sum of an 8-vector over the 16 lanes of a half-warp (xor offsets 8..1).  On
-// return, lane l holds the total of component (l >> 1) & 7 when (l & 1) == 0.
-__device__ __forceinline__ float half_reduce8(float (&v)[8], int lane) {
-    const bool b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
+// Sum of an 8-vector over the 8 lanes that share a row (xor offsets 4, 2, 1).
+// On return, lane l holds the total of component l & 7.  Fixed order.
+__device__ __forceinline__ float row_reduce8(float (&v)[8], int lane) {
+    const bool b2 = lane & 4, b1 = lane & 2, b0 = lane & 1;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const float send = b3 ? v[i] : v[i + 4];
-        const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
-        v[i] = (b3 ? v[i + 4] : v[i]) + recv;
+        const float send = b2 ? v[i] : v[i + 4];
+        const float recv = __shfl_xor_sync(0xffffffffu, send, 4);
+        v[i] = (b2 ? v[i + 4] : v[i]) + recv;
     }
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-        const float send = b2 ? v[i] : v[i + 2];
-        const float recv = __shfl_xor_sync(0xffffffffu, send, 4);
-        v[i] = (b2 ? v[i + 2] : v[i]) + recv;
-    }
-    {
-        const float send = b1 ? v[0] : v[1];
+        const float send = b1 ? v[i] : v[i + 2];
         const float recv = __shfl_xor_sync(0xffffffffu, send, 2);
-        v[0] = (b1 ? v[1] : v[0]) + recv;
+        v[i] = (b1 ? v[i + 2] : v[i]) + recv;
     }
-    return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+    const float send = b0 ? v[0] : v[1];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+    return (b0 ? v[1] : v[0]) + recv;
+}
+
+// Sum over the four row groups of a warp (lanes with equal lane & 7).
+__device__ __forceinline__ float warp_rows_sum(float v) {
+    v += __shfl_xor_sync(0xffffffffu, v, 8);
+    v += __shfl_xor_sync(0xffffffffu, v, 16);
+    return v;
+}
+
+// Cluster sum of part[idx] over the CL ranks, rank 0 first, loads issued first.
+__device__ __forceinline__ float cluster_sum(cg::cluster_group& cluster, float* part, int idx,
+                                             int CL) {
+    float v[kMaxCluster];
+#pragma unroll
+    for (int q = 0; q < kMaxCluster; ++q) v[q] = q < CL ? cluster.map_shared_rank(part, q)[idx] : 0.f;
+    float s = v[0];
+#pragma unroll
+    for (int q = 1; q < kMaxCluster; ++q)
+        if (q < CL) s += v[q];
+    return s;
 }
 
 // ---------------------------------------------------------------- dY pass
-// Shared memory: red[kWarps][(kRJ + 1) * kCols] (per-warp partials) and
-// part[(kRJ + 1) * kCols] (this CTA's partial, read by the cluster).
 template <typename T>
 __global__ void __launch_bounds__(kThreads) k4_dy_kernel(
     const T* __restrict__ dY, const float* __restrict__ B, const float* __restrict__ xA, int M,
@@ -100,23 +117,20 @@ __global__ void __launch_bounds__(kThreads) k4_dy_kernel(
     constexpr int kW = (kRJ + 1) * kCols;
     __shared__ float red[kWarps][kW];
     __shared__ float part[kW];
+    pdl_trigger();
+    pdl_wait();
     cg::cluster_group cluster = cg::this_cluster();
     const int CL = static_cast<int>(cluster.num_blocks());
     const int crank = static_cast<int>(cluster.block_rank());
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int half = lane >> 4, cl = lane & 15;
+    const int rg = lane / kLanesPerRow, cl = lane % kLanesPerRow;
     const int cb = blockIdx.x;
     const int c0 = cb * kCols + cl * 8;
     const int mbeg = blockIdx.y * RM;
     const int mend = min(M, mbeg + RM);
     const bool vec = (N % 8) == 0;
+    const int rowoff = warp * kRowsPerWarp + rg;
 
-    float bv[kRJ][8];
-#pragma unroll
-    for (int j = 0; j < kRJ; ++j)
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-            bv[j][e] = (j0 + j < r && c0 + e < N) ? __ldg(B + static_cast<size_t>(j0 + j) * N + c0 + e) : 0.f;
     float db[kRJ][8];
     float dbi[8];
 #pragma unroll
@@ -125,9 +139,11 @@ __global__ void __launch_bounds__(kThreads) k4_dy_kernel(
 #pragma unroll
         for (int j = 0; j < kRJ; ++j) db[j][e] = 0.f;
     }
+    float bv[kRJ][8];
+    bool have_b = false;
 
-    const int rowoff = 2 * warp + half;
     for (int pb = mbeg; pb < mend; pb += kRowsPerPass * kPassesInFlight) {
+        // every load of the pass group first: dY rows, their xA rows (and B once)
         float v[kPassesInFlight][8];
         float xr[kPassesInFlight][kRJ];
 #pragma unroll
@@ -141,6 +157,15 @@ __global__ void __launch_bounds__(kThreads) k4_dy_kernel(
 #pragma unroll
             for (int j = 0; j < kRJ; ++j)
                 xr[u][j] = (ok && j0 + j < r) ? __ldg(xA + static_cast<size_t>(m) * r + j0 + j) : 0.f;
+        }
+        if (!have_b) {
+#pragma unroll
+            for (int j = 0; j < kRJ; ++j)
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    bv[j][e] = (j0 + j < r && c0 + e < N) ? __ldg(B + static_cast<size_t>(j0 + j) * N + c0 + e)
+                                                          : 0.f;
+            have_b = true;
         }
 #pragma unroll
         for (int u = 0; u < kPassesInFlight; ++u) {
@@ -157,21 +182,19 @@ __global__ void __launch_bounds__(kThreads) k4_dy_kernel(
             }
 #pragma unroll
             for (int e = 0; e < 8; ++e) dbi[e] += v[u][e];
-            const float gs = half_reduce8(g, lane);  // all lanes take part
-            const int jj = (cl >> 1) & 7;
-            if (m < mend && (cl & 1) == 0 && j0 + jj < r)
-                Gp[(static_cast<size_t>(cb) * M + m) * r + j0 + jj] = gs;
+            const float gs = row_reduce8(g, lane);  // all lanes take part
+            if (m < mend && j0 + cl < r) Gp[(static_cast<size_t>(cb) * M + m) * r + j0 + cl] = gs;
         }
     }
 
-    // the two rows of a warp -> one partial per warp, then the warps in order
+    // the four row groups of a warp, then the warps in order
 #pragma unroll
     for (int j = 0; j < kRJ; ++j)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) db[j][e] += __shfl_xor_sync(0xffffffffu, db[j][e], 16);
+        for (int e = 0; e < 8; ++e) db[j][e] = warp_rows_sum(db[j][e]);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) dbi[e] += __shfl_xor_sync(0xffffffffu, dbi[e], 16);
-    if (half == 0) {
+    for (int e = 0; e < 8; ++e) dbi[e] = warp_rows_sum(dbi[e]);
+    if (rg == 0) {
 #pragma unroll
         for (int j = 0; j < kRJ; ++j)
 #pragma unroll
@@ -199,11 +222,7 @@ __global__ void __launch_bounds__(kThreads) k4_dy_kernel(
         if (n >= N) continue;
         if (j < kRJ && j0 + j >= r) continue;
         if (j == kRJ && !with_bias) continue;
-        float s = 0.f;
-        for (int q = 0; q < CL; ++q) {
-            const float* rp = cluster.map_shared_rank(part, q);
-            s = q == 0 ? rp[j * kCols + cc] : s + rp[j * kCols + cc];
-        }
+        const float s = cluster_sum(cluster, part, j * kCols + cc, CL);
         if (j < kRJ) dB[static_cast<size_t>(j0 + j) * N + n] = cscale * s;
         else dbias[n] = s;
     }
@@ -219,18 +238,21 @@ __global__ void __launch_bounds__(kThreads) k4_x_kernel(
     constexpr int kW = kCols * kRJ;
     __shared__ float red[kWarps][kW];
     __shared__ float part[kW];
-    __shared__ float sG[kXRowBlock][kRJ];
+    __shared__ __align__(16) float sG[kXRowBlock][kRJ];
+    pdl_trigger();
+    pdl_wait();
     cg::cluster_group cluster = cg::this_cluster();
     const int CL = static_cast<int>(cluster.num_blocks());
     const int crank = static_cast<int>(cluster.block_rank());
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int half = lane >> 4, cl = lane & 15;
+    const int rg = lane / kLanesPerRow, cl = lane % kLanesPerRow;
     const int cb = blockIdx.x;
     const int c0 = cb * kCols + cl * 8;
     const int mbeg = blockIdx.y * RM;
     const int mend = min(M, mbeg + RM);
     const bool vec = (K % 8) == 0;
     const size_t gslice = static_cast<size_t>(M) * r;
+    const int rowoff = warp * kRowsPerWarp + rg;
 
     float acc[8][kRJ];
 #pragma unroll
@@ -238,52 +260,45 @@ __global__ void __launch_bounds__(kThreads) k4_x_kernel(
 #pragma unroll
         for (int j = 0; j < kRJ; ++j) acc[e][j] = 0.f;
 
-    const int rowoff = 2 * warp + half;
     for (int rb = mbeg; rb < mend; rb += kXRowBlock) {
         const int rbe = min(mend, rb + kXRowBlock);
+        // this block's X rows go out before G is staged
+        float v[kXRowBlock / kRowsPerPass][8];
+#pragma unroll
+        for (int u = 0; u < kXRowBlock / kRowsPerPass; ++u) {
+            const int m = rb + u * kRowsPerPass + rowoff;
+            if (m < rbe) load8<T>(X + static_cast<size_t>(m) * K, c0, K, vec, v[u]);
+            else
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[u][e] = 0.f;
+        }
         __syncthreads();  // the previous block's G is no longer read
         for (int i = threadIdx.x; i < kXRowBlock * kRJ; i += kThreads) {
             const int rr = i / kRJ, j = i % kRJ;
             const int m = rb + rr;
-            float s = 0.f;
-            if (m < rbe && j0 + j < r) {
-                const float* p = Gp + static_cast<size_t>(m) * r + j0 + j;
-                s = __ldg(p);
-                for (int b = 1; b < ncb; ++b) s += __ldg(p + b * gslice);
-            }
-            sG[rr][j] = s;
+            sG[rr][j] = (m < rbe && j0 + j < r)
+                            ? sum_slices(Gp + static_cast<size_t>(m) * r + j0 + j, gslice, ncb)
+                            : 0.f;
         }
         __syncthreads();
-        for (int pb = rb; pb < rbe; pb += kRowsPerPass * kPassesInFlight) {
-            float v[kPassesInFlight][8];
 #pragma unroll
-            for (int u = 0; u < kPassesInFlight; ++u) {
-                const int m = pb + u * kRowsPerPass + rowoff;
-                if (m < rbe) load8<T>(X + static_cast<size_t>(m) * K, c0, K, vec, v[u]);
-                else
+        for (int u = 0; u < kXRowBlock / kRowsPerPass; ++u) {
+            const int rr = u * kRowsPerPass + rowoff;
+            const float4 g0 = *reinterpret_cast<const float4*>(&sG[rr][0]);
+            const float4 g1 = *reinterpret_cast<const float4*>(&sG[rr][4]);
+            const float g[kRJ] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) v[u][e] = 0.f;
-            }
+            for (int e = 0; e < 8; ++e)
 #pragma unroll
-            for (int u = 0; u < kPassesInFlight; ++u) {
-                const int rr = pb - rb + u * kRowsPerPass + rowoff;
-                if (rr >= kXRowBlock) break;
-                const float4 g0 = *reinterpret_cast<const float4*>(&sG[rr][0]);
-                const float4 g1 = *reinterpret_cast<const float4*>(&sG[rr][4]);
-                const float g[kRJ] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-#pragma unroll
-                    for (int j = 0; j < kRJ; ++j) acc[e][j] = fmaf(v[u][e], g[j], acc[e][j]);
-            }
+                for (int j = 0; j < kRJ; ++j) acc[e][j] = fmaf(v[u][e], g[j], acc[e][j]);
         }
     }
 
 #pragma unroll
     for (int e = 0; e < 8; ++e)
 #pragma unroll
-        for (int j = 0; j < kRJ; ++j) acc[e][j] += __shfl_xor_sync(0xffffffffu, acc[e][j], 16);
-    if (half == 0) {
+        for (int j = 0; j < kRJ; ++j) acc[e][j] = warp_rows_sum(acc[e][j]);
+    if (rg == 0) {
 #pragma unroll
         for (int e = 0; e < 8; ++e)
 #pragma unroll
@@ -304,12 +319,7 @@ __global__ void __launch_bounds__(kThreads) k4_x_kernel(
         const int cc = cbeg + i / kRJ, j = i % kRJ;
         const int k = cb * kCols + cc;
         if (k >= K || j0 + j >= r) continue;
-        float s = 0.f;
-        for (int q = 0; q < CL; ++q) {
-            const float* rp = cluster.map_shared_rank(part, q);
-            s = q == 0 ? rp[cc * kRJ + j] : s + rp[cc * kRJ + j];
-        }
-        dA[static_cast<size_t>(k) * r + j0 + j] = cscale * s;
+        dA[static_cast<size_t>(k) * r + j0 + j] = cscale * cluster_sum(cluster, part, cc * kRJ + j, CL);
     }
     cluster.sync();
 }
@@ -317,34 +327,19 @@ __global__ void __launch_bounds__(kThreads) k4_x_kernel(
 // G[m,j] = sum_b Gp[b][m,j] (only when a caller asks for G itself).
 __global__ void k4_g_reduce_kernel(const float* __restrict__ Gp, int ncb, size_t n,
                                    float* __restrict__ G) {
+    pdl_trigger();
+    pdl_wait();
     for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
-         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-        float s = Gp[i];
-        for (int b = 1; b < ncb; ++b) s += Gp[static_cast<size_t>(b) * n + i];
-        G[i] = s;
-    }
+         i += static_cast<size_t>(gridDim.x) * blockDim.x)
+        G[i] = sum_slices(Gp + i, n, ncb);
 }
 
-int cluster_for(int M) {
+// Cluster size along the rows.  The dY pass runs one CTA per SM (its
+// accumulators fill the register file), so it takes clusters of at most 4:
+// clusters of 8 such CTAs do not all fit in one wave of the GPCs.
+int cluster_for(int M, int max_cl) {
     int cl = (M + 63) / 64;
-    return cl > kMaxCluster ? kMaxCluster : (cl < 1 ? 1 : cl);
-}
-
-template <typename Kern, typename... Args>
-cudaError_t launch_clustered(Kern kern, dim3 grid, int cl, cudaStream_t s, Args... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = cl;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, args...);
+    return cl > max_cl ? max_cl : (cl < 1 ? 1 : cl);
 }
 
 }  // namespace
@@ -358,41 +353,43 @@ size_t rank_workspace_floats(int M, int N, int r) {
 cudaError_t launch_rank_dy(Act act, const void* dY, const float* B, const float* xA, int M, int N,
                            int r, float c, float* Gp, float* dB, float* dbias, float* G,
                            cudaStream_t s) {
-    const int cl = cluster_for(M);
+    const int cl = cluster_for(M, 4);
     const int RM = (M + cl - 1) / cl;
     const dim3 grid(rank_col_blocks(N), cl);
     for (int j0 = 0; j0 < r; j0 += kRJ) {
         cudaError_t e;
         if (act == kBF16)
-            e = launch_clustered(k4_dy_kernel<__nv_bfloat16>, grid, cl, s,
-                                 static_cast<const __nv_bfloat16*>(dY), B, xA, M, N, r, j0, RM, c,
-                                 Gp, dB, dbias);
+            e = launch_k(k4_dy_kernel<__nv_bfloat16>, grid, dim3(kThreads), 0, s, cl,
+                         static_cast<const __nv_bfloat16*>(dY), B, xA, M, N, r, j0, RM, c, Gp, dB,
+                         dbias);
         else
-            e = launch_clustered(k4_dy_kernel<float>, grid, cl, s, static_cast<const float*>(dY), B,
-                                 xA, M, N, r, j0, RM, c, Gp, dB, dbias);
+            e = launch_k(k4_dy_kernel<float>, grid, dim3(kThreads), 0, s, cl,
+                         static_cast<const float*>(dY), B, xA, M, N, r, j0, RM, c, Gp, dB, dbias);
         if (e != cudaSuccess) return e;
     }
     if (G) {
         const size_t n = static_cast<size_t>(M) * r;
         const int blocks = static_cast<int>((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
-        k4_g_reduce_kernel<<<blocks, 256, 0, s>>>(Gp, rank_col_blocks(N), n, G);
+        cudaError_t e = launch_k(k4_g_reduce_kernel, dim3(blocks), dim3(256), 0, s, 1,
+                                 static_cast<const float*>(Gp), rank_col_blocks(N), n, G);
+        if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
 }
 
 cudaError_t launch_rank_x(Act act, const void* X, const float* Gp, int ncb, int M, int K, int r,
                           float c, float* dA, cudaStream_t s) {
-    const int cl = cluster_for(M);
+    const int cl = cluster_for(M, kMaxCluster);
     const int RM = (M + cl - 1) / cl;
     const dim3 grid(rank_col_blocks(K), cl);
     for (int j0 = 0; j0 < r; j0 += kRJ) {
         cudaError_t e;
         if (act == kBF16)
-            e = launch_clustered(k4_x_kernel<__nv_bfloat16>, grid, cl, s,
-                                 static_cast<const __nv_bfloat16*>(X), Gp, ncb, M, K, r, j0, RM, c, dA);
+            e = launch_k(k4_x_kernel<__nv_bfloat16>, grid, dim3(kThreads), 0, s, cl,
+                         static_cast<const __nv_bfloat16*>(X), Gp, ncb, M, K, r, j0, RM, c, dA);
         else
-            e = launch_clustered(k4_x_kernel<float>, grid, cl, s, static_cast<const float*>(X), Gp,
-                                 ncb, M, K, r, j0, RM, c, dA);
+            e = launch_k(k4_x_kernel<float>, grid, dim3(kThreads), 0, s, cl,
+                         static_cast<const float*>(X), Gp, ncb, M, K, r, j0, RM, c, dA);
         if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();

@@ -26,6 +26,17 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
     return t;
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while its predecessor on the stream still runs.
+// pdl_wait() blocks until every predecessor grid has completed and its
+// memory is visible (a no-op for ordinary launches); every kernel here calls
+// it before its first global-memory read or write.  pdl_trigger() lets the
+// successor start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ bool elect_one() {
     uint32_t pred = 0;
     asm volatile(
@@ -273,6 +284,26 @@ struct ActIO<__nv_bfloat16> {
     static __device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
     static __device__ __forceinline__ __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
 };
+
+// sum_{b < n} p[b * stride] in ascending b, with eight loads in flight.
+__device__ __forceinline__ float sum_slices(const float* __restrict__ p, size_t stride, int n) {
+    float s = 0.f;
+    int b = 0;
+    for (; b + 8 <= n; b += 8) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = __ldg(p + (b + u) * stride);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) s = (b + u == 0) ? v[u] : s + v[u];
+    }
+    float t[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) t[u] = (b + u < n) ? __ldg(p + (b + u) * stride) : 0.f;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+        if (b + u < n) s = (b + u == 0) ? t[u] : s + t[u];
+    return s;
+}
 
 // Symmetric abs-max int8 code: clamp(rne(v * inv), -127, 127), fp32 product
 // rounded once.

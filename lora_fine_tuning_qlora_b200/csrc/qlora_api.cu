@@ -136,6 +136,11 @@ int tile_override(const char* name) {
     return val;
 }
 
+bool pdl_enabled() {
+    static const bool on = tile_override("QLORA_PDL") != 0;
+    return on;
+}
+
 int sm_count() {
     static int cache[64] = {0};
     int dev = 0;

@@ -16,6 +16,8 @@ __device__ __forceinline__ bool positive(T v) {
 
 template <typename T>
 __global__ void relu_kernel(T* __restrict__ y, size_t n, bool vec) {
+    pdl_trigger();
+    pdl_wait();
     constexpr int kV = 16 / sizeof(T);
     const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
     size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
@@ -37,6 +39,8 @@ __global__ void relu_kernel(T* __restrict__ y, size_t n, bool vec) {
 
 template <typename T>
 __global__ void relu_backward_kernel(T* __restrict__ g, const T* __restrict__ h, size_t n, bool vec) {
+    pdl_trigger();
+    pdl_wait();
     constexpr int kV = 16 / sizeof(T);
     const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
     size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
@@ -71,22 +75,19 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 cudaError_t launch_relu(Act act, void* y, size_t n, cudaStream_t s) {
     const bool vec = aligned16(y);
     if (act == kBF16)
-        relu_kernel<__nv_bfloat16><<<grid_for(n / 8 + 1), 256, 0, s>>>(static_cast<__nv_bfloat16*>(y),
-                                                                       n, vec);
-    else
-        relu_kernel<float><<<grid_for(n / 4 + 1), 256, 0, s>>>(static_cast<float*>(y), n, vec);
-    return cudaGetLastError();
+        return launch_k(relu_kernel<__nv_bfloat16>, dim3(grid_for(n / 8 + 1)), dim3(256), 0, s, 1,
+                        static_cast<__nv_bfloat16*>(y), n, vec);
+    return launch_k(relu_kernel<float>, dim3(grid_for(n / 4 + 1)), dim3(256), 0, s, 1,
+                    static_cast<float*>(y), n, vec);
 }
 
 cudaError_t launch_relu_backward(Act act, void* g, const void* h, size_t n, cudaStream_t s) {
     const bool vec = aligned16(g) && aligned16(h);
     if (act == kBF16)
-        relu_backward_kernel<__nv_bfloat16><<<grid_for(n / 8 + 1), 256, 0, s>>>(
-            static_cast<__nv_bfloat16*>(g), static_cast<const __nv_bfloat16*>(h), n, vec);
-    else
-        relu_backward_kernel<float><<<grid_for(n / 4 + 1), 256, 0, s>>>(
-            static_cast<float*>(g), static_cast<const float*>(h), n, vec);
-    return cudaGetLastError();
+        return launch_k(relu_backward_kernel<__nv_bfloat16>, dim3(grid_for(n / 8 + 1)), dim3(256), 0, s,
+                        1, static_cast<__nv_bfloat16*>(g), static_cast<const __nv_bfloat16*>(h), n, vec);
+    return launch_k(relu_backward_kernel<float>, dim3(grid_for(n / 4 + 1)), dim3(256), 0, s, 1,
+                    static_cast<float*>(g), static_cast<const float*>(h), n, vec);
 }
 
 }  // namespace qlora
