@@ -140,6 +140,44 @@ int qlora_backward(const qlora_layer_desc* d, int M, const void* X, const void* 
                    const float* xA, void* dX, float* dA, float* dB, float* dbias,
                    void* workspace, size_t workspace_bytes, void* stream);
 
+/* Size of the static scratch behind qlora_backward_noalloc (8 MiB per device). */
+#define QLORA_NOALLOC_SCRATCH_BYTES (8 * 1024 * 1024)
+
+/*
+ * qlora_backward without a workspace argument (the pages have no counterpart:
+ * it is a calling convention, not part of the method).  Same arguments,
+ * results and error codes as qlora_backward, minus workspace/workspace_bytes.
+ *
+ * Who it is for: callers that must not allocate device memory at the point
+ * of the call and hold no spare buffer to lend, e.g. code that runs inside
+ * an allocator's own callbacks, a host that forbids allocation once its
+ * steady state begins, or a runtime whose memory pool is already committed.
+ * The scratch it needs (the per-column-block G slices of the rank-r backward)
+ * is a file-scope device array of QLORA_NOALLOC_SCRATCH_BYTES reserved when
+ * the library's module is loaded on a device; the call itself allocates no
+ * device memory.  Nothing in the scratch has to start at zero: each call
+ * writes every scratch element it reads before reading it.
+ *
+ * Limit: the layer needs ceil(N/64) * M * r * 4 bytes of scratch (rounded up
+ * to 256); a call that needs more than QLORA_NOALLOC_SCRATCH_BYTES returns
+ * QLORA_ESHAPE with a message stating both sizes, before any launch.  Use
+ * qlora_backward with a workspace for such layers.
+ *
+ * Set-up: the first call on each device (with that device current) looks up
+ * the device addresses of the scratch and of the status word with
+ * cudaGetSymbolAddress and caches them; a failed lookup returns QLORA_ECUDA.
+ * Make the first call on a device before any stream capture begins.
+ *
+ * Concurrency: all calls on one device share the one scratch.  Calls issued
+ * to the same stream are ordered and safe; calls that can overlap on the
+ * device (different streams without ordering between them, or several host
+ * threads) race on the scratch and give undefined results.
+ */
+int qlora_backward_noalloc(const qlora_layer_desc* d, int M, const void* X, const void* dY,
+                           const int8_t* Wq, const float* sw, const float* A, const float* B,
+                           const float* xA, void* dX, float* dA, float* dB, float* dbias,
+                           void* stream);
+
 /* ------------------------------------------------------------------------
  * Step-level entry points.  qlora_forward is qlora_quantize_input followed
  * by qlora_gemm_forward; qlora_backward is qlora_lora_grad_dy, then

@@ -1,6 +1,7 @@
 // qlora_api.cu -- the C ABI of libqlora.so (declared in include/qlora.h):
 // argument validation, workspace layout, tensor-map encoding and the launch
 // sequence of each call.  No device memory is allocated here.
+#include <cstdio>
 #include <cstdlib>
 #include <map>
 #include <mutex>
@@ -167,6 +168,39 @@ cudaError_t ensure_smem_attr(const void* func, int bytes) {
     return e;
 }
 
+}  // namespace qlora
+
+namespace qlora {
+namespace {
+
+// Scratch of qlora_backward_noalloc: the G slices of the rank-r backward live
+// in this file-scope array (one copy per device, reserved when the module is
+// loaded on that device) instead of a caller-supplied workspace.  Every
+// element the three passes read is written by the dY pass of the same call
+// first, so nothing in it has to start at zero.
+__device__ __align__(256) unsigned char g_noalloc_scratch[QLORA_NOALLOC_SCRATCH_BYTES];
+
+uint8_t* g_noalloc_ptr[64] = {nullptr};
+
+// Device address of the scratch on the current device, looked up once per
+// device (with that device current) and cached.
+cudaError_t noalloc_scratch(uint8_t** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_ptr[dev] = static_cast<uint8_t*>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
 }  // namespace qlora
 
 using namespace qlora;
@@ -444,6 +478,64 @@ int qlora_relu_backward(void* dY, const void* Y, size_t n, qlora_dtype dtype, vo
     return cuda_status(launch_relu_backward(dtype == QLORA_BF16 ? kBF16 : kF32, dY, Y, n,
                                             static_cast<cudaStream_t>(stream)),
                        "relu backward launch");
+}
+
+int qlora_backward_noalloc(const qlora_layer_desc* d, int M, const void* X, const void* dY,
+                           const int8_t* Wq, const float* sw, const float* A, const float* B,
+                           const float* xA, void* dX, float* dA, float* dB, float* dbias,
+                           void* stream) {
+    int rc = check_layer(d, M);
+    if (rc != QLORA_OK) return rc;
+    QL_REQUIRE(X && dY && Wq && sw && A && B && xA && dA && dB, QLORA_EINVAL,
+               "NULL pointer argument");
+    QL_REQUIRE(aligned(X, 16) && aligned(dY, 16) && aligned(Wq, 16) && (!dX || aligned(dX, 16)),
+               QLORA_EALIGN, "X, dY, dX, Wq must be 16-byte aligned");
+    QL_REQUIRE(aligned(sw, 4) && aligned(A, 4) && aligned(B, 4) && aligned(xA, 4) &&
+                   aligned(dA, 4) && aligned(dB, 4) && (!dbias || aligned(dbias, 4)),
+               QLORA_EALIGN, "fp32 vectors must be 4-byte aligned");
+    const WsLayout w = layout_for(*d, M);
+    if (w.bwd_total > QLORA_NOALLOC_SCRATCH_BYTES) {
+        char msg[256];
+        snprintf(msg, sizeof msg,
+                 "qlora_backward_noalloc: M=%d, N=%d, r=%d needs %zu bytes of scratch, above the "
+                 "%d-byte static scratch; use qlora_backward with a caller-supplied workspace",
+                 M, d->N, d->r, w.bwd_total, QLORA_NOALLOC_SCRATCH_BYTES);
+        return fail(QLORA_ESHAPE, msg);
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M == 0) {
+        rc = cuda_status(cudaMemsetAsync(dA, 0, sizeof(float) * d->K * d->r, s), "memset dA");
+        if (rc == QLORA_OK)
+            rc = cuda_status(cudaMemsetAsync(dB, 0, sizeof(float) * d->r * d->N, s), "memset dB");
+        if (rc == QLORA_OK && dbias)
+            rc = cuda_status(cudaMemsetAsync(dbias, 0, sizeof(float) * d->N, s), "memset dbias");
+        return rc;
+    }
+    uint8_t* scratch = nullptr;
+    rc = cuda_status(noalloc_scratch(&scratch), "static scratch address");
+    if (rc != QLORA_OK) return rc;
+    int* status = status_ptr();
+    QL_REQUIRE(status, QLORA_ECUDA, "no CUDA device");
+    float* gp = reinterpret_cast<float*>(scratch + w.gp);
+    const float c = lora_scale(d);
+    rc = cuda_status(launch_rank_dy(act_of(d), dY, B, xA, M, d->N, d->r, c, gp, dB, dbias,
+                                    nullptr, s),
+                     "dY pass launch");
+    if (rc != QLORA_OK) return rc;
+    if (dX) {
+        DxEpilogue ep;
+        ep.Gp = gp;
+        ep.ncb = w.ncb;
+        ep.A = A;
+        ep.r = d->r;
+        ep.c = c;
+        ep.dX = dX;
+        rc = cuda_status(launch_gemm_dx(act_of(d), dY, Wq, sw, M, d->N, d->K, ep, status, s),
+                         "dX GEMM launch");
+        if (rc != QLORA_OK) return rc;
+    }
+    return cuda_status(launch_rank_x(act_of(d), X, gp, w.ncb, M, d->K, d->r, c, dA, s),
+                       "X pass launch");
 }
 
 }  // extern "C"

@@ -30,7 +30,7 @@ EXPORTED = ("qlora_quantize_weight", "qlora_workspace_bytes", "qlora_forward",
             "qlora_backward", "qlora_merge", "qlora_last_error", "qlora_device_status",
             "qlora_version", "qlora_relu", "qlora_relu_backward", "qlora_quantize_input",
             "qlora_gemm_forward", "qlora_lora_grad_dy", "qlora_gemm_dx", "qlora_lora_grad_x",
-            "qlora_selftest_wait_timeout")
+            "qlora_selftest_wait_timeout", "qlora_backward_noalloc")
 
 
 class QLoraError(RuntimeError):
@@ -64,6 +64,9 @@ def _load():
     lib.qlora_backward.argtypes = [ctypes.POINTER(LayerDesc), I, P, P, P, P, P, P, P, P, P, P,
                                    P, P, ctypes.c_size_t, P]
     lib.qlora_backward.restype = I
+    lib.qlora_backward_noalloc.argtypes = [ctypes.POINTER(LayerDesc), I, P, P, P, P, P, P, P, P,
+                                           P, P, P, P]
+    lib.qlora_backward_noalloc.restype = I
     lib.qlora_merge.argtypes = [ctypes.POINTER(LayerDesc), P, P, P, P, P, P, P]
     lib.qlora_merge.restype = I
     lib.qlora_last_error.restype = ctypes.c_char_p
@@ -171,6 +174,14 @@ def qlora_backward(d: LayerDesc, M: int, X, dY, Wq, sw, A, B, xA, dX, dA, dB, db
     _check(_lib.qlora_backward(ctypes.byref(d), int(M), _ptr(X), _ptr(dY), _ptr(Wq), _ptr(sw),
                                _ptr(A), _ptr(B), _ptr(xA), _ptr(dX), _ptr(dA), _ptr(dB),
                                _ptr(dbias), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def qlora_backward_noalloc(d: LayerDesc, M: int, X, dY, Wq, sw, A, B, xA, dX, dA, dB, dbias,
+                           stream=None):
+    """qlora_backward with the library's static scratch instead of a workspace."""
+    _check(_lib.qlora_backward_noalloc(ctypes.byref(d), int(M), _ptr(X), _ptr(dY), _ptr(Wq),
+                                       _ptr(sw), _ptr(A), _ptr(B), _ptr(xA), _ptr(dX), _ptr(dA),
+                                       _ptr(dB), _ptr(dbias), _stream(stream)))
 
 
 def qlora_merge(d: LayerDesc, Wq, sw, A, B, Wq_out, sw_out, stream=None):
