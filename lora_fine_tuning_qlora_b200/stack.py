@@ -34,10 +34,8 @@ class MLPStack:
         self.dX = torch.empty((batch, layers[0].K), dtype=self.act, device=dev)
         self.dbias = [torch.empty((L.N,), dtype=torch.float32, device=dev) for L in layers]
         Kmax = max(L.K for L in layers)
-        rmax = max(L.r for L in layers)
         self.Xq = torch.empty((batch, Kmax), dtype=torch.int8, device=dev)
         self.sx = torch.empty((batch,), dtype=torch.float32, device=dev)
-        self.Gr = torch.empty((batch, rmax), dtype=torch.float32, device=dev)
         # the LoRA gradients live in one flat buffer (one all-reduce in data
         # parallel runs); dA[i], dB[i] are views into it
         sizes = [L.K * L.r + L.r * L.N for L in layers]
@@ -82,8 +80,8 @@ class MLPStack:
 
     def _run(self, stream=None, events=None):
         """One step.  ``events`` optionally maps a step name ("gemm_forward"
-        or "gemm_dx") to a list of (start, end) CUDA events per layer that
-        are recorded around that step's launch."""
+        or "gemm_dx") to a per-layer list of (start, end) CUDA events, or
+        None for a layer that is not timed, recorded around that launch."""
         L_ = self.layers
         n = len(L_)
         D = self.descs
@@ -93,11 +91,11 @@ class MLPStack:
         h = self.X
         for i, L in enumerate(L_):
             qlora.qlora_quantize_input(D[i], M, h, L.A, self.Xq, self.sx, self.xA[i], stream)
-            if ev_f:
+            if ev_f and ev_f[i]:
                 ev_f[i][0].record()
             qlora.qlora_gemm_forward(D[i], M, self.Xq, self.sx, L.Wq, L.sw, L.bias, self.xA[i],
                                      L.B, self.H[i], None, stream)
-            if ev_f:
+            if ev_f and ev_f[i]:
                 ev_f[i][1].record()
             if i < n - 1:
                 qlora.qlora_relu(self.H[i], stream)
@@ -111,19 +109,23 @@ class MLPStack:
             dX = self.dX if i == 0 else self.G[i - 1]
             qlora.qlora_lora_grad_dy(D[i], M, g, L.B, self.xA[i], self.dB[i], self.dbias[i],
                                      self.ws, None, stream)
-            if ev_d:
+            if ev_d and ev_d[i]:
                 ev_d[i][0].record()
             qlora.qlora_gemm_dx(D[i], M, g, L.Wq, L.sw, L.A, dX, self.ws, stream)
-            if ev_d:
+            if ev_d and ev_d[i]:
                 ev_d[i][1].record()
             qlora.qlora_lora_grad_x(D[i], M, x_in, self.dA[i], self.ws, stream)
             g = dX
 
-    def make_events(self, kinds=("gemm_dx",)):
-        """Timing events (graph-capturable) around the given steps, per layer."""
+    def make_events(self, kinds=("gemm_dx",), layers=None):
+        """Timing events (graph-capturable) around the given steps of the
+        given layers (all layers when None).  An event pair between two
+        kernels orders them, so each timed launch loses its overlap with its
+        neighbours; time a few layers to keep the step itself unperturbed."""
+        sel = set(range(len(self.layers)) if layers is None else layers)
         return {k: [(torch.cuda.Event(enable_timing=True, external=True),
-                     torch.cuda.Event(enable_timing=True, external=True))
-                    for _ in self.layers] for k in kinds}
+                     torch.cuda.Event(enable_timing=True, external=True)) if i in sel else None
+                    for i in range(len(self.layers))] for k in kinds}
 
     def capture(self, warmup: int = 1, events=None):
         """Records one step into a CUDA graph (after `warmup` eager steps)."""
