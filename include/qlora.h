@@ -158,10 +158,12 @@ int qlora_backward(const qlora_layer_desc* d, int M, const void* X, const void* 
  * device memory.  Nothing in the scratch has to start at zero: each call
  * writes every scratch element it reads before reading it.
  *
- * Limit: the layer needs ceil(N/64) * M * r * 4 bytes of scratch (rounded up
- * to 256); a call that needs more than QLORA_NOALLOC_SCRATCH_BYTES returns
- * QLORA_ESHAPE with a message stating both sizes, before any launch.  Use
- * qlora_backward with a workspace for such layers.
+ * Limit: the layer needs S * M * r * 4 bytes of scratch for its S slices of
+ * G (S = ceil(N/128) for bf16 layers with N a multiple of 8, else
+ * ceil(N/64)), plus M * r * 4 bytes for G itself when S > 8, each part
+ * rounded up to 256.  A call that needs more than QLORA_NOALLOC_SCRATCH_BYTES
+ * returns QLORA_ESHAPE with a message stating both sizes, before any launch.
+ * Use qlora_backward with a workspace for such layers.
  *
  * Set-up: the first call on each device (with that device current) looks up
  * the device addresses of the scratch and of the status word with

@@ -49,19 +49,33 @@ cudaError_t launch_gemm_dx(Act act, const void* dY, const int8_t* Wq, const floa
                            int N, int K, const DxEpilogue& ep, int* status, cudaStream_t s);
 
 // ---------------------------------------------------------------- K4
-// Column blocks of the passes (= number of G slices for N columns).
-int rank_col_blocks(int N);
-// fp32 workspace of the G slices: rank_col_blocks(N) * M * r.
-size_t rank_workspace_floats(int M, int N, int r);
+// The dY pass runs on the tensor cores for bf16 activations whose rows TMA
+// can describe (N a multiple of 8), in 128-column blocks; otherwise on CUDA
+// cores in 64-column blocks.  The X pass likewise (K is always a multiple of 16).
+bool rank_dy_tc(Act act, int N);
+// Column blocks of the dY pass = number of G slices it writes.
+int rank_col_blocks(Act act, int N);
+// Consumers add up to this many G slices themselves; above it the slices are
+// added once into G (launch_g_reduce) and the consumers read G.
+constexpr int kMaxDirectSlices = 8;
 
-// Pass over dY: G slices into Gp, final dB and dbias (dbias may be null),
-// and, when G is not null, the summed G [M,r] as well.
+// Pass over dY: G slices into Gp, final dB and dbias (dbias may be null).
 cudaError_t launch_rank_dy(Act act, const void* dY, const float* B, const float* xA, int M, int N,
-                           int r, float c, float* Gp, float* dB, float* dbias, float* G,
+                           int r, float c, float* Gp, float* dB, float* dbias, int* status,
                            cudaStream_t s);
-// Pass over X: final dA from X and the ncb G slices.
-cudaError_t launch_rank_x(Act act, const void* X, const float* Gp, int ncb, int M, int K, int r,
-                          float c, float* dA, cudaStream_t s);
+// G [M,r] = the ncb slices of Gp added in ascending order.
+cudaError_t launch_g_reduce(const float* Gp, int ncb, int M, int r, float* G, cudaStream_t s);
+// Pass over X: final dA from X and G given as nsl slices (nsl = 1: G itself).
+cudaError_t launch_rank_x(Act act, const void* X, const float* G, int nsl, int M, int K, int r,
+                          float c, float* dA, int* status, cudaStream_t s);
+
+// tensor-core passes (k4_rank_tc.cu)
+int rank_tc_col_blocks(int C);
+cudaError_t launch_rank_dy_tc(const void* dY, const float* B, const float* xA, int M, int N, int r,
+                              float c, float* Gp, float* dB, float* dbias, int* status,
+                              cudaStream_t s);
+cudaError_t launch_rank_x_tc(const void* X, const float* G, int nsl, int M, int K, int r, float c,
+                             float* dA, int* status, cudaStream_t s);
 
 // ---------------------------------------------------------------- KM
 cudaError_t launch_merge(const int8_t* Wq, const float* sw, const float* A, const float* B, int K,

@@ -8,9 +8,11 @@
 // ("How to fine-tune the 4-bit model?" thread: the LoRA factors are the
 // trainable fp32 weights and the backward needs the A @ B.T-style adapter
 // products; "Parameter-efficient fine-tuning of GPT-2 with LoRA", "LoRA
-// equation", for the shapes.)  These are far too thin for tensor cores: each
-// pass streams its matrix once from HBM with 128-bit loads and does 2r FMAs
-// per element on CUDA cores.
+// equation", for the shapes.)  This file holds the CUDA-core passes, used
+// for fp32 activations (where the sums must stay fp32 throughout) and for dY
+// rows that TMA cannot describe; bf16 layers run the tensor-core passes of
+// k4_rank_tc.cu.  Each pass here streams its matrix once from HBM with
+// 128-bit loads and does 2r FMAs per element.
 //
 // Layout of the work: a CTA owns 64 columns (8 lanes x 8, so a warp covers
 // four rows per load) and a chunk of rows; the CL <= 8 CTAs that own the
@@ -20,7 +22,8 @@
 // rank, so dB, dbias and dA leave the kernel final, with a fixed summation
 // order (deterministic) and no second launch.  G's per-row sums over the
 // column blocks stay as partial slices Gp in the workspace; the two
-// consumers (the dX GEMM and the X pass) add the slices up themselves.
+// consumers (the dX GEMM and the X pass) add the slices up themselves, or
+// read G once launch_g_reduce has added many slices.
 #include <cooperative_groups.h>
 
 #include "internal.h"
@@ -344,18 +347,20 @@ int cluster_for(int M, int max_cl) {
 
 }  // namespace
 
-int rank_col_blocks(int N) { return (N + kCols - 1) / kCols; }
+bool rank_dy_tc(Act act, int N) { return act == kBF16 && N % 8 == 0; }
 
-size_t rank_workspace_floats(int M, int N, int r) {
-    return static_cast<size_t>(rank_col_blocks(N)) * M * r;
+int rank_col_blocks(Act act, int N) {
+    return rank_dy_tc(act, N) ? rank_tc_col_blocks(N) : (N + kCols - 1) / kCols;
 }
 
 cudaError_t launch_rank_dy(Act act, const void* dY, const float* B, const float* xA, int M, int N,
-                           int r, float c, float* Gp, float* dB, float* dbias, float* G,
+                           int r, float c, float* Gp, float* dB, float* dbias, int* status,
                            cudaStream_t s) {
+    if (rank_dy_tc(act, N))
+        return launch_rank_dy_tc(dY, B, xA, M, N, r, c, Gp, dB, dbias, status, s);
     const int cl = cluster_for(M, 4);
     const int RM = (M + cl - 1) / cl;
-    const dim3 grid(rank_col_blocks(N), cl);
+    const dim3 grid((N + kCols - 1) / kCols, cl);
     for (int j0 = 0; j0 < r; j0 += kRJ) {
         cudaError_t e;
         if (act == kBF16)
@@ -367,29 +372,30 @@ cudaError_t launch_rank_dy(Act act, const void* dY, const float* B, const float*
                          static_cast<const float*>(dY), B, xA, M, N, r, j0, RM, c, Gp, dB, dbias);
         if (e != cudaSuccess) return e;
     }
-    if (G) {
-        const size_t n = static_cast<size_t>(M) * r;
-        const int blocks = static_cast<int>((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
-        cudaError_t e = launch_k(k4_g_reduce_kernel, dim3(blocks), dim3(256), 0, s, 1,
-                                 static_cast<const float*>(Gp), rank_col_blocks(N), n, G);
-        if (e != cudaSuccess) return e;
-    }
     return cudaGetLastError();
 }
 
-cudaError_t launch_rank_x(Act act, const void* X, const float* Gp, int ncb, int M, int K, int r,
-                          float c, float* dA, cudaStream_t s) {
+cudaError_t launch_g_reduce(const float* Gp, int ncb, int M, int r, float* G, cudaStream_t s) {
+    const size_t n = static_cast<size_t>(M) * r;
+    const int blocks = static_cast<int>((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
+    return launch_k(k4_g_reduce_kernel, dim3(blocks < 1 ? 1 : blocks), dim3(256), 0, s, 1, Gp, ncb,
+                    n, G);
+}
+
+cudaError_t launch_rank_x(Act act, const void* X, const float* G, int nsl, int M, int K, int r,
+                          float c, float* dA, int* status, cudaStream_t s) {
+    if (act == kBF16 && K % 8 == 0) return launch_rank_x_tc(X, G, nsl, M, K, r, c, dA, status, s);
     const int cl = cluster_for(M, kMaxCluster);
     const int RM = (M + cl - 1) / cl;
-    const dim3 grid(rank_col_blocks(K), cl);
+    const dim3 grid((K + kCols - 1) / kCols, cl);
     for (int j0 = 0; j0 < r; j0 += kRJ) {
         cudaError_t e;
         if (act == kBF16)
             e = launch_k(k4_x_kernel<__nv_bfloat16>, grid, dim3(kThreads), 0, s, cl,
-                         static_cast<const __nv_bfloat16*>(X), Gp, ncb, M, K, r, j0, RM, c, dA);
+                         static_cast<const __nv_bfloat16*>(X), G, nsl, M, K, r, j0, RM, c, dA);
         else
             e = launch_k(k4_x_kernel<float>, grid, dim3(kThreads), 0, s, cl,
-                         static_cast<const float*>(X), Gp, ncb, M, K, r, j0, RM, c, dA);
+                         static_cast<const float*>(X), G, nsl, M, K, r, j0, RM, c, dA);
         if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();

@@ -1,0 +1,426 @@
+// k4_rank_tc.cu -- the rank-r passes of the LoRA backward on the tensor cores
+// (bf16 activations):
+//
+//   dY pass:  Gp[b][m,j] = sum_{n in block b} dY[m,n] B[j,n]      (G slices)
+//             dB[j,n]    = c * sum_m xA[m,j] dY[m,n]
+//             dbias[n]   = sum_m dY[m,n]
+//   X pass:   dA[k,j]    = c * sum_m X[m,k] G[m,j]               (G = sum_b Gp[b])
+//
+// ("How to fine-tune the 4-bit model?" thread: the adapter's A B^T-style
+// products drive the gradient; "Parameter-efficient fine-tuning of GPT-2
+// with LoRA", "LoRA equation", for the shapes.)
+//
+// A CTA owns 128 columns of the activation T (dY or X) and a run of 128-row
+// tiles.  Each tile arrives by TMA as two [128 rows x 64 columns] boxes with
+// the 128-byte swizzle, and the one copy in shared memory is read two ways
+// by tcgen05.mma.kind::f16 (bf16 in, fp32 accumulate in TMEM):
+//   * K-major (rows = M dimension, columns = contraction): T . Bcat^T gives
+//     the tile's G rows (dY pass only);
+//   * MN-major (columns = M dimension, rows = contraction): T^T . Vcat sums
+//     over the tile's rows into a [128 columns x NV] accumulator that stays
+//     in TMEM across all the CTA's tiles: dB^T and dbias (dY pass), dA (X pass).
+// The fp32 factors enter as bf16 head + remainder pairs (v = hi + lo to
+// 16 significant bits; every bf16 x bf16 product is exact in fp32), so the
+// sums carry fp32-level accuracy.  Vcat holds [xA_hi | xA_lo | 1] (dY pass;
+// the ones column yields dbias) or [G_hi | G_lo] (X pass); Bcat holds
+// [B_hi | B_lo].  The head and remainder halves sit RP = roundup(r, 16)
+// columns apart in TMEM, so one 16-column load of each gives 16 sums.
+//
+// The CL <= 8 CTAs that share a column block form a cluster along the rows
+// and add their [128 x r] partials through distributed shared memory in rank
+// order: dB, dbias and dA leave the kernel final and deterministic.
+//
+// Warps: 0 TMA producer, 1 TMEM owner + MMA issuer, 2..5 operand tables and
+// epilogues (warp w owns TMEM lane quarter w % 4).
+#include <cooperative_groups.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace qlora {
+
+namespace {
+
+constexpr int kTileRows = 128;
+constexpr int kTileCols = 128;
+constexpr int kBoxCols = 64;                         // one 128-byte swizzle row of bf16
+constexpr uint32_t kBoxBytes = kTileRows * kBoxCols * 2;
+constexpr uint32_t kTileBytes = 2 * kBoxBytes;
+constexpr int kWorkers = 4;
+constexpr int kThreads = 64 + 32 * kWorkers;
+constexpr int kMaxCluster = 8;
+constexpr uint32_t kTabSbo = (kTileCols / 8) * 128;  // 8-row group stride of a 128-wide table
+
+struct RankTcArgs {
+    const float* V;      // dY pass: xA [M, r]; X pass: G slices (nsl of them) or G
+    int nsl;             // X pass: slices to add (1 = G itself)
+    const float* B;      // dY pass: B [r, C]
+    float* Gp;           // dY pass: G slices [ceil(C/128)][M, r]
+    float* out;          // dY pass: dB [r, C]; X pass: dA [C, r]
+    float* dbias;        // dY pass: [C] or nullptr
+    int M, C, r;
+    int tiles_per_cta;   // 128-row tiles per CTA
+    float c;
+};
+
+// Shared-memory and TMEM layout for rank r (same on host and device).
+struct RtLayout {
+    int RP, NG, NV, JP;
+    uint32_t vtab, bcat, part, bar, total;
+    uint32_t tmem_cols, d_col, g_col;
+    __host__ __device__ RtLayout(bool dy, int r) {
+        RP = (r + 15) / 16 * 16;
+        NG = dy ? 2 * RP : 0;
+        NV = dy ? 2 * RP + 16 : 2 * RP;
+        JP = dy ? r + 1 : r;
+        vtab = 2 * kTileBytes;
+        bcat = vtab + 2 * static_cast<uint32_t>(NV) * 256;
+        part = bcat + static_cast<uint32_t>(NG) * 256;
+        bar = part + ((kTileCols * JP * 4 + 15) / 16) * 16;
+        total = bar + 128;
+        d_col = 0;
+        g_col = static_cast<uint32_t>(NV);
+        const uint32_t need = static_cast<uint32_t>(NV + 2 * NG);
+        tmem_cols = 32;
+        while (tmem_cols < need) tmem_cols <<= 1;
+    }
+};
+
+// Byte offset of element (row, k) of a K-major bf16 operand table that is 128
+// elements long in K, no swizzle: 8-row x 16-byte core matrices, K-adjacent
+// ones 128 B apart (leading byte offset), 8-row groups 2048 B apart (stride
+// byte offset).
+__device__ __forceinline__ uint32_t ktab_off(int row, int k) {
+    return static_cast<uint32_t>((row >> 3) * kTabSbo + (k >> 3) * 128 + (row & 7) * 16 +
+                                 (k & 7) * 2);
+}
+
+__device__ __forceinline__ void put_split(uint8_t* tab, int row_hi, int row_lo, int k, float v) {
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+    *reinterpret_cast<__nv_bfloat16*>(tab + ktab_off(row_hi, k)) = hi;
+    *reinterpret_cast<__nv_bfloat16*>(tab + ktab_off(row_lo, k)) = lo;
+}
+
+template <bool kDy>
+__global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_constant__ CUtensorMap tmT,
+                                                              RankTcArgs a, int* status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const RtLayout L(kDy, a.r);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar);
+    uint64_t* full = bars;        // [2] tile landed
+    uint64_t* vready = bars + 2;  // [2] Vcat table written
+    uint64_t* empty = bars + 4;   // [2] tile and table consumed by the MMAs
+    uint64_t* gfull = bars + 6;   // [2] G accumulator ready
+    uint64_t* gempty = bars + 8;  // [2] G accumulator read out
+    uint64_t* dfull = bars + 10;  // column accumulator final
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+    float* part = reinterpret_cast<float*>(smem + L.part);
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const int CL = static_cast<int>(cluster.num_blocks());
+    const int crank = static_cast<int>(cluster.block_rank());
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int cb = blockIdx.x;
+    const int col0 = cb * kTileCols;
+    const int mtiles = (a.M + kTileRows - 1) / kTileRows;
+    const int t0 = blockIdx.y * a.tiles_per_cta;
+    const int t1 = min(mtiles, t0 + a.tiles_per_cta);
+    const int nt = t1 > t0 ? t1 - t0 : 0;
+    pdl_trigger();
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&vready[s], kWorkers);
+            mbar_init(&empty[s], 1);
+            mbar_init(&gfull[s], 1);
+            mbar_init(&gempty[s], kWorkers);
+        }
+        mbar_init(dfull, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, L.tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    pdl_wait();  // nothing above read global memory
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmT);
+            for (int i = 0; i < nt; ++i) {
+                const int s = i & 1;
+                if (i >= 2 && !mbar_wait(&empty[s], ((i >> 1) - 1) & 1, status)) break;
+                uint8_t* dst = smem + s * kTileBytes;
+                const int m0 = (t0 + i) * kTileRows;
+                mbar_arrive_expect_tx(&full[s], kTileBytes);
+                tma_load_2d(dst, &tmT, &full[s], col0, m0);
+                tma_load_2d(dst + kBoxBytes, &tmT, &full[s], col0 + kBoxCols, m0);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t tiles = smem_u32(smem);
+            const uint32_t vt = smem_u32(smem + L.vtab);
+            const uint32_t bt = smem_u32(smem + L.bcat);
+            const uint32_t id_g = idesc_bf16(128, L.NG, false, false);
+            const uint32_t id_d = idesc_bf16(128, L.NV, true, false);
+            bool ok = true;
+            for (int i = 0; i < nt; ++i) {
+                const int s = i & 1;
+                if (!mbar_wait(&full[s], (i >> 1) & 1, status) ||
+                    !mbar_wait(&vready[s], (i >> 1) & 1, status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t tb = tiles + s * kTileBytes;
+                if constexpr (kDy) {
+                    // G rows of this tile: T (K-major) x Bcat
+                    if (i >= 2 && !mbar_wait(&gempty[s], ((i >> 1) - 1) & 1, status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kTileCols / 16; ++kk) {
+                        const uint64_t ad = smem_desc(tb + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16,
+                                                      1024, kLayoutSw128);
+                        const uint64_t bd = smem_desc(bt + kk * 256, 128, kTabSbo, kLayoutNone);
+                        mma_bf16(tmem + L.g_col + s * L.NG, ad, bd, id_g, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&gfull[s]);
+                }
+                // column sums: T^T (MN-major, the two boxes 64 columns apart) x Vcat
+#pragma unroll
+                for (int kk = 0; kk < kTileRows / 16; ++kk) {
+                    const uint64_t ad = smem_desc(tb + kk * 2048, kBoxBytes, 1024, kLayoutSw128);
+                    const uint64_t bd =
+                        smem_desc(vt + s * L.NV * 256 + kk * 256, 128, kTabSbo, kLayoutNone);
+                    mma_bf16(tmem + L.d_col, ad, bd, id_d, (i > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(&empty[s]);
+            }
+            if (ok) mma_commit(dfull);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------ tables, epilogues
+        const int wq = warp & 3;
+        const int rr = wq * 32 + lane;  // tile row for the tables; column for the readback
+        const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+        bool ok = true;
+        if constexpr (kDy) {
+            // Bcat[j][n] = B[j, col0 + n] as head (rows 0..RP) and remainder (RP..2RP)
+            uint8_t* bt = smem + L.bcat;
+            const int n = col0 + rr;
+            for (int j = 0; j < L.RP; ++j) {
+                const float v = (j < a.r && n < a.C) ? __ldg(a.B + static_cast<size_t>(j) * a.C + n) : 0.f;
+                put_split(bt, j, L.RP + j, rr, v);
+            }
+        }
+        auto g_epilogue = [&](int i) {
+            const int b = i & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(&gfull[b], (i >> 1) & 1, status));
+            if (!ok) return;
+            tc_fence_after();
+            const int m = (t0 + i) * kTileRows + rr;
+            const uint32_t base = tmem + lane_base + L.g_col + b * L.NG;
+            float* g = a.Gp + (static_cast<size_t>(cb) * a.M + m) * a.r;
+            for (int c0 = 0; c0 < L.RP; c0 += 16) {
+                uint32_t hi[16], lo[16];
+                tmem_ld16(base + c0, hi);
+                tmem_ld16(base + L.RP + c0, lo);
+                tmem_ld_wait();
+                if (m < a.M) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        if (c0 + e < a.r) g[c0 + e] = __uint_as_float(hi[e]) + __uint_as_float(lo[e]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&gempty[b]);
+        };
+        for (int i = 0; i < nt && ok; ++i) {
+            const int s = i & 1;
+            const int m = (t0 + i) * kTileRows + rr;
+            ok = __all_sync(0xffffffffu,
+                            i < 2 || mbar_wait(&empty[s], ((i >> 1) - 1) & 1, status));
+            if (!ok) break;
+            uint8_t* vt = smem + L.vtab + s * L.NV * 256;
+            const bool mok = m < a.M;
+            for (int j0 = 0; j0 < L.RP; j0 += 8) {
+                float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                if (mok && j0 < a.r) {
+                    const int nv = min(8, a.r - j0);
+                    const float* p = a.V + static_cast<size_t>(m) * a.r + j0;
+                    if constexpr (kDy) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            if (e < nv) v[e] = __ldg(p + e);
+                    } else {
+                        // G = the slices added in ascending order
+                        const size_t stride = static_cast<size_t>(a.M) * a.r;
+#pragma unroll 4
+                        for (int b = 0; b < a.nsl; ++b, p += stride)
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                if (e < nv) v[e] += __ldg(p + e);
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) put_split(vt, j0 + e, L.RP + j0 + e, rr, v[e]);
+            }
+            if constexpr (kDy) {
+                const __nv_bfloat16 one = __float2bfloat16_rn(mok ? 1.f : 0.f);
+                const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
+                *reinterpret_cast<__nv_bfloat16*>(vt + ktab_off(2 * L.RP, rr)) = one;
+                for (int j = 2 * L.RP + 1; j < L.NV; ++j)
+                    *reinterpret_cast<__nv_bfloat16*>(vt + ktab_off(j, rr)) = zero;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&vready[s]);
+            if constexpr (kDy) {
+                if (i >= 1) g_epilogue(i - 1);
+            }
+        }
+        if constexpr (kDy) {
+            if (ok && nt >= 1) g_epilogue(nt - 1);
+        }
+        // this CTA's column partials: part[col][j] (and the dbias column)
+        float* pc = part + rr * L.JP;
+        if (ok && nt > 0) ok = __all_sync(0xffffffffu, mbar_wait(dfull, 0, status));
+        if (ok && nt > 0) {
+            tc_fence_after();
+            const uint32_t base = tmem + lane_base + L.d_col;
+            for (int c0 = 0; c0 < L.RP; c0 += 16) {
+                uint32_t hi[16], lo[16];
+                tmem_ld16(base + c0, hi);
+                tmem_ld16(base + L.RP + c0, lo);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    if (c0 + e < a.r) pc[c0 + e] = __uint_as_float(hi[e]) + __uint_as_float(lo[e]);
+            }
+            if constexpr (kDy) {
+                uint32_t ones[16];
+                tmem_ld16(base + 2 * L.RP, ones);
+                tmem_ld_wait();
+                pc[a.r] = __uint_as_float(ones[0]);
+            }
+        } else {
+            for (int j = 0; j < L.JP; ++j) pc[j] = 0.f;
+        }
+        __syncwarp();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, L.tmem_cols);
+    }
+
+    // cluster sum of the partials, rank by rank; rank q finalises its slice
+    cluster.sync();
+    const int per = (kTileCols + CL - 1) / CL;
+    const int cbeg = crank * per;
+    const int cend = min(kTileCols, cbeg + per);
+    const int width = cend - cbeg;
+    if (width > 0) {
+        for (int idx = threadIdx.x; idx < L.JP * width; idx += kThreads) {
+            int j, cc;
+            if constexpr (kDy) {  // dB is [r, C]: consecutive threads take consecutive columns
+                j = idx / width;
+                cc = cbeg + idx % width;
+            } else {              // dA is [C, r]: consecutive threads take consecutive ranks
+                cc = cbeg + idx / L.JP;
+                j = idx % L.JP;
+            }
+            const int col = col0 + cc;
+            if (col >= a.C) continue;
+            if (kDy && j == a.r && a.dbias == nullptr) continue;
+            float sum = 0.f;
+            for (int q = 0; q < CL; ++q) sum += cluster.map_shared_rank(part, q)[cc * L.JP + j];
+            if constexpr (kDy) {
+                if (j < a.r) a.out[static_cast<size_t>(j) * a.C + col] = a.c * sum;
+                else a.dbias[col] = sum;
+            } else {
+                a.out[static_cast<size_t>(col) * a.r + j] = a.c * sum;
+            }
+        }
+    }
+    cluster.sync();
+}
+
+template <bool kDy>
+cudaError_t launch_tc(const void* T, RankTcArgs a, int* status, cudaStream_t s) {
+    CUtensorMap tm;
+    if (!make_tmap_2d(&tm, T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.C,
+                      static_cast<uint64_t>(a.C) * 2, kTileRows, kBoxCols,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    const RtLayout L(kDy, a.r);
+    const size_t smem = L.total + 1024;
+    auto kern = k4_rank_tc_kernel<kDy>;
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    // rows split over a cluster of CL CTAs, every CTA at least one tile;
+    // CTAs too large for two per SM take clusters of at most 4 (clusters of
+    // 8 single-CTA SMs do not all fit one wave of the GPCs)
+    const int max_cl = smem > 110 * 1024 ? 4 : kMaxCluster;
+    const int mtiles = (a.M + kTileRows - 1) / kTileRows;
+    a.tiles_per_cta = (mtiles + max_cl - 1) / max_cl;
+    const int cl = (mtiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
+    const dim3 grid((a.C + kTileCols - 1) / kTileCols, cl);
+    return launch_k(kern, grid, dim3(kThreads), smem, s, cl, tm, a, status);
+}
+
+}  // namespace
+
+int rank_tc_col_blocks(int C) { return (C + kTileCols - 1) / kTileCols; }
+
+cudaError_t launch_rank_dy_tc(const void* dY, const float* B, const float* xA, int M, int N, int r,
+                              float c, float* Gp, float* dB, float* dbias, int* status,
+                              cudaStream_t s) {
+    RankTcArgs a{};
+    a.V = xA;
+    a.nsl = 1;
+    a.B = B;
+    a.Gp = Gp;
+    a.out = dB;
+    a.dbias = dbias;
+    a.M = M;
+    a.C = N;
+    a.r = r;
+    a.c = c;
+    return launch_tc<true>(dY, a, status, s);
+}
+
+cudaError_t launch_rank_x_tc(const void* X, const float* G, int nsl, int M, int K, int r, float c,
+                             float* dA, int* status, cudaStream_t s) {
+    RankTcArgs a{};
+    a.V = G;
+    a.nsl = nsl;
+    a.out = dA;
+    a.M = M;
+    a.C = K;
+    a.r = r;
+    a.c = c;
+    return launch_tc<false>(X, a, status, s);
+}
+
+}  // namespace qlora

@@ -67,24 +67,36 @@ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 
 // Forward: Xq [M,K] int8 and sx [M] fp32.  Backward: the G slices
 // Gp [ncb][M,r] fp32 (written by the dY pass, read by the dX GEMM and the X
-// pass).  The two uses do not overlap in time.
+// pass) and, when there are more than kMaxDirectSlices slices, their sum
+// G [M,r].  The two uses do not overlap in time.
 struct WsLayout {
     size_t xq, sx, fwd_total;
-    size_t gp, bwd_total;
+    size_t gp, g, bwd_total;
     int ncb;
+    bool reduce;  // consumers read G (added once) instead of the slices
     size_t total;
 };
 
 WsLayout layout_for(const qlora_layer_desc& d, int M) {
     WsLayout w{};
+    const Act act = d.act_dtype == QLORA_BF16 ? kBF16 : kF32;
     w.xq = 0;
     w.sx = align256(static_cast<size_t>(M) * d.K);
     w.fwd_total = w.sx + align256(static_cast<size_t>(M) * 4);
+    w.ncb = rank_col_blocks(act, d.N);
+    w.reduce = w.ncb > kMaxDirectSlices;
     w.gp = 0;
-    w.ncb = rank_col_blocks(d.N);
-    w.bwd_total = align256(rank_workspace_floats(M, d.N, d.r) * 4);
+    w.g = align256(static_cast<size_t>(w.ncb) * M * d.r * 4);
+    w.bwd_total = w.g + (w.reduce ? align256(static_cast<size_t>(M) * d.r * 4) : 0);
     w.total = w.fwd_total > w.bwd_total ? w.fwd_total : w.bwd_total;
     return w;
+}
+
+// Where the consumers read G: the slices themselves, or G once added up.
+const float* g_source(const WsLayout& w, const void* ws, int* nsl) {
+    const uint8_t* b = static_cast<const uint8_t*>(ws);
+    *nsl = w.reduce ? 1 : w.ncb;
+    return reinterpret_cast<const float*>(b + (w.reduce ? w.g : w.gp));
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -156,15 +168,18 @@ int sm_count() {
 }
 
 cudaError_t ensure_smem_attr(const void* func, int bytes) {
+    // largest dynamic shared memory size set so far, per (device, kernel):
+    // some kernels size their shared memory by the rank at run time
     static std::mutex mu;
-    static std::set<std::pair<int, const void*>> done;
+    static std::map<std::pair<int, const void*>, int> done;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lk(mu);
-    if (done.count({dev, func})) return cudaSuccess;
+    auto it = done.find({dev, func});
+    if (it != done.end() && it->second >= bytes) return cudaSuccess;
     e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess) done.insert({dev, func});
+    if (e == cudaSuccess) done[{dev, func}] = bytes;
     return e;
 }
 
@@ -324,10 +339,20 @@ int qlora_lora_grad_dy(const qlora_layer_desc* d, int M, const void* dY, const f
     }
     const WsLayout w = layout_for(*d, M);
     QL_REQUIRE(workspace_bytes >= w.total, QLORA_EINVAL, "workspace too small");
+    int* status = status_ptr();
+    QL_REQUIRE(status, QLORA_ECUDA, "no CUDA device");
     float* gp = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.gp);
-    return cuda_status(launch_rank_dy(act_of(d), dY, B, xA, M, d->N, d->r, lora_scale(d), gp, dB,
-                                      dbias, G, s),
-                       "dY pass launch");
+    rc = cuda_status(launch_rank_dy(act_of(d), dY, B, xA, M, d->N, d->r, lora_scale(d), gp, dB,
+                                    dbias, status, s),
+                     "dY pass launch");
+    if (rc == QLORA_OK && w.reduce)
+        rc = cuda_status(launch_g_reduce(gp, w.ncb, M, d->r,
+                                         reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.g),
+                                         s),
+                         "G reduction launch");
+    if (rc == QLORA_OK && G)
+        rc = cuda_status(launch_g_reduce(gp, w.ncb, M, d->r, G, s), "G reduction launch");
+    return rc;
 }
 
 int qlora_gemm_dx(const qlora_layer_desc* d, int M, const void* dY, const int8_t* Wq,
@@ -345,8 +370,7 @@ int qlora_gemm_dx(const qlora_layer_desc* d, int M, const void* dY, const int8_t
     int* status = status_ptr();
     QL_REQUIRE(status, QLORA_ECUDA, "no CUDA device");
     DxEpilogue ep;
-    ep.Gp = reinterpret_cast<const float*>(static_cast<const uint8_t*>(workspace) + w.gp);
-    ep.ncb = w.ncb;
+    ep.Gp = g_source(w, workspace, &ep.ncb);
     ep.A = A;
     ep.r = d->r;
     ep.c = lora_scale(d);
@@ -368,8 +392,12 @@ int qlora_lora_grad_x(const qlora_layer_desc* d, int M, const void* X, float* dA
     if (M == 0) return cuda_status(cudaMemsetAsync(dA, 0, sizeof(float) * d->K * d->r, s), "memset dA");
     const WsLayout w = layout_for(*d, M);
     QL_REQUIRE(workspace_bytes >= w.total, QLORA_EINVAL, "workspace too small");
-    const float* gp = reinterpret_cast<const float*>(static_cast<const uint8_t*>(workspace) + w.gp);
-    return cuda_status(launch_rank_x(act_of(d), X, gp, w.ncb, M, d->K, d->r, lora_scale(d), dA, s),
+    int* status = status_ptr();
+    QL_REQUIRE(status, QLORA_ECUDA, "no CUDA device");
+    int nsl = 0;
+    const float* g = g_source(w, workspace, &nsl);
+    return cuda_status(launch_rank_x(act_of(d), X, g, nsl, M, d->K, d->r, lora_scale(d), dA, status,
+                                     s),
                        "X pass launch");
 }
 
@@ -518,14 +546,20 @@ int qlora_backward_noalloc(const qlora_layer_desc* d, int M, const void* X, cons
     QL_REQUIRE(status, QLORA_ECUDA, "no CUDA device");
     float* gp = reinterpret_cast<float*>(scratch + w.gp);
     const float c = lora_scale(d);
-    rc = cuda_status(launch_rank_dy(act_of(d), dY, B, xA, M, d->N, d->r, c, gp, dB, dbias,
-                                    nullptr, s),
+    rc = cuda_status(launch_rank_dy(act_of(d), dY, B, xA, M, d->N, d->r, c, gp, dB, dbias, status,
+                                    s),
                      "dY pass launch");
+    if (rc == QLORA_OK && w.reduce)
+        rc = cuda_status(launch_g_reduce(gp, w.ncb, M, d->r, reinterpret_cast<float*>(scratch + w.g),
+                                         s),
+                         "G reduction launch");
     if (rc != QLORA_OK) return rc;
+    int nsl = 0;
+    const float* g = g_source(w, scratch, &nsl);
     if (dX) {
         DxEpilogue ep;
-        ep.Gp = gp;
-        ep.ncb = w.ncb;
+        ep.Gp = g;
+        ep.ncb = nsl;
         ep.A = A;
         ep.r = d->r;
         ep.c = c;
@@ -534,7 +568,7 @@ int qlora_backward_noalloc(const qlora_layer_desc* d, int M, const void* X, cons
                          "dX GEMM launch");
         if (rc != QLORA_OK) return rc;
     }
-    return cuda_status(launch_rank_x(act_of(d), X, gp, w.ncb, M, d->K, d->r, c, dA, s),
+    return cuda_status(launch_rank_x(act_of(d), X, g, nsl, M, d->K, d->r, c, dA, status, s),
                        "X pass launch");
 }
 

@@ -68,13 +68,17 @@ class MLPStack:
     def launches_per_step(self) -> int:
         """Kernels this library launches in one step (for the benchmark)."""
         n = 0
+        bf16 = self.act == torch.bfloat16
         for i, L in enumerate(self.layers):
             n += 2                                   # quantize+xA, int8 GEMM
             n += 1 if i < len(self.layers) - 1 else 0  # ReLU
-            rj = (L.r + 7) // 8
-            n += rj                                  # dY pass(es), cluster-reduced
+            rj = (L.r + 7) // 8                      # CUDA-core passes: 8 ranks per launch
+            dy_tc = bf16 and L.N % 8 == 0            # tensor-core dY pass, 128-column blocks
+            n += 1 if dy_tc else rj                  # dY pass
+            ncb = -(-L.N // 128) if dy_tc else -(-L.N // 64)
+            n += 1 if ncb > 8 else 0                 # G slices added once
             n += 1                                   # dX GEMM
-            n += rj                                  # X pass(es), cluster-reduced
+            n += 1 if bf16 else rj                   # X pass
             n += 1 if i < len(self.layers) - 1 else 0  # ReLU backward
         return n
 
