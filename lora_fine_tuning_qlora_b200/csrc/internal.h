@@ -95,6 +95,13 @@ cudaError_t launch_selftest_wait(int* status, unsigned long long limit_ns, cudaS
 bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem_bytes,
                   uint64_t rows, uint64_t cols, uint64_t pitch_bytes, uint32_t box_rows,
                   uint32_t box_cols, CUtensorMapSwizzle swizzle);
+// A [rows, cols] row-major matrix seen as [rows][cols / blk][blk] (cols a
+// multiple of blk), 128-byte swizzle: one box of box_blocks consecutive
+// blk-wide column blocks x box_rows rows lands as box_blocks [box_rows x blk]
+// tiles one after another in shared memory.
+bool make_tmap_3d_blocks(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                         int elem_bytes, uint64_t rows, uint64_t cols, uint32_t blk,
+                         uint32_t box_rows, uint32_t box_blocks);
 
 // Number of SMs of the current device (cached per device).
 int sm_count();

@@ -30,7 +30,7 @@ namespace qlora {
 
 namespace {
 
-constexpr int kBKn = 64;  // contraction (n) per stage: one 128-byte row of bf16
+constexpr int kBlkN = 64;  // one 128-byte swizzle row of bf16: the dY block a 2-D box covers
 constexpr int kDqWarps = 8;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * (kDqWarps + kEpiWarps);
@@ -39,6 +39,10 @@ constexpr int kSmemLimit = 232448;
 template <int MSUB, int BN, int RMAX>
 struct K3Cfg {
     static constexpr int kBM = 128 * MSUB;
+    // contraction (n) per stage: 128 (two 64-column dY blocks in one 3-D TMA
+    // box), 64 for the 256-row tiles so that two stages fit
+    static constexpr int kBKn = MSUB == 2 ? 64 : 128;
+    static constexpr int kBlk = kBKn / kBlkN;
     // rank <= 16: c G A^T runs on the tensor cores as tf32 MMAs into the same
     // fp32 accumulator (operand tables c*G [kBM x kKL] and A [BN x kKL] per
     // accumulator buffer); larger ranks fall back to CUDA-core FMAs.
@@ -48,18 +52,14 @@ struct K3Cfg {
     static constexpr int kAtBytes = kLoraMMA ? BN * kKL * 4 : 0;
     static constexpr int kASub = 128 * kBKn * 2;       // one dY sub-tile, bf16
     static constexpr int kABytes = MSUB * kASub;
-    static constexpr int kQBytes = kBKn * BN;          // int8 kernel tile
     static constexpr int kWBytes = kBKn * BN * 2;      // de-quantized bf16 tile
-    static constexpr int kStageBytes = kABytes + kQBytes + kWBytes;
+    static constexpr int kStageBytes = kABytes + kWBytes;
     static constexpr int kStgBytes = kEpiWarps * 32 * stage_pitch<__nv_bfloat16>();
     static constexpr int kParamBytes = 2 * (kGtBytes + kAtBytes);
     static constexpr int kFixed = kStgBytes + kParamBytes + 512 + 1024;
     static constexpr int kStagesFit = (kSmemLimit - kFixed) / kStageBytes;
     static constexpr int STAGES = kStagesFit > 8 ? 8 : kStagesFit;
     static_assert(STAGES >= 2, "shared memory budget");
-    // de-quantize warps per ring stage (warps beyond STAGES * kDqPerStage idle)
-    static constexpr int kDqPerStage = kDqWarps / STAGES > 0 ? kDqWarps / STAGES : 1;
-    static_assert(STAGES <= kDqWarps, "one de-quantize warp per stage at least");
     static constexpr int kStgOff = STAGES * kStageBytes;
     static constexpr int kTabOff = kStgOff + kStgBytes;
     static constexpr int kBarOff = kTabOff + kParamBytes;
@@ -128,11 +128,12 @@ __device__ __forceinline__ void dequant16(const uint4 raw, float scale, uint32_t
 
 template <int MSUB, int BN, int RMAX>
 __global__ void __launch_bounds__(kThreads, 1)
-    k3_dx_dequant_kernel(const __grid_constant__ CUtensorMap tmDY,
-                         const __grid_constant__ CUtensorMap tmQ, const float* __restrict__ sw,
-                         int M, int N, int K, DxEpilogue ep, int* status) {
+    k3_dx_dequant_kernel(const __grid_constant__ CUtensorMap tmDY, int dy3d,
+                         const int8_t* __restrict__ Wq, const float* __restrict__ sw, int M, int N,
+                         int K, DxEpilogue ep, int* status) {
     using C = K3Cfg<MSUB, BN, RMAX>;
     constexpr int S = C::STAGES;
+    constexpr int kBKn = C::kBKn;
     constexpr uint32_t kLbo = (kBKn / 8) * 1024;  // MN-block stride of the bf16 tile
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -180,12 +181,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------ producer
         if (lane == 0) {
             tma_prefetch_desc(&tmDY);
-            tma_prefetch_desc(&tmQ);
             int g = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
                 const int m0 = (t / num_k) * C::kBM;
-                const int k0 = (t % num_k) * BN;
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
                     const int s = g % S;
                     if (g >= S && !mbar_wait(&empty[s], ((g / S) - 1) & 1, status)) {
@@ -193,11 +192,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     uint8_t* sa = smem + s * C::kStageBytes;
-                    mbar_arrive_expect_tx(&full[s], C::kABytes + C::kQBytes);
+                    mbar_arrive_expect_tx(&full[s], C::kABytes);
 #pragma unroll
-                    for (int ms = 0; ms < MSUB; ++ms)
-                        tma_load_2d(sa + ms * C::kASub, &tmDY, &full[s], kb * kBKn, m0 + 128 * ms);
-                    tma_load_2d(sa + C::kABytes, &tmQ, &full[s], k0, kb * kBKn);
+                    for (int ms = 0; ms < MSUB; ++ms) {
+                        // the stage's kBlk 64-column blocks, consecutive in shared memory
+                        if (dy3d) {
+                            tma_load_3d(sa + ms * C::kASub, &tmDY, &full[s], 0, m0 + 128 * ms,
+                                        kb * C::kBlk);
+                        } else {
+#pragma unroll
+                            for (int b = 0; b < C::kBlk; ++b)
+                                tma_load_2d(sa + ms * C::kASub + b * (128 * kBlkN * 2), &tmDY, &full[s],
+                                            (kb * C::kBlk + b) * kBlkN, m0 + 128 * ms);
+                        }
+                    }
                 }
             }
         }
@@ -222,14 +230,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc_fence_after();
                     const uint32_t a_base = smem_u32(smem + s * C::kStageBytes);
-                    const uint32_t w_base = a_base + C::kABytes + C::kQBytes;
+                    const uint32_t w_base = a_base + C::kABytes;
 #pragma unroll
                     for (int kk = 0; kk < kBKn / 16; ++kk) {
                         const uint64_t bd = smem_desc(w_base + kk * 2048, kLbo, 1024, kLayoutSw128);
 #pragma unroll
                         for (int ms = 0; ms < MSUB; ++ms) {
-                            const uint64_t ad = smem_desc(a_base + ms * C::kASub + kk * 32, 16, 1024,
-                                                          kLayoutSw128);
+                            // 16-column step kk: block kk / 4 of the sub-tile, 32 bytes per step within it
+                            const uint64_t ad = smem_desc(
+                                a_base + ms * C::kASub + (kk >> 2) * (128 * kBlkN * 2) + (kk & 3) * 32, 16,
+                                1024, kLayoutSw128);
                             mma_bf16(tmem + ab * C::kAccCols + ms * BN, ad, bd, idesc, (kb | kk) != 0);
                         }
                     }
@@ -263,9 +273,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp < 2 + kDqWarps) {
         // ------------------------------------------------------ de-quantize
         // All eight warps convert every stage, each its own slice of the
-        // chunks, walking the stages in order (so every barrier phase is
-        // awaited in turn); a warp's row scales are loaded before it waits
-        // for the stage, so no global load sits on the conversion path.
+        // 16-byte chunks, walking the stages in order (so every barrier phase
+        // is awaited in turn).  The int8 codes and row scales come straight
+        // from global memory into registers, S stages ahead of their use (a
+        // ring slot u per ring stage u), so neither a TMA box nor a load
+        // latency sits on the conversion path; a stage only waits for its
+        // bf16 slot to be released by the MMAs that read it last.
         const int dw = warp - 2;  // 0 .. 7
         constexpr int kChunksPerRow = BN / 16;
         constexpr int kChunks = kBKn * kChunksPerRow;
@@ -273,38 +286,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         static_assert(kChunks % (32 * kDqWarps) == 0, "chunks per stage");
         const int my_tiles = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
         const int total_kb = my_tiles * nkb;
-        for (int g = 0; g < total_kb; ++g) {
-            const int s = g % S;
+        uint4 qr[S][kPerLane];
+        float sr[S][kPerLane];
+        auto fetch = [&](int g, uint4 (&q)[kPerLane], float (&sc)[kPerLane]) {
+            const int t = blockIdx.x + (g / nkb) * gridDim.x;
+            const int k0 = (t % num_k) * BN;
             const int kb = g % nkb;
-            float scl[kPerLane];
 #pragma unroll
             for (int i = 0; i < kPerLane; ++i) {
-                const int n = kb * kBKn + (dw * 32 + lane + i * 32 * kDqWarps) / kChunksPerRow;
-                scl[i] = n < N ? __ldg(sw + n) : 0.f;
+                const int c = dw * 32 + lane + i * 32 * kDqWarps;
+                const int n = kb * kBKn + c / kChunksPerRow;
+                const int k = k0 + (c % kChunksPerRow) * 16;
+                const bool in = g < total_kb && n < N && k < K;
+                q[i] = in ? __ldg(reinterpret_cast<const uint4*>(Wq + static_cast<size_t>(n) * K + k))
+                          : make_uint4(0u, 0u, 0u, 0u);
+                sc[i] = in ? __ldg(sw + n) : 0.f;
             }
-            if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (g / S) & 1, status))) break;
-            {
-                const uint8_t* sq = smem + s * C::kStageBytes + C::kABytes;
-                uint8_t* wt = smem + s * C::kStageBytes + C::kABytes + C::kQBytes;
+        };
+#pragma unroll
+        for (int u = 0; u < S; ++u) fetch(u, qr[u], sr[u]);
+        bool live = true;
+        for (int g0 = 0; g0 < total_kb && live; g0 += S) {
+#pragma unroll
+            for (int u = 0; u < S; ++u) {
+                const int g = g0 + u;  // ring stage g % S == u
+                if (g >= total_kb) break;
+                if (g >= S &&
+                    !__all_sync(0xffffffffu, mbar_wait(&empty[u], ((g / S) - 1) & 1, status))) {
+                    live = false;
+                    break;
+                }
+                uint8_t* wt = smem + u * C::kStageBytes + C::kABytes;
 #pragma unroll
                 for (int i = 0; i < kPerLane; ++i) {
                     const int c = dw * 32 + lane + i * 32 * kDqWarps;
                     const int nr = c / kChunksPerRow;   // contraction row within the stage
                     const int kc = c % kChunksPerRow;   // 16 output columns
-                    const float scale = scl[i];
-                    const uint4 raw = *reinterpret_cast<const uint4*>(sq + nr * BN + kc * 16);
                     uint32_t o[8];
-                    dequant16(raw, scale, o);
+                    dequant16(qr[u][i], sr[u][i], o);
                     const int mn = kc * 16;
                     *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn, nr, kLbo)) =
                         make_uint4(o[0], o[1], o[2], o[3]);
                     *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn + 8, nr, kLbo)) =
                         make_uint4(o[4], o[5], o[6], o[7]);
                 }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&wready[u]);
+                fetch(g + S, qr[u], sr[u]);
             }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&wready[s]);
         }
         __syncwarp();
     } else {
@@ -399,24 +429,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int MSUB, int BN, int RMAX>
-cudaError_t launch_tc(const CUtensorMap& tdy, const CUtensorMap& tq, const float* sw, int M, int N,
-                      int K, const DxEpilogue& ep, int* status, cudaStream_t s) {
+cudaError_t launch_tc(const void* dY, const int8_t* Wq, const float* sw, int M, int N, int K,
+                      const DxEpilogue& ep, int* status, cudaStream_t s) {
     using C = K3Cfg<MSUB, BN, RMAX>;
     auto kern = k3_dx_dequant_kernel<MSUB, BN, RMAX>;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), C::kTotal);
     if (e != cudaSuccess) return e;
+    // dY as [row][64-column block][64] (one 3-D box per stage) when the rows
+    // split into whole blocks; otherwise one 2-D box per 64-column block
+    CUtensorMap tdy;
+    const int dy3d = (N % kBlkN) == 0 ? 1 : 0;
+    const bool ok =
+        dy3d ? make_tmap_3d_blocks(&tdy, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, kBlkN, 128,
+                                   C::kBlk)
+             : make_tmap_2d(&tdy, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N,
+                            static_cast<uint64_t>(N) * 2, 128, kBlkN, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return cudaErrorInvalidValue;
     const int tiles = ((M + C::kBM - 1) / C::kBM) * ((K + BN - 1) / BN);
     const int grid = tiles < sm_count() ? tiles : sm_count();
-    return launch_k(kern, dim3(grid), dim3(kThreads), C::kTotal, s, 1, tdy, tq, sw, M, N, K, ep,
+    return launch_k(kern, dim3(grid), dim3(kThreads), C::kTotal, s, 1, tdy, dy3d, Wq, sw, M, N, K, ep,
                     status);
 }
 
 template <int RMAX>
-cudaError_t launch_tc_cfg(int cfg, const CUtensorMap& tdy, const CUtensorMap& tq, const float* sw,
-                          int M, int N, int K, const DxEpilogue& ep, int* status, cudaStream_t s) {
-    if (cfg == 0) return launch_tc<2, 128, RMAX>(tdy, tq, sw, M, N, K, ep, status, s);
-    if (cfg == 1) return launch_tc<1, 128, RMAX>(tdy, tq, sw, M, N, K, ep, status, s);
-    return launch_tc<1, 64, RMAX>(tdy, tq, sw, M, N, K, ep, status, s);
+cudaError_t launch_tc_cfg(int cfg, const void* dY, const int8_t* Wq, const float* sw, int M, int N,
+                          int K, const DxEpilogue& ep, int* status, cudaStream_t s) {
+    if (cfg == 0) return launch_tc<2, 128, RMAX>(dY, Wq, sw, M, N, K, ep, status, s);
+    if (cfg == 1) return launch_tc<1, 128, RMAX>(dY, Wq, sw, M, N, K, ep, status, s);
+    return launch_tc<1, 64, RMAX>(dY, Wq, sw, M, N, K, ep, status, s);
 }
 
 // ---------------------------------------------------------------- SIMT path
@@ -514,18 +554,10 @@ cudaError_t launch_gemm_dx(Act act, const void* dY, const int8_t* Wq, const floa
     else if (ntiles(128, 128) >= sms) cfg = 1;
     const int forced = tile_override("QLORA_DX_TILE");  // tuning: 0, 1 or 2
     if (forced >= 0 && forced <= 2) cfg = forced;
-    const int bn = cfg == 2 ? 64 : 128;
-    CUtensorMap tdy, tq;
-    if (!make_tmap_2d(&tdy, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N,
-                      static_cast<uint64_t>(N) * 2, 128, kBKn, CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
-    if (!make_tmap_2d(&tq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, kBKn, bn,
-                      CU_TENSOR_MAP_SWIZZLE_NONE))
-        return cudaErrorInvalidValue;
-    if (ep.r <= 4) return launch_tc_cfg<4>(cfg, tdy, tq, sw, M, N, K, ep, status, s);
-    if (ep.r <= 8) return launch_tc_cfg<8>(cfg, tdy, tq, sw, M, N, K, ep, status, s);
-    if (ep.r <= 16) return launch_tc_cfg<16>(cfg, tdy, tq, sw, M, N, K, ep, status, s);
-    return launch_tc_cfg<64>(cfg, tdy, tq, sw, M, N, K, ep, status, s);
+    if (ep.r <= 4) return launch_tc_cfg<4>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
+    if (ep.r <= 8) return launch_tc_cfg<8>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
+    if (ep.r <= 16) return launch_tc_cfg<16>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
+    return launch_tc_cfg<64>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
 }
 
 }  // namespace qlora

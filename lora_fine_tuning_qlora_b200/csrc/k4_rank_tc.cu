@@ -26,9 +26,12 @@
 // [B_hi | B_lo].  The head and remainder halves sit RP = roundup(r, 16)
 // columns apart in TMEM, so one 16-column load of each gives 16 sums.
 //
-// The CL <= 8 CTAs that share a column block form a cluster along the rows
-// and add their [128 x r] partials through distributed shared memory in rank
-// order: dB, dbias and dA leave the kernel final and deterministic.
+// The CL <= 8 CTAs that share a column block form a cluster along the rows.
+// Each CTA owns 128/CL of the block's columns: every CTA stores its partials
+// for those columns into the owner's shared memory (distributed shared
+// memory) and arrives on the owner's mbarrier; the owner adds the CL partials
+// in rank order, so dB, dbias and dA leave the kernel final and
+// deterministic, with no cluster-wide barrier at the end.
 //
 // Warps: 0 TMA producer, 1 TMEM owner + MMA issuer, 2..5 operand tables and
 // epilogues (warp w owns TMEM lane quarter w % 4).
@@ -68,7 +71,7 @@ struct RankTcArgs {
 // Shared-memory and TMEM layout for rank r (same on host and device).
 struct RtLayout {
     int RP, NG, NV, JP;
-    uint32_t vtab, bcat, part, bar, total;
+    uint32_t vtab, bcat, recv, bar, total;
     uint32_t tmem_cols, d_col, g_col;
     __host__ __device__ RtLayout(bool dy, int r) {
         RP = (r + 15) / 16 * 16;
@@ -77,8 +80,8 @@ struct RtLayout {
         JP = dy ? r + 1 : r;
         vtab = 2 * kTileBytes;
         bcat = vtab + 2 * static_cast<uint32_t>(NV) * 256;
-        part = bcat + static_cast<uint32_t>(NG) * 256;
-        bar = part + ((kTileCols * JP * 4 + 15) / 16) * 16;
+        recv = bcat + static_cast<uint32_t>(NG) * 256;
+        bar = recv + (((kTileCols + kMaxCluster) * JP * 4 + 15) / 16) * 16;
         total = bar + 128;
         d_col = 0;
         g_col = static_cast<uint32_t>(NV);
@@ -106,7 +109,7 @@ __device__ __forceinline__ void put_split(uint8_t* tab, int row_hi, int row_lo, 
 
 template <bool kDy>
 __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_constant__ CUtensorMap tmT,
-                                                              RankTcArgs a, int* status) {
+                                                              int t3d, RankTcArgs a, int* status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -118,8 +121,10 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
     uint64_t* gfull = bars + 6;   // [2] G accumulator ready
     uint64_t* gempty = bars + 8;  // [2] G accumulator read out
     uint64_t* dfull = bars + 10;  // column accumulator final
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
-    float* part = reinterpret_cast<float*>(smem + L.part);
+    uint64_t* rbar = bars + 11;   // every CTA of the cluster delivered this CTA's column slice
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+    // recv[q][c][j]: partial of CTA q for column cbeg + c of this CTA's slice
+    float* recv = reinterpret_cast<float*>(smem + L.recv);
 
     cg::cluster_group cluster = cg::this_cluster();
     const int CL = static_cast<int>(cluster.num_blocks());
@@ -131,6 +136,10 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
     const int t0 = blockIdx.y * a.tiles_per_cta;
     const int t1 = min(mtiles, t0 + a.tiles_per_cta);
     const int nt = t1 > t0 ? t1 - t0 : 0;
+    // the 128 columns are split over the cluster: CTA q sums columns [q*per, q*per + per)
+    const int per = (kTileCols + CL - 1) / CL;
+    const int cbeg = crank * per;
+    const int cend = min(kTileCols, cbeg + per);
     pdl_trigger();
 
     if (threadIdx.x == 0) {
@@ -142,6 +151,7 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
             mbar_init(&gempty[s], kWorkers);
         }
         mbar_init(dfull, 1);
+        mbar_init(rbar, static_cast<uint32_t>(CL * (cend > cbeg ? cend - cbeg : 1)));
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -152,6 +162,8 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // no CTA of the cluster arrives on another's barrier before all are initialised
+    cluster_arrive_relaxed();
     pdl_wait();  // nothing above read global memory
 
     if (warp == 0) {
@@ -164,11 +176,16 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
                 uint8_t* dst = smem + s * kTileBytes;
                 const int m0 = (t0 + i) * kTileRows;
                 mbar_arrive_expect_tx(&full[s], kTileBytes);
-                tma_load_2d(dst, &tmT, &full[s], col0, m0);
-                tma_load_2d(dst + kBoxBytes, &tmT, &full[s], col0 + kBoxCols, m0);
+                if (t3d) {  // both 64-column blocks in one box
+                    tma_load_3d(dst, &tmT, &full[s], 0, m0, col0 / kBoxCols);
+                } else {
+                    tma_load_2d(dst, &tmT, &full[s], col0, m0);
+                    tma_load_2d(dst + kBoxBytes, &tmT, &full[s], col0 + kBoxCols, m0);
+                }
             }
         }
         __syncwarp();
+        cluster_wait();
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -216,6 +233,7 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
             if (ok) mma_commit(dfull);
         }
         __syncwarp();
+        cluster_wait();
     } else {
         // ------------------------------------------------------ tables, epilogues
         const int wq = warp & 3;
@@ -272,13 +290,16 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
                         for (int e = 0; e < 8; ++e)
                             if (e < nv) v[e] = __ldg(p + e);
                     } else {
-                        // G = the slices added in ascending order
+                        // G = the slices added in ascending order, every load issued at once
                         const size_t stride = static_cast<size_t>(a.M) * a.r;
-#pragma unroll 4
-                        for (int b = 0; b < a.nsl; ++b, p += stride)
 #pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                if (e < nv) v[e] += __ldg(p + e);
+                        for (int b = 0; b < kMaxDirectSlices; ++b)
+                            if (b < a.nsl)
+#pragma unroll
+                                for (int e = 0; e < 8; ++e)
+                                    if (e < nv) v[e] += __ldg(p + b * stride + e);
+                        for (int b = kMaxDirectSlices; b < a.nsl; ++b)
+                            for (int e = 0; e < nv; ++e) v[e] += __ldg(p + b * stride + e);
                     }
                 }
 #pragma unroll
@@ -301,8 +322,11 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
         if constexpr (kDy) {
             if (ok && nt >= 1) g_epilogue(nt - 1);
         }
-        // this CTA's column partials: part[col][j] (and the dbias column)
-        float* pc = part + rr * L.JP;
+        // this CTA's partial of column rr goes to the CTA that owns the column
+        cluster_wait();  // every CTA of the cluster has initialised its barriers
+        const int owner = rr / per;
+        const uint32_t dst = dsmem_addr(recv + (crank * per + rr - owner * per) * L.JP,
+                                        static_cast<uint32_t>(owner));
         if (ok && nt > 0) ok = __all_sync(0xffffffffu, mbar_wait(dfull, 0, status));
         if (ok && nt > 0) {
             tc_fence_after();
@@ -314,17 +338,19 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
                 tmem_ld_wait();
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
-                    if (c0 + e < a.r) pc[c0 + e] = __uint_as_float(hi[e]) + __uint_as_float(lo[e]);
+                    if (c0 + e < a.r)
+                        dsmem_st(dst + 4 * (c0 + e), __uint_as_float(hi[e]) + __uint_as_float(lo[e]));
             }
             if constexpr (kDy) {
                 uint32_t ones[16];
                 tmem_ld16(base + 2 * L.RP, ones);
                 tmem_ld_wait();
-                pc[a.r] = __uint_as_float(ones[0]);
+                dsmem_st(dst + 4 * a.r, __uint_as_float(ones[0]));
             }
         } else {
-            for (int j = 0; j < L.JP; ++j) pc[j] = 0.f;
+            for (int j = 0; j < L.JP; ++j) dsmem_st(dst + 4 * j, 0.f);
         }
+        mbar_arrive_remote(dsmem_addr(rbar, static_cast<uint32_t>(owner)));
         __syncwarp();
     }
     tc_fence_before();
@@ -334,27 +360,26 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
         tmem_dealloc(tmem, L.tmem_cols);
     }
 
-    // cluster sum of the partials, rank by rank; rank q finalises its slice
-    cluster.sync();
-    const int per = (kTileCols + CL - 1) / CL;
-    const int cbeg = crank * per;
-    const int cend = min(kTileCols, cbeg + per);
+    // this CTA's slice of the columns: the CL partials added in rank order.
+    // Once every CTA's partials have arrived nothing reads or writes this
+    // CTA's shared memory from outside, so it may exit without a cluster barrier.
     const int width = cend - cbeg;
-    if (width > 0) {
+    const bool got = mbar_wait_cluster(rbar, 0, status);
+    if (got && width > 0) {
         for (int idx = threadIdx.x; idx < L.JP * width; idx += kThreads) {
             int j, cc;
             if constexpr (kDy) {  // dB is [r, C]: consecutive threads take consecutive columns
                 j = idx / width;
-                cc = cbeg + idx % width;
+                cc = idx % width;
             } else {              // dA is [C, r]: consecutive threads take consecutive ranks
-                cc = cbeg + idx / L.JP;
+                cc = idx / L.JP;
                 j = idx % L.JP;
             }
-            const int col = col0 + cc;
+            const int col = col0 + cbeg + cc;
             if (col >= a.C) continue;
             if (kDy && j == a.r && a.dbias == nullptr) continue;
             float sum = 0.f;
-            for (int q = 0; q < CL; ++q) sum += cluster.map_shared_rank(part, q)[cc * L.JP + j];
+            for (int q = 0; q < CL; ++q) sum += recv[(q * per + cc) * L.JP + j];
             if constexpr (kDy) {
                 if (j < a.r) a.out[static_cast<size_t>(j) * a.C + col] = a.c * sum;
                 else a.dbias[col] = sum;
@@ -363,16 +388,21 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
             }
         }
     }
-    cluster.sync();
 }
 
 template <bool kDy>
 cudaError_t launch_tc(const void* T, RankTcArgs a, int* status, cudaStream_t s) {
+    // T as [row][64-column block][64] when its rows split into whole blocks
+    // (one box per tile), else one 2-D box per 64-column block
     CUtensorMap tm;
-    if (!make_tmap_2d(&tm, T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.C,
-                      static_cast<uint64_t>(a.C) * 2, kTileRows, kBoxCols,
-                      CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
+    const int t3d = (a.C % kBoxCols) == 0 ? 1 : 0;
+    const bool ok =
+        t3d ? make_tmap_3d_blocks(&tm, T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.C, kBoxCols,
+                                  kTileRows, 2)
+            : make_tmap_2d(&tm, T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.C,
+                           static_cast<uint64_t>(a.C) * 2, kTileRows, kBoxCols,
+                           CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return cudaErrorInvalidValue;
     const RtLayout L(kDy, a.r);
     const size_t smem = L.total + 1024;
     auto kern = k4_rank_tc_kernel<kDy>;
@@ -386,7 +416,7 @@ cudaError_t launch_tc(const void* T, RankTcArgs a, int* status, cudaStream_t s) 
     a.tiles_per_cta = (mtiles + max_cl - 1) / max_cl;
     const int cl = (mtiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
     const dim3 grid((a.C + kTileCols - 1) / kTileCols, cl);
-    return launch_k(kern, grid, dim3(kThreads), smem, s, cl, tm, a, status);
+    return launch_k(kern, grid, dim3(kThreads), smem, s, cl, tm, t3d, a, status);
 }
 
 }  // namespace

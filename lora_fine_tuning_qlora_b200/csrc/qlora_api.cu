@@ -137,6 +137,22 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
     return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_3d_blocks(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                         int elem_bytes, uint64_t rows, uint64_t cols, uint32_t blk,
+                         uint32_t box_rows, uint32_t box_blocks) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || cols % blk != 0) return false;
+    const uint64_t eb = static_cast<uint64_t>(elem_bytes);
+    cuuint64_t dims[3] = {blk, rows, cols / blk};
+    cuuint64_t strides[2] = {cols * eb, blk * eb};
+    cuuint32_t box[3] = {blk, box_rows, box_blocks};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, dtype, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 int tile_override(const char* name) {
     static std::mutex mu;
     static std::map<std::string, int> cache;
