@@ -23,9 +23,19 @@ class MLPStack:
         self.M = batch
         self.act = layers[0].act
         dev = torch.device(device)
-        # the largest workspace over the layers serves all of them
+        # the largest workspace over the layers serves all of them; two of them
+        # alternate between layers in the backward, so that a layer's X pass
+        # (on the side stream) can still read its G while the next layer's
+        # dY pass writes the other one
         need = max(qlora.qlora_workspace_bytes(L.desc(), batch) for L in layers)
         self.ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        self.ws_alt = torch.empty(need, dtype=torch.uint8, device=dev)
+        # the X pass (dA) feeds nothing in the backward but the final gradient,
+        # so it runs on a side stream, overlapping the next layers' dY passes
+        # and dX GEMMs, which carry the critical path
+        self.side = torch.cuda.Stream(device=dev)
+        self.ev_g = [torch.cuda.Event() for _ in layers]  # layer's G is in its workspace
+        self.ev_x = [torch.cuda.Event() for _ in layers]  # layer's X pass is done
         self.X = torch.zeros((batch, layers[0].K), dtype=self.act, device=dev)
         self.dY = torch.zeros((batch, layers[-1].N), dtype=self.act, device=dev)
         self.H = [torch.empty((batch, L.N), dtype=self.act, device=dev) for L in layers]
@@ -91,35 +101,44 @@ class MLPStack:
         D = self.descs
         M = self.M
         ev_f = events.get("gemm_forward") if events else None
+        fwd = stream if stream is not None else torch.cuda.current_stream()
         ev_d = events.get("gemm_dx") if events else None
         h = self.X
         for i, L in enumerate(L_):
             qlora.qlora_quantize_input(D[i], M, h, L.A, self.Xq, self.sx, self.xA[i], stream)
             if ev_f and ev_f[i]:
-                ev_f[i][0].record()
+                ev_f[i][0].record(fwd)
             qlora.qlora_gemm_forward(D[i], M, self.Xq, self.sx, L.Wq, L.sw, L.bias, self.xA[i],
                                      L.B, self.H[i], None, stream)
             if ev_f and ev_f[i]:
-                ev_f[i][1].record()
+                ev_f[i][1].record(fwd)
             if i < n - 1:
                 qlora.qlora_relu(self.H[i], stream)
             h = self.H[i]
+        main = stream if stream is not None else torch.cuda.current_stream()
         g = self.dY
         for i in range(n - 1, -1, -1):
             L = L_[i]
+            ws = self.ws if i % 2 == 0 else self.ws_alt
             if i < n - 1:
-                qlora.qlora_relu_backward(g, self.H[i], stream)
+                qlora.qlora_relu_backward(g, self.H[i], main)
             x_in = self.X if i == 0 else self.H[i - 1]
             dX = self.dX if i == 0 else self.G[i - 1]
+            if i + 2 < n:
+                main.wait_event(self.ev_x[i + 2])  # the X pass that read this workspace
             qlora.qlora_lora_grad_dy(D[i], M, g, L.B, self.xA[i], self.dB[i], self.dbias[i],
-                                     self.ws, None, stream)
+                                     ws, None, main)
+            self.ev_g[i].record(main)
             if ev_d and ev_d[i]:
-                ev_d[i][0].record()
-            qlora.qlora_gemm_dx(D[i], M, g, L.Wq, L.sw, L.A, dX, self.ws, stream)
+                ev_d[i][0].record(main)
+            qlora.qlora_gemm_dx(D[i], M, g, L.Wq, L.sw, L.A, dX, ws, main)
             if ev_d and ev_d[i]:
-                ev_d[i][1].record()
-            qlora.qlora_lora_grad_x(D[i], M, x_in, self.dA[i], self.ws, stream)
+                ev_d[i][1].record(main)
+            self.side.wait_event(self.ev_g[i])
+            qlora.qlora_lora_grad_x(D[i], M, x_in, self.dA[i], ws, self.side)
+            self.ev_x[i].record(self.side)
             g = dX
+        main.wait_stream(self.side)
 
     def make_events(self, kinds=("gemm_dx",), layers=None):
         """Timing events (graph-capturable) around the given steps of the
