@@ -210,6 +210,19 @@ int qlora_lora_grad_dy(const qlora_layer_desc* d, int M, const void* dY, const f
                        const float* xA, float* dB, float* dbias, float* G, void* workspace,
                        size_t workspace_bytes, void* stream);
 
+/* a3 in two halves, for callers that put G on their critical path and the
+ * parameter gradients on another stream:
+ *   qlora_lora_g      : G = dY B^T into the workspace, exactly as
+ *                       qlora_lora_grad_dy leaves it for a4 and a5;
+ *   qlora_lora_grad_b : dB = c * xA^T dY [r,N] and, if dbias is not NULL,
+ *                       dbias = column sums of dY [N]; touches no workspace.
+ * Together they give the same results as qlora_lora_grad_dy, each with one
+ * more read of dY.  Deterministic. */
+int qlora_lora_g(const qlora_layer_desc* d, int M, const void* dY, const float* B,
+                 void* workspace, size_t workspace_bytes, void* stream);
+int qlora_lora_grad_b(const qlora_layer_desc* d, int M, const void* dY, const float* xA,
+                      float* dB, float* dbias, void* stream);
+
 /* a4: dX = dY (Wq * sw)^T + c * G A^T [M,K], G from the workspace that a3
  * filled; the int8 kernel is de-quantized tile by tile in shared memory
  * ("How to fine-tune the 4-bit model?": de-quantize in place before the

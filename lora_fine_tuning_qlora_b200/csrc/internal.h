@@ -59,7 +59,8 @@ int rank_col_blocks(Act act, int N);
 // added once into G (launch_g_reduce) and the consumers read G.
 constexpr int kMaxDirectSlices = 8;
 
-// Pass over dY: G slices into Gp, final dB and dbias (dbias may be null).
+// Pass over dY: G slices into Gp, final dB and dbias.  Gp or dB may be null
+// (that half is skipped); dbias may be null.
 cudaError_t launch_rank_dy(Act act, const void* dY, const float* B, const float* xA, int M, int N,
                            int r, float c, float* Gp, float* dB, float* dbias, int* status,
                            cudaStream_t s);

@@ -159,15 +159,16 @@ __global__ void __launch_bounds__(kThreads) k4_dy_kernel(
                 for (int e = 0; e < 8; ++e) v[u][e] = 0.f;
 #pragma unroll
             for (int j = 0; j < kRJ; ++j)
-                xr[u][j] = (ok && j0 + j < r) ? __ldg(xA + static_cast<size_t>(m) * r + j0 + j) : 0.f;
+                xr[u][j] = (xA && ok && j0 + j < r) ? __ldg(xA + static_cast<size_t>(m) * r + j0 + j) : 0.f;
         }
         if (!have_b) {
 #pragma unroll
             for (int j = 0; j < kRJ; ++j)
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
-                    bv[j][e] = (j0 + j < r && c0 + e < N) ? __ldg(B + static_cast<size_t>(j0 + j) * N + c0 + e)
-                                                          : 0.f;
+                    bv[j][e] = (B && j0 + j < r && c0 + e < N)
+                                   ? __ldg(B + static_cast<size_t>(j0 + j) * N + c0 + e)
+                                   : 0.f;
             have_b = true;
         }
 #pragma unroll
@@ -186,7 +187,7 @@ __global__ void __launch_bounds__(kThreads) k4_dy_kernel(
 #pragma unroll
             for (int e = 0; e < 8; ++e) dbi[e] += v[u][e];
             const float gs = row_reduce8(g, lane);  // all lanes take part
-            if (m < mend && j0 + cl < r) Gp[(static_cast<size_t>(cb) * M + m) * r + j0 + cl] = gs;
+            if (Gp && m < mend && j0 + cl < r) Gp[(static_cast<size_t>(cb) * M + m) * r + j0 + cl] = gs;
         }
     }
 
@@ -223,7 +224,7 @@ __global__ void __launch_bounds__(kThreads) k4_dy_kernel(
         const int cc = cbeg + i % (cend - cbeg);
         const int n = cb * kCols + cc;
         if (n >= N) continue;
-        if (j < kRJ && j0 + j >= r) continue;
+        if (j < kRJ && (j0 + j >= r || dB == nullptr)) continue;
         if (j == kRJ && !with_bias) continue;
         const float s = cluster_sum(cluster, part, j * kCols + cc, CL);
         if (j < kRJ) dB[static_cast<size_t>(j0 + j) * N + n] = cscale * s;

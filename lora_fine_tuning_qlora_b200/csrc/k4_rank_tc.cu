@@ -8,39 +8,38 @@
 //
 // ("How to fine-tune the 4-bit model?" thread: the adapter's A B^T-style
 // products drive the gradient; "Parameter-efficient fine-tuning of GPT-2
-// with LoRA", "LoRA equation", for the shapes.)
+// with LoRA", "LoRA equation", for the shapes.)  The dY pass also runs as
+// two halves, G alone and dB + dbias alone, so that a caller can put G on
+// its critical path and the parameter gradients elsewhere.
 //
 // A CTA owns 128 columns of the activation T (dY or X) and a run of 128-row
-// tiles.  Each tile arrives by TMA as two [128 rows x 64 columns] boxes with
-// the 128-byte swizzle, and the one copy in shared memory is read two ways
-// by tcgen05.mma.kind::f16 (bf16 in, fp32 accumulate in TMEM):
+// tiles.  Each tile arrives by TMA (one 3-D box of two 64-column blocks, or
+// two 2-D boxes) with the 128-byte swizzle, and the one copy in shared
+// memory is read two ways by tcgen05.mma.kind::f16 (bf16 in, fp32
+// accumulate in TMEM):
 //   * K-major (rows = M dimension, columns = contraction): T . Bcat^T gives
-//     the tile's G rows (dY pass only);
+//     the tile's G rows;
 //   * MN-major (columns = M dimension, rows = contraction): T^T . Vcat sums
 //     over the tile's rows into a [128 columns x NV] accumulator that stays
-//     in TMEM across all the CTA's tiles: dB^T and dbias (dY pass), dA (X pass).
+//     in TMEM across all the CTA's tiles: dB^T and dbias, or dA.
 // The fp32 factors enter as bf16 head + remainder pairs (v = hi + lo to
 // 16 significant bits; every bf16 x bf16 product is exact in fp32), so the
-// sums carry fp32-level accuracy.  Vcat holds [xA_hi | xA_lo | 1] (dY pass;
-// the ones column yields dbias) or [G_hi | G_lo] (X pass); Bcat holds
-// [B_hi | B_lo].  The head and remainder halves sit RP = roundup(r, 16)
-// columns apart in TMEM, so one 16-column load of each gives 16 sums.
+// sums carry fp32-level accuracy.  Vcat holds [xA_hi | xA_lo | 1] (the ones
+// column yields dbias) or [G_hi | G_lo]; Bcat holds [B_hi | B_lo].  The head
+// and remainder halves sit RP = roundup(r, 16) columns apart in TMEM, so one
+// 16-column load of each gives 16 sums.
 //
-// The CL <= 8 CTAs that share a column block form a cluster along the rows.
-// Each CTA owns 128/CL of the block's columns: every CTA stores its partials
-// for those columns into the owner's shared memory (distributed shared
-// memory) and arrives on the owner's mbarrier; the owner adds the CL partials
-// in rank order, so dB, dbias and dA leave the kernel final and
-// deterministic, with no cluster-wide barrier at the end.
+// Column sums: the CL <= 8 CTAs that share a column block form a cluster
+// along the rows.  Each CTA owns 128/CL of the block's columns: every CTA
+// stores its partials for those columns into the owner's shared memory
+// (distributed shared memory) and arrives on the owner's mbarrier; the owner
+// adds the CL partials in rank order, so dB, dbias and dA leave the kernel
+// final and deterministic, with no cluster-wide barrier at the end.
 //
 // Warps: 0 TMA producer, 1 TMEM owner + MMA issuer, 2..5 operand tables and
 // epilogues (warp w owns TMEM lane quarter w % 4).
-#include <cooperative_groups.h>
-
 #include "internal.h"
 #include "ptx.cuh"
-
-namespace cg = cooperative_groups;
 
 namespace qlora {
 
@@ -56,13 +55,20 @@ constexpr int kThreads = 64 + 32 * kWorkers;
 constexpr int kMaxCluster = 8;
 constexpr uint32_t kTabSbo = (kTileCols / 8) * 128;  // 8-row group stride of a 128-wide table
 
+// What one launch computes.
+struct Parts {
+    bool g;     // G slices from T . B^T
+    bool d;     // column sums T^T . V (dB or dA), reduced over the cluster
+    bool ones;  // a ones column in V (dbias)
+};
+
 struct RankTcArgs {
-    const float* V;      // dY pass: xA [M, r]; X pass: G slices (nsl of them) or G
-    int nsl;             // X pass: slices to add (1 = G itself)
-    const float* B;      // dY pass: B [r, C]
-    float* Gp;           // dY pass: G slices [ceil(C/128)][M, r]
-    float* out;          // dY pass: dB [r, C]; X pass: dA [C, r]
-    float* dbias;        // dY pass: [C] or nullptr
+    const float* V;      // column sums: xA [M, r] (nsl = 1) or the nsl slices of G
+    int nsl;
+    const float* B;      // G: B [r, C]
+    float* Gp;           // G: slices out [ceil(C/128)][M, r]
+    float* out;          // column sums: dB [r, C] (with ones) or dA [C, r]
+    float* dbias;        // with ones: [C] or nullptr
     int M, C, r;
     int tiles_per_cta;   // 128-row tiles per CTA
     float c;
@@ -73,11 +79,11 @@ struct RtLayout {
     int RP, NG, NV, JP;
     uint32_t vtab, bcat, recv, bar, total;
     uint32_t tmem_cols, d_col, g_col;
-    __host__ __device__ RtLayout(bool dy, int r) {
+    __host__ __device__ RtLayout(Parts p, int r) {
         RP = (r + 15) / 16 * 16;
-        NG = dy ? 2 * RP : 0;
-        NV = dy ? 2 * RP + 16 : 2 * RP;
-        JP = dy ? r + 1 : r;
+        NG = p.g ? 2 * RP : 0;
+        NV = p.d ? 2 * RP + (p.ones ? 16 : 0) : 0;
+        JP = p.d ? r + (p.ones ? 1 : 0) : 0;
         vtab = 2 * kTileBytes;
         bcat = vtab + 2 * static_cast<uint32_t>(NV) * 256;
         recv = bcat + static_cast<uint32_t>(NG) * 256;
@@ -107,13 +113,13 @@ __device__ __forceinline__ void put_split(uint8_t* tab, int row_hi, int row_lo, 
     *reinterpret_cast<__nv_bfloat16*>(tab + ktab_off(row_lo, k)) = lo;
 }
 
-template <bool kDy>
+template <bool kG, bool kD, bool kOnes>
 __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_constant__ CUtensorMap tmT,
                                                               int t3d, RankTcArgs a, int* status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    const RtLayout L(kDy, a.r);
+    const RtLayout L(Parts{kG, kD, kOnes}, a.r);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar);
     uint64_t* full = bars;        // [2] tile landed
     uint64_t* vready = bars + 2;  // [2] Vcat table written
@@ -126,9 +132,11 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
     // recv[q][c][j]: partial of CTA q for column cbeg + c of this CTA's slice
     float* recv = reinterpret_cast<float*>(smem + L.recv);
 
-    cg::cluster_group cluster = cg::this_cluster();
-    const int CL = static_cast<int>(cluster.num_blocks());
-    const int crank = static_cast<int>(cluster.block_rank());
+    uint32_t CL = 1, crank = 0;
+    if constexpr (kD) {
+        asm("mov.u32 %0, %%cluster_nctarank;" : "=r"(CL));
+        asm("mov.u32 %0, %%cluster_ctarank;" : "=r"(crank));
+    }
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int cb = blockIdx.x;
     const int col0 = cb * kTileCols;
@@ -137,8 +145,8 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
     const int t1 = min(mtiles, t0 + a.tiles_per_cta);
     const int nt = t1 > t0 ? t1 - t0 : 0;
     // the 128 columns are split over the cluster: CTA q sums columns [q*per, q*per + per)
-    const int per = (kTileCols + CL - 1) / CL;
-    const int cbeg = crank * per;
+    const int per = (kTileCols + static_cast<int>(CL) - 1) / static_cast<int>(CL);
+    const int cbeg = static_cast<int>(crank) * per;
     const int cend = min(kTileCols, cbeg + per);
     pdl_trigger();
 
@@ -163,7 +171,7 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     // no CTA of the cluster arrives on another's barrier before all are initialised
-    cluster_arrive_relaxed();
+    if constexpr (kD) cluster_arrive_relaxed();
     pdl_wait();  // nothing above read global memory
 
     if (warp == 0) {
@@ -185,26 +193,28 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
             }
         }
         __syncwarp();
-        cluster_wait();
+        if constexpr (kD) cluster_wait();
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t tiles = smem_u32(smem);
             const uint32_t vt = smem_u32(smem + L.vtab);
             const uint32_t bt = smem_u32(smem + L.bcat);
-            const uint32_t id_g = idesc_bf16(128, L.NG, false, false);
-            const uint32_t id_d = idesc_bf16(128, L.NV, true, false);
+            const uint32_t id_g = idesc_bf16(128, kG ? L.NG : 16, false, false);
+            const uint32_t id_d = idesc_bf16(128, kD ? L.NV : 16, true, false);
             bool ok = true;
             for (int i = 0; i < nt; ++i) {
                 const int s = i & 1;
+                // Vcat of this tile (column sums), or the Bcat table once (G alone)
+                const bool need_v = kD || i == 0;
                 if (!mbar_wait(&full[s], (i >> 1) & 1, status) ||
-                    !mbar_wait(&vready[s], (i >> 1) & 1, status)) {
+                    (need_v && !mbar_wait(&vready[s], (i >> 1) & 1, status))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t tb = tiles + s * kTileBytes;
-                if constexpr (kDy) {
+                if constexpr (kG) {
                     // G rows of this tile: T (K-major) x Bcat
                     if (i >= 2 && !mbar_wait(&gempty[s], ((i >> 1) - 1) & 1, status)) {
                         ok = false;
@@ -220,33 +230,47 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
                     }
                     mma_commit(&gfull[s]);
                 }
-                // column sums: T^T (MN-major, the two boxes 64 columns apart) x Vcat
+                if constexpr (kD) {
+                    // column sums: T^T (MN-major, the two blocks 64 columns apart) x Vcat
 #pragma unroll
-                for (int kk = 0; kk < kTileRows / 16; ++kk) {
-                    const uint64_t ad = smem_desc(tb + kk * 2048, kBoxBytes, 1024, kLayoutSw128);
-                    const uint64_t bd =
-                        smem_desc(vt + s * L.NV * 256 + kk * 256, 128, kTabSbo, kLayoutNone);
-                    mma_bf16(tmem + L.d_col, ad, bd, id_d, (i > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kTileRows / 16; ++kk) {
+                        const uint64_t ad = smem_desc(tb + kk * 2048, kBoxBytes, 1024, kLayoutSw128);
+                        const uint64_t bd =
+                            smem_desc(vt + s * L.NV * 256 + kk * 256, 128, kTabSbo, kLayoutNone);
+                        mma_bf16(tmem + L.d_col, ad, bd, id_d, (i > 0 || kk > 0) ? 1u : 0u);
+                    }
                 }
                 mma_commit(&empty[s]);
             }
-            if (ok) mma_commit(dfull);
+            if (kD && ok) mma_commit(dfull);
         }
         __syncwarp();
-        cluster_wait();
+        if constexpr (kD) cluster_wait();
     } else {
         // ------------------------------------------------------ tables, epilogues
         const int wq = warp & 3;
         const int rr = wq * 32 + lane;  // tile row for the tables; column for the readback
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         bool ok = true;
-        if constexpr (kDy) {
-            // Bcat[j][n] = B[j, col0 + n] as head (rows 0..RP) and remainder (RP..2RP)
+        if constexpr (kG) {
+            // Bcat[j][n] = B[j, col0 + n] as head (rows 0..RP) and remainder (RP..2RP),
+            // eight loads in flight per round
             uint8_t* bt = smem + L.bcat;
             const int n = col0 + rr;
-            for (int j = 0; j < L.RP; ++j) {
-                const float v = (j < a.r && n < a.C) ? __ldg(a.B + static_cast<size_t>(j) * a.C + n) : 0.f;
-                put_split(bt, j, L.RP + j, rr, v);
+            for (int j0 = 0; j0 < L.RP; j0 += 8) {
+                float v[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    v[e] = (j0 + e < a.r && n < a.C) ? __ldg(a.B + static_cast<size_t>(j0 + e) * a.C + n)
+                                                     : 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) put_split(bt, j0 + e, L.RP + j0 + e, rr, v[e]);
+            }
+            if constexpr (!kD) {
+                // G alone: the MMAs of the first tile wait for this table on vready[0]
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&vready[0]);
             }
         }
         auto g_epilogue = [&](int i) {
@@ -272,25 +296,25 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
             __syncwarp();
             if (lane == 0) mbar_arrive(&gempty[b]);
         };
-        for (int i = 0; i < nt && ok; ++i) {
-            const int s = i & 1;
-            const int m = (t0 + i) * kTileRows + rr;
-            ok = __all_sync(0xffffffffu,
-                            i < 2 || mbar_wait(&empty[s], ((i >> 1) - 1) & 1, status));
-            if (!ok) break;
-            uint8_t* vt = smem + L.vtab + s * L.NV * 256;
-            const bool mok = m < a.M;
-            for (int j0 = 0; j0 < L.RP; j0 += 8) {
-                float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                if (mok && j0 < a.r) {
-                    const int nv = min(8, a.r - j0);
-                    const float* p = a.V + static_cast<size_t>(m) * a.r + j0;
-                    if constexpr (kDy) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            if (e < nv) v[e] = __ldg(p + e);
-                    } else {
-                        // G = the slices added in ascending order, every load issued at once
+        if constexpr (kG && !kD) {
+            // the Bcat table is the only operand the workers write
+            for (int i = 0; i < nt && ok; ++i) g_epilogue(i);
+        }
+        if constexpr (kD) {
+            for (int i = 0; i < nt && ok; ++i) {
+                const int s = i & 1;
+                const int m = (t0 + i) * kTileRows + rr;
+                ok = __all_sync(0xffffffffu,
+                                i < 2 || mbar_wait(&empty[s], ((i >> 1) - 1) & 1, status));
+                if (!ok) break;
+                uint8_t* vt = smem + L.vtab + s * L.NV * 256;
+                const bool mok = m < a.M;
+                for (int j0 = 0; j0 < L.RP; j0 += 8) {
+                    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    if (mok && j0 < a.r) {
+                        const int nv = min(8, a.r - j0);
+                        const float* p = a.V + static_cast<size_t>(m) * a.r + j0;
+                        // V = the nsl slices added in ascending order, every load issued at once
                         const size_t stride = static_cast<size_t>(a.M) * a.r;
 #pragma unroll
                         for (int b = 0; b < kMaxDirectSlices; ++b)
@@ -301,56 +325,56 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
                         for (int b = kMaxDirectSlices; b < a.nsl; ++b)
                             for (int e = 0; e < nv; ++e) v[e] += __ldg(p + b * stride + e);
                     }
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) put_split(vt, j0 + e, L.RP + j0 + e, rr, v[e]);
                 }
+                if constexpr (kOnes) {
+                    const __nv_bfloat16 one = __float2bfloat16_rn(mok ? 1.f : 0.f);
+                    const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
+                    *reinterpret_cast<__nv_bfloat16*>(vt + ktab_off(2 * L.RP, rr)) = one;
+                    for (int j = 2 * L.RP + 1; j < L.NV; ++j)
+                        *reinterpret_cast<__nv_bfloat16*>(vt + ktab_off(j, rr)) = zero;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&vready[s]);
+                if constexpr (kG) {
+                    if (i >= 1) g_epilogue(i - 1);
+                }
+            }
+            if constexpr (kG) {
+                if (ok && nt >= 1) g_epilogue(nt - 1);
+            }
+            // this CTA's partial of column rr goes to the CTA that owns the column
+            cluster_wait();  // every CTA of the cluster has initialised its barriers
+            const int owner = rr / per;
+            const uint32_t dst = dsmem_addr(recv + (static_cast<int>(crank) * per + rr - owner * per) * L.JP,
+                                            static_cast<uint32_t>(owner));
+            if (ok && nt > 0) ok = __all_sync(0xffffffffu, mbar_wait(dfull, 0, status));
+            if (ok && nt > 0) {
+                tc_fence_after();
+                const uint32_t base = tmem + lane_base + L.d_col;
+                for (int c0 = 0; c0 < L.RP; c0 += 16) {
+                    uint32_t hi[16], lo[16];
+                    tmem_ld16(base + c0, hi);
+                    tmem_ld16(base + L.RP + c0, lo);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 8; ++e) put_split(vt, j0 + e, L.RP + j0 + e, rr, v[e]);
+                    for (int e = 0; e < 16; ++e)
+                        if (c0 + e < a.r)
+                            dsmem_st(dst + 4 * (c0 + e), __uint_as_float(hi[e]) + __uint_as_float(lo[e]));
+                }
+                if constexpr (kOnes) {
+                    uint32_t ones[16];
+                    tmem_ld16(base + 2 * L.RP, ones);
+                    tmem_ld_wait();
+                    dsmem_st(dst + 4 * a.r, __uint_as_float(ones[0]));
+                }
+            } else {
+                for (int j = 0; j < L.JP; ++j) dsmem_st(dst + 4 * j, 0.f);
             }
-            if constexpr (kDy) {
-                const __nv_bfloat16 one = __float2bfloat16_rn(mok ? 1.f : 0.f);
-                const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
-                *reinterpret_cast<__nv_bfloat16*>(vt + ktab_off(2 * L.RP, rr)) = one;
-                for (int j = 2 * L.RP + 1; j < L.NV; ++j)
-                    *reinterpret_cast<__nv_bfloat16*>(vt + ktab_off(j, rr)) = zero;
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&vready[s]);
-            if constexpr (kDy) {
-                if (i >= 1) g_epilogue(i - 1);
-            }
+            mbar_arrive_remote(dsmem_addr(rbar, static_cast<uint32_t>(owner)));
         }
-        if constexpr (kDy) {
-            if (ok && nt >= 1) g_epilogue(nt - 1);
-        }
-        // this CTA's partial of column rr goes to the CTA that owns the column
-        cluster_wait();  // every CTA of the cluster has initialised its barriers
-        const int owner = rr / per;
-        const uint32_t dst = dsmem_addr(recv + (crank * per + rr - owner * per) * L.JP,
-                                        static_cast<uint32_t>(owner));
-        if (ok && nt > 0) ok = __all_sync(0xffffffffu, mbar_wait(dfull, 0, status));
-        if (ok && nt > 0) {
-            tc_fence_after();
-            const uint32_t base = tmem + lane_base + L.d_col;
-            for (int c0 = 0; c0 < L.RP; c0 += 16) {
-                uint32_t hi[16], lo[16];
-                tmem_ld16(base + c0, hi);
-                tmem_ld16(base + L.RP + c0, lo);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    if (c0 + e < a.r)
-                        dsmem_st(dst + 4 * (c0 + e), __uint_as_float(hi[e]) + __uint_as_float(lo[e]));
-            }
-            if constexpr (kDy) {
-                uint32_t ones[16];
-                tmem_ld16(base + 2 * L.RP, ones);
-                tmem_ld_wait();
-                dsmem_st(dst + 4 * a.r, __uint_as_float(ones[0]));
-            }
-        } else {
-            for (int j = 0; j < L.JP; ++j) dsmem_st(dst + 4 * j, 0.f);
-        }
-        mbar_arrive_remote(dsmem_addr(rbar, static_cast<uint32_t>(owner)));
         __syncwarp();
     }
     tc_fence_before();
@@ -359,38 +383,40 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
         tc_fence_after();
         tmem_dealloc(tmem, L.tmem_cols);
     }
-
-    // this CTA's slice of the columns: the CL partials added in rank order.
-    // Once every CTA's partials have arrived nothing reads or writes this
-    // CTA's shared memory from outside, so it may exit without a cluster barrier.
-    const int width = cend - cbeg;
-    const bool got = mbar_wait_cluster(rbar, 0, status);
-    if (got && width > 0) {
-        for (int idx = threadIdx.x; idx < L.JP * width; idx += kThreads) {
-            int j, cc;
-            if constexpr (kDy) {  // dB is [r, C]: consecutive threads take consecutive columns
-                j = idx / width;
-                cc = idx % width;
-            } else {              // dA is [C, r]: consecutive threads take consecutive ranks
-                cc = idx / L.JP;
-                j = idx % L.JP;
-            }
-            const int col = col0 + cbeg + cc;
-            if (col >= a.C) continue;
-            if (kDy && j == a.r && a.dbias == nullptr) continue;
-            float sum = 0.f;
-            for (int q = 0; q < CL; ++q) sum += recv[(q * per + cc) * L.JP + j];
-            if constexpr (kDy) {
-                if (j < a.r) a.out[static_cast<size_t>(j) * a.C + col] = a.c * sum;
-                else a.dbias[col] = sum;
-            } else {
-                a.out[static_cast<size_t>(col) * a.r + j] = a.c * sum;
+    if constexpr (kD) {
+        // this CTA's slice of the columns: the CL partials added in rank order.
+        // Once every CTA's partials have arrived nothing reads or writes this
+        // CTA's shared memory from outside, so it may exit without a cluster
+        // barrier.
+        const int width = cend - cbeg;
+        const bool got = mbar_wait_cluster(rbar, 0, status);
+        if (got && width > 0) {
+            for (int idx = threadIdx.x; idx < L.JP * width; idx += kThreads) {
+                int j, cc;
+                if constexpr (kOnes) {  // dB is [r, C]: consecutive threads take consecutive columns
+                    j = idx / width;
+                    cc = idx % width;
+                } else {                // dA is [C, r]: consecutive threads take consecutive ranks
+                    cc = idx / L.JP;
+                    j = idx % L.JP;
+                }
+                const int col = col0 + cbeg + cc;
+                if (col >= a.C) continue;
+                if (kOnes && j == a.r && a.dbias == nullptr) continue;
+                float sum = 0.f;
+                for (int q = 0; q < static_cast<int>(CL); ++q) sum += recv[(q * per + cc) * L.JP + j];
+                if constexpr (kOnes) {
+                    if (j < a.r) a.out[static_cast<size_t>(j) * a.C + col] = a.c * sum;
+                    else a.dbias[col] = sum;
+                } else {
+                    a.out[static_cast<size_t>(col) * a.r + j] = a.c * sum;
+                }
             }
         }
     }
 }
 
-template <bool kDy>
+template <bool kG, bool kD, bool kOnes>
 cudaError_t launch_tc(const void* T, RankTcArgs a, int* status, cudaStream_t s) {
     // T as [row][64-column block][64] when its rows split into whole blocks
     // (one box per tile), else one 2-D box per 64-column block
@@ -403,19 +429,32 @@ cudaError_t launch_tc(const void* T, RankTcArgs a, int* status, cudaStream_t s) 
                            static_cast<uint64_t>(a.C) * 2, kTileRows, kBoxCols,
                            CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return cudaErrorInvalidValue;
-    const RtLayout L(kDy, a.r);
+    const RtLayout L(Parts{kG, kD, kOnes}, a.r);
     const size_t smem = L.total + 1024;
-    auto kern = k4_rank_tc_kernel<kDy>;
+    auto kern = k4_rank_tc_kernel<kG, kD, kOnes>;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    // rows split over a cluster of CL CTAs, every CTA at least one tile;
-    // CTAs too large for two per SM take clusters of at most 4 (clusters of
-    // 8 single-CTA SMs do not all fit one wave of the GPCs)
-    const int max_cl = smem > 110 * 1024 ? 4 : kMaxCluster;
     const int mtiles = (a.M + kTileRows - 1) / kTileRows;
-    a.tiles_per_cta = (mtiles + max_cl - 1) / max_cl;
-    const int cl = (mtiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
-    const dim3 grid((a.C + kTileCols - 1) / kTileCols, cl);
+    int cl = 1;
+    int rows_grid;
+    if (kD) {
+        // rows split over a cluster of CL CTAs, every CTA at least one tile;
+        // CTAs too large for two per SM take clusters of at most 4 (clusters
+        // of 8 single-CTA SMs do not all fit one wave of the GPCs)
+        const int max_cl = smem > 110 * 1024 ? 4 : kMaxCluster;
+        a.tiles_per_cta = (mtiles + max_cl - 1) / max_cl;
+        cl = (mtiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
+        rows_grid = cl;
+    } else {
+        // G alone needs no reduction over rows: one 128-row tile per CTA,
+        // unless that makes more than a few waves of CTAs
+        const long long cbs = (a.C + kTileCols - 1) / kTileCols;
+        a.tiles_per_cta = 1;
+        while (cbs * ((mtiles + a.tiles_per_cta - 1) / a.tiles_per_cta) > 4LL * sm_count())
+            a.tiles_per_cta *= 2;
+        rows_grid = (mtiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
+    }
+    const dim3 grid((a.C + kTileCols - 1) / kTileCols, rows_grid);
     return launch_k(kern, grid, dim3(kThreads), smem, s, cl, tm, t3d, a, status);
 }
 
@@ -437,7 +476,10 @@ cudaError_t launch_rank_dy_tc(const void* dY, const float* B, const float* xA, i
     a.C = N;
     a.r = r;
     a.c = c;
-    return launch_tc<true>(dY, a, status, s);
+    if (Gp && dB) return launch_tc<true, true, true>(dY, a, status, s);
+    if (Gp) return launch_tc<true, false, false>(dY, a, status, s);
+    if (dB) return launch_tc<false, true, true>(dY, a, status, s);
+    return cudaSuccess;
 }
 
 cudaError_t launch_rank_x_tc(const void* X, const float* G, int nsl, int M, int K, int r, float c,
@@ -450,7 +492,7 @@ cudaError_t launch_rank_x_tc(const void* X, const float* G, int nsl, int M, int 
     a.C = K;
     a.r = r;
     a.c = c;
-    return launch_tc<false>(X, a, status, s);
+    return launch_tc<false, true, false>(X, a, status, s);
 }
 
 }  // namespace qlora

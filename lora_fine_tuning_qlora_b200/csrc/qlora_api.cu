@@ -371,6 +371,54 @@ int qlora_lora_grad_dy(const qlora_layer_desc* d, int M, const void* dY, const f
     return rc;
 }
 
+int qlora_lora_g(const qlora_layer_desc* d, int M, const void* dY, const float* B,
+                 void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_layer(d, M);
+    if (rc != QLORA_OK) return rc;
+    QL_REQUIRE(dY && B && workspace, QLORA_EINVAL, "NULL pointer argument");
+    QL_REQUIRE(aligned(dY, 16) && aligned(workspace, 256), QLORA_EALIGN,
+               "dY must be 16-byte aligned, workspace 256-byte aligned");
+    QL_REQUIRE(aligned(B, 4), QLORA_EALIGN, "fp32 vectors must be 4-byte aligned");
+    if (M == 0) return QLORA_OK;
+    const WsLayout w = layout_for(*d, M);
+    QL_REQUIRE(workspace_bytes >= w.total, QLORA_EINVAL, "workspace too small");
+    int* status = status_ptr();
+    QL_REQUIRE(status, QLORA_ECUDA, "no CUDA device");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float* gp = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.gp);
+    rc = cuda_status(launch_rank_dy(act_of(d), dY, B, nullptr, M, d->N, d->r, lora_scale(d), gp,
+                                    nullptr, nullptr, status, s),
+                     "G pass launch");
+    if (rc == QLORA_OK && w.reduce)
+        rc = cuda_status(launch_g_reduce(gp, w.ncb, M, d->r,
+                                         reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.g),
+                                         s),
+                         "G reduction launch");
+    return rc;
+}
+
+int qlora_lora_grad_b(const qlora_layer_desc* d, int M, const void* dY, const float* xA,
+                      float* dB, float* dbias, void* stream) {
+    int rc = check_layer(d, M);
+    if (rc != QLORA_OK) return rc;
+    QL_REQUIRE(dY && xA && dB, QLORA_EINVAL, "NULL pointer argument");
+    QL_REQUIRE(aligned(dY, 16), QLORA_EALIGN, "dY must be 16-byte aligned");
+    QL_REQUIRE(aligned(xA, 4) && aligned(dB, 4) && (!dbias || aligned(dbias, 4)), QLORA_EALIGN,
+               "fp32 vectors must be 4-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M == 0) {
+        rc = cuda_status(cudaMemsetAsync(dB, 0, sizeof(float) * d->r * d->N, s), "memset dB");
+        if (rc == QLORA_OK && dbias)
+            rc = cuda_status(cudaMemsetAsync(dbias, 0, sizeof(float) * d->N, s), "memset dbias");
+        return rc;
+    }
+    int* status = status_ptr();
+    QL_REQUIRE(status, QLORA_ECUDA, "no CUDA device");
+    return cuda_status(launch_rank_dy(act_of(d), dY, nullptr, xA, M, d->N, d->r, lora_scale(d),
+                                      nullptr, dB, dbias, status, s),
+                       "dB pass launch");
+}
+
 int qlora_gemm_dx(const qlora_layer_desc* d, int M, const void* dY, const int8_t* Wq,
                   const float* sw, const float* A, void* dX, const void* workspace,
                   size_t workspace_bytes, void* stream) {

@@ -30,7 +30,8 @@ EXPORTED = ("qlora_quantize_weight", "qlora_workspace_bytes", "qlora_forward",
             "qlora_backward", "qlora_merge", "qlora_last_error", "qlora_device_status",
             "qlora_version", "qlora_relu", "qlora_relu_backward", "qlora_quantize_input",
             "qlora_gemm_forward", "qlora_lora_grad_dy", "qlora_gemm_dx", "qlora_lora_grad_x",
-            "qlora_selftest_wait_timeout", "qlora_backward_noalloc")
+            "qlora_selftest_wait_timeout", "qlora_backward_noalloc", "qlora_lora_g",
+            "qlora_lora_grad_b")
 
 
 class QLoraError(RuntimeError):
@@ -82,10 +83,12 @@ def _load():
     lib.qlora_quantize_input.argtypes = [D, I, P, P, P, P, P, P]
     lib.qlora_gemm_forward.argtypes = [D, I, P, P, P, P, P, P, P, P, P, P]
     lib.qlora_lora_grad_dy.argtypes = [D, I, P, P, P, P, P, P, P, Z, P]
+    lib.qlora_lora_g.argtypes = [D, I, P, P, P, Z, P]
+    lib.qlora_lora_grad_b.argtypes = [D, I, P, P, P, P, P]
     lib.qlora_gemm_dx.argtypes = [D, I, P, P, P, P, P, P, Z, P]
     lib.qlora_lora_grad_x.argtypes = [D, I, P, P, P, Z, P]
     for f in (lib.qlora_quantize_input, lib.qlora_gemm_forward, lib.qlora_lora_grad_dy,
-              lib.qlora_gemm_dx, lib.qlora_lora_grad_x):
+              lib.qlora_lora_g, lib.qlora_lora_grad_b, lib.qlora_gemm_dx, lib.qlora_lora_grad_x):
         f.restype = I
     lib.qlora_selftest_wait_timeout.argtypes = [ctypes.c_uint, P]
     lib.qlora_selftest_wait_timeout.restype = I
@@ -204,6 +207,18 @@ def qlora_lora_grad_dy(d: LayerDesc, M: int, dY, B, xA, dB, dbias, ws, G=None, s
     writes the summed G too when a tensor is given)."""
     _check(_lib.qlora_lora_grad_dy(ctypes.byref(d), int(M), _ptr(dY), _ptr(B), _ptr(xA), _ptr(dB),
                                    _ptr(dbias), _ptr(G), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def qlora_lora_g(d: LayerDesc, M: int, dY, B, ws, stream=None):
+    """G = dY B^T into `ws` (the first half of qlora_lora_grad_dy)."""
+    _check(_lib.qlora_lora_g(ctypes.byref(d), int(M), _ptr(dY), _ptr(B), _ptr(ws), ws.numel(),
+                             _stream(stream)))
+
+
+def qlora_lora_grad_b(d: LayerDesc, M: int, dY, xA, dB, dbias, stream=None):
+    """dB and dbias (the second half of qlora_lora_grad_dy)."""
+    _check(_lib.qlora_lora_grad_b(ctypes.byref(d), int(M), _ptr(dY), _ptr(xA), _ptr(dB),
+                                  _ptr(dbias), _stream(stream)))
 
 
 def qlora_gemm_dx(d: LayerDesc, M: int, dY, Wq, sw, A, dX, ws, stream=None):

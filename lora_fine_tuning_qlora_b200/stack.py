@@ -30,9 +30,9 @@ class MLPStack:
         need = max(qlora.qlora_workspace_bytes(L.desc(), batch) for L in layers)
         self.ws = torch.empty(need, dtype=torch.uint8, device=dev)
         self.ws_alt = torch.empty(need, dtype=torch.uint8, device=dev)
-        # the X pass (dA) feeds nothing in the backward but the final gradient,
-        # so it runs on a side stream, overlapping the next layers' dY passes
-        # and dX GEMMs, which carry the critical path
+        # only G feeds the next layer's gradient: the G pass and the dX GEMM
+        # carry the critical path, while each layer's dB/dbias pass and X pass
+        # (dA) run on a side stream, overlapping the next layers
         self.side = torch.cuda.Stream(device=dev)
         self.ev_g = [torch.cuda.Event() for _ in layers]  # layer's G is in its workspace
         self.ev_x = [torch.cuda.Event() for _ in layers]  # layer's X pass is done
@@ -83,8 +83,8 @@ class MLPStack:
             n += 2                                   # quantize+xA, int8 GEMM
             n += 1 if i < len(self.layers) - 1 else 0  # ReLU
             rj = (L.r + 7) // 8                      # CUDA-core passes: 8 ranks per launch
-            dy_tc = bf16 and L.N % 8 == 0            # tensor-core dY pass, 128-column blocks
-            n += 1 if dy_tc else rj                  # dY pass
+            dy_tc = bf16 and L.N % 8 == 0            # tensor-core dY passes, 128-column blocks
+            n += 2 if dy_tc else 2 * rj              # G pass + dB/dbias pass
             ncb = -(-L.N // 128) if dy_tc else -(-L.N // 64)
             n += 1 if ncb > 8 else 0                 # G slices added once
             n += 1                                   # dX GEMM
@@ -126,8 +126,7 @@ class MLPStack:
             dX = self.dX if i == 0 else self.G[i - 1]
             if i + 2 < n:
                 main.wait_event(self.ev_x[i + 2])  # the X pass that read this workspace
-            qlora.qlora_lora_grad_dy(D[i], M, g, L.B, self.xA[i], self.dB[i], self.dbias[i],
-                                     ws, None, main)
+            qlora.qlora_lora_g(D[i], M, g, L.B, ws, main)
             self.ev_g[i].record(main)
             if ev_d and ev_d[i]:
                 ev_d[i][0].record(main)
@@ -135,6 +134,7 @@ class MLPStack:
             if ev_d and ev_d[i]:
                 ev_d[i][1].record(main)
             self.side.wait_event(self.ev_g[i])
+            qlora.qlora_lora_grad_b(D[i], M, g, self.xA[i], self.dB[i], self.dbias[i], self.side)
             qlora.qlora_lora_grad_x(D[i], M, x_in, self.dA[i], ws, self.side)
             self.ev_x[i].record(self.side)
             g = dX

@@ -237,6 +237,54 @@ def test_step_level_calls_match_composite(q):
     assert_close(to_np(G), G_ref, "bf16", "G")
 
 
+@pytest.mark.parametrize("M,K,N,r,act", [(200, 384, 264, 8, "bf16"), (333, 784, 1024, 4, "bf16"),
+                                          (96, 256, 10, 8, "bf16"), (64, 784, 128, 4, "f32"),
+                                          (70, 128, 2304, 16, "bf16")])
+def test_split_dy_pass_matches_grad_dy(q, M, K, N, r, act):
+    """qlora_lora_g followed by qlora_lora_grad_b (on another stream) gives
+    the results of qlora_lora_grad_dy: the same dB and dbias, and a
+    workspace from which a4 and a5 give the same dX and dA; dB, dA and G
+    also against the oracle."""
+    spec = _edge_spec(M, K, N, r, act=act, seed=M + N)
+    d = inputs.layer_inputs(spec)
+    from parity import device_layer, act_torch
+    layer = device_layer(spec, d, q)
+    tdt = act_torch(act)
+    X = torch.from_numpy(d["X"]).to(tdt).cuda()
+    dY = torch.from_numpy(d["dY"]).to(tdt).cuda()
+    D = layer.desc()
+    ws1 = q.workspace(D, M)
+    ws2 = q.workspace(D, M)
+    _, xA = q.forward(layer, X, ws1)
+    dB1 = torch.empty((r, N), device="cuda"); db1 = torch.empty((N,), device="cuda")
+    q.qlora_lora_grad_dy(D, M, dY, layer.B, xA, dB1, db1, ws1)
+    dB2 = torch.full((r, N), float("nan"), device="cuda")
+    db2 = torch.full((N,), float("nan"), device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    q.qlora_lora_g(D, M, dY, layer.B, ws2)
+    with torch.cuda.stream(side):
+        q.qlora_lora_grad_b(D, M, dY, xA, dB2, db2, side)
+    torch.cuda.current_stream().wait_stream(side)
+    outs = []
+    for ws in (ws1, ws2):
+        dX = torch.empty((M, K), dtype=tdt, device="cuda")
+        dA = torch.empty((K, r), device="cuda")
+        q.qlora_gemm_dx(D, M, dY, layer.Wq, layer.sw, layer.A, dX, ws)
+        q.qlora_lora_grad_x(D, M, X, dA, ws)
+        outs.append((dX, dA))
+    torch.cuda.synchronize()
+    assert q.qlora_device_status() == 0
+    assert torch.equal(dB1, dB2) and torch.equal(db1, db2)
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    ref = oracle.backward(oracle.to_act(d["X"], act), oracle.to_act(d["dY"], act),
+                          *oracle.quantize_weight(d["W"]), d["A"], d["B"], spec.alpha,
+                          want_dx=False, act=act)
+    assert_close(to_np(dB2), ref["dB"], act, "dB")
+    assert_close(to_np(db2), ref["dbias"], act, "dbias")
+    assert_close(to_np(outs[1][1]), ref["dA"], act, "dA")
+
+
 def test_relu_kernels(q):
     """The stack's elementwise ReLU and its backward, aligned and unaligned."""
     rng = np.random.Generator(np.random.PCG64(21))
