@@ -32,13 +32,17 @@ namespace {
 
 constexpr int kBlkN = 64;  // one 128-byte swizzle row of bf16: the dY block a 2-D box covers
 constexpr int kDqWarps = 8;
-constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * (kDqWarps + kEpiWarps);
 constexpr int kSmemLimit = 232448;
 
 template <int MSUB, int BN, int RMAX>
 struct K3Cfg {
     static constexpr int kBM = 128 * MSUB;
+    // epilogue warps: two per TMEM lane quarter (row sub-tiles, or column
+    // halves), one for the 128 x 64 tiles, whose four extra MMA issuers would
+    // otherwise leave too few registers per thread
+    static constexpr int kEpiWarps = (MSUB == 1 && BN == 64) ? 4 : 8;
+    static constexpr int kEpiPerQuarter = kEpiWarps / 4;
+    static_assert(MSUB == 1 || kEpiWarps == 8, "one epilogue warp pair per row sub-tile");
     // contraction (n) per stage: 128 (two 64-column dY blocks in one 3-D TMA
     // box), 64 for the 256-row tiles so that two stages fit
     static constexpr int kBKn = MSUB == 2 ? 64 : 128;
@@ -64,9 +68,20 @@ struct K3Cfg {
     static constexpr int kTabOff = kStgOff + kStgBytes;
     static constexpr int kBarOff = kTabOff + kParamBytes;
     static constexpr int kTotal = kBarOff + 512 + 1024;
-    static constexpr uint32_t kAccCols = MSUB * BN;     // one accumulator buffer
-    static constexpr uint32_t kTmemCols = 2 * kAccCols;
+    // A tcgen05.mma holds its issuing thread ~0.1 us whatever its N, so the
+    // contraction of a tile is split over kChains MMA-issuing warps, each with
+    // its own TMEM accumulator (added in chain order by the epilogue); two
+    // tile buffers of kChains accumulators fill the 512 TMEM columns.
+    static constexpr int kChains = (MSUB == 1 && BN == 64) ? 4 : (MSUB == 1 ? 2 : 1);
+    static constexpr uint32_t kAccCols = MSUB * BN;             // one chain's accumulator
+    static constexpr uint32_t kBufCols = kChains * kAccCols;    // one tile buffer
+    static constexpr uint32_t kTmemCols = 2 * kBufCols;
     static_assert(kTmemCols <= 512, "TMEM");
+    static_assert((kBKn / 16) % kChains == 0, "k-steps per chain");
+    // warps: producer, kChains MMA issuers, de-quantize, epilogue
+    static constexpr int kDqWarp0 = 1 + kChains;
+    static constexpr int kEpiWarp0 = kDqWarp0 + kDqWarps;
+    static constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 };
 
 // byte offset of the 16-byte chunk holding bf16 elements (mn .. mn+7, kr) in
@@ -127,7 +142,7 @@ __device__ __forceinline__ void dequant16(const uint4 raw, float scale, uint32_t
 }
 
 template <int MSUB, int BN, int RMAX>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
     k3_dx_dequant_kernel(const __grid_constant__ CUtensorMap tmDY, int dy3d,
                          const int8_t* __restrict__ Wq, const float* __restrict__ sw, int M, int N,
                          int K, DxEpilogue ep, int* status) {
@@ -158,12 +173,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&wready[s], kDqWarps);  // every de-quantize warp, once per fill
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], C::kChains);  // every MMA issuer, once per use
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], kEpiWarps);
-            mbar_init(&lready[b], kEpiWarps);
+            mbar_init(&tfull[b], C::kChains);
+            mbar_init(&tempty[b], C::kEpiWarps);
+            mbar_init(&lready[b], C::kEpiWarps);
         }
         fence_mbar_init();
     }
@@ -210,8 +225,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------ MMA issuer
+    } else if (warp < C::kDqWarp0) {
+        // ------------------------------------------------------ MMA issuers
+        // issuer ch takes the k-steps ch, ch + kChains, ... of every stage
+        // into its own accumulator; issuer 0 also adds the rank-r term
+        const int ch = warp - 1;
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16(128, BN, false, true);
             int g = 0, i = 0;
@@ -232,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t a_base = smem_u32(smem + s * C::kStageBytes);
                     const uint32_t w_base = a_base + C::kABytes;
 #pragma unroll
-                    for (int kk = 0; kk < kBKn / 16; ++kk) {
+                    for (int kk = ch; kk < kBKn / 16; kk += C::kChains) {
                         const uint64_t bd = smem_desc(w_base + kk * 2048, kLbo, 1024, kLayoutSw128);
 #pragma unroll
                         for (int ms = 0; ms < MSUB; ++ms) {
@@ -240,12 +258,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const uint64_t ad = smem_desc(
                                 a_base + ms * C::kASub + (kk >> 2) * (128 * kBlkN * 2) + (kk & 3) * 32, 16,
                                 1024, kLayoutSw128);
-                            mma_bf16(tmem + ab * C::kAccCols + ms * BN, ad, bd, idesc, (kb | kk) != 0);
+                            mma_bf16(tmem + ab * C::kBufCols + ch * C::kAccCols + ms * BN, ad, bd, idesc,
+                                     (kb > 0 || kk > ch) ? 1u : 0u);
                         }
                     }
                     mma_commit(&empty[s]);
                 }
-                if constexpr (C::kLoraMMA) {
+                if (C::kLoraMMA && ch == 0) {
                     // + (c G) A^T: tf32 MMAs from the tables the epilogue warps wrote
                     if (ok && !mbar_wait(&lready[ab], use & 1, status)) ok = false;
                     if (ok) {
@@ -261,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int ms = 0; ms < MSUB; ++ms) {
                                 const uint64_t ad =
                                     smem_desc(gt + ms * 16 * kSbo + ks * 256, 128, kSbo, kLayoutNone);
-                                mma_tf32(tmem + ab * C::kAccCols + ms * BN, ad, bd, tdesc, 1);
+                                mma_tf32(tmem + ab * C::kBufCols + ms * BN, ad, bd, tdesc, 1);
                             }
                         }
                     }
@@ -270,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp < 2 + kDqWarps) {
+    } else if (warp < C::kEpiWarp0) {
         // ------------------------------------------------------ de-quantize
         // All eight warps convert every stage, each its own slice of the
         // 16-byte chunks, walking the stages in order (so every barrier phase
@@ -279,32 +298,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ring slot u per ring stage u), so neither a TMA box nor a load
         // latency sits on the conversion path; a stage only waits for its
         // bf16 slot to be released by the MMAs that read it last.
-        const int dw = warp - 2;  // 0 .. 7
+        const int dw = warp - C::kDqWarp0;  // 0 .. 7
         constexpr int kChunksPerRow = BN / 16;
         constexpr int kChunks = kBKn * kChunksPerRow;
         constexpr int kPerLane = kChunks / (32 * kDqWarps);
         static_assert(kChunks % (32 * kDqWarps) == 0, "chunks per stage");
         const int my_tiles = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
         const int total_kb = my_tiles * nkb;
+        // The loads are unconditional, from addresses clamped into the
+        // matrices, and a chunk outside them is zeroed through its scale when
+        // it is converted: a select on a just-loaded register would make the
+        // warp wait out the load right here.
         uint4 qr[S][kPerLane];
         float sr[S][kPerLane];
-        auto fetch = [&](int g, uint4 (&q)[kPerLane], float (&sc)[kPerLane]) {
+        uint32_t inb[S];  // bit i: chunk i of the ring slot lies inside the matrices
+        auto fetch = [&](int g, uint4 (&q)[kPerLane], float (&sc)[kPerLane], uint32_t& in_bits) {
             const int t = blockIdx.x + (g / nkb) * gridDim.x;
             const int k0 = (t % num_k) * BN;
             const int kb = g % nkb;
+            in_bits = 0;
 #pragma unroll
             for (int i = 0; i < kPerLane; ++i) {
                 const int c = dw * 32 + lane + i * 32 * kDqWarps;
                 const int n = kb * kBKn + c / kChunksPerRow;
                 const int k = k0 + (c % kChunksPerRow) * 16;
-                const bool in = g < total_kb && n < N && k < K;
-                q[i] = in ? __ldg(reinterpret_cast<const uint4*>(Wq + static_cast<size_t>(n) * K + k))
-                          : make_uint4(0u, 0u, 0u, 0u);
-                sc[i] = in ? __ldg(sw + n) : 0.f;
+                if (g < total_kb && n < N && k < K) in_bits |= 1u << i;
+                const int nc = n < N ? n : N - 1;
+                const int kc = k < K ? k : K - 16;
+                q[i] = __ldg(reinterpret_cast<const uint4*>(Wq + static_cast<size_t>(nc) * K + kc));
+                sc[i] = __ldg(sw + nc);
             }
         };
 #pragma unroll
-        for (int u = 0; u < S; ++u) fetch(u, qr[u], sr[u]);
+        for (int u = 0; u < S; ++u) fetch(u, qr[u], sr[u], inb[u]);
         bool live = true;
         for (int g0 = 0; g0 < total_kb && live; g0 += S) {
 #pragma unroll
@@ -323,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int nr = c / kChunksPerRow;   // contraction row within the stage
                     const int kc = c % kChunksPerRow;   // 16 output columns
                     uint32_t o[8];
-                    dequant16(qr[u][i], sr[u][i], o);
+                    dequant16(qr[u][i], (inb[u] >> i) & 1u ? sr[u][i] : 0.f, o);
                     const int mn = kc * 16;
                     *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn, nr, kLbo)) =
                         make_uint4(o[0], o[1], o[2], o[3]);
@@ -333,16 +359,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&wready[u]);
-                fetch(g + S, qr[u], sr[u]);
+                fetch(g + S, qr[u], sr[u], inb[u]);
             }
         }
         __syncwarp();
     } else {
         // ------------------------------------------------------ epilogue
-        const int ew = warp - 2 - kDqWarps;  // 0 .. 7
+        const int ew = warp - C::kEpiWarp0;  // 0 .. 7
         const int q = warp & 3;              // TMEM lane quarter of this warp
-        const int sub = ew >> 2;             // MSUB == 2: row sub-tile, else column half
-        const int et = threadIdx.x - 64 - 32 * kDqWarps;
+        const int sub = ew >> 2;             // MSUB == 2: row sub-tile, else column part
+        const int et = threadIdx.x - 32 * C::kEpiWarp0;
         uint8_t* stg = smem + C::kStgOff + ew * 32 * stage_pitch<__nv_bfloat16>();
         __nv_bfloat16* dX = static_cast<__nv_bfloat16*>(ep.dX);
         int i = 0;
@@ -356,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // c*G rows m0.. and A rows k0.. (zero outside the matrices)
                 uint8_t* gt = tabs + ab * (C::kGtBytes + C::kAtBytes);
                 uint8_t* at = gt + C::kGtBytes;
-                for (int e = et; e < C::kBM * C::kKL; e += 32 * kEpiWarps) {
+                for (int e = et; e < C::kBM * C::kKL; e += 32 * C::kEpiWarps) {
                     const int rr = e / C::kKL, j = e % C::kKL;
                     const int m = m0 + rr;
                     const float g = (m < M && j < ep.r) ? g_row(ep, M, m, j) * ep.c : 0.f;
@@ -364,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tf32_split(g, hi, lo);
                     *reinterpret_cast<float*>(gt + kmajor_tf32_offset(rr, j, C::kKL)) = hi;
                 }
-                for (int e = et; e < BN * C::kKL; e += 32 * kEpiWarps) {
+                for (int e = et; e < BN * C::kKL; e += 32 * C::kEpiWarps) {
                     const int cc = e / C::kKL, j = e % C::kKL;
                     const int k = k0 + cc;
                     const float a = (k < K && j < ep.r) ? ep.A[static_cast<size_t>(k) * ep.r + j] : 0.f;
@@ -389,20 +415,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[ab], use & 1, status));
             if (!ok) break;
             tc_fence_after();
-            const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * C::kAccCols +
+            const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * C::kBufCols +
                                    msub * BN;
-            const int cbeg = MSUB == 2 ? 0 : sub * (BN / 2);
-            const int cend = MSUB == 2 ? BN : (sub + 1) * (BN / 2);
+            const int cbeg = MSUB == 2 ? 0 : sub * (BN / C::kEpiPerQuarter);
+            const int cend = MSUB == 2 ? BN : (sub + 1) * (BN / C::kEpiPerQuarter);
 #pragma unroll 1
             for (int col = cbeg; col < cend; col += kEpiCols) {
+                // the chains' partial sums, added in chain order
                 uint32_t v[kEpiCols];
+                float part[kEpiCols];
                 tmem_ld16(tbase + col, v);
                 tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < kEpiCols; ++e) part[e] = __uint_as_float(v[e]);
+#pragma unroll
+                for (int ch = 1; ch < C::kChains; ++ch) {
+                    tmem_ld16(tbase + ch * C::kAccCols + col, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < kEpiCols; ++e) part[e] += __uint_as_float(v[e]);
+                }
                 float y[kEpiCols];
 #pragma unroll
                 for (int e = 0; e < kEpiCols; ++e) {
                     const int c = col + e;
-                    float acc = __uint_as_float(v[e]);
+                    float acc = part[e];
                     if constexpr (!C::kLoraMMA) {
                         const int k = k0 + c;
                         if (k < K)
@@ -447,7 +484,7 @@ cudaError_t launch_tc(const void* dY, const int8_t* Wq, const float* sw, int M, 
     if (!ok) return cudaErrorInvalidValue;
     const int tiles = ((M + C::kBM - 1) / C::kBM) * ((K + BN - 1) / BN);
     const int grid = tiles < sm_count() ? tiles : sm_count();
-    return launch_k(kern, dim3(grid), dim3(kThreads), C::kTotal, s, 1, tdy, dy3d, Wq, sw, M, N, K, ep,
+    return launch_k(kern, dim3(grid), dim3(C::kThreads), C::kTotal, s, 1, tdy, dy3d, Wq, sw, M, N, K, ep,
                     status);
 }
 
