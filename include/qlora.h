@@ -201,6 +201,16 @@ int qlora_gemm_forward(const qlora_layer_desc* d, int M, const int8_t* Xq, const
                        const int8_t* Wq, const float* sw, const float* bias, const float* xA,
                        const float* B, void* Y, int32_t* acc, void* stream);
 
+/* a2 for a layer followed by a ReLU, as the hidden layers of the MLP in
+ * "Introduce QLoRA-like technique" (benchmark script: Dense layers with ReLU
+ * between them; the ReLU is not part of the layer): the same Y, then
+ * Y = max(Y, 0) in the epilogue, bit-identical to qlora_gemm_forward followed
+ * by qlora_relu, without the second pass over Y.  acc, if not NULL, still
+ * receives the raw accumulator. */
+int qlora_gemm_forward_relu(const qlora_layer_desc* d, int M, const int8_t* Xq, const float* sx,
+                            const int8_t* Wq, const float* sw, const float* bias, const float* xA,
+                            const float* B, void* Y, int32_t* acc, void* stream);
+
 /* a3: one pass over dY: dB = c * xA^T dY [r,N] and, if dbias is not NULL,
  * dbias = column sums of dY [N]; G = dY B^T is left in the workspace (as
  * per-column-block slices) for the a4 and a5 calls that follow on the same
@@ -230,6 +240,14 @@ int qlora_lora_grad_b(const qlora_layer_desc* d, int M, const void* dY, const fl
 int qlora_gemm_dx(const qlora_layer_desc* d, int M, const void* dY, const int8_t* Wq,
                   const float* sw, const float* A, void* dX, const void* workspace,
                   size_t workspace_bytes, void* stream);
+
+/* a4 for a layer whose input X [M,K] (act_dtype, 16-byte aligned) is the
+ * output of a ReLU: dX is taken back through that ReLU as well, dX = 0 where
+ * X <= 0, in the epilogue; bit-identical to qlora_gemm_dx followed by
+ * qlora_relu_backward(dX, X), without the second pass over dX. */
+int qlora_gemm_dx_relu(const qlora_layer_desc* d, int M, const void* dY, const int8_t* Wq,
+                       const float* sw, const float* A, const void* X, void* dX,
+                       const void* workspace, size_t workspace_bytes, void* stream);
 
 /* a5: one pass over X: dA = c * X^T G [K,r], G from the workspace that a3
  * filled.  Deterministic. */

@@ -30,6 +30,7 @@ struct FwdEpilogue {
     float c;
     void* Y;            // [M,N] act
     int32_t* acc;       // [M,N] debug copy or null
+    int relu;           // 1: Y = max(Y, 0) (the ReLU that follows the layer in an MLP)
 };
 // Y = (Xq Wq^T) sx sw + bias + c xA B with the tcgen05 int8 GEMM.
 cudaError_t launch_gemm_i8_fwd(Act act, const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
@@ -43,6 +44,8 @@ struct DxEpilogue {
     int r;
     float c;
     void* dX;         // [M,K] act
+    const void* gate; // [M,K] act or null: dX = 0 where gate <= 0 (the layer input came
+                      // out of a ReLU, whose backward this applies)
 };
 // dX = dY (Wq sw)^T + c G A^T.  tcgen05 bf16 path when possible, else SIMT.
 cudaError_t launch_gemm_dx(Act act, const void* dY, const int8_t* Wq, const float* sw, int M,

@@ -32,7 +32,7 @@ namespace qlora {
 namespace {
 
 constexpr int kBM = 128;
-constexpr int kBK = 128;  // int8 elements per k-block: one 128-byte swizzle row
+constexpr int kBlkK = 128;        // int8 elements per 128-byte swizzle row (one TMA block)
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory
@@ -46,11 +46,15 @@ struct K2Cfg {
     static constexpr int kXtBytes = kLoraMMA ? kBM * kKL * 4 : 0;
     static constexpr int kBtBytes = kLoraMMA ? BN * kKL * 4 : 0;
     static constexpr int kBufBytes = kTerms * (kXtBytes + kBtBytes) + BN * 4 * 2;  // + sw, bias
+    static constexpr int kStgBytes = kEpiWarps * 32 * stage_pitch<OutT>();
+    static constexpr int kFixed = kStgBytes + 2 * kBufBytes + 512 + 1024;
+    // k per stage: two 128-byte blocks (one 3-D TMA box per operand) where
+    // two such stages fit, else one
+    static constexpr int kBlk = (kSmemLimit - kFixed) / ((kBM + BN) * 2 * kBlkK) >= 2 ? 2 : 1;
+    static constexpr int kBK = kBlk * kBlkK;
     static constexpr int kABytes = kBM * kBK;
     static constexpr int kBBytes = BN * kBK;
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kStgBytes = kEpiWarps * 32 * stage_pitch<OutT>();
-    static constexpr int kFixed = kStgBytes + 2 * kBufBytes + 512 + 1024;
     static constexpr int kStagesFit = (kSmemLimit - kFixed) / kStageBytes;
     static constexpr int STAGES = kStagesFit > 8 ? 8 : kStagesFit;
     static_assert(STAGES >= 2, "shared memory budget");
@@ -66,7 +70,7 @@ struct K2Cfg {
 template <int BN, typename OutT, int RMAX>
 __global__ void __launch_bounds__(kThreads, 1)
     k2_gemm_i8_lora_kernel(const __grid_constant__ CUtensorMap tmA,
-                           const __grid_constant__ CUtensorMap tmB, int M, int N, int K,
+                           const __grid_constant__ CUtensorMap tmB, int k3d, int M, int N, int K,
                            FwdEpilogue ep, int* status) {
     using C = K2Cfg<BN, OutT, RMAX>;
     constexpr int S = C::STAGES;
@@ -84,7 +88,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lane = threadIdx.x % 32;
     const int num_n = (N + BN - 1) / BN;
     const int tiles = ((M + kBM - 1) / kBM) * num_n;
-    const int nkb = (K + kBK - 1) / kBK;
+    const int nkb = (K + C::kBK - 1) / C::kBK;
     pdl_trigger();
 
     if (threadIdx.x == 0) {
@@ -127,8 +131,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     uint8_t* sa = smem + s * C::kStageBytes;
                     mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-                    tma_load_2d(sa, &tmA, &full[s], kb * kBK, m0);
-                    tma_load_2d(sa + C::kABytes, &tmB, &full[s], kb * kBK, n0);
+                    // each operand's two k-blocks, consecutive in shared memory
+                    if (k3d) {
+                        tma_load_3d(sa, &tmA, &full[s], 0, m0, kb * C::kBlk);
+                        tma_load_3d(sa + C::kABytes, &tmB, &full[s], 0, n0, kb * C::kBlk);
+                    } else {
+#pragma unroll
+                        for (int b = 0; b < C::kBlk; ++b) {
+                            tma_load_2d(sa + b * (kBM * kBlkK), &tmA, &full[s], (kb * C::kBlk + b) * kBlkK,
+                                        m0);
+                            tma_load_2d(sa + C::kABytes + b * (BN * kBlkK), &tmB, &full[s],
+                                        (kb * C::kBlk + b) * kBlkK, n0);
+                        }
+                    }
                 }
             }
         }
@@ -155,9 +170,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t a_base = smem_u32(smem + s * C::kStageBytes);
                     const uint32_t b_base = a_base + C::kABytes;
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 32; ++kk) {
-                        const uint64_t ad = smem_desc(a_base + kk * 32, 16, 1024, kLayoutSw128);
-                        const uint64_t bd = smem_desc(b_base + kk * 32, 16, 1024, kLayoutSw128);
+                    for (int kk = 0; kk < C::kBK / 32; ++kk) {
+                        // 32-byte step kk: block kk / 4, 32 bytes per step within it
+                        const uint64_t ad = smem_desc(a_base + (kk >> 2) * (kBM * kBlkK) + (kk & 3) * 32, 16,
+                                                      1024, kLayoutSw128);
+                        const uint64_t bd = smem_desc(b_base + (kk >> 2) * (BN * kBlkK) + (kk & 3) * 32, 16,
+                                                      1024, kLayoutSw128);
                         mma_i8(dacc, ad, bd, idesc, (kb | kk) != 0);
                     }
                     mma_commit(&empty[s]);
@@ -298,6 +316,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
+                if (ep.relu) {
+#pragma unroll
+                    for (int e = 0; e < kEpiCols; ++e) y[e] = y[e] > 0.f ? y[e] : 0.f;
+                }
                 if (ep.acc && row_ok) {
                     for (int e = 0; e < kEpiCols; ++e)
                         if (n0 + col + e < N)
@@ -320,31 +342,46 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int BN, typename OutT, int RMAX>
-cudaError_t launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K,
+cudaError_t launch_cfg(const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
                        const FwdEpilogue& ep, int* status, cudaStream_t s) {
     using C = K2Cfg<BN, OutT, RMAX>;
+    // Xq and Wq as [row][k-block of 128][128] (one 3-D box per operand and
+    // stage) when K splits into whole blocks, else one 2-D box per block
+    CUtensorMap ta, tb;
+    const int k3d = (K % kBlkK) == 0 ? 1 : 0;
+    bool ok;
+    if (k3d)
+        ok = make_tmap_3d_blocks(&ta, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, kBlkK, kBM, C::kBlk) &&
+             make_tmap_3d_blocks(&tb, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, kBlkK, BN, C::kBlk);
+    else
+        ok = make_tmap_2d(&ta, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, K, kBM, kBlkK,
+                          CU_TENSOR_MAP_SWIZZLE_128B) &&
+             make_tmap_2d(&tb, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, BN, kBlkK,
+                          CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return cudaErrorInvalidValue;
     auto kern = k2_gemm_i8_lora_kernel<BN, OutT, RMAX>;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), C::kTotal);
     if (e != cudaSuccess) return e;
     const int tiles = ((M + kBM - 1) / kBM) * ((N + BN - 1) / BN);
     const int grid = tiles < sm_count() ? tiles : sm_count();
-    return launch_k(kern, dim3(grid), dim3(kThreads), C::kTotal, s, 1, ta, tb, M, N, K, ep, status);
+    return launch_k(kern, dim3(grid), dim3(kThreads), C::kTotal, s, 1, ta, tb, k3d, M, N, K, ep,
+                    status);
 }
 
 template <typename OutT, int RMAX>
-cudaError_t launch_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K,
+cudaError_t launch_bn(int bn, const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
                       const FwdEpilogue& ep, int* status, cudaStream_t s) {
-    if (bn == 128) return launch_cfg<128, OutT, RMAX>(ta, tb, M, N, K, ep, status, s);
-    return launch_cfg<64, OutT, RMAX>(ta, tb, M, N, K, ep, status, s);
+    if (bn == 128) return launch_cfg<128, OutT, RMAX>(Xq, Wq, M, N, K, ep, status, s);
+    return launch_cfg<64, OutT, RMAX>(Xq, Wq, M, N, K, ep, status, s);
 }
 
 template <typename OutT>
-cudaError_t launch_r(int bn, const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K,
+cudaError_t launch_r(int bn, const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
                      const FwdEpilogue& ep, int* status, cudaStream_t s) {
-    if (ep.r <= 4) return launch_bn<OutT, 4>(bn, ta, tb, M, N, K, ep, status, s);
-    if (ep.r <= 8) return launch_bn<OutT, 8>(bn, ta, tb, M, N, K, ep, status, s);
-    if (ep.r <= 16) return launch_bn<OutT, 16>(bn, ta, tb, M, N, K, ep, status, s);
-    return launch_bn<OutT, 64>(bn, ta, tb, M, N, K, ep, status, s);
+    if (ep.r <= 4) return launch_bn<OutT, 4>(bn, Xq, Wq, M, N, K, ep, status, s);
+    if (ep.r <= 8) return launch_bn<OutT, 8>(bn, Xq, Wq, M, N, K, ep, status, s);
+    if (ep.r <= 16) return launch_bn<OutT, 16>(bn, Xq, Wq, M, N, K, ep, status, s);
+    return launch_bn<OutT, 64>(bn, Xq, Wq, M, N, K, ep, status, s);
 }
 
 }  // namespace
@@ -356,15 +393,8 @@ cudaError_t launch_gemm_i8_fwd(Act act, const int8_t* Xq, const int8_t* Wq, int 
     int bn = mt * ((N + 127) / 128) >= sm_count() ? 128 : 64;
     const int forced = tile_override("QLORA_FWD_BN");  // tuning: 64 or 128
     if (forced == 64 || forced == 128) bn = forced;
-    CUtensorMap ta, tb;
-    if (!make_tmap_2d(&ta, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, K, kBM, kBK,
-                      CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
-    if (!make_tmap_2d(&tb, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, bn, kBK,
-                      CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
-    if (act == kBF16) return launch_r<__nv_bfloat16>(bn, ta, tb, M, N, K, ep, status, s);
-    return launch_r<float>(bn, ta, tb, M, N, K, ep, status, s);
+    if (act == kBF16) return launch_r<__nv_bfloat16>(bn, Xq, Wq, M, N, K, ep, status, s);
+    return launch_r<float>(bn, Xq, Wq, M, N, K, ep, status, s);
 }
 
 }  // namespace qlora

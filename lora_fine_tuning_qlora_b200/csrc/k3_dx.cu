@@ -448,6 +448,19 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
                     }
                     y[e] = acc;
                 }
+                if (ep.gate && row_ok && k0 + col < K) {
+                    // backward of the ReLU that produced this layer's input
+                    const uint4* gp = reinterpret_cast<const uint4*>(
+                        static_cast<const __nv_bfloat16*>(ep.gate) + static_cast<size_t>(row) * K + k0 + col);
+                    const uint4 g0 = __ldg(gp), g1 = __ldg(gp + 1);
+                    const __nv_bfloat16* gh0 = reinterpret_cast<const __nv_bfloat16*>(&g0);
+                    const __nv_bfloat16* gh1 = reinterpret_cast<const __nv_bfloat16*>(&g1);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        if (!(__bfloat162float(gh0[e]) > 0.f)) y[e] = 0.f;
+                        if (!(__bfloat162float(gh1[e]) > 0.f)) y[8 + e] = 0.f;
+                    }
+                }
                 store_block<__nv_bfloat16>(stg, y, lane, dX, static_cast<size_t>(K), row0, M, k0 + col,
                                            K, true);
             }
@@ -565,7 +578,9 @@ __global__ void __launch_bounds__(256) k3_dx_simt_kernel(const T* __restrict__ d
             float l = 0.f;
             for (int jj = 0; jj < ep.r; ++jj)
                 l = fmaf(sG[ty + 16 * i][jj], ep.A[static_cast<size_t>(k) * ep.r + jj], l);
-            dX[static_cast<size_t>(m) * K + k] = ActIO<T>::from_f(acc[i][j] + ep.c * l);
+            const bool pass =
+                !ep.gate || ActIO<T>::to_f(static_cast<const T*>(ep.gate)[static_cast<size_t>(m) * K + k]) > 0.f;
+            dX[static_cast<size_t>(m) * K + k] = ActIO<T>::from_f(pass ? acc[i][j] + ep.c * l : 0.f);
         }
     }
 }

@@ -255,16 +255,21 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
         if constexpr (kG) {
             // Bcat[j][n] = B[j, col0 + n] as head (rows 0..RP) and remainder (RP..2RP),
             // eight loads in flight per round
+            // (loads from clamped addresses first, the zeroing of entries
+            // outside B after them, so that no select waits on a single load)
             uint8_t* bt = smem + L.bcat;
             const int n = col0 + rr;
+            const int nc = n < a.C ? n : a.C - 1;
             for (int j0 = 0; j0 < L.RP; j0 += 8) {
                 float v[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    v[e] = (j0 + e < a.r && n < a.C) ? __ldg(a.B + static_cast<size_t>(j0 + e) * a.C + n)
-                                                     : 0.f;
+                for (int e = 0; e < 8; ++e) {
+                    const int jc = j0 + e < a.r ? j0 + e : a.r - 1;
+                    v[e] = __ldg(a.B + static_cast<size_t>(jc) * a.C + nc);
+                }
 #pragma unroll
-                for (int e = 0; e < 8; ++e) put_split(bt, j0 + e, L.RP + j0 + e, rr, v[e]);
+                for (int e = 0; e < 8; ++e)
+                    put_split(bt, j0 + e, L.RP + j0 + e, rr, (j0 + e < a.r && n < a.C) ? v[e] : 0.f);
             }
             if constexpr (!kD) {
                 // G alone: the MMAs of the first tile wait for this table on vready[0]

@@ -306,9 +306,10 @@ int qlora_quantize_input(const qlora_layer_desc* d, int M, const void* X, const 
                        "input quantizer launch");
 }
 
-int qlora_gemm_forward(const qlora_layer_desc* d, int M, const int8_t* Xq, const float* sx,
-                       const int8_t* Wq, const float* sw, const float* bias, const float* xA,
-                       const float* B, void* Y, int32_t* acc, void* stream) {
+static int gemm_forward_impl(const qlora_layer_desc* d, int M, const int8_t* Xq, const float* sx,
+                             const int8_t* Wq, const float* sw, const float* bias,
+                             const float* xA, const float* B, void* Y, int32_t* acc, int relu,
+                             void* stream) {
     int rc = check_layer(d, M);
     if (rc != QLORA_OK) return rc;
     QL_REQUIRE(Xq && sx && Wq && sw && xA && B && Y, QLORA_EINVAL, "NULL pointer argument");
@@ -330,9 +331,22 @@ int qlora_gemm_forward(const qlora_layer_desc* d, int M, const int8_t* Xq, const
     ep.c = lora_scale(d);
     ep.Y = Y;
     ep.acc = acc;
+    ep.relu = relu;
     return cuda_status(launch_gemm_i8_fwd(act_of(d), Xq, Wq, M, d->N, d->K, ep, status,
                                           static_cast<cudaStream_t>(stream)),
                        "int8 GEMM launch");
+}
+
+int qlora_gemm_forward(const qlora_layer_desc* d, int M, const int8_t* Xq, const float* sx,
+                       const int8_t* Wq, const float* sw, const float* bias, const float* xA,
+                       const float* B, void* Y, int32_t* acc, void* stream) {
+    return gemm_forward_impl(d, M, Xq, sx, Wq, sw, bias, xA, B, Y, acc, 0, stream);
+}
+
+int qlora_gemm_forward_relu(const qlora_layer_desc* d, int M, const int8_t* Xq, const float* sx,
+                            const int8_t* Wq, const float* sw, const float* bias, const float* xA,
+                            const float* B, void* Y, int32_t* acc, void* stream) {
+    return gemm_forward_impl(d, M, Xq, sx, Wq, sw, bias, xA, B, Y, acc, 1, stream);
 }
 
 int qlora_lora_grad_dy(const qlora_layer_desc* d, int M, const void* dY, const float* B,
@@ -419,15 +433,16 @@ int qlora_lora_grad_b(const qlora_layer_desc* d, int M, const void* dY, const fl
                        "dB pass launch");
 }
 
-int qlora_gemm_dx(const qlora_layer_desc* d, int M, const void* dY, const int8_t* Wq,
-                  const float* sw, const float* A, void* dX, const void* workspace,
-                  size_t workspace_bytes, void* stream) {
+static int gemm_dx_impl(const qlora_layer_desc* d, int M, const void* dY, const int8_t* Wq,
+                        const float* sw, const float* A, const void* gate, void* dX,
+                        const void* workspace, size_t workspace_bytes, void* stream) {
     int rc = check_layer(d, M);
     if (rc != QLORA_OK) return rc;
     QL_REQUIRE(dY && Wq && sw && A && dX && workspace, QLORA_EINVAL, "NULL pointer argument");
     QL_REQUIRE(aligned(dY, 16) && aligned(Wq, 16) && aligned(dX, 16) && aligned(workspace, 256),
                QLORA_EALIGN, "dY, Wq and dX must be 16-byte aligned, workspace 256-byte aligned");
     QL_REQUIRE(aligned(sw, 4) && aligned(A, 4), QLORA_EALIGN, "fp32 vectors must be 4-byte aligned");
+    QL_REQUIRE(!gate || aligned(gate, 16), QLORA_EALIGN, "X must be 16-byte aligned");
     if (M == 0) return QLORA_OK;
     const WsLayout w = layout_for(*d, M);
     QL_REQUIRE(workspace_bytes >= w.total, QLORA_EINVAL, "workspace too small");
@@ -439,9 +454,23 @@ int qlora_gemm_dx(const qlora_layer_desc* d, int M, const void* dY, const int8_t
     ep.r = d->r;
     ep.c = lora_scale(d);
     ep.dX = dX;
+    ep.gate = gate;
     return cuda_status(launch_gemm_dx(act_of(d), dY, Wq, sw, M, d->N, d->K, ep, status,
                                       static_cast<cudaStream_t>(stream)),
                        "dX GEMM launch");
+}
+
+int qlora_gemm_dx(const qlora_layer_desc* d, int M, const void* dY, const int8_t* Wq,
+                  const float* sw, const float* A, void* dX, const void* workspace,
+                  size_t workspace_bytes, void* stream) {
+    return gemm_dx_impl(d, M, dY, Wq, sw, A, nullptr, dX, workspace, workspace_bytes, stream);
+}
+
+int qlora_gemm_dx_relu(const qlora_layer_desc* d, int M, const void* dY, const int8_t* Wq,
+                       const float* sw, const float* A, const void* X, void* dX,
+                       const void* workspace, size_t workspace_bytes, void* stream) {
+    if (!X) return fail(QLORA_EINVAL, "NULL pointer argument");
+    return gemm_dx_impl(d, M, dY, Wq, sw, A, X, dX, workspace, workspace_bytes, stream);
 }
 
 int qlora_lora_grad_x(const qlora_layer_desc* d, int M, const void* X, float* dA,
@@ -628,6 +657,7 @@ int qlora_backward_noalloc(const qlora_layer_desc* d, int M, const void* X, cons
         ep.r = d->r;
         ep.c = c;
         ep.dX = dX;
+        ep.gate = nullptr;
         rc = cuda_status(launch_gemm_dx(act_of(d), dY, Wq, sw, M, d->N, d->K, ep, status, s),
                          "dX GEMM launch");
         if (rc != QLORA_OK) return rc;

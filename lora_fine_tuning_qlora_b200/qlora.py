@@ -31,7 +31,7 @@ EXPORTED = ("qlora_quantize_weight", "qlora_workspace_bytes", "qlora_forward",
             "qlora_version", "qlora_relu", "qlora_relu_backward", "qlora_quantize_input",
             "qlora_gemm_forward", "qlora_lora_grad_dy", "qlora_gemm_dx", "qlora_lora_grad_x",
             "qlora_selftest_wait_timeout", "qlora_backward_noalloc", "qlora_lora_g",
-            "qlora_lora_grad_b")
+            "qlora_lora_grad_b", "qlora_gemm_forward_relu", "qlora_gemm_dx_relu")
 
 
 class QLoraError(RuntimeError):
@@ -86,9 +86,12 @@ def _load():
     lib.qlora_lora_g.argtypes = [D, I, P, P, P, Z, P]
     lib.qlora_lora_grad_b.argtypes = [D, I, P, P, P, P, P]
     lib.qlora_gemm_dx.argtypes = [D, I, P, P, P, P, P, P, Z, P]
+    lib.qlora_gemm_forward_relu.argtypes = [D, I, P, P, P, P, P, P, P, P, P, P]
+    lib.qlora_gemm_dx_relu.argtypes = [D, I, P, P, P, P, P, P, P, Z, P]
     lib.qlora_lora_grad_x.argtypes = [D, I, P, P, P, Z, P]
     for f in (lib.qlora_quantize_input, lib.qlora_gemm_forward, lib.qlora_lora_grad_dy,
-              lib.qlora_lora_g, lib.qlora_lora_grad_b, lib.qlora_gemm_dx, lib.qlora_lora_grad_x):
+              lib.qlora_lora_g, lib.qlora_lora_grad_b, lib.qlora_gemm_dx, lib.qlora_lora_grad_x,
+              lib.qlora_gemm_forward_relu, lib.qlora_gemm_dx_relu):
         f.restype = I
     lib.qlora_selftest_wait_timeout.argtypes = [ctypes.c_uint, P]
     lib.qlora_selftest_wait_timeout.restype = I
@@ -207,6 +210,20 @@ def qlora_lora_grad_dy(d: LayerDesc, M: int, dY, B, xA, dB, dbias, ws, G=None, s
     writes the summed G too when a tensor is given)."""
     _check(_lib.qlora_lora_grad_dy(ctypes.byref(d), int(M), _ptr(dY), _ptr(B), _ptr(xA), _ptr(dB),
                                    _ptr(dbias), _ptr(G), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def qlora_gemm_forward_relu(d: LayerDesc, M: int, Xq, sx, Wq, sw, bias, xA, B, Y, acc=None,
+                            stream=None):
+    """qlora_gemm_forward with the following ReLU in its epilogue."""
+    _check(_lib.qlora_gemm_forward_relu(ctypes.byref(d), int(M), _ptr(Xq), _ptr(sx), _ptr(Wq),
+                                        _ptr(sw), _ptr(bias), _ptr(xA), _ptr(B), _ptr(Y), _ptr(acc),
+                                        _stream(stream)))
+
+
+def qlora_gemm_dx_relu(d: LayerDesc, M: int, dY, Wq, sw, A, X, dX, ws, stream=None):
+    """qlora_gemm_dx taken back through the ReLU that produced X."""
+    _check(_lib.qlora_gemm_dx_relu(ctypes.byref(d), int(M), _ptr(dY), _ptr(Wq), _ptr(sw), _ptr(A),
+                                   _ptr(X), _ptr(dX), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def qlora_lora_g(d: LayerDesc, M: int, dY, B, ws, stream=None):

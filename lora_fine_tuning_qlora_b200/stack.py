@@ -1,11 +1,13 @@
 """The MNIST MLP workload as a stack of int8-LoRA Dense layers on one GPU.
 
-784 -> 1024, 31 x (1024 -> 1024), 1024 -> 10 with a plain ReLU between
-layers ("Introduce QLoRA-like technique", benchmark.py and its Results
-table), batch 1024, bf16 activations, rank-8 adapters.  One ``step`` is the
-forward through every layer and the backward through every layer (dX, dA,
-dB of each), all through the C ABI into preallocated device buffers, so a
-step can be captured into a CUDA graph and replayed.
+784 -> 1024, 31 x (1024 -> 1024), 1024 -> 10 with a ReLU between layers
+("Introduce QLoRA-like technique", benchmark.py and its Results table),
+batch 1024, bf16 activations, rank-8 adapters.  One ``step`` is the forward
+through every layer and the backward through every layer (dX, dA, dB of
+each), all through the C ABI into preallocated device buffers, so a step can
+be captured into a CUDA graph and replayed.  The ReLU runs in the epilogues:
+the forward GEMM of a hidden layer writes max(Y, 0), and the dX GEMM of a
+layer whose input came out of a ReLU zeroes dX where that input is <= 0.
 """
 from __future__ import annotations
 
@@ -80,16 +82,14 @@ class MLPStack:
         n = 0
         bf16 = self.act == torch.bfloat16
         for i, L in enumerate(self.layers):
-            n += 2                                   # quantize+xA, int8 GEMM
-            n += 1 if i < len(self.layers) - 1 else 0  # ReLU
+            n += 2                                   # quantize+xA, int8 GEMM (+ ReLU)
             rj = (L.r + 7) // 8                      # CUDA-core passes: 8 ranks per launch
             dy_tc = bf16 and L.N % 8 == 0            # tensor-core dY passes, 128-column blocks
             n += 2 if dy_tc else 2 * rj              # G pass + dB/dbias pass
             ncb = -(-L.N // 128) if dy_tc else -(-L.N // 64)
             n += 1 if ncb > 8 else 0                 # G slices added once
-            n += 1                                   # dX GEMM
+            n += 1                                   # dX GEMM (+ ReLU backward)
             n += 1 if bf16 else rj                   # X pass
-            n += 1 if i < len(self.layers) - 1 else 0  # ReLU backward
         return n
 
     def _run(self, stream=None, events=None):
@@ -108,20 +108,18 @@ class MLPStack:
             qlora.qlora_quantize_input(D[i], M, h, L.A, self.Xq, self.sx, self.xA[i], stream)
             if ev_f and ev_f[i]:
                 ev_f[i][0].record(fwd)
-            qlora.qlora_gemm_forward(D[i], M, self.Xq, self.sx, L.Wq, L.sw, L.bias, self.xA[i],
-                                     L.B, self.H[i], None, stream)
+            # hidden layers: the ReLU that follows runs in the GEMM's epilogue
+            gemm = qlora.qlora_gemm_forward_relu if i < n - 1 else qlora.qlora_gemm_forward
+            gemm(D[i], M, self.Xq, self.sx, L.Wq, L.sw, L.bias, self.xA[i], L.B, self.H[i], None,
+                 stream)
             if ev_f and ev_f[i]:
                 ev_f[i][1].record(fwd)
-            if i < n - 1:
-                qlora.qlora_relu(self.H[i], stream)
             h = self.H[i]
         main = stream if stream is not None else torch.cuda.current_stream()
         g = self.dY
         for i in range(n - 1, -1, -1):
             L = L_[i]
             ws = self.ws if i % 2 == 0 else self.ws_alt
-            if i < n - 1:
-                qlora.qlora_relu_backward(g, self.H[i], main)
             x_in = self.X if i == 0 else self.H[i - 1]
             dX = self.dX if i == 0 else self.G[i - 1]
             if i + 2 < n:
@@ -130,10 +128,15 @@ class MLPStack:
             self.ev_g[i].record(main)
             if ev_d and ev_d[i]:
                 ev_d[i][0].record(main)
-            qlora.qlora_gemm_dx(D[i], M, g, L.Wq, L.sw, L.A, dX, ws, main)
+            if i > 0:
+                # dX taken back through the ReLU that produced this layer's input
+                qlora.qlora_gemm_dx_relu(D[i], M, g, L.Wq, L.sw, L.A, x_in, dX, ws, main)
+            else:
+                qlora.qlora_gemm_dx(D[i], M, g, L.Wq, L.sw, L.A, dX, ws, main)
             if ev_d and ev_d[i]:
                 ev_d[i][1].record(main)
-            self.side.wait_event(self.ev_g[i])
+            # a timed dX GEMM runs alone: the side stream waits for its end event
+            self.side.wait_event(ev_d[i][1] if ev_d and ev_d[i] else self.ev_g[i])
             qlora.qlora_lora_grad_b(D[i], M, g, self.xA[i], self.dB[i], self.dbias[i], self.side)
             qlora.qlora_lora_grad_x(D[i], M, x_in, self.dA[i], ws, self.side)
             self.ev_x[i].record(self.side)
@@ -144,7 +147,9 @@ class MLPStack:
         """Timing events (graph-capturable) around the given steps of the
         given layers (all layers when None).  An event pair between two
         kernels orders them, so each timed launch loses its overlap with its
-        neighbours; time a few layers to keep the step itself unperturbed."""
+        neighbours, and a timed dX GEMM also keeps that layer's side-stream
+        passes waiting until it ends; time a few layers to keep the step
+        itself close to unperturbed."""
         sel = set(range(len(self.layers)) if layers is None else layers)
         return {k: [(torch.cuda.Event(enable_timing=True, external=True),
                      torch.cuda.Event(enable_timing=True, external=True)) if i in sel else None

@@ -285,6 +285,45 @@ def test_split_dy_pass_matches_grad_dy(q, M, K, N, r, act):
     assert_close(to_np(outs[1][1]), ref["dA"], act, "dA")
 
 
+@pytest.mark.parametrize("M,K,N,r,act", [(200, 384, 264, 8, "bf16"), (96, 256, 10, 8, "bf16"),
+                                          (64, 784, 128, 4, "f32")])
+def test_fused_relu_entry_points(q, M, K, N, r, act):
+    """qlora_gemm_forward_relu == qlora_relu(qlora_gemm_forward) and
+    qlora_gemm_dx_relu == qlora_relu_backward(qlora_gemm_dx, X), bit for bit,
+    on the tensor-core and CUDA-core paths."""
+    spec = _edge_spec(M, K, N, r, act=act, seed=3 * M + N)
+    d = inputs.layer_inputs(spec)
+    from parity import device_layer, act_torch
+    layer = device_layer(spec, d, q)
+    tdt = act_torch(act)
+    X = torch.from_numpy(d["X"]).to(tdt).cuda()
+    X = torch.where(torch.arange(K, device="cuda") % 3 == 0, -X.abs(), X)  # plenty of X <= 0
+    dY = torch.from_numpy(d["dY"]).to(tdt).cuda()
+    D = layer.desc()
+    ws = q.workspace(D, M)
+    Xq = torch.empty((M, K), dtype=torch.int8, device="cuda")
+    sx = torch.empty((M,), device="cuda")
+    xA = torch.empty((M, r), device="cuda")
+    q.qlora_quantize_input(D, M, X, layer.A, Xq, sx, xA)
+    Y1 = torch.empty((M, N), dtype=tdt, device="cuda")
+    Y2 = torch.empty_like(Y1)
+    q.qlora_gemm_forward(D, M, Xq, sx, layer.Wq, layer.sw, layer.bias, xA, layer.B, Y1)
+    q.qlora_relu(Y1)
+    q.qlora_gemm_forward_relu(D, M, Xq, sx, layer.Wq, layer.sw, layer.bias, xA, layer.B, Y2)
+    dB = torch.empty((r, N), device="cuda")
+    q.qlora_lora_grad_dy(D, M, dY, layer.B, xA, dB, None, ws)
+    dX1 = torch.empty((M, K), dtype=tdt, device="cuda")
+    dX2 = torch.full_like(dX1, float("nan"))
+    q.qlora_gemm_dx(D, M, dY, layer.Wq, layer.sw, layer.A, dX1, ws)
+    q.qlora_relu_backward(dX1, X)
+    q.qlora_gemm_dx_relu(D, M, dY, layer.Wq, layer.sw, layer.A, X, dX2, ws)
+    torch.cuda.synchronize()
+    assert q.qlora_device_status() == 0
+    assert torch.equal(Y1, Y2)
+    assert torch.equal(dX1, dX2)
+    assert (Y2 >= 0).all() and (dX2[X <= 0] == 0).all()
+
+
 def test_relu_kernels(q):
     """The stack's elementwise ReLU and its backward, aligned and unaligned."""
     rng = np.random.Generator(np.random.PCG64(21))
