@@ -67,37 +67,55 @@ template <int RP>
 __host__ __device__ constexpr int a_chunk_floats() { return 8 * RP + 4; }
 
 // Stages A rows [k0, k0 + 8*chunks) into shared memory (zero outside K / r).
+// Every round issues all its loads (from addresses clamped into A) before
+// any of them is used, so a round costs one memory latency; a select on each
+// freshly loaded value would wait out the loads one by one.
 template <int RP>
 __device__ __forceinline__ void stage_a(float* sA, const float* __restrict__ A, int K, int r,
                                         int k0, int chunks) {
+    constexpr int kU = 8;  // loads in flight per thread
     if (r == RP && (reinterpret_cast<uintptr_t>(A) & 15) == 0) {
-        // rows of A are RP floats: copy 16-byte vectors, four in flight per thread
+        // rows of A are RP floats: copy 16-byte vectors
         constexpr int V = 2 * RP;  // float4 per 8-row chunk
         const int n4 = chunks * V;
         const int kmax4 = (K - k0) * RP / 4;  // float4 that lie inside A
+        const int lim = n4 < kmax4 ? n4 : kmax4;
         const float4* src = reinterpret_cast<const float4*>(A + static_cast<size_t>(k0) * RP);
         float4* dst = reinterpret_cast<float4*>(sA);
-        for (int base = threadIdx.x; base < n4; base += 4 * blockDim.x) {
-            float4 v[4];
+        for (int base = threadIdx.x; base < n4; base += kU * blockDim.x) {
+            float4 v[kU];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < kU; ++u) {
                 const int idx = base + u * blockDim.x;
-                v[u] = (idx < n4 && idx < kmax4) ? __ldg(src + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[u] = __ldg(src + (idx < lim ? idx : lim - 1));
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < kU; ++u) {
                 const int idx = base + u * blockDim.x;
-                if (idx < n4) dst[(idx / V) * (V + 1) + idx % V] = v[u];
+                if (idx < n4)
+                    dst[(idx / V) * (V + 1) + idx % V] = idx < lim ? v[u] : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
         return;
     }
     const int n = chunks * 8 * RP;
-    for (int idx = threadIdx.x; idx < n; idx += blockDim.x) {
-        const int kl = idx / RP, j = idx % RP;
-        const int k = k0 + kl;
-        sA[(kl >> 3) * a_chunk_floats<RP>() + (kl & 7) * RP + j] =
-            (k < K && j < r) ? __ldg(A + static_cast<size_t>(k) * r + j) : 0.f;
+    for (int base = threadIdx.x; base < n; base += kU * blockDim.x) {
+        float v[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int idx = base + u * blockDim.x;
+            const int kl = idx / RP, j = idx % RP;
+            const int k = k0 + kl < K ? k0 + kl : K - 1;
+            v[u] = __ldg(A + static_cast<size_t>(k) * r + (j < r ? j : r - 1));
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int idx = base + u * blockDim.x;
+            const int kl = idx / RP, j = idx % RP;
+            if (idx < n)
+                sA[(kl >> 3) * a_chunk_floats<RP>() + (kl & 7) * RP + j] =
+                    (k0 + kl < K && j < r) ? v[u] : 0.f;
+        }
     }
 }
 

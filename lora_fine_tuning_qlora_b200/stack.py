@@ -38,6 +38,7 @@ class MLPStack:
         self.side = torch.cuda.Stream(device=dev)
         self.ev_g = [torch.cuda.Event() for _ in layers]  # layer's G is in its workspace
         self.ev_x = [torch.cuda.Event() for _ in layers]  # layer's X pass is done
+        self.ev_dx = [torch.cuda.Event() for _ in layers]  # layer's dX GEMM is done (timed layers)
         self.X = torch.zeros((batch, layers[0].K), dtype=self.act, device=dev)
         self.dY = torch.zeros((batch, layers[-1].N), dtype=self.act, device=dev)
         self.H = [torch.empty((batch, L.N), dtype=self.act, device=dev) for L in layers]
@@ -135,8 +136,11 @@ class MLPStack:
                 qlora.qlora_gemm_dx(D[i], M, g, L.Wq, L.sw, L.A, dX, ws, main)
             if ev_d and ev_d[i]:
                 ev_d[i][1].record(main)
-            # a timed dX GEMM runs alone: the side stream waits for its end event
-            self.side.wait_event(ev_d[i][1] if ev_d and ev_d[i] else self.ev_g[i])
+                self.ev_dx[i].record(main)
+            # a timed dX GEMM runs alone: the side stream waits until it ends
+            # (through an ordinary event: a timing event cannot carry a stream
+            # into a graph capture)
+            self.side.wait_event(self.ev_dx[i] if ev_d and ev_d[i] else self.ev_g[i])
             qlora.qlora_lora_grad_b(D[i], M, g, self.xA[i], self.dB[i], self.dbias[i], self.side)
             qlora.qlora_lora_grad_x(D[i], M, x_in, self.dA[i], ws, self.side)
             self.ev_x[i].record(self.side)
