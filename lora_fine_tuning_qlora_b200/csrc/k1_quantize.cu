@@ -24,6 +24,7 @@ constexpr int kThreads = 256;
 constexpr int kChunk = 8;    // elements per 128-bit (bf16) / 2x128-bit (f32) load
 constexpr int kMaxCPT = 8;   // chunks per thread held in registers
 constexpr int kSmemCap = 200 * 1024;
+constexpr int kSlicedSmem = 96 * 1024;  // A slice of the sliced kernel: two CTAs per SM
 
 template <typename T>
 struct Chunk8;
@@ -299,6 +300,114 @@ __global__ void __launch_bounds__(kThreads) k1_quantize_rows_long_kernel(
     }
 }
 
+// Rows whose x.A operand A does not fit in shared memory.  A CTA takes 32
+// rows, four per warp, and sweeps them twice: the abs-max of each row, then,
+// A slice by A slice (each slice staged once for all 32 rows instead of once
+// per row), the quantization of the slice's chunks and their part of x.A.
+// Eight 8-element chunks of a row are loaded before any is used, and the A
+// slices are sized for two CTAs per SM, so that enough bytes are in flight
+// per SM to cover the memory latency.
+template <typename T, int RP>
+__global__ void __launch_bounds__(kThreads) k1_quantize_rows_sliced_kernel(
+    const T* __restrict__ X, const float* __restrict__ A, int M, int K, int r, int a_chunks,
+    int8_t* __restrict__ Xq, float* __restrict__ sx, float* __restrict__ xA) {
+    constexpr int kRowsPerWarp = 4;
+    constexpr int kRows = kRowsPerWarp * (kThreads / 32);
+    constexpr int kU = 8;
+    pdl_trigger();
+    pdl_wait();
+    extern __shared__ float4 smem_f4[];
+    float* sA = reinterpret_cast<float*>(smem_f4);
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int nchunks = K / kChunk;
+    const int m0 = blockIdx.x * kRows + warp * kRowsPerWarp;
+    float inv[kRowsPerWarp];
+#pragma unroll
+    for (int q = 0; q < kRowsPerWarp; ++q) {
+        const int m = m0 + q;
+        float amax = 0.f;
+        if (m < M) {
+            const T* xr = X + static_cast<size_t>(m) * K;
+            for (int ch = lane; ch < nchunks; ch += 32 * kU) {
+                float v[kU][8];
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    const int c = ch + 32 * u;
+                    Chunk8<T>::load(xr + static_cast<size_t>(c < nchunks ? c : nchunks - 1) * kChunk, v[u]);
+                }
+#pragma unroll
+                for (int u = 0; u < kU; ++u)
+                    if (ch + 32 * u < nchunks)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[u][e]));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        inv[q] = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
+        if (m < M && lane == 0) sx[m] = __fdiv_rn(amax, 127.0f);
+    }
+    float acc[kRowsPerWarp][RP];
+#pragma unroll
+    for (int q = 0; q < kRowsPerWarp; ++q)
+#pragma unroll
+        for (int j = 0; j < RP; ++j) acc[q][j] = 0.f;
+    for (int c0 = 0; c0 < nchunks; c0 += a_chunks) {
+        const int c1 = c0 + a_chunks < nchunks ? c0 + a_chunks : nchunks;
+        __syncthreads();  // the previous slice is no longer read
+        stage_a<RP>(sA, A, K, r, c0 * kChunk, c1 - c0);
+        __syncthreads();
+#pragma unroll
+        for (int q = 0; q < kRowsPerWarp; ++q) {
+            const int m = m0 + q;
+            if (m >= M) continue;  // warp-uniform
+            const T* xr = X + static_cast<size_t>(m) * K;
+            int8_t* qr = Xq + static_cast<size_t>(m) * K;
+            for (int ch = c0 + lane; ch < c1; ch += 32 * kU) {
+                float v[kU][8];
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    const int c = ch + 32 * u;
+                    Chunk8<T>::load(xr + static_cast<size_t>(c < c1 ? c : c1 - 1) * kChunk, v[u]);
+                }
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    const int c = ch + 32 * u;
+                    if (c < c1) {
+                        *reinterpret_cast<uint2*>(qr + static_cast<size_t>(c) * kChunk) = pack8(v[u], inv[q]);
+                        chunk_fma<RP>(sA + (c - c0) * a_chunk_floats<RP>(), v[u], acc[q]);
+                    }
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < kRowsPerWarp; ++q) {
+        const int m = m0 + q;
+#pragma unroll
+        for (int j = 0; j < RP; ++j) {
+            float v = acc[q][j];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if (m < M && lane == 0 && j < r) xA[static_cast<size_t>(m) * r + j] = v;
+        }
+    }
+}
+
+template <typename T, int RP>
+cudaError_t launch_sliced(const T* X, const float* A, int M, int K, int r, int8_t* Xq, float* sx,
+                          float* xA, cudaStream_t s) {
+    const int nchunks = K / kChunk;
+    const int cap_chunks = kSlicedSmem / (a_chunk_floats<RP>() * 4);
+    const int a_chunks = nchunks <= cap_chunks ? nchunks : cap_chunks;
+    auto kern = k1_quantize_rows_sliced_kernel<T, RP>;
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), kSmemCap);
+    if (e != cudaSuccess) return e;
+    constexpr int kRows = 4 * (kThreads / 32);
+    return launch_k(kern, dim3((M + kRows - 1) / kRows), dim3(kThreads),
+                    a_chunks * a_chunk_floats<RP>() * 4, s, 1, X, A, M, K, r, a_chunks, Xq, sx, xA);
+}
+
 template <typename T, int TPR, int RP>
 cudaError_t launch_tpr(const T* X, const float* A, int M, int K, int r, int8_t* Xq, float* sx,
                        float* xA, cudaStream_t s) {
@@ -322,6 +431,11 @@ template <typename T, int RP>
 cudaError_t launch_rows_rp(const T* X, const float* A, int M, int K, int r, int8_t* Xq, float* sx,
                            float* xA, cudaStream_t s) {
     const int nchunks = K / kChunk;
+    // A too large for shared memory: slices staged once per 32 rows
+    if constexpr (RP <= 16) {
+        if (nchunks > kSmemCap / (a_chunk_floats<RP>() * 4))
+            return launch_sliced<T, RP>(X, A, M, K, r, Xq, sx, xA, s);
+    }
     if (nchunks <= 32 * kMaxCPT) return launch_tpr<T, 32, RP>(X, A, M, K, r, Xq, sx, xA, s);
     if (nchunks <= 64 * kMaxCPT) return launch_tpr<T, 64, RP>(X, A, M, K, r, Xq, sx, xA, s);
     if (nchunks <= 128 * kMaxCPT) return launch_tpr<T, 128, RP>(X, A, M, K, r, Xq, sx, xA, s);

@@ -46,7 +46,8 @@ def test_single_fp32_layer(q):
 
 
 @pytest.mark.parametrize("M,K,N,r", [(300, 784, 520, 8), (129, 256, 136, 4), (1, 64, 16, 1),
-                                     (200, 1040, 264, 16), (70, 128, 24, 64)])
+                                     (200, 1040, 264, 16), (70, 128, 24, 64),
+                                     (100, 4096, 136, 16)])
 def test_bf16_layer_tiles_and_ragged_tails(q, M, K, N, r):
     spec = inputs.LayerSpec("ragged", M=M, K=K, N=N, r=r, alpha=2.0 * r, act="bf16",
                             x_dist="normal", w_dist="glorot", a_dist="he_uniform", b_std=0.01,
@@ -54,7 +55,7 @@ def test_bf16_layer_tiles_and_ragged_tails(q, M, K, N, r):
     run_and_compare(spec, q)
 
 
-@pytest.mark.parametrize("M,K,N,r", [(96, 784, 128, 4), (33, 1040, 10, 8)])
+@pytest.mark.parametrize("M,K,N,r", [(96, 784, 128, 4), (33, 1040, 10, 8), (40, 12288, 72, 4)])
 def test_fp32_layer_shapes(q, M, K, N, r):
     spec = inputs.LayerSpec("f32", M=M, K=K, N=N, r=r, alpha=r, act="f32", x_dist="normal",
                             w_dist="glorot", a_dist="he_uniform", b_std=0.01,
