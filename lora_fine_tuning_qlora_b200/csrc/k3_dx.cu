@@ -72,12 +72,16 @@ struct K3Cfg {
     // contraction of a tile is split over kChains MMA-issuing warps, each with
     // its own TMEM accumulator (added in chain order by the epilogue); two
     // tile buffers of kChains accumulators fill the 512 TMEM columns.
-    static constexpr int kChains = (MSUB == 1 && BN == 64) ? 4 : (MSUB == 1 ? 2 : 1);
+    // The 256-row tiles give each 128-row sub-tile its own issuer instead
+    // (kSplitRows): the two sub-tile accumulators are separate already.
+    static constexpr int kChains = (MSUB == 1 && BN == 64) ? 4 : 2;
+    static constexpr bool kSplitRows = MSUB == 2;
+    static constexpr int kKChains = kSplitRows ? 1 : kChains;  // accumulators added by the epilogue
     static constexpr uint32_t kAccCols = MSUB * BN;             // one chain's accumulator
-    static constexpr uint32_t kBufCols = kChains * kAccCols;    // one tile buffer
+    static constexpr uint32_t kBufCols = kKChains * kAccCols;   // one tile buffer
     static constexpr uint32_t kTmemCols = 2 * kBufCols;
     static_assert(kTmemCols <= 512, "TMEM");
-    static_assert((kBKn / 16) % kChains == 0, "k-steps per chain");
+    static_assert(kSplitRows ? kChains == MSUB : (kBKn / 16) % kChains == 0, "work per issuer");
     // warps: producer, kChains MMA issuers, de-quantize, epilogue
     static constexpr int kDqWarp0 = 1 + kChains;
     static constexpr int kEpiWarp0 = kDqWarp0 + kDqWarps;
@@ -228,8 +232,10 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
     } else if (warp < C::kDqWarp0) {
         // ------------------------------------------------------ MMA issuers
         // issuer ch takes the k-steps ch, ch + kChains, ... of every stage
-        // into its own accumulator; issuer 0 also adds the rank-r term
+        // into its own accumulator, or (256-row tiles) every k-step of
+        // sub-tile ch; each issuer adds the rank-r term of its rows
         const int ch = warp - 1;
+        constexpr int kKStep = C::kSplitRows ? 1 : C::kChains;
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16(128, BN, false, true);
             int g = 0, i = 0;
@@ -250,21 +256,24 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
                     const uint32_t a_base = smem_u32(smem + s * C::kStageBytes);
                     const uint32_t w_base = a_base + C::kABytes;
 #pragma unroll
-                    for (int kk = ch; kk < kBKn / 16; kk += C::kChains) {
+                    for (int kk = C::kSplitRows ? 0 : ch; kk < kBKn / 16; kk += kKStep) {
                         const uint64_t bd = smem_desc(w_base + kk * 2048, kLbo, 1024, kLayoutSw128);
 #pragma unroll
                         for (int ms = 0; ms < MSUB; ++ms) {
+                            if (C::kSplitRows && ms != ch) continue;
                             // 16-column step kk: block kk / 4 of the sub-tile, 32 bytes per step within it
                             const uint64_t ad = smem_desc(
                                 a_base + ms * C::kASub + (kk >> 2) * (128 * kBlkN * 2) + (kk & 3) * 32, 16,
                                 1024, kLayoutSw128);
-                            mma_bf16(tmem + ab * C::kBufCols + ch * C::kAccCols + ms * BN, ad, bd, idesc,
-                                     (kb > 0 || kk > ch) ? 1u : 0u);
+                            const uint32_t d = C::kSplitRows ? tmem + ab * C::kBufCols + ms * BN
+                                                             : tmem + ab * C::kBufCols + ch * C::kAccCols;
+                            const bool first = C::kSplitRows ? (kb == 0 && kk == 0) : (kb == 0 && kk == ch);
+                            mma_bf16(d, ad, bd, idesc, first ? 0u : 1u);
                         }
                     }
                     mma_commit(&empty[s]);
                 }
-                if (C::kLoraMMA && ch == 0) {
+                if (C::kLoraMMA && (C::kSplitRows || ch == 0)) {
                     // + (c G) A^T: tf32 MMAs from the tables the epilogue warps wrote
                     if (ok && !mbar_wait(&lready[ab], use & 1, status)) ok = false;
                     if (ok) {
@@ -278,6 +287,7 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
                             const uint64_t bd = smem_desc(at + ks * 256, 128, kSbo, kLayoutNone);
 #pragma unroll
                             for (int ms = 0; ms < MSUB; ++ms) {
+                                if (C::kSplitRows && ms != ch) continue;
                                 const uint64_t ad =
                                     smem_desc(gt + ms * 16 * kSbo + ks * 256, 128, kSbo, kLayoutNone);
                                 mma_tf32(tmem + ab * C::kBufCols + ms * BN, ad, bd, tdesc, 1);
@@ -429,7 +439,7 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
 #pragma unroll
                 for (int e = 0; e < kEpiCols; ++e) part[e] = __uint_as_float(v[e]);
 #pragma unroll
-                for (int ch = 1; ch < C::kChains; ++ch) {
+                for (int ch = 1; ch < C::kKChains; ++ch) {
                     tmem_ld16(tbase + ch * C::kAccCols + col, v);
                     tmem_ld_wait();
 #pragma unroll
