@@ -47,6 +47,7 @@ struct K3Cfg {
     // box), 64 for the 256-row tiles so that two stages fit
     static constexpr int kBKn = MSUB == 2 ? 64 : 128;
     static constexpr int kBlk = kBKn / kBlkN;
+    static_assert(MSUB == 1 || kBlk == 1, "one dY box per stage covers the sub-tiles of one block");
     // rank <= 16: c G A^T runs on the tensor cores as tf32 MMAs into the same
     // fp32 accumulator (operand tables c*G [kBM x kKL] and A [BN x kKL] per
     // accumulator buffer); larger ranks fall back to CUDA-core FMAs.
@@ -212,18 +213,16 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
                     }
                     uint8_t* sa = smem + s * C::kStageBytes;
                     mbar_arrive_expect_tx(&full[s], C::kABytes);
+                    // all kBM rows in one box: the stage's kBlk 64-column blocks
+                    // (MSUB == 1), or both 128-row sub-tiles of one block (MSUB
+                    // == 2), consecutive in shared memory
+                    if (dy3d) {
+                        tma_load_3d(sa, &tmDY, &full[s], 0, m0, kb * C::kBlk);
+                    } else {
 #pragma unroll
-                    for (int ms = 0; ms < MSUB; ++ms) {
-                        // the stage's kBlk 64-column blocks, consecutive in shared memory
-                        if (dy3d) {
-                            tma_load_3d(sa + ms * C::kASub, &tmDY, &full[s], 0, m0 + 128 * ms,
-                                        kb * C::kBlk);
-                        } else {
-#pragma unroll
-                            for (int b = 0; b < C::kBlk; ++b)
-                                tma_load_2d(sa + ms * C::kASub + b * (128 * kBlkN * 2), &tmDY, &full[s],
-                                            (kb * C::kBlk + b) * kBlkN, m0 + 128 * ms);
-                        }
+                        for (int b = 0; b < C::kBlk; ++b)
+                            tma_load_2d(sa + b * (C::kBM * kBlkN * 2), &tmDY, &full[s],
+                                        (kb * C::kBlk + b) * kBlkN, m0);
                     }
                 }
             }
@@ -500,10 +499,10 @@ cudaError_t launch_tc(const void* dY, const int8_t* Wq, const float* sw, int M, 
     CUtensorMap tdy;
     const int dy3d = (N % kBlkN) == 0 ? 1 : 0;
     const bool ok =
-        dy3d ? make_tmap_3d_blocks(&tdy, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, kBlkN, 128,
+        dy3d ? make_tmap_3d_blocks(&tdy, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, kBlkN, C::kBM,
                                    C::kBlk)
              : make_tmap_2d(&tdy, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N,
-                            static_cast<uint64_t>(N) * 2, 128, kBlkN, CU_TENSOR_MAP_SWIZZLE_128B);
+                            static_cast<uint64_t>(N) * 2, C::kBM, kBlkN, CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return cudaErrorInvalidValue;
     const int tiles = ((M + C::kBM - 1) / C::kBM) * ((K + BN - 1) / BN);
     const int grid = tiles < sm_count() ? tiles : sm_count();
