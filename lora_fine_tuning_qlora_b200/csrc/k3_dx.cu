@@ -10,16 +10,26 @@
 // kernel and the LoRA factors enter dX.
 //
 // tcgen05 path (bf16 activations, N a multiple of 8): persistent, one CTA
-// per SM, a tile is (128 * MSUB) rows x BN columns of dX, 18 warps:
-//   warp 0       TMA producer: MSUB dY tiles [128 x 64 bf16] (128B swizzle,
-//                K-major) and the int8 kernel tile Wq[n0:n0+64, k0:k0+BN]
-//   warp 1       TMEM owner and MMA issuer: MSUB x tcgen05.mma.kind::f16
-//                (bf16 in, fp32 accumulate), M=128, N=BN, K=16, all sharing
-//                one de-quantized B tile; two TMEM accumulators per
-//                sub-tile so tile i+1's main loop overlaps tile i's epilogue
-//   warps 2..9   de-quantize every int8 stage into a bf16 tile laid out as
-//                the MN-major 128B-swizzled B operand
-//   warps 10..17 epilogue: + c G A^T, staged coalesced stores of dX
+// per SM, a tile is (128 * MSUB) rows x BN columns of dX; a stage covers 128
+// (MSUB = 1) or 64 (MSUB = 2) rows of the contraction.  Warps:
+//   warp 0        TMA producer: one box per stage with all the tile's dY rows
+//                 (128B swizzle, K-major; a 3-D view of dY gives two 64-column
+//                 blocks in one box when N is a multiple of 64)
+//   warps 1..C    MMA issuers (C = 4, or 2): tcgen05.mma.kind::f16 (bf16 in,
+//                 fp32 accumulate), M=128, N=BN, K=16.  A tcgen05.mma holds
+//                 its issuing thread ~0.1 us whatever its N, so the 128 x 64
+//                 and 128 x 128 tiles split every stage's k-steps over C
+//                 issuers, each with its own TMEM accumulator, and the 256-row
+//                 tiles give each 128-row sub-tile its own issuer; two tile
+//                 buffers so tile i+1's main loop overlaps tile i's epilogue.
+//                 Warp 1 owns the TMEM allocation.
+//   8 warps       de-quantize: load their int8 code chunks and row scales
+//                 from global memory into registers S stages ahead, and
+//                 convert every stage into a bf16 tile laid out as the
+//                 MN-major 128B-swizzled B operand
+//   4 or 8 warps  epilogue: c G A^T (tf32 MMAs from tables they write), the
+//                 accumulators added in chain order, an optional ReLU-backward
+//                 gate, staged coalesced stores of dX
 // SIMT path: fp32 activations, or rows of dY that the Tensor Memory
 // Accelerator cannot describe (N*2 bytes not a multiple of 16).
 #include "internal.h"
@@ -60,7 +70,10 @@ struct K3Cfg {
     static constexpr int kWBytes = kBKn * BN * 2;      // de-quantized bf16 tile
     static constexpr int kStageBytes = kABytes + kWBytes;
     static constexpr int kStgBytes = kEpiWarps * 32 * stage_pitch<__nv_bfloat16>();
-    static constexpr int kParamBytes = 2 * (kGtBytes + kAtBytes);
+    // one set of rank-r operand tables: the epilogue warps write a tile's
+    // tables only after the previous tile's accumulator (and with it that
+    // tile's rank-r MMAs) is complete, so two sets are never live at once
+    static constexpr int kParamBytes = kGtBytes + kAtBytes;
     static constexpr int kFixed = kStgBytes + kParamBytes + 512 + 1024;
     static constexpr int kStagesFit = (kSmemLimit - kFixed) / kStageBytes;
     static constexpr int STAGES = kStagesFit > 8 ? 8 : kStagesFit;
@@ -165,7 +178,7 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
     uint64_t* tempty = tfull + 2;  // [2]
     uint64_t* lready = tempty + 2; // [2] rank-r operand tables written
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lready + 2);
-    uint8_t* tabs = smem + C::kTabOff;  // [2] x (c*G table, A table)
+    uint8_t* tabs = smem + C::kTabOff;  // c*G table, A table
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
@@ -279,7 +292,7 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
                         tc_fence_after();
                         constexpr uint32_t tdesc = idesc_tf32(128, BN);
                         constexpr uint32_t kSbo = (C::kKL / 4) * 128;
-                        const uint32_t gt = smem_u32(tabs + ab * (C::kGtBytes + C::kAtBytes));
+                        const uint32_t gt = smem_u32(tabs);
                         const uint32_t at = gt + C::kGtBytes;
 #pragma unroll
                         for (int ks = 0; ks < C::kKL / 8; ++ks) {
@@ -389,7 +402,7 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
             if constexpr (C::kLoraMMA) {
                 // operand tables of this tile's rank-r product, tf32-rounded:
                 // c*G rows m0.. and A rows k0.. (zero outside the matrices)
-                uint8_t* gt = tabs + ab * (C::kGtBytes + C::kAtBytes);
+                uint8_t* gt = tabs;
                 uint8_t* at = gt + C::kGtBytes;
                 for (int e = et; e < C::kBM * C::kKL; e += 32 * C::kEpiWarps) {
                     const int rr = e / C::kKL, j = e % C::kKL;
