@@ -3,8 +3,9 @@
 
 One step = forward and backward (dX, dA, dB, dbias of every layer) through
 the MNIST MLP stack of int8-LoRA Dense layers: 784 -> 1024, 31 x 1024 ->
-1024, 1024 -> 10, plain ReLU between layers, batch 1024 per GPU, bf16
-activations, rank 8, alpha 8 (seeded synthetic data and weights).  With N
+1024, 1024 -> 10, ReLU between layers (run in the GEMM epilogues), batch
+1024 per GPU, bf16 activations, rank 8, alpha 8 (seeded synthetic data and
+weights).  With N
 GPUs (torchrun, one process per GPU) every rank runs its own batch and the
 LoRA gradients are summed with one NCCL all-reduce per step (weak scaling).
 
