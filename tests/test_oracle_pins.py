@@ -240,6 +240,61 @@ def test_forward_B_zero_is_base_layer():
     np.testing.assert_array_equal(b0["dX"], bb["dX"])
 
 
+def test_rank_one_adapter_is_an_outer_product_update():
+    """r = 1: the adapter's contribution Y(B) - Y(B = 0) = c (X a) b is an
+    outer product of two vectors, i.e. a matrix of rank exactly one (its
+    second singular value vanishes), equal to numpy's outer product."""
+    rng = _rng(7)
+    M, K, N = 11, 24, 9
+    X = rng.normal(0, 1, (M, K)).astype(np.float32)
+    W = rng.normal(0, 0.05, (K, N)).astype(np.float32)
+    Wq, sw = oracle.quantize_weight(W)
+    a = rng.normal(0, 0.2, (K, 1))
+    b = rng.normal(0, 0.2, (1, N))
+    bias = rng.normal(0, 0.01, N)
+    delta = (oracle.forward(X, Wq, sw, bias, a, b, 3.0)["y"]
+             - oracle.forward(X, Wq, sw, bias, a, np.zeros((1, N)), 3.0)["y"])
+    sv = np.linalg.svd(delta, compute_uv=False)
+    assert sv[1] <= 1e-12 * sv[0]
+    np.testing.assert_allclose(delta, 3.0 * np.outer(X.astype(np.float64) @ a[:, 0], b[0]),
+                               rtol=1e-9, atol=1e-12)
+
+
+def test_columns_at_plus_minus_amax_quantize_to_127():
+    """A kernel whose every entry is +-a in its column quantizes to codes
+    +-127 only, with scale a / 127."""
+    rng = _rng(8)
+    K, N = 33, 7
+    amp = rng.uniform(0.1, 2.0, N).astype(np.float32)
+    W = (np.where(rng.integers(0, 2, (K, N)) == 1, 1.0, -1.0) * amp[None, :]).astype(np.float32)
+    Wq, sw = oracle.quantize_weight(W)
+    np.testing.assert_array_equal(np.abs(Wq.astype(np.int32)), 127)
+    np.testing.assert_array_equal(np.sign(Wq.T.astype(np.int32)), np.sign(W).astype(np.int32))
+    np.testing.assert_allclose(sw.astype(np.float64), amp.astype(np.float64) / 127.0, rtol=2 ** -23)
+
+
+def test_single_input_feature():
+    """K = 1: each input row is its own abs-max, so it quantizes to +-127 (or
+    0) and the base product is x * fl(q_w s_w) up to the fp32 roundings of the
+    two scales; the adapter term is c x a b."""
+    rng = _rng(9)
+    M, N, r = 6, 5, 2
+    X = rng.normal(0, 1, (M, 1)).astype(np.float32)
+    X[2, 0] = 0.0
+    W = rng.normal(0, 0.1, (1, N)).astype(np.float32)
+    Wq, sw = oracle.quantize_weight(W)
+    A = rng.normal(0, 0.3, (1, r))
+    B = rng.normal(0, 0.3, (r, N))
+    bias = rng.normal(0, 0.01, N)
+    out = oracle.forward(X, Wq, sw, bias, A, B, 4.0)
+    assert set(np.abs(out["xq"].astype(np.int32)).ravel().tolist()) <= {0, 127}
+    assert out["xq"][2, 0] == 0 and out["sx"][2] == 0.0
+    Xd = X.astype(np.float64)
+    Wd = Wq.T.astype(np.float64) * sw.astype(np.float64)[None, :]
+    ref = Xd @ Wd + bias[None, :] + (4.0 / r) * (Xd @ A) @ B
+    np.testing.assert_allclose(out["y"], ref, rtol=1e-6, atol=1e-9)
+
+
 # --------------------------------------------------------------------------
 # backward: central differences
 # --------------------------------------------------------------------------
