@@ -254,6 +254,21 @@ int qlora_gemm_dx_relu(const qlora_layer_desc* d, int M, const void* dY, const i
 int qlora_lora_grad_x(const qlora_layer_desc* d, int M, const void* X, float* dA,
                       const void* workspace, size_t workspace_bytes, void* stream);
 
+/* Launch policy of the column-sum passes on the tensor cores (bf16 layers):
+ * the dB/dbias half of a3 (qlora_lora_grad_dy, qlora_lora_grad_b) and a5
+ * (qlora_lora_grad_x).  They sum over the M rows; by default the rows of a
+ * 128-column block are spread over a cluster of up to 8 CTAs, which gives
+ * the lowest latency for a pass that runs alone.  rows > 0 makes every CTA
+ * cover at least that many rows (rounded up to 128), so a pass occupies
+ * fewer SMs for longer: the choice for passes that run on a side stream
+ * beside a larger kernel that needs the SMs.  rows == 0 restores the
+ * default.  Results change only by the fp32 rounding of the different
+ * grouping and stay deterministic for a given setting.  Process-wide, for
+ * launches made after the call (a captured graph keeps the launch shape it
+ * was captured with); returns the previous setting, or QLORA_EINVAL for rows
+ * outside [0, 2^24].  The pages have no counterpart. */
+int qlora_set_rank_pass_rows(int rows);
+
 /*
  * Lossy merge ("Introduce QLoRA-like technique", Results footnote: merging
  * LoRA weights into int8 kernels is lossy; "How to fine-tune the 4-bit

@@ -145,6 +145,8 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
 // Tile-shape override for tuning sweeps: the integer value of environment
 // variable `name`, read once, or -1 when it is unset.
 int tile_override(const char* name);
+// Minimum rows per CTA of the column-sum passes (dB/dbias, dA); 0 = default.
+int rank_pass_rows();
 
 // Sets the dynamic shared memory limit of `func` once per device.
 cudaError_t ensure_smem_attr(const void* func, int bytes);

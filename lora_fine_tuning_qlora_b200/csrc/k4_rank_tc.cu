@@ -448,6 +448,9 @@ cudaError_t launch_tc(const void* T, RankTcArgs a, int* status, cudaStream_t s) 
         // of 8 single-CTA SMs do not all fit one wave of the GPCs)
         const int max_cl = smem > 110 * 1024 ? 4 : kMaxCluster;
         a.tiles_per_cta = (mtiles + max_cl - 1) / max_cl;
+        // a caller's minimum rows per CTA (fewer CTAs that stay longer)
+        const int want = (rank_pass_rows() + kTileRows - 1) / kTileRows;
+        if (want > a.tiles_per_cta) a.tiles_per_cta = want;
         cl = (mtiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
         rows_grid = cl;
     } else {

@@ -4,6 +4,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <map>
+#include <atomic>
 #include <mutex>
 #include <set>
 #include <string>
@@ -164,6 +165,12 @@ int tile_override(const char* name) {
     cache[name] = val;
     return val;
 }
+
+namespace {
+std::atomic<int> g_rank_pass_rows{0};
+}
+
+int rank_pass_rows() { return g_rank_pass_rows.load(std::memory_order_relaxed); }
 
 bool pdl_enabled() {
     static const bool on = tile_override("QLORA_PDL") != 0;
@@ -471,6 +478,11 @@ int qlora_gemm_dx_relu(const qlora_layer_desc* d, int M, const void* dY, const i
                        const void* workspace, size_t workspace_bytes, void* stream) {
     if (!X) return fail(QLORA_EINVAL, "NULL pointer argument");
     return gemm_dx_impl(d, M, dY, Wq, sw, A, X, dX, workspace, workspace_bytes, stream);
+}
+
+int qlora_set_rank_pass_rows(int rows) {
+    if (rows < 0 || rows > (1 << 24)) return fail(QLORA_EINVAL, "rows per CTA must be in [0, 2^24]");
+    return g_rank_pass_rows.exchange(rows);
 }
 
 int qlora_lora_grad_x(const qlora_layer_desc* d, int M, const void* X, float* dA,

@@ -31,7 +31,8 @@ EXPORTED = ("qlora_quantize_weight", "qlora_workspace_bytes", "qlora_forward",
             "qlora_version", "qlora_relu", "qlora_relu_backward", "qlora_quantize_input",
             "qlora_gemm_forward", "qlora_lora_grad_dy", "qlora_gemm_dx", "qlora_lora_grad_x",
             "qlora_selftest_wait_timeout", "qlora_backward_noalloc", "qlora_lora_g",
-            "qlora_lora_grad_b", "qlora_gemm_forward_relu", "qlora_gemm_dx_relu")
+            "qlora_lora_grad_b", "qlora_gemm_forward_relu", "qlora_gemm_dx_relu",
+            "qlora_set_rank_pass_rows")
 
 
 class QLoraError(RuntimeError):
@@ -93,6 +94,8 @@ def _load():
               lib.qlora_lora_g, lib.qlora_lora_grad_b, lib.qlora_gemm_dx, lib.qlora_lora_grad_x,
               lib.qlora_gemm_forward_relu, lib.qlora_gemm_dx_relu):
         f.restype = I
+    lib.qlora_set_rank_pass_rows.argtypes = [I]
+    lib.qlora_set_rank_pass_rows.restype = I
     lib.qlora_selftest_wait_timeout.argtypes = [ctypes.c_uint, P]
     lib.qlora_selftest_wait_timeout.restype = I
     return lib
@@ -246,6 +249,15 @@ def qlora_gemm_dx(d: LayerDesc, M: int, dY, Wq, sw, A, dX, ws, stream=None):
 def qlora_lora_grad_x(d: LayerDesc, M: int, X, dA, ws, stream=None):
     _check(_lib.qlora_lora_grad_x(ctypes.byref(d), int(M), _ptr(X), _ptr(dA), _ptr(ws), ws.numel(),
                                   _stream(stream)))
+
+
+def qlora_set_rank_pass_rows(rows: int) -> int:
+    """Minimum rows per CTA of the dB/dbias and dA passes (0: the default,
+    lowest-latency spread); returns the previous setting."""
+    prev = _lib.qlora_set_rank_pass_rows(int(rows))
+    if prev < 0:
+        _check(prev)
+    return prev
 
 
 def qlora_relu(Y: torch.Tensor, stream=None):

@@ -20,6 +20,9 @@ from . import qlora
 
 
 class MLPStack:
+    # rows per CTA of the dB/dbias and dA passes on the side stream
+    SIDE_PASS_ROWS = 256
+
     def __init__(self, layers: List[qlora.Layer], batch: int, device="cuda"):
         self.layers = layers
         self.M = batch
@@ -117,6 +120,19 @@ class MLPStack:
                 ev_f[i][1].record(fwd)
             h = self.H[i]
         main = stream if stream is not None else torch.cuda.current_stream()
+        # the side-stream passes cover 256 rows per CTA: half the CTAs of the
+        # default spread, so that they leave the SMs to the dX GEMMs
+        prev = qlora.qlora_set_rank_pass_rows(self.SIDE_PASS_ROWS)
+        try:
+            self._backward(main, ev_d)
+        finally:
+            qlora.qlora_set_rank_pass_rows(prev)
+
+    def _backward(self, main, ev_d):
+        L_ = self.layers
+        n = len(L_)
+        D = self.descs
+        M = self.M
         g = self.dY
         for i in range(n - 1, -1, -1):
             L = L_[i]

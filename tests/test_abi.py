@@ -113,3 +113,15 @@ def test_binding_refuses_host_tensors(q):
     W = torch.zeros((32, 16))
     with pytest.raises(ValueError):
         q.quantize_weight(W)
+
+
+def test_rank_pass_rows_setting(q):
+    """qlora_set_rank_pass_rows returns the previous setting and refuses
+    negative values (no GPU needed)."""
+    lib = q.lib()
+    prev = lib.qlora_set_rank_pass_rows(256)
+    assert prev == 0
+    assert lib.qlora_set_rank_pass_rows(0) == 256
+    assert lib.qlora_set_rank_pass_rows(-1) == -1
+    assert b"rows per CTA" in lib.qlora_last_error()
+    assert lib.qlora_set_rank_pass_rows(0) == 0

@@ -286,6 +286,47 @@ def test_split_dy_pass_matches_grad_dy(q, M, K, N, r, act):
     assert_close(to_np(outs[1][1]), ref["dA"], act, "dA")
 
 
+@pytest.mark.parametrize("M,K,N,r", [(1024, 1024, 1024, 8), (1000, 784, 264, 4), (3000, 256, 512, 16)])
+def test_rank_pass_rows_setting(q, M, K, N, r):
+    """With 256 and 1024 rows per CTA (and back at the default) the dB/dbias
+    and dA passes still match the oracle, and two calls with the same
+    setting agree bit for bit."""
+    spec = _edge_spec(M, K, N, r, seed=M + 11 * N)
+    d = inputs.layer_inputs(spec)
+    from parity import device_layer
+    layer = device_layer(spec, d, q)
+    X = torch.from_numpy(d["X"]).to(torch.bfloat16).cuda()
+    dY = torch.from_numpy(d["dY"]).to(torch.bfloat16).cuda()
+    D = layer.desc()
+    ws = q.workspace(D, M)
+    _, xA = q.forward(layer, X, ws)
+    q.qlora_lora_g(D, M, dY, layer.B, ws)
+    ref = oracle.backward(oracle.to_act(d["X"], "bf16"), oracle.to_act(d["dY"], "bf16"),
+                          *oracle.quantize_weight(d["W"]), d["A"], d["B"], spec.alpha,
+                          want_dx=False, act="bf16")
+    try:
+        for rows in (256, 1024, 0):
+            assert q.qlora_set_rank_pass_rows(rows) in (0, 256, 1024)
+            outs = []
+            for _ in range(2):
+                dB = torch.full((r, N), float("nan"), device="cuda")
+                db = torch.full((N,), float("nan"), device="cuda")
+                dA = torch.full((K, r), float("nan"), device="cuda")
+                q.qlora_lora_grad_b(D, M, dY, xA, dB, db)
+                q.qlora_lora_grad_x(D, M, X, dA, ws)
+                outs.append((dB, db, dA))
+            torch.cuda.synchronize()
+            assert q.qlora_device_status() == 0
+            for a_, b_ in zip(*outs):
+                assert torch.equal(a_, b_)
+            dB, db, dA = outs[0]
+            assert_close(to_np(dB), ref["dB"], "bf16", "dB rows=%d" % rows)
+            assert_close(to_np(db), ref["dbias"], "bf16", "dbias rows=%d" % rows)
+            assert_close(to_np(dA), ref["dA"], "bf16", "dA rows=%d" % rows)
+    finally:
+        q.qlora_set_rank_pass_rows(0)
+
+
 @pytest.mark.parametrize("M,K,N,r,act", [(200, 384, 264, 8, "bf16"), (96, 256, 10, 8, "bf16"),
                                           (64, 784, 128, 4, "f32")])
 def test_fused_relu_entry_points(q, M, K, N, r, act):
