@@ -620,12 +620,21 @@ cudaError_t launch_gemm_dx(Act act, const void* dY, const int8_t* Wq, const floa
         return launch_k(k3_dx_simt_kernel<float>, grid, dim3(256), 0, s, 1,
                         static_cast<const float*>(dY), Wq, sw, M, N, K, ep);
     }
-    // tile shape: the largest that still gives every SM a tile
+    // tile shape: the least estimated main-loop time, i.e. waves of
+    // persistent CTAs x stages per tile x the measured pace of one stage on
+    // B200 (128x64 tiles: 0.88 us per 128-deep stage; 128x128: 1.30 us;
+    // 256x128: 0.91 us per 64-deep stage)
     const int sms = sm_count();
-    auto ntiles = [&](int bm, int bn) { return ((M + bm - 1) / bm) * ((K + bn - 1) / bn); };
+    auto cost = [&](int bm, int bn, int bkn, double pace) {
+        const long long tiles = static_cast<long long>((M + bm - 1) / bm) * ((K + bn - 1) / bn);
+        const long long waves = (tiles + sms - 1) / sms;
+        return static_cast<double>(waves) * ((N + bkn - 1) / bkn) * pace;
+    };
+    const double c0 = cost(256, 128, 64, 0.91), c1 = cost(128, 128, 128, 1.30),
+                 c2 = cost(128, 64, 128, 0.88);
     int cfg = 2;
-    if (ntiles(256, 128) >= sms) cfg = 0;
-    else if (ntiles(128, 128) >= sms) cfg = 1;
+    if (c1 < c2 && c1 <= c0) cfg = 1;
+    else if (c0 < c2 && c0 < c1) cfg = 0;
     const int forced = tile_override("QLORA_DX_TILE");  // tuning: 0, 1 or 2
     if (forced >= 0 && forced <= 2) cfg = forced;
     if (ep.r <= 4) return launch_tc_cfg<4>(cfg, dY, Wq, sw, M, N, K, ep, status, s);

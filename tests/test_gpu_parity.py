@@ -47,7 +47,7 @@ def test_single_fp32_layer(q):
 
 @pytest.mark.parametrize("M,K,N,r", [(300, 784, 520, 8), (129, 256, 136, 4), (1, 64, 16, 1),
                                      (200, 1040, 264, 16), (70, 128, 24, 64),
-                                     (100, 4096, 136, 16)])
+                                     (100, 4096, 136, 16), (1000, 1296, 264, 8)])
 def test_bf16_layer_tiles_and_ragged_tails(q, M, K, N, r):
     spec = inputs.LayerSpec("ragged", M=M, K=K, N=N, r=r, alpha=2.0 * r, act="bf16",
                             x_dist="normal", w_dist="glorot", a_dist="he_uniform", b_std=0.01,
