@@ -16,6 +16,7 @@ from parity import assert_close, to_np
     ("btnh,nhd->btd", "bt", "nh", "d"),     # attention output
     ("abc,cde->abde", "ab", "c", "de"),
     ("ab,bc->ac", "a", "b", "c"),           # Dense
+    ("ab,bcd->acd", "a", "b", "cd"),        # the float8 PR's EinsumDense example
 ])
 def test_plan_splits_axes(eq, batch, contracted, free):
     p = einsum.plan(eq)
@@ -27,7 +28,10 @@ def test_plan_splits_axes(eq, batch, contracted, free):
                                 "btd,dnh->bnth",    # output axes permuted
                                 "ab,cd->abcd",      # no contraction
                                 "btd,hdn->btnh",    # contraction not on the leading kernel axes
-                                "ab,bb->ab"])       # repeated axis
+                                "ab,bb->ab",        # repeated axis
+                                # the float8 PR's speed test: the kernel shares axes a and b
+                                # with the output, a batched GEMM with one kernel per (a, b)
+                                "abcde,aebf->adbcf"])
 def test_plan_rejects_other_equations(eq):
     assert not einsum.supported(eq)
     with pytest.raises(ValueError):
