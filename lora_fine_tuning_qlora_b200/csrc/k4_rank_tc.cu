@@ -306,6 +306,8 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
             for (int i = 0; i < nt && ok; ++i) g_epilogue(i);
         }
         if constexpr (kD) {
+            // rows of V in whole 8-float groups at 16-byte alignment
+            const bool vec4 = (a.r % 8) == 0 && (reinterpret_cast<uintptr_t>(a.V) & 15) == 0;
             for (int i = 0; i < nt && ok; ++i) {
                 const int s = i & 1;
                 const int m = (t0 + i) * kTileRows + rr;
@@ -316,7 +318,33 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
                 const bool mok = m < a.M;
                 for (int j0 = 0; j0 < L.RP; j0 += 8) {
                     float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                    if (mok && j0 < a.r) {
+                    bool vdone = false;
+                    if constexpr (!kG) {
+                      if (mok && j0 < a.r && vec4) {
+                        vdone = true;
+                        // V = the nsl slices added in ascending order: eight
+                        // slices' rows in flight as 16-byte loads, then the adds
+                        const float4* p4 = reinterpret_cast<const float4*>(a.V + static_cast<size_t>(m) * a.r + j0);
+                        const size_t st4 = static_cast<size_t>(a.M) * a.r / 4;
+                        for (int b0 = 0; b0 < a.nsl; b0 += 8) {
+                            float4 lo[8], hi[8];
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                const size_t b = static_cast<size_t>(b0 + u < a.nsl ? b0 + u : b0);
+                                lo[u] = __ldg(p4 + b * st4);
+                                hi[u] = __ldg(p4 + b * st4 + 1);
+                            }
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                if (b0 + u < a.nsl) {
+                                    v[0] += lo[u].x; v[1] += lo[u].y; v[2] += lo[u].z; v[3] += lo[u].w;
+                                    v[4] += hi[u].x; v[5] += hi[u].y; v[6] += hi[u].z; v[7] += hi[u].w;
+                                }
+                            }
+                        }
+                      }
+                    }
+                    if (!vdone && mok && j0 < a.r) {
                         const int nv = min(8, a.r - j0);
                         const float* p = a.V + static_cast<size_t>(m) * a.r + j0;
                         // V = the nsl slices added in ascending order, every load issued at once
