@@ -22,6 +22,9 @@ What each routine follows (page title, section):
     through the input quantizer.
   * merge -- Keras PR 19356 Results footnote (lossy merge) and the 4-bit
     thread (de-quantize, add the LoRA, re-quantize).
+  * quantize_weight_int4 / unpack_int4 / merge_int4 -- packed 4-bit kernels:
+    keras-llm-light, "Simplified Int4Variable quantization" (two int4 values
+    per int8 byte) and the 4-bit thread; the readings are in the C file.
 
 Pins: every routine here is checked by ``tests/test_oracle_pins.py`` against
 closed forms, brute force, finite differences and printed values (see
@@ -76,6 +79,9 @@ def _lib():
             lib.orc_backward.argtypes = [L, L, L, L, D, P, P, P, P, P, P,
                                          ctypes.c_int, P, P, P, P, P]
             lib.orc_merge.argtypes = [P, P, P, P, L, L, L, F, P, P]
+            lib.orc_quantize_weight_int4.argtypes = [P, L, L, P, P]
+            lib.orc_unpack_int4.argtypes = [P, L, L, P]
+            lib.orc_merge_int4.argtypes = [P, P, P, P, L, L, L, F, P, P]
             lib.orc_round_bf16.argtypes = [D]
             lib.orc_round_bf16.restype = D
             lib.orc_round_bf16_array.argtypes = [P, L, P]
@@ -216,6 +222,46 @@ def merge(Wq, sw, A, B, alpha):
     sw2 = np.empty_like(sw)
     _lib().orc_merge(_p(Wq), _p(sw), _p(A), _p(B), K, N, r, float(c), _p(Wq2), _p(sw2))
     return Wq2, sw2
+
+
+# --------------------------------------------------------------------------
+# packed int4 kernels (the int8 layer with 4-bit codes; readings in the C file)
+# --------------------------------------------------------------------------
+def quantize_weight_int4(W):
+    """W [K,N] float32 (K even) -> (Wp [N, K/2] uint8 packed codes, sw [N] float32)."""
+    W = _c(W, np.float32)
+    K, N = W.shape
+    if K % 2:
+        raise ValueError("K must be even to pack two codes per byte")
+    Wp = np.empty((N, K // 2), np.uint8)
+    sw = np.empty((N,), np.float32)
+    _lib().orc_quantize_weight_int4(_p(W), K, N, _p(Wp), _p(sw))
+    return Wp, sw
+
+
+def unpack_int4(Wp):
+    """Wp [N, K/2] uint8 -> Wq [N, K] int8 codes (the layer's forward and
+    backward are the int8 ones with these codes)."""
+    Wp = _c(Wp, np.uint8)
+    N, K2 = Wp.shape
+    Wq = np.empty((N, 2 * K2), np.int8)
+    _lib().orc_unpack_int4(_p(Wp), N, 2 * K2, _p(Wq))
+    return Wq
+
+
+def merge_int4(Wp, sw, A, B, alpha):
+    """Lossy merge of an int4 layer -> (Wp' [N, K/2] uint8, sw' [N] float32)."""
+    Wq = unpack_int4(Wp)
+    sw = _c(sw, np.float32)
+    A = _c(A, np.float32)
+    B = _c(B, np.float32)
+    N, K = Wq.shape
+    r = A.shape[1]
+    c = np.float32(np.float32(alpha) / np.float32(r))
+    Wp2 = np.empty((N, K // 2), np.uint8)
+    sw2 = np.empty_like(sw)
+    _lib().orc_merge_int4(_p(Wq), _p(sw), _p(A), _p(B), K, N, r, float(c), _p(Wp2), _p(sw2))
+    return Wp2, sw2
 
 
 def round_bf16(x):

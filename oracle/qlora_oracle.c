@@ -304,6 +304,87 @@ void orc_merge(const int8_t* Wq, const float* sw, const float* A, const float* B
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* Packed int4 kernels ("Simplified Int4Variable quantization" in the         */
+/* keras-llm-light description: two int4 values stored in one int8 byte;     */
+/* "How to fine-tune the 4-bit model?": a 4-bit integer kernel, frozen, with  */
+/* an fp32 LoRA, de-quantized in place; merge = de-quantize, add the LoRA,    */
+/* re-quantize).  Readings where the pages are silent:                        */
+/*   - the int4 quantizer is the int8 one with 7 in place of 127: per output  */
+/*     channel, s = amax / 7, q = clamp(round_half_even(v * (7 / amax)),      */
+/*     -7, 7), fp32, one rounding per operation (15 levels, symmetric);       */
+/*   - packing runs along K: byte j of channel n holds code 2j in its low     */
+/*     nibble and code 2j+1 in its high nibble, each as a two's-complement    */
+/*     nibble; K is even;                                                     */
+/*   - an int4 layer computes exactly what the int8 layer computes with the   */
+/*     unpacked codes in place of the int8 codes (forward, backward), and its */
+/*     merge re-quantizes the merged kernel to int4.                          */
+/* ------------------------------------------------------------------------ */
+static float quantize_vector_int4(const float* v, long n, long stride, int8_t* q) {
+    float amax = 0.0f;
+    for (long i = 0; i < n; ++i) {
+        float a = fabsf(v[i * stride]);
+        if (a > amax) amax = a;
+    }
+    float inv = (amax > 0.0f) ? 7.0f / amax : 0.0f;
+    for (long i = 0; i < n; ++i) {
+        float t = v[i * stride] * inv;      /* one fp32 rounding */
+        float r = rintf(t);                 /* round half to even */
+        if (r > 7.0f) r = 7.0f;
+        if (r < -7.0f) r = -7.0f;
+        q[i] = (int8_t)r;
+    }
+    return amax / 7.0f;
+}
+
+static void pack_int4_row(const int8_t* q, long K, uint8_t* out) {
+    for (long j = 0; j < K / 2; ++j) {
+        unsigned lo = (unsigned)q[2 * j] & 0xFu;
+        unsigned hi = (unsigned)q[2 * j + 1] & 0xFu;
+        out[j] = (uint8_t)(lo | (hi << 4));
+    }
+}
+
+/* W [K,N] fp32 -> Wp [N, K/2] packed codes, sw [N]. */
+void orc_quantize_weight_int4(const float* W, long K, long N, uint8_t* Wp, float* sw) {
+    #pragma omp parallel for schedule(static)
+    for (long n = 0; n < N; ++n) {
+        int8_t* q = (int8_t*)malloc((size_t)K);
+        sw[n] = quantize_vector_int4(W + n, K, N, q);
+        pack_int4_row(q, K, Wp + n * (K / 2));
+        free(q);
+    }
+}
+
+/* Wp [N, K/2] -> Wq [N,K] int8 codes in [-8, 7]. */
+void orc_unpack_int4(const uint8_t* Wp, long N, long K, int8_t* Wq) {
+    for (long n = 0; n < N; ++n) {
+        for (long j = 0; j < K / 2; ++j) {
+            int lo = Wp[n * (K / 2) + j] & 0xF;
+            int hi = (Wp[n * (K / 2) + j] >> 4) & 0xF;
+            Wq[n * K + 2 * j] = (int8_t)(lo >= 8 ? lo - 16 : lo);
+            Wq[n * K + 2 * j + 1] = (int8_t)(hi >= 8 ? hi - 16 : hi);
+        }
+    }
+}
+
+/* Lossy merge of an int4 layer (given its unpacked codes): the merged entries
+ * of the int8 merge, re-quantized per channel to int4 and packed. */
+void orc_merge_int4(const int8_t* Wq, const float* sw, const float* A, const float* B,
+                    long K, long N, long r, float c, uint8_t* Wp_out, float* sw_out) {
+    #pragma omp parallel for schedule(static)
+    for (long n = 0; n < N; ++n) {
+        float* col = (float*)malloc(sizeof(float) * (size_t)K);
+        int8_t* q = (int8_t*)malloc((size_t)K);
+        for (long k = 0; k < K; ++k)
+            col[k] = merged_entry(Wq, sw, A, B, K, N, r, c, k, n);
+        sw_out[n] = quantize_vector_int4(col, K, 1, q);
+        pack_int4_row(q, K, Wp_out + n * (K / 2));
+        free(q);
+        free(col);
+    }
+}
+
 /*
  * Round an fp64 value to the nearest bfloat16 (8-bit significand, the fp32
  * exponent range), ties to even, returned as fp64.  Used where a layer's

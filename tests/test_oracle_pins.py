@@ -540,3 +540,101 @@ def test_input_generator_is_deterministic_and_shaped():
     assert a["X"].shape == (16, 256) and a["W"].shape == (256, 128)
     assert a["A"].shape == (256, 4) and a["B"].shape == (4, 128)
     assert np.abs(a["W"]).max() <= 1.0
+
+
+# --------------------------------------------------------------------------
+# packed int4 kernels
+# --------------------------------------------------------------------------
+def test_int4_byte_layout_by_hand():
+    """One channel, K = 4: amax = 7/8 gives 7/amax = 8 exactly, so the codes
+    are w * 8 = (-7, 3, 0, -1).  Packed two per byte, even k in the low
+    nibble, as two's-complement nibbles: 0x39 (low 9 = -7, high 3) and 0xF0
+    (low 0, high F = -1)."""
+    W = np.array([[-7 / 8], [3 / 8], [0.0], [-1 / 8]], np.float32)
+    Wp, sw = oracle.quantize_weight_int4(W)
+    assert Wp.shape == (1, 2) and Wp.dtype == np.uint8
+    assert Wp[0, 0] == 0x39 and Wp[0, 1] == 0xF0
+    assert sw[0] == np.float32(0.125)
+    np.testing.assert_array_equal(oracle.unpack_int4(Wp), [[-7, 3, 0, -1]])
+
+
+def test_int4_ties_round_half_to_even():
+    """amax = 7/8 (7/amax = 8): w = k/16 for odd k lands exactly on .5 and
+    rounds to the even neighbour: 2.5 -> 2, 3.5 -> 4, -0.5 -> 0, 1.5 -> 2,
+    -2.5 -> -2, 6.5 -> 6."""
+    vals = [7 / 8, 2.5 / 8, 3.5 / 8, -0.5 / 8, 1.5 / 8, -2.5 / 8, 6.5 / 8, 0.0]
+    W = np.array(vals, np.float32)[:, None]
+    Wp, _ = oracle.quantize_weight_int4(W)
+    np.testing.assert_array_equal(oracle.unpack_int4(Wp)[0], [7, 2, 4, 0, 2, -2, 6, 0])
+
+
+def test_int4_every_code_survives_packing_in_both_nibbles():
+    """Brute force over all 15 x 15 pairs of codes: a channel holding the
+    pair (q0, q1) next to +-7 reference entries quantizes and unpacks to
+    exactly those codes, in either position of the byte."""
+    codes = list(range(-7, 8))
+    cols = []
+    for q0 in codes:
+        for q1 in codes:
+            cols.append([q0, q1, 7, -7])
+    W = (np.array(cols, np.float32).T * np.float32(0.25))  # amax 7/4: 7/amax = 4 exactly
+    Wp, sw = oracle.quantize_weight_int4(W)
+    np.testing.assert_array_equal(oracle.unpack_int4(Wp), np.array(cols, np.int8))
+    np.testing.assert_array_equal(sw, np.float32(0.25))
+
+
+def test_int4_quantizer_properties():
+    """Random channels: every nonzero channel reaches code +-7 at its abs-max,
+    codes are monotone in w within a channel, every entry lies within half a
+    step of its de-quantized value (plus the fp32 rounding of w * 7/amax),
+    and an all-zero channel gets codes 0 and scale 0."""
+    rng = _rng(11)
+    K, N = 64, 12
+    W = rng.standard_t(3, (K, N)).astype(np.float32) * 0.02
+    W[:, 5] = 0.0
+    Wp, sw = oracle.quantize_weight_int4(W)
+    q = oracle.unpack_int4(Wp).astype(np.int32)  # [N, K]
+    assert sw[5] == 0.0 and not q[5].any()
+    for n in range(N):
+        if n == 5:
+            continue
+        k = int(np.argmax(np.abs(W[:, n])))
+        assert abs(q[n, k]) == 7 and np.sign(q[n, k]) == np.sign(W[k, n])
+        order = np.argsort(W[:, n], kind="stable")
+        assert (np.diff(q[n, order]) >= 0).all()
+        amax = float(np.abs(W[:, n]).max())
+        err = np.abs(W[:, n].astype(np.float64) - q[n] * float(sw[n]))
+        assert (err <= (0.5 + 2 ** -20) * amax / 7).all()
+    assert q.min() >= -7 and q.max() <= 7
+
+
+def test_int4_merge_of_a_zero_adapter_keeps_the_codes():
+    """B = 0: every merged entry is fl(q s), which re-quantizes to the same
+    codes (the relative error of fl(q s) * fl(7 / fl(7 s)) is far below half
+    a step), with a scale within one ulp of s."""
+    rng = _rng(12)
+    K, N, r = 32, 9, 4
+    W = rng.normal(0, 0.05, (K, N)).astype(np.float32)
+    Wp, sw = oracle.quantize_weight_int4(W)
+    A = rng.normal(0, 0.3, (K, r)).astype(np.float32)
+    Wp2, sw2 = oracle.merge_int4(Wp, sw, A, np.zeros((r, N), np.float32), 8.0)
+    np.testing.assert_array_equal(oracle.unpack_int4(Wp2), oracle.unpack_int4(Wp))
+    np.testing.assert_allclose(sw2, sw, rtol=2 ** -23)
+
+
+def test_int4_merge_of_a_rank_one_power_of_two_adapter():
+    """All codes 0 and a rank-one adapter of powers of two: the merged
+    channel n is c a_k b_n (every product exact), so its codes are
+    rne(7 a_k / max|a|) and its scale c |b_n| max|a| / 7."""
+    K, N = 6, 3
+    a = np.array([1.0, -0.5, 0.25, -1.0, 0.125, 0.5], np.float32)
+    b = np.array([2.0, -0.25, 1.0], np.float32)
+    Wp = np.zeros((N, K // 2), np.uint8)
+    sw = np.full((N,), 0.01, np.float32)
+    Wp2, sw2 = oracle.merge_int4(Wp, sw, a[:, None], b[None, :], 2.0)  # c = 2 / 1
+    # 7 * a / max|a| = 7, -3.5, 1.75, -7, 0.875, 3.5 -> rne: 7, -4, 2, -7, 1, 4
+    want = np.array([7, -4, 2, -7, 1, 4], np.int8)
+    q = oracle.unpack_int4(Wp2)
+    for n in range(N):
+        np.testing.assert_array_equal(q[n], want * int(np.sign(b[n])))
+        assert sw2[n] == np.float32(np.float32(2.0 * abs(b[n]) * 1.0) / np.float32(7.0))
