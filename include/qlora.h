@@ -269,6 +269,45 @@ int qlora_lora_grad_x(const qlora_layer_desc* d, int M, const void* X, float* dA
  * outside [0, 2^24].  The pages have no counterpart. */
 int qlora_set_rank_pass_rows(int rows);
 
+/* ------------------------------------------------------------------------
+ * Packed int4 frozen kernels (keras-llm-light, "Simplified Int4Variable
+ * quantization": two int4 values in one int8 byte; "How to fine-tune the
+ * 4-bit model?": a frozen 4-bit kernel under an fp32 LoRA, de-quantized in
+ * place before the matrix unit).  Reading (the pages give no formula): the
+ * int8 quantizer with 7 in place of 127, per output channel n,
+ *   sw[n] = amax / 7,  q[n,k] = clamp(rne(W[k,n] * (7 / amax)), -7, 7)
+ * in fp32, one rounding per operation; Wp [N, K/2] bytes, byte j of row n
+ * holding q[n,2j] in its low nibble and q[n,2j+1] in its high nibble (two's
+ * complement).  An int4 layer computes exactly what the int8 layer computes
+ * with these codes as its Wq.  K must be a multiple of 32
+ * (QLORA_EUNSUPPORTED otherwise); Wp is 16-byte aligned.
+ *
+ * Forward: expand the codes once with qlora_unpack_int4 into an int8 [N, K]
+ * buffer the caller owns and run qlora_forward / qlora_gemm_forward on it
+ * (the codes lie in [-7, 7]); the dX GEMM reads the packed codes directly.
+ * ------------------------------------------------------------------------ */
+
+/* a0 for int4: W [K,N] fp32 -> Wp [N, K/2] packed codes, sw [N].  Bit-exact. */
+int qlora_quantize_weight_int4(const float* W, int K, int N, uint8_t* Wp, float* sw,
+                               void* stream);
+
+/* Wp [N, K/2] -> Wq [N, K] int8 codes in [-8, 7] (Wq 16-byte aligned).  Bit-exact. */
+int qlora_unpack_int4(const uint8_t* Wp, int K, int N, int8_t* Wq, void* stream);
+
+/* a4 with packed int4 codes: dX = dY (q * sw)^T + c * G A^T, the nibbles
+ * de-quantized in shared memory; G from the workspace as qlora_gemm_dx.
+ * Bit-identical to qlora_gemm_dx given the unpacked codes. */
+int qlora_gemm_dx_int4(const qlora_layer_desc* d, int M, const void* dY, const uint8_t* Wp,
+                       const float* sw, const float* A, void* dX, const void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* a6 for int4: the merged kernel of qlora_merge (same operations, same
+ * order), re-quantized per channel to int4 and packed into Wp_out [N, K/2],
+ * sw_out [N].  Bit-exact.  Outputs must not alias the inputs. */
+int qlora_merge_int4(const qlora_layer_desc* d, const uint8_t* Wp, const float* sw,
+                     const float* A, const float* B, uint8_t* Wp_out, float* sw_out,
+                     void* stream);
+
 /*
  * Lossy merge ("Introduce QLoRA-like technique", Results footnote: merging
  * LoRA weights into int8 kernels is lossy; "How to fine-tune the 4-bit

@@ -48,8 +48,10 @@ struct DxEpilogue {
                       // out of a ReLU, whose backward this applies)
 };
 // dX = dY (Wq sw)^T + c G A^T.  tcgen05 bf16 path when possible, else SIMT.
+// w4: Wq holds packed int4 codes [N, K/2] (K % 32 == 0).
 cudaError_t launch_gemm_dx(Act act, const void* dY, const int8_t* Wq, const float* sw, int M,
-                           int N, int K, const DxEpilogue& ep, int* status, cudaStream_t s);
+                           int N, int K, const DxEpilogue& ep, int* status, cudaStream_t s,
+                           bool w4 = false);
 
 // ---------------------------------------------------------------- K4
 // The dY pass runs on the tensor cores for bf16 activations whose rows TMA
@@ -82,6 +84,13 @@ cudaError_t launch_rank_x_tc(const void* X, const float* G, int nsl, int M, int 
                              float* dA, int* status, cudaStream_t s);
 
 // ---------------------------------------------------------------- KM
+cudaError_t launch_merge_int4(const uint8_t* Wp, const float* sw, const float* A, const float* B,
+                              int K, int N, int r, float c, uint8_t* Wp_out, float* sw_out,
+                              cudaStream_t s);
+// Packed int4 kernels (two codes per byte, even k in the low nibble; K % 32 == 0).
+cudaError_t launch_quantize_weight_int4(const float* W, int K, int N, uint8_t* Wp, float* sw,
+                                        cudaStream_t s);
+cudaError_t launch_unpack_int4(const uint8_t* Wp, int K, int N, int8_t* Wq, cudaStream_t s);
 cudaError_t launch_merge(const int8_t* Wq, const float* sw, const float* A, const float* B, int K,
                          int N, int r, float c, int8_t* Wq_out, float* sw_out, cudaStream_t s);
 

@@ -23,7 +23,8 @@
 //                 tiles give each 128-row sub-tile its own issuer; two tile
 //                 buffers so tile i+1's main loop overlaps tile i's epilogue.
 //                 Warp 1 owns the TMEM allocation.
-//   8 warps       de-quantize: load their int8 code chunks and row scales
+//   8 warps       de-quantize: load their code chunks (int8, or packed int4
+//                 unpacked to int8 first) and row scales
 //                 from global memory into registers S stages ahead, and
 //                 convert every stage into a bf16 tile laid out as the
 //                 MN-major 128B-swizzled B operand
@@ -159,7 +160,9 @@ __device__ __forceinline__ void dequant16(const uint4 raw, float scale, uint32_t
     }
 }
 
-template <int MSUB, int BN, int RMAX>
+// W4: Wq holds packed int4 codes [N, K/2] (two per byte, even k in the low
+// nibble) instead of int8 codes [N, K]; a 16-byte fetch then carries 32 codes.
+template <int MSUB, int BN, int RMAX, bool W4>
 __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
     k3_dx_dequant_kernel(const __grid_constant__ CUtensorMap tmDY, int dy3d,
                          const int8_t* __restrict__ Wq, const float* __restrict__ sw, int M, int N,
@@ -321,7 +324,9 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
         // latency sits on the conversion path; a stage only waits for its
         // bf16 slot to be released by the MMAs that read it last.
         const int dw = warp - C::kDqWarp0;  // 0 .. 7
-        constexpr int kChunksPerRow = BN / 16;
+        constexpr int kCodes = W4 ? 32 : 16;  // codes per 16-byte chunk
+        constexpr int kChunksPerRow = BN / kCodes;
+        const size_t row_bytes = W4 ? static_cast<size_t>(K) / 2 : static_cast<size_t>(K);
         constexpr int kChunks = kBKn * kChunksPerRow;
         constexpr int kPerLane = kChunks / (32 * kDqWarps);
         static_assert(kChunks % (32 * kDqWarps) == 0, "chunks per stage");
@@ -343,11 +348,12 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
             for (int i = 0; i < kPerLane; ++i) {
                 const int c = dw * 32 + lane + i * 32 * kDqWarps;
                 const int n = kb * kBKn + c / kChunksPerRow;
-                const int k = k0 + (c % kChunksPerRow) * 16;
+                const int k = k0 + (c % kChunksPerRow) * kCodes;
                 if (g < total_kb && n < N && k < K) in_bits |= 1u << i;
                 const int nc = n < N ? n : N - 1;
-                const int kc = k < K ? k : K - 16;
-                q[i] = __ldg(reinterpret_cast<const uint4*>(Wq + static_cast<size_t>(nc) * K + kc));
+                const int kc = k < K ? k : K - kCodes;
+                q[i] = __ldg(reinterpret_cast<const uint4*>(Wq + static_cast<size_t>(nc) * row_bytes +
+                                                            (W4 ? kc / 2 : kc)));
                 sc[i] = __ldg(sw + nc);
             }
         };
@@ -369,14 +375,30 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
                 for (int i = 0; i < kPerLane; ++i) {
                     const int c = dw * 32 + lane + i * 32 * kDqWarps;
                     const int nr = c / kChunksPerRow;   // contraction row within the stage
-                    const int kc = c % kChunksPerRow;   // 16 output columns
+                    const int kc = c % kChunksPerRow;   // kCodes output columns
+                    const float scale = (inb[u] >> i) & 1u ? sr[u][i] : 0.f;
+                    const int mn = kc * kCodes;
                     uint32_t o[8];
-                    dequant16(qr[u][i], (inb[u] >> i) & 1u ? sr[u][i] : 0.f, o);
-                    const int mn = kc * 16;
-                    *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn, nr, kLbo)) =
-                        make_uint4(o[0], o[1], o[2], o[3]);
-                    *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn + 8, nr, kLbo)) =
-                        make_uint4(o[4], o[5], o[6], o[7]);
+                    if constexpr (W4) {
+                        uint4 lo, hi;
+                        unpack_int4x32(qr[u][i], lo, hi);
+                        dequant16(lo, scale, o);
+                        *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn, nr, kLbo)) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
+                        *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn + 8, nr, kLbo)) =
+                            make_uint4(o[4], o[5], o[6], o[7]);
+                        dequant16(hi, scale, o);
+                        *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn + 16, nr, kLbo)) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
+                        *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn + 24, nr, kLbo)) =
+                            make_uint4(o[4], o[5], o[6], o[7]);
+                    } else {
+                        dequant16(qr[u][i], scale, o);
+                        *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn, nr, kLbo)) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
+                        *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn + 8, nr, kLbo)) =
+                            make_uint4(o[4], o[5], o[6], o[7]);
+                    }
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -500,11 +522,11 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
     }
 }
 
-template <int MSUB, int BN, int RMAX>
+template <int MSUB, int BN, int RMAX, bool W4>
 cudaError_t launch_tc(const void* dY, const int8_t* Wq, const float* sw, int M, int N, int K,
                       const DxEpilogue& ep, int* status, cudaStream_t s) {
     using C = K3Cfg<MSUB, BN, RMAX>;
-    auto kern = k3_dx_dequant_kernel<MSUB, BN, RMAX>;
+    auto kern = k3_dx_dequant_kernel<MSUB, BN, RMAX, W4>;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), C::kTotal);
     if (e != cudaSuccess) return e;
     // dY as [row][64-column block][64] (one 3-D box per stage) when the rows
@@ -523,12 +545,21 @@ cudaError_t launch_tc(const void* dY, const int8_t* Wq, const float* sw, int M, 
                     status);
 }
 
-template <int RMAX>
+template <int RMAX, bool W4>
 cudaError_t launch_tc_cfg(int cfg, const void* dY, const int8_t* Wq, const float* sw, int M, int N,
                           int K, const DxEpilogue& ep, int* status, cudaStream_t s) {
-    if (cfg == 0) return launch_tc<2, 128, RMAX>(dY, Wq, sw, M, N, K, ep, status, s);
-    if (cfg == 1) return launch_tc<1, 128, RMAX>(dY, Wq, sw, M, N, K, ep, status, s);
-    return launch_tc<1, 64, RMAX>(dY, Wq, sw, M, N, K, ep, status, s);
+    if (cfg == 0) return launch_tc<2, 128, RMAX, W4>(dY, Wq, sw, M, N, K, ep, status, s);
+    if (cfg == 1) return launch_tc<1, 128, RMAX, W4>(dY, Wq, sw, M, N, K, ep, status, s);
+    return launch_tc<1, 64, RMAX, W4>(dY, Wq, sw, M, N, K, ep, status, s);
+}
+
+template <bool W4>
+cudaError_t launch_tc_r(int cfg, const void* dY, const int8_t* Wq, const float* sw, int M, int N,
+                        int K, const DxEpilogue& ep, int* status, cudaStream_t s) {
+    if (ep.r <= 4) return launch_tc_cfg<4, W4>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
+    if (ep.r <= 8) return launch_tc_cfg<8, W4>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
+    if (ep.r <= 16) return launch_tc_cfg<16, W4>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
+    return launch_tc_cfg<64, W4>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
 }
 
 // ---------------------------------------------------------------- SIMT path
@@ -538,7 +569,7 @@ cudaError_t launch_tc_cfg(int cfg, const void* dY, const int8_t* Wq, const float
 constexpr int kSB = 64;
 constexpr int kSN = 16;
 
-template <typename T>
+template <typename T, bool W4>
 __global__ void __launch_bounds__(256) k3_dx_simt_kernel(const T* __restrict__ dY,
                                                          const int8_t* __restrict__ Wq,
                                                          const float* __restrict__ sw, int M,
@@ -561,7 +592,15 @@ __global__ void __launch_bounds__(256) k3_dx_simt_kernel(const T* __restrict__ d
             const int n = n0 + nn, k = k0 + kk;
             float w = 0.f;
             if (n < N && k < K) {
-                w = __fmul_rn(static_cast<float>(Wq[static_cast<size_t>(n) * K + k]), __ldg(sw + n));
+                int code;
+                if constexpr (W4) {
+                    const int b = reinterpret_cast<const uint8_t*>(Wq)[static_cast<size_t>(n) * (K / 2) + k / 2];
+                    const int nib = (k & 1) ? (b >> 4) & 0xF : b & 0xF;
+                    code = nib >= 8 ? nib - 16 : nib;
+                } else {
+                    code = Wq[static_cast<size_t>(n) * K + k];
+                }
+                w = __fmul_rn(static_cast<float>(code), __ldg(sw + n));
                 if constexpr (sizeof(T) == 2) w = __bfloat162float(__float2bfloat16_rn(w));
             }
             sW[nn][kk] = w;
@@ -610,15 +649,19 @@ __global__ void __launch_bounds__(256) k3_dx_simt_kernel(const T* __restrict__ d
 }  // namespace
 
 cudaError_t launch_gemm_dx(Act act, const void* dY, const int8_t* Wq, const float* sw, int M,
-                           int N, int K, const DxEpilogue& ep, int* status, cudaStream_t s) {
+                           int N, int K, const DxEpilogue& ep, int* status, cudaStream_t s, bool w4) {
     const bool tc = act == kBF16 && (N % 8) == 0;
     if (!tc) {
         dim3 grid((K + kSB - 1) / kSB, (M + kSB - 1) / kSB);
         if (act == kBF16)
-            return launch_k(k3_dx_simt_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, 1,
-                            static_cast<const __nv_bfloat16*>(dY), Wq, sw, M, N, K, ep);
-        return launch_k(k3_dx_simt_kernel<float>, grid, dim3(256), 0, s, 1,
-                        static_cast<const float*>(dY), Wq, sw, M, N, K, ep);
+            return w4 ? launch_k(k3_dx_simt_kernel<__nv_bfloat16, true>, grid, dim3(256), 0, s, 1,
+                                 static_cast<const __nv_bfloat16*>(dY), Wq, sw, M, N, K, ep)
+                      : launch_k(k3_dx_simt_kernel<__nv_bfloat16, false>, grid, dim3(256), 0, s, 1,
+                                 static_cast<const __nv_bfloat16*>(dY), Wq, sw, M, N, K, ep);
+        return w4 ? launch_k(k3_dx_simt_kernel<float, true>, grid, dim3(256), 0, s, 1,
+                             static_cast<const float*>(dY), Wq, sw, M, N, K, ep)
+                  : launch_k(k3_dx_simt_kernel<float, false>, grid, dim3(256), 0, s, 1,
+                             static_cast<const float*>(dY), Wq, sw, M, N, K, ep);
     }
     // tile shape: the least estimated main-loop time, i.e. waves of
     // persistent CTAs x stages per tile x the measured pace of one stage on
@@ -637,10 +680,8 @@ cudaError_t launch_gemm_dx(Act act, const void* dY, const int8_t* Wq, const floa
     else if (c0 < c2 && c0 < c1) cfg = 0;
     const int forced = tile_override("QLORA_DX_TILE");  // tuning: 0, 1 or 2
     if (forced >= 0 && forced <= 2) cfg = forced;
-    if (ep.r <= 4) return launch_tc_cfg<4>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
-    if (ep.r <= 8) return launch_tc_cfg<8>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
-    if (ep.r <= 16) return launch_tc_cfg<16>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
-    return launch_tc_cfg<64>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
+    return w4 ? launch_tc_r<true>(cfg, dY, Wq, sw, M, N, K, ep, status, s)
+              : launch_tc_r<false>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
 }
 
 }  // namespace qlora

@@ -375,6 +375,34 @@ __device__ __forceinline__ float sum_slices(const float* __restrict__ p, size_t 
 
 // Symmetric abs-max int8 code: clamp(rne(v * inv), -127, 127), fp32 product
 // rounded once.
+// 32 packed int4 codes (16 bytes; byte j holds code 2j in its low nibble and
+// code 2j+1 in its high nibble, two's complement) -> the same 32 codes as
+// int8 bytes in order (lo: codes 0..15, hi: codes 16..31).  Each nibble is
+// sign-extended within its byte ((x ^ 8) - 8, byte-wise), then the low and
+// high nibbles of each byte are interleaved back into k order.
+__device__ __forceinline__ void unpack_int4x32(const uint4 raw, uint4& lo, uint4& hi) {
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t ev = __vsub4((w[i] & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);
+        const uint32_t od = __vsub4(((w[i] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);
+        o[2 * i] = __byte_perm(ev, od, 0x5140);
+        o[2 * i + 1] = __byte_perm(ev, od, 0x7362);
+    }
+    lo = make_uint4(o[0], o[1], o[2], o[3]);
+    hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// Symmetric abs-max code with L levels on each side: clamp(rne(v * inv), -L, L).
+template <int L>
+__device__ __forceinline__ int quant_code_l(float v, float inv) {
+    int q = __float2int_rn(__fmul_rn(v, inv));
+    q = q > L ? L : q;
+    q = q < -L ? -L : q;
+    return q;
+}
+
 __device__ __forceinline__ int quant_code(float v, float inv) {
     int q = __float2int_rn(__fmul_rn(v, inv));
     q = q > 127 ? 127 : q;

@@ -442,9 +442,12 @@ int qlora_lora_grad_b(const qlora_layer_desc* d, int M, const void* dY, const fl
 
 static int gemm_dx_impl(const qlora_layer_desc* d, int M, const void* dY, const int8_t* Wq,
                         const float* sw, const float* A, const void* gate, void* dX,
-                        const void* workspace, size_t workspace_bytes, void* stream) {
+                        const void* workspace, size_t workspace_bytes, void* stream,
+                        bool w4 = false) {
     int rc = check_layer(d, M);
     if (rc != QLORA_OK) return rc;
+    QL_REQUIRE(!w4 || d->K % 32 == 0, QLORA_EUNSUPPORTED,
+               "packed int4 kernels need K a multiple of 32 (16-byte rows of codes)");
     QL_REQUIRE(dY && Wq && sw && A && dX && workspace, QLORA_EINVAL, "NULL pointer argument");
     QL_REQUIRE(aligned(dY, 16) && aligned(Wq, 16) && aligned(dX, 16) && aligned(workspace, 256),
                QLORA_EALIGN, "dY, Wq and dX must be 16-byte aligned, workspace 256-byte aligned");
@@ -463,7 +466,7 @@ static int gemm_dx_impl(const qlora_layer_desc* d, int M, const void* dY, const 
     ep.dX = dX;
     ep.gate = gate;
     return cuda_status(launch_gemm_dx(act_of(d), dY, Wq, sw, M, d->N, d->K, ep, status,
-                                      static_cast<cudaStream_t>(stream)),
+                                      static_cast<cudaStream_t>(stream), w4),
                        "dX GEMM launch");
 }
 
@@ -584,6 +587,60 @@ int qlora_merge(const qlora_layer_desc* d, const int8_t* Wq, const float* sw, co
     return cuda_status(launch_merge(Wq, sw, A, B, d->K, d->N, d->r, c, Wq_out, sw_out,
                                     static_cast<cudaStream_t>(stream)),
                        "merge launch");
+}
+
+// ---------------------------------------------------------------------------
+// packed int4 kernels
+// ---------------------------------------------------------------------------
+static int check_int4_shape(int K, int N) {
+    if (K < 1 || N < 1) return fail(QLORA_ESHAPE, "K and N must be >= 1");
+    if (K % 32 != 0)
+        return fail(QLORA_EUNSUPPORTED, "packed int4 kernels need K a multiple of 32 (16-byte rows of codes)");
+    return QLORA_OK;
+}
+
+int qlora_quantize_weight_int4(const float* W, int K, int N, uint8_t* Wp, float* sw, void* stream) {
+    if (!W || !Wp || !sw) return fail(QLORA_EINVAL, "NULL pointer argument");
+    int rc = check_int4_shape(K, N);
+    if (rc != QLORA_OK) return rc;
+    if (!aligned(W, 4) || !aligned(sw, 4) || !aligned(Wp, 16))
+        return fail(QLORA_EALIGN, "misaligned pointer (W, sw 4 B; Wp 16 B)");
+    return cuda_status(launch_quantize_weight_int4(W, K, N, Wp, sw, static_cast<cudaStream_t>(stream)),
+                       "quantize_weight_int4 launch");
+}
+
+int qlora_unpack_int4(const uint8_t* Wp, int K, int N, int8_t* Wq, void* stream) {
+    if (!Wp || !Wq) return fail(QLORA_EINVAL, "NULL pointer argument");
+    int rc = check_int4_shape(K, N);
+    if (rc != QLORA_OK) return rc;
+    if (!aligned(Wp, 16) || !aligned(Wq, 16)) return fail(QLORA_EALIGN, "Wp and Wq must be 16-byte aligned");
+    return cuda_status(launch_unpack_int4(Wp, K, N, Wq, static_cast<cudaStream_t>(stream)),
+                       "unpack_int4 launch");
+}
+
+int qlora_gemm_dx_int4(const qlora_layer_desc* d, int M, const void* dY, const uint8_t* Wp,
+                       const float* sw, const float* A, void* dX, const void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    return gemm_dx_impl(d, M, dY, reinterpret_cast<const int8_t*>(Wp), sw, A, nullptr, dX, workspace,
+                        workspace_bytes, stream, true);
+}
+
+int qlora_merge_int4(const qlora_layer_desc* d, const uint8_t* Wp, const float* sw, const float* A,
+                     const float* B, uint8_t* Wp_out, float* sw_out, void* stream) {
+    int rc = check_desc(d);
+    if (rc != QLORA_OK) return rc;
+    rc = check_int4_shape(d->K, d->N);
+    if (rc != QLORA_OK) return rc;
+    if (!Wp || !sw || !A || !B || !Wp_out || !sw_out) return fail(QLORA_EINVAL, "NULL pointer argument");
+    if (!aligned(Wp, 16) || !aligned(Wp_out, 16))
+        return fail(QLORA_EALIGN, "Wp and Wp_out must be 16-byte aligned");
+    if (!aligned(sw, 4) || !aligned(A, 4) || !aligned(B, 4) || !aligned(sw_out, 4))
+        return fail(QLORA_EALIGN, "fp32 vectors must be 4-byte aligned");
+    if (Wp_out == Wp || sw_out == sw) return fail(QLORA_EINVAL, "merge outputs alias its inputs");
+    const float c = d->alpha / static_cast<float>(d->r);
+    return cuda_status(launch_merge_int4(Wp, sw, A, B, d->K, d->N, d->r, c, Wp_out, sw_out,
+                                         static_cast<cudaStream_t>(stream)),
+                       "merge_int4 launch");
 }
 
 int qlora_selftest_wait_timeout(unsigned int limit_us, void* stream) {

@@ -32,7 +32,8 @@ EXPORTED = ("qlora_quantize_weight", "qlora_workspace_bytes", "qlora_forward",
             "qlora_gemm_forward", "qlora_lora_grad_dy", "qlora_gemm_dx", "qlora_lora_grad_x",
             "qlora_selftest_wait_timeout", "qlora_backward_noalloc", "qlora_lora_g",
             "qlora_lora_grad_b", "qlora_gemm_forward_relu", "qlora_gemm_dx_relu",
-            "qlora_set_rank_pass_rows")
+            "qlora_set_rank_pass_rows", "qlora_quantize_weight_int4", "qlora_unpack_int4",
+            "qlora_gemm_dx_int4", "qlora_merge_int4")
 
 
 class QLoraError(RuntimeError):
@@ -93,6 +94,13 @@ def _load():
     for f in (lib.qlora_quantize_input, lib.qlora_gemm_forward, lib.qlora_lora_grad_dy,
               lib.qlora_lora_g, lib.qlora_lora_grad_b, lib.qlora_gemm_dx, lib.qlora_lora_grad_x,
               lib.qlora_gemm_forward_relu, lib.qlora_gemm_dx_relu):
+        f.restype = I
+    lib.qlora_quantize_weight_int4.argtypes = [P, I, I, P, P, P]
+    lib.qlora_unpack_int4.argtypes = [P, I, I, P, P]
+    lib.qlora_gemm_dx_int4.argtypes = [D, I, P, P, P, P, P, P, Z, P]
+    lib.qlora_merge_int4.argtypes = [D, P, P, P, P, P, P, P]
+    for f in (lib.qlora_quantize_weight_int4, lib.qlora_unpack_int4, lib.qlora_gemm_dx_int4,
+              lib.qlora_merge_int4):
         f.restype = I
     lib.qlora_set_rank_pass_rows.argtypes = [I]
     lib.qlora_set_rank_pass_rows.restype = I
@@ -249,6 +257,38 @@ def qlora_gemm_dx(d: LayerDesc, M: int, dY, Wq, sw, A, dX, ws, stream=None):
 def qlora_lora_grad_x(d: LayerDesc, M: int, X, dA, ws, stream=None):
     _check(_lib.qlora_lora_grad_x(ctypes.byref(d), int(M), _ptr(X), _ptr(dA), _ptr(ws), ws.numel(),
                                   _stream(stream)))
+
+
+def quantize_weight_int4(W: torch.Tensor, stream=None):
+    """W [K, N] fp32 -> (Wp [N, K/2] uint8 packed int4 codes, sw [N] fp32)."""
+    K, N = W.shape
+    W = W.float().contiguous()
+    Wp = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    sw = torch.empty((N,), dtype=torch.float32, device=W.device)
+    _check(_lib.qlora_quantize_weight_int4(_ptr(W), K, N, _ptr(Wp), _ptr(sw), _stream(stream)))
+    return Wp, sw
+
+
+def unpack_int4(Wp: torch.Tensor, stream=None) -> torch.Tensor:
+    """Wp [N, K/2] -> int8 codes [N, K] (the forward's Wq)."""
+    N, K2 = Wp.shape
+    Wq = torch.empty((N, 2 * K2), dtype=torch.int8, device=Wp.device)
+    _check(_lib.qlora_unpack_int4(_ptr(Wp), 2 * K2, N, _ptr(Wq), _stream(stream)))
+    return Wq
+
+
+def qlora_gemm_dx_int4(d: LayerDesc, M: int, dY, Wp, sw, A, dX, ws, stream=None):
+    _check(_lib.qlora_gemm_dx_int4(ctypes.byref(d), int(M), _ptr(dY), _ptr(Wp), _ptr(sw), _ptr(A),
+                                   _ptr(dX), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def merge_int4(d: LayerDesc, Wp, sw, A, B, stream=None):
+    """Lossy merge of an int4 layer -> (Wp' [N, K/2], sw' [N])."""
+    Wp2 = torch.empty_like(Wp)
+    sw2 = torch.empty_like(sw)
+    _check(_lib.qlora_merge_int4(ctypes.byref(d), _ptr(Wp), _ptr(sw), _ptr(A), _ptr(B), _ptr(Wp2),
+                                 _ptr(sw2), _stream(stream)))
+    return Wp2, sw2
 
 
 def qlora_set_rank_pass_rows(rows: int) -> int:

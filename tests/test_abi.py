@@ -14,7 +14,7 @@ def _header_functions():
     with open(os.path.join(ROOT, "include", "qlora.h")) as f:
         text = f.read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(qlora_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(qlora_[a-z0-9_]+)\s*\(", text)))
 
 
 @pytest.fixture(scope="module")
@@ -125,3 +125,25 @@ def test_rank_pass_rows_setting(q):
     assert lib.qlora_set_rank_pass_rows(-1) == -1
     assert b"rows per CTA" in lib.qlora_last_error()
     assert lib.qlora_set_rank_pass_rows(0) == 0
+
+
+def test_int4_calls_reject_bad_arguments(q):
+    """The packed int4 calls need K a multiple of 32 and 16-byte aligned code
+    buffers; they refuse anything else before launching (fake pointers)."""
+    import torch
+    P = ctypes.c_void_p
+    lib = q.lib()
+    assert lib.qlora_quantize_weight_int4(P(0x1000), 48, 8, P(0x2000), P(0x3000), None) == -5
+    assert lib.qlora_quantize_weight_int4(P(0x1000), 64, 8, P(0x2008), P(0x3000), None) == -2
+    assert lib.qlora_quantize_weight_int4(None, 64, 8, P(0x2000), P(0x3000), None) == -1
+    assert lib.qlora_unpack_int4(P(0x1000), 80, 8, P(0x2000), None) == -5
+    assert lib.qlora_unpack_int4(P(0x1000), 64, 8, P(0x2004), None) == -2
+    d = q.desc(784, 128, 4, 4.0, torch.bfloat16)  # K % 32 == 16
+    assert lib.qlora_merge_int4(ctypes.byref(d), P(0x1000), P(0x2000), P(0x3000), P(0x4000),
+                                P(0x5000), P(0x6000), None) == -5
+    assert lib.qlora_gemm_dx_int4(ctypes.byref(d), 64, P(0x1000), P(0x2000), P(0x3000), P(0x4000),
+                                  P(0x5000), P(0x6000), 1 << 30, None) == -5
+    assert b"multiple of 32" in lib.qlora_last_error()
+    d = q.desc(1024, 128, 4, 4.0, torch.bfloat16)
+    assert lib.qlora_merge_int4(ctypes.byref(d), P(0x1000), P(0x2000), P(0x3000), P(0x4000),
+                                P(0x1000), P(0x6000), None) == -1  # output aliases input

@@ -380,3 +380,82 @@ def test_relu_kernels(q):
             torch.cuda.synchronize()
             assert torch.equal(y.float(), ref)
             assert torch.equal(g.float(), (ref > 0).float())
+
+
+# ---------------------------------------------------------------- packed int4
+@pytest.mark.parametrize("K,N", [(1024, 1024), (768, 2304), (32, 10), (4096, 136)])
+def test_int4_quantize_and_unpack_bit_exact(q, K, N):
+    """The int4 quantizer and the unpack kernel against the oracle, byte for
+    byte, on heavy-tailed kernels with a zero channel and exact .5 ties."""
+    rng = np.random.Generator(np.random.PCG64(K + 3 * N))
+    W = (rng.standard_t(3, (K, N)) * 0.02).astype(np.float32)
+    W[:, 0] = 0.0
+    if N > 2:
+        W[:, 1] = 0.0
+        W[:4, 1] = np.array([7 / 8, 2.5 / 8, -3.5 / 8, 0.5 / 8], np.float32)
+    Wp, sw = q.quantize_weight_int4(torch.from_numpy(W).cuda())
+    Wq = q.unpack_int4(Wp)
+    torch.cuda.synchronize()
+    Wp_o, sw_o = oracle.quantize_weight_int4(W)
+    np.testing.assert_array_equal(Wp.cpu().numpy(), Wp_o)
+    np.testing.assert_array_equal(to_np(sw).view(np.uint32), sw_o.view(np.uint32))
+    np.testing.assert_array_equal(Wq.cpu().numpy(), oracle.unpack_int4(Wp_o))
+
+
+@pytest.mark.parametrize("M,K,N,r,act", [(1024, 1024, 1024, 8, "bf16"),   # 128x64 tiles
+                                          (333, 768, 2304, 4, "bf16"),
+                                          (1000, 1312, 264, 8, "bf16"),   # 128x128 tiles
+                                          (4096, 768, 768, 4, "bf16"),    # 256x128 tiles
+                                          (96, 256, 10, 8, "bf16"),       # CUDA-core dX
+                                          (64, 256, 128, 4, "f32")])      # fp32 activations
+def test_int4_layer_matches_oracle(q, M, K, N, r, act):
+    """An int4 layer: forward on the unpacked codes (accumulator bit-exact), dX
+    from the packed codes bit-identical to the int8 path on the unpacked codes
+    and within tolerance of the oracle, dA/dB/dbias against the oracle, and
+    the int4 merge bit-exact."""
+    spec = _edge_spec(M, K, N, r, act=act, seed=5 * M + K)
+    d = inputs.layer_inputs(spec)
+    from parity import act_torch
+    tdt = act_torch(act)
+    Wp, sw = q.quantize_weight_int4(torch.from_numpy(d["W"]).cuda())
+    Wq8 = q.unpack_int4(Wp)
+    layer = q.Layer(Wq=Wq8, sw=sw, bias=torch.from_numpy(d["bias"]).cuda(),
+                    A=torch.from_numpy(d["A"]).cuda(), B=torch.from_numpy(d["B"]).cuda(),
+                    alpha=spec.alpha, act=tdt)
+    D = layer.desc()
+    X = torch.from_numpy(d["X"]).to(tdt).cuda()
+    dY = torch.from_numpy(d["dY"]).to(tdt).cuda()
+    ws = q.workspace(D, M)
+    Y, xA, (xq, sx, acc) = q.forward(layer, X, ws, debug=True)
+    dB = torch.empty((r, N), device="cuda")
+    db = torch.empty((N,), device="cuda")
+    q.qlora_lora_grad_dy(D, M, dY, layer.B, xA, dB, db, ws)
+    dX4 = torch.full((M, K), float("nan"), dtype=tdt, device="cuda")
+    dX8 = torch.empty((M, K), dtype=tdt, device="cuda")
+    q.qlora_gemm_dx_int4(D, M, dY, Wp, sw, layer.A, dX4, ws)
+    q.qlora_gemm_dx(D, M, dY, Wq8, sw, layer.A, dX8, ws)
+    dA = torch.empty((K, r), device="cuda")
+    q.qlora_lora_grad_x(D, M, X, dA, ws)
+    Wp2, sw2 = q.merge_int4(D, Wp, sw, layer.A, layer.B)
+    torch.cuda.synchronize()
+    assert q.qlora_device_status() == 0
+    assert torch.equal(dX4, dX8)
+
+    Wp_o, sw_o = oracle.quantize_weight_int4(d["W"])
+    codes = oracle.unpack_int4(Wp_o)
+    rows = np.arange(M) if M <= 1024 else np.unique(np.concatenate(
+        [[0, M - 1], np.random.Generator(np.random.PCG64(M)).choice(M, 192, replace=False)]))
+    f = oracle.forward(d["X"][rows], codes, sw_o, d["bias"], d["A"], d["B"], spec.alpha)
+    np.testing.assert_array_equal(to_np(acc)[rows], f["acc"])
+    assert_close(to_np(Y)[rows], f["y"], act, "Y")
+    b_rows = oracle.backward(d["X"][rows], d["dY"][rows], codes, sw_o, d["A"], d["B"], spec.alpha,
+                             want_dx=True, act=act)
+    assert_close(to_np(dX4)[rows], b_rows["dX"], act, "dX (int4)")
+    b_full = oracle.backward(d["X"], d["dY"], codes, sw_o, d["A"], d["B"], spec.alpha,
+                             want_dx=False, act=act)
+    assert_close(to_np(dA), b_full["dA"], act, "dA")
+    assert_close(to_np(dB), b_full["dB"], act, "dB")
+    assert_close(to_np(db), b_full["dbias"], act, "dbias")
+    Wp2_o, sw2_o = oracle.merge_int4(Wp_o, sw_o, d["A"], d["B"], spec.alpha)
+    np.testing.assert_array_equal(Wp2.cpu().numpy(), Wp2_o)
+    np.testing.assert_array_equal(to_np(sw2).view(np.uint32), sw2_o.view(np.uint32))
