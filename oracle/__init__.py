@@ -22,6 +22,10 @@ What each routine follows (page title, section):
     through the input quantizer.
   * merge -- Keras PR 19356 Results footnote (lossy merge) and the 4-bit
     thread (de-quantize, add the LoRA, re-quantize).
+  * quantize_outlier_int8 / dequantize_outlier_int8 / percentile / round_fp16
+    -- outlier-compensated int8 kernels: keras-llm-light, "Weights
+    quantization" and "Simplified Int8Variable quantization"; the readings
+    are in the C file.
   * quantize_weight_int4 / unpack_int4 / merge_int4 -- packed 4-bit kernels:
     keras-llm-light, "Simplified Int4Variable quantization" (two int4 values
     per int8 byte) and the 4-bit thread; the readings are in the C file.
@@ -82,6 +86,13 @@ def _lib():
             lib.orc_quantize_weight_int4.argtypes = [P, L, L, P, P]
             lib.orc_unpack_int4.argtypes = [P, L, L, P]
             lib.orc_merge_int4.argtypes = [P, P, P, P, L, L, L, F, P, P]
+            lib.orc_percentile.argtypes = [P, L, D]
+            lib.orc_percentile.restype = D
+            lib.orc_round_fp16.argtypes = [D]
+            lib.orc_round_fp16.restype = D
+            lib.orc_quantize_outlier_int8.argtypes = [P, L, P, P, P, P]
+            lib.orc_quantize_outlier_int8.restype = L
+            lib.orc_dequantize_outlier_int8.argtypes = [P, P, P, L, F, F, P]
             lib.orc_round_bf16.argtypes = [D]
             lib.orc_round_bf16.restype = D
             lib.orc_round_bf16_array.argtypes = [P, L, P]
@@ -262,6 +273,46 @@ def merge_int4(Wp, sw, A, B, alpha):
     sw2 = np.empty_like(sw)
     _lib().orc_merge_int4(_p(Wq), _p(sw), _p(A), _p(B), K, N, r, float(c), _p(Wp2), _p(sw2))
     return Wp2, sw2
+
+
+# --------------------------------------------------------------------------
+# outlier-compensated int8 kernels (keras-llm-light; readings in the C file)
+# --------------------------------------------------------------------------
+def percentile(v, p):
+    """Percentile p of the entries of v (linear interpolation), fp64."""
+    v = _c(np.asarray(v).ravel(), np.float32)
+    return float(_lib().orc_percentile(_p(v), v.size, float(p)))
+
+
+def round_fp16(x):
+    """Round an fp64 value to the nearest IEEE half, ties to even, as fp64."""
+    return float(_lib().orc_round_fp16(float(x)))
+
+
+def quantize_outlier_int8(W):
+    """W (any shape) float32 -> dict of codes (uint8, W's shape), is_outlier
+    (bool), outlier values (fp16 values as float32, 0 elsewhere), lo, hi,
+    scale, bias and the outlier count."""
+    W = _c(W, np.float32)
+    n = W.size
+    codes = np.empty(W.shape, np.uint8)
+    is_out = np.empty(W.shape, np.uint8)
+    vals = np.empty(W.shape, np.float32)
+    par = np.empty(4, np.float32)
+    count = _lib().orc_quantize_outlier_int8(_p(W), n, _p(codes), _p(is_out), _p(vals), _p(par))
+    return {"codes": codes, "is_outlier": is_out.astype(bool), "values": vals, "lo": par[0],
+            "hi": par[1], "scale": par[2], "bias": par[3], "count": int(count)}
+
+
+def dequantize_outlier_int8(q):
+    """The rebuilt fp32 kernel of a quantize_outlier_int8 result."""
+    codes = _c(q["codes"], np.uint8)
+    is_out = _c(q["is_outlier"].astype(np.uint8), np.uint8)
+    vals = _c(q["values"], np.float32)
+    W = np.empty(codes.shape, np.float32)
+    _lib().orc_dequantize_outlier_int8(_p(codes), _p(is_out), _p(vals), codes.size,
+                                       float(q["scale"]), float(q["bias"]), _p(W))
+    return W
 
 
 def round_bf16(x):

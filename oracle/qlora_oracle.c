@@ -385,6 +385,110 @@ void orc_merge_int4(const int8_t* Wq, const float* sw, const float* A, const flo
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* Outlier-compensated int8 kernels (keras-llm-light, "Weights               */
+/* quantization" and "Simplified Int8Variable quantization": a simplified    */
+/* LLM.int8(); the weights are quantized after removing outliers with a 99.9 */
+/* percentile cutoff, the outliers are kept in a sparse (row, col, value)    */
+/* list in fp16, and the kernel is rebuilt as bias + value * scale with the  */
+/* outliers written back; the block summary stores such kernels as uint8).   */
+/* Readings where the pages are silent:                                      */
+/*   - one affine code per tensor: lo and hi are the 0.1th and 99.9th        */
+/*     percentiles of all entries (linear interpolation between order        */
+/*     statistics, in fp64, then stored as fp32);                            */
+/*   - outliers are the entries strictly below lo or strictly above hi;     */
+/*     they are stored as fp16 (round to nearest even);                      */
+/*   - scale = fl32((hi - lo) / 255), bias = lo, and every other entry gets  */
+/*     value = clamp(rne(fl32(fl32(w - bias) / scale)), 0, 255) (0 when      */
+/*     scale == 0);                                                          */
+/*   - rebuilt entry = fl32(bias + fl32(value * scale)), or the outlier's    */
+/*     fp16 value widened to fp32.                                           */
+/* ------------------------------------------------------------------------ */
+static int cmp_float(const void* a, const void* b) {
+    float x = *(const float*)a, y = *(const float*)b;
+    return (x > y) - (x < y);
+}
+
+/* Percentile p (in [0, 100]) of n floats, linear interpolation between the
+ * order statistics at position (n - 1) * p / 100. */
+double orc_percentile(const float* v, long n, double p) {
+    float* s = (float*)malloc(sizeof(float) * (size_t)n);
+    memcpy(s, v, sizeof(float) * (size_t)n);
+    qsort(s, (size_t)n, sizeof(float), cmp_float);
+    double h = (double)(n - 1) * p / 100.0;
+    long i = (long)floor(h);
+    if (i >= n - 1) i = n - 1;
+    double frac = h - (double)i;
+    double q = (double)s[i];
+    if (i + 1 < n && frac > 0.0) q += frac * ((double)s[i + 1] - (double)s[i]);
+    free(s);
+    return q;
+}
+
+/*
+ * Round an fp64 value to the nearest IEEE half (11-bit significand, normal
+ * range from 2^-14, subnormal quantum 2^-24), ties to even, as fp64.
+ */
+double orc_round_fp16(double x) {
+    if (x == 0.0 || !isfinite(x)) return x;
+    int e;
+    frexp(x, &e);                 /* |x| in [2^(e-1), 2^e) */
+    if (e - 1 < -14) e = -13;     /* subnormal range: fixed quantum 2^-24 */
+    double ulp = ldexp(1.0, e - 11);
+    double q = rint(x / ulp) * ulp;
+    if (fabs(q) > 65504.0) q = copysign(INFINITY, x);
+    return q;
+}
+
+/*
+ * W [n] fp32 -> codes [n] uint8, outlier flags [n] (0, or 1 for an outlier),
+ * outlier values [n] (fp16 values as fp32, 0 elsewhere), and
+ * par = {lo, hi, scale, bias}.  Returns the number of outliers.
+ */
+long orc_quantize_outlier_int8(const float* W, long n, uint8_t* codes, uint8_t* is_out,
+                               float* out_val, float* par) {
+    float lo = (float)orc_percentile(W, n, 0.1);
+    float hi = (float)orc_percentile(W, n, 99.9);
+    float scale = (hi - lo) / 255.0f;
+    float bias = lo;
+    long count = 0;
+    for (long i = 0; i < n; ++i) {
+        float w = W[i];
+        if (w < lo || w > hi) {
+            is_out[i] = 1;
+            out_val[i] = (float)orc_round_fp16((double)w);
+            codes[i] = 0;
+            ++count;
+            continue;
+        }
+        is_out[i] = 0;
+        out_val[i] = 0.0f;
+        float r = 0.0f;
+        if (scale > 0.0f) {
+            float d = w - bias;           /* one fp32 rounding */
+            float t = d / scale;          /* one fp32 rounding */
+            r = rintf(t);
+            if (r < 0.0f) r = 0.0f;
+            if (r > 255.0f) r = 255.0f;
+        }
+        codes[i] = (uint8_t)r;
+    }
+    par[0] = lo;
+    par[1] = hi;
+    par[2] = scale;
+    par[3] = bias;
+    return count;
+}
+
+/* Rebuilds the kernel: bias + value * scale, outliers written back. */
+void orc_dequantize_outlier_int8(const uint8_t* codes, const uint8_t* is_out, const float* out_val,
+                                 long n, float scale, float bias, float* W) {
+    for (long i = 0; i < n; ++i) {
+        float v = (float)codes[i] * scale;   /* one fp32 rounding */
+        W[i] = is_out[i] ? out_val[i] : bias + v;
+    }
+}
+
 /*
  * Round an fp64 value to the nearest bfloat16 (8-bit significand, the fp32
  * exponent range), ties to even, returned as fp64.  Used where a layer's

@@ -638,3 +638,82 @@ def test_int4_merge_of_a_rank_one_power_of_two_adapter():
     for n in range(N):
         np.testing.assert_array_equal(q[n], want * int(np.sign(b[n])))
         assert sw2[n] == np.float32(np.float32(2.0 * abs(b[n]) * 1.0) / np.float32(7.0))
+
+
+# --------------------------------------------------------------------------
+# outlier-compensated int8 kernels
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("p", [0.1, 99.9, 50.0, 0.0, 100.0, 37.25])
+def test_percentile_is_numpys_linear_percentile(p):
+    """The cutoffs use the order-statistic interpolation that numpy's
+    percentile uses by default."""
+    rng = _rng(21)
+    for n in (1, 2, 999, 1001, 5000):
+        v = rng.normal(0, 1, n).astype(np.float32)
+        assert oracle.percentile(v, p) == pytest.approx(np.percentile(v.astype(np.float64), p),
+                                                        rel=1e-12, abs=1e-12)
+
+
+def test_round_fp16_is_ieee_half():
+    """Round to nearest even into IEEE half: numpy's float16 conversion, on
+    normal values, exact ties, subnormals and overflow."""
+    rng = _rng(22)
+    xs = list(rng.normal(0, 100, 2000)) + list(rng.normal(0, 1e-5, 500))
+    xs += [1 + 2 ** -11, 1 + 3 * 2 ** -11, 2 ** -24 * 1.5, 2 ** -25, 65504.0, 65520.0, 1e6,
+           -2 ** -14 * (1 + 2 ** -10), 0.0]
+    with np.errstate(over="ignore"):  # 65520 and 1e6 overflow to inf, as they should
+        for x in xs:
+            assert oracle.round_fp16(x) == float(np.float16(x)), x
+
+
+def _order_stat_outliers(n):
+    """Entries strictly outside the 0.1th / 99.9th percentiles of n distinct
+    values, per side: with h = (n - 1) / 1000, floor(h) + 1 when h is not an
+    integer (the cutoff lies strictly between two order statistics), h when
+    it is (the cutoff is an order statistic)."""
+    h = (n - 1) / 1000
+    return int(h) + 1 if h != int(h) else int(h)
+
+
+@pytest.mark.parametrize("n", [500, 1001, 3200, 20001])
+def test_outlier_count_and_exact_outliers(n):
+    """The number of outliers matches the order-statistic count on both
+    sides, the outliers come back as their fp16 values, and every other entry
+    comes back within half a step (scale / 2) of itself, with codes in
+    [0, 255]."""
+    rng = _rng(23 + n)
+    W = (rng.standard_t(3, n) * 0.05).astype(np.float32)
+    q = oracle.quantize_outlier_int8(W)
+    assert q["count"] == 2 * _order_stat_outliers(n)
+    R = oracle.dequantize_outlier_int8(q)
+    o = q["is_outlier"]
+    assert (W[o] < q["lo"]).sum() == _order_stat_outliers(n)
+    np.testing.assert_array_equal(R[o], np.array([float(np.float16(w)) for w in W[o]], np.float32))
+    err = np.abs(R[~o].astype(np.float64) - W[~o])
+    assert (err <= float(q["scale"]) * (0.5 + 2 ** -16) + 2 ** -22 * np.abs(W[~o])).all()
+    assert q["codes"][o].max(initial=0) == 0
+    assert q["codes"].max() <= 255
+
+
+def test_outlier_cutoffs_that_are_entries_quantize_to_0_and_255():
+    """n = 1001 values: (n - 1) / 1000 = 1, so the cutoffs are the second
+    smallest and second largest entries; they quantize to 0 and 255, and the
+    two extremes are the only outliers."""
+    rng = _rng(24)
+    W = rng.permutation(np.linspace(-1, 1, 1001)).astype(np.float32)
+    W[np.argmin(W)] = -40.0
+    W[np.argmax(W)] = 17.0
+    q = oracle.quantize_outlier_int8(W)
+    s = np.sort(W)
+    assert q["lo"] == s[1] and q["hi"] == s[-2]
+    assert q["count"] == 2 and set(W[q["is_outlier"]].tolist()) == {-40.0, 17.0}
+    assert q["codes"][W == s[1]][0] == 0 and q["codes"][W == s[-2]][0] == 255
+
+
+def test_constant_kernel_has_no_outliers_and_rebuilds_exactly():
+    """All entries equal: both cutoffs are that value, the scale is 0, every
+    code is 0 and the rebuilt kernel is the constant itself."""
+    W = np.full((7, 9), -0.3125, np.float32)
+    q = oracle.quantize_outlier_int8(W)
+    assert q["count"] == 0 and q["scale"] == 0.0 and not q["codes"].any()
+    np.testing.assert_array_equal(oracle.dequantize_outlier_int8(q), W)
