@@ -282,9 +282,9 @@ int qlora_set_rank_pass_rows(int rows);
  * with these codes as its Wq.  K must be a multiple of 32
  * (QLORA_EUNSUPPORTED otherwise); Wp is 16-byte aligned.
  *
- * Forward: expand the codes once with qlora_unpack_int4 into an int8 [N, K]
- * buffer the caller owns and run qlora_forward / qlora_gemm_forward on it
- * (the codes lie in [-7, 7]); the dX GEMM reads the packed codes directly.
+ * qlora_gemm_forward_int4 and qlora_gemm_dx_int4 read the packed codes
+ * directly and expand them in shared memory.  qlora_unpack_int4 gives the
+ * int8 codes for the composite calls (qlora_forward, qlora_backward).
  * ------------------------------------------------------------------------ */
 
 /* a0 for int4: W [K,N] fp32 -> Wp [N, K/2] packed codes, sw [N].  Bit-exact. */
@@ -293,6 +293,16 @@ int qlora_quantize_weight_int4(const float* W, int K, int N, uint8_t* Wp, float*
 
 /* Wp [N, K/2] -> Wq [N, K] int8 codes in [-8, 7] (Wq 16-byte aligned).  Bit-exact. */
 int qlora_unpack_int4(const uint8_t* Wp, int K, int N, int8_t* Wq, void* stream);
+
+/* a2 with packed int4 codes: the int8 GEMM and epilogue of qlora_gemm_forward
+ * on the codes, which dedicated warps expand from Wp into each stage's int8
+ * tile.  Bit-identical to qlora_gemm_forward given the unpacked codes.  It
+ * needs no int8 copy of the kernel, but at K >= 4096 the expansion paces the
+ * stages and it runs at about half the speed of qlora_gemm_forward; there,
+ * qlora_unpack_int4 once followed by qlora_gemm_forward is faster. */
+int qlora_gemm_forward_int4(const qlora_layer_desc* d, int M, const int8_t* Xq, const float* sx,
+                            const uint8_t* Wp, const float* sw, const float* bias, const float* xA,
+                            const float* B, void* Y, int32_t* acc, void* stream);
 
 /* a4 with packed int4 codes: dX = dY (q * sw)^T + c * G A^T, the nibbles
  * de-quantized in shared memory; G from the workspace as qlora_gemm_dx.

@@ -33,8 +33,9 @@ struct FwdEpilogue {
     int relu;           // 1: Y = max(Y, 0) (the ReLU that follows the layer in an MLP)
 };
 // Y = (Xq Wq^T) sx sw + bias + c xA B with the tcgen05 int8 GEMM.
+// w4: Wq holds packed int4 codes [N, K/2] (K % 32 == 0), expanded in shared memory.
 cudaError_t launch_gemm_i8_fwd(Act act, const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
-                               const FwdEpilogue& ep, int* status, cudaStream_t s);
+                               const FwdEpilogue& ep, int* status, cudaStream_t s, bool w4 = false);
 
 // ---------------------------------------------------------------- K3
 struct DxEpilogue {

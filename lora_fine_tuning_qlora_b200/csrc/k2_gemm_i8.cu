@@ -35,6 +35,10 @@ constexpr int kBM = 128;
 constexpr int kBlkK = 128;        // int8 elements per 128-byte swizzle row (one TMA block)
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kUnpackWarps = 4;  // packed int4 kernels: warps that expand the codes per stage
+
+template <bool W4>
+__host__ __device__ constexpr int k2_threads() { return kThreads + (W4 ? 32 * kUnpackWarps : 0); }
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory
 
 template <int BN, typename OutT, int RMAX>
@@ -67,11 +71,15 @@ struct K2Cfg {
     static_assert(kTmemCols <= 512, "TMEM");
 };
 
-template <int BN, typename OutT, int RMAX>
-__global__ void __launch_bounds__(kThreads, 1)
+// W4: the kernel is packed int4 codes Wp [N, K/2] (two per byte, even k in
+// the low nibble) instead of int8 codes behind tmB; warps 10..13 expand each
+// stage's codes into the int8 tile the TMA would have written (128B swizzle,
+// K-major), and the MMA waits for them as well as for the Xq tile.
+template <int BN, typename OutT, int RMAX, bool W4>
+__global__ void __launch_bounds__(k2_threads<W4>(), 1)
     k2_gemm_i8_lora_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmB, int k3d, int M, int N, int K,
-                           FwdEpilogue ep, int* status) {
+                           const uint8_t* __restrict__ Wp, FwdEpilogue ep, int* status) {
     using C = K2Cfg<BN, OutT, RMAX>;
     constexpr int S = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -82,7 +90,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* tfull = empty + S;    // [2]
     uint64_t* tempty = tfull + 2;   // [2]
     uint64_t* lready = tempty + 2;  // [2] rank-r operand tables written
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lready + 2);
+    uint64_t* wready = lready + 2;  // [S] packed int4 kernels: the stage's int8 codes written
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wready + S);
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
@@ -101,6 +110,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&tempty[b], kEpiWarps);
             mbar_init(&lready[b], 1);
         }
+        if constexpr (W4)
+            for (int s = 0; s < S; ++s) mbar_init(&wready[s], kUnpackWarps);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -130,18 +141,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     uint8_t* sa = smem + s * C::kStageBytes;
-                    mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+                    mbar_arrive_expect_tx(&full[s], W4 ? C::kABytes : C::kStageBytes);
                     // each operand's two k-blocks, consecutive in shared memory
                     if (k3d) {
                         tma_load_3d(sa, &tmA, &full[s], 0, m0, kb * C::kBlk);
-                        tma_load_3d(sa + C::kABytes, &tmB, &full[s], 0, n0, kb * C::kBlk);
+                        if constexpr (!W4) tma_load_3d(sa + C::kABytes, &tmB, &full[s], 0, n0, kb * C::kBlk);
                     } else {
 #pragma unroll
                         for (int b = 0; b < C::kBlk; ++b) {
                             tma_load_2d(sa + b * (kBM * kBlkK), &tmA, &full[s], (kb * C::kBlk + b) * kBlkK,
                                         m0);
-                            tma_load_2d(sa + C::kABytes + b * (BN * kBlkK), &tmB, &full[s],
-                                        (kb * C::kBlk + b) * kBlkK, n0);
+                            if constexpr (!W4)
+                                tma_load_2d(sa + C::kABytes + b * (BN * kBlkK), &tmB, &full[s],
+                                            (kb * C::kBlk + b) * kBlkK, n0);
                         }
                     }
                 }
@@ -162,7 +174,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t dacc = tmem + ab * C::kAccCols;
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
                     const int s = g % S;
-                    if (!mbar_wait(&full[s], (g / S) & 1, status)) {
+                    if (!mbar_wait(&full[s], (g / S) & 1, status) ||
+                        (W4 && !mbar_wait(&wready[s], (g / S) & 1, status))) {
                         ok = false;
                         break;
                     }
@@ -208,6 +221,62 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 if (ok) mma_commit(&tfull[ab]);
+            }
+        }
+        __syncwarp();
+    } else if (W4 && warp >= 2 + kEpiWarps) {
+        // ------------------------------------------------------ int4 unpack
+        // Stage g's Wq tile, as the TMA would have written it: k-block b of
+        // row n at b * BN * 128 + n * 128, its 16-byte chunk c at position
+        // c ^ (n % 8).  One packed 16-byte chunk (32 codes) gives int8 chunks
+        // 2p and 2p + 1 of a row; chunks outside the matrix are written as
+        // zeros.  The loads go out before the wait for the stage to be free.
+        const int ut = (warp - 2 - kEpiWarps) * 32 + lane;
+        constexpr int kPerRow = C::kBlk * 4;  // packed chunks of one row per stage
+        constexpr int kItems = BN * kPerRow;
+        constexpr int kPer = kItems / (32 * kUnpackWarps);
+        static_assert(kItems % (32 * kUnpackWarps) == 0, "packed chunks per unpack thread");
+        const size_t row_bytes = static_cast<size_t>(K) / 2;
+        int g = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            const int n0 = (t % num_n) * BN;
+            for (int kb = 0; kb < nkb; ++kb, ++g) {
+                const int s = g % S;
+                uint4 raw[kPer];
+                uint32_t inb = 0;
+#pragma unroll
+                for (int i = 0; i < kPer; ++i) {
+                    const int e = ut + i * 32 * kUnpackWarps;
+                    const int n = n0 + e / kPerRow;
+                    const int rem = e % kPerRow;
+                    const int k = kb * C::kBK + (rem / 4) * kBlkK + (rem % 4) * 32;
+                    if (n < N && k < K) inb |= 1u << i;
+                    const int nc = n < N ? n : N - 1;
+                    const int kc = k < K ? k : K - 32;
+                    raw[i] = __ldg(reinterpret_cast<const uint4*>(Wp + static_cast<size_t>(nc) * row_bytes + kc / 2));
+                }
+                if (g >= S && !__all_sync(0xffffffffu, mbar_wait(&empty[s], ((g / S) - 1) & 1, status))) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* wb = smem + s * C::kStageBytes + C::kABytes;
+#pragma unroll
+                for (int i = 0; i < kPer; ++i) {
+                    const int e = ut + i * 32 * kUnpackWarps;
+                    const int n = e / kPerRow;
+                    const int rem = e % kPerRow;
+                    const int p = rem % 4;
+                    uint4 lo, hi;
+                    unpack_int4x32(raw[i], lo, hi);
+                    if (!((inb >> i) & 1u)) lo = hi = make_uint4(0u, 0u, 0u, 0u);
+                    uint8_t* row = wb + (rem / 4) * (BN * kBlkK) + n * kBlkK;
+                    *reinterpret_cast<uint4*>(row + (((2 * p) ^ (n & 7)) << 4)) = lo;
+                    *reinterpret_cast<uint4*>(row + (((2 * p + 1) ^ (n & 7)) << 4)) = hi;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&wready[s]);
             }
         }
         __syncwarp();
@@ -341,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int BN, typename OutT, int RMAX>
+template <int BN, typename OutT, int RMAX, bool W4>
 cudaError_t launch_cfg(const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
                        const FwdEpilogue& ep, int* status, cudaStream_t s) {
     using C = K2Cfg<BN, OutT, RMAX>;
@@ -350,51 +419,56 @@ cudaError_t launch_cfg(const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
     CUtensorMap ta, tb;
     const int k3d = (K % kBlkK) == 0 ? 1 : 0;
     bool ok;
+    // (packed int4 kernels: no map for the codes, which the unpack warps load)
     if (k3d)
         ok = make_tmap_3d_blocks(&ta, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, kBlkK, kBM, C::kBlk) &&
-             make_tmap_3d_blocks(&tb, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, kBlkK, BN, C::kBlk);
+             (W4 || make_tmap_3d_blocks(&tb, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, kBlkK, BN, C::kBlk));
     else
         ok = make_tmap_2d(&ta, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, K, kBM, kBlkK,
                           CU_TENSOR_MAP_SWIZZLE_128B) &&
-             make_tmap_2d(&tb, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, BN, kBlkK,
-                          CU_TENSOR_MAP_SWIZZLE_128B);
+             (W4 || make_tmap_2d(&tb, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, BN, kBlkK,
+                                 CU_TENSOR_MAP_SWIZZLE_128B));
     if (!ok) return cudaErrorInvalidValue;
-    auto kern = k2_gemm_i8_lora_kernel<BN, OutT, RMAX>;
+    if (W4) tb = ta;  // unused
+    auto kern = k2_gemm_i8_lora_kernel<BN, OutT, RMAX, W4>;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), C::kTotal);
     if (e != cudaSuccess) return e;
     const int tiles = ((M + kBM - 1) / kBM) * ((N + BN - 1) / BN);
     const int grid = tiles < sm_count() ? tiles : sm_count();
-    return launch_k(kern, dim3(grid), dim3(kThreads), C::kTotal, s, 1, ta, tb, k3d, M, N, K, ep,
-                    status);
+    return launch_k(kern, dim3(grid), dim3(k2_threads<W4>()), C::kTotal, s, 1, ta, tb, k3d, M, N, K,
+                    W4 ? reinterpret_cast<const uint8_t*>(Wq) : nullptr, ep, status);
 }
 
-template <typename OutT, int RMAX>
+template <typename OutT, int RMAX, bool W4>
 cudaError_t launch_bn(int bn, const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
                       const FwdEpilogue& ep, int* status, cudaStream_t s) {
-    if (bn == 128) return launch_cfg<128, OutT, RMAX>(Xq, Wq, M, N, K, ep, status, s);
-    return launch_cfg<64, OutT, RMAX>(Xq, Wq, M, N, K, ep, status, s);
+    if (bn == 128) return launch_cfg<128, OutT, RMAX, W4>(Xq, Wq, M, N, K, ep, status, s);
+    return launch_cfg<64, OutT, RMAX, W4>(Xq, Wq, M, N, K, ep, status, s);
 }
 
-template <typename OutT>
+template <typename OutT, bool W4>
 cudaError_t launch_r(int bn, const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
                      const FwdEpilogue& ep, int* status, cudaStream_t s) {
-    if (ep.r <= 4) return launch_bn<OutT, 4>(bn, Xq, Wq, M, N, K, ep, status, s);
-    if (ep.r <= 8) return launch_bn<OutT, 8>(bn, Xq, Wq, M, N, K, ep, status, s);
-    if (ep.r <= 16) return launch_bn<OutT, 16>(bn, Xq, Wq, M, N, K, ep, status, s);
-    return launch_bn<OutT, 64>(bn, Xq, Wq, M, N, K, ep, status, s);
+    if (ep.r <= 4) return launch_bn<OutT, 4, W4>(bn, Xq, Wq, M, N, K, ep, status, s);
+    if (ep.r <= 8) return launch_bn<OutT, 8, W4>(bn, Xq, Wq, M, N, K, ep, status, s);
+    if (ep.r <= 16) return launch_bn<OutT, 16, W4>(bn, Xq, Wq, M, N, K, ep, status, s);
+    return launch_bn<OutT, 64, W4>(bn, Xq, Wq, M, N, K, ep, status, s);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_i8_fwd(Act act, const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
-                               const FwdEpilogue& ep, int* status, cudaStream_t s) {
+                               const FwdEpilogue& ep, int* status, cudaStream_t s, bool w4) {
     // Tile width: 128 columns unless that leaves SMs without a tile.
     const int mt = (M + kBM - 1) / kBM;
     int bn = mt * ((N + 127) / 128) >= sm_count() ? 128 : 64;
     const int forced = tile_override("QLORA_FWD_BN");  // tuning: 64 or 128
     if (forced == 64 || forced == 128) bn = forced;
-    if (act == kBF16) return launch_r<__nv_bfloat16>(bn, Xq, Wq, M, N, K, ep, status, s);
-    return launch_r<float>(bn, Xq, Wq, M, N, K, ep, status, s);
+    if (act == kBF16)
+        return w4 ? launch_r<__nv_bfloat16, true>(bn, Xq, Wq, M, N, K, ep, status, s)
+                  : launch_r<__nv_bfloat16, false>(bn, Xq, Wq, M, N, K, ep, status, s);
+    return w4 ? launch_r<float, true>(bn, Xq, Wq, M, N, K, ep, status, s)
+              : launch_r<float, false>(bn, Xq, Wq, M, N, K, ep, status, s);
 }
 
 }  // namespace qlora

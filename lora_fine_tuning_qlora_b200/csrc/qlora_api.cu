@@ -316,9 +316,11 @@ int qlora_quantize_input(const qlora_layer_desc* d, int M, const void* X, const 
 static int gemm_forward_impl(const qlora_layer_desc* d, int M, const int8_t* Xq, const float* sx,
                              const int8_t* Wq, const float* sw, const float* bias,
                              const float* xA, const float* B, void* Y, int32_t* acc, int relu,
-                             void* stream) {
+                             void* stream, bool w4 = false) {
     int rc = check_layer(d, M);
     if (rc != QLORA_OK) return rc;
+    QL_REQUIRE(!w4 || d->K % 32 == 0, QLORA_EUNSUPPORTED,
+               "packed int4 kernels need K a multiple of 32 (16-byte rows of codes)");
     QL_REQUIRE(Xq && sx && Wq && sw && xA && B && Y, QLORA_EINVAL, "NULL pointer argument");
     QL_REQUIRE(aligned(Xq, 16) && aligned(Wq, 16) && aligned(Y, 16), QLORA_EALIGN,
                "Xq, Wq and Y must be 16-byte aligned");
@@ -340,7 +342,7 @@ static int gemm_forward_impl(const qlora_layer_desc* d, int M, const int8_t* Xq,
     ep.acc = acc;
     ep.relu = relu;
     return cuda_status(launch_gemm_i8_fwd(act_of(d), Xq, Wq, M, d->N, d->K, ep, status,
-                                          static_cast<cudaStream_t>(stream)),
+                                          static_cast<cudaStream_t>(stream), w4),
                        "int8 GEMM launch");
 }
 
@@ -616,6 +618,13 @@ int qlora_unpack_int4(const uint8_t* Wp, int K, int N, int8_t* Wq, void* stream)
     if (!aligned(Wp, 16) || !aligned(Wq, 16)) return fail(QLORA_EALIGN, "Wp and Wq must be 16-byte aligned");
     return cuda_status(launch_unpack_int4(Wp, K, N, Wq, static_cast<cudaStream_t>(stream)),
                        "unpack_int4 launch");
+}
+
+int qlora_gemm_forward_int4(const qlora_layer_desc* d, int M, const int8_t* Xq, const float* sx,
+                            const uint8_t* Wp, const float* sw, const float* bias, const float* xA,
+                            const float* B, void* Y, int32_t* acc, void* stream) {
+    return gemm_forward_impl(d, M, Xq, sx, reinterpret_cast<const int8_t*>(Wp), sw, bias, xA, B, Y,
+                             acc, 0, stream, true);
 }
 
 int qlora_gemm_dx_int4(const qlora_layer_desc* d, int M, const void* dY, const uint8_t* Wp,

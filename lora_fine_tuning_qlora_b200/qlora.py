@@ -33,7 +33,7 @@ EXPORTED = ("qlora_quantize_weight", "qlora_workspace_bytes", "qlora_forward",
             "qlora_selftest_wait_timeout", "qlora_backward_noalloc", "qlora_lora_g",
             "qlora_lora_grad_b", "qlora_gemm_forward_relu", "qlora_gemm_dx_relu",
             "qlora_set_rank_pass_rows", "qlora_quantize_weight_int4", "qlora_unpack_int4",
-            "qlora_gemm_dx_int4", "qlora_merge_int4")
+            "qlora_gemm_dx_int4", "qlora_merge_int4", "qlora_gemm_forward_int4")
 
 
 class QLoraError(RuntimeError):
@@ -98,6 +98,8 @@ def _load():
     lib.qlora_quantize_weight_int4.argtypes = [P, I, I, P, P, P]
     lib.qlora_unpack_int4.argtypes = [P, I, I, P, P]
     lib.qlora_gemm_dx_int4.argtypes = [D, I, P, P, P, P, P, P, Z, P]
+    lib.qlora_gemm_forward_int4.argtypes = [D, I, P, P, P, P, P, P, P, P, P, P]
+    lib.qlora_gemm_forward_int4.restype = I
     lib.qlora_merge_int4.argtypes = [D, P, P, P, P, P, P, P]
     for f in (lib.qlora_quantize_weight_int4, lib.qlora_unpack_int4, lib.qlora_gemm_dx_int4,
               lib.qlora_merge_int4):
@@ -275,6 +277,14 @@ def unpack_int4(Wp: torch.Tensor, stream=None) -> torch.Tensor:
     Wq = torch.empty((N, 2 * K2), dtype=torch.int8, device=Wp.device)
     _check(_lib.qlora_unpack_int4(_ptr(Wp), 2 * K2, N, _ptr(Wq), _stream(stream)))
     return Wq
+
+
+def qlora_gemm_forward_int4(d: LayerDesc, M: int, Xq, sx, Wp, sw, bias, xA, B, Y, acc=None,
+                            stream=None):
+    """qlora_gemm_forward on packed int4 codes Wp [N, K/2]."""
+    _check(_lib.qlora_gemm_forward_int4(ctypes.byref(d), int(M), _ptr(Xq), _ptr(sx), _ptr(Wp),
+                                        _ptr(sw), _ptr(bias), _ptr(xA), _ptr(B), _ptr(Y), _ptr(acc),
+                                        _stream(stream)))
 
 
 def qlora_gemm_dx_int4(d: LayerDesc, M: int, dY, Wp, sw, A, dX, ws, stream=None):

@@ -147,3 +147,12 @@ def test_int4_calls_reject_bad_arguments(q):
     d = q.desc(1024, 128, 4, 4.0, torch.bfloat16)
     assert lib.qlora_merge_int4(ctypes.byref(d), P(0x1000), P(0x2000), P(0x3000), P(0x4000),
                                 P(0x1000), P(0x6000), None) == -1  # output aliases input
+
+
+def test_int4_forward_rejects_k_not_multiple_of_32(q):
+    import torch
+    P = ctypes.c_void_p
+    d = q.desc(784, 128, 4, 4.0, torch.bfloat16)
+    rc = q.lib().qlora_gemm_forward_int4(ctypes.byref(d), 64, P(0x1000), P(0x2000), P(0x3000),
+                                         P(0x4000), None, P(0x5000), P(0x6000), P(0x7000), None, None)
+    assert rc == -5

@@ -407,12 +407,14 @@ def test_int4_quantize_and_unpack_bit_exact(q, K, N):
                                           (1000, 1312, 264, 8, "bf16"),   # 128x128 tiles
                                           (4096, 768, 768, 4, "bf16"),    # 256x128 tiles
                                           (96, 256, 10, 8, "bf16"),       # CUDA-core dX
-                                          (64, 256, 128, 4, "f32")])      # fp32 activations
+                                          (64, 256, 128, 4, "f32"),       # fp32 activations
+                                          (200, 800, 264, 16, "bf16")])   # K % 128 == 32: ragged k-block
 def test_int4_layer_matches_oracle(q, M, K, N, r, act):
-    """An int4 layer: forward on the unpacked codes (accumulator bit-exact), dX
-    from the packed codes bit-identical to the int8 path on the unpacked codes
-    and within tolerance of the oracle, dA/dB/dbias against the oracle, and
-    the int4 merge bit-exact."""
+    """An int4 layer: the forward from the packed codes bit-identical to the
+    int8 forward on the unpacked codes (accumulator bit-exact against the
+    oracle), dX from the packed codes bit-identical to the int8 path and
+    within tolerance of the oracle, dA/dB/dbias against the oracle, and the
+    int4 merge bit-exact."""
     spec = _edge_spec(M, K, N, r, act=act, seed=5 * M + K)
     d = inputs.layer_inputs(spec)
     from parity import act_torch
@@ -437,9 +439,14 @@ def test_int4_layer_matches_oracle(q, M, K, N, r, act):
     dA = torch.empty((K, r), device="cuda")
     q.qlora_lora_grad_x(D, M, X, dA, ws)
     Wp2, sw2 = q.merge_int4(D, Wp, sw, layer.A, layer.B)
+    # the forward from the packed codes, against the int8 forward on the unpacked ones
+    Y4 = torch.full_like(Y, float("nan"))
+    acc4 = torch.full_like(acc, -1)
+    q.qlora_gemm_forward_int4(D, M, xq, sx, Wp, sw, layer.bias, xA, layer.B, Y4, acc4)
     torch.cuda.synchronize()
     assert q.qlora_device_status() == 0
     assert torch.equal(dX4, dX8)
+    assert torch.equal(acc4, acc) and torch.equal(Y4, Y)
 
     Wp_o, sw_o = oracle.quantize_weight_int4(d["W"])
     codes = oracle.unpack_int4(Wp_o)
