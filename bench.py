@@ -1,18 +1,26 @@
 #!/usr/bin/env python3
 """Benchmark of the int8-LoRA Dense hot path on B200.
 
-One step = forward and backward (dX, dA, dB, dbias of every layer) through
-the MNIST MLP stack of int8-LoRA Dense layers: 784 -> 1024, 31 x 1024 ->
-1024, 1024 -> 10, ReLU between layers (run in the GEMM epilogues), batch
-1024 per GPU, bf16 activations, rank 8, alpha 8 (seeded synthetic data and
-weights).  With N
-GPUs (torchrun, one process per GPU) every rank runs its own batch and the
-LoRA gradients are summed with one NCCL all-reduce per step (weak scaling).
+Headline: one step = forward and backward (dX, dA, dB, dbias) of one
+int8-LoRA Dense layer with a 4096 x 4096 kernel at M = 16384 tokens, bf16
+activations, a rank-4 adapter (alpha 8): the largest single-GPU shape of the
+4096-wide layer sweep ("How to fine-tune the 4-bit model?" thread, the
+arithmetic-intensity argument for a 4096-wide layer).  With N GPUs (torchrun,
+one process per GPU) every rank runs its own 16384 tokens and the LoRA
+gradients are summed with one NCCL all-reduce per step (weak scaling).
+
+Beside the headline, the same JSON line carries a ``configs`` list: every
+layer of every benchmark workload (the single fp32 layer, the MNIST MLP
+stack, the GPT-2 base projections, the Gemma-2B projections at M = 512 and
+4096, the 4096-wide layer at M = 16 ... 16384), each with its step time, its
+TFLOP/s, the step roofline t_roof / t_measured, and every launch group's
+time and fraction of its own roofline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--no-configs] [--only SUBSTRING]
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle on
-a bounded row sample of the same workload, on the host cores.
+a bounded row sample of the headline layer, on the host cores.
 """
 from __future__ import annotations
 
@@ -20,6 +28,7 @@ import argparse
 import hashlib
 import json
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -31,9 +40,17 @@ sys.path.insert(0, ROOT)
 
 METRIC = "int8-LoRA Dense fwd+bwd TFLOP/s per step; % of B200 i8/bf16 TC and HBM roofline"
 UNIT = "TFLOP/s"
-WORKLOAD = "mnist_mlp_stack_33x_int8_lora_dense_bf16_b1024_r8"
+HEAD_M = 16384
+WORKLOAD = "dense4096_m16384_bf16_r4"
 L2_FLUSH_BYTES = 384 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PART_KERNELS = {
+    "quantize_input": ("k1_quantize_rows_kernel", "hbm"),
+    "gemm_forward": ("k2_gemm_i8_lora_kernel", "tensor_i8"),
+    "lora_grad_dy": ("k4_rank_tc_kernel (dY pass)", "hbm"),
+    "gemm_dx": ("k3_dx_dequant_kernel", "tensor_bf16"),
+    "lora_grad_x": ("k4_rank_tc_kernel (X pass)", "hbm"),
+}
 
 
 def log(*a):
@@ -45,62 +62,73 @@ def load_peaks():
     try:
         with open(p) as f:
             d = json.load(f)
-        return d, "measured"
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"]))}, \
+            "measured"
     except Exception:
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def config_dict(n_gpus, batch):
-    return {"workload": WORKLOAD, "layers": 33, "dims": "784-1024x32-10", "batch_per_gpu": batch,
-            "global_batch": batch * n_gpus, "rank": 8, "alpha": 8.0, "act": "bf16",
-            "forward_gemm": "int8 tcgen05", "dx_gemm": "bf16 tcgen05 (int8 dequant in smem)",
-            "l2": "flushed between timed steps (384 MiB write)",
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return platform.processor() or "unknown"
+
+
+def head_config(n_gpus):
+    return {"workload": WORKLOAD, "M_per_gpu": HEAD_M, "K": 4096, "N": 4096, "rank": 4,
+            "alpha": 8.0, "act": "bf16", "global_batch": HEAD_M * n_gpus, "seq_len": None,
+            "forward_gemm": "int8 tcgen05 (K2)", "dx_gemm": "bf16 tcgen05, int8 de-quantized in smem (K3)",
+            "l2": "inputs larger than L2, and flushed between timed steps (384 MiB write)",
             "parallelism": "dp%d" % n_gpus}
 
 
 # --------------------------------------------------------------------------
 # CPU oracle timing (cpu_baseline and the reference arm)
 # --------------------------------------------------------------------------
-def oracle_stack_sample(rows, specs, data):
-    """Runs the oracle's stack on the first `rows` rows; returns seconds."""
-    import numpy as np
+def oracle_layer_rows(data, spec, Wq, sw, rows):
+    """The oracle's forward + backward of the layer on its first `rows` rows;
+    returns seconds."""
     import oracle
-    layers = []
-    for s, L in zip(specs, data["layers"]):
-        Wq, sw = oracle.quantize_weight(L["W"])
-        layers.append({"Wq": Wq, "sw": sw, "bias": L["bias"], "A": L["A"], "B": L["B"],
-                       "alpha": s.alpha})
     X = data["X"][:rows]
     dY = data["dY"][:rows]
     t0 = time.perf_counter()
-    oracle.mlp_stack(X, layers, dY, "bf16")
+    oracle.forward(X, Wq, sw, data["bias"], data["A"], data["B"], spec.alpha)
+    oracle.backward(X, dY, Wq, sw, data["A"], data["B"], spec.alpha, want_dx=True, act=spec.act)
     return time.perf_counter() - t0
 
 
-def stack_flops(specs, rows):
-    tot = 0.0
-    for s in specs:
-        tot += 4.0 * rows * s.N * s.K
-        tot += 2.0 * rows * s.r * (2 * s.K + 2 * s.N) + 2.0 * rows * s.r * (s.K + s.N)
-    return tot
+def layer_flops(M, K, N, r):
+    return 4.0 * M * N * K + 2.0 * M * r * (2 * K + 2 * N) + 2.0 * M * r * (K + N)
 
 
-def calibrate_rows(specs, data, target_s):
-    t = oracle_stack_sample(16, specs, data)
-    rows = int(16 * target_s / max(t, 1e-3))
-    rows = max(16, min(1024, (rows // 16) * 16))
-    return rows
-
-
-def cpu_baseline(specs, data, target_s=12.0):
+def oracle_setup(spec, data):
     import oracle
     oracle.set_threads(os.cpu_count() or 1)
-    rows = calibrate_rows(specs, data, target_s)
-    t = oracle_stack_sample(rows, specs, data)
-    return {"value": stack_flops(specs, rows) / t / 1e12, "unit": UNIT,
-            "cores": oracle.get_threads(), "kind": "oracle",
-            "sample": "oracle MLP stack fwd+bwd on the first %d of 1024 rows (all 33 layers), "
-                      "%.1f s" % (rows, t)}
+    Wq, sw = oracle.quantize_weight(data["W"])
+    return Wq, sw
+
+
+def calibrate_rows(spec, data, Wq, sw, target_s):
+    t = oracle_layer_rows(data, spec, Wq, sw, 4)
+    rows = int(4 * target_s / max(t, 1e-3))
+    return max(4, min(spec.M, rows))
+
+
+def cpu_baseline(spec, data, target_s=12.0):
+    import oracle
+    Wq, sw = oracle_setup(spec, data)
+    rows = calibrate_rows(spec, data, Wq, sw, target_s)
+    t = oracle_layer_rows(data, spec, Wq, sw, rows)
+    return {"value": layer_flops(rows, spec.K, spec.N, spec.r) / t / 1e12, "unit": UNIT,
+            "cores": oracle.get_threads(), "cpu": cpu_model(), "kind": "oracle",
+            "sample": "oracle forward+backward of the %dx%d layer on the first %d of %d rows "
+                      "(dA, dB over those rows), %.1f s" % (spec.K, spec.N, rows, spec.M, t)}
 
 
 def run_reference(args):
@@ -110,25 +138,25 @@ def run_reference(args):
         return 0
     import oracle
     from lora_fine_tuning_qlora_b200 import inputs
-    oracle.set_threads(os.cpu_count() or 1)
-    specs = inputs.mlp_stack()
-    data = inputs.mlp_stack_inputs(specs)
+    spec = inputs.dense4096(HEAD_M)
+    data = inputs.layer_inputs(spec)
+    Wq, sw = oracle_setup(spec, data)
     per_step = max(0.5, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
-    rows = calibrate_rows(specs, data, per_step)
+    rows = calibrate_rows(spec, data, Wq, sw, per_step)
     for _ in range(args.warmup):
-        oracle_stack_sample(rows, specs, data)
-    times = [oracle_stack_sample(rows, specs, data) for _ in range(args.steps)]
+        oracle_layer_rows(data, spec, Wq, sw, rows)
+    times = [oracle_layer_rows(data, spec, Wq, sw, rows) for _ in range(args.steps)]
     tot = sum(times)
-    value = stack_flops(specs, rows) * args.steps / tot / 1e12
+    value = layer_flops(rows, spec.K, spec.N, spec.r) * args.steps / tot / 1e12
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_dict(world, 1024),
+            "config": head_config(world),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.get_threads(),
-                             "kind": "oracle",
-                             "sample": "oracle MLP stack fwd+bwd on the first %d of 1024 rows per "
-                                       "step (all 33 layers)" % rows},
+                             "cpu": cpu_model(), "kind": "oracle",
+                             "sample": "oracle forward+backward of the 4096x4096 layer on the "
+                                       "first %d of %d rows per step" % (rows, HEAD_M)},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -200,7 +228,7 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------
-# our arm
+# roofline arithmetic
 # --------------------------------------------------------------------------
 def source_sha(*names):
     h = hashlib.sha256()
@@ -210,24 +238,195 @@ def source_sha(*names):
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel_key, src_files):
-    """Per-launch DRAM bytes of `kernel_key` from the committed ncu summary,
-    if the kernel's source has not changed since the capture."""
+TRAFFIC_SOURCES = {
+    "k1_quantize_rows_kernel": ["k1_quantize.cu", "ptx.cuh"],
+    "k2_gemm_i8_lora_kernel": ["k2_gemm_i8.cu", "ptx.cuh", "tile_epilogue.cuh"],
+    "k3_dx_dequant_kernel": ["k3_dx.cu", "ptx.cuh", "tile_epilogue.cuh"],
+    "k4_rank_tc_kernel (dY pass)": ["k4_rank_tc.cu", "ptx.cuh"],
+    "k4_rank_tc_kernel (X pass)": ["k4_rank_tc.cu", "ptx.cuh"],
+}
+
+
+def profiled_traffic(kernel, workload):
+    """Per-launch DRAM bytes of `kernel` on `workload` from the committed ncu
+    summary, if the kernel's sources have not changed since the capture."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             d = json.load(f)
-        e = d[kernel_key]
-        if e.get("source_sha") == source_sha(*src_files):
+        e = d[kernel + " @ " + workload]
+        if e.get("source_sha") == source_sha(*TRAFFIC_SOURCES[kernel]):
             return e["dram_bytes_per_launch"]
     except Exception:
         pass
     return None
 
 
+class Roof:
+    def __init__(self, peaks):
+        self.bw = peaks["hbm_gbs"] * 1e9
+        self.bf16 = peaks["bf16_tflops"] * 1e12
+        self.i8 = 2.0 * self.bf16  # nominal int8:bf16 dense ratio
+
+    def part(self, name, us, M, K, N, r, e):
+        """Achieved rate and fractions of one launch group."""
+        from lora_fine_tuning_qlora_b200.step import algorithmic_bytes
+        by = algorithmic_bytes(M, K, N, r, e)[name]
+        t = us * 1e-6
+        kern, bound = PART_KERNELS[name]
+        d = {"us": us, "kernel": kern, "bytes": by, "GB/s": by / t / 1e9}
+        if bound == "hbm":
+            d.update({"bound": "hbm", "frac_hbm": by / t / self.bw})
+            d["t_roof_us"] = by / self.bw * 1e6
+        else:
+            fl = 2.0 * M * N * K
+            peak = self.i8 if bound == "tensor_i8" else self.bf16
+            d.update({"bound": bound, "T(FL)OP/s": fl / t / 1e12, "frac_tensor": fl / t / peak,
+                      "frac_hbm": by / t / self.bw})
+            d["t_roof_us"] = max(fl / peak, by / self.bw) * 1e6
+        d["frac_roof"] = d["t_roof_us"] / us
+        return d
+
+    def step_roof_us(self, M, K, N, r, e):
+        """t_roof of one fwd+bwd step: the int8 GEMM and the dX GEMM each at
+        the slower of their tensor and byte bounds, plus the byte-bound
+        passes (input quantizer, dY pass, X pass) at HBM bandwidth."""
+        from lora_fine_tuning_qlora_b200.step import algorithmic_bytes
+        b = algorithmic_bytes(M, K, N, r, e)
+        fl = 2.0 * M * N * K
+        t = max(fl / self.i8, b["gemm_forward"] / self.bw) + max(fl / self.bf16, b["gemm_dx"] / self.bw)
+        t += (b["quantize_input"] + b["lora_grad_dy"] + b["lora_grad_x"]) / self.bw
+        return t * 1e6
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+def make_step(spec, dev, data=None):
+    import torch
+    from lora_fine_tuning_qlora_b200 import inputs, qlora, step
+    d = data if data is not None else inputs.layer_inputs(spec)
+    act = torch.bfloat16 if spec.act == "bf16" else torch.float32
+    Wq, sw = qlora.quantize_weight(torch.from_numpy(d["W"]).to(dev))
+    bias = torch.from_numpy(d["bias"]).to(dev) if d["bias"] is not None else None
+    layer = qlora.Layer(Wq=Wq, sw=sw, bias=bias, A=torch.from_numpy(d["A"]).to(dev),
+                        B=torch.from_numpy(d["B"]).to(dev), alpha=spec.alpha, act=act)
+    st = step.LayerStep(layer, spec.M, dev)
+    st.X.copy_(torch.from_numpy(d["X"]).to(act))
+    st.dY.copy_(torch.from_numpy(d["dY"]).to(act))
+    return st, d
+
+
+def time_graph(replay, steps, warmup, flush, between=None):
+    """Mean ms of `replay()` over `steps` replays, L2 flushed before each."""
+    import torch
+    for _ in range(warmup):
+        flush.zero_()
+        replay()
+    torch.cuda.synchronize()
+    s = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for k in range(steps):
+        flush.zero_()
+        s[k].record()
+        replay()
+        e[k].record()
+        if between:
+            between(k)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in zip(s, e)]
+
+
+def layer_entry(spec, dev, flush, roof, steps, warmup, data=None):
+    """Step time and per-launch-group times of one layer workload."""
+    import torch
+    from lora_fine_tuning_qlora_b200 import step as step_mod
+    st, _ = make_step(spec, dev, data)
+    e = 2 if spec.act == "bf16" else 4
+    st.capture(warmup=1)
+    plain = st.graph
+    ms = time_graph(st.replay, steps, warmup, flush)
+    ev = st.make_events()
+    st.capture(warmup=0, events=ev)
+    per = {p: [] for p in step_mod.PARTS}
+
+    def collect(k):
+        torch.cuda.synchronize()
+        for p in step_mod.PARTS:
+            per[p].append(ev[p][0].elapsed_time(ev[p][1]))
+
+    time_graph(st.replay, steps, 1, flush, between=collect)
+    step_us = 1e3 * statistics.median(ms)
+    M, K, N, r = spec.M, spec.K, spec.N, spec.r
+    t_roof = roof.step_roof_us(M, K, N, r, e)
+    ent = {"workload": spec.name, "M": M, "K": K, "N": N, "r": r, "act": spec.act,
+           "step_us": step_us, "tflops": st.flops() / (step_us * 1e-6) / 1e12,
+           "t_roof_us": t_roof, "roof_frac": t_roof / step_us,
+           "kernels": {p: roof.part(p, 1e3 * statistics.median(per[p]), M, K, N, r, e)
+                       for p in step_mod.PARTS}}
+    st.graph = None
+    del plain
+    return ent, st
+
+
+def mlp_entry(dev, flush, roof, steps, warmup):
+    import torch  # noqa: F401
+    from lora_fine_tuning_qlora_b200 import inputs, stack
+    specs = inputs.mlp_stack()
+    data = inputs.mlp_stack_inputs(specs)
+    net = stack.MLPStack.from_inputs(specs, data, device=dev)
+    import torch as T
+    net.X.copy_(T.from_numpy(data["X"]).to(T.bfloat16))
+    net.dY.copy_(T.from_numpy(data["dY"]).to(T.bfloat16))
+    net.capture(warmup=1)
+    ms = time_graph(net.replay, steps, warmup, flush)
+    step_us = 1e3 * statistics.median(ms)
+    t_roof = sum(roof.step_roof_us(s.M, s.K, s.N, s.r, 2) for s in specs)
+    net.graph = None
+    return {"workload": "mnist_mlp_stack_33x_b1024_bf16_r8", "layers": len(specs),
+            "step_us": step_us, "tflops": net.flops_per_step() / (step_us * 1e-6) / 1e12,
+            "t_roof_us": t_roof, "roof_frac": t_roof / step_us,
+            "note": "33 layers (784-1024x32-10), ReLU fused in the GEMM epilogues, side-stream "
+                    "dB/dA passes, one CUDA graph"}
+
+
+def merge_entry(st, flush, roof, steps):
+    """qlora_merge of a 4096x4096 layer: reads Wq twice, writes Wq' and sw'."""
+    import torch
+    from lora_fine_tuning_qlora_b200 import qlora
+    L = st.layer
+    Wq2 = torch.empty_like(L.Wq)
+    sw2 = torch.empty_like(L.sw)
+    d = L.desc()
+    ms = time_graph(lambda: qlora.qlora_merge(d, L.Wq, L.sw, L.A, L.B, Wq2, sw2), steps, 3, flush)
+    us = 1e3 * statistics.median(ms)
+    by = 2.0 * L.K * L.N + 4.0 * L.N + 4.0 * L.r * (L.K + L.N) + L.K * L.N + 4.0 * L.N
+    return {"kernel": "km_merge_kernel", "K": L.K, "N": L.N, "us": us, "bytes": by,
+            "GB/s": by / (us * 1e-6) / 1e9, "frac_hbm": by / (us * 1e-6) / roof.bw}
+
+
+def all_configs(dev, flush, roof, steps, only):
+    from lora_fine_tuning_qlora_b200 import inputs
+    specs = [inputs.single_fp32()] + inputs.gpt2_base() + inputs.gemma_2b(512) + \
+        inputs.gemma_2b(4096) + [inputs.dense4096(m) for m in inputs.DENSE4096_M if m != HEAD_M]
+    out = []
+    if not only or "mlp" in only:
+        out.append(mlp_entry(dev, flush, roof, steps, 3))
+    merge = None
+    for s in specs:
+        if only and only not in s.name:
+            continue
+        ent, st = layer_entry(s, dev, flush, roof, steps, 3)
+        if s.name.startswith("dense4096") and merge is None:
+            merge = merge_entry(st, flush, roof, steps)
+        out.append(ent)
+        del st
+    return out, merge
+
+
 def run_ours(args):
     import torch
-    from lora_fine_tuning_qlora_b200 import dp, inputs, stack
+    from lora_fine_tuning_qlora_b200 import dp, inputs, step as step_mod
 
     rank, local, world = dp.init("nccl")
     if world != args.gpus:
@@ -236,30 +435,27 @@ def run_ours(args):
         raise SystemExit("bench.py needs a CUDA device")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    peaks, peak_src = load_peaks()
+    roof = Roof(peaks)
 
-    specs = inputs.mlp_stack()
-    data = inputs.mlp_stack_inputs(specs)
-    # weak scaling: every rank draws its own batch; the weights are shared
+    # weak scaling: every rank draws its own tokens; the weights are shared
+    spec = inputs.dense4096(HEAD_M)
+    data = inputs.layer_inputs(spec)
     if world > 1:
-        rspecs = [inputs.scaled(s, seed=dp.rank_seed(s.seed, rank)) for s in specs]
-        rd = inputs.mlp_stack_inputs(rspecs)
-        data = {"layers": data["layers"], "X": rd["X"], "dY": rd["dY"]}
-    net = stack.MLPStack.from_inputs(specs, data, device=dev)
-    X_dev = torch.from_numpy(data["X"]).to(torch.bfloat16).to(dev)
-    dY_dev = torch.from_numpy(data["dY"]).to(torch.bfloat16).to(dev)
-    net.X.copy_(X_dev)
-    net.dY.copy_(dY_dev)
-    # per-kernel events on a few interior 1024x1024 layers only: an event pair
-    # serialises the kernel it brackets, so timing every layer slows the step
-    mid = [i for i, s in enumerate(specs) if s.K == 1024 and s.N == 1024][3::8]
-    events = net.make_events(("gemm_forward", "gemm_dx"), layers=mid)
-    net.capture(warmup=1, events=events)
+        rd = inputs.layer_inputs(inputs.scaled(spec, seed=dp.rank_seed(spec.seed, rank)))
+        data = dict(data, X=rd["X"], dY=rd["dY"])
+    st, _ = make_step(spec, dev, data)
+    flops = st.flops()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    flops = net.flops_per_step()
+    # the timed graph brackets every launch group with events on the launching
+    # stream; the kernels are long enough (tens to hundreds of us) that the
+    # event pairs cost them little
+    ev = st.make_events()
+    st.capture(warmup=1, events=ev)
 
     def one_step():
-        net.replay()
-        dp.allreduce_grads(net.grad_flat)
+        st.replay()
+        dp.allreduce_grads(st.grad_flat)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -269,7 +465,7 @@ def run_ours(args):
     # ---------------- timed region (device time, L2 flushed between steps)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    kt = {"gemm_forward": [], "gemm_dx": []}
+    per = {p: [] for p in step_mod.PARTS}
     gpu_id = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[local] \
         if os.environ.get("CUDA_VISIBLE_DEVICES") else str(local)
     dp.barrier(dev)
@@ -280,9 +476,10 @@ def run_ours(args):
             starts[k].record()
             one_step()
             ends[k].record()
+            # the graph's events hold the latest replay: read them before the next
             ends[k].synchronize()
-            for name in kt:
-                kt[name].extend(events[name][i][0].elapsed_time(events[name][i][1]) for i in mid)
+            for p in step_mod.PARTS:
+                per[p].append(ev[p][0].elapsed_time(ev[p][1]))
         torch.cuda.synchronize()
     dp.barrier(dev)
     total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
@@ -292,7 +489,7 @@ def run_ours(args):
     # ---------------- end to end through the public API with host buffers
     Xh = torch.from_numpy(data["X"]).to(torch.bfloat16).pin_memory()
     dYh = torch.from_numpy(data["dY"]).to(torch.bfloat16).pin_memory()
-    gh = torch.empty(net.grad_flat.shape, dtype=torch.float32).pin_memory()
+    gh = torch.empty(st.grad_flat.shape, dtype=torch.float32).pin_memory()
     e_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     e_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     dp.barrier(dev)
@@ -300,10 +497,10 @@ def run_ours(args):
     for k in range(args.steps):
         flush.zero_()
         e_s[k].record()
-        net.X.copy_(Xh, non_blocking=True)
-        net.dY.copy_(dYh, non_blocking=True)
+        st.X.copy_(Xh, non_blocking=True)
+        st.dY.copy_(dYh, non_blocking=True)
         one_step()
-        gh.copy_(net.grad_flat, non_blocking=True)
+        gh.copy_(st.grad_flat, non_blocking=True)
         e_e[k].record()
     torch.cuda.synchronize()
     dp.barrier(dev)
@@ -312,46 +509,59 @@ def run_ours(args):
     h2d = Xh.numel() * 2 + dYh.numel() * 2
     d2h = gh.numel() * 4
 
-    # ---------------- roofline of the dominant kernel
-    peaks, peak_src = load_peaks()
-    fwd_ms = statistics.mean(kt["gemm_forward"])
-    dx_ms = statistics.mean(kt["gemm_dx"])
-    fl_launch = 2.0 * 1024 * 1024 * 1024
-    if dx_ms >= fwd_ms:
-        dom, ms = "gemm_dx (k3_dx_dequant_kernel, 1024x1024x1024 bf16)", dx_ms
-        peak = peaks["bf16_tflops"]
-        peak_note = "%s bf16 dense burst" % peak_src
-        traffic = profiled_traffic("k3_dx_dequant_kernel", ["k3_dx.cu", "ptx.cuh"])
+    # ---------------- roofline of the dominant kernel and of the step
+    M, K, N, r = spec.M, spec.K, spec.N, spec.r
+    kern = {p: roof.part(p, 1e3 * statistics.mean(per[p]), M, K, N, r, 2) for p in step_mod.PARTS}
+    dom = max(kern, key=lambda p: kern[p]["us"])
+    kd = kern[dom]
+    name, bound = PART_KERNELS[dom]
+    if bound == "hbm":
+        roofline = {"bound": "hbm", "achieved": kd["GB/s"], "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": kd["frac_hbm"]}
     else:
-        dom, ms = "gemm_forward (k2_gemm_i8_lora_kernel, 1024x1024x1024 int8)", fwd_ms
-        peak = 2.0 * peaks["bf16_tflops"]
-        peak_note = "%s bf16 dense burst x 2 (nominal int8:bf16 ratio)" % peak_src
-        traffic = profiled_traffic("k2_gemm_i8_lora_kernel", ["k2_gemm_i8.cu", "ptx.cuh"])
-    achieved = fl_launch / (ms * 1e-3) / 1e12
-    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved / peak, "traffic": traffic, "kernel": dom,
-            "peak_source": peak_note, "avg_launch_us": ms * 1e3,
-            "launches_timed": len(kt["gemm_dx"]),
-            "other": {"gemm_forward_us": fwd_ms * 1e3, "gemm_dx_us": dx_ms * 1e3}}
+        peak = peaks["bf16_tflops"] * (2.0 if bound == "tensor_i8" else 1.0)
+        roofline = {"bound": "tensor", "achieved": kd["T(FL)OP/s"], "peak": peak,
+                    "unit": "TFLOP/s", "frac": kd["frac_tensor"]}
+    roofline.update({
+        "traffic": profiled_traffic(name, WORKLOAD), "kernel": "%s (%s, %dx%dx%d bf16)" % (name, dom, M, K, N),
+        "peak_source": "%s %s" % (peak_src, "HBM copy" if bound == "hbm" else
+                                  "bf16 dense burst" + (" x 2 (nominal int8:bf16 ratio)"
+                                                        if bound == "tensor_i8" else "")),
+        "avg_launch_us": kd["us"], "algorithmic_per_launch": kd["bytes"] if bound == "hbm"
+        else 2.0 * M * N * K, "launches_timed": len(per[dom])})
+    t_roof = roof.step_roof_us(M, K, N, r, 2)
+    ms_step = total_ms / args.steps
+    step_roof = {"t_roof_us": t_roof, "t_measured_us": 1e3 * ms_step,
+                 "frac": t_roof / (1e3 * ms_step),
+                 "rule": "max(2MNK/P_i8, bytes_fwd/BW) + max(2MNK/P_bf16, bytes_dx/BW) + "
+                         "(bytes_quantize + bytes_dY_pass + bytes_X_pass)/BW"}
+
+    configs, merge = None, None
+    if rank == 0 and world == 1 and not args.no_configs:
+        st.graph = None
+        configs, merge = all_configs(dev, flush, roof, args.config_steps, args.only)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(specs, data)
+        cpu = cpu_baseline(spec, data)
 
     clk = clocks.summary()
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+                "ms_per_step": ms_step, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-                "data": "synthetic (seeded; random-init weights of the MNIST MLP shapes)",
-                "config": config_dict(world, 1024),
+                "data": "synthetic (seeded; random-init weights of the 4096x4096 layer)",
+                "config": head_config(world),
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},
-                "gpu_launches": net.launches_per_step() * args.steps,
-                "roofline": roof, "cpu_baseline": cpu, "clocks": clk}
+                "gpu_launches": st.launches_per_step() * args.steps,
+                "roofline": roofline, "step_roofline": step_roof, "kernels": kern,
+                "cpu_baseline": cpu, "clocks": clk,
+                "peaks": dict(peaks, source=peak_src),
+                "merge": merge, "configs": configs}
         print(json.dumps(line), flush=True)
-    net.graph = None
+    st.graph = None
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -365,6 +575,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="headline only")
+    ap.add_argument("--config-steps", type=int, default=10, help="timed steps per config layer")
+    ap.add_argument("--only", default="", help="time only the config layers whose name contains this")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         log("warmup raised to 3")
