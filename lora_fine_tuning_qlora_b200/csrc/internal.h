@@ -14,7 +14,7 @@ enum Act { kF32 = 0, kBF16 = 1 };
 // ---------------------------------------------------------------- K1 / a0
 // Xq, sx (bit-exact quantization) and xA = X . A, one pass over X.
 cudaError_t launch_quantize_rows(Act act, const void* X, const float* A, int M, int K, int r,
-                                 int8_t* Xq, float* sx, float* xA, cudaStream_t s);
+                                 int8_t* Xq, float* sx, float* xA, int* status, cudaStream_t s);
 // W [K,N] fp32 -> Wq [N,K], sw [N].
 cudaError_t launch_quantize_weight(const float* W, int K, int N, int8_t* Wq, float* sw,
                                    cudaStream_t s);
@@ -123,8 +123,6 @@ int sm_count();
 // Launches `kern` with programmatic stream serialization (the kernel starts
 // while its predecessor drains; it calls pdl_wait() before touching global
 // memory), optionally as thread-block clusters of cluster_y CTAs along y.
-// Disabled (ordinary serialization) when QLORA_PDL=0.
-bool pdl_enabled();
 template <typename... KArgs, typename... Args>
 cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                      int cluster_y, Args... args) {
@@ -135,11 +133,9 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
     int n = 0;
-    if (pdl_enabled()) {
-        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[n].val.programmaticStreamSerializationAllowed = 1;
-        ++n;
-    }
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
     if (cluster_y > 1) {
         attr[n].id = cudaLaunchAttributeClusterDimension;
         attr[n].val.clusterDim.x = 1;
@@ -152,9 +148,6 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
     return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
-// Tile-shape override for tuning sweeps: the integer value of environment
-// variable `name`, read once, or -1 when it is unset.
-int tile_override(const char* name);
 // Minimum rows per CTA of the column-sum passes (dB/dbias, dA); 0 = default.
 int rank_pass_rows();
 

@@ -15,6 +15,7 @@
 // walks over many row groups, so A is read from L2 once per CTA, not per row.
 #include "internal.h"
 #include "ptx.cuh"
+#include "tile_epilogue.cuh"
 
 namespace qlora {
 
@@ -449,6 +450,356 @@ cudaError_t launch_rows_rp(const T* X, const float* A, int M, int K, int r, int8
                     K, r, a_chunks, Xq, sx, xA);
 }
 
+// ------------------------------------------------------------------ staged K1
+// bf16 rows, rank <= 8, rows of at most 256 * CPT 8-element chunks.
+//
+// Rows stream through a ring of shared-memory stages, each filled by one
+// bulk copy of R consecutive rows (four per row group, up to 32 KB), so that
+// a CTA keeps up to five stages (160 KB) of loads in flight with one
+// instruction per stage.  Eight consumer warps form row groups of TPR threads
+// (TPR a multiple of 32 covering the row); a thread owns one or two 8-element
+// chunks of the row and holds the matching rows of A in registers, so x.A
+// costs no shared-memory traffic.
+// Per stage a row group takes two sweeps over its staged rows: the abs-max,
+// then the codes (written as 8-byte stores) and the x.A partial sums, as
+// paired fp32 FMAs over neighbouring elements (the two lanes of a pair are
+// added at the end).  Both reductions over the group's threads go through a
+// transposing warp butterfly (one shuffle per value and lane step) and,
+// across warps, one named barrier each.
+namespace staged {
+// consumer threads: row groups of TPR threads, 256 in all (eight warps: more
+// warps, at one chunk per thread, measured slower at 16384 x 4096)
+template <int RP>
+__host__ __device__ constexpr int max_cons() { return 256; }
+template <int TPR, int RP>
+__host__ __device__ constexpr int groups() { return max_cons<RP>() / TPR; }
+template <int TPR, int RP>
+__host__ __device__ constexpr int cons() { return groups<TPR, RP>() * TPR; }
+constexpr int kRPG = 4;                 // rows per group per stage
+constexpr int kSmemBudget = 160 * 1024;
+constexpr int kMaxStages = 8;
+}  // namespace staged
+
+struct StagedArgs {
+    const __nv_bfloat16* X;
+    const float* A;
+    int M, K, r;
+    int8_t* Xq;
+    float* sx;
+    float* xA;
+    int rows_per_stage;    // R = groups * kRPG
+    uint32_t stage_bytes;  // R * K * 2, rounded up to 128
+    int nstages;           // ring depth S
+    int stages_total;      // ceil(M / R)
+};
+
+// 8 bf16 (16 bytes) -> 8 floats (exact)
+__device__ __forceinline__ void bf16x8_to_f(const uint4 u, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+// Symmetric abs-max codes of 8 values: rne(fl(v * inv)).  The products are
+// rounded to fp32 first (paired multiplies), then converted with round half
+// to even; |fl(v * inv)| <= 127 * (1 + 2^-24)^2 < 127.5, so no clamp is
+// reached.  (The rounding has to stay a separate step: a fused multiply-add
+// with 1.5 * 2^23 would round the exact product instead and break ties such
+// as v = amax / 2 differently.)  The low byte of each int is the code.
+__device__ __forceinline__ uint2 codes8(const float (&f)[8], unsigned long long inv2) {
+    uint32_t b[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        unsigned long long y;
+        asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(pk2(f[2 * i], f[2 * i + 1])), "l"(inv2));
+        float lo, hi;
+        unpk2(y, lo, hi);
+        b[2 * i] = static_cast<uint32_t>(__float2int_rn(lo));
+        b[2 * i + 1] = static_cast<uint32_t>(__float2int_rn(hi));
+    }
+    const uint32_t w0 = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+    const uint32_t w1 = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
+    return make_uint2(w0, w1);
+}
+
+template <int TPR, int CPT, int RP>
+__global__ void __launch_bounds__(staged::cons<TPR, RP>() + 32, 1)
+    k1_quantize_rows_staged_kernel(StagedArgs a, int* status) {
+    using namespace staged;
+    constexpr int kCons = cons<TPR, RP>();
+    constexpr int G = groups<TPR, RP>();  // row groups
+    constexpr int W = TPR / 32;     // warps per group
+    constexpr int V = kRPG * RP;    // x.A partial sums per thread and stage
+    static_assert(V <= 32, "transposed reduction width");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~static_cast<uintptr_t>(127));
+    const int S = a.nstages;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(S) * a.stage_bytes);
+    uint64_t* empty = full + kMaxStages;
+    float* redA = reinterpret_cast<float*>(empty + kMaxStages);  // [G][kRPG][W]
+    float* redX = redA + G * kRPG * W;                           // [G][W][V]
+    int* abort_flag = reinterpret_cast<int*>(redX + G * W * V);  // [G]
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int K = a.K;
+    const int nch = K >> 3;
+    const int R = a.rows_per_stage;
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kCons / 32);
+        }
+        for (int g = 0; g < G; ++g) abort_flag[g] = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    pdl_trigger();
+    pdl_wait();
+
+    if (warp == kCons / 32) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            int k = 0;
+            for (int st = blockIdx.x; st < a.stages_total; st += gridDim.x, ++k) {
+                const int slot = k % S;
+                if (k >= S && !mbar_wait(&empty[slot], ((k / S) - 1) & 1, status)) break;
+                const int row0 = st * R;
+                const int rows = min(R, a.M - row0);
+                const uint32_t bytes = static_cast<uint32_t>(rows) * static_cast<uint32_t>(K) * 2u;
+                mbar_arrive_expect_tx(&full[slot], bytes);
+                bulk_load(smem + static_cast<size_t>(slot) * a.stage_bytes,
+                          a.X + static_cast<size_t>(row0) * K, bytes, &full[slot]);
+            }
+            // every copy issued has landed before the CTA may exit
+            for (int j = k > S ? k - S : 0; j < k; ++j) mbar_wait(&full[j % S], (j / S) & 1, status);
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------- consumers
+    const int g = tid / TPR;
+    const int t = tid % TPR;
+    const int w = t >> 5;
+    // rows of A for this thread's chunks, as (A[k][j], A[k+1][j]) pairs of
+    // neighbouring k (k = 8c + 2p)
+    unsigned long long a2[CPT][4][RP];
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const int c = t + i * TPR;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const int k = c < nch ? c * 8 + 2 * p : 0;
+#pragma unroll
+            for (int j = 0; j < RP; ++j) {
+                const bool in = c < nch && j < a.r;
+                const float v0 = in ? __ldg(a.A + static_cast<size_t>(k) * a.r + j) : 0.f;
+                const float v1 = in ? __ldg(a.A + static_cast<size_t>(k + 1) * a.r + j) : 0.f;
+                a2[i][p][j] = pk2(v0, v1);
+            }
+        }
+    }
+
+    int k = 0;
+    for (int st = blockIdx.x; st < a.stages_total; st += gridDim.x, ++k) {
+        const int slot = k % S;
+        bool ok = mbar_wait(&full[slot], (k / S) & 1, status);
+        ok = __all_sync(0xffffffffu, ok);
+        const uint8_t* gbase = smem + static_cast<size_t>(slot) * a.stage_bytes +
+                               static_cast<size_t>(g * kRPG) * K * 2;
+        const int m0 = st * R + g * kRPG;
+
+        // ---- sweep 1: abs-max of each row
+        float amax[kRPG];
+#pragma unroll
+        for (int q = 0; q < kRPG; ++q) {
+            __nv_bfloat162 m2 = __float2bfloat162_rn(0.f);
+            if (ok) {
+#pragma unroll
+                for (int i = 0; i < CPT; ++i) {
+                    const int c = t + i * TPR;
+                    if (c < nch) {
+                        const uint4 u = *reinterpret_cast<const uint4*>(gbase + static_cast<size_t>(q) * K * 2 + c * 16);
+                        const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                        for (int h = 0; h < 4; ++h)
+                            m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&wv[h])));
+                    }
+                }
+            }
+            amax[q] = fmaxf(__low2float(m2), __high2float(m2));
+        }
+        {
+            float v[kRPG];
+#pragma unroll
+            for (int q = 0; q < kRPG; ++q) v[q] = amax[q];
+            const float x = xreduce<kRPG, true>(v);
+            if constexpr (W == 1) {
+#pragma unroll
+                for (int q = 0; q < kRPG; ++q) amax[q] = __shfl_sync(0xffffffffu, x, xreduce_lane<kRPG>(q));
+            } else {
+                if ((lane & (32 / kRPG - 1)) == 0) redA[(g * kRPG + xreduce_index<kRPG>(lane)) * W + w] = x;
+                if (!ok) abort_flag[g] = 1;
+                named_bar_sync(1 + g, TPR);
+                if (abort_flag[g]) break;
+#pragma unroll
+                for (int q = 0; q < kRPG; ++q) {
+                    float mx = redA[(g * kRPG + q) * W];
+#pragma unroll
+                    for (int ww = 1; ww < W; ++ww) mx = fmaxf(mx, redA[(g * kRPG + q) * W + ww]);
+                    amax[q] = mx;
+                }
+            }
+        }
+        if (!ok) break;
+
+        // ---- sweep 2: codes and x.A (xa[q][j] holds two partial sums)
+        unsigned long long xa[kRPG][RP];
+#pragma unroll
+        for (int q = 0; q < kRPG; ++q)
+#pragma unroll
+            for (int j = 0; j < RP; ++j) xa[q][j] = 0ull;
+#pragma unroll
+        for (int q = 0; q < kRPG; ++q) {
+            const float inv = amax[q] > 0.f ? __fdiv_rn(127.0f, amax[q]) : 0.f;
+            const unsigned long long inv2 = pk2(inv, inv);
+            const int m = m0 + q;
+            int8_t* qrow = a.Xq + static_cast<size_t>(m) * K;
+#pragma unroll
+            for (int i = 0; i < CPT; ++i) {
+                const int c = t + i * TPR;
+                if (c < nch) {
+                    const uint4 u = *reinterpret_cast<const uint4*>(gbase + static_cast<size_t>(q) * K * 2 + c * 16);
+                    float f[8];
+                    bf16x8_to_f(u, f);
+                    const uint2 cw = codes8(f, inv2);
+                    if (m < a.M) *reinterpret_cast<uint2*>(qrow + c * 8) = cw;
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        const unsigned long long x2 = pk2(f[2 * p], f[2 * p + 1]);
+#pragma unroll
+                        for (int j = 0; j < RP; ++j) fma2(xa[q][j], x2, a2[i][p][j]);
+                    }
+                }
+            }
+        }
+        // the stage's rows are no longer read: release the slot
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+        if (t < kRPG && m0 + t < a.M) {
+            float am = amax[0];
+#pragma unroll
+            for (int q = 1; q < kRPG; ++q) am = t == q ? amax[q] : am;
+            a.sx[m0 + t] = __fdiv_rn(am, 127.0f);
+        }
+
+        float v[V];
+#pragma unroll
+        for (int q = 0; q < kRPG; ++q)
+#pragma unroll
+            for (int j = 0; j < RP; ++j) {
+                float lo, hi;
+                unpk2(xa[q][j], lo, hi);
+                v[q * RP + j] = lo + hi;
+            }
+        const float x = xreduce<V, false>(v);
+        const int idx = xreduce_index<V>(lane);
+        if constexpr (W == 1) {
+            if ((lane & (32 / V - 1)) == 0) {
+                const int q = idx / RP, j = idx % RP;
+                if (m0 + q < a.M && j < a.r) a.xA[static_cast<size_t>(m0 + q) * a.r + j] = x;
+            }
+        } else {
+            if ((lane & (32 / V - 1)) == 0) redX[(g * W + w) * V + idx] = x;
+            named_bar_sync(1 + g, TPR);
+            if (t < V) {
+                float sum = redX[(g * W) * V + t];
+#pragma unroll
+                for (int ww = 1; ww < W; ++ww) sum += redX[(g * W + ww) * V + t];
+                const int q = t / RP, j = t % RP;
+                if (m0 + q < a.M && j < a.r) a.xA[static_cast<size_t>(m0 + q) * a.r + j] = sum;
+            }
+        }
+    }
+}
+
+template <int TPR, int CPT, int RP>
+cudaError_t launch_staged(const __nv_bfloat16* X, const float* A, int M, int K, int r, int8_t* Xq,
+                          float* sx, float* xA, int* status, cudaStream_t s) {
+    using namespace staged;
+    constexpr int G = groups<TPR, RP>();
+    constexpr int W = TPR / 32;
+    constexpr int V = kRPG * RP;
+    StagedArgs a{};
+    a.X = X;
+    a.A = A;
+    a.M = M;
+    a.K = K;
+    a.r = r;
+    a.Xq = Xq;
+    a.sx = sx;
+    a.xA = xA;
+    a.rows_per_stage = G * kRPG;
+    a.stage_bytes = (static_cast<uint32_t>(a.rows_per_stage) * K * 2u + 127u) & ~127u;
+    int S = kSmemBudget / static_cast<int>(a.stage_bytes);
+    S = S > kMaxStages ? kMaxStages : S;
+    if (S < 2) return cudaErrorInvalidValue;
+    a.nstages = S;
+    a.stages_total = (M + a.rows_per_stage - 1) / a.rows_per_stage;
+    const size_t smem = 128 + static_cast<size_t>(S) * a.stage_bytes + 2 * kMaxStages * 8 +
+                        4 * (G * kRPG * W + G * W * V + G);
+    auto kern = k1_quantize_rows_staged_kernel<TPR, CPT, RP>;
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const int grid = a.stages_total < sm_count() ? a.stages_total : sm_count();
+    return launch_k(kern, dim3(grid), dim3(cons<TPR, RP>() + 32), smem, s, 1, a, status);
+}
+
+template <int CPT, int RP>
+cudaError_t launch_staged_cpt(int nch, const __nv_bfloat16* X, const float* A, int M, int K, int r,
+                              int8_t* Xq, float* sx, float* xA, int* status, cudaStream_t s) {
+    constexpr int cap = staged::max_cons<RP>();
+    const int need = (nch + CPT - 1) / CPT;  // threads per row
+    if (need <= 32) return launch_staged<32, CPT, RP>(X, A, M, K, r, Xq, sx, xA, status, s);
+    if (need <= 64) return launch_staged<64, CPT, RP>(X, A, M, K, r, Xq, sx, xA, status, s);
+    if (need <= 96) return launch_staged<96, CPT, RP>(X, A, M, K, r, Xq, sx, xA, status, s);
+    if (need <= 128) return launch_staged<128, CPT, RP>(X, A, M, K, r, Xq, sx, xA, status, s);
+    if (need <= 192) return launch_staged<192, CPT, RP>(X, A, M, K, r, Xq, sx, xA, status, s);
+    if (need <= 256) return launch_staged<256, CPT, RP>(X, A, M, K, r, Xq, sx, xA, status, s);
+    if constexpr (cap >= 512) {
+        if (need <= 384) return launch_staged<384, CPT, RP>(X, A, M, K, r, Xq, sx, xA, status, s);
+        if (need <= 512) return launch_staged<512, CPT, RP>(X, A, M, K, r, Xq, sx, xA, status, s);
+    }
+    return cudaErrorNotSupported;
+}
+
+// one chunk per thread while a row fits the consumer threads, else two
+template <int RP>
+cudaError_t launch_staged_rp(const __nv_bfloat16* X, const float* A, int M, int K, int r,
+                             int8_t* Xq, float* sx, float* xA, int* status, cudaStream_t s) {
+    const int nch = K / 8;
+    if (nch <= staged::max_cons<RP>())
+        return launch_staged_cpt<1, RP>(nch, X, A, M, K, r, Xq, sx, xA, status, s);
+    if constexpr (RP <= 4) {
+        if (nch <= 2 * staged::max_cons<RP>())
+            return launch_staged_cpt<2, RP>(nch, X, A, M, K, r, Xq, sx, xA, status, s);
+    }
+    return cudaErrorNotSupported;
+}
+
+// The staged kernel when it applies (bf16, r <= 8, rows short enough for the
+// consumer threads at one or two chunks each); cudaErrorNotSupported otherwise.
+cudaError_t launch_rows_staged(const __nv_bfloat16* X, const float* A, int M, int K, int r,
+                               int8_t* Xq, float* sx, float* xA, int* status, cudaStream_t s) {
+    if (r <= 4) return launch_staged_rp<4>(X, A, M, K, r, Xq, sx, xA, status, s);
+    if (r <= 8) return launch_staged_rp<8>(X, A, M, K, r, Xq, sx, xA, status, s);
+    return cudaErrorNotSupported;
+}
+
 template <typename T>
 cudaError_t launch_rows_t(const T* X, const float* A, int M, int K, int r, int8_t* Xq, float* sx,
                           float* xA, cudaStream_t s) {
@@ -512,9 +863,13 @@ __global__ void __launch_bounds__(256) k_quantize_weight_kernel(const float* __r
 }  // namespace
 
 cudaError_t launch_quantize_rows(Act act, const void* X, const float* A, int M, int K, int r,
-                                 int8_t* Xq, float* sx, float* xA, cudaStream_t s) {
-    if (act == kBF16)
+                                 int8_t* Xq, float* sx, float* xA, int* status, cudaStream_t s) {
+    if (act == kBF16) {
+        const cudaError_t e = launch_rows_staged(static_cast<const __nv_bfloat16*>(X), A, M, K, r,
+                                                 Xq, sx, xA, status, s);
+        if (e != cudaErrorNotSupported) return e;
         return launch_rows_t(static_cast<const __nv_bfloat16*>(X), A, M, K, r, Xq, sx, xA, s);
+    }
     return launch_rows_t(static_cast<const float*>(X), A, M, K, r, Xq, sx, xA, s);
 }
 

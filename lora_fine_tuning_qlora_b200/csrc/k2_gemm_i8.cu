@@ -41,7 +41,7 @@ template <bool W4>
 __host__ __device__ constexpr int k2_threads() { return kThreads + (W4 ? 32 * kUnpackWarps : 0); }
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory
 
-template <int BN, typename OutT, int RMAX>
+template <int BN, typename OutT, int RMAX, bool SPLIT = false>
 struct K2Cfg {
     static constexpr bool kLoraMMA = RMAX <= 16;
     static constexpr bool kSplit = sizeof(OutT) == 4;      // 3 x tf32 for fp32 outputs
@@ -51,7 +51,12 @@ struct K2Cfg {
     static constexpr int kBtBytes = kLoraMMA ? BN * kKL * 4 : 0;
     static constexpr int kBufBytes = kTerms * (kXtBytes + kBtBytes) + BN * 4 * 2;  // + sw, bias
     static constexpr int kStgBytes = kEpiWarps * 32 * stage_pitch<OutT>();
-    static constexpr int kFixed = kStgBytes + 2 * kBufBytes + 512 + 1024;
+    // split-K: the partial accumulators of this CTA's rows from every CTA of
+    // the cluster, [S][128 / S rows][BN] int32, rows padded by 16 bytes
+    // (conflict-free 16-byte accesses by per-lane rows)
+    static constexpr int kRedPitch = BN + 4;
+    static constexpr int kRedBytes = SPLIT ? kBM * kRedPitch * 4 : 0;
+    static constexpr int kFixed = kStgBytes + 2 * kBufBytes + kRedBytes + 512 + 1024;
     // k per stage: two 128-byte blocks (one 3-D TMA box per operand) where
     // two such stages fit, else one
     static constexpr int kBlk = (kSmemLimit - kFixed) / ((kBM + BN) * 2 * kBlkK) >= 2 ? 2 : 1;
@@ -64,10 +69,12 @@ struct K2Cfg {
     static_assert(STAGES >= 2, "shared memory budget");
     static constexpr int kStgOff = STAGES * kStageBytes;
     static constexpr int kBufOff = kStgOff + kStgBytes;
-    static constexpr int kBarOff = kBufOff + 2 * kBufBytes;
+    static constexpr int kRedOff = kBufOff + 2 * kBufBytes;
+    static constexpr int kBarOff = kRedOff + kRedBytes;
     static constexpr int kTotal = kBarOff + 512 + 1024;
     static constexpr uint32_t kAccCols = 2 * BN;             // int32 acc + fp32 rank-r acc
-    static constexpr uint32_t kTmemCols = 2 * kAccCols;
+    // split-K CTAs take one tile each: one accumulator buffer
+    static constexpr uint32_t kTmemCols = SPLIT ? kAccCols : 2 * kAccCols;
     static_assert(kTmemCols <= 512, "TMEM");
 };
 
@@ -75,12 +82,22 @@ struct K2Cfg {
 // the low nibble) instead of int8 codes behind tmB; warps 10..13 expand each
 // stage's codes into the int8 tile the TMA would have written (128B swizzle,
 // K-major), and the MMA waits for them as well as for the Xq tile.
-template <int BN, typename OutT, int RMAX, bool W4>
+//
+// SPLIT: split-K for grids that would leave SMs idle.  The grid is tiles x S
+// (S = 2, 4 or 8) with clusters of the S CTAs of one tile (along y); CTA s
+// runs k-blocks [s nkb / S, (s+1) nkb / S) of its tile.  Rows
+// [s 128/S, (s+1) 128/S) of the tile belong to CTA s: every CTA stores its
+// int32 partial of those rows into CTA s's shared memory (distributed shared
+// memory, one slot per CTA) and arrives on CTA s's barrier; CTA s adds the S
+// slots (in slot order) and runs the epilogue of its rows.  Every CTA issues
+// the rank-r MMAs of the whole tile (a few tf32 MMAs) and uses its rows.
+template <int BN, typename OutT, int RMAX, bool W4, bool SPLIT>
 __global__ void __launch_bounds__(k2_threads<W4>(), 1)
     k2_gemm_i8_lora_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmB, int k3d, int M, int N, int K,
                            const uint8_t* __restrict__ Wp, FwdEpilogue ep, int* status) {
-    using C = K2Cfg<BN, OutT, RMAX>;
+    using C = K2Cfg<BN, OutT, RMAX, SPLIT>;
+    static_assert(!(SPLIT && W4), "split-K runs on int8 codes");
     constexpr int S = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -91,13 +108,18 @@ __global__ void __launch_bounds__(k2_threads<W4>(), 1)
     uint64_t* tempty = tfull + 2;   // [2]
     uint64_t* lready = tempty + 2;  // [2] rank-r operand tables written
     uint64_t* wready = lready + 2;  // [S] packed int4 kernels: the stage's int8 codes written
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wready + S);
+    uint64_t* rbar = wready + S;    // split-K leader: every CTA's partial has been added
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + 1);
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     const int num_n = (N + BN - 1) / BN;
     const int tiles = ((M + kBM - 1) / kBM) * num_n;
     const int nkb = (K + C::kBK - 1) / C::kBK;
+    const int split = SPLIT ? static_cast<int>(blockIdx.y) : 0;
+    const int nsplit = SPLIT ? static_cast<int>(gridDim.y) : 1;
+    const int kb0 = split * nkb / nsplit;
+    const int kb1 = (split + 1) * nkb / nsplit;
     pdl_trigger();
 
     if (threadIdx.x == 0) {
@@ -112,8 +134,10 @@ __global__ void __launch_bounds__(k2_threads<W4>(), 1)
         }
         if constexpr (W4)
             for (int s = 0; s < S; ++s) mbar_init(&wready[s], kUnpackWarps);
+        if constexpr (SPLIT) mbar_init(rbar, 2u * kBM);  // every CTA: its rows' partials, two column halves
         fence_mbar_init();
     }
+
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
@@ -122,6 +146,9 @@ __global__ void __launch_bounds__(k2_threads<W4>(), 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // split-K: no CTA stores into another's slots before that CTA's barrier
+    // is initialised (every warp waits on this arrival once, below)
+    if constexpr (SPLIT) cluster_arrive();
     pdl_wait();  // the prologue above touched no global memory
 
     if (warp == 0) {
@@ -134,7 +161,7 @@ __global__ void __launch_bounds__(k2_threads<W4>(), 1)
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
                 const int m0 = (t / num_n) * kBM;
                 const int n0 = (t % num_n) * BN;
-                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                for (int kb = kb0; kb < kb1; ++kb, ++g) {
                     const int s = g % S;
                     if (g >= S && !mbar_wait(&empty[s], ((g / S) - 1) & 1, status)) {
                         ok = false;
@@ -160,6 +187,7 @@ __global__ void __launch_bounds__(k2_threads<W4>(), 1)
             }
         }
         __syncwarp();
+        if constexpr (SPLIT) cluster_wait();
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -172,7 +200,7 @@ __global__ void __launch_bounds__(k2_threads<W4>(), 1)
                 if (use > 0 && !mbar_wait(&tempty[ab], (use - 1) & 1, status)) break;
                 tc_fence_after();
                 const uint32_t dacc = tmem + ab * C::kAccCols;
-                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                for (int kb = kb0; kb < kb1; ++kb, ++g) {
                     const int s = g % S;
                     if (!mbar_wait(&full[s], (g / S) & 1, status) ||
                         (W4 && !mbar_wait(&wready[s], (g / S) & 1, status))) {
@@ -189,7 +217,7 @@ __global__ void __launch_bounds__(k2_threads<W4>(), 1)
                                                       1024, kLayoutSw128);
                         const uint64_t bd = smem_desc(b_base + (kk >> 2) * (BN * kBlkK) + (kk & 3) * 32, 16,
                                                       1024, kLayoutSw128);
-                        mma_i8(dacc, ad, bd, idesc, (kb | kk) != 0);
+                        mma_i8(dacc, ad, bd, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
                     }
                     mma_commit(&empty[s]);
                 }
@@ -224,6 +252,7 @@ __global__ void __launch_bounds__(k2_threads<W4>(), 1)
             }
         }
         __syncwarp();
+        if constexpr (SPLIT) cluster_wait();
     } else if (W4 && warp >= 2 + kEpiWarps) {
         // ------------------------------------------------------ int4 unpack
         // Stage g's Wq tile, as the TMA would have written it: k-block b of
@@ -241,7 +270,7 @@ __global__ void __launch_bounds__(k2_threads<W4>(), 1)
         bool ok = true;
         for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
             const int n0 = (t % num_n) * BN;
-            for (int kb = 0; kb < nkb; ++kb, ++g) {
+            for (int kb = kb0; kb < kb1; ++kb, ++g) {
                 const int s = g % S;
                 uint4 raw[kPer];
                 uint32_t inb = 0;
@@ -351,15 +380,67 @@ __global__ void __launch_bounds__(k2_threads<W4>(), 1)
                     xa[j] = (row_ok && j < ep.r) ? ep.xA[static_cast<size_t>(row) * ep.r + j] * ep.c : 0.f;
             }
 
-            const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[ab], use & 1, status));
-            if (!ok) break;
+            bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[ab], use & 1, status));
             tc_fence_after();
             const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * C::kAccCols;
+            // split-K: this CTA's rows of the tile and where this lane's row lives
+            const int R = kBM / nsplit;
+            const int trow = q * 32 + lane;
+            const int own_lo = split * R;
+            int* slots = reinterpret_cast<int*>(smem + C::kRedOff);
+            if constexpr (SPLIT) {
+                cluster_wait();
+                const int owner = trow / R;
+                const uint32_t dst = dsmem_addr(slots + (split * R + trow % R) * C::kRedPitch,
+                                                static_cast<uint32_t>(owner));
+                if (ok) {
+#pragma unroll 1
+                    for (int col = half * (BN / 2); col < (half + 1) * (BN / 2); col += kEpiCols) {
+                        uint32_t v[kEpiCols];
+                        tmem_ld16(tbase + col, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < kEpiCols; e += 4)
+                            dsmem_st_v4(dst + 4u * static_cast<uint32_t>(col + e), v[e], v[e + 1], v[e + 2],
+                                        v[e + 3]);
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive_remote(dsmem_addr(rbar, static_cast<uint32_t>(owner)));
+                // every CTA's slots of this CTA's rows have landed
+                ok = __all_sync(0xffffffffu, mbar_wait_cluster(rbar, 0, status) && ok);
+                tc_fence_after();
+                if (own_lo >= q * 32 + 32 || own_lo + R <= q * 32) break;  // no rows of mine here
+            }
+            if (!ok) break;
+            const int row_min = SPLIT ? m0 + own_lo : 0;
+            const int row_lim = SPLIT ? min(M, m0 + own_lo + R) : M;
+            const bool own_row = !SPLIT || (trow >= own_lo && trow < own_lo + R);
 #pragma unroll 1
             for (int col = half * (BN / 2); col < (half + 1) * (BN / 2); col += kEpiCols) {
                 uint32_t v[kEpiCols];
                 uint32_t l[kEpiCols];
-                tmem_ld16(tbase + col, v);
+                if constexpr (SPLIT) {
+                    // the S partials of this row, added in slot order
+#pragma unroll
+                    for (int e = 0; e < kEpiCols; ++e) v[e] = 0u;
+                    if (own_row) {
+                        for (int sp = 0; sp < nsplit; ++sp) {
+                            const uint4* p = reinterpret_cast<const uint4*>(
+                                slots + (sp * R + trow - own_lo) * C::kRedPitch + col);
+#pragma unroll
+                            for (int e4 = 0; e4 < kEpiCols / 4; ++e4) {
+                                const uint4 w = p[e4];
+                                v[4 * e4 + 0] += w.x;
+                                v[4 * e4 + 1] += w.y;
+                                v[4 * e4 + 2] += w.z;
+                                v[4 * e4 + 3] += w.w;
+                            }
+                        }
+                    }
+                } else {
+                    tmem_ld16(tbase + col, v);
+                }
                 if constexpr (C::kLoraMMA) tmem_ld16(tbase + BN + col, l);
                 tmem_ld_wait();
                 float y[kEpiCols];
@@ -389,12 +470,13 @@ __global__ void __launch_bounds__(k2_threads<W4>(), 1)
 #pragma unroll
                     for (int e = 0; e < kEpiCols; ++e) y[e] = y[e] > 0.f ? y[e] : 0.f;
                 }
-                if (ep.acc && row_ok) {
+                if (ep.acc && row_ok && own_row) {
                     for (int e = 0; e < kEpiCols; ++e)
                         if (n0 + col + e < N)
                             ep.acc[static_cast<size_t>(row) * N + n0 + col + e] = static_cast<int32_t>(v[e]);
                 }
-                store_block<OutT>(stg, y, lane, Y, static_cast<size_t>(N), row0, M, n0 + col, N, vec);
+                store_block<OutT>(stg, y, lane, Y, static_cast<size_t>(N), row0, row_lim, n0 + col, N, vec,
+                                  row_min);
             }
             tc_fence_before();
             __syncwarp();
@@ -410,10 +492,10 @@ __global__ void __launch_bounds__(k2_threads<W4>(), 1)
     }
 }
 
-template <int BN, typename OutT, int RMAX, bool W4>
+template <int BN, typename OutT, int RMAX, bool W4, bool SPLIT = false>
 cudaError_t launch_cfg(const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
-                       const FwdEpilogue& ep, int* status, cudaStream_t s) {
-    using C = K2Cfg<BN, OutT, RMAX>;
+                       const FwdEpilogue& ep, int* status, cudaStream_t s, int nsplit = 1) {
+    using C = K2Cfg<BN, OutT, RMAX, SPLIT>;
     // Xq and Wq as [row][k-block of 128][128] (one 3-D box per operand and
     // stage) when K splits into whole blocks, else one 2-D box per block
     CUtensorMap ta, tb;
@@ -430,10 +512,13 @@ cudaError_t launch_cfg(const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
                                  CU_TENSOR_MAP_SWIZZLE_128B));
     if (!ok) return cudaErrorInvalidValue;
     if (W4) tb = ta;  // unused
-    auto kern = k2_gemm_i8_lora_kernel<BN, OutT, RMAX, W4>;
+    auto kern = k2_gemm_i8_lora_kernel<BN, OutT, RMAX, W4, SPLIT>;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), C::kTotal);
     if (e != cudaSuccess) return e;
     const int tiles = ((M + kBM - 1) / kBM) * ((N + BN - 1) / BN);
+    if constexpr (SPLIT)
+        return launch_k(kern, dim3(tiles, nsplit), dim3(k2_threads<W4>()), C::kTotal, s, nsplit, ta, tb,
+                        k3d, M, N, K, static_cast<const uint8_t*>(nullptr), ep, status);
     const int grid = tiles < sm_count() ? tiles : sm_count();
     return launch_k(kern, dim3(grid), dim3(k2_threads<W4>()), C::kTotal, s, 1, ta, tb, k3d, M, N, K,
                     W4 ? reinterpret_cast<const uint8_t*>(Wq) : nullptr, ep, status);
@@ -457,13 +542,34 @@ cudaError_t launch_r(int bn, const int8_t* Xq, const int8_t* Wq, int M, int N, i
 
 }  // namespace
 
+// Split-K factor for a bf16 layer whose 128 x 128 tiles would leave more than
+// half the SMs idle: the largest power of two (2, 4 or 8: one cluster, and
+// whole slices of the 128 tile rows) with tiles x S <= SMs and at least two
+// k-blocks per CTA; 1 = no split.
+int fwd_split(int M, int N, int K) {
+    using C = K2Cfg<128, __nv_bfloat16, 4, true>;
+    const int tiles = ((M + kBM - 1) / kBM) * ((N + 127) / 128);
+    const int nkb = (K + C::kBK - 1) / C::kBK;
+    int sp = 1;
+    while (sp < 8 && 2 * sp * tiles <= sm_count() && 2 * (2 * sp) <= nkb) sp *= 2;
+    return sp;
+}
+
 cudaError_t launch_gemm_i8_fwd(Act act, const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
                                const FwdEpilogue& ep, int* status, cudaStream_t s, bool w4) {
+    if (act == kBF16 && !w4 && ep.r <= 16) {
+        const int sp = fwd_split(M, N, K);
+        if (sp > 1) {
+            if (ep.r <= 4)
+                return launch_cfg<128, __nv_bfloat16, 4, false, true>(Xq, Wq, M, N, K, ep, status, s, sp);
+            if (ep.r <= 8)
+                return launch_cfg<128, __nv_bfloat16, 8, false, true>(Xq, Wq, M, N, K, ep, status, s, sp);
+            return launch_cfg<128, __nv_bfloat16, 16, false, true>(Xq, Wq, M, N, K, ep, status, s, sp);
+        }
+    }
     // Tile width: 128 columns unless that leaves SMs without a tile.
     const int mt = (M + kBM - 1) / kBM;
     int bn = mt * ((N + 127) / 128) >= sm_count() ? 128 : 64;
-    const int forced = tile_override("QLORA_FWD_BN");  // tuning: 64 or 128
-    if (forced == 64 || forced == 128) bn = forced;
     if (act == kBF16)
         return w4 ? launch_r<__nv_bfloat16, true>(bn, Xq, Wq, M, N, K, ep, status, s)
                   : launch_r<__nv_bfloat16, false>(bn, Xq, Wq, M, N, K, ep, status, s);

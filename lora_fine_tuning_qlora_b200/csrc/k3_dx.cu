@@ -678,8 +678,6 @@ cudaError_t launch_gemm_dx(Act act, const void* dY, const int8_t* Wq, const floa
     int cfg = 2;
     if (c1 < c2 && c1 <= c0) cfg = 1;
     else if (c0 < c2 && c0 < c1) cfg = 0;
-    const int forced = tile_override("QLORA_DX_TILE");  // tuning: 0, 1 or 2
-    if (forced >= 0 && forced <= 2) cfg = forced;
     return w4 ? launch_tc_r<true>(cfg, dY, Wq, sw, M, N, K, ep, status, s)
               : launch_tc_r<false>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
 }

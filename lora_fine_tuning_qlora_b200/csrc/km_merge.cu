@@ -99,20 +99,194 @@ __global__ void __launch_bounds__(kThreads) km_merge_kernel(const uint8_t* __res
     }
 }
 
+// ---------------------------------------------------------------- tiled merge
+// Ranks up to 8.  A CTA takes kNB = 8 output channels; each thread owns 16
+// consecutive k (one 16-byte chunk of int8 codes, or 8 bytes of packed int4)
+// per 4096-wide step of k and holds those rows of A in registers (eight at a
+// time), so A is read once per CTA and sweep, and reused for all eight
+// channels.  Sweep 1 forms w' and its per-channel abs-max, sweep 2 reads the
+// codes again (mostly from L2), recomputes w' with the same operations and
+// writes the new codes.  The arithmetic per element is the one of
+// merged_value, in the same order, so the result is bit-identical to it.
+constexpr int kNB = 8;
+constexpr int kKStep = kThreads * 16;
+
+// 16 int8 codes (k order) -> exact floats, by placing each code (offset by
+// 128) in the low mantissa byte of 2^23 and subtracting 2^23 + 128
+__device__ __forceinline__ void codes_to_f(const uint4 raw, float (&f)[16]) {
+    const uint32_t w[4] = {raw.x ^ 0x80808080u, raw.y ^ 0x80808080u, raw.z ^ 0x80808080u,
+                           raw.w ^ 0x80808080u};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[4 * i + 0] = __fsub_rn(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7540)), 8388736.0f);
+        f[4 * i + 1] = __fsub_rn(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7541)), 8388736.0f);
+        f[4 * i + 2] = __fsub_rn(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7542)), 8388736.0f);
+        f[4 * i + 3] = __fsub_rn(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7543)), 8388736.0f);
+    }
+}
+
+template <bool W4, int RP>
+__global__ void __launch_bounds__(kThreads, RP <= 4 ? 2 : 1) km_merge_tiled_kernel(const uint8_t* __restrict__ Wq,
+                                                                  const float* __restrict__ sw,
+                                                                  const float* __restrict__ A,
+                                                                  const float* __restrict__ B, int K,
+                                                                  int N, int r, float c,
+                                                                  uint8_t* __restrict__ Wq_out,
+                                                                  float* __restrict__ sw_out) {
+    constexpr float kLevels = W4 ? 7.0f : 127.0f;
+    __shared__ float sB[RP][kNB];
+    __shared__ float sS[kNB];
+    __shared__ float red[kThreads / 32][kNB];
+    __shared__ float s_amax[kNB];
+    pdl_trigger();
+    pdl_wait();
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int n0 = blockIdx.x * kNB;
+    if (t < RP * kNB) {
+        const int j = t / kNB, nb = t % kNB;
+        sB[j][nb] = (j < r && n0 + nb < N) ? B[static_cast<size_t>(j) * N + n0 + nb] : 0.f;
+    }
+    if (t < kNB) sS[t] = n0 + t < N ? sw[n0 + t] : 0.f;
+    __syncthreads();
+    const size_t row_bytes = W4 ? static_cast<size_t>(K) / 2 : static_cast<size_t>(K);
+
+    auto load_chunk = [&](int n, int k0) -> uint4 {
+        const uint8_t* p = Wq + static_cast<size_t>(n) * row_bytes;
+        if constexpr (W4) {
+            const uint2 v = __ldg(reinterpret_cast<const uint2*>(p + k0 / 2));
+            uint4 lo, hi;
+            unpack_int4x32(make_uint4(v.x, v.y, 0u, 0u), lo, hi);
+            return lo;  // codes k0 .. k0 + 15
+        } else {
+            return __ldg(reinterpret_cast<const uint4*>(p + k0));
+        }
+    };
+    // A rows k0 .. k0 + 7
+    auto load_a = [&](int k0, float (&a)[8][RP]) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+#pragma unroll
+            for (int j = 0; j < RP; ++j)
+                a[e][j] = j < r ? __ldg(A + static_cast<size_t>(k0 + e) * r + j) : 0.f;
+    };
+    // w'(k) for 8 k of channel nb (codes q), in the merge's fixed order
+    auto merged8 = [&](const float* q, int nb, const float (&a)[8][RP], float (&wp)[8]) {
+        const float s = sS[nb];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float w = __fmul_rn(q[e], s);
+            float d = __fmul_rn(a[e][0], sB[0][nb]);
+#pragma unroll
+            for (int j = 1; j < RP; ++j)
+                if (j < r) d = __fadd_rn(d, __fmul_rn(a[e][j], sB[j][nb]));
+            wp[e] = __fadd_rn(w, __fmul_rn(c, d));
+        }
+    };
+
+    float amax[kNB];
+#pragma unroll
+    for (int nb = 0; nb < kNB; ++nb) amax[nb] = 0.f;
+    for (int ks = 0; ks < K; ks += kKStep) {
+        const int k0 = ks + t * 16;
+        if (k0 >= K) break;
+        uint4 raw[kNB];
+#pragma unroll
+        for (int nb = 0; nb < kNB; ++nb)
+            raw[nb] = n0 + nb < N ? load_chunk(n0 + nb, k0) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float a[8][RP];
+            load_a(k0 + 8 * h, a);
+#pragma unroll
+            for (int nb = 0; nb < kNB; ++nb) {
+                float q[16], wp[8];
+                codes_to_f(raw[nb], q);
+                merged8(q + 8 * h, nb, a, wp);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) amax[nb] = fmaxf(amax[nb], fabsf(wp[e]));
+            }
+        }
+    }
+    {
+        const float x = xreduce<kNB, true>(amax);
+        if ((lane & (32 / kNB - 1)) == 0) red[warp][xreduce_index<kNB>(lane)] = x;
+    }
+    __syncthreads();
+    if (t < kNB) {
+        float m = red[0][t];
+#pragma unroll
+        for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[w][t]);
+        s_amax[t] = m;
+        if (n0 + t < N) sw_out[n0 + t] = __fdiv_rn(m, kLevels);
+    }
+    __syncthreads();
+
+    for (int ks = 0; ks < K; ks += kKStep) {
+        const int k0 = ks + t * 16;
+        if (k0 >= K) break;
+        uint4 raw[kNB];
+#pragma unroll
+        for (int nb = 0; nb < kNB; ++nb)
+            raw[nb] = n0 + nb < N ? load_chunk(n0 + nb, k0) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float a[8][RP];
+            load_a(k0 + 8 * h, a);
+#pragma unroll
+            for (int nb = 0; nb < kNB; ++nb) {
+                const int n = n0 + nb;
+                if (n >= N) break;
+                float q[16], wp[8];
+                codes_to_f(raw[nb], q);
+                merged8(q + 8 * h, nb, a, wp);
+                const float m = s_amax[nb];
+                const float inv = m > 0.f ? __fdiv_rn(kLevels, m) : 0.f;
+                uint8_t* orow = Wq_out + static_cast<size_t>(n) * row_bytes;
+                if constexpr (W4) {
+                    uint32_t v = 0u;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        v |= (static_cast<uint32_t>(quant_code_l<7>(wp[e], inv)) & 0xFu) << (4 * e);
+                    *reinterpret_cast<uint32_t*>(orow + (k0 + 8 * h) / 2) = v;
+                } else {
+                    uint32_t v[2] = {0u, 0u};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        v[e / 4] |= (static_cast<uint32_t>(quant_code(wp[e], inv)) & 0xFFu) << (8 * (e % 4));
+                    *reinterpret_cast<uint2*>(orow + k0 + 8 * h) = make_uint2(v[0], v[1]);
+                }
+            }
+        }
+    }
+}
+
+template <bool W4>
+cudaError_t launch_merge_t(const uint8_t* Wq, const float* sw, const float* A, const float* B,
+                           int K, int N, int r, float c, uint8_t* Wq_out, float* sw_out,
+                           cudaStream_t s) {
+    const dim3 grid((N + kNB - 1) / kNB);
+    if (r <= 4)
+        return launch_k(km_merge_tiled_kernel<W4, 4>, grid, dim3(kThreads), 0, s, 1, Wq, sw, A, B, K,
+                        N, r, c, Wq_out, sw_out);
+    if (r <= 8)
+        return launch_k(km_merge_tiled_kernel<W4, 8>, grid, dim3(kThreads), 0, s, 1, Wq, sw, A, B, K,
+                        N, r, c, Wq_out, sw_out);
+    km_merge_kernel<W4><<<N, kThreads, 0, s>>>(Wq, sw, A, B, K, N, r, c, Wq_out, sw_out);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_merge(const int8_t* Wq, const float* sw, const float* A, const float* B, int K,
                          int N, int r, float c, int8_t* Wq_out, float* sw_out, cudaStream_t s) {
-    km_merge_kernel<false><<<N, kThreads, 0, s>>>(reinterpret_cast<const uint8_t*>(Wq), sw, A, B, K,
-                                                  N, r, c, reinterpret_cast<uint8_t*>(Wq_out), sw_out);
-    return cudaGetLastError();
+    return launch_merge_t<false>(reinterpret_cast<const uint8_t*>(Wq), sw, A, B, K, N, r, c,
+                                 reinterpret_cast<uint8_t*>(Wq_out), sw_out, s);
 }
 
 cudaError_t launch_merge_int4(const uint8_t* Wp, const float* sw, const float* A, const float* B,
                               int K, int N, int r, float c, uint8_t* Wp_out, float* sw_out,
                               cudaStream_t s) {
-    km_merge_kernel<true><<<N, kThreads, 0, s>>>(Wp, sw, A, B, K, N, r, c, Wp_out, sw_out);
-    return cudaGetLastError();
+    return launch_merge_t<true>(Wp, sw, A, B, K, N, r, c, Wp_out, sw_out, s);
 }
 
 }  // namespace qlora

@@ -102,6 +102,12 @@ __device__ __forceinline__ void cluster_arrive_relaxed() {
     asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
 
+// arrive with release semantics: this thread's earlier shared-memory writes
+// are visible to every thread of the cluster that completes the wait
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void cluster_wait() {
     asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
 }
@@ -116,6 +122,20 @@ __device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
 
 __device__ __forceinline__ void dsmem_st(uint32_t addr, float v) {
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+// 16-byte store to a shared-memory address of a CTA of the cluster.
+__device__ __forceinline__ void dsmem_st_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                            uint32_t d) {
+    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b),
+                 "r"(c), "r"(d)
+                 : "memory");
+}
+
+// Atomic add of v to the int32 at a shared-memory address of a CTA of the
+// cluster (integer sums are exact whatever the order of the adds).
+__device__ __forceinline__ void dsmem_red_add(uint32_t addr, int v) {
+    asm volatile("red.relaxed.cluster.shared::cluster.add.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
 // Arrives on an mbarrier of another CTA of the cluster, releasing this
@@ -179,6 +199,19 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+// Untiled bulk copy of `bytes` contiguous bytes from global memory into this
+// CTA's shared memory, completing a transaction of that size on `bar`.  Both
+// addresses are 16-byte aligned and `bytes` is a multiple of 16 at the call
+// sites.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
 
@@ -333,6 +366,77 @@ __device__ __forceinline__ void tf32_split(float x, float& hi, float& lo) {
     asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(x));
     hi = __uint_as_float(h);
     lo = x - hi;
+}
+
+// ---------------------------------------------------------------------------
+// packed fp32 pairs (one instruction for two lanes of arithmetic, each lane
+// rounded like its scalar counterpart)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ unsigned long long pk2(float a, float b) {
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+__device__ __forceinline__ void unpk2(unsigned long long v, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+
+// d = a * b + d, lane-wise, fused (one rounding per lane)
+__device__ __forceinline__ void fma2(unsigned long long& d, unsigned long long a, unsigned long long b) {
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
+}
+
+// ---------------------------------------------------------------------------
+// warp reductions
+// ---------------------------------------------------------------------------
+// Sum (or max) of the V values v[] over the warp's 32 lanes, transposed:
+// returns one total per lane, lane l holding value xreduce_index<V>(l).
+// Every halving step sends half of the live values and keeps the other half.
+template <int V, bool MAX>
+__device__ __forceinline__ float xreduce(float (&v)[V]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int n = V, off = 16; n > 1; n >>= 1, off >>= 1) {
+        const bool up = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+            const float send = up ? v[i] : v[i + n / 2];
+            const float keep = up ? v[i + n / 2] : v[i];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, off);
+            v[i] = MAX ? fmaxf(keep, recv) : keep + recv;
+        }
+    }
+    float x = v[0];
+#pragma unroll
+    for (int off = 32 / V / 2; off >= 1; off >>= 1) {
+        const float y = __shfl_xor_sync(0xffffffffu, x, off);
+        x = MAX ? fmaxf(x, y) : x + y;
+    }
+    return x;
+}
+
+template <int V>
+__device__ __forceinline__ int xreduce_index(int lane) {
+    int idx = 0;
+#pragma unroll
+    for (int n = V, off = 16; n > 1; n >>= 1, off >>= 1)
+        if (lane & off) idx += n / 2;
+    return idx;
+}
+
+// a lane that holds value q after xreduce<V>
+template <int V>
+__device__ __forceinline__ int xreduce_lane(int q) {
+    int l = 0;
+#pragma unroll
+    for (int n = V, off = 16; n > 1; n >>= 1, off >>= 1) {
+        if (q >= n / 2) {
+            l |= off;
+            q -= n / 2;
+        }
+    }
+    return l;
 }
 
 // ---------------------------------------------------------------------------

@@ -154,28 +154,11 @@ bool make_tmap_3d_blocks(CUtensorMap* map, const void* base, CUtensorMapDataType
     return r == CUDA_SUCCESS;
 }
 
-int tile_override(const char* name) {
-    static std::mutex mu;
-    static std::map<std::string, int> cache;
-    std::lock_guard<std::mutex> lk(mu);
-    auto it = cache.find(name);
-    if (it != cache.end()) return it->second;
-    const char* v = std::getenv(name);
-    const int val = (v && *v) ? std::atoi(v) : -1;
-    cache[name] = val;
-    return val;
-}
-
 namespace {
 std::atomic<int> g_rank_pass_rows{0};
 }
 
 int rank_pass_rows() { return g_rank_pass_rows.load(std::memory_order_relaxed); }
-
-bool pdl_enabled() {
-    static const bool on = tile_override("QLORA_PDL") != 0;
-    return on;
-}
 
 int sm_count() {
     static int cache[64] = {0};
@@ -308,7 +291,9 @@ int qlora_quantize_input(const qlora_layer_desc* d, int M, const void* X, const 
     QL_REQUIRE(aligned(A, 4) && aligned(sx, 4) && aligned(xA, 4), QLORA_EALIGN,
                "fp32 vectors must be 4-byte aligned");
     if (M == 0) return QLORA_OK;
-    return cuda_status(launch_quantize_rows(act_of(d), X, A, M, d->K, d->r, Xq, sx, xA,
+    int* status = status_ptr();
+    QL_REQUIRE(status, QLORA_ECUDA, "no CUDA device");
+    return cuda_status(launch_quantize_rows(act_of(d), X, A, M, d->K, d->r, Xq, sx, xA, status,
                                             static_cast<cudaStream_t>(stream)),
                        "input quantizer launch");
 }

@@ -30,12 +30,12 @@ __device__ __forceinline__ uint32_t pack2(float a, float b, __nv_bfloat16*) {
 // Writes the 16 values of this lane's row into the warp's staging buffer,
 // then the warp stores the 32 x 16 block to global memory with 16-byte
 // stores (rows row0 .. row0+31, columns n .. n+15 of a row-major [M, ldo]
-// matrix).  Rows >= M and columns >= N are skipped; when `vec` is false
+// matrix).  Rows >= M or < row_min and columns >= N are skipped; when `vec` is false
 // (row pitch not a multiple of 16 bytes) the copy-out is element by element.
 template <typename OutT>
 __device__ __forceinline__ void store_block(uint8_t* stg, const float (&v)[kEpiCols], int lane,
                                             OutT* __restrict__ out, size_t ldo, int row0, int M,
-                                            int n, int N, bool vec) {
+                                            int n, int N, bool vec, int row_min = 0) {
     constexpr int P = stage_pitch<OutT>();
     uint8_t* my = stg + lane * P;
     if constexpr (sizeof(OutT) == 2) {
@@ -66,7 +66,7 @@ __device__ __forceinline__ void store_block(uint8_t* stg, const float (&v)[kEpiC
         const int ch = lane % kChunks;
         const int gr = row0 + rr;
         const int gn = n + ch * kElems;
-        if (gr < M && gn < N) {
+        if (gr < M && gr >= row_min && gn < N) {
             const uint4 val = *reinterpret_cast<const uint4*>(stg + rr * P + ch * 16);
             OutT* dst = out + static_cast<size_t>(gr) * ldo + gn;
             if (vec && gn + kElems <= N) {

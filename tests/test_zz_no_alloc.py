@@ -1,7 +1,10 @@
 """qlora_backward_noalloc: the backward with the library's static scratch in
-place of a caller-supplied workspace.  Two calls in a row through the C ABI
-must each agree with qlora_backward (the workspace entry point) on the same
-inputs, within the tolerance the parity tests use for the layer's dtype.
+place of a caller-supplied workspace.  Both entry points run the same
+deterministic kernels in the same order, so two calls in a row through the C
+ABI must each give results bit-identical to qlora_backward (the workspace
+entry point) on the same inputs, even after a call on a larger layer with
+other inputs has left different data in the shared scratch; one case is also
+checked against the CPU oracle within the parity tolerance.
 
 Collected last on purpose: it must also pass after every other test has run
 in the same process, as well as alone in a fresh one."""
@@ -12,6 +15,7 @@ import torch
 
 from lora_fine_tuning_qlora_b200 import inputs
 
+import oracle
 from parity import act_torch, assert_close, device_layer, to_np
 
 
@@ -55,6 +59,19 @@ def test_noalloc_backward_matches_workspace_backward(q, spec):
     _, xA = q.forward(layer, X, ws)
     want_dbias = layer.bias is not None
 
+    # first fill the shared scratch with another layer's data: more rows and
+    # more G slices than the layer under test, other inputs
+    big = inputs.scaled(spec, M=spec.M + 77, N=spec.N + 136 if spec.N % 8 == 0 else spec.N,
+                        seed=spec.seed + 17)
+    db = inputs.layer_inputs(big)
+    lb = device_layer(big, db, q)
+    Xb = torch.from_numpy(db["X"]).to(tdt).to(dev)
+    dYb = torch.from_numpy(db["dY"]).to(tdt).to(dev)
+    wsb = q.workspace(lb.desc(), big.M, dev)
+    _, xAb = q.forward(lb, Xb, wsb)
+    q.qlora_backward_noalloc(lb.desc(), big.M, Xb, dYb, lb.Wq, lb.sw, lb.A, lb.B, xAb,
+                             *_grads(q, lb, big.M, dev, lb.bias is not None))
+
     # two scratch-free calls in a row, each into fresh outputs
     runs = []
     for _ in range(2):
@@ -75,8 +92,17 @@ def test_noalloc_backward_matches_workspace_backward(q, spec):
         for name, g, r in zip(names, out, ref):
             if r is None:
                 continue
-            act = spec.act if name == "dX" else ("f32" if spec.act == "f32" else "bf16")
-            assert_close(to_np(g), to_np(r), act, "call %d %s" % (i + 1, name))
+            assert torch.equal(g, r), "call %d %s differs from qlora_backward" % (i + 1, name)
+
+    # and the second call against the oracle
+    Wq_o, sw_o = oracle.quantize_weight(d["W"])
+    b = oracle.backward(d["X"], d["dY"], Wq_o, sw_o, d["A"], d["B"], spec.alpha, want_dx=True,
+                        act=spec.act)
+    for name, g in zip(names, runs[1]):
+        if g is None:
+            continue
+        act = spec.act if name == "dX" else ("f32" if spec.act == "f32" else "bf16")
+        assert_close(to_np(g), b[name], act, "oracle vs call 2 %s" % name)
 
 
 def test_noalloc_rejects_layers_above_the_static_scratch(q):
