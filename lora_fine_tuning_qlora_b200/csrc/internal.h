@@ -53,6 +53,11 @@ struct DxEpilogue {
 cudaError_t launch_gemm_dx(Act act, const void* dY, const int8_t* Wq, const float* sw, int M,
                            int N, int K, const DxEpilogue& ep, int* status, cudaStream_t s,
                            bool w4 = false);
+// The bf16 dX GEMM on CTA pairs (256 x 256 tiles, k3_dx_pair.cu): for N a
+// multiple of 64, rank <= 16 and at least one wave of pair tiles.
+bool gemm_dx_pair_applies(int M, int N, int K, int r);
+cudaError_t launch_gemm_dx_pair(const void* dY, const int8_t* Wq, const float* sw, int M, int N,
+                                int K, const DxEpilogue& ep, int* status, cudaStream_t s, bool w4);
 
 // ---------------------------------------------------------------- K4
 // The dY pass runs on the tensor cores for bf16 activations whose rows TMA
@@ -150,6 +155,27 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
 
 // Minimum rows per CTA of the column-sum passes (dB/dbias, dA); 0 = default.
 int rank_pass_rows();
+
+// launch_k with thread-block clusters of cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kx(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                      int cluster_x, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster_x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
 
 // Sets the dynamic shared memory limit of `func` once per device.
 cudaError_t ensure_smem_attr(const void* func, int bytes);

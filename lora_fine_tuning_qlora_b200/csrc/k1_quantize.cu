@@ -503,23 +503,17 @@ __device__ __forceinline__ void bf16x8_to_f(const uint4 u, float (&f)[8]) {
     }
 }
 
-// Symmetric abs-max codes of 8 values: rne(fl(v * inv)).  The products are
-// rounded to fp32 first (paired multiplies), then converted with round half
-// to even; |fl(v * inv)| <= 127 * (1 + 2^-24)^2 < 127.5, so no clamp is
-// reached.  (The rounding has to stay a separate step: a fused multiply-add
-// with 1.5 * 2^23 would round the exact product instead and break ties such
-// as v = amax / 2 differently.)  The low byte of each int is the code.
-__device__ __forceinline__ uint2 codes8(const float (&f)[8], unsigned long long inv2) {
+// Symmetric abs-max codes of 8 values: rne(fl(v * inv)).  The product is
+// rounded to fp32 (__fmul_rn, never contracted into a fused multiply-add),
+// then 1.5 * 2^23 is added (__fadd_rn): for |p| < 2^22 the sum rounds p to the
+// nearest integer, ties to even, and its low byte is the two's-complement
+// code.  |fl(v * inv)| <= 127 * (1 + 2^-24)^2 < 127.5, so no clamp is reached.
+// Both steps run on the FMA pipe (a float-to-int conversion would use the
+// narrow conversion pipe for every element).
+__device__ __forceinline__ uint2 codes8(const float (&f)[8], float inv) {
     uint32_t b[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        unsigned long long y;
-        asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(pk2(f[2 * i], f[2 * i + 1])), "l"(inv2));
-        float lo, hi;
-        unpk2(y, lo, hi);
-        b[2 * i] = static_cast<uint32_t>(__float2int_rn(lo));
-        b[2 * i + 1] = static_cast<uint32_t>(__float2int_rn(hi));
-    }
+    for (int i = 0; i < 8; ++i) b[i] = __float_as_uint(__fadd_rn(__fmul_rn(f[i], inv), 12582912.0f));
     const uint32_t w0 = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
     const uint32_t w1 = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
     return make_uint2(w0, w1);
@@ -666,7 +660,6 @@ __global__ void __launch_bounds__(staged::cons<TPR, RP>() + 32, 1)
 #pragma unroll
         for (int q = 0; q < kRPG; ++q) {
             const float inv = amax[q] > 0.f ? __fdiv_rn(127.0f, amax[q]) : 0.f;
-            const unsigned long long inv2 = pk2(inv, inv);
             const int m = m0 + q;
             int8_t* qrow = a.Xq + static_cast<size_t>(m) * K;
 #pragma unroll
@@ -676,7 +669,7 @@ __global__ void __launch_bounds__(staged::cons<TPR, RP>() + 32, 1)
                     const uint4 u = *reinterpret_cast<const uint4*>(gbase + static_cast<size_t>(q) * K * 2 + c * 16);
                     float f[8];
                     bf16x8_to_f(u, f);
-                    const uint2 cw = codes8(f, inv2);
+                    const uint2 cw = codes8(f, inv);
                     if (m < a.M) *reinterpret_cast<uint2*>(qrow + c * 8) = cw;
 #pragma unroll
                     for (int p = 0; p < 4; ++p) {

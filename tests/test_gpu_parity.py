@@ -50,7 +50,10 @@ def test_single_fp32_layer(q):
                                      (100, 4096, 136, 16), (1000, 1296, 264, 8),
                                      # few output tiles: split-K forward (clusters of 2..8 CTAs)
                                      (100, 2048, 520, 4), (16, 4096, 4096, 4), (250, 3072, 264, 8),
-                                     (333, 1024, 1000, 8)])
+                                     (333, 1024, 1000, 8),
+                                     # dX on CTA pairs (256 x 256 tiles): ragged M (the last
+                                     # tile's second CTA wholly outside) and ragged K
+                                     (850, 4736, 640, 4), (1100, 4736, 192, 16)])
 def test_bf16_layer_tiles_and_ragged_tails(q, M, K, N, r):
     spec = inputs.LayerSpec("ragged", M=M, K=K, N=N, r=r, alpha=2.0 * r, act="bf16",
                             x_dist="normal", w_dist="glorot", a_dist="he_uniform", b_std=0.01,
@@ -335,7 +338,8 @@ def test_rank_pass_rows_setting(q, M, K, N, r):
 
 
 @pytest.mark.parametrize("M,K,N,r,act", [(200, 384, 264, 8, "bf16"), (96, 256, 10, 8, "bf16"),
-                                          (64, 784, 128, 4, "f32"), (300, 2048, 264, 8, "bf16")])
+                                          (64, 784, 128, 4, "f32"), (300, 2048, 264, 8, "bf16"),
+                                          (600, 8192, 256, 8, "bf16")])
 def test_fused_relu_entry_points(q, M, K, N, r, act):
     """qlora_gemm_forward_relu == qlora_relu(qlora_gemm_forward) and
     qlora_gemm_dx_relu == qlora_relu_backward(qlora_gemm_dx, X), bit for bit,
@@ -415,7 +419,8 @@ def test_int4_quantize_and_unpack_bit_exact(q, K, N):
                                           (4096, 768, 768, 4, "bf16"),    # 256x128 tiles
                                           (96, 256, 10, 8, "bf16"),       # CUDA-core dX
                                           (64, 256, 128, 4, "f32"),       # fp32 activations
-                                          (200, 800, 264, 16, "bf16")])   # K % 128 == 32: ragged k-block
+                                          (200, 800, 264, 16, "bf16"),    # K % 128 == 32: ragged k-block
+                                          (850, 4736, 640, 4, "bf16")])   # CTA-pair dX
 def test_int4_layer_matches_oracle(q, M, K, N, r, act):
     """An int4 layer: the forward from the packed codes bit-identical to the
     int8 forward on the unpacked codes (accumulator bit-exact against the
