@@ -80,6 +80,8 @@ struct K3Cfg {
     static constexpr int kStagesFit = (kSmemLimit - kFixed) / kStageBytes;
     static constexpr int STAGES = kStagesFit > 8 ? 8 : kStagesFit;
     static_assert(STAGES >= 2, "shared memory budget");
+    // de-quantize stage groups: four where the stages divide into them
+    static constexpr int kDqGroups = STAGES % 4 == 0 ? 4 : (STAGES % 2 == 0 ? 2 : 1);
     static constexpr int kStgOff = STAGES * kStageBytes;
     static constexpr int kTabOff = kStgOff + kStgBytes;
     static constexpr int kBarOff = kTabOff + kParamBytes;
@@ -137,7 +139,7 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&wready[s], kDqWarps);  // every de-quantize warp, once per fill
+            mbar_init(&wready[s], kDqWarps / C::kDqGroups);  // the stage group's warps
             mbar_init(&empty[s], C::kChains);  // every MMA issuer, once per use
         }
         for (int b = 0; b < 2; ++b) {
@@ -260,55 +262,74 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
         __syncwarp();
     } else if (warp < C::kEpiWarp0) {
         // ------------------------------------------------------ de-quantize
-        // All eight warps convert every stage, each its own slice of the
-        // 16-byte chunks, walking the stages in order (so every barrier phase
-        // is awaited in turn).  The int8 codes and row scales come straight
-        // from global memory into registers, S stages ahead of their use (a
-        // ring slot u per ring stage u), so neither a TMA box nor a load
-        // latency sits on the conversion path; a stage only waits for its
-        // bf16 slot to be released by the MMAs that read it last.
+        // The eight warps form kDqGroups groups; group q converts the stages
+        // g = q, q + kDqGroups, ... (all of a stage's codes), so a warp has
+        // kDqGroups stage-times for each of its stages and the pace is set by
+        // the warps' throughput, not by the latency of one stage's
+        // load-convert-store-signal chain.  The codes and row scales of a
+        // group's next S / kDqGroups stages are held in registers (loaded
+        // that many group stages ahead); a chunk outside the matrices is
+        // zeroed through its scale.  The stage and tile cursors advance
+        // without divisions.
+        constexpr int kDqGroups = C::kDqGroups;
+        constexpr int kWPG = kDqWarps / kDqGroups;
         const int dw = warp - C::kDqWarp0;  // 0 .. 7
+        const int grp = dw / kWPG;
+        const int gw = dw % kWPG;
         constexpr int kCodes = W4 ? 32 : 16;  // codes per 16-byte chunk
         constexpr int kChunksPerRow = BN / kCodes;
         const size_t row_bytes = W4 ? static_cast<size_t>(K) / 2 : static_cast<size_t>(K);
         constexpr int kChunks = kBKn * kChunksPerRow;
-        constexpr int kPerLane = kChunks / (32 * kDqWarps);
-        static_assert(kChunks % (32 * kDqWarps) == 0, "chunks per stage");
+        constexpr int kPerLane = kChunks / (32 * kWPG);
+        static_assert(kChunks % (32 * kWPG) == 0, "chunks per stage");
+        constexpr int P = S / kDqGroups;  // register ring of a group
+        static_assert(S % kDqGroups == 0, "stages per group");
         const int my_tiles = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
         const int total_kb = my_tiles * nkb;
-        // The loads are unconditional, from addresses clamped into the
-        // matrices, and a chunk outside them is zeroed through its scale when
-        // it is converted: a select on a just-loaded register would make the
-        // warp wait out the load right here.
-        uint4 qr[S][kPerLane];
-        float sr[S][kPerLane];
-        uint32_t inb[S];  // bit i: chunk i of the ring slot lies inside the matrices
-        auto fetch = [&](int g, uint4 (&q)[kPerLane], float (&sc)[kPerLane], uint32_t& in_bits) {
-            const int t = blockIdx.x + (g / nkb) * gridDim.x;
-            const int k0 = (t % num_k) * BN;
-            const int kb = g % nkb;
+        // fetch cursor: stage g = grp + kDqGroups * j -> (tile ft of this CTA, block fkb)
+        int fj = 0, ft = 0, fkb = grp;
+        while (fkb >= nkb) { fkb -= nkb; ++ft; }
+        int fk0 = ((static_cast<int>(blockIdx.x) + ft * static_cast<int>(gridDim.x)) % num_k) * BN;
+        uint4 qr[P][kPerLane];
+        float sr[P][kPerLane];
+        uint32_t inb[P];  // bit i: chunk i of the ring slot lies inside the matrices
+        auto fetch = [&](uint4 (&q)[kPerLane], float (&sc)[kPerLane], uint32_t& in_bits) {
+            const bool live_g = grp + kDqGroups * fj < total_kb;
             in_bits = 0;
 #pragma unroll
             for (int i = 0; i < kPerLane; ++i) {
-                const int c = dw * 32 + lane + i * 32 * kDqWarps;
-                const int n = kb * kBKn + c / kChunksPerRow;
-                const int k = k0 + (c % kChunksPerRow) * kCodes;
-                if (g < total_kb && n < N && k < K) in_bits |= 1u << i;
+                const int c = gw * 32 + lane + i * 32 * kWPG;
+                const int n = fkb * kBKn + c / kChunksPerRow;
+                const int k = fk0 + (c % kChunksPerRow) * kCodes;
+                if (live_g && n < N && k < K) in_bits |= 1u << i;
                 const int nc = n < N ? n : N - 1;
                 const int kc = k < K ? k : K - kCodes;
                 q[i] = __ldg(reinterpret_cast<const uint4*>(Wq + static_cast<size_t>(nc) * row_bytes +
                                                             (W4 ? kc / 2 : kc)));
                 sc[i] = __ldg(sw + nc);
             }
+            ++fj;
+            fkb += kDqGroups;
+            bool moved = false;
+            while (fkb >= nkb) {
+                fkb -= nkb;
+                ++ft;
+                moved = true;
+            }
+            if (moved) fk0 = ((static_cast<int>(blockIdx.x) + ft * static_cast<int>(gridDim.x)) % num_k) * BN;
         };
 #pragma unroll
-        for (int u = 0; u < S; ++u) fetch(u, qr[u], sr[u], inb[u]);
+        for (int v = 0; v < P; ++v) fetch(qr[v], sr[v], inb[v]);
         bool live = true;
-        for (int g0 = 0; g0 < total_kb && live; g0 += S) {
+        for (int j0 = 0; live; j0 += P) {
 #pragma unroll
-            for (int u = 0; u < S; ++u) {
-                const int g = g0 + u;  // ring stage g % S == u
-                if (g >= total_kb) break;
+            for (int v = 0; v < P; ++v) {
+                const int g = grp + kDqGroups * (j0 + v);
+                if (g >= total_kb) {
+                    live = false;
+                    break;
+                }
+                const int u = grp + kDqGroups * v;  // shared-memory stage: g % S
                 if (g >= S &&
                     !__all_sync(0xffffffffu, mbar_wait(&empty[u], ((g / S) - 1) & 1, status))) {
                     live = false;
@@ -317,15 +338,15 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
                 uint8_t* wt = smem + u * C::kStageBytes + C::kABytes;
 #pragma unroll
                 for (int i = 0; i < kPerLane; ++i) {
-                    const int c = dw * 32 + lane + i * 32 * kDqWarps;
+                    const int c = gw * 32 + lane + i * 32 * kWPG;
                     const int nr = c / kChunksPerRow;   // contraction row within the stage
                     const int kc = c % kChunksPerRow;   // kCodes output columns
-                    const float scale = (inb[u] >> i) & 1u ? sr[u][i] : 0.f;
+                    const float scale = (inb[v] >> i) & 1u ? sr[v][i] : 0.f;
                     const int mn = kc * kCodes;
                     uint32_t o[8];
                     if constexpr (W4) {
                         uint4 lo, hi;
-                        unpack_int4x32(qr[u][i], lo, hi);
+                        unpack_int4x32(qr[v][i], lo, hi);
                         dequant16(lo, scale, o);
                         *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn, nr, kLbo)) =
                             make_uint4(o[0], o[1], o[2], o[3]);
@@ -337,7 +358,7 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
                         *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn + 24, nr, kLbo)) =
                             make_uint4(o[4], o[5], o[6], o[7]);
                     } else {
-                        dequant16(qr[u][i], scale, o);
+                        dequant16(qr[v][i], scale, o);
                         *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn, nr, kLbo)) =
                             make_uint4(o[0], o[1], o[2], o[3]);
                         *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn + 8, nr, kLbo)) =
@@ -347,7 +368,7 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&wready[u]);
-                fetch(g + S, qr[u], sr[u], inb[u]);
+                fetch(qr[v], sr[v], inb[v]);
             }
         }
         __syncwarp();

@@ -37,15 +37,8 @@
 // adds the CL partials in rank order, so dB, dbias and dA leave the kernel
 // final and deterministic, with no cluster-wide barrier at the end.
 //
-// Warps: 0 TMA producer; 1 and 2 MMA issuers (warp 1 owns TMEM): a
-// tcgen05.mma holds its issuing thread about as long as a 128 x 32 MMA takes
-// to run, so the G chain and the column sums of a tile go to different
-// issuers.  For ranks up to 16 the column sums always accumulate the even and
-// the odd 16-row steps into two accumulators (added in that order at the
-// end), so that a pass with column sums alone can give each to its own issuer
-// and still match the combined pass bit for bit (larger ranks keep one
-// accumulator and one issuer, within the 512 TMEM columns); 3..6 operand
-// tables and epilogues (warp w owns TMEM lane quarter w % 4).
+// Warps: 0 TMA producer, 1 TMEM owner + MMA issuer, 2..5 operand tables and
+// epilogues (warp w owns TMEM lane quarter w % 4).
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -59,8 +52,7 @@ constexpr int kBoxCols = 64;                         // one 128-byte swizzle row
 constexpr uint32_t kBoxBytes = kTileRows * kBoxCols * 2;
 constexpr uint32_t kTileBytes = 2 * kBoxBytes;
 constexpr int kWorkers = 4;
-constexpr int kIssuers = 2;
-constexpr int kThreads = 32 * (1 + kIssuers) + 32 * kWorkers;
+constexpr int kThreads = 64 + 32 * kWorkers;
 constexpr int kMaxCluster = 8;
 constexpr uint32_t kTabSbo = (kTileCols / 8) * 128;  // 8-row group stride of a 128-wide table
 
@@ -88,7 +80,6 @@ struct RtLayout {
     int RP, NG, NV, JP;
     uint32_t vtab, bcat, recv, bar, total;
     uint32_t tmem_cols, d_col, g_col;
-    int nd;  // column-sum accumulators: the even and the odd 16-row steps (ranks <= 16)
     __host__ __device__ RtLayout(Parts p, int r) {
         RP = (r + 15) / 16 * 16;
         NG = p.g ? 2 * RP : 0;
@@ -99,10 +90,9 @@ struct RtLayout {
         recv = bcat + static_cast<uint32_t>(NG) * 256;
         bar = recv + (((kTileCols + kMaxCluster) * JP * 4 + 15) / 16) * 16;
         total = bar + 128;
-        nd = (p.d && RP <= 16) ? 2 : 1;
         d_col = 0;
-        g_col = static_cast<uint32_t>(nd * NV);
-        const uint32_t need = static_cast<uint32_t>(nd * NV + 2 * NG);
+        g_col = static_cast<uint32_t>(NV);
+        const uint32_t need = static_cast<uint32_t>(NV + 2 * NG);
         tmem_cols = 32;
         while (tmem_cols < need) tmem_cols <<= 1;
     }
@@ -165,12 +155,11 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
         for (int s = 0; s < 2; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&vready[s], kWorkers);
-            // every issuer that reads the tile
-            mbar_init(&empty[s], (kG && kD) || (kD && L.nd == 2) ? 2u : 1u);
+            mbar_init(&empty[s], 1);
             mbar_init(&gfull[s], 1);
             mbar_init(&gempty[s], kWorkers);
         }
-        mbar_init(dfull, (kD && !kG && L.nd == 2) ? 2u : 1u);
+        mbar_init(dfull, 1);
         mbar_init(rbar, static_cast<uint32_t>(CL * (cend > cbeg ? cend - cbeg : 1)));
         fence_mbar_init();
     }
@@ -206,28 +195,19 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
         }
         __syncwarp();
         if constexpr (kD) cluster_wait();
-    } else if (warp <= kIssuers) {
-        // ------------------------------------------------------ MMA issuers
-        // G and column sums: issuer 0 runs the G chain, issuer 1 both column-sum
-        // accumulators.  Column sums alone: issuer q runs the 16-row steps of
-        // parity q into accumulator q.  G alone: issuer 0.
-        const int iss = warp - 1;
-        const bool do_g = kG && iss == 0;
-        const bool do_d = kD && (kG ? iss == 1 : (L.nd == 2 || iss == 0));
-        if (lane == 0 && (do_g || do_d)) {
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (lane == 0) {
             const uint32_t tiles = smem_u32(smem);
             const uint32_t vt = smem_u32(smem + L.vtab);
             const uint32_t bt = smem_u32(smem + L.bcat);
             const uint32_t id_g = idesc_bf16(128, kG ? L.NG : 16, false, false);
             const uint32_t id_d = idesc_bf16(128, kD ? L.NV : 16, true, false);
-            const int kk0 = (kG || L.nd == 1) ? 0 : iss;
-            const int kks = (kG || L.nd == 1) ? 1 : 2;
             bool ok = true;
             for (int i = 0; i < nt; ++i) {
                 const int s = i & 1;
-                // the D chain needs this tile's Vcat; the G chain the Bcat table
-                // (written before the first tile's Vcat, or signalled alone)
-                const bool need_v = do_d || i == 0;
+                // Vcat of this tile (column sums), or the Bcat table once (G alone)
+                const bool need_v = kD || i == 0;
                 if (!mbar_wait(&full[s], (i >> 1) & 1, status) ||
                     (need_v && !mbar_wait(&vready[s], (i >> 1) & 1, status))) {
                     ok = false;
@@ -235,7 +215,7 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
                 }
                 tc_fence_after();
                 const uint32_t tb = tiles + s * kTileBytes;
-                if (do_g) {
+                if constexpr (kG) {
                     // G rows of this tile: T (K-major) x Bcat
                     if (i >= 2 && !mbar_wait(&gempty[s], ((i >> 1) - 1) & 1, status)) {
                         ok = false;
@@ -251,21 +231,19 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
                     }
                     mma_commit(&gfull[s]);
                 }
-                if (do_d) {
+                if constexpr (kD) {
                     // column sums: T^T (MN-major, the two blocks 64 columns apart) x Vcat
 #pragma unroll
-                    for (int kk = kk0; kk < kTileRows / 16; kk += kks) {
+                    for (int kk = 0; kk < kTileRows / 16; ++kk) {
                         const uint64_t ad = smem_desc(tb + kk * 2048, kBoxBytes, 1024, kLayoutSw128);
                         const uint64_t bd =
                             smem_desc(vt + s * L.NV * 256 + kk * 256, 128, kTabSbo, kLayoutNone);
-                        const int acc = L.nd == 2 ? (kk & 1) : 0;
-                        const uint32_t dacc = tmem + L.d_col + static_cast<uint32_t>(acc * L.NV);
-                        mma_bf16(dacc, ad, bd, id_d, (i > 0 || kk >= L.nd) ? 1u : 0u);
+                        mma_bf16(tmem + L.d_col, ad, bd, id_d, (i > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
-                if (kD || do_g) mma_commit(&empty[s]);
+                mma_commit(&empty[s]);
             }
-            if (do_d && ok) mma_commit(dfull);
+            if (kD && ok) mma_commit(dfull);
         }
         __syncwarp();
         if constexpr (kD) cluster_wait();
@@ -331,79 +309,58 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
         if constexpr (kD) {
             // rows of V in whole 8-float groups at 16-byte alignment
             const bool vec4 = (a.r % 8) == 0 && (reinterpret_cast<uintptr_t>(a.V) & 15) == 0;
-            // V of one 8-column group of row m: the nsl slices added in ascending order
-            auto vals = [&](int j0, int m, bool mok, float (&v)[8]) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = 0.f;
-                bool vdone = false;
-                if constexpr (!kG) {
-                  if (mok && j0 < a.r && vec4) {
-                    vdone = true;
-                    // V = the nsl slices added in ascending order: eight
-                    // slices' rows in flight as 16-byte loads, then the adds
-                    const float4* p4 = reinterpret_cast<const float4*>(a.V + static_cast<size_t>(m) * a.r + j0);
-                    const size_t st4 = static_cast<size_t>(a.M) * a.r / 4;
-                    for (int b0 = 0; b0 < a.nsl; b0 += 8) {
-                        float4 lo[8], hi[8];
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const size_t b = static_cast<size_t>(b0 + u < a.nsl ? b0 + u : b0);
-                            lo[u] = __ldg(p4 + b * st4);
-                            hi[u] = __ldg(p4 + b * st4 + 1);
-                        }
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            if (b0 + u < a.nsl) {
-                                v[0] += lo[u].x; v[1] += lo[u].y; v[2] += lo[u].z; v[3] += lo[u].w;
-                                v[4] += hi[u].x; v[5] += hi[u].y; v[6] += hi[u].z; v[7] += hi[u].w;
-                            }
-                        }
-                    }
-                  }
-                }
-                if (!vdone && mok && j0 < a.r) {
-                    const int nv = min(8, a.r - j0);
-                    const float* p = a.V + static_cast<size_t>(m) * a.r + j0;
-                    // V = the nsl slices added in ascending order, every load issued at once
-                    const size_t stride = static_cast<size_t>(a.M) * a.r;
-#pragma unroll
-                    for (int b = 0; b < kMaxDirectSlices; ++b)
-                        if (b < a.nsl)
-#pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                if (e < nv) v[e] += __ldg(p + b * stride + e);
-                    for (int b = kMaxDirectSlices; b < a.nsl; ++b)
-                        for (int e = 0; e < nv; ++e) v[e] += __ldg(p + b * stride + e);
-                }
-            };
             for (int i = 0; i < nt && ok; ++i) {
                 const int s = i & 1;
                 const int m = (t0 + i) * kTileRows + rr;
-                const bool mok = m < a.M;
+                ok = __all_sync(0xffffffffu,
+                                i < 2 || mbar_wait(&empty[s], ((i >> 1) - 1) & 1, status));
+                if (!ok) break;
                 uint8_t* vt = smem + L.vtab + s * L.NV * 256;
-                if (L.RP == 16) {
-                    // ranks <= 16: this row's V is read before the wait for the
-                    // table slot, so the loads overlap the MMAs of the tile before
-                    float v0[8], v1[8];
-                    vals(0, m, mok, v0);
-                    vals(8, m, mok, v1);
-                    ok = __all_sync(0xffffffffu,
-                                    i < 2 || mbar_wait(&empty[s], ((i >> 1) - 1) & 1, status));
-                    if (!ok) break;
+                const bool mok = m < a.M;
+                for (int j0 = 0; j0 < L.RP; j0 += 8) {
+                    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    bool vdone = false;
+                    if constexpr (!kG) {
+                      if (mok && j0 < a.r && vec4) {
+                        vdone = true;
+                        // V = the nsl slices added in ascending order: eight
+                        // slices' rows in flight as 16-byte loads, then the adds
+                        const float4* p4 = reinterpret_cast<const float4*>(a.V + static_cast<size_t>(m) * a.r + j0);
+                        const size_t st4 = static_cast<size_t>(a.M) * a.r / 4;
+                        for (int b0 = 0; b0 < a.nsl; b0 += 8) {
+                            float4 lo[8], hi[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) put_split(vt, e, L.RP + e, rr, v0[e]);
+                            for (int u = 0; u < 8; ++u) {
+                                const size_t b = static_cast<size_t>(b0 + u < a.nsl ? b0 + u : b0);
+                                lo[u] = __ldg(p4 + b * st4);
+                                hi[u] = __ldg(p4 + b * st4 + 1);
+                            }
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) put_split(vt, 8 + e, L.RP + 8 + e, rr, v1[e]);
-                } else {
-                    ok = __all_sync(0xffffffffu,
-                                    i < 2 || mbar_wait(&empty[s], ((i >> 1) - 1) & 1, status));
-                    if (!ok) break;
-                    for (int j0 = 0; j0 < L.RP; j0 += 8) {
-                        float v[8];
-                        vals(j0, m, mok, v);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) put_split(vt, j0 + e, L.RP + j0 + e, rr, v[e]);
+                            for (int u = 0; u < 8; ++u) {
+                                if (b0 + u < a.nsl) {
+                                    v[0] += lo[u].x; v[1] += lo[u].y; v[2] += lo[u].z; v[3] += lo[u].w;
+                                    v[4] += hi[u].x; v[5] += hi[u].y; v[6] += hi[u].z; v[7] += hi[u].w;
+                                }
+                            }
+                        }
+                      }
                     }
+                    if (!vdone && mok && j0 < a.r) {
+                        const int nv = min(8, a.r - j0);
+                        const float* p = a.V + static_cast<size_t>(m) * a.r + j0;
+                        // V = the nsl slices added in ascending order, every load issued at once
+                        const size_t stride = static_cast<size_t>(a.M) * a.r;
+#pragma unroll
+                        for (int b = 0; b < kMaxDirectSlices; ++b)
+                            if (b < a.nsl)
+#pragma unroll
+                                for (int e = 0; e < 8; ++e)
+                                    if (e < nv) v[e] += __ldg(p + b * stride + e);
+                        for (int b = kMaxDirectSlices; b < a.nsl; ++b)
+                            for (int e = 0; e < nv; ++e) v[e] += __ldg(p + b * stride + e);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) put_split(vt, j0 + e, L.RP + j0 + e, rr, v[e]);
                 }
                 if constexpr (kOnes) {
                     const __nv_bfloat16 one = __float2bfloat16_rn(mok ? 1.f : 0.f);
@@ -436,32 +393,16 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
                     tmem_ld16(base + c0, hi);
                     tmem_ld16(base + L.RP + c0, lo);
                     tmem_ld_wait();
-                    float sum[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) sum[e] = __uint_as_float(hi[e]) + __uint_as_float(lo[e]);
-                    if (L.nd == 2) {
-                        // the second issuer's accumulator, added after the first
-                        tmem_ld16(base + L.NV + c0, hi);
-                        tmem_ld16(base + L.NV + L.RP + c0, lo);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) sum[e] += __uint_as_float(hi[e]) + __uint_as_float(lo[e]);
-                    }
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
-                        if (c0 + e < a.r) dsmem_st(dst + 4 * (c0 + e), sum[e]);
+                        if (c0 + e < a.r)
+                            dsmem_st(dst + 4 * (c0 + e), __uint_as_float(hi[e]) + __uint_as_float(lo[e]));
                 }
                 if constexpr (kOnes) {
                     uint32_t ones[16];
                     tmem_ld16(base + 2 * L.RP, ones);
                     tmem_ld_wait();
-                    float db = __uint_as_float(ones[0]);
-                    if (L.nd == 2) {
-                        tmem_ld16(base + L.NV + 2 * L.RP, ones);
-                        tmem_ld_wait();
-                        db += __uint_as_float(ones[0]);
-                    }
-                    dsmem_st(dst + 4 * a.r, db);
+                    dsmem_st(dst + 4 * a.r, __uint_as_float(ones[0]));
                 }
             } else {
                 for (int j = 0; j < L.JP; ++j) dsmem_st(dst + 4 * j, 0.f);
