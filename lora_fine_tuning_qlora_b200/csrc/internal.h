@@ -37,6 +37,12 @@ struct FwdEpilogue {
 cudaError_t launch_gemm_i8_fwd(Act act, const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
                                const FwdEpilogue& ep, int* status, cudaStream_t s, bool w4 = false);
 
+// The forward GEMM on CTA pairs (256 x 256 tiles, k2_gemm_i8_pair.cu): bf16
+// outputs, rank <= 16, at least one wave of pair tiles.
+bool gemm_fwd_pair_applies(Act act, int M, int N, int K, int r);
+cudaError_t launch_gemm_i8_fwd_pair(const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
+                                    const FwdEpilogue& ep, int* status, cudaStream_t s);
+
 // ---------------------------------------------------------------- K3
 struct DxEpilogue {
     const float* Gp;  // [ncb][M,r] slices of G = dY B^T (G = sum of the slices)

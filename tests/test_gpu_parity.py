@@ -53,7 +53,9 @@ def test_single_fp32_layer(q):
                                      (333, 1024, 1000, 8),
                                      # dX on CTA pairs (256 x 256 tiles): ragged M (the last
                                      # tile's second CTA wholly outside) and ragged K
-                                     (850, 4736, 640, 4), (1100, 4736, 192, 16)])
+                                     (850, 4736, 640, 4), (1100, 4736, 192, 16),
+                                     # forward on CTA pairs: ragged M, N
+                                     (1000, 1040, 4744, 8)])
 def test_bf16_layer_tiles_and_ragged_tails(q, M, K, N, r):
     spec = inputs.LayerSpec("ragged", M=M, K=K, N=N, r=r, alpha=2.0 * r, act="bf16",
                             x_dist="normal", w_dist="glorot", a_dist="he_uniform", b_std=0.01,
@@ -339,7 +341,7 @@ def test_rank_pass_rows_setting(q, M, K, N, r):
 
 @pytest.mark.parametrize("M,K,N,r,act", [(200, 384, 264, 8, "bf16"), (96, 256, 10, 8, "bf16"),
                                           (64, 784, 128, 4, "f32"), (300, 2048, 264, 8, "bf16"),
-                                          (600, 8192, 256, 8, "bf16")])
+                                          (600, 8192, 256, 8, "bf16"), (2048, 512, 9216, 4, "bf16")])
 def test_fused_relu_entry_points(q, M, K, N, r, act):
     """qlora_gemm_forward_relu == qlora_relu(qlora_gemm_forward) and
     qlora_gemm_dx_relu == qlora_relu_backward(qlora_gemm_dx, X), bit for bit,
