@@ -168,7 +168,10 @@ int qlora_backward(const qlora_layer_desc* d, int M, const void* X, const void* 
  * Set-up: the first call on each device (with that device current) looks up
  * the device addresses of the scratch and of the status word with
  * cudaGetSymbolAddress and caches them; a failed lookup returns QLORA_ECUDA.
- * Make the first call on a device before any stream capture begins.
+ * Make the first call on a device before any stream capture begins.  The
+ * cached addresses belong to the device's current context: after
+ * cudaDeviceReset (or anything else that destroys that context) they are
+ * stale, and this entry point must not be called again in the process.
  *
  * Concurrency: all calls on one device share the one scratch.  Calls issued
  * to the same stream are ordered and safe; calls that can overlap on the
@@ -265,7 +268,9 @@ int qlora_lora_grad_x(const qlora_layer_desc* d, int M, const void* X, float* dA
  * default.  Results change only by the fp32 rounding of the different
  * grouping and stay deterministic for a given setting.  Process-wide, for
  * launches made after the call (a captured graph keeps the launch shape it
- * was captured with); returns the previous setting, or QLORA_EINVAL for rows
+ * was captured with): one value shared by every caller in the process, so a
+ * caller that changes it should restore it around its own launches (the MLP
+ * stack does); returns the previous setting, or QLORA_EINVAL for rows
  * outside [0, 2^24].  The pages have no counterpart. */
 int qlora_set_rank_pass_rows(int rows);
 
