@@ -25,7 +25,9 @@ What each routine follows (page title, section):
   * quantize_outlier_int8 / dequantize_outlier_int8 / percentile / round_fp16
     -- outlier-compensated int8 kernels: keras-llm-light, "Weights
     quantization" and "Simplified Int8Variable quantization"; the readings
-    are in the C file.
+    are in the C file.  forward_outlier / backward_outlier compose them into
+    the layer (the rebuilt kernel in the activation dtype, unquantized
+    activations; numpy fp64 matmuls as the products).
   * quantize_weight_int4 / unpack_int4 / merge_int4 -- packed 4-bit kernels:
     keras-llm-light, "Simplified Int4Variable quantization" (two int4 values
     per int8 byte) and the 4-bit thread; the readings are in the C file.
@@ -313,6 +315,44 @@ def dequantize_outlier_int8(q):
     _lib().orc_dequantize_outlier_int8(_p(codes), _p(is_out), _p(vals), codes.size,
                                        float(q["scale"]), float(q["bias"]), _p(W))
     return W
+
+
+def outlier_kernel(q, act_dtype):
+    """The kernel an outlier-compensated layer multiplies with: the rebuilt
+    fp32 kernel of quantize_outlier_int8 (same shape as W, [K, N]), stored in
+    the activation dtype (rounded to bf16 for bf16 layers), as fp64."""
+    return to_act(dequantize_outlier_int8(q).astype(np.float64), act_dtype)
+
+
+def forward_outlier(X, q, bias, A, B, alpha, act_dtype):
+    """One outlier-compensated int8-LoRA Dense forward (keras-llm-light,
+    "Simplified Int8Variable quantization": the kernel is rebuilt from its
+    codes and outliers, and the activations are not quantized; "Parameter-
+    efficient fine-tuning of GPT-2 with LoRA", "LoRA equation"):
+    y = X . Wr + bias + c (X . A) . B in fp64, Wr = outlier_kernel(q, act).
+    Returns dict xA, y."""
+    Xd = np.asarray(X, np.float64)
+    Wr = outlier_kernel(q, act_dtype)
+    c = float(alpha) / float(A.shape[1])
+    xA = lora_down(Xd, A)
+    y = Xd @ Wr + c * (xA @ np.asarray(B, np.float64))
+    if bias is not None:
+        y = y + np.asarray(bias, np.float64)[None, :]
+    return {"xA": xA, "y": y}
+
+
+def backward_outlier(X, dY, q, A, B, alpha, act_dtype):
+    """Its backward in fp64: G = dY B^T, dX = dY Wr^T + c G A^T,
+    dA = c X^T G, dB = c (X A)^T dY, dbias = sum_m dY."""
+    Xd = np.asarray(X, np.float64)
+    dYd = np.asarray(dY, np.float64)
+    Ad = np.asarray(A, np.float64)
+    Bd = np.asarray(B, np.float64)
+    c = float(alpha) / float(Ad.shape[1])
+    Wr = outlier_kernel(q, act_dtype)
+    G = dYd @ Bd.T
+    return {"G": G, "dX": dYd @ Wr.T + c * (G @ Ad.T), "dA": c * (Xd.T @ G),
+            "dB": c * (lora_down(Xd, A).T @ dYd), "dbias": dYd.sum(axis=0)}
 
 
 def round_bf16(x):

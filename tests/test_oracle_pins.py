@@ -717,3 +717,73 @@ def test_constant_kernel_has_no_outliers_and_rebuilds_exactly():
     q = oracle.quantize_outlier_int8(W)
     assert q["count"] == 0 and q["scale"] == 0.0 and not q["codes"].any()
     np.testing.assert_array_equal(oracle.dequantize_outlier_int8(q), W)
+
+
+# ---------------------------------------------------------------- outlier layer
+def _outlier_layer(seed, K=24, N=20, M=7, r=3):
+    rng = _rng(seed)
+    W = (rng.normal(0, 0.02, size=(K, N))).astype(np.float32)
+    W.reshape(-1)[rng.choice(K * N, size=3, replace=False)] *= 20.0
+    X = rng.normal(size=(M, K))
+    A = rng.uniform(-0.2, 0.2, size=(K, r)).astype(np.float32)
+    B = rng.normal(0, 0.1, size=(r, N)).astype(np.float32)
+    bias = rng.normal(0, 0.01, size=(N,)).astype(np.float32)
+    dY = rng.normal(size=(M, N))
+    return W, X, A, B, bias, dY
+
+
+def test_outlier_layer_with_zero_adapter_is_the_rebuilt_kernel_product():
+    """B = 0: the forward is X . Wr + bias, with Wr the rebuilt kernel (codes
+    and fp16 outliers) checked entry by entry against the quantizer's own
+    pieces: an outlier entry is its fp16 value, every other entry is
+    bias + code * scale in fp32."""
+    W, X, A, B, bias, _ = _outlier_layer(31)
+    q = oracle.quantize_outlier_int8(W)
+    f = oracle.forward_outlier(X, q, bias, A, np.zeros_like(B), 2.0, "f32")
+    Wr = np.where(q["is_outlier"], q["values"],
+                  np.float32(q["bias"]) + q["codes"].astype(np.float32) * np.float32(q["scale"]))
+    np.testing.assert_allclose(f["y"], X @ Wr.astype(np.float64) + bias.astype(np.float64),
+                               rtol=1e-12, atol=1e-12)
+    # 480 entries: both cutoffs fall between the two most extreme order
+    # statistics, so exactly one outlier on each side
+    assert q["count"] == int(q["is_outlier"].sum()) == 2
+
+
+def test_outlier_layer_gradients_are_central_differences():
+    """The outlier layer is linear in X, A and B (nothing is quantized at run
+    time), so dX, dA and dB equal central differences of the forward of the
+    loss sum(dY * y) to rounding."""
+    W, X, A, B, bias, dY = _outlier_layer(32, K=6, N=5, M=3, r=2)
+    q = oracle.quantize_outlier_int8(W)
+    alpha = 3.0
+    g = oracle.backward_outlier(X, dY, q, A, B, alpha, "f32")
+    A64, B64 = A.astype(np.float64), B.astype(np.float64)
+
+    def loss(Xv, Av, Bv):
+        Wr = oracle.outlier_kernel(q, "f32")
+        y = Xv @ Wr + bias.astype(np.float64) + (alpha / A.shape[1]) * (Xv @ Av) @ Bv
+        return float((dY * y).sum())
+
+    h = 1e-6
+    for name, base in (("dX", X.copy()), ("dA", A64.copy()), ("dB", B64.copy())):
+        num = np.zeros_like(base)
+        for idx in np.ndindex(base.shape):
+            p, m = base.copy(), base.copy()
+            p[idx] += h
+            m[idx] -= h
+            args_p = {"dX": (p, A64, B64), "dA": (X, p, B64), "dB": (X, A64, p)}[name]
+            args_m = {"dX": (m, A64, B64), "dA": (X, m, B64), "dB": (X, A64, m)}[name]
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        np.testing.assert_allclose(g[name], num, rtol=1e-6, atol=1e-8, err_msg=name)
+    np.testing.assert_allclose(g["dbias"], dY.sum(axis=0), rtol=1e-12)
+
+
+def test_outlier_kernel_in_bf16_is_the_rounded_rebuilt_kernel():
+    """For bf16 layers the rebuilt kernel enters the products rounded to bf16
+    (torch's conversion), like every operand of a bf16 layer."""
+    import torch
+    W, *_ = _outlier_layer(33)
+    q = oracle.quantize_outlier_int8(W)
+    Wr = oracle.dequantize_outlier_int8(q)
+    ref = torch.from_numpy(Wr).to(torch.bfloat16).float().numpy().astype(np.float64)
+    np.testing.assert_array_equal(oracle.outlier_kernel(q, "bf16"), ref)
