@@ -323,6 +323,81 @@ int qlora_merge_int4(const qlora_layer_desc* d, const uint8_t* Wp, const float* 
                      const float* A, const float* B, uint8_t* Wp_out, float* sw_out,
                      void* stream);
 
+/* ------------------------------------------------------------------------
+ * Outlier-compensated int8 kernels (keras-llm-light, "Weights
+ * quantization": the weights are quantized after the outliers beyond a
+ * 99.9 percentile cutoff are taken out and kept in fp16; "Simplified
+ * Int8Variable quantization": the kernel is rebuilt as bias + code * scale
+ * with the outliers written back, and the activations are not quantized).
+ *
+ * Reading (the pages give no formula): one affine code per tensor.  lo and
+ * hi are the 0.1th and 99.9th percentiles of all K*N entries of W (linear
+ * interpolation between the order statistics at (K*N - 1) p / 100, in fp64,
+ * stored as fp32).  Entries strictly below lo or above hi are outliers,
+ * kept as fp16 (round to nearest even) with code 0; scale = fl32((hi - lo) /
+ * 255), bias = lo, and every other entry gets
+ *   code = clamp(rne(fl32(fl32(w - bias) / scale)), 0, 255)   (0 if scale == 0).
+ * The rebuilt kernel is Wr = fl32(bias + fl32(code * scale)), the fp16 value
+ * at the outliers; a bf16 layer rounds Wr to bf16 before the tensor cores.
+ *
+ * Storage (struct qlora_outlier_kernel, all device memory owned by the caller):
+ *   codes_nk [N,K] uint8 (16-byte aligned; the dX GEMM's layout)
+ *   codes_kn [K,N] uint8 (16-byte aligned; the forward GEMM's layout)
+ *   par [4] fp32: lo, hi, scale, bias
+ *   start_nk [N * ceil(K/128) + 1] int32, ent_nk [cap] uint32: the outliers of
+ *     row n, columns 128b .. 128b+127 of codes_nk are ent_nk[start_nk[n *
+ *     ceil(K/128) + b] .. start_nk[n * ceil(K/128) + b + 1]), each entry
+ *     (column - 128b) << 16 | fp16 bits; the order inside a bucket is not
+ *     specified
+ *   start_kn [K * ceil(N/128) + 1], ent_kn [cap]: the same for codes_kn
+ *   cap: entries of ent_nk and of ent_kn, at least qlora_outlier_cap(K, N)
+ * The layer: Y = X Wr + bias + c (X A) B; its backward as qlora_backward with
+ * Wr in place of Wq * sw.  Layer constraints as for int8 layers (K a multiple
+ * of 16); bf16 layers run on the tensor cores when N is a multiple of 16.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    uint8_t* codes_nk;
+    uint8_t* codes_kn;
+    float* par;
+    int* start_nk;
+    uint32_t* ent_nk;
+    int* start_kn;
+    uint32_t* ent_kn;
+    int cap;
+} qlora_outlier_kernel;
+
+/* Upper bound on the number of outliers of a K x N kernel (the entries
+ * strictly outside the two percentiles): (i_lo + 1) + (K*N - 1 - i_hi) with
+ * i = floor((K*N - 1) p / 100).  0 for an invalid shape. */
+size_t qlora_outlier_cap(int K, int N);
+
+/* Bytes of scratch that qlora_outlier_quantize needs (256-byte aligned). */
+size_t qlora_outlier_workspace_bytes(int K, int N);
+
+/* a0 for outlier-compensated kernels: W [K,N] fp32 -> every member of *q.
+ * Codes, par and the set of outliers in each bucket are bit-exact with the
+ * reading above.  K >= 1, N >= 1, K*N < 2^31; q is a host pointer. */
+int qlora_outlier_quantize(const float* W, int K, int N, const qlora_outlier_kernel* q,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* Forward of an outlier-compensated layer: xA = X A [M,r], then
+ * Y = X Wr + bias + c xA B, the kernel rebuilt tile by tile in shared memory
+ * (codes_kn, ent_kn) in front of the tensor cores.  bias may be NULL.
+ * workspace: at least qlora_workspace_bytes(d, M). */
+int qlora_outlier_forward(const qlora_layer_desc* d, int M, const void* X,
+                          const qlora_outlier_kernel* q, const float* bias, const float* A,
+                          const float* B, void* Y, float* xA, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/* Backward of an outlier-compensated layer: G = dY B^T, dX = dY Wr^T +
+ * c G A^T (codes_nk, ent_nk; dX may be NULL), dA = c X^T G, dB = c xA^T dY,
+ * dbias = column sums of dY (may be NULL).  The parameter gradients are the
+ * passes of qlora_backward.  Deterministic. */
+int qlora_outlier_backward(const qlora_layer_desc* d, int M, const void* X, const void* dY,
+                           const qlora_outlier_kernel* q, const float* A, const float* B,
+                           const float* xA, void* dX, float* dA, float* dB, float* dbias,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
 /*
  * Lossy merge ("Introduce QLoRA-like technique", Results footnote: merging
  * LoRA weights into int8 kernels is lossy; "How to fine-tune the 4-bit

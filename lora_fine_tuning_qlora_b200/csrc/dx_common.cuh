@@ -7,6 +7,8 @@
 #include "internal.h"
 #include "ptx.cuh"
 
+#include <cuda_fp16.h>
+
 namespace qlora {
 
 // byte offset of the 16-byte chunk holding bf16 elements (mn .. mn+7, kr) in
@@ -64,6 +66,51 @@ __device__ __forceinline__ void dequant16(const uint4 raw, float scale, uint32_t
         asm("mov.b64 {%0, %1}, %2;" : "=f"(c), "=f"(d) : "l"(hi));
         o[2 * i] = pack_bf16x2(a, b);
         o[2 * i + 1] = pack_bf16x2(c, d);
+    }
+}
+
+// Element (k, j) of the rank-r epilogue's factor (A for dX; B^T for a forward
+// run on the dX kernels).
+__device__ __forceinline__ float a_at(const DxEpilogue& ep, int k, int j) {
+    return __ldg(ep.A + static_cast<size_t>(k) * (ep.a_ks ? ep.a_ks : ep.r) +
+                 static_cast<size_t>(j) * ep.a_js);
+}
+
+// 16 uint8 affine codes -> 8 words of packed bf16 pairs holding
+// bf16(fl32(bias + fl32(code * scale))) (the rebuilt outlier-compensated
+// kernel; the two roundings stay separate, as the reading fixes).
+__device__ __forceinline__ void dequant16_affine(const uint4 raw, float scale, float bias,
+                                                 uint32_t (&o)[8]) {
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float v[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const float code = __fsub_rn(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7540 + b)),
+                                         8388608.0f);
+            v[b] = __fadd_rn(bias, __fmul_rn(code, scale));
+        }
+        o[2 * i] = pack_bf16x2(v[0], v[1]);
+        o[2 * i + 1] = pack_bf16x2(v[2], v[3]);
+    }
+}
+
+// Writes the outliers of contraction row `row` (global), columns
+// [c0, c0 + width) of the layout (c0 % 128 + width <= 128), into a stage's
+// MN-major 128B-swizzled bf16 tile at contraction row `nr` (column c0 -> 0).
+__device__ __forceinline__ void patch_outliers(const OutlierArgs& ol, int row, int c0, int width,
+                                               uint8_t* tile, int nr, uint32_t lbo) {
+    const int blk = c0 >> 7, off = c0 & 127;
+    const size_t b = static_cast<size_t>(row) * ol.nb + blk;
+    const int e0 = __ldg(ol.start + b), e1 = __ldg(ol.start + b + 1);
+    for (int e = e0; e < e1; ++e) {
+        const uint32_t v = __ldg(ol.ent + e);
+        const int col = static_cast<int>(v >> 16) - off;
+        if (col < 0 || col >= width) continue;
+        const float f = __half2float(__ushort_as_half(static_cast<unsigned short>(v & 0xFFFFu)));
+        *reinterpret_cast<__nv_bfloat16*>(tile + mn_sw128_offset(col & ~7, nr, lbo) + (col & 7) * 2) =
+            __float2bfloat16_rn(f);
     }
 }
 

@@ -44,16 +44,50 @@ cudaError_t launch_gemm_i8_fwd_pair(const int8_t* Xq, const int8_t* Wq, int M, i
                                     const FwdEpilogue& ep, int* status, cudaStream_t s);
 
 // ---------------------------------------------------------------- K3
+// Outlier-compensated int8 kernel as a GEMM operand (outlier.cu): uint8
+// affine codes [rows, cols] with rows the contraction, one scale and bias per
+// tensor (par[2], par[3]), and the fp16 outliers of every (row, 128-column
+// block) in ent[start[row * nb + block] .. start[row * nb + block + 1]), each
+// (column within the block << 16) | fp16 bits.
+struct OutlierArgs {
+    const float* par;
+    const int* start;
+    const uint32_t* ent;
+    int nb;  // 128-column blocks per row
+};
+
 struct DxEpilogue {
     const float* Gp;  // [ncb][M,r] slices of G = dY B^T (G = sum of the slices)
     int ncb;
-    const float* A;   // [K,r]
+    const float* A;   // element (k, j) at A[k * a_ks + j * a_js]; [K,r] when a_ks = 0
     int r;
     float c;
     void* dX;         // [M,K] act
     const void* gate; // [M,K] act or null: dX = 0 where gate <= 0 (the layer input came
                       // out of a ReLU, whose backward this applies)
+    int a_ks = 0;     // 0: r
+    int a_js = 1;
+    const float* bias = nullptr;      // [K] added per output column, or null
+    OutlierArgs ol{};  // ol.par != nullptr: outlier-compensated codes instead of int8 / int4
 };
+
+// The one-off quantization of an outlier-compensated int8 kernel W [K,N]
+// (outlier.cu): codes in both layouts, affine parameters, bucketed outliers.
+struct OutlierKernel {
+    uint8_t* codes_nk;  // [N,K]
+    uint8_t* codes_kn;  // [K,N]
+    float* par;         // [4] lo, hi, scale, bias
+    int* start_nk;      // [N * ceil(K/128) + 1]
+    uint32_t* ent_nk;   // [cap]
+    int* start_kn;      // [K * ceil(N/128) + 1]
+    uint32_t* ent_kn;   // [cap]
+    int cap;
+};
+size_t outlier_buckets_nk(int K, int N);
+size_t outlier_buckets_kn(int K, int N);
+size_t outlier_workspace_bytes(int K, int N);
+cudaError_t launch_quantize_outlier(const float* W, int K, int N, const OutlierKernel& q,
+                                    void* workspace, cudaStream_t s);
 // dX = dY (Wq sw)^T + c G A^T.  tcgen05 bf16 path when possible, else SIMT.
 // w4: Wq holds packed int4 codes [N, K/2] (K % 32 == 0).
 cudaError_t launch_gemm_dx(Act act, const void* dY, const int8_t* Wq, const float* sw, int M,

@@ -106,9 +106,12 @@ struct K3Cfg {
     static constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 };
 
-// W4: Wq holds packed int4 codes [N, K/2] (two per byte, even k in the low
-// nibble) instead of int8 codes [N, K]; a 16-byte fetch then carries 32 codes.
-template <int MSUB, int BN, int RMAX, bool W4>
+// MODE 0: int8 codes [N, K] with a scale per contraction row.  MODE 1: packed
+// int4 codes [N, K/2] (two per byte, even k in the low nibble); a 16-byte
+// fetch then carries 32 codes.  MODE 2: uint8 affine codes of an
+// outlier-compensated kernel (ep.ol), whose fp16 outliers are written over
+// the de-quantized tile.
+template <int MSUB, int BN, int RMAX, int MODE>
 __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
     k3_dx_dequant_kernel(const __grid_constant__ CUtensorMap tmDY, int dy3d,
                          const int8_t* __restrict__ Wq, const float* __restrict__ sw, int M, int N,
@@ -116,6 +119,7 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
     using C = K3Cfg<MSUB, BN, RMAX>;
     constexpr int S = C::STAGES;
     constexpr int kBKn = C::kBKn;
+    constexpr bool W4 = MODE == 1;
     constexpr uint32_t kLbo = (kBKn / 8) * 1024;  // MN-block stride of the bf16 tile
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -293,6 +297,11 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
         uint4 qr[P][kPerLane];
         float sr[P][kPerLane];
         uint32_t inb[P];  // bit i: chunk i of the ring slot lies inside the matrices
+        float ascale = 0.f, abias = 0.f;  // MODE 2: the tensor's affine parameters
+        if constexpr (MODE == 2) {
+            ascale = __ldg(ep.ol.par + 2);
+            abias = __ldg(ep.ol.par + 3);
+        }
         auto fetch = [&](uint4 (&q)[kPerLane], float (&sc)[kPerLane], uint32_t& in_bits) {
             const bool live_g = grp + kDqGroups * fj < total_kb;
             in_bits = 0;
@@ -306,7 +315,7 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
                 const int kc = k < K ? k : K - kCodes;
                 q[i] = __ldg(reinterpret_cast<const uint4*>(Wq + static_cast<size_t>(nc) * row_bytes +
                                                             (W4 ? kc / 2 : kc)));
-                sc[i] = __ldg(sw + nc);
+                sc[i] = MODE == 2 ? 1.f : __ldg(sw + nc);
             }
             ++fj;
             fkb += kDqGroups;
@@ -358,11 +367,31 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
                         *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn + 24, nr, kLbo)) =
                             make_uint4(o[4], o[5], o[6], o[7]);
                     } else {
-                        dequant16(qr[v][i], scale, o);
+                        if constexpr (MODE == 2) {
+                            // outside the matrices: zero through the affine parameters
+                            const bool in = (inb[v] >> i) & 1u;
+                            dequant16_affine(qr[v][i], in ? ascale : 0.f, in ? abias : 0.f, o);
+                        } else {
+                            dequant16(qr[v][i], scale, o);
+                        }
                         *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn, nr, kLbo)) =
                             make_uint4(o[0], o[1], o[2], o[3]);
                         *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn + 8, nr, kLbo)) =
                             make_uint4(o[4], o[5], o[6], o[7]);
+                    }
+                }
+                if constexpr (MODE == 2) {
+                    // The warp wrote whole tile rows nr = kRW gw + (c % 32) /
+                    // kChunksPerRow + kRW kWPG i (kRW rows per 32 chunks);
+                    // its lanes now write those rows' outliers.
+                    constexpr int kRW = 32 / kChunksPerRow;
+                    __syncwarp();
+                    const int t = static_cast<int>(blockIdx.x) + (g / nkb) * static_cast<int>(gridDim.x);
+                    const int c0 = (t % num_k) * BN;
+                    for (int idx = lane; idx < kPerLane * kRW; idx += 32) {
+                        const int nr = gw * kRW + idx % kRW + kRW * kWPG * (idx / kRW);
+                        const int n = (g % nkb) * kBKn + nr;
+                        if (n < N && c0 < K) patch_outliers(ep.ol, n, c0, BN, wt, nr, kLbo);
                     }
                 }
                 fence_proxy_async_smem();
@@ -402,7 +431,7 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
                 for (int e = et; e < BN * C::kKL; e += 32 * C::kEpiWarps) {
                     const int cc = e / C::kKL, j = e % C::kKL;
                     const int k = k0 + cc;
-                    const float a = (k < K && j < ep.r) ? ep.A[static_cast<size_t>(k) * ep.r + j] : 0.f;
+                    const float a = (k < K && j < ep.r) ? a_at(ep, k, j) : 0.f;
                     float hi, lo;
                     tf32_split(a, hi, lo);
                     *reinterpret_cast<float*>(at + kmajor_tf32_offset(cc, j, C::kKL)) = hi;
@@ -452,9 +481,9 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
                     if constexpr (!C::kLoraMMA) {
                         const int k = k0 + c;
                         if (k < K)
-                            for (int j = 0; j < ep.r; ++j)
-                                acc = fmaf(gr[j], __ldg(ep.A + static_cast<size_t>(k) * ep.r + j), acc);
+                            for (int j = 0; j < ep.r; ++j) acc = fmaf(gr[j], a_at(ep, k, j), acc);
                     }
+                    if (ep.bias && k0 + c < K) acc += __ldg(ep.bias + k0 + c);
                     y[e] = acc;
                 }
                 if (ep.gate && row_ok && k0 + col < K) {
@@ -487,11 +516,11 @@ __global__ void __launch_bounds__(K3Cfg<MSUB, BN, RMAX>::kThreads, 1)
     }
 }
 
-template <int MSUB, int BN, int RMAX, bool W4>
+template <int MSUB, int BN, int RMAX, int MODE>
 cudaError_t launch_tc(const void* dY, const int8_t* Wq, const float* sw, int M, int N, int K,
                       const DxEpilogue& ep, int* status, cudaStream_t s) {
     using C = K3Cfg<MSUB, BN, RMAX>;
-    auto kern = k3_dx_dequant_kernel<MSUB, BN, RMAX, W4>;
+    auto kern = k3_dx_dequant_kernel<MSUB, BN, RMAX, MODE>;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), C::kTotal);
     if (e != cudaSuccess) return e;
     // dY as [row][64-column block][64] (one 3-D box per stage) when the rows
@@ -510,21 +539,21 @@ cudaError_t launch_tc(const void* dY, const int8_t* Wq, const float* sw, int M, 
                     status);
 }
 
-template <int RMAX, bool W4>
+template <int RMAX, int MODE>
 cudaError_t launch_tc_cfg(int cfg, const void* dY, const int8_t* Wq, const float* sw, int M, int N,
                           int K, const DxEpilogue& ep, int* status, cudaStream_t s) {
-    if (cfg == 0) return launch_tc<2, 128, RMAX, W4>(dY, Wq, sw, M, N, K, ep, status, s);
-    if (cfg == 1) return launch_tc<1, 128, RMAX, W4>(dY, Wq, sw, M, N, K, ep, status, s);
-    return launch_tc<1, 64, RMAX, W4>(dY, Wq, sw, M, N, K, ep, status, s);
+    if (cfg == 0) return launch_tc<2, 128, RMAX, MODE>(dY, Wq, sw, M, N, K, ep, status, s);
+    if (cfg == 1) return launch_tc<1, 128, RMAX, MODE>(dY, Wq, sw, M, N, K, ep, status, s);
+    return launch_tc<1, 64, RMAX, MODE>(dY, Wq, sw, M, N, K, ep, status, s);
 }
 
-template <bool W4>
+template <int MODE>
 cudaError_t launch_tc_r(int cfg, const void* dY, const int8_t* Wq, const float* sw, int M, int N,
                         int K, const DxEpilogue& ep, int* status, cudaStream_t s) {
-    if (ep.r <= 4) return launch_tc_cfg<4, W4>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
-    if (ep.r <= 8) return launch_tc_cfg<8, W4>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
-    if (ep.r <= 16) return launch_tc_cfg<16, W4>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
-    return launch_tc_cfg<64, W4>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
+    if (ep.r <= 4) return launch_tc_cfg<4, MODE>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
+    if (ep.r <= 8) return launch_tc_cfg<8, MODE>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
+    if (ep.r <= 16) return launch_tc_cfg<16, MODE>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
+    return launch_tc_cfg<64, MODE>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
 }
 
 // ---------------------------------------------------------------- SIMT path
@@ -534,7 +563,7 @@ cudaError_t launch_tc_r(int cfg, const void* dY, const int8_t* Wq, const float* 
 constexpr int kSB = 64;
 constexpr int kSN = 16;
 
-template <typename T, bool W4>
+template <typename T, int MODE>
 __global__ void __launch_bounds__(256) k3_dx_simt_kernel(const T* __restrict__ dY,
                                                          const int8_t* __restrict__ Wq,
                                                          const float* __restrict__ sw, int M,
@@ -557,18 +586,40 @@ __global__ void __launch_bounds__(256) k3_dx_simt_kernel(const T* __restrict__ d
             const int n = n0 + nn, k = k0 + kk;
             float w = 0.f;
             if (n < N && k < K) {
-                int code;
-                if constexpr (W4) {
-                    const int b = reinterpret_cast<const uint8_t*>(Wq)[static_cast<size_t>(n) * (K / 2) + k / 2];
-                    const int nib = (k & 1) ? (b >> 4) & 0xF : b & 0xF;
-                    code = nib >= 8 ? nib - 16 : nib;
+                if constexpr (MODE == 2) {
+                    const int code = reinterpret_cast<const uint8_t*>(Wq)[static_cast<size_t>(n) * K + k];
+                    w = __fadd_rn(__ldg(ep.ol.par + 3), __fmul_rn(static_cast<float>(code), __ldg(ep.ol.par + 2)));
                 } else {
-                    code = Wq[static_cast<size_t>(n) * K + k];
+                    int code;
+                    if constexpr (MODE == 1) {
+                        const int b = reinterpret_cast<const uint8_t*>(Wq)[static_cast<size_t>(n) * (K / 2) + k / 2];
+                        const int nib = (k & 1) ? (b >> 4) & 0xF : b & 0xF;
+                        code = nib >= 8 ? nib - 16 : nib;
+                    } else {
+                        code = Wq[static_cast<size_t>(n) * K + k];
+                    }
+                    w = __fmul_rn(static_cast<float>(code), __ldg(sw + n));
                 }
-                w = __fmul_rn(static_cast<float>(code), __ldg(sw + n));
                 if constexpr (sizeof(T) == 2) w = __bfloat162float(__float2bfloat16_rn(w));
             }
             sW[nn][kk] = w;
+        }
+        if constexpr (MODE == 2) {
+            // the outliers of the 16 contraction rows, columns k0 .. k0+63
+            __syncthreads();
+            if (threadIdx.x < kSN && n0 + static_cast<int>(threadIdx.x) < N) {
+                const int n = n0 + threadIdx.x;
+                const size_t b = static_cast<size_t>(n) * ep.ol.nb + (k0 >> 7);
+                const int e1 = __ldg(ep.ol.start + b + 1);
+                for (int e = __ldg(ep.ol.start + b); e < e1; ++e) {
+                    const uint32_t v = __ldg(ep.ol.ent + e);
+                    const int col = static_cast<int>(v >> 16) - (k0 & 127);
+                    if (col < 0 || col >= kSB) continue;
+                    float f = __half2float(__ushort_as_half(static_cast<unsigned short>(v & 0xFFFFu)));
+                    if constexpr (sizeof(T) == 2) f = __bfloat162float(__float2bfloat16_rn(f));
+                    sW[threadIdx.x][col] = f;
+                }
+            }
         }
         __syncthreads();
 #pragma unroll
@@ -602,11 +653,11 @@ __global__ void __launch_bounds__(256) k3_dx_simt_kernel(const T* __restrict__ d
             const int k = k0 + tx + 16 * j;
             if (k >= K) continue;
             float l = 0.f;
-            for (int jj = 0; jj < ep.r; ++jj)
-                l = fmaf(sG[ty + 16 * i][jj], ep.A[static_cast<size_t>(k) * ep.r + jj], l);
+            for (int jj = 0; jj < ep.r; ++jj) l = fmaf(sG[ty + 16 * i][jj], a_at(ep, k, jj), l);
             const bool pass =
                 !ep.gate || ActIO<T>::to_f(static_cast<const T*>(ep.gate)[static_cast<size_t>(m) * K + k]) > 0.f;
-            dX[static_cast<size_t>(m) * K + k] = ActIO<T>::from_f(pass ? acc[i][j] + ep.c * l : 0.f);
+            const float b = ep.bias ? __ldg(ep.bias + k) : 0.f;
+            dX[static_cast<size_t>(m) * K + k] = ActIO<T>::from_f(pass ? acc[i][j] + ep.c * l + b : 0.f);
         }
     }
 }
@@ -615,18 +666,21 @@ __global__ void __launch_bounds__(256) k3_dx_simt_kernel(const T* __restrict__ d
 
 cudaError_t launch_gemm_dx(Act act, const void* dY, const int8_t* Wq, const float* sw, int M,
                            int N, int K, const DxEpilogue& ep, int* status, cudaStream_t s, bool w4) {
-    const bool tc = act == kBF16 && (N % 8) == 0;
+    const bool tc = act == kBF16 && (N % 8) == 0 && (!ep.ol.par || (K % 16) == 0);
+    const int mode = ep.ol.par ? 2 : (w4 ? 1 : 0);
     if (!tc) {
         dim3 grid((K + kSB - 1) / kSB, (M + kSB - 1) / kSB);
-        if (act == kBF16)
-            return w4 ? launch_k(k3_dx_simt_kernel<__nv_bfloat16, true>, grid, dim3(256), 0, s, 1,
-                                 static_cast<const __nv_bfloat16*>(dY), Wq, sw, M, N, K, ep)
-                      : launch_k(k3_dx_simt_kernel<__nv_bfloat16, false>, grid, dim3(256), 0, s, 1,
-                                 static_cast<const __nv_bfloat16*>(dY), Wq, sw, M, N, K, ep);
-        return w4 ? launch_k(k3_dx_simt_kernel<float, true>, grid, dim3(256), 0, s, 1,
-                             static_cast<const float*>(dY), Wq, sw, M, N, K, ep)
-                  : launch_k(k3_dx_simt_kernel<float, false>, grid, dim3(256), 0, s, 1,
-                             static_cast<const float*>(dY), Wq, sw, M, N, K, ep);
+        if (act == kBF16) {
+            auto kern = mode == 2 ? k3_dx_simt_kernel<__nv_bfloat16, 2>
+                                  : (mode == 1 ? k3_dx_simt_kernel<__nv_bfloat16, 1>
+                                               : k3_dx_simt_kernel<__nv_bfloat16, 0>);
+            return launch_k(kern, grid, dim3(256), 0, s, 1, static_cast<const __nv_bfloat16*>(dY), Wq,
+                            sw, M, N, K, ep);
+        }
+        auto kern = mode == 2 ? k3_dx_simt_kernel<float, 2>
+                              : (mode == 1 ? k3_dx_simt_kernel<float, 1> : k3_dx_simt_kernel<float, 0>);
+        return launch_k(kern, grid, dim3(256), 0, s, 1, static_cast<const float*>(dY), Wq, sw, M, N, K,
+                        ep);
     }
     if (gemm_dx_pair_applies(M, N, K, ep.r))
         return launch_gemm_dx_pair(dY, Wq, sw, M, N, K, ep, status, s, w4);
@@ -645,8 +699,9 @@ cudaError_t launch_gemm_dx(Act act, const void* dY, const int8_t* Wq, const floa
     int cfg = 2;
     if (c1 < c2 && c1 <= c0) cfg = 1;
     else if (c0 < c2 && c0 < c1) cfg = 0;
-    return w4 ? launch_tc_r<true>(cfg, dY, Wq, sw, M, N, K, ep, status, s)
-              : launch_tc_r<false>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
+    if (mode == 2) return launch_tc_r<2>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
+    return w4 ? launch_tc_r<1>(cfg, dY, Wq, sw, M, N, K, ep, status, s)
+              : launch_tc_r<0>(cfg, dY, Wq, sw, M, N, K, ep, status, s);
 }
 
 }  // namespace qlora

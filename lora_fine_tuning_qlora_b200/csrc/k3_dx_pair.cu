@@ -58,7 +58,7 @@ struct PairCfg {
     static constexpr int kWBytes = kPK * (kPN / 2) * 2;   // de-quantized half tile: 16 KB
     static constexpr int kStageBytes = kABytes + kWBytes;
     static constexpr int kStgBytes = kEpiW * 32 * stage_pitch<__nv_bfloat16>();
-    static constexpr int kATabBytes = kPN * RP * 4;       // A rows of the tile's 256 columns
+    static constexpr int kATabBytes = kPN * (RP + 1) * 4;  // A rows (+ bias) of the tile's 256 columns
     static constexpr int kFixed = kStgBytes + kATabBytes + 512 + 1024;
     static constexpr int kStagesFit = (kPSmemLimit - kFixed) / kStageBytes;
     static constexpr int STAGES = 4;  // a multiple of the stage groups (more measured no faster)
@@ -71,13 +71,17 @@ struct PairCfg {
     static constexpr uint32_t kTmemCols = 2 * kAccCols;   // two buffers: all 512 columns
 };
 
-template <int RP, bool W4>
+// MODE: 0 int8 codes with a scale per contraction row; 1 packed int4 codes;
+// 2 outlier-compensated uint8 affine codes (ep.ol) with their fp16 outliers
+// written over the de-quantized tile.
+template <int RP, int MODE>
 __global__ void __launch_bounds__(kPThreads, 1)
     k3_dx_pair_kernel(const __grid_constant__ CUtensorMap tmDY, const int8_t* __restrict__ Wq,
                       const float* __restrict__ sw, int M, int N, int K, DxEpilogue ep,
                       int* status) {
     using C = PairCfg<RP>;
     constexpr int S = C::STAGES;
+    constexpr bool W4 = MODE == 1;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -88,6 +92,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     uint64_t* tempty = tfull + 2;                                     // [2] (CTA 0)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
     float* sAt = reinterpret_cast<float*>(smem + C::kATabOff);        // [256][RP]
+    float* sBias = sAt + kPN * RP;                                     // [256]
 
     const uint32_t rank = cluster_ctarank();
     const int warp = threadIdx.x / 32;
@@ -217,6 +222,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
         uint4 qr[P][kPerLane];
         float sr[P][kPerLane];
         uint32_t inb[P];
+        float ascale = 0.f, abias = 0.f;  // MODE 2: the tensor's affine parameters
+        if constexpr (MODE == 2) {
+            ascale = __ldg(ep.ol.par + 2);
+            abias = __ldg(ep.ol.par + 3);
+        }
         auto fetch = [&](uint4 (&q)[kPerLane], float (&sc)[kPerLane], uint32_t& in_bits) {
             const bool live_g = grp + kDqGroups * fj < total_kb;
             in_bits = 0;
@@ -230,7 +240,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 const int kc = k < K ? k : K - kCodes;
                 q[i] = __ldg(reinterpret_cast<const uint4*>(Wq + static_cast<size_t>(nc) * row_bytes +
                                                             (W4 ? kc / 2 : kc)));
-                sc[i] = __ldg(sw + nc);
+                sc[i] = MODE == 2 ? 1.f : __ldg(sw + nc);
             }
             // advance to the group's next stage
             ++fj;
@@ -283,12 +293,30 @@ __global__ void __launch_bounds__(kPThreads, 1)
                         *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn + 24, nr, kPLbo)) =
                             make_uint4(o[4], o[5], o[6], o[7]);
                     } else {
-                        dequant16(qr[v][i], scale, o);
+                        if constexpr (MODE == 2) {
+                            // outside the matrices: zero through the affine parameters
+                            const bool in = (inb[v] >> i) & 1u;
+                            dequant16_affine(qr[v][i], in ? ascale : 0.f, in ? abias : 0.f, o);
+                        } else {
+                            dequant16(qr[v][i], scale, o);
+                        }
                         *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn, nr, kPLbo)) =
                             make_uint4(o[0], o[1], o[2], o[3]);
                         *reinterpret_cast<uint4*>(wt + mn_sw128_offset(mn + 8, nr, kPLbo)) =
                             make_uint4(o[4], o[5], o[6], o[7]);
                     }
+                }
+                if constexpr (MODE == 2) {
+                    // The warp wrote whole tile rows nr = 4 gw + (c % 32) / 8 +
+                    // 4 kDqWPG i; each lane writes the outliers of one of them.
+                    static_assert(kPerLane * (32 / kChunksPerRow) == 32, "one row per lane");
+                    __syncwarp();
+                    const int nr = gw * (32 / kChunksPerRow) + (lane % (32 / kChunksPerRow)) +
+                                   (32 / kChunksPerRow) * kDqWPG * (lane / (32 / kChunksPerRow));
+                    const int n = (g % nkb) * kPK + nr;
+                    const int t = pair + (g / nkb) * npairs;
+                    const int c0 = (t % num_kt) * kPN + static_cast<int>(rank) * kHalf;
+                    if (n < N && c0 < K) patch_outliers(ep.ol, n, c0, kHalf, wt, nr, kPLbo);
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -316,10 +344,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
             const int k0 = (t % num_kt) * kPN;
             // A rows of the tile's columns (the last tile's reads are done)
             named_bar_sync(1, 32 * kEpiW);
+            for (int col = et; col < kPN; col += 32 * kEpiW)
+                sBias[col] = (ep.bias && k0 + col < K) ? __ldg(ep.bias + k0 + col) : 0.f;
             for (int e = et; e < kPN * RP; e += 32 * kEpiW) {
                 const int col = e / RP, j = e % RP;
                 const int k = k0 + col;
-                sAt[e] = (k < K && j < ep.r) ? __ldg(ep.A + static_cast<size_t>(k) * ep.r + j) : 0.f;
+                sAt[e] = (k < K && j < ep.r) ? a_at(ep, k, j) : 0.f;
             }
             named_bar_sync(1, 32 * kEpiW);
             const int row0 = m0 + q * 32;
@@ -341,7 +371,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #pragma unroll
                 for (int e = 0; e < kEpiCols; ++e) {
                     const float4* a4 = reinterpret_cast<const float4*>(sAt + (col + e) * RP);
-                    float acc = __uint_as_float(v[e]);
+                    float acc = __uint_as_float(v[e]) + sBias[col + e];
 #pragma unroll
                     for (int j4 = 0; j4 < RP / 4; ++j4) {
                         const float4 a = a4[j4];
@@ -388,11 +418,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
     }
 }
 
-template <int RP, bool W4>
+template <int RP, int MODE>
 cudaError_t launch_pair_t(const void* dY, const int8_t* Wq, const float* sw, int M, int N, int K,
                           const DxEpilogue& ep, int* status, cudaStream_t s) {
     using C = PairCfg<RP>;
-    auto kern = k3_dx_pair_kernel<RP, W4>;
+    auto kern = k3_dx_pair_kernel<RP, MODE>;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), C::kTotal);
     if (e != cudaSuccess) return e;
     // dY as [row][64-column block][64]: one box of 128 rows x one block per stage
@@ -413,16 +443,19 @@ bool gemm_dx_pair_applies(int M, int N, int K, int r) {
     return tiles >= sm_count() / 2;
 }
 
+template <int MODE>
+cudaError_t launch_pair_mode(const void* dY, const int8_t* Wq, const float* sw, int M, int N,
+                             int K, const DxEpilogue& ep, int* status, cudaStream_t s) {
+    if (ep.r <= 4) return launch_pair_t<4, MODE>(dY, Wq, sw, M, N, K, ep, status, s);
+    if (ep.r <= 8) return launch_pair_t<8, MODE>(dY, Wq, sw, M, N, K, ep, status, s);
+    return launch_pair_t<16, MODE>(dY, Wq, sw, M, N, K, ep, status, s);
+}
+
 cudaError_t launch_gemm_dx_pair(const void* dY, const int8_t* Wq, const float* sw, int M, int N,
                                 int K, const DxEpilogue& ep, int* status, cudaStream_t s, bool w4) {
-    if (ep.r <= 4)
-        return w4 ? launch_pair_t<4, true>(dY, Wq, sw, M, N, K, ep, status, s)
-                  : launch_pair_t<4, false>(dY, Wq, sw, M, N, K, ep, status, s);
-    if (ep.r <= 8)
-        return w4 ? launch_pair_t<8, true>(dY, Wq, sw, M, N, K, ep, status, s)
-                  : launch_pair_t<8, false>(dY, Wq, sw, M, N, K, ep, status, s);
-    return w4 ? launch_pair_t<16, true>(dY, Wq, sw, M, N, K, ep, status, s)
-              : launch_pair_t<16, false>(dY, Wq, sw, M, N, K, ep, status, s);
+    if (ep.ol.par) return launch_pair_mode<2>(dY, Wq, sw, M, N, K, ep, status, s);
+    return w4 ? launch_pair_mode<1>(dY, Wq, sw, M, N, K, ep, status, s)
+              : launch_pair_mode<0>(dY, Wq, sw, M, N, K, ep, status, s);
 }
 
 }  // namespace qlora

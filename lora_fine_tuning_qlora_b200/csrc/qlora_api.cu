@@ -1,6 +1,7 @@
 // qlora_api.cu -- the C ABI of libqlora.so (declared in include/qlora.h):
 // argument validation, workspace layout, tensor-map encoding and the launch
 // sequence of each call.  No device memory is allocated here.
+#include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <map>
@@ -635,6 +636,152 @@ int qlora_merge_int4(const qlora_layer_desc* d, const uint8_t* Wp, const float* 
     return cuda_status(launch_merge_int4(Wp, sw, A, B, d->K, d->N, d->r, c, Wp_out, sw_out,
                                          static_cast<cudaStream_t>(stream)),
                        "merge_int4 launch");
+}
+
+// ---------------------------------------------------------------------------
+// outlier-compensated int8 kernels
+// ---------------------------------------------------------------------------
+static long pct_index(long n, double p) {
+    // the same fp64 expression as the device's percentile positions
+    const double h = static_cast<double>(n - 1) * p / 100.0;
+    long i = static_cast<long>(floor(h));
+    return i > n - 1 ? n - 1 : i;
+}
+
+size_t qlora_outlier_cap(int K, int N) {
+    if (K < 1 || N < 1) return 0;
+    const long n = static_cast<long>(K) * N;
+    return static_cast<size_t>((pct_index(n, 0.1) + 1) + (n - 1 - pct_index(n, 99.9)));
+}
+
+size_t qlora_outlier_workspace_bytes(int K, int N) {
+    if (K < 1 || N < 1) return 0;
+    return outlier_workspace_bytes(K, N);
+}
+
+static int check_outlier(const qlora_outlier_kernel* q, int K, int N) {
+    QL_REQUIRE(q, QLORA_EINVAL, "NULL outlier kernel");
+    QL_REQUIRE(q->codes_nk && q->codes_kn && q->par && q->start_nk && q->ent_nk && q->start_kn &&
+                   q->ent_kn,
+               QLORA_EINVAL, "NULL member of the outlier kernel");
+    QL_REQUIRE(aligned(q->codes_nk, 16) && aligned(q->codes_kn, 16), QLORA_EALIGN,
+               "outlier codes must be 16-byte aligned");
+    QL_REQUIRE(aligned(q->par, 4) && aligned(q->start_nk, 4) && aligned(q->ent_nk, 4) &&
+                   aligned(q->start_kn, 4) && aligned(q->ent_kn, 4),
+               QLORA_EALIGN, "outlier tables must be 4-byte aligned");
+    QL_REQUIRE(q->cap >= 0 && static_cast<size_t>(q->cap) >= qlora_outlier_cap(K, N), QLORA_EINVAL,
+               "outlier capacity below qlora_outlier_cap(K, N)");
+    return QLORA_OK;
+}
+
+int qlora_outlier_quantize(const float* W, int K, int N, const qlora_outlier_kernel* q,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+    QL_REQUIRE(W && workspace, QLORA_EINVAL, "NULL pointer argument");
+    QL_REQUIRE(K >= 1 && N >= 1, QLORA_ESHAPE, "K and N must be >= 1");
+    QL_REQUIRE(static_cast<long>(K) * N < (1L << 31), QLORA_ESHAPE, "K * N must be below 2^31");
+    int rc = check_outlier(q, K, N);
+    if (rc != QLORA_OK) return rc;
+    QL_REQUIRE(aligned(W, 4) && aligned(workspace, 256), QLORA_EALIGN,
+               "W must be 4-byte aligned, workspace 256-byte aligned");
+    QL_REQUIRE(workspace_bytes >= outlier_workspace_bytes(K, N), QLORA_EINVAL, "workspace too small");
+    OutlierKernel k{q->codes_nk, q->codes_kn, q->par, q->start_nk, q->ent_nk, q->start_kn, q->ent_kn,
+                    q->cap};
+    return cuda_status(launch_quantize_outlier(W, K, N, k, workspace, static_cast<cudaStream_t>(stream)),
+                       "outlier quantizer launch");
+}
+
+int qlora_outlier_forward(const qlora_layer_desc* d, int M, const void* X,
+                          const qlora_outlier_kernel* q, const float* bias, const float* A,
+                          const float* B, void* Y, float* xA, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+    int rc = check_layer(d, M);
+    if (rc != QLORA_OK) return rc;
+    QL_REQUIRE(X && A && B && Y && xA && workspace, QLORA_EINVAL, "NULL pointer argument");
+    rc = check_outlier(q, d->K, d->N);
+    if (rc != QLORA_OK) return rc;
+    QL_REQUIRE(aligned(X, 16) && aligned(Y, 16) && aligned(workspace, 256), QLORA_EALIGN,
+               "X and Y must be 16-byte aligned, workspace 256-byte aligned");
+    QL_REQUIRE(aligned(A, 4) && aligned(B, 4) && aligned(xA, 4) && (!bias || aligned(bias, 4)),
+               QLORA_EALIGN, "fp32 vectors must be 4-byte aligned");
+    if (M == 0) return QLORA_OK;
+    const WsLayout w = layout_for(*d, M);
+    QL_REQUIRE(workspace_bytes >= w.total, QLORA_EINVAL, "workspace too small");
+    int* status = status_ptr();
+    QL_REQUIRE(status, QLORA_ECUDA, "no CUDA device");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    // xA from the input pass (its int8 rows go to the workspace unused: the
+    // layer's activations are not quantized)
+    rc = cuda_status(launch_quantize_rows(act_of(d), X, A, M, d->K, d->r,
+                                          reinterpret_cast<int8_t*>(ws + w.xq),
+                                          reinterpret_cast<float*>(ws + w.sx), xA, status, s),
+                     "input pass launch");
+    if (rc != QLORA_OK) return rc;
+    // Y = X Wr + bias + c xA B on the de-quantizing GEMM: contraction over K
+    // (the rows of codes_kn), output columns N, rank-r factor B^T
+    DxEpilogue ep;
+    ep.Gp = xA;
+    ep.ncb = 1;
+    ep.A = B;
+    ep.a_ks = 1;
+    ep.a_js = d->N;
+    ep.r = d->r;
+    ep.c = lora_scale(d);
+    ep.dX = Y;
+    ep.gate = nullptr;
+    ep.bias = bias;
+    ep.ol = OutlierArgs{q->par, q->start_kn, q->ent_kn, (d->N + 127) / 128};
+    return cuda_status(launch_gemm_dx(act_of(d), X, reinterpret_cast<const int8_t*>(q->codes_kn),
+                                      nullptr, M, d->K, d->N, ep, status, s),
+                       "outlier forward GEMM launch");
+}
+
+int qlora_outlier_backward(const qlora_layer_desc* d, int M, const void* X, const void* dY,
+                           const qlora_outlier_kernel* q, const float* A, const float* B,
+                           const float* xA, void* dX, float* dA, float* dB, float* dbias,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_layer(d, M);
+    if (rc != QLORA_OK) return rc;
+    QL_REQUIRE(X && dY && A && B && xA && dA && dB && workspace, QLORA_EINVAL,
+               "NULL pointer argument");
+    rc = check_outlier(q, d->K, d->N);
+    if (rc != QLORA_OK) return rc;
+    QL_REQUIRE(aligned(X, 16) && aligned(dY, 16) && (!dX || aligned(dX, 16)) &&
+                   aligned(workspace, 256),
+               QLORA_EALIGN, "X, dY, dX must be 16-byte aligned, workspace 256-byte aligned");
+    QL_REQUIRE(aligned(A, 4) && aligned(B, 4) && aligned(xA, 4) && aligned(dA, 4) &&
+                   aligned(dB, 4) && (!dbias || aligned(dbias, 4)),
+               QLORA_EALIGN, "fp32 vectors must be 4-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M == 0) {
+        rc = cuda_status(cudaMemsetAsync(dA, 0, sizeof(float) * d->K * d->r, s), "memset dA");
+        if (rc == QLORA_OK)
+            rc = cuda_status(cudaMemsetAsync(dB, 0, sizeof(float) * d->r * d->N, s), "memset dB");
+        if (rc == QLORA_OK && dbias)
+            rc = cuda_status(cudaMemsetAsync(dbias, 0, sizeof(float) * d->N, s), "memset dbias");
+        return rc;
+    }
+    const WsLayout w = layout_for(*d, M);
+    QL_REQUIRE(workspace_bytes >= w.total, QLORA_EINVAL, "workspace too small");
+    rc = qlora_lora_grad_dy(d, M, dY, B, xA, dB, dbias, nullptr, workspace, workspace_bytes, stream);
+    if (rc != QLORA_OK) return rc;
+    if (dX) {
+        int* status = status_ptr();
+        QL_REQUIRE(status, QLORA_ECUDA, "no CUDA device");
+        DxEpilogue ep;
+        ep.Gp = g_source(w, workspace, &ep.ncb);
+        ep.A = A;
+        ep.r = d->r;
+        ep.c = lora_scale(d);
+        ep.dX = dX;
+        ep.gate = nullptr;
+        ep.ol = OutlierArgs{q->par, q->start_nk, q->ent_nk, (d->K + 127) / 128};
+        rc = cuda_status(launch_gemm_dx(act_of(d), dY, reinterpret_cast<const int8_t*>(q->codes_nk),
+                                        nullptr, M, d->N, d->K, ep, status, s),
+                         "outlier dX GEMM launch");
+        if (rc != QLORA_OK) return rc;
+    }
+    return qlora_lora_grad_x(d, M, X, dA, workspace, workspace_bytes, stream);
 }
 
 int qlora_selftest_wait_timeout(unsigned int limit_us, void* stream) {

@@ -33,7 +33,9 @@ EXPORTED = ("qlora_quantize_weight", "qlora_workspace_bytes", "qlora_forward",
             "qlora_selftest_wait_timeout", "qlora_backward_noalloc", "qlora_lora_g",
             "qlora_lora_grad_b", "qlora_gemm_forward_relu", "qlora_gemm_dx_relu",
             "qlora_set_rank_pass_rows", "qlora_quantize_weight_int4", "qlora_unpack_int4",
-            "qlora_gemm_dx_int4", "qlora_merge_int4", "qlora_gemm_forward_int4")
+            "qlora_gemm_dx_int4", "qlora_merge_int4", "qlora_gemm_forward_int4",
+            "qlora_outlier_cap", "qlora_outlier_workspace_bytes", "qlora_outlier_quantize",
+            "qlora_outlier_forward", "qlora_outlier_backward")
 
 
 class QLoraError(RuntimeError):
@@ -49,6 +51,14 @@ class LayerDesc(ctypes.Structure):
 
 class Debug(ctypes.Structure):
     _fields_ = [("xq", ctypes.c_void_p), ("sx", ctypes.c_void_p), ("acc", ctypes.c_void_p)]
+
+
+class OutlierKernelStruct(ctypes.Structure):
+    """qlora_outlier_kernel: device pointers of an outlier-compensated kernel."""
+    _fields_ = [("codes_nk", ctypes.c_void_p), ("codes_kn", ctypes.c_void_p),
+                ("par", ctypes.c_void_p), ("start_nk", ctypes.c_void_p),
+                ("ent_nk", ctypes.c_void_p), ("start_kn", ctypes.c_void_p),
+                ("ent_kn", ctypes.c_void_p), ("cap", ctypes.c_int)]
 
 
 def _load():
@@ -103,6 +113,16 @@ def _load():
     lib.qlora_merge_int4.argtypes = [D, P, P, P, P, P, P, P]
     for f in (lib.qlora_quantize_weight_int4, lib.qlora_unpack_int4, lib.qlora_gemm_dx_int4,
               lib.qlora_merge_int4):
+        f.restype = I
+    OK = ctypes.POINTER(OutlierKernelStruct)
+    lib.qlora_outlier_cap.argtypes = [I, I]
+    lib.qlora_outlier_cap.restype = Z
+    lib.qlora_outlier_workspace_bytes.argtypes = [I, I]
+    lib.qlora_outlier_workspace_bytes.restype = Z
+    lib.qlora_outlier_quantize.argtypes = [P, I, I, OK, P, Z, P]
+    lib.qlora_outlier_forward.argtypes = [D, I, P, OK, P, P, P, P, P, P, Z, P]
+    lib.qlora_outlier_backward.argtypes = [D, I, P, P, OK, P, P, P, P, P, P, P, P, Z, P]
+    for f in (lib.qlora_outlier_quantize, lib.qlora_outlier_forward, lib.qlora_outlier_backward):
         f.restype = I
     lib.qlora_set_rank_pass_rows.argtypes = [I]
     lib.qlora_set_rank_pass_rows.restype = I
@@ -299,6 +319,89 @@ def merge_int4(d: LayerDesc, Wp, sw, A, B, stream=None):
     _check(_lib.qlora_merge_int4(ctypes.byref(d), _ptr(Wp), _ptr(sw), _ptr(A), _ptr(B), _ptr(Wp2),
                                  _ptr(sw2), _stream(stream)))
     return Wp2, sw2
+
+
+@dataclass
+class OutlierKernel:
+    """Device buffers of an outlier-compensated uint8 kernel of a K x N
+    weight (layouts of include/qlora.h, qlora_outlier_kernel)."""
+
+    K: int
+    N: int
+    codes_nk: torch.Tensor  # [N, K] uint8
+    codes_kn: torch.Tensor  # [K, N] uint8
+    par: torch.Tensor       # [4] fp32: lo, hi, scale, bias
+    start_nk: torch.Tensor  # [N * ceil(K/128) + 1] int32
+    ent_nk: torch.Tensor    # [cap] int32 (uint32 entries)
+    start_kn: torch.Tensor  # [K * ceil(N/128) + 1] int32
+    ent_kn: torch.Tensor    # [cap] int32
+
+    def struct(self) -> OutlierKernelStruct:
+        return OutlierKernelStruct(self.codes_nk.data_ptr(), self.codes_kn.data_ptr(),
+                                   self.par.data_ptr(), self.start_nk.data_ptr(),
+                                   self.ent_nk.data_ptr(), self.start_kn.data_ptr(),
+                                   self.ent_kn.data_ptr(), int(self.ent_nk.numel()))
+
+    @property
+    def count(self) -> int:
+        """Number of outliers (reads the device tables)."""
+        return int(self.start_nk[-1].item())
+
+
+def qlora_outlier_cap(K: int, N: int) -> int:
+    return int(_lib.qlora_outlier_cap(int(K), int(N)))
+
+
+def qlora_outlier_workspace_bytes(K: int, N: int) -> int:
+    return int(_lib.qlora_outlier_workspace_bytes(int(K), int(N)))
+
+
+def outlier_kernel_buffers(K: int, N: int, device=None) -> OutlierKernel:
+    dev = device or "cuda"
+    cap = max(qlora_outlier_cap(K, N), 1)
+    nbk, nbn = (K + 127) // 128, (N + 127) // 128
+    return OutlierKernel(
+        K, N, torch.empty((N, K), dtype=torch.uint8, device=dev),
+        torch.empty((K, N), dtype=torch.uint8, device=dev),
+        torch.empty((4,), dtype=torch.float32, device=dev),
+        torch.empty((N * nbk + 1,), dtype=torch.int32, device=dev),
+        torch.empty((cap,), dtype=torch.int32, device=dev),
+        torch.empty((K * nbn + 1,), dtype=torch.int32, device=dev),
+        torch.empty((cap,), dtype=torch.int32, device=dev))
+
+
+def qlora_outlier_quantize(W: torch.Tensor, q: OutlierKernel, ws: torch.Tensor, stream=None):
+    K, N = W.shape
+    assert W.dtype == torch.float32 and (q.K, q.N) == (K, N)
+    st = q.struct()
+    _check(_lib.qlora_outlier_quantize(_ptr(W), K, N, ctypes.byref(st), _ptr(ws), ws.numel(),
+                                       _stream(stream)))
+
+
+def quantize_outlier(W: torch.Tensor, stream=None) -> OutlierKernel:
+    """W [K, N] fp32 -> its outlier-compensated kernel (fresh buffers)."""
+    K, N = W.shape
+    W = W.float().contiguous()
+    q = outlier_kernel_buffers(K, N, W.device)
+    ws = torch.empty(qlora_outlier_workspace_bytes(K, N), dtype=torch.uint8, device=W.device)
+    qlora_outlier_quantize(W, q, ws, stream)
+    return q
+
+
+def qlora_outlier_forward(d: LayerDesc, M: int, X, q: OutlierKernel, bias, A, B, Y, xA, ws,
+                          stream=None):
+    st = q.struct()
+    _check(_lib.qlora_outlier_forward(ctypes.byref(d), int(M), _ptr(X), ctypes.byref(st), _ptr(bias),
+                                      _ptr(A), _ptr(B), _ptr(Y), _ptr(xA), _ptr(ws), ws.numel(),
+                                      _stream(stream)))
+
+
+def qlora_outlier_backward(d: LayerDesc, M: int, X, dY, q: OutlierKernel, A, B, xA, dX, dA, dB,
+                           dbias, ws, stream=None):
+    st = q.struct()
+    _check(_lib.qlora_outlier_backward(ctypes.byref(d), int(M), _ptr(X), _ptr(dY), ctypes.byref(st),
+                                       _ptr(A), _ptr(B), _ptr(xA), _ptr(dX), _ptr(dA), _ptr(dB),
+                                       _ptr(dbias), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def qlora_set_rank_pass_rows(rows: int) -> int:
