@@ -423,6 +423,60 @@ def merge_entry(st, flush, roof, steps):
             "GB/s": by / (us * 1e-6) / 1e9, "frac_hbm": by / (us * 1e-6) / roof.bw}
 
 
+def outlier_entry(spec, dev, flush, roof, steps, warmup):
+    """fwd+bwd of the outlier-compensated variant of a layer: the uint8 affine
+    kernel rebuilt (with its fp16 outliers) tile by tile in shared memory in
+    front of the bf16 tensor cores, in both directions."""
+    import torch
+    from lora_fine_tuning_qlora_b200 import inputs, qlora
+    d = inputs.layer_inputs(spec)
+    act = torch.bfloat16
+    M, K, N, r = spec.M, spec.K, spec.N, spec.r
+    qk = qlora.quantize_outlier(torch.from_numpy(d["W"]).to(dev))
+    X = torch.from_numpy(d["X"]).to(act).to(dev)
+    dY = torch.from_numpy(d["dY"]).to(act).to(dev)
+    A = torch.from_numpy(d["A"]).to(dev)
+    B = torch.from_numpy(d["B"]).to(dev)
+    bias = torch.from_numpy(d["bias"]).to(dev)
+    desc = qlora.desc(K, N, r, spec.alpha, act)
+    ws = qlora.workspace(desc, M, dev)
+    Y = torch.empty((M, N), dtype=act, device=dev)
+    xA = torch.empty((M, r), dtype=torch.float32, device=dev)
+    dX = torch.empty((M, K), dtype=act, device=dev)
+    dA = torch.empty((K, r), dtype=torch.float32, device=dev)
+    dB = torch.empty((r, N), dtype=torch.float32, device=dev)
+    db = torch.empty((N,), dtype=torch.float32, device=dev)
+
+    def run():
+        qlora.qlora_outlier_forward(desc, M, X, qk, bias, A, B, Y, xA, ws)
+        qlora.qlora_outlier_backward(desc, M, X, dY, qk, A, B, xA, dX, dA, dB, db, ws)
+
+    run()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run()
+    ms = time_graph(g.replay, steps, warmup, flush)
+    step_us = 1e3 * statistics.median(ms)
+    e = 2
+    fl = 2.0 * M * N * K
+    # both GEMMs on bf16 tensor cores; the forward reads X, the uint8 codes and
+    # writes Y; the input pass reads X and writes xA
+    from lora_fine_tuning_qlora_b200.step import algorithmic_bytes
+    b = algorithmic_bytes(M, K, N, r, e)
+    fwd_bytes = M * K * e + K * N + M * N * e + 4.0 * (N + M * r + r * N)
+    t_roof = (max(fl / roof.bf16, fwd_bytes / roof.bw) + max(fl / roof.bf16, b["gemm_dx"] / roof.bw)
+              + (M * K * e + 4.0 * M * r + b["lora_grad_dy"] + b["lora_grad_x"]) / roof.bw) * 1e6
+    flops = 4.0 * M * N * K + 2.0 * M * r * (2 * K + 2 * N) + 2.0 * M * r * (K + N)
+    del g
+    return {"workload": spec.name.replace("gpt2_", "gpt2_outlier_"), "M": M, "K": K, "N": N, "r": r,
+            "act": "bf16", "outliers": qk.count, "step_us": step_us,
+            "tflops": flops / (step_us * 1e-6) / 1e12, "t_roof_us": t_roof,
+            "roof_frac": t_roof / step_us,
+            "note": "outlier-compensated uint8 kernel, rebuilt in shared memory before bf16 "
+                    "tensor cores in both directions"}
+
+
 def all_configs(dev, flush, roof, steps, only):
     from lora_fine_tuning_qlora_b200 import inputs
     specs = [inputs.single_fp32()] + inputs.gpt2_base() + inputs.gemma_2b(512) + \
@@ -439,6 +493,10 @@ def all_configs(dev, flush, roof, steps, only):
             merge = merge_entry(st, flush, roof, steps)
         out.append(ent)
         del st
+    for s in inputs.gpt2_base():
+        if only and only not in s.name.replace("gpt2_", "gpt2_outlier_"):
+            continue
+        out.append(outlier_entry(s, dev, flush, roof, steps, 3))
     return out, merge
 
 

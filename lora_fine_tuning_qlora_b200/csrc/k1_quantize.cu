@@ -467,8 +467,9 @@ cudaError_t launch_rows_rp(const T* X, const float* A, int M, int K, int r, int8
 // transposing warp butterfly (one shuffle per value and lane step) and,
 // across warps, one named barrier each.
 namespace staged {
-// consumer threads: row groups of TPR threads, 256 in all (eight warps: more
-// warps, at one chunk per thread, measured slower at 16384 x 4096)
+// consumer threads: row groups of TPR threads, 256 in all (eight warps: 512,
+// at one chunk per thread, measured slower at 16384 x 4096: the per-stage
+// reductions over twice the warps cost more than the extra warps hide)
 template <int RP>
 __host__ __device__ constexpr int max_cons() { return 256; }
 template <int TPR, int RP>
@@ -609,6 +610,7 @@ __global__ void __launch_bounds__(staged::cons<TPR, RP>() + 32, 1)
 
         // ---- sweep 1: abs-max of each row
         float amax[kRPG];
+        float inv[kRPG];  // 127 / amax (0 for a zero row)
 #pragma unroll
         for (int q = 0; q < kRPG; ++q) {
             __nv_bfloat162 m2 = __float2bfloat162_rn(0.f);
@@ -635,17 +637,30 @@ __global__ void __launch_bounds__(staged::cons<TPR, RP>() + 32, 1)
             if constexpr (W == 1) {
 #pragma unroll
                 for (int q = 0; q < kRPG; ++q) amax[q] = __shfl_sync(0xffffffffu, x, xreduce_lane<kRPG>(q));
+#pragma unroll
+                for (int q = 0; q < kRPG; ++q) inv[q] = amax[q] > 0.f ? __fdiv_rn(127.0f, amax[q]) : 0.f;
             } else {
-                if ((lane & (32 / kRPG - 1)) == 0) redA[(g * kRPG + xreduce_index<kRPG>(lane)) * W + w] = x;
+                constexpr int kLPR = 32 / kRPG;  // lanes holding one row's value
+                const int qr = xreduce_index<kRPG>(lane);
+                if ((lane & (kLPR - 1)) == 0) redA[(g * kRPG + qr) * W + w] = x;
                 if (!ok) abort_flag[g] = 1;
                 named_bar_sync(1 + g, TPR);
                 if (abort_flag[g]) break;
+                // the kLPR lanes of row qr share its W warp maxima, then every
+                // lane takes the four row maxima from one lane of each row
+                float mx = 0.f;
+#pragma unroll
+                for (int ww = lane & (kLPR - 1); ww < W; ww += kLPR)
+                    mx = fmaxf(mx, redA[(g * kRPG + qr) * W + ww]);
+#pragma unroll
+                for (int off = 1; off < kLPR; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+#pragma unroll
+                // one division per row, in the row's lanes
+                const float iv = mx > 0.f ? __fdiv_rn(127.0f, mx) : 0.f;
 #pragma unroll
                 for (int q = 0; q < kRPG; ++q) {
-                    float mx = redA[(g * kRPG + q) * W];
-#pragma unroll
-                    for (int ww = 1; ww < W; ++ww) mx = fmaxf(mx, redA[(g * kRPG + q) * W + ww]);
-                    amax[q] = mx;
+                    amax[q] = __shfl_sync(0xffffffffu, mx, xreduce_lane<kRPG>(q));
+                    inv[q] = __shfl_sync(0xffffffffu, iv, xreduce_lane<kRPG>(q));
                 }
             }
         }
@@ -659,7 +674,6 @@ __global__ void __launch_bounds__(staged::cons<TPR, RP>() + 32, 1)
             for (int j = 0; j < RP; ++j) xa[q][j] = 0ull;
 #pragma unroll
         for (int q = 0; q < kRPG; ++q) {
-            const float inv = amax[q] > 0.f ? __fdiv_rn(127.0f, amax[q]) : 0.f;
             const int m = m0 + q;
             int8_t* qrow = a.Xq + static_cast<size_t>(m) * K;
 #pragma unroll
@@ -669,7 +683,7 @@ __global__ void __launch_bounds__(staged::cons<TPR, RP>() + 32, 1)
                     const uint4 u = *reinterpret_cast<const uint4*>(gbase + static_cast<size_t>(q) * K * 2 + c * 16);
                     float f[8];
                     bf16x8_to_f(u, f);
-                    const uint2 cw = codes8(f, inv);
+                    const uint2 cw = codes8(f, inv[q]);
                     if (m < a.M) *reinterpret_cast<uint2*>(qrow + c * 8) = cw;
 #pragma unroll
                     for (int p = 0; p < 4; ++p) {
@@ -709,12 +723,18 @@ __global__ void __launch_bounds__(staged::cons<TPR, RP>() + 32, 1)
         } else {
             if ((lane & (32 / V - 1)) == 0) redX[(g * W + w) * V + idx] = x;
             named_bar_sync(1 + g, TPR);
-            if (t < V) {
-                float sum = redX[(g * W) * V + t];
+            if (t < 32) {
+                // the group's first warp: 32 / V lanes per value, each adding
+                // every (32 / V)-th warp's partial, then a shuffle
+                constexpr int kLPV = 32 / V;
+                const int vi = t / kLPV;
+                float sum = 0.f;
 #pragma unroll
-                for (int ww = 1; ww < W; ++ww) sum += redX[(g * W + ww) * V + t];
-                const int q = t / RP, j = t % RP;
-                if (m0 + q < a.M && j < a.r) a.xA[static_cast<size_t>(m0 + q) * a.r + j] = sum;
+                for (int ww = t % kLPV; ww < W; ww += kLPV) sum += redX[(g * W + ww) * V + vi];
+#pragma unroll
+                for (int off = 1; off < kLPV; off <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+                const int q = vi / RP, j = vi % RP;
+                if ((t % kLPV) == 0 && m0 + q < a.M && j < a.r) a.xA[static_cast<size_t>(m0 + q) * a.r + j] = sum;
             }
         }
     }

@@ -134,6 +134,34 @@ def test_zero_rows_and_exact_ties(q):
     assert_close(to_np(Y), f["y"], "bf16", "Y")
 
 
+@pytest.mark.parametrize("M,K,r", [(16384, 4096, 4), (5000, 4096, 3), (8192, 3072, 4),
+                                   (8200, 4096, 8), (4096, 768, 4), (12000, 2048, 2)])
+def test_quantize_input_large_shapes(q, M, K, r):
+    """a1 alone at the sizes where the staged input quantizer runs (rows
+    streamed through shared memory by bulk copies), every row: codes and
+    row scales bit-exact, xA within the bf16 tolerance.  Zero rows and a
+    ragged last stage included."""
+    rng = np.random.Generator(np.random.PCG64(M + K + r))
+    X = inputs.round_to_act(rng.standard_normal((M, K), dtype=np.float32), "bf16")
+    X[M // 2, :] = 0.0
+    X[M - 1, :] = 0.0
+    X[M - 1, K - 1] = 3.0
+    A = rng.uniform(-1 / 64, 1 / 64, (K, r)).astype(np.float32)
+    d = q.desc(K, 64, r, float(r), torch.bfloat16)
+    Xt = torch.from_numpy(X).to(torch.bfloat16).cuda()
+    At = torch.from_numpy(A).cuda()
+    Xq = torch.empty((M, K), dtype=torch.int8, device="cuda")
+    sx = torch.empty((M,), device="cuda")
+    xA = torch.empty((M, r), device="cuda")
+    q.qlora_quantize_input(d, M, Xt, At, Xq, sx, xA)
+    torch.cuda.synchronize()
+    assert q.qlora_device_status() == 0
+    xq_o, sx_o = oracle.quantize_rows(X)
+    np.testing.assert_array_equal(to_np(Xq), xq_o)
+    np.testing.assert_array_equal(to_np(sx).view(np.uint32), sx_o.view(np.uint32))
+    assert_close(to_np(xA), oracle.lora_down(X, A), "bf16", "xA")
+
+
 def test_empty_batch(q):
     spec = _edge_spec(1, 64, 32, 4)
     d = inputs.layer_inputs(spec)
