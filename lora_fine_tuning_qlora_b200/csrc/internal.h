@@ -99,6 +99,16 @@ bool gemm_dx_pair_applies(int M, int N, int K, int r);
 cudaError_t launch_gemm_dx_pair(const void* dY, const int8_t* Wq, const float* sw, int M, int N,
                                 int K, const DxEpilogue& ep, int* status, cudaStream_t s, bool w4);
 
+// Few tokens (M <= 64, rank <= 16, fewer large tiles than SMs): tokens on
+// the MMA's N, output channels on its M, the contraction split over a
+// cluster (small_m.cu).  int8 or packed int4 codes (w4) with a scale per
+// row; not the outlier-compensated kernels.
+bool small_m_applies(int M, int out_channels, int r);
+cudaError_t launch_gemm_i8_fwd_small(Act act, const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
+                                     const FwdEpilogue& ep, int* status, cudaStream_t s, bool w4);
+cudaError_t launch_gemm_dx_small(const void* dY, const int8_t* Wq, const float* sw, int M, int N, int K,
+                                 const DxEpilogue& ep, int* status, cudaStream_t s, bool w4);
+
 // ---------------------------------------------------------------- K4
 // The dY pass runs on the tensor cores for bf16 activations whose rows TMA
 // can describe (N a multiple of 8), in 128-column blocks; otherwise on CUDA

@@ -559,6 +559,7 @@ int fwd_split(int M, int N, int K) {
 
 cudaError_t launch_gemm_i8_fwd(Act act, const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
                                const FwdEpilogue& ep, int* status, cudaStream_t s, bool w4) {
+    if (small_m_applies(M, N, ep.r)) return launch_gemm_i8_fwd_small(act, Xq, Wq, M, N, K, ep, status, s, w4);
     if (!w4 && gemm_fwd_pair_applies(act, M, N, K, ep.r))
         return launch_gemm_i8_fwd_pair(Xq, Wq, M, N, K, ep, status, s);
     if (act == kBF16 && !w4 && ep.r <= 16) {

@@ -682,6 +682,8 @@ cudaError_t launch_gemm_dx(Act act, const void* dY, const int8_t* Wq, const floa
         return launch_k(kern, grid, dim3(256), 0, s, 1, static_cast<const float*>(dY), Wq, sw, M, N, K,
                         ep);
     }
+    if (mode != 2 && !ep.bias && small_m_applies(M, K, ep.r))
+        return launch_gemm_dx_small(dY, Wq, sw, M, N, K, ep, status, s, w4);
     if (gemm_dx_pair_applies(M, N, K, ep.r))
         return launch_gemm_dx_pair(dY, Wq, sw, M, N, K, ep, status, s, w4);
     // tile shape: the least estimated main-loop time, i.e. waves of

@@ -55,7 +55,10 @@ def test_single_fp32_layer(q):
                                      # tile's second CTA wholly outside) and ragged K
                                      (850, 4736, 640, 4), (1100, 4736, 192, 16),
                                      # forward on CTA pairs: ragged M, N
-                                     (1000, 1040, 4744, 8)])
+                                     (1000, 1040, 4744, 8),
+                                     # few tokens: tokens on the MMA's N, split-K clusters,
+                                     # ragged channels and contraction
+                                     (57, 1040, 200, 16), (64, 4096, 1000, 4), (9, 2048, 4096, 8)])
 def test_bf16_layer_tiles_and_ragged_tails(q, M, K, N, r):
     spec = inputs.LayerSpec("ragged", M=M, K=K, N=N, r=r, alpha=2.0 * r, act="bf16",
                             x_dist="normal", w_dist="glorot", a_dist="he_uniform", b_std=0.01,
@@ -369,7 +372,8 @@ def test_rank_pass_rows_setting(q, M, K, N, r):
 
 @pytest.mark.parametrize("M,K,N,r,act", [(200, 384, 264, 8, "bf16"), (96, 256, 10, 8, "bf16"),
                                           (64, 784, 128, 4, "f32"), (300, 2048, 264, 8, "bf16"),
-                                          (600, 8192, 256, 8, "bf16"), (2048, 512, 9216, 4, "bf16")])
+                                          (600, 8192, 256, 8, "bf16"), (2048, 512, 9216, 4, "bf16"),
+                                          (48, 1024, 768, 8, "bf16")])
 def test_fused_relu_entry_points(q, M, K, N, r, act):
     """qlora_gemm_forward_relu == qlora_relu(qlora_gemm_forward) and
     qlora_gemm_dx_relu == qlora_relu_backward(qlora_gemm_dx, X), bit for bit,
@@ -444,6 +448,8 @@ def test_int4_quantize_and_unpack_bit_exact(q, K, N):
 
 
 @pytest.mark.parametrize("M,K,N,r,act", [(1024, 1024, 1024, 8, "bf16"),   # 128x64 tiles
+                                          (40, 2048, 1000, 4, "bf16"),    # few tokens
+                                          (17, 1056, 4096, 8, "f32"),     # few tokens, fp32 outputs
                                           (333, 768, 2304, 4, "bf16"),
                                           (1000, 1312, 264, 8, "bf16"),   # 128x128 tiles
                                           (4096, 768, 768, 4, "bf16"),    # 256x128 tiles
