@@ -41,7 +41,7 @@ cudaError_t launch_gemm_i8_fwd(Act act, const int8_t* Xq, const int8_t* Wq, int 
 // outputs, rank <= 16, at least one wave of pair tiles.
 bool gemm_fwd_pair_applies(Act act, int M, int N, int K, int r);
 cudaError_t launch_gemm_i8_fwd_pair(const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
-                                    const FwdEpilogue& ep, int* status, cudaStream_t s);
+                                    const FwdEpilogue& ep, int* status, cudaStream_t s, bool w4);
 
 // ---------------------------------------------------------------- K3
 // Outlier-compensated int8 kernel as a GEMM operand (outlier.cu): uint8

@@ -41,7 +41,7 @@ template <bool W4>
 __host__ __device__ constexpr int k2_threads() { return kThreads + (W4 ? 32 * kUnpackWarps : 0); }
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory
 
-template <int BN, typename OutT, int RMAX, bool SPLIT = false>
+template <int BN, typename OutT, int RMAX, bool SPLIT = false, bool W4 = false>
 struct K2Cfg {
     static constexpr bool kLoraMMA = RMAX <= 16;
     static constexpr bool kSplit = sizeof(OutT) == 4;      // 3 x tf32 for fp32 outputs
@@ -59,11 +59,14 @@ struct K2Cfg {
     static constexpr int kFixed = kStgBytes + 2 * kBufBytes + kRedBytes + 512 + 1024;
     // k per stage: two 128-byte blocks (one 3-D TMA box per operand) where
     // two such stages fit, else one
-    static constexpr int kBlk = (kSmemLimit - kFixed) / ((kBM + BN) * 2 * kBlkK) >= 2 ? 2 : 1;
+    // (packed int4 kernels: the stage also holds the packed codes, BN x kBK/2)
+    static constexpr int kBlk =
+        (kSmemLimit - kFixed) / ((kBM + BN + (W4 ? BN / 2 : 0)) * 2 * kBlkK) >= 2 ? 2 : 1;
     static constexpr int kBK = kBlk * kBlkK;
     static constexpr int kABytes = kBM * kBK;
     static constexpr int kBBytes = BN * kBK;
-    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kPBytes = W4 ? BN * kBK / 2 : 0;
+    static constexpr int kStageBytes = kABytes + kBBytes + kPBytes;
     static constexpr int kStagesFit = (kSmemLimit - kFixed) / kStageBytes;
     static constexpr int STAGES = kStagesFit > 8 ? 8 : kStagesFit;
     static_assert(STAGES >= 2, "shared memory budget");
@@ -79,9 +82,10 @@ struct K2Cfg {
 };
 
 // W4: the kernel is packed int4 codes Wp [N, K/2] (two per byte, even k in
-// the low nibble) instead of int8 codes behind tmB; warps 10..13 expand each
-// stage's codes into the int8 tile the TMA would have written (128B swizzle,
-// K-major), and the MMA waits for them as well as for the Xq tile.
+// the low nibble) instead of int8 codes; tmB then maps Wp, and the TMA brings
+// each stage's packed tile ([BN rows][kBK/2 bytes], no swizzle) with the Xq
+// tile.  Warps 10..13 expand it into the int8 tile the TMA would have written
+// for int8 codes (128B swizzle, K-major), and the MMA waits for them as well.
 //
 // SPLIT: split-K for grids that would leave SMs idle.  The grid is tiles x S
 // (S = 2, 4 or 8) with clusters of the S CTAs of one tile (along y); CTA s
@@ -96,7 +100,7 @@ __global__ void __launch_bounds__(k2_threads<W4>(), 1)
     k2_gemm_i8_lora_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmB, int k3d, int M, int N, int K,
                            const uint8_t* __restrict__ Wp, FwdEpilogue ep, int* status) {
-    using C = K2Cfg<BN, OutT, RMAX, SPLIT>;
+    using C = K2Cfg<BN, OutT, RMAX, SPLIT, W4>;
     static_assert(!(SPLIT && W4), "split-K runs on int8 codes");
     constexpr int S = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -168,7 +172,9 @@ __global__ void __launch_bounds__(k2_threads<W4>(), 1)
                         break;
                     }
                     uint8_t* sa = smem + s * C::kStageBytes;
-                    mbar_arrive_expect_tx(&full[s], W4 ? C::kABytes : C::kStageBytes);
+                    mbar_arrive_expect_tx(&full[s], W4 ? C::kABytes + C::kPBytes : C::kStageBytes);
+                    if constexpr (W4)
+                        tma_load_2d(sa + C::kABytes + C::kBBytes, &tmB, &full[s], kb * (C::kBK / 2), n0);
                     // each operand's two k-blocks, consecutive in shared memory
                     if (k3d) {
                         tma_load_3d(sa, &tmA, &full[s], 0, m0, kb * C::kBlk);
@@ -258,38 +264,34 @@ __global__ void __launch_bounds__(k2_threads<W4>(), 1)
         // Stage g's Wq tile, as the TMA would have written it: k-block b of
         // row n at b * BN * 128 + n * 128, its 16-byte chunk c at position
         // c ^ (n % 8).  One packed 16-byte chunk (32 codes) gives int8 chunks
-        // 2p and 2p + 1 of a row; chunks outside the matrix are written as
-        // zeros.  The loads go out before the wait for the stage to be free.
+        // 2p and 2p + 1 of a row; outside the matrix the TMA's zero fill gives
+        // zero codes.  The stage's int8 area is free once its packed codes
+        // have landed: the producer refills a stage only after its MMAs.
         const int ut = (warp - 2 - kEpiWarps) * 32 + lane;
         constexpr int kPerRow = C::kBlk * 4;  // packed chunks of one row per stage
         constexpr int kItems = BN * kPerRow;
         constexpr int kPer = kItems / (32 * kUnpackWarps);
         static_assert(kItems % (32 * kUnpackWarps) == 0, "packed chunks per unpack thread");
-        const size_t row_bytes = static_cast<size_t>(K) / 2;
+        (void)Wp;
         int g = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-            const int n0 = (t % num_n) * BN;
             for (int kb = kb0; kb < kb1; ++kb, ++g) {
                 const int s = g % S;
-                uint4 raw[kPer];
-                uint32_t inb = 0;
-#pragma unroll
-                for (int i = 0; i < kPer; ++i) {
-                    const int e = ut + i * 32 * kUnpackWarps;
-                    const int n = n0 + e / kPerRow;
-                    const int rem = e % kPerRow;
-                    const int k = kb * C::kBK + (rem / 4) * kBlkK + (rem % 4) * 32;
-                    if (n < N && k < K) inb |= 1u << i;
-                    const int nc = n < N ? n : N - 1;
-                    const int kc = k < K ? k : K - 32;
-                    raw[i] = __ldg(reinterpret_cast<const uint4*>(Wp + static_cast<size_t>(nc) * row_bytes + kc / 2));
-                }
-                if (g >= S && !__all_sync(0xffffffffu, mbar_wait(&empty[s], ((g / S) - 1) & 1, status))) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (g / S) & 1, status))) {
                     ok = false;
                     break;
                 }
                 uint8_t* wb = smem + s * C::kStageBytes + C::kABytes;
+                const uint8_t* pk = wb + C::kBBytes;
+                uint4 raw[kPer];
+#pragma unroll
+                for (int i = 0; i < kPer; ++i) {
+                    const int e = ut + i * 32 * kUnpackWarps;
+                    const int n = e / kPerRow;
+                    const int rem = e % kPerRow;
+                    raw[i] = *reinterpret_cast<const uint4*>(pk + n * (C::kBK / 2) + (rem / 4) * 64 + (rem % 4) * 16);
+                }
 #pragma unroll
                 for (int i = 0; i < kPer; ++i) {
                     const int e = ut + i * 32 * kUnpackWarps;
@@ -298,7 +300,6 @@ __global__ void __launch_bounds__(k2_threads<W4>(), 1)
                     const int p = rem % 4;
                     uint4 lo, hi;
                     unpack_int4x32(raw[i], lo, hi);
-                    if (!((inb >> i) & 1u)) lo = hi = make_uint4(0u, 0u, 0u, 0u);
                     uint8_t* row = wb + (rem / 4) * (BN * kBlkK) + n * kBlkK;
                     *reinterpret_cast<uint4*>(row + (((2 * p) ^ (n & 7)) << 4)) = lo;
                     *reinterpret_cast<uint4*>(row + (((2 * p + 1) ^ (n & 7)) << 4)) = hi;
@@ -495,13 +496,14 @@ __global__ void __launch_bounds__(k2_threads<W4>(), 1)
 template <int BN, typename OutT, int RMAX, bool W4, bool SPLIT = false>
 cudaError_t launch_cfg(const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
                        const FwdEpilogue& ep, int* status, cudaStream_t s, int nsplit = 1) {
-    using C = K2Cfg<BN, OutT, RMAX, SPLIT>;
+    using C = K2Cfg<BN, OutT, RMAX, SPLIT, W4>;
     // Xq and Wq as [row][k-block of 128][128] (one 3-D box per operand and
     // stage) when K splits into whole blocks, else one 2-D box per block
     CUtensorMap ta, tb;
     const int k3d = (K % kBlkK) == 0 ? 1 : 0;
     bool ok;
-    // (packed int4 kernels: no map for the codes, which the unpack warps load)
+    // (packed int4 kernels: tmB maps the packed codes [N, K/2], one box of
+    // [BN rows][kBK/2 bytes] per stage)
     if (k3d)
         ok = make_tmap_3d_blocks(&ta, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, kBlkK, kBM, C::kBlk) &&
              (W4 || make_tmap_3d_blocks(&tb, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, kBlkK, BN, C::kBlk));
@@ -510,8 +512,10 @@ cudaError_t launch_cfg(const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
                           CU_TENSOR_MAP_SWIZZLE_128B) &&
              (W4 || make_tmap_2d(&tb, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, BN, kBlkK,
                                  CU_TENSOR_MAP_SWIZZLE_128B));
+    if (W4)
+        ok = ok && make_tmap_2d(&tb, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, K / 2, BN, C::kBK / 2,
+                                CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return cudaErrorInvalidValue;
-    if (W4) tb = ta;  // unused
     auto kern = k2_gemm_i8_lora_kernel<BN, OutT, RMAX, W4, SPLIT>;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), C::kTotal);
     if (e != cudaSuccess) return e;
@@ -560,8 +564,8 @@ int fwd_split(int M, int N, int K) {
 cudaError_t launch_gemm_i8_fwd(Act act, const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
                                const FwdEpilogue& ep, int* status, cudaStream_t s, bool w4) {
     if (small_m_applies(M, N, ep.r)) return launch_gemm_i8_fwd_small(act, Xq, Wq, M, N, K, ep, status, s, w4);
-    if (!w4 && gemm_fwd_pair_applies(act, M, N, K, ep.r))
-        return launch_gemm_i8_fwd_pair(Xq, Wq, M, N, K, ep, status, s);
+    if (gemm_fwd_pair_applies(act, M, N, K, ep.r))
+        return launch_gemm_i8_fwd_pair(Xq, Wq, M, N, K, ep, status, s, w4);
     if (act == kBF16 && !w4 && ep.r <= 16) {
         const int sp = fwd_split(M, N, K);
         if (sp > 1) {

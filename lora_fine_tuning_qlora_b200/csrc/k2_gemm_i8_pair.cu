@@ -23,6 +23,13 @@
 // epilogue warp of both CTAs (CTA-scope release).  Every wait is bounded.
 // The epilogue applies both scales, the bias and the rank-r term on CUDA
 // cores (fp32), from per-tile tables of sw, bias and B.
+//
+// W4 (packed int4 codes Wp [N, K/2]): each CTA's TMA brings its stage's
+// packed tile ([128 rows][64 bytes], no swizzle) onto a barrier of its own
+// (pfull), warps 6..9 expand it into the int8 tile the TMA would have written
+// (16-byte chunk c of row n at c ^ (n % 8)) and arrive on CTA 0's wready
+// (CTA-scope release: the tile stays in the writer's shared memory, published
+// to the tensor cores by a proxy fence); the MMA waits for both CTAs' tiles.
 #include "internal.h"
 #include "ptx.cuh"
 #include "tile_epilogue.cuh"
@@ -35,14 +42,17 @@ constexpr int kQM = 128;             // rows per CTA (256 per pair)
 constexpr int kQN = 256;             // output columns per pair tile (128 of Wq per CTA)
 constexpr int kQK = 128;             // int8 k per stage: one 128-byte swizzle row
 constexpr int kQEpi = 4;             // epilogue warps
-constexpr int kQThreads = 32 * (2 + kQEpi);
+constexpr int kQUnpack = 4;          // W4: warps that expand the packed codes
+template <bool W4>
+__host__ __device__ constexpr int q_threads() { return 32 * (2 + kQEpi + (W4 ? kQUnpack : 0)); }
 constexpr int kQSmemLimit = 232448;
 
-template <int RP>
+template <int RP, bool W4>
 struct PairFwdCfg {
     static constexpr int kABytes = kQM * kQK;             // Xq rows of this CTA: 16 KB
     static constexpr int kBBytes = (kQN / 2) * kQK;       // Wq rows of this CTA: 16 KB
-    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kPBytes = W4 ? (kQN / 2) * kQK / 2 : 0;  // packed codes: 8 KB
+    static constexpr int kStageBytes = kABytes + kBBytes + kPBytes;
     static constexpr int kStgBytes = kQEpi * 32 * stage_pitch<__nv_bfloat16>();
     static constexpr int kTabBytes = kQN * (RP + 2) * 4;  // B rows, sw, bias of the tile's columns
     static constexpr int kFixed = kStgBytes + kTabBytes + 512 + 1024;
@@ -53,16 +63,17 @@ struct PairFwdCfg {
     static constexpr int kTabOff = kStgOff + kStgBytes;
     static constexpr int kBarOff = kTabOff + kTabBytes;
     static constexpr int kTotal = kBarOff + 512 + 1024;
+    static_assert(6 * 8 * 4 + 8 * 4 <= 512, "barrier area");
     static constexpr uint32_t kAccCols = kQN;             // int32 accumulator: 256 columns
     static constexpr uint32_t kTmemCols = 2 * kAccCols;   // two buffers: all 512 columns
 };
 
-template <int RP>
-__global__ void __launch_bounds__(kQThreads, 1)
+template <int RP, bool W4>
+__global__ void __launch_bounds__(q_threads<W4>(), 1)
     k2_gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmB, int M, int N, int K,
                            FwdEpilogue ep, int* status) {
-    using C = PairFwdCfg<RP>;
+    using C = PairFwdCfg<RP, W4>;
     constexpr int S = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -71,7 +82,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
     uint64_t* empty = full + S;                                       // [S]
     uint64_t* tfull = empty + S;                                      // [2]
     uint64_t* tempty = tfull + 2;                                     // [2] (CTA 0)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+    uint64_t* pfull = tempty + 2;                                     // [S] W4: packed tile landed
+    uint64_t* wready = pfull + S;                                     // [S] W4 (CTA 0): both tiles expanded
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wready + S);
     float* sB = reinterpret_cast<float*>(smem + C::kTabOff);          // [256][RP]
     float* sSw = sB + kQN * RP;                                        // [256]
     float* sBias = sSw + kQN;                                          // [256]
@@ -95,6 +108,11 @@ __global__ void __launch_bounds__(kQThreads, 1)
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], 2 * kQEpi);
         }
+        if constexpr (W4)
+            for (int s = 0; s < S; ++s) {
+                mbar_init(&pfull[s], 1);
+                mbar_init(&wready[s], 2 * kQUnpack);
+            }
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -128,7 +146,17 @@ __global__ void __launch_bounds__(kQThreads, 1)
                         break;
                     }
                     uint8_t* sa = smem + s * C::kStageBytes;
-                    if (rank == 0) {
+                    if constexpr (W4) {
+                        // Xq of both CTAs on CTA 0's full; each CTA's packed codes on its own pfull
+                        if (rank == 0) {
+                            mbar_arrive_expect_tx(&full[s], 2 * C::kABytes);
+                            tma_load_2d(sa, &tmA, &full[s], kb * kQK, m0);
+                        } else {
+                            tma_load_2d_pair(sa, &tmA, full0 + 8u * static_cast<uint32_t>(s), kb * kQK, m0);
+                        }
+                        mbar_arrive_expect_tx(&pfull[s], C::kPBytes);
+                        tma_load_2d(sa + C::kABytes + C::kBBytes, &tmB, &pfull[s], kb * (kQK / 2), n0);
+                    } else if (rank == 0) {
                         mbar_arrive_expect_tx(&full[s], 2 * C::kStageBytes);
                         tma_load_2d(sa, &tmA, &full[s], kb * kQK, m0);
                         tma_load_2d(sa + C::kABytes, &tmB, &full[s], kb * kQK, n0);
@@ -155,7 +183,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
                 const uint32_t dacc = tmem + ab * C::kAccCols;
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
                     const int s = g % S;
-                    if (!mbar_wait(&full[s], (g / S) & 1, status)) {
+                    if (!mbar_wait(&full[s], (g / S) & 1, status) ||
+                        (W4 && !mbar_wait(&wready[s], (g / S) & 1, status))) {
                         ok = false;
                         break;
                     }
@@ -171,6 +200,46 @@ __global__ void __launch_bounds__(kQThreads, 1)
                     mma_commit_pair(&empty[s], 0x3);
                 }
                 if (ok) mma_commit_pair(&tfull[ab], 0x3);
+            }
+        }
+        __syncwarp();
+    } else if (W4 && warp >= 2 + kQEpi) {
+        // ------------------------------------------------------ int4 expand (W4)
+        const int t = threadIdx.x - 32 * (2 + kQEpi);  // 0 .. 127
+        const uint32_t wready0 = dsmem_addr(wready, 0);
+        int g = 0;
+        bool ok = true;
+        for (int tt = pair; tt < tiles && ok; tt += npairs) {
+            for (int kb = 0; kb < nkb; ++kb, ++g) {
+                const int s = g % S;
+                if (!__all_sync(0xffffffffu, mbar_wait(&pfull[s], (g / S) & 1, status))) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* wb = smem + s * C::kStageBytes + C::kABytes;
+                const uint8_t* pk = wb + C::kBBytes;
+                uint4 raw[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int e = t + u * 128;
+                    raw[u] = *reinterpret_cast<const uint4*>(pk + (e >> 2) * 64 + (e & 3) * 16);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int e = t + u * 128;
+                    const int n = e >> 2, p = e & 3;
+                    uint4 lo, hi;
+                    unpack_int4x32(raw[u], lo, hi);
+                    uint8_t* row = wb + n * kQK;
+                    *reinterpret_cast<uint4*>(row + (((2 * p) ^ (n & 7)) << 4)) = lo;
+                    *reinterpret_cast<uint4*>(row + (((2 * p + 1) ^ (n & 7)) << 4)) = hi;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    if (rank == 0) mbar_arrive(&wready[s]);
+                    else mbar_arrive_remote_cta(wready0 + 8u * static_cast<uint32_t>(s));
+                }
             }
         }
         __syncwarp();
@@ -267,22 +336,24 @@ __global__ void __launch_bounds__(kQThreads, 1)
     }
 }
 
-template <int RP>
+template <int RP, bool W4>
 cudaError_t launch_fwd_pair_t(const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
                               const FwdEpilogue& ep, int* status, cudaStream_t s) {
-    using C = PairFwdCfg<RP>;
-    auto kern = k2_gemm_i8_pair_kernel<RP>;
+    using C = PairFwdCfg<RP, W4>;
+    auto kern = k2_gemm_i8_pair_kernel<RP, W4>;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), C::kTotal);
     if (e != cudaSuccess) return e;
     CUtensorMap ta, tb;
-    if (!make_tmap_2d(&ta, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, K, kQM, kQK,
-                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap_2d(&tb, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, kQN / 2, kQK,
-                      CU_TENSOR_MAP_SWIZZLE_128B))
+    const bool bok = W4 ? make_tmap_2d(&tb, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, K / 2,
+                                       kQN / 2, kQK / 2, CU_TENSOR_MAP_SWIZZLE_NONE)
+                        : make_tmap_2d(&tb, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, kQN / 2, kQK,
+                                       CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!bok || !make_tmap_2d(&ta, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, K, kQM, kQK,
+                              CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     const int tiles = ((M + 2 * kQM - 1) / (2 * kQM)) * ((N + kQN - 1) / kQN);
     const int pairs = tiles < sm_count() / 2 ? tiles : sm_count() / 2;
-    return launch_kx(kern, dim3(2 * pairs), dim3(kQThreads), C::kTotal, s, 2, ta, tb, M, N, K, ep,
+    return launch_kx(kern, dim3(2 * pairs), dim3(q_threads<W4>()), C::kTotal, s, 2, ta, tb, M, N, K, ep,
                      status);
 }
 
@@ -295,10 +366,15 @@ bool gemm_fwd_pair_applies(Act act, int M, int N, int K, int r) {
 }
 
 cudaError_t launch_gemm_i8_fwd_pair(const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
-                                    const FwdEpilogue& ep, int* status, cudaStream_t s) {
-    if (ep.r <= 4) return launch_fwd_pair_t<4>(Xq, Wq, M, N, K, ep, status, s);
-    if (ep.r <= 8) return launch_fwd_pair_t<8>(Xq, Wq, M, N, K, ep, status, s);
-    return launch_fwd_pair_t<16>(Xq, Wq, M, N, K, ep, status, s);
+                                    const FwdEpilogue& ep, int* status, cudaStream_t s, bool w4) {
+    if (ep.r <= 4)
+        return w4 ? launch_fwd_pair_t<4, true>(Xq, Wq, M, N, K, ep, status, s)
+                  : launch_fwd_pair_t<4, false>(Xq, Wq, M, N, K, ep, status, s);
+    if (ep.r <= 8)
+        return w4 ? launch_fwd_pair_t<8, true>(Xq, Wq, M, N, K, ep, status, s)
+                  : launch_fwd_pair_t<8, false>(Xq, Wq, M, N, K, ep, status, s);
+    return w4 ? launch_fwd_pair_t<16, true>(Xq, Wq, M, N, K, ep, status, s)
+              : launch_fwd_pair_t<16, false>(Xq, Wq, M, N, K, ep, status, s);
 }
 
 }  // namespace qlora

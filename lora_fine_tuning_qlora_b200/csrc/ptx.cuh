@@ -584,8 +584,10 @@ __device__ __forceinline__ void unpack_int4x32(const uint4 raw, uint4& lo, uint4
     uint32_t o[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint32_t ev = __vsub4((w[i] & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);
-        const uint32_t od = __vsub4(((w[i] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);
+        // per byte, a nibble n becomes the signed byte n - 16 [n >= 8] as
+        // ((n ^ 8) + 0x78) ^ 0x80: the add never carries out of its byte
+        const uint32_t ev = (((w[i] & 0x0F0F0F0Fu) ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
+        const uint32_t od = ((((w[i] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
         o[2 * i] = __byte_perm(ev, od, 0x5140);
         o[2 * i + 1] = __byte_perm(ev, od, 0x7362);
     }

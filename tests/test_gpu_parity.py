@@ -449,6 +449,8 @@ def test_int4_quantize_and_unpack_bit_exact(q, K, N):
 
 @pytest.mark.parametrize("M,K,N,r,act", [(1024, 1024, 1024, 8, "bf16"),   # 128x64 tiles
                                           (40, 2048, 1000, 4, "bf16"),    # few tokens
+                                          (2304, 2048, 4096, 4, "bf16"),  # forward on CTA pairs
+                                          (2100, 1056, 2600, 8, "bf16"),  # CTA pairs, ragged M, N, k-block
                                           (17, 1056, 4096, 8, "f32"),     # few tokens, fp32 outputs
                                           (333, 768, 2304, 4, "bf16"),
                                           (1000, 1312, 264, 8, "bf16"),   # 128x128 tiles
