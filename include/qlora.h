@@ -423,6 +423,19 @@ int qlora_merge(const qlora_layer_desc* d, const int8_t* Wq, const float* sw,
 int qlora_relu(void* Y, size_t n, qlora_dtype dtype, void* stream);
 int qlora_relu_backward(void* dY, const void* Y, size_t n, qlora_dtype dtype, void* stream);
 
+/*
+ * Axis permutation of a row-major tensor (EinsumDense layouts: "Introduce
+ * float8 training", the speed test's "abcde,aebf->adbcf"; an equation whose
+ * operands are not a plain reshape of a Dense layer's is brought to
+ * [batch, kept, contracted] order before the layer and back after it).
+ * src has `ndim` (1..8) axes of extents shape[]; dst axis d is src axis
+ * perm[d], i.e. dst[i_0, .., i_{ndim-1}] = src[j] with j_{perm[d]} = i_d.
+ * elem_bytes is 1, 2, 4 or 8; both buffers are device memory aligned to it
+ * and must not overlap.  Bit-exact (a copy).
+ */
+int qlora_permute(const void* src, void* dst, int ndim, const int64_t* shape, const int* perm,
+                  int elem_bytes, void* stream);
+
 /* Message for the last non-OK status returned on the calling thread. */
 const char* qlora_last_error(void);
 

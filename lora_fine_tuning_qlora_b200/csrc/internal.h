@@ -109,6 +109,12 @@ cudaError_t launch_gemm_i8_fwd_small(Act act, const int8_t* Xq, const int8_t* Wq
 cudaError_t launch_gemm_dx_small(const void* dY, const int8_t* Wq, const float* sw, int M, int N, int K,
                                  const DxEpilogue& ep, int* status, cudaStream_t s, bool w4);
 
+// Axis permutation of a row-major tensor of up to kMaxPermAxes axes
+// (permute.cu): dst axis d is src axis perm[d].
+constexpr int kMaxPermAxes = 8;
+cudaError_t launch_permute(const void* src, void* dst, int nd, const long long* shape, const int* perm,
+                           int elem_bytes, cudaStream_t s);
+
 // ---------------------------------------------------------------- K4
 // The dY pass runs on the tensor cores for bf16 activations whose rows TMA
 // can describe (N a multiple of 8), in 128-column blocks; otherwise on CUDA

@@ -784,6 +784,28 @@ int qlora_outlier_backward(const qlora_layer_desc* d, int M, const void* X, cons
     return qlora_lora_grad_x(d, M, X, dA, workspace, workspace_bytes, stream);
 }
 
+int qlora_permute(const void* src, void* dst, int ndim, const int64_t* shape, const int* perm,
+                  int elem_bytes, void* stream) {
+    QL_REQUIRE(src && dst && shape && perm, QLORA_EINVAL, "NULL pointer argument");
+    QL_REQUIRE(ndim >= 1 && ndim <= kMaxPermAxes, QLORA_ESHAPE, "ndim must be in [1, 8]");
+    QL_REQUIRE(elem_bytes == 1 || elem_bytes == 2 || elem_bytes == 4 || elem_bytes == 8, QLORA_EINVAL,
+               "elem_bytes must be 1, 2, 4 or 8");
+    QL_REQUIRE(aligned(src, elem_bytes) && aligned(dst, elem_bytes), QLORA_EALIGN,
+               "src and dst must be aligned to the element size");
+    QL_REQUIRE(src != dst, QLORA_EINVAL, "src and dst must not alias");
+    long long sh[kMaxPermAxes];
+    bool seen[kMaxPermAxes] = {false};
+    for (int d = 0; d < ndim; ++d) {
+        QL_REQUIRE(shape[d] >= 0, QLORA_ESHAPE, "negative extent");
+        QL_REQUIRE(perm[d] >= 0 && perm[d] < ndim && !seen[perm[d]], QLORA_EINVAL,
+                   "perm must be a permutation of 0 .. ndim-1");
+        seen[perm[d]] = true;
+        sh[d] = static_cast<long long>(shape[d]);
+    }
+    return cuda_status(launch_permute(src, dst, ndim, sh, perm, elem_bytes, static_cast<cudaStream_t>(stream)),
+                       "permute launch");
+}
+
 int qlora_selftest_wait_timeout(unsigned int limit_us, void* stream) {
     QL_REQUIRE(limit_us >= 1 && limit_us <= 2000000, QLORA_EINVAL, "limit_us must be in [1, 2e6]");
     int* status = status_ptr();

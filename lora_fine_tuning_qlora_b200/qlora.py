@@ -35,7 +35,7 @@ EXPORTED = ("qlora_quantize_weight", "qlora_workspace_bytes", "qlora_forward",
             "qlora_set_rank_pass_rows", "qlora_quantize_weight_int4", "qlora_unpack_int4",
             "qlora_gemm_dx_int4", "qlora_merge_int4", "qlora_gemm_forward_int4",
             "qlora_outlier_cap", "qlora_outlier_workspace_bytes", "qlora_outlier_quantize",
-            "qlora_outlier_forward", "qlora_outlier_backward")
+            "qlora_outlier_forward", "qlora_outlier_backward", "qlora_permute")
 
 
 class QLoraError(RuntimeError):
@@ -124,6 +124,8 @@ def _load():
     lib.qlora_outlier_backward.argtypes = [D, I, P, P, OK, P, P, P, P, P, P, P, P, Z, P]
     for f in (lib.qlora_outlier_quantize, lib.qlora_outlier_forward, lib.qlora_outlier_backward):
         f.restype = I
+    lib.qlora_permute.argtypes = [P, P, I, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int), I, P]
+    lib.qlora_permute.restype = I
     lib.qlora_set_rank_pass_rows.argtypes = [I]
     lib.qlora_set_rank_pass_rows.restype = I
     lib.qlora_selftest_wait_timeout.argtypes = [ctypes.c_uint, P]
@@ -402,6 +404,25 @@ def qlora_outlier_backward(d: LayerDesc, M: int, X, dY, q: OutlierKernel, A, B, 
     _check(_lib.qlora_outlier_backward(ctypes.byref(d), int(M), _ptr(X), _ptr(dY), ctypes.byref(st),
                                        _ptr(A), _ptr(B), _ptr(xA), _ptr(dX), _ptr(dA), _ptr(dB),
                                        _ptr(dbias), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def qlora_permute(src: torch.Tensor, perm, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """dst = src with its axes permuted (dst axis d is src axis perm[d]), by
+    the library's kernel; returns dst (contiguous)."""
+    perm = [int(p) for p in perm]
+    nd = src.dim()
+    if sorted(perm) != list(range(nd)):
+        raise ValueError("perm must be a permutation of 0 .. %d" % (nd - 1))
+    shape = [src.shape[p] for p in perm]
+    dst = out if out is not None else torch.empty(shape, dtype=src.dtype, device=src.device)
+    if tuple(dst.shape) != tuple(shape) or dst.dtype != src.dtype:
+        raise ValueError("out has the wrong shape or dtype")
+    if src.numel() == 0:
+        return dst
+    sh = (ctypes.c_int64 * nd)(*src.shape)
+    pm = (ctypes.c_int * nd)(*perm)
+    _check(_lib.qlora_permute(_ptr(src), _ptr(dst), nd, sh, pm, src.element_size(), _stream(stream)))
+    return dst
 
 
 def qlora_set_rank_pass_rows(rows: int) -> int:
