@@ -32,9 +32,14 @@ What each routine follows (page title, section):
     keras-llm-light, "Simplified Int4Variable quantization" (two int4 values
     per int8 byte) and the 4-bit thread; the readings are in the C file.
 
+  * float8 (submodule ``oracle.float8``, numpy) -- the float8 training
+    recipe, "Introduce float8 training" (Keras PR 19488): E4M3 / E5M2
+    codes, delayed scaling from an amax history, the float8 Dense layer's
+    forward and backward; its readings are in the submodule's header.
+
 Pins: every routine here is checked by ``tests/test_oracle_pins.py`` against
 closed forms, brute force, finite differences and printed values (see
-``tests/golden/``).
+``tests/golden/``); the float8 submodule by ``tests/test_oracle_float8.py``.
 """
 from __future__ import annotations
 
