@@ -436,6 +436,48 @@ int qlora_relu_backward(void* dY, const void* Y, size_t n, qlora_dtype dtype, vo
 int qlora_permute(const void* src, void* dst, int ndim, const int64_t* shape, const int* perm,
                   int elem_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * The float8 training recipe ("Introduce float8 training", Keras PR 19488:
+ * quantization mode "float8", per-tensor scale and amax_history updated
+ * every step, the output-gradient scale, float8 matmuls on float8 tensor
+ * cores).  The page gives no formula; the library's reading:
+ *   formats   inputs and kernel E4M3 (largest finite 448), the output
+ *             gradient E5M2 (largest finite 57344); codes as uint8
+ *   quantize  q = fp8(satfinite(fl32(T / s))), round to nearest, ties to
+ *             even, s the scale stored by the previous step (delayed
+ *             scaling)
+ *   state     after quantizing, s' = fl32(h / fp8_max) with h the largest
+ *             entry of the amax history before this step (s' = s when h is
+ *             0 or not finite), and the history becomes
+ *             [amax(|T|), H[0], .., H[L-2]] (newest first, oldest dropped)
+ *   layer     Y = (Xq Wq) s_x s_w + bias, dX = (dYq Wq^T) s_g s_w,
+ *             dW = (Xq^T dYq) s_x s_g, dbias = column sums of dY
+ * ------------------------------------------------------------------------ */
+typedef enum { QLORA_FP8_E4M3 = 0, QLORA_FP8_E5M2 = 1 } qlora_fp8_format;
+
+/* Scratch of qlora_fp8_quantize (one word; 256 for alignment). */
+#define QLORA_FP8_WORKSPACE_BYTES 256
+
+/* Quantizes T [rows, cols] (dtype) with the scale *scale_in into q [rows,
+ * cols] and, if qt is not NULL, its transpose qt [cols, rows] (the K-major
+ * operand of the backward GEMMs), then writes the next scale to *scale_out
+ * and updates amax_history [history_len] in place, as above.  scale_in,
+ * scale_out and amax_history are device memory; scale_out must not alias
+ * scale_in (keep two and swap them every step).  Codes, scale and history
+ * are bit-exact with the reading above. */
+int qlora_fp8_quantize(const void* T, int rows, int cols, qlora_dtype dtype, qlora_fp8_format fmt,
+                       const float* scale_in, float* scale_out, float* amax_history, int history_len,
+                       uint8_t* q, uint8_t* qt, void* workspace, size_t workspace_bytes, void* stream);
+
+/* C [M,N] = (A B^T) * (*scale_a) * (*scale_b) (+ bias[n]), A [M,K] and
+ * B [N,K] float8 codes (both K-major, K a multiple of 16), products on
+ * tcgen05.mma.kind::f8f6f4 with fp32 accumulation; C in c_dtype (bf16
+ * rounded to nearest even).  bias may be NULL; scales are device pointers.
+ * A, B and C 16-byte aligned. */
+int qlora_fp8_gemm(const uint8_t* A, qlora_fp8_format fmt_a, const uint8_t* B, qlora_fp8_format fmt_b,
+                   int M, int N, int K, const float* scale_a, const float* scale_b, const float* bias,
+                   void* C, qlora_dtype c_dtype, void* stream);
+
 /* Message for the last non-OK status returned on the calling thread. */
 const char* qlora_last_error(void);
 

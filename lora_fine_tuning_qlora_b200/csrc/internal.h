@@ -115,6 +115,20 @@ constexpr int kMaxPermAxes = 8;
 cudaError_t launch_permute(const void* src, void* dst, int nd, const long long* shape, const int* perm,
                            int elem_bytes, cudaStream_t s);
 
+// The float8 recipe (fp8.cu).  Formats of the codes:
+constexpr int kFp8E4M3 = 0;
+constexpr int kFp8E5M2 = 1;
+// Codes of T [R, Cc] with the stored scale *scale_in (row-major q and, if
+// qt != null, transposed qt [Cc, R]); then *scale_out and the history hist
+// [L] of delayed scaling.  amax_word: one word of device scratch.
+cudaError_t launch_fp8_quantize(Act act, const void* T, int R, int Cc, const float* scale_in, float* scale_out,
+                                float* hist, int L, int fmt, uint8_t* q, uint8_t* qt, unsigned int* amax_word,
+                                cudaStream_t s);
+// C [M,N] = (A [M,K] B [N,K]^T) * sa * sb (+ bias [N]); K-major fp8 codes.
+cudaError_t launch_fp8_gemm(const uint8_t* A, int afmt, const uint8_t* B, int bfmt, int M, int N, int K,
+                            const float* sa, const float* sb, const float* bias, void* C, Act out, int* status,
+                            cudaStream_t s);
+
 // ---------------------------------------------------------------- K4
 // The dY pass runs on the tensor cores for bf16 activations whose rows TMA
 // can describe (N a multiple of 8), in 128-column blocks; otherwise on CUDA

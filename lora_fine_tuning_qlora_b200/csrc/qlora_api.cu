@@ -806,6 +806,55 @@ int qlora_permute(const void* src, void* dst, int ndim, const int64_t* shape, co
                        "permute launch");
 }
 
+// ---------------------------------------------------------------------------
+// the float8 recipe
+// ---------------------------------------------------------------------------
+int qlora_fp8_quantize(const void* T, int rows, int cols, qlora_dtype dtype, qlora_fp8_format fmt,
+                       const float* scale_in, float* scale_out, float* amax_history, int history_len,
+                       uint8_t* q, uint8_t* qt, void* workspace, size_t workspace_bytes, void* stream) {
+    QL_REQUIRE(T && scale_in && scale_out && amax_history && q && workspace, QLORA_EINVAL,
+               "NULL pointer argument");
+    QL_REQUIRE(rows >= 1 && cols >= 1 && history_len >= 1, QLORA_ESHAPE,
+               "rows, cols and history_len must be >= 1");
+    QL_REQUIRE(static_cast<long long>(rows) * cols < (1LL << 40), QLORA_ESHAPE, "tensor too large");
+    QL_REQUIRE(dtype == QLORA_F32 || dtype == QLORA_BF16, QLORA_EINVAL, "unknown dtype");
+    QL_REQUIRE(fmt == QLORA_FP8_E4M3 || fmt == QLORA_FP8_E5M2, QLORA_EINVAL, "unknown float8 format");
+    QL_REQUIRE(scale_out != scale_in, QLORA_EINVAL, "scale_out must not alias scale_in");
+    QL_REQUIRE(aligned(T, dtype == QLORA_BF16 ? 2 : 4) && aligned(scale_in, 4) && aligned(scale_out, 4) &&
+                   aligned(amax_history, 4) && aligned(workspace, 4),
+               QLORA_EALIGN, "misaligned pointer");
+    QL_REQUIRE(workspace_bytes >= QLORA_FP8_WORKSPACE_BYTES, QLORA_EINVAL, "workspace too small");
+    return cuda_status(launch_fp8_quantize(dtype == QLORA_BF16 ? kBF16 : kF32, T, rows, cols, scale_in,
+                                           scale_out, amax_history, history_len,
+                                           fmt == QLORA_FP8_E4M3 ? kFp8E4M3 : kFp8E5M2, q, qt,
+                                           static_cast<unsigned int*>(workspace),
+                                           static_cast<cudaStream_t>(stream)),
+                       "float8 quantizer launch");
+}
+
+int qlora_fp8_gemm(const uint8_t* A, qlora_fp8_format fmt_a, const uint8_t* B, qlora_fp8_format fmt_b,
+                   int M, int N, int K, const float* scale_a, const float* scale_b, const float* bias,
+                   void* C, qlora_dtype c_dtype, void* stream) {
+    QL_REQUIRE(A && B && scale_a && scale_b && C, QLORA_EINVAL, "NULL pointer argument");
+    QL_REQUIRE(M >= 1 && N >= 1 && K >= 1, QLORA_ESHAPE, "M, N and K must be >= 1");
+    QL_REQUIRE(K % 16 == 0, QLORA_EUNSUPPORTED, "K must be a multiple of 16 (16-byte rows of codes)");
+    QL_REQUIRE((fmt_a == QLORA_FP8_E4M3 || fmt_a == QLORA_FP8_E5M2) &&
+                   (fmt_b == QLORA_FP8_E4M3 || fmt_b == QLORA_FP8_E5M2),
+               QLORA_EINVAL, "unknown float8 format");
+    QL_REQUIRE(c_dtype == QLORA_F32 || c_dtype == QLORA_BF16, QLORA_EINVAL, "unknown dtype");
+    QL_REQUIRE(aligned(A, 16) && aligned(B, 16) && aligned(C, 16), QLORA_EALIGN,
+               "A, B and C must be 16-byte aligned");
+    QL_REQUIRE(aligned(scale_a, 4) && aligned(scale_b, 4) && (!bias || aligned(bias, 4)), QLORA_EALIGN,
+               "fp32 vectors must be 4-byte aligned");
+    int* status = status_ptr();
+    QL_REQUIRE(status, QLORA_ECUDA, "no CUDA device");
+    return cuda_status(launch_fp8_gemm(A, fmt_a == QLORA_FP8_E4M3 ? kFp8E4M3 : kFp8E5M2, B,
+                                       fmt_b == QLORA_FP8_E4M3 ? kFp8E4M3 : kFp8E5M2, M, N, K, scale_a,
+                                       scale_b, bias, C, c_dtype == QLORA_BF16 ? kBF16 : kF32, status,
+                                       static_cast<cudaStream_t>(stream)),
+                       "float8 GEMM launch");
+}
+
 int qlora_selftest_wait_timeout(unsigned int limit_us, void* stream) {
     QL_REQUIRE(limit_us >= 1 && limit_us <= 2000000, QLORA_EINVAL, "limit_us must be in [1, 2e6]");
     int* status = status_ptr();

@@ -35,7 +35,8 @@ EXPORTED = ("qlora_quantize_weight", "qlora_workspace_bytes", "qlora_forward",
             "qlora_set_rank_pass_rows", "qlora_quantize_weight_int4", "qlora_unpack_int4",
             "qlora_gemm_dx_int4", "qlora_merge_int4", "qlora_gemm_forward_int4",
             "qlora_outlier_cap", "qlora_outlier_workspace_bytes", "qlora_outlier_quantize",
-            "qlora_outlier_forward", "qlora_outlier_backward", "qlora_permute")
+            "qlora_outlier_forward", "qlora_outlier_backward", "qlora_permute",
+            "qlora_fp8_quantize", "qlora_fp8_gemm")
 
 
 class QLoraError(RuntimeError):
@@ -124,6 +125,10 @@ def _load():
     lib.qlora_outlier_backward.argtypes = [D, I, P, P, OK, P, P, P, P, P, P, P, P, Z, P]
     for f in (lib.qlora_outlier_quantize, lib.qlora_outlier_forward, lib.qlora_outlier_backward):
         f.restype = I
+    lib.qlora_fp8_quantize.argtypes = [P, I, I, I, I, P, P, P, I, P, P, P, Z, P]
+    lib.qlora_fp8_quantize.restype = I
+    lib.qlora_fp8_gemm.argtypes = [P, I, P, I, I, I, I, P, P, P, P, I, P]
+    lib.qlora_fp8_gemm.restype = I
     lib.qlora_permute.argtypes = [P, P, I, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int), I, P]
     lib.qlora_permute.restype = I
     lib.qlora_set_rank_pass_rows.argtypes = [I]
@@ -423,6 +428,32 @@ def qlora_permute(src: torch.Tensor, perm, out: Optional[torch.Tensor] = None, s
     pm = (ctypes.c_int * nd)(*perm)
     _check(_lib.qlora_permute(_ptr(src), _ptr(dst), nd, sh, pm, src.element_size(), _stream(stream)))
     return dst
+
+
+FP8_E4M3 = 0
+FP8_E5M2 = 1
+FP8_WORKSPACE_BYTES = 256
+
+
+def qlora_fp8_quantize(T: torch.Tensor, fmt: int, scale_in, scale_out, history, q, qt=None, ws=None,
+                       stream=None):
+    """Codes of T [rows, cols] with *scale_in into q (and its transpose into
+    qt), then the next scale into scale_out and the rolled amax history."""
+    rows, cols = T.shape
+    if ws is None:
+        ws = torch.empty(FP8_WORKSPACE_BYTES, dtype=torch.uint8, device=T.device)
+    _check(_lib.qlora_fp8_quantize(_ptr(T), rows, cols, act_code(T.dtype), int(fmt), _ptr(scale_in),
+                                   _ptr(scale_out), _ptr(history), history.numel(), _ptr(q), _ptr(qt),
+                                   _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def qlora_fp8_gemm(A, fmt_a: int, B, fmt_b: int, scale_a, scale_b, bias, C, stream=None):
+    """C [M,N] = (A [M,K] B [N,K]^T) * scale_a * scale_b (+ bias)."""
+    M, K = A.shape
+    N = B.shape[0]
+    assert B.shape[1] == K and tuple(C.shape) == (M, N)
+    _check(_lib.qlora_fp8_gemm(_ptr(A), int(fmt_a), _ptr(B), int(fmt_b), M, N, K, _ptr(scale_a),
+                               _ptr(scale_b), _ptr(bias), _ptr(C), act_code(C.dtype), _stream(stream)))
 
 
 def qlora_set_rank_pass_rows(rows: int) -> int:
