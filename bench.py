@@ -477,6 +477,44 @@ def outlier_entry(spec, dev, flush, roof, steps, warmup):
                     "tensor cores in both directions"}
 
 
+def float8_entry(name, M, K, N, dev, flush, roof, steps, warmup):
+    """One training step of a float8 Dense layer ("Introduce float8 training"):
+    three delayed-scaling quantizations (E4M3 input and kernel, E5M2 output
+    gradient), the forward, dX and dW GEMMs on float8 tensor cores, and the
+    bias gradient.  The float8 peak is twice the measured bf16 peak (the
+    nominal dense ratio)."""
+    import torch
+    from lora_fine_tuning_qlora_b200.float8 import Float8Dense
+    g = torch.Generator(device="cpu").manual_seed(M + K + N)
+    W = (torch.randn(K, N, generator=g) * 0.02).to(dev)
+    bias = torch.zeros(N, device=dev)
+    X = torch.randn(M, K, generator=g).to(torch.bfloat16).to(dev)
+    dY = (torch.randn(M, N, generator=g) * 1e-2).to(torch.bfloat16).to(dev)
+    lay = Float8Dense(W, bias, torch.bfloat16, history_len=1024)
+
+    def run():
+        _, ctx = lay.forward(X)
+        lay.backward(ctx, dY)
+
+    run()
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        run()
+    ms = time_graph(gr.replay, steps, warmup, flush)
+    step_us = 1e3 * statistics.median(ms)
+    fl = 6.0 * M * N * K
+    peak8 = 2.0 * roof.bf16
+    # bytes: the three tensors read, their codes written twice (row-major and
+    # transposed), the GEMMs' outputs
+    by = 2.0 * (M * K + M * N) + 4.0 * K * N + 2.0 * (M * K + K * N + M * N) + 2.0 * (M * N + M * K) + 4.0 * K * N
+    t_roof = (fl / peak8 + by / roof.bw) * 1e6
+    del gr
+    return {"workload": name, "M": M, "K": K, "N": N, "act": "bf16", "recipe": "float8 (E4M3 x, W; E5M2 dY)",
+            "step_us": step_us, "tflops": fl / (step_us * 1e-6) / 1e12, "t_roof_us": t_roof,
+            "roof_frac": t_roof / step_us, "frac_fp8_peak": fl / (step_us * 1e-6) / peak8}
+
+
 def all_configs(dev, flush, roof, steps, only):
     from lora_fine_tuning_qlora_b200 import inputs
     specs = [inputs.single_fp32()] + inputs.gpt2_base() + inputs.gemma_2b(512) + \
@@ -497,6 +535,11 @@ def all_configs(dev, flush, roof, steps, only):
         if only and only not in s.name.replace("gpt2_", "gpt2_outlier_"):
             continue
         out.append(outlier_entry(s, dev, flush, roof, steps, 3))
+    for name, M, K, N in (("float8_gpt2_mlp_up_4096x768x3072", 4096, 768, 3072),
+                          ("float8_dense4096_16384x4096x4096", 16384, 4096, 4096)):
+        if only and only not in name:
+            continue
+        out.append(float8_entry(name, M, K, N, dev, flush, roof, steps, 3))
     return out, merge
 
 

@@ -19,10 +19,11 @@
 //                        the float bits (non-negative floats order as
 //                        unsigned integers)
 //   fp8_state_kernel     one block: the new scale and the rolled history
-//   fp8_gemm_kernel      C = (A B^T) sa sb (+ bias): one 128 x 128 tile per
-//                        CTA, both operands K-major fp8 by TMA (128-byte
-//                        swizzle, 128 k per stage), 4 MMAs of K = 32 per
-//                        stage into a TMEM accumulator, four epilogue warps
+//   fp8_gemm_kernel      C = (A B^T) sa sb (+ bias): one 128 x 256 (or 128 x
+//                        128) tile per CTA, both operands K-major fp8 by TMA
+//                        (128-byte swizzle, 128 k per stage), 4 MMAs of
+//                        K = 32 per stage into a TMEM accumulator, four
+//                        epilogue warps
 #include "internal.h"
 #include "ptx.cuh"
 #include "tile_epilogue.cuh"
@@ -126,11 +127,17 @@ __global__ void __launch_bounds__(1024) fp8_state_kernel(const unsigned int* __r
 
 namespace {
 
-constexpr int kGM = 128, kGN = 128, kGK = 128;  // tile rows, columns, k bytes per stage
-constexpr int kGStages = 6;
+constexpr int kGM = 128, kGK = 128;  // tile rows, k bytes per stage
 constexpr int kGEpi = 4;
 constexpr int kGThreads = 32 * (2 + kGEpi);
-constexpr uint32_t kGStage = (kGM + kGN) * kGK;  // 32 KB
+// BN = 256 columns per tile where the output is wide enough (an MMA of
+// N = 256 keeps the tensor pipe busy for about as long as one takes to
+// issue), else 128; as many stages as fit 192 KB.
+template <int BN>
+struct GCfg {
+    static constexpr uint32_t kStage = (kGM + BN) * kGK;
+    static constexpr int kStages = (192 * 1024) / kStage > 8 ? 8 : (192 * 1024) / kStage;
+};
 
 // kind::f8f6f4 instruction descriptor: fp32 D; A and B formats (E4M3 0,
 // E5M2 1) in bits [7,10) and [10,13); both K-major; N >> 3, M >> 4.
@@ -149,7 +156,7 @@ __device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_
         : "memory");
 }
 
-template <typename OutT>
+template <typename OutT, int BN>
 __global__ void __launch_bounds__(kGThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
                     int N, int K, uint32_t idesc, const float* __restrict__ sa, const float* __restrict__ sb,
@@ -157,6 +164,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    constexpr int kGStages = GCfg<BN>::kStages;
+    constexpr uint32_t kGStage = GCfg<BN>::kStage;
+    constexpr int kGN = BN;
     constexpr uint32_t kStgOff = kGStages * kGStage;
     constexpr uint32_t kBarOff = kStgOff + kGEpi * 32 * stage_pitch<OutT>();
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOff);
@@ -175,7 +185,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(tslot, 128);
+        tmem_alloc(tslot, BN);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -246,7 +256,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 128);
+        tmem_dealloc(tmem, BN);
     }
 }
 
@@ -274,19 +284,28 @@ cudaError_t launch_fp8_gemm(const uint8_t* A, int afmt, const uint8_t* B, int bf
                             cudaStream_t s) {
     CUtensorMap ta, tb;
     if (!make_tmap_2d(&ta, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, K, kGM, kGK, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, kGN, kGK, CU_TENSOR_MAP_SWIZZLE_128B))
+        !make_tmap_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, 128, kGK, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    const uint32_t id = idesc_f8(kGM, kGN, afmt, bfmt);
-    const dim3 grid((N + kGN - 1) / kGN, (M + kGM - 1) / kGM);
-    auto run = [&](auto kern, size_t pitch) -> cudaError_t {
-        const size_t smem = kGStages * kGStage + kGEpi * 32 * pitch + 256 + 1024;
+    const int bn = N >= 256 ? 256 : 128;
+    CUtensorMap tb2;
+    if (!make_tmap_2d(&tb2, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, bn, kGK, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    (void)tb;
+    const uint32_t id = idesc_f8(kGM, bn, afmt, bfmt);
+    const dim3 grid((N + bn - 1) / bn, (M + kGM - 1) / kGM);
+    auto run = [&](auto kern, size_t stage_bytes_total, size_t pitch) -> cudaError_t {
+        const size_t smem = stage_bytes_total + kGEpi * 32 * pitch + 256 + 1024;
         cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
         if (e != cudaSuccess) return e;
-        return launch_k(kern, grid, dim3(kGThreads), smem, s, 1, ta, tb, M, N, K, id, sa, sb, bias, C, status);
+        return launch_k(kern, grid, dim3(kGThreads), smem, s, 1, ta, tb2, M, N, K, id, sa, sb, bias, C, status);
     };
+    constexpr size_t r128 = static_cast<size_t>(GCfg<128>::kStages) * GCfg<128>::kStage;
+    constexpr size_t r256 = static_cast<size_t>(GCfg<256>::kStages) * GCfg<256>::kStage;
     if (out == kBF16)
-        return run(fp8_gemm_kernel<__nv_bfloat16>, stage_pitch<__nv_bfloat16>());
-    return run(fp8_gemm_kernel<float>, stage_pitch<float>());
+        return bn == 256 ? run(fp8_gemm_kernel<__nv_bfloat16, 256>, r256, stage_pitch<__nv_bfloat16>())
+                         : run(fp8_gemm_kernel<__nv_bfloat16, 128>, r128, stage_pitch<__nv_bfloat16>());
+    return bn == 256 ? run(fp8_gemm_kernel<float, 256>, r256, stage_pitch<float>())
+                     : run(fp8_gemm_kernel<float, 128>, r128, stage_pitch<float>());
 }
 
 }  // namespace qlora
