@@ -307,16 +307,18 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     }
                 }
                 if constexpr (MODE == 2) {
-                    // The warp wrote whole tile rows nr = 4 gw + (c % 32) / 8 +
-                    // 4 kDqWPG i; each lane writes the outliers of one of them.
-                    static_assert(kPerLane * (32 / kChunksPerRow) == 32, "one row per lane");
+                    // The warp wrote whole tile rows nr = kRW gw + (c % 32) /
+                    // kChunksPerRow + kRW kDqWPG i (kRW rows per 32 chunks);
+                    // its lanes now write those rows' outliers.
+                    constexpr int kRW = 32 / kChunksPerRow;
                     __syncwarp();
-                    const int nr = gw * (32 / kChunksPerRow) + (lane % (32 / kChunksPerRow)) +
-                                   (32 / kChunksPerRow) * kDqWPG * (lane / (32 / kChunksPerRow));
-                    const int n = (g % nkb) * kPK + nr;
                     const int t = pair + (g / nkb) * npairs;
                     const int c0 = (t % num_kt) * kPN + static_cast<int>(rank) * kHalf;
-                    if (n < N && c0 < K) patch_outliers(ep.ol, n, c0, kHalf, wt, nr, kPLbo);
+                    for (int idx = lane; idx < kPerLane * kRW; idx += 32) {
+                        const int nr = gw * kRW + idx % kRW + kRW * kDqWPG * (idx / kRW);
+                        const int n = (g % nkb) * kPK + nr;
+                        if (n < N && c0 < K) patch_outliers(ep.ol, n, c0, kHalf, wt, nr, kPLbo);
+                    }
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
