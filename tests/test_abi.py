@@ -156,3 +156,42 @@ def test_int4_forward_rejects_k_not_multiple_of_32(q):
     rc = q.lib().qlora_gemm_forward_int4(ctypes.byref(d), 64, P(0x1000), P(0x2000), P(0x3000),
                                          P(0x4000), None, P(0x5000), P(0x6000), P(0x7000), None, None)
     assert rc == -5
+
+
+def test_new_entry_points_reject_bad_arguments(q):
+    """The outlier, float8 and permutation calls validate before any launch
+    (fake device addresses are never dereferenced)."""
+    lib = ctypes.CDLL(q.LIB_PATH)
+    P = ctypes.c_void_p
+    fake = P(4096)
+    # permutation: not a permutation, too many axes, NULL
+    sh = (ctypes.c_int64 * 2)(4, 4)
+    assert lib.qlora_permute(fake, P(8192), 2, sh, (ctypes.c_int * 2)(0, 0), 4, None) == -1
+    sh9 = (ctypes.c_int64 * 9)(*([2] * 9))
+    assert lib.qlora_permute(fake, P(8192), 9, sh9, (ctypes.c_int * 9)(*range(9)), 4, None) == -3
+    assert lib.qlora_permute(None, P(8192), 2, sh, (ctypes.c_int * 2)(1, 0), 4, None) == -1
+    # float8 GEMM: K not a multiple of 16; unknown format
+    lib.qlora_fp8_gemm.argtypes = [P, ctypes.c_int, P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                   ctypes.c_int, P, P, P, P, ctypes.c_int, P]
+    assert lib.qlora_fp8_gemm(fake, 0, fake, 0, 16, 16, 24, fake, fake, None, fake, 1, None) == -5
+    assert lib.qlora_fp8_gemm(fake, 7, fake, 0, 16, 16, 32, fake, fake, None, fake, 1, None) == -1
+    # float8 quantizer: the next scale must not overwrite the one in use
+    lib.qlora_fp8_quantize.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P,
+                                       ctypes.c_int, P, P, P, ctypes.c_size_t, P]
+    assert lib.qlora_fp8_quantize(fake, 4, 4, 1, 0, fake, fake, P(8192), 16, P(12288), None, P(16384), 256,
+                                  None) == -1
+    # outlier kernel: capacity below the bound, NULL member
+    cap = q.qlora_outlier_cap(256, 256)
+    assert cap == (int((256 * 256 - 1) * 0.1 / 100) + 1) + (256 * 256 - 1 - int((256 * 256 - 1) * 99.9 / 100))
+    ok = q.OutlierKernelStruct(4096, 8192, 12288, 16384, 20480, 24576, 28672, cap)
+    small = q.OutlierKernelStruct(4096, 8192, 12288, 16384, 20480, 24576, 28672, cap - 1)
+    ws = P(32768)
+    nbytes = q.qlora_outlier_workspace_bytes(256, 256)
+    assert lib.qlora_outlier_quantize(fake, 256, 256, ctypes.byref(small), ws, nbytes, None) == -1
+    nul = q.OutlierKernelStruct(4096, 0, 12288, 16384, 20480, 24576, 28672, cap)
+    assert lib.qlora_outlier_quantize(fake, 256, 256, ctypes.byref(nul), ws, nbytes, None) == -1
+    assert lib.qlora_outlier_quantize(fake, 256, 256, ctypes.byref(ok), ws, nbytes - 1, None) == -1
+    # the outlier layer refuses a K that is not a multiple of 16
+    d = q.desc(100, 64, 4, 4.0, __import__("torch").bfloat16)
+    assert lib.qlora_outlier_forward(ctypes.byref(d), 8, fake, ctypes.byref(ok), None, fake, fake, fake, fake,
+                                     ws, 1 << 20, None) == -5
