@@ -22,6 +22,26 @@ __device__ __forceinline__ uint32_t mn_sw128_offset(int mn, int kr, uint32_t lbo
     return mb * lbo + kg * 1024 + row * 128 + ((chunk ^ row) << 4);
 }
 
+// Chunk c of a de-quantize stage -> (contraction row nr, 16-byte chunk kc of
+// that row), CPR chunks per row.  With 8 chunks per row (two 64-element MN
+// blocks) the plain row-major order puts chunks kc and kc + 4 of one row,
+// which land on the same shared-memory banks one MN block apart, in the same
+// 8-lane phase of a 16-byte store; instead every 8 consecutive chunks cover
+// two rows of opposite parity and four chunks of one MN block, so the
+// swizzled positions ((kc % 4) * 2 ^ row) of a phase are all distinct.  The
+// rows a warp covers are the same set as in row-major order.
+template <int CPR>
+__device__ __forceinline__ void chunk_rc(int c, int& nr, int& kc) {
+    if constexpr (CPR == 8) {
+        const int rest = c >> 3;
+        nr = 2 * (rest >> 1) + ((c >> 2) & 1);
+        kc = (c & 3) + 4 * (rest & 1);
+    } else {
+        nr = c / CPR;
+        kc = c % CPR;
+    }
+}
+
 // G[m,j] = sum over the column-block slices of G (fixed order).
 __device__ __forceinline__ float g_row(const DxEpilogue& ep, int M, int m, int j) {
     return sum_slices(ep.Gp + static_cast<size_t>(m) * ep.r + j, static_cast<size_t>(M) * ep.r,

@@ -233,8 +233,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #pragma unroll
             for (int i = 0; i < kPerLane; ++i) {
                 const int c = gw * 32 + lane + i * 32 * kDqWPG;
-                const int n = fkb * kPK + c / kChunksPerRow;
-                const int k = fk0 + (c % kChunksPerRow) * kCodes;
+                int cr, cc;
+                chunk_rc<kChunksPerRow>(c, cr, cc);
+                const int n = fkb * kPK + cr;
+                const int k = fk0 + cc * kCodes;
                 if (live_g && n < N && k < K) in_bits |= 1u << i;
                 const int nc = n < N ? n : N - 1;
                 const int kc = k < K ? k : K - kCodes;
@@ -274,8 +276,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #pragma unroll
                 for (int i = 0; i < kPerLane; ++i) {
                     const int c = gw * 32 + lane + i * 32 * kDqWPG;
-                    const int nr = c / kChunksPerRow;
-                    const int kc = c % kChunksPerRow;
+                    int nr, kc;
+                    chunk_rc<kChunksPerRow>(c, nr, kc);
                     const float scale = (inb[v] >> i) & 1u ? sr[v][i] : 0.f;
                     const int mn = kc * kCodes;
                     uint32_t o[8];
