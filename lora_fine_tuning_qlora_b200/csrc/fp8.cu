@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(256) fp8_quantize_kernel(const T* __restrict__
     pdl_trigger();
     pdl_wait();
     const float s = __ldg(scale);
-    const int r0 = blockIdx.y * kQT, c0 = blockIdx.x * kQT;
+    const int r0 = blockIdx.x * kQT, c0 = blockIdx.y * kQT;
     const int tx = threadIdx.x % kQT, ty = threadIdx.x / kQT;  // 32 x 8
     float mx = 0.f;
     for (int rr = ty; rr < kQT; rr += 8) {
@@ -79,6 +79,142 @@ __global__ void __launch_bounds__(256) fp8_quantize_kernel(const T* __restrict__
         for (int cc = ty; cc < kQT; cc += 8) {
             const int c = c0 + cc, r = r0 + tx;
             if (c < Cc && r < R) qt[static_cast<size_t>(c) * R + r] = tile[tx][cc];
+        }
+    }
+}
+
+// The same quantizer for aligned layouts (T 16-byte aligned, cols % 8 == 0,
+// q 8-byte aligned; qt 16-byte aligned with rows % 16 == 0): one 128 x 128
+// tile per block of 256 threads.  Each thread loads eight 8-value chunks
+// (16-byte loads, all in flight before the first is used), converts two
+// values per cvt and stores 8 codes per 8-byte store; the codes also go to
+// a 16 KB shared tile (32 words a row, word w of row r at w ^ 4 ((r / 16) %
+// 8), so that both the 8-byte stores and the column reads below are free of
+// bank conflicts).  For qt each thread then reads a 16-row x 4-column block,
+// transposes it four 4 x 4 byte blocks at a time with byte permutes and
+// writes four 16-byte runs of qt rows; eight threads cover 128 contiguous
+// bytes of one qt row.
+constexpr int kFR = 128, kFC = 128, kFThreads = 256;
+constexpr int kFChunks = kFR * kFC / 8 / kFThreads;  // 8 chunks of 8 values per thread
+
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, uint32_t (&raw)[8]) {
+    const uint4 r = __ldg(reinterpret_cast<const uint4*>(p));
+    raw[0] = r.x;
+    raw[1] = r.y;
+    raw[2] = r.z;
+    raw[3] = r.w;
+}
+__device__ __forceinline__ void load8(const float* p, uint32_t (&raw)[8]) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint4 b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
+    raw[0] = a.x;
+    raw[1] = a.y;
+    raw[2] = a.z;
+    raw[3] = a.w;
+    raw[4] = b.x;
+    raw[5] = b.y;
+    raw[6] = b.z;
+    raw[7] = b.w;
+}
+__device__ __forceinline__ float val8(const uint32_t (&raw)[8], int i, const __nv_bfloat16*) {
+    return __uint_as_float((i & 1) ? (raw[i >> 1] & 0xffff0000u) : (raw[i >> 1] << 16));
+}
+__device__ __forceinline__ float val8(const uint32_t (&raw)[8], int i, const float*) {
+    return __uint_as_float(raw[i]);
+}
+
+template <int FMT>
+__device__ __forceinline__ uint32_t cvt2(float lo, float hi) {
+    const __nv_fp8x2_storage_t c = __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE,
+                                                            FMT == kFp8E4M3 ? __NV_E4M3 : __NV_E5M2);
+    return static_cast<uint32_t>(c);
+}
+
+// rows (w0..w3) x 4 byte columns -> 4 columns (c0..c3) x 4 rows
+__device__ __forceinline__ void transpose4x4(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, uint32_t& c0,
+                                             uint32_t& c1, uint32_t& c2, uint32_t& c3) {
+    const uint32_t t0 = __byte_perm(w0, w1, 0x5140);  // w0.b0 w1.b0 w0.b1 w1.b1
+    const uint32_t t1 = __byte_perm(w0, w1, 0x7362);  // w0.b2 w1.b2 w0.b3 w1.b3
+    const uint32_t t2 = __byte_perm(w2, w3, 0x5140);
+    const uint32_t t3 = __byte_perm(w2, w3, 0x7362);
+    c0 = __byte_perm(t0, t2, 0x5410);
+    c1 = __byte_perm(t0, t2, 0x7632);
+    c2 = __byte_perm(t1, t3, 0x5410);
+    c3 = __byte_perm(t1, t3, 0x7632);
+}
+
+template <typename T, int FMT>
+__global__ void __launch_bounds__(kFThreads) fp8_quantize_tiled_kernel(const T* __restrict__ src, int R, int Cc,
+                                                                      const float* __restrict__ scale,
+                                                                      uint8_t* __restrict__ q,
+                                                                      uint8_t* __restrict__ qt,
+                                                                      unsigned int* __restrict__ amax_bits) {
+    __shared__ __align__(16) uint32_t tile[kFR * kFC / 4];
+    __shared__ float wmax[kFThreads / 32];
+    pdl_trigger();
+    pdl_wait();
+    const int t = threadIdx.x;
+    const int r0 = blockIdx.x * kFR, c0 = blockIdx.y * kFC;
+    const int j = t % 16;  // this thread's 8-column chunk in every row it handles
+    const int gc = c0 + 8 * j;
+    uint32_t raw[kFChunks][8];
+#pragma unroll
+    for (int u = 0; u < kFChunks; ++u) {
+        const int gr = r0 + t / 16 + 16 * u;
+        if (gr < R && gc < Cc) load8(src + static_cast<size_t>(gr) * Cc + gc, raw[u]);
+        else
+#pragma unroll
+            for (int i = 0; i < 8; ++i) raw[u][i] = 0u;
+    }
+    const float s = __ldg(scale);
+    float mx = 0.f;
+#pragma unroll
+    for (int u = 0; u < kFChunks; ++u) {
+        const int row = t / 16 + 16 * u;
+        const int gr = r0 + row;
+        float x[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float v = val8(raw[u], i, src);
+            mx = fmaxf(mx, fabsf(v));
+            x[i] = __fdiv_rn(v, s);
+        }
+        const uint32_t lo = cvt2<FMT>(x[0], x[1]) | (cvt2<FMT>(x[2], x[3]) << 16);
+        const uint32_t hi = cvt2<FMT>(x[4], x[5]) | (cvt2<FMT>(x[6], x[7]) << 16);
+        if (gr < R && gc < Cc)
+            *reinterpret_cast<uint2*>(q + static_cast<size_t>(gr) * Cc + gc) = make_uint2(lo, hi);
+        const int w = (2 * j) ^ (((row >> 4) & 7) << 2);
+        *reinterpret_cast<uint2*>(&tile[row * 32 + w]) = make_uint2(lo, hi);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (t % 32 == 0) wmax[t / 32] = mx;
+    __syncthreads();
+    if (t == 0) {
+        float m = wmax[0];
+#pragma unroll
+        for (int i = 1; i < kFThreads / 32; ++i) m = fmaxf(m, wmax[i]);
+        atomicMax(amax_bits, __float_as_uint(m));
+    }
+    if (qt) {
+        const int seg = t % 8, c4 = t / 8;
+        const int gr = r0 + 16 * seg;
+        if (gr < R) {
+            uint32_t col[4][4];  // [column of the quad][group of 4 rows]
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                uint32_t w[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) w[i] = tile[(16 * seg + 4 * g + i) * 32 + (c4 ^ (seg << 2))];
+                transpose4x4(w[0], w[1], w[2], w[3], col[0][g], col[1][g], col[2][g], col[3][g]);
+            }
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int c = c0 + 4 * c4 + jj;
+                if (c < Cc)
+                    *reinterpret_cast<uint4*>(qt + static_cast<size_t>(c) * R + gr) =
+                        make_uint4(col[jj][0], col[jj][1], col[jj][2], col[jj][3]);
+            }
         }
     }
 }
@@ -260,6 +396,227 @@ __global__ void __launch_bounds__(kGThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------------------
+// The same product on CTA pairs, for outputs of at least one 256 x 256 tile
+// per pair of SMs: a cluster of two CTAs computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2.kind::f8f6f4 (M = 256, N = 256, K = 32); CTA r
+// loads A rows [128 r, +128) and B rows [128 r, +128) of the tile, 128 k per
+// stage (TMA, K-major, 128-byte swizzle) and holds its 128 rows x 256 columns
+// of the fp32 accumulator in TMEM.  Each CTA then streams half as many bytes
+// per MMA as in the one-CTA kernel.  Persistent: pair p takes tiles p,
+// p + pairs, ...; the accumulator is double-buffered (512 TMEM columns) so
+// the epilogue of one tile overlaps the main loop of the next.
+// Warps: 0 TMA producer; 1 TMEM owner and, in CTA 0, the MMA issuer; 2..5
+// epilogue.  full[s] (CTA 0) completes when the four boxes of stage s have
+// landed; the commits arrive on empty[s] and tfull[b] of both CTAs;
+// tempty[b] (CTA 0) takes one arrival from each epilogue warp of both CTAs.
+// ---------------------------------------------------------------------------
+constexpr int kPM = 128;   // rows per CTA (256 per pair)
+constexpr int kPN = 256;   // output columns per pair tile (128 B rows per CTA)
+constexpr int kPSmemLimit = 232448;
+
+template <typename OutT>
+struct PCfg {
+    static constexpr int kABytes = kPM * kGK;
+    static constexpr int kBBytes = (kPN / 2) * kGK;
+    static constexpr int kStageBytes = kABytes + kBBytes;  // 32 KB
+    static constexpr int kStgBytes = kGEpi * 32 * stage_pitch<OutT>();
+    static constexpr int kTabBytes = kPN * 4;              // bias of the tile's columns
+    static constexpr int kFixed = kStgBytes + kTabBytes + 512 + 1024;
+    static constexpr int kFit = (kPSmemLimit - kFixed) / kStageBytes;
+    static constexpr int S = kFit > 6 ? 6 : kFit;
+    static_assert(S >= 4, "shared memory budget");
+    static constexpr int kStgOff = S * kStageBytes;
+    static constexpr int kTabOff = kStgOff + kStgBytes;
+    static constexpr int kBarOff = kTabOff + kTabBytes;
+    static constexpr int kTotal = kBarOff + 512 + 1024;
+    static_assert((2 * S + 4) * 8 + 4 <= 512, "barrier area");
+    static constexpr uint32_t kAccCols = kPN;
+    static constexpr uint32_t kTmemCols = 2 * kAccCols;
+};
+
+__device__ __forceinline__ void mma_f8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+template <typename OutT>
+__global__ void __launch_bounds__(kGThreads, 1)
+    fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                         int M, int N, int K, uint32_t idesc, const float* __restrict__ sa,
+                         const float* __restrict__ sb, const float* __restrict__ bias, OutT* __restrict__ C,
+                         int* status) {
+    using P = PCfg<OutT>;
+    constexpr int S = P::S;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + P::kBarOff);  // [S] (CTA 0)
+    uint64_t* empty = full + S;                                       // [S]
+    uint64_t* tfull = empty + S;                                      // [2]
+    uint64_t* tempty = tfull + 2;                                     // [2] (CTA 0)
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(tempty + 2);
+    float* sBias = reinterpret_cast<float*>(smem + P::kTabOff);
+
+    const uint32_t rank = cluster_ctarank();
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int pair = static_cast<int>(blockIdx.x) / 2;
+    const int npairs = static_cast<int>(gridDim.x) / 2;
+    const int num_nt = (N + kPN - 1) / kPN;
+    const int tiles = ((M + 2 * kPM - 1) / (2 * kPM)) * num_nt;
+    const int nkb = (K + kGK - 1) / kGK;
+    pdl_trigger();
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 2 * kGEpi);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tslot, P::kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+    // neither CTA signals the other's barriers before both have initialised them
+    cluster_arrive();
+    cluster_wait();
+    pdl_wait();  // nothing above touched global memory
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmA);
+            tma_prefetch_desc(&tmB);
+            const uint32_t full0 = dsmem_addr(full, 0);  // CTA 0's full[0]
+            int g = 0;
+            bool ok = true;
+            for (int t = pair; t < tiles && ok; t += npairs) {
+                const int m0 = (t / num_nt) * 2 * kPM + static_cast<int>(rank) * kPM;
+                const int n0 = (t % num_nt) * kPN + static_cast<int>(rank) * (kPN / 2);
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s = g % S;
+                    if (g >= S && !mbar_wait(&empty[s], ((g / S) - 1) & 1, status)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* st = smem + s * P::kStageBytes;
+                    if (rank == 0) {
+                        mbar_arrive_expect_tx(&full[s], 2 * P::kStageBytes);
+                        tma_load_2d(st, &tmA, &full[s], kb * kGK, m0);
+                        tma_load_2d(st + P::kABytes, &tmB, &full[s], kb * kGK, n0);
+                    } else {
+                        const uint32_t fb = full0 + 8u * static_cast<uint32_t>(s);
+                        tma_load_2d_pair(st, &tmA, fb, kb * kGK, m0);
+                        tma_load_2d_pair(st + P::kABytes, &tmB, fb, kb * kGK, n0);
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer (CTA 0)
+        if (rank == 0 && lane == 0) {
+            int g = 0, i = 0;
+            bool ok = true;
+            for (int t = pair; t < tiles && ok; t += npairs, ++i) {
+                const int ab = i & 1;
+                const int use = i >> 1;
+                if (use > 0 && !mbar_wait(&tempty[ab], (use - 1) & 1, status)) break;
+                tc_fence_after();
+                const uint32_t dacc = tmem + ab * P::kAccCols;
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s = g % S;
+                    if (!mbar_wait(&full[s], (g / S) & 1, status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(smem + s * P::kStageBytes);
+                    const uint32_t b_base = a_base + P::kABytes;
+#pragma unroll
+                    for (int kk = 0; kk < kGK / 32; ++kk) {
+                        const uint64_t ad = smem_desc(a_base + kk * 32, 16, 1024, kLayoutSw128);
+                        const uint64_t bd = smem_desc(b_base + kk * 32, 16, 1024, kLayoutSw128);
+                        mma_f8_pair(dacc, ad, bd, idesc, (kb != 0 || kk != 0) ? 1u : 0u);
+                    }
+                    mma_commit_pair(&empty[s], 0x3);
+                }
+                if (ok) mma_commit_pair(&tfull[ab], 0x3);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------ epilogue
+        const int ew = warp - 2;  // 0 .. 3
+        const int q = warp & 3;   // TMEM lane quarter of this warp
+        const int et = threadIdx.x - 64;
+        uint8_t* stg = smem + P::kStgOff + ew * 32 * stage_pitch<OutT>();
+        const bool vec = ((static_cast<size_t>(N) * sizeof(OutT)) % 16) == 0;
+        const uint32_t tempty0 = dsmem_addr(tempty, 0);
+        const float sab = __fmul_rn(__ldg(sa), __ldg(sb));
+        int i = 0;
+        for (int t = pair; t < tiles; t += npairs, ++i) {
+            const int ab = i & 1;
+            const int use = i >> 1;
+            const int m0 = (t / num_nt) * 2 * kPM + static_cast<int>(rank) * kPM;
+            const int n0 = (t % num_nt) * kPN;
+            // the tile's bias (the last tile's reads are done)
+            named_bar_sync(1, 32 * kGEpi);
+            for (int col = et; col < kPN; col += 32 * kGEpi) {
+                const int n = n0 + col;
+                sBias[col] = (bias && n < N) ? __ldg(bias + n) : 0.f;
+            }
+            named_bar_sync(1, 32 * kGEpi);
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[ab], use & 1, status));
+            if (!ok) break;
+            tc_fence_after();
+            const int row0 = m0 + q * 32;
+            const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * P::kAccCols;
+            if (nkb > 0) {
+#pragma unroll 1
+                for (int col = 0; col < kPN; col += kEpiCols) {
+                    uint32_t v[kEpiCols];
+                    tmem_ld16(tbase + col, v);
+                    tmem_ld_wait();
+                    float y[kEpiCols];
+#pragma unroll
+                    for (int e = 0; e < kEpiCols; ++e) y[e] = fmaf(__uint_as_float(v[e]), sab, sBias[col + e]);
+                    store_block<OutT>(stg, y, lane, C, static_cast<size_t>(N), row0, M, n0 + col, N, vec);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (rank == 0) mbar_arrive(&tempty[ab]);
+                else mbar_arrive_remote_cta(tempty0 + 8u * static_cast<uint32_t>(ab));
+            }
+        }
+        __syncwarp();
+    }
+    tc_fence_before();
+    __syncthreads();
+    // both CTAs are done with the pair's TMEM and with each other's barriers
+    cluster_arrive();
+    cluster_wait();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, P::kTmemCols);
+    }
+}
 }  // namespace
 
 cudaError_t launch_fp8_quantize(Act act, const void* T, int R, int Cc, const float* scale_in, float* scale_out,
@@ -267,12 +624,35 @@ cudaError_t launch_fp8_quantize(Act act, const void* T, int R, int Cc, const flo
                                 cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(amax_word, 0, sizeof(unsigned int), s);
     if (e != cudaSuccess) return e;
-    const dim3 grid((Cc + kQT - 1) / kQT, (R + kQT - 1) / kQT);
-    e = act == kBF16
-            ? launch_k(fp8_quantize_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, 1,
-                       static_cast<const __nv_bfloat16*>(T), R, Cc, scale_in, fmt, q, qt, amax_word)
-            : launch_k(fp8_quantize_kernel<float>, grid, dim3(256), 0, s, 1, static_cast<const float*>(T), R,
-                       Cc, scale_in, fmt, q, qt, amax_word);
+    const auto al = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; };
+    const bool tiled = al(T, 16) && Cc % 8 == 0 && al(q, 8) && (!qt || (al(qt, 16) && R % 16 == 0)) &&
+                       (Cc + kFC - 1) / kFC <= 65535;
+    if (tiled) {
+        const dim3 grid((R + kFR - 1) / kFR, (Cc + kFC - 1) / kFC);
+        if (act == kBF16) {
+            const auto* src = static_cast<const __nv_bfloat16*>(T);
+            e = fmt == kFp8E4M3
+                    ? launch_k(fp8_quantize_tiled_kernel<__nv_bfloat16, kFp8E4M3>, grid, dim3(kFThreads), 0, s, 1,
+                               src, R, Cc, scale_in, q, qt, amax_word)
+                    : launch_k(fp8_quantize_tiled_kernel<__nv_bfloat16, kFp8E5M2>, grid, dim3(kFThreads), 0, s, 1,
+                               src, R, Cc, scale_in, q, qt, amax_word);
+        } else {
+            const auto* src = static_cast<const float*>(T);
+            e = fmt == kFp8E4M3
+                    ? launch_k(fp8_quantize_tiled_kernel<float, kFp8E4M3>, grid, dim3(kFThreads), 0, s, 1, src, R,
+                               Cc, scale_in, q, qt, amax_word)
+                    : launch_k(fp8_quantize_tiled_kernel<float, kFp8E5M2>, grid, dim3(kFThreads), 0, s, 1, src, R,
+                               Cc, scale_in, q, qt, amax_word);
+        }
+    } else {
+        if ((Cc + kQT - 1) / kQT > 65535) return cudaErrorInvalidValue;
+        const dim3 grid((R + kQT - 1) / kQT, (Cc + kQT - 1) / kQT);
+        e = act == kBF16
+                ? launch_k(fp8_quantize_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, 1,
+                           static_cast<const __nv_bfloat16*>(T), R, Cc, scale_in, fmt, q, qt, amax_word)
+                : launch_k(fp8_quantize_kernel<float>, grid, dim3(256), 0, s, 1, static_cast<const float*>(T), R,
+                           Cc, scale_in, fmt, q, qt, amax_word);
+    }
     if (e != cudaSuccess) return e;
     const float fmax = fmt == kFp8E4M3 ? 448.0f : 57344.0f;
     return launch_k(fp8_state_kernel, dim3(1), dim3(1024), 0, s, 1, static_cast<const unsigned int*>(amax_word),
@@ -290,7 +670,21 @@ cudaError_t launch_fp8_gemm(const uint8_t* A, int afmt, const uint8_t* B, int bf
     CUtensorMap tb2;
     if (!make_tmap_2d(&tb2, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, bn, kGK, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    (void)tb;
+    const int pair_tiles = ((M + 2 * kPM - 1) / (2 * kPM)) * ((N + kPN - 1) / kPN);
+    if (pair_tiles >= sm_count() / 2) {
+        // CTA pairs, persistent: one pair per two SMs; tb holds 128-row boxes of B
+        const int pairs = pair_tiles < sm_count() / 2 ? pair_tiles : sm_count() / 2;
+        const uint32_t idp = idesc_f8(2 * kPM, kPN, afmt, bfmt);
+        auto runp = [&](auto kern, int total) -> cudaError_t {
+            cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), total);
+            if (e != cudaSuccess) return e;
+            return launch_kx(kern, dim3(2 * pairs), dim3(kGThreads), static_cast<size_t>(total), s, 2, ta, tb, M,
+                             N, K, idp, sa, sb, bias, C, status);
+        };
+        if (out == kBF16)
+            return runp(fp8_gemm_pair_kernel<__nv_bfloat16>, PCfg<__nv_bfloat16>::kTotal);
+        return runp(fp8_gemm_pair_kernel<float>, PCfg<float>::kTotal);
+    }
     const uint32_t id = idesc_f8(kGM, bn, afmt, bfmt);
     const dim3 grid((N + bn - 1) / bn, (M + kGM - 1) / kGM);
     auto run = [&](auto kern, size_t stage_bytes_total, size_t pitch) -> cudaError_t {

@@ -31,13 +31,20 @@ def _fmt(q, name):
     return q.FP8_E4M3 if name == f8.E4M3 else q.FP8_E5M2
 
 
-@pytest.mark.parametrize("R,C,dtype,fmt,scale,L", [
-    (300, 784, torch.bfloat16, f8.E4M3, 0.01, 7),
-    (129, 1000, torch.float32, f8.E5M2, 1e-4, 1024),
-    (64, 64, torch.bfloat16, f8.E5M2, 3.0, 1500),     # history longer than one block
-    (1, 16, torch.float32, f8.E4M3, 1.0, 1),
+@pytest.mark.parametrize("R,C,dtype,fmt,scale,L,with_qt", [
+    # 8-aligned columns but rows % 16 != 0 with the transpose: the scalar kernel
+    (300, 784, torch.bfloat16, f8.E4M3, 0.01, 7, True),
+    (129, 1000, torch.float32, f8.E5M2, 1e-4, 1024, True),
+    (1, 16, torch.float32, f8.E4M3, 1.0, 1, True),
+    (37, 30, torch.bfloat16, f8.E4M3, 0.5, 3, True),   # columns not a multiple of 8
+    # the 128 x 128 tiled kernel: whole and ragged tiles, both formats and types
+    (64, 64, torch.bfloat16, f8.E5M2, 3.0, 1500, True),  # history longer than one block
+    (304, 1000, torch.bfloat16, f8.E4M3, 0.01, 16, True),
+    (2000, 520, torch.float32, f8.E5M2, 1e-3, 16, True),
+    (1024, 384, torch.float32, f8.E4M3, 0.02, 16, True),
+    (301, 136, torch.bfloat16, f8.E5M2, 2e-3, 4, False),  # no transpose: any row count
 ])
-def test_quantize_state_bit_exact(q, R, C, dtype, fmt, scale, L):
+def test_quantize_state_bit_exact(q, R, C, dtype, fmt, scale, L, with_qt):
     rng = np.random.Generator(np.random.PCG64(R + C))
     T = (rng.standard_normal((R, C)) * rng.choice([1e-6, 1.0, 40.0, 1e4], (R, C))).astype(np.float32)
     Tt = torch.from_numpy(T).to(dtype).cuda()
@@ -48,12 +55,13 @@ def test_quantize_state_bit_exact(q, R, C, dtype, fmt, scale, L):
     s_out = torch.full((1,), -1.0, dtype=torch.float32, device="cuda")
     h = torch.from_numpy(hist).cuda()
     qq = torch.empty((R, C), dtype=torch.uint8, device="cuda")
-    qt = torch.empty((C, R), dtype=torch.uint8, device="cuda")
+    qt = torch.empty((C, R), dtype=torch.uint8, device="cuda") if with_qt else None
     q.qlora_fp8_quantize(Tt, _fmt(q, fmt), s_in, s_out, h, qq, qt)
     torch.cuda.synchronize()
     codes, amax, new = f8.step_tensor(Tv, {"scale": np.float32(scale), "history": hist}, fmt)
     np.testing.assert_array_equal(qq.cpu().numpy(), codes)
-    np.testing.assert_array_equal(qt.cpu().numpy(), codes.T)
+    if with_qt:
+        np.testing.assert_array_equal(qt.cpu().numpy(), codes.T)
     assert to_np(s_out)[0] == new["scale"]
     np.testing.assert_array_equal(to_np(h), new["history"])
 
@@ -75,6 +83,12 @@ def test_zero_history_keeps_the_scale(q):
     (200, 264, 1024, f8.E5M2, f8.E4M3, torch.bfloat16),  # gradient x kernel
     (768, 384, 512, f8.E4M3, f8.E5M2, torch.float32),    # input^T x gradient
     (1, 16, 16, f8.E4M3, f8.E4M3, torch.float32),
+    # CTA pairs (at least one 256 x 256 tile per two SMs): the last tile's
+    # second half of rows and of columns wholly outside, ragged k-block
+    (2148, 2100, 784, f8.E5M2, f8.E4M3, torch.bfloat16),
+    # CTA pairs, several tiles per pair: both accumulator buffers and the
+    # stage ring wrap
+    (4096, 4096, 256, f8.E4M3, f8.E5M2, torch.float32),
 ])
 def test_fp8_gemm(q, M, N, K, fa, fb, out):
     rng = np.random.Generator(np.random.PCG64(M * N + K))
@@ -91,13 +105,35 @@ def test_fp8_gemm(q, M, N, K, fa, fb, out):
                      torch.tensor([sa], device="cuda"), torch.tensor([sb], device="cuda"),
                      torch.from_numpy(bias).cuda(), C)
     torch.cuda.synchronize()
-    ref = (f8.decode(A, fa) @ f8.decode(B, fb).T) * (np.float64(sa) * np.float64(sb)) + bias[None, :]
+    da, db = f8.decode(A, fa), f8.decode(B, fb)
+    sab = np.float64(sa) * np.float64(sb)
+    ref = (da @ db.T) * sab + bias[None, :]
     got = to_np(C)
-    if out == torch.bfloat16:
-        assert_close(got, ref, "bf16", "C")
-    else:
-        err = np.abs(got - ref).max() / max(np.abs(ref).max(), 1e-30)
-        assert err <= F32_SUM_RTOL, err
+    # per element: the fp32 sum of K exact products errs by at most
+    # K u sum_k |a_k b_k| in any order (u = 2^-24; 2u allowed), then one
+    # rounding to the output type (2^-8 relative for bf16, 2^-23 for fp32)
+    sum_abs = (np.abs(da) @ np.abs(db).T) * sab
+    out_u = 2.0 ** -8 if out == torch.bfloat16 else 2.0 ** -23
+    tol = K * 2.0 ** -23 * sum_abs + out_u * np.abs(ref) + 1e-30
+    bad = np.abs(got - ref) > tol
+    assert not bad.any(), (int(bad.sum()), np.argwhere(bad)[0])
+
+
+@pytest.mark.parametrize("M,N,K,out", [(300, 520, 784, torch.bfloat16), (2148, 2100, 784, torch.float32)])
+def test_fp8_gemm_zero_operand_gives_the_bias(q, M, N, K, out):
+    """A = 0: every output is its column's bias rounded once to the output
+    type (0 * s + b is exact), so a bias taken from the wrong column, or an
+    output written to the wrong place, shows bit for bit."""
+    rng = np.random.Generator(np.random.PCG64(M + N))
+    A = torch.zeros((M, K), dtype=torch.uint8, device="cuda")
+    B = torch.from_numpy(rng.integers(0, 0x70, (N, K), dtype=np.uint8)).cuda()
+    bias = torch.from_numpy(rng.normal(0, 1, N).astype(np.float32)).cuda()
+    C = torch.full((M, N), 7.0, dtype=out, device="cuda")
+    one = torch.ones(1, device="cuda")
+    q.qlora_fp8_gemm(A, q.FP8_E4M3, B, q.FP8_E4M3, one, one, bias, C)
+    torch.cuda.synchronize()
+    want = bias.to(out)[None, :].expand(M, N)
+    assert torch.equal(C, want)
 
 
 @pytest.mark.parametrize("M,K,N,act", [(512, 768, 768, torch.bfloat16), (256, 1024, 320, torch.float32)])
