@@ -469,6 +469,23 @@ int qlora_fp8_quantize(const void* T, int rows, int cols, qlora_dtype dtype, qlo
                        const float* scale_in, float* scale_out, float* amax_history, int history_len,
                        uint8_t* q, uint8_t* qt, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Bytes of workspace qlora_fp8_quantize_colsum needs for T [rows, cols]
+ * (0 for an empty shape). */
+size_t qlora_fp8_colsum_workspace_bytes(int rows, int cols);
+
+/* qlora_fp8_quantize plus colsum[c] = sum_r T[r, c] in fp32 (the bias
+ * gradient when T is the output gradient dY), read in the same pass as the
+ * codes.  The sum's order is fixed (8-row runs, then 128-row tiles, then
+ * the tiles in order), so repeated calls give the same bits.  Needs T
+ * 16-byte aligned, cols % 8 == 0, q 8-byte aligned and qt NULL or 16-byte
+ * aligned with rows % 16 == 0 (else QLORA_EUNSUPPORTED); workspace: device
+ * memory, 256-byte aligned, of at least
+ * qlora_fp8_colsum_workspace_bytes(rows, cols) bytes. */
+int qlora_fp8_quantize_colsum(const void* T, int rows, int cols, qlora_dtype dtype, qlora_fp8_format fmt,
+                              const float* scale_in, float* scale_out, float* amax_history, int history_len,
+                              uint8_t* q, uint8_t* qt, float* colsum, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
 /* C [M,N] = (A B^T) * (*scale_a) * (*scale_b) (+ bias[n]), A [M,K] and
  * B [N,K] float8 codes (both K-major, K a multiple of 16), products on
  * tcgen05.mma.kind::f8f6f4 with fp32 accumulation; C in c_dtype (bf16

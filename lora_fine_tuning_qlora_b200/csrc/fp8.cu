@@ -143,14 +143,38 @@ __device__ __forceinline__ void transpose4x4(uint32_t w0, uint32_t w1, uint32_t 
     c3 = __byte_perm(t1, t3, 0x7632);
 }
 
-template <typename T, int FMT>
+// Column sums (CS): each thread adds its 8 columns over its 8 rows, the 16
+// threads of a column chunk are added in a fixed order through shared
+// memory, and the tile's sums go to part[row tile][col].  The last block of
+// a column strip to finish (a counter per strip; it resets the counter)
+// adds the strip's partials over the row tiles in a fixed order, so the
+// result does not depend on which block finishes last.
+__device__ __forceinline__ float sum_strided_cg(const float* p, size_t stride, int n) {
+    float s = 0.f;
+    int b = 0;
+    for (; b + 8 <= n; b += 8) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = __ldcg(p + (b + u) * stride);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) s += v[u];
+    }
+    for (; b < n; ++b) s += __ldcg(p + b * stride);
+    return s;
+}
+
+template <typename T, int FMT, bool CS>
 __global__ void __launch_bounds__(kFThreads) fp8_quantize_tiled_kernel(const T* __restrict__ src, int R, int Cc,
                                                                       const float* __restrict__ scale,
                                                                       uint8_t* __restrict__ q,
                                                                       uint8_t* __restrict__ qt,
-                                                                      unsigned int* __restrict__ amax_bits) {
+                                                                      unsigned int* __restrict__ amax_bits,
+                                                                      float* part, unsigned int* cnt,
+                                                                      float* __restrict__ colsum) {
     __shared__ __align__(16) uint32_t tile[kFR * kFC / 4];
+    __shared__ __align__(16) float csm[CS ? 16 * kFC : 1];
     __shared__ float wmax[kFThreads / 32];
+    __shared__ int last;
     pdl_trigger();
     pdl_wait();
     const int t = threadIdx.x;
@@ -168,6 +192,9 @@ __global__ void __launch_bounds__(kFThreads) fp8_quantize_tiled_kernel(const T* 
     }
     const float s = __ldg(scale);
     float mx = 0.f;
+    float cs[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) cs[i] = 0.f;
 #pragma unroll
     for (int u = 0; u < kFChunks; ++u) {
         const int row = t / 16 + 16 * u;
@@ -177,6 +204,7 @@ __global__ void __launch_bounds__(kFThreads) fp8_quantize_tiled_kernel(const T* 
         for (int i = 0; i < 8; ++i) {
             const float v = val8(raw[u], i, src);
             mx = fmaxf(mx, fabsf(v));
+            if constexpr (CS) cs[i] += v;
             x[i] = __fdiv_rn(v, s);
         }
         const uint32_t lo = cvt2<FMT>(x[0], x[1]) | (cvt2<FMT>(x[2], x[3]) << 16);
@@ -189,12 +217,43 @@ __global__ void __launch_bounds__(kFThreads) fp8_quantize_tiled_kernel(const T* 
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     if (t % 32 == 0) wmax[t / 32] = mx;
+    if constexpr (CS) {
+        float4* d = reinterpret_cast<float4*>(&csm[(t / 16) * kFC + 8 * j]);
+        d[0] = make_float4(cs[0], cs[1], cs[2], cs[3]);
+        d[1] = make_float4(cs[4], cs[5], cs[6], cs[7]);
+    }
     __syncthreads();
     if (t == 0) {
         float m = wmax[0];
 #pragma unroll
         for (int i = 1; i < kFThreads / 32; ++i) m = fmaxf(m, wmax[i]);
         atomicMax(amax_bits, __float_as_uint(m));
+    }
+    if constexpr (CS) {
+        if (t < kFC) {
+            float p = 0.f;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) p += csm[k * kFC + t];
+            if (c0 + t < Cc) part[static_cast<size_t>(blockIdx.x) * Cc + c0 + t] = p;
+        }
+        __threadfence();
+        __syncthreads();
+        if (t == 0) last = atomicAdd(&cnt[blockIdx.y], 1u) == gridDim.x - 1;
+        __syncthreads();
+        if (last) {
+            __threadfence();
+            // two threads a column: row tiles h, h + 2, .. each, then h = 0 + h = 1
+            const int col = t % kFC, h = t / kFC;
+            const int nrt = static_cast<int>(gridDim.x);
+            float v = 0.f;
+            if (c0 + col < Cc && h < nrt)
+                v = sum_strided_cg(part + static_cast<size_t>(h) * Cc + c0 + col, 2 * static_cast<size_t>(Cc),
+                                   (nrt - h + 1) / 2);
+            csm[h * kFC + col] = v;
+            __syncthreads();
+            if (h == 0 && c0 + col < Cc) colsum[c0 + col] = csm[col] + csm[kFC + col];
+            if (t == 0) cnt[blockIdx.y] = 0u;
+        }
     }
     if (qt) {
         const int seg = t % 8, c4 = t / 8;
@@ -619,30 +678,57 @@ __global__ void __launch_bounds__(kGThreads, 1)
 }
 }  // namespace
 
-cudaError_t launch_fp8_quantize(Act act, const void* T, int R, int Cc, const float* scale_in, float* scale_out,
-                                float* hist, int L, int fmt, uint8_t* q, uint8_t* qt, unsigned int* amax_word,
-                                cudaStream_t s) {
-    cudaError_t e = cudaMemsetAsync(amax_word, 0, sizeof(unsigned int), s);
-    if (e != cudaSuccess) return e;
+bool fp8_tiled_applies(const void* T, int R, int Cc, const uint8_t* q, const uint8_t* qt) {
     const auto al = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; };
-    const bool tiled = al(T, 16) && Cc % 8 == 0 && al(q, 8) && (!qt || (al(qt, 16) && R % 16 == 0)) &&
-                       (Cc + kFC - 1) / kFC <= 65535;
+    return al(T, 16) && Cc % 8 == 0 && al(q, 8) && (!qt || (al(qt, 16) && R % 16 == 0)) &&
+           (Cc + kFC - 1) / kFC <= 65535;
+}
+
+// workspace: the amax word; with column sums, a counter per 128-column strip
+// and, from the next 256-byte boundary, the partial sums [row tiles][Cc]
+static size_t colsum_part_offset(int Cc) {
+    const size_t head = 4 + 4 * static_cast<size_t>((Cc + kFC - 1) / kFC);
+    return (head + 255) / 256 * 256;
+}
+
+size_t fp8_colsum_ws_bytes(int R, int Cc) {
+    return colsum_part_offset(Cc) + 4 * static_cast<size_t>((R + kFR - 1) / kFR) * static_cast<size_t>(Cc);
+}
+
+cudaError_t launch_fp8_quantize(Act act, const void* T, int R, int Cc, const float* scale_in, float* scale_out,
+                                float* hist, int L, int fmt, uint8_t* q, uint8_t* qt, void* ws, float* colsum,
+                                cudaStream_t s) {
+    unsigned int* amax_word = static_cast<unsigned int*>(ws);
+    unsigned int* cnt = amax_word + 1;
+    float* part = colsum ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + colsum_part_offset(Cc)) : nullptr;
+    const size_t zero_bytes = colsum ? 4 + 4 * static_cast<size_t>((Cc + kFC - 1) / kFC) : 4;
+    cudaError_t e = cudaMemsetAsync(ws, 0, zero_bytes, s);
+    if (e != cudaSuccess) return e;
+    const bool tiled = fp8_tiled_applies(T, R, Cc, q, qt);
+    if (colsum && !tiled) return cudaErrorInvalidValue;
     if (tiled) {
         const dim3 grid((R + kFR - 1) / kFR, (Cc + kFC - 1) / kFC);
-        if (act == kBF16) {
-            const auto* src = static_cast<const __nv_bfloat16*>(T);
-            e = fmt == kFp8E4M3
-                    ? launch_k(fp8_quantize_tiled_kernel<__nv_bfloat16, kFp8E4M3>, grid, dim3(kFThreads), 0, s, 1,
-                               src, R, Cc, scale_in, q, qt, amax_word)
-                    : launch_k(fp8_quantize_tiled_kernel<__nv_bfloat16, kFp8E5M2>, grid, dim3(kFThreads), 0, s, 1,
-                               src, R, Cc, scale_in, q, qt, amax_word);
+        auto go = [&](auto kern, auto src) {
+            return launch_k(kern, grid, dim3(kFThreads), 0, s, 1, src, R, Cc, scale_in, q, qt, amax_word, part, cnt,
+                            colsum);
+        };
+        const auto* sb = static_cast<const __nv_bfloat16*>(T);
+        const auto* sf = static_cast<const float*>(T);
+        const bool e4 = fmt == kFp8E4M3;
+        if (colsum) {
+            if (act == kBF16)
+                e = e4 ? go(fp8_quantize_tiled_kernel<__nv_bfloat16, kFp8E4M3, true>, sb)
+                       : go(fp8_quantize_tiled_kernel<__nv_bfloat16, kFp8E5M2, true>, sb);
+            else
+                e = e4 ? go(fp8_quantize_tiled_kernel<float, kFp8E4M3, true>, sf)
+                       : go(fp8_quantize_tiled_kernel<float, kFp8E5M2, true>, sf);
         } else {
-            const auto* src = static_cast<const float*>(T);
-            e = fmt == kFp8E4M3
-                    ? launch_k(fp8_quantize_tiled_kernel<float, kFp8E4M3>, grid, dim3(kFThreads), 0, s, 1, src, R,
-                               Cc, scale_in, q, qt, amax_word)
-                    : launch_k(fp8_quantize_tiled_kernel<float, kFp8E5M2>, grid, dim3(kFThreads), 0, s, 1, src, R,
-                               Cc, scale_in, q, qt, amax_word);
+            if (act == kBF16)
+                e = e4 ? go(fp8_quantize_tiled_kernel<__nv_bfloat16, kFp8E4M3, false>, sb)
+                       : go(fp8_quantize_tiled_kernel<__nv_bfloat16, kFp8E5M2, false>, sb);
+            else
+                e = e4 ? go(fp8_quantize_tiled_kernel<float, kFp8E4M3, false>, sf)
+                       : go(fp8_quantize_tiled_kernel<float, kFp8E5M2, false>, sf);
         }
     } else {
         if ((Cc + kQT - 1) / kQT > 65535) return cudaErrorInvalidValue;

@@ -120,10 +120,18 @@ constexpr int kFp8E4M3 = 0;
 constexpr int kFp8E5M2 = 1;
 // Codes of T [R, Cc] with the stored scale *scale_in (row-major q and, if
 // qt != null, transposed qt [Cc, R]); then *scale_out and the history hist
-// [L] of delayed scaling.  amax_word: one word of device scratch.
+// [L] of delayed scaling.  ws: device scratch (the amax word; with column
+// sums, fp8_colsum_ws_bytes).  colsum [Cc] (optional): the column sums of T
+// in fp32.
 cudaError_t launch_fp8_quantize(Act act, const void* T, int R, int Cc, const float* scale_in, float* scale_out,
-                                float* hist, int L, int fmt, uint8_t* q, uint8_t* qt, unsigned int* amax_word,
+                                float* hist, int L, int fmt, uint8_t* q, uint8_t* qt, void* ws, float* colsum,
                                 cudaStream_t s);
+// Whether the 128 x 128 tiled quantizer takes this layout (T 16-byte
+// aligned, Cc % 8 == 0, q 8-byte aligned, qt null or 16-byte aligned with
+// R % 16 == 0); column sums need it.
+bool fp8_tiled_applies(const void* T, int R, int Cc, const uint8_t* q, const uint8_t* qt);
+// Workspace bytes of a quantization with column sums of T [R, Cc].
+size_t fp8_colsum_ws_bytes(int R, int Cc);
 // C [M,N] = (A [M,K] B [N,K]^T) * sa * sb (+ bias [N]); K-major fp8 codes.
 cudaError_t launch_fp8_gemm(const uint8_t* A, int afmt, const uint8_t* B, int bfmt, int M, int N, int K,
                             const float* sa, const float* sb, const float* bias, void* C, Act out, int* status,

@@ -826,9 +826,39 @@ int qlora_fp8_quantize(const void* T, int rows, int cols, qlora_dtype dtype, qlo
     QL_REQUIRE(workspace_bytes >= QLORA_FP8_WORKSPACE_BYTES, QLORA_EINVAL, "workspace too small");
     return cuda_status(launch_fp8_quantize(dtype == QLORA_BF16 ? kBF16 : kF32, T, rows, cols, scale_in,
                                            scale_out, amax_history, history_len,
-                                           fmt == QLORA_FP8_E4M3 ? kFp8E4M3 : kFp8E5M2, q, qt,
-                                           static_cast<unsigned int*>(workspace),
-                                           static_cast<cudaStream_t>(stream)),
+                                           fmt == QLORA_FP8_E4M3 ? kFp8E4M3 : kFp8E5M2, q, qt, workspace,
+                                           nullptr, static_cast<cudaStream_t>(stream)),
+                       "float8 quantizer launch");
+}
+
+size_t qlora_fp8_colsum_workspace_bytes(int rows, int cols) {
+    if (rows < 1 || cols < 1) return 0;
+    return fp8_colsum_ws_bytes(rows, cols);
+}
+
+int qlora_fp8_quantize_colsum(const void* T, int rows, int cols, qlora_dtype dtype, qlora_fp8_format fmt,
+                              const float* scale_in, float* scale_out, float* amax_history, int history_len,
+                              uint8_t* q, uint8_t* qt, float* colsum, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+    QL_REQUIRE(T && scale_in && scale_out && amax_history && q && colsum && workspace, QLORA_EINVAL,
+               "NULL pointer argument");
+    QL_REQUIRE(rows >= 1 && cols >= 1 && history_len >= 1, QLORA_ESHAPE,
+               "rows, cols and history_len must be >= 1");
+    QL_REQUIRE(static_cast<long long>(rows) * cols < (1LL << 40), QLORA_ESHAPE, "tensor too large");
+    QL_REQUIRE(dtype == QLORA_F32 || dtype == QLORA_BF16, QLORA_EINVAL, "unknown dtype");
+    QL_REQUIRE(fmt == QLORA_FP8_E4M3 || fmt == QLORA_FP8_E5M2, QLORA_EINVAL, "unknown float8 format");
+    QL_REQUIRE(scale_out != scale_in, QLORA_EINVAL, "scale_out must not alias scale_in");
+    QL_REQUIRE(aligned(scale_in, 4) && aligned(scale_out, 4) && aligned(amax_history, 4) && aligned(colsum, 4) &&
+                   aligned(workspace, 256),
+               QLORA_EALIGN, "misaligned pointer (workspace: 256 bytes)");
+    QL_REQUIRE(fp8_tiled_applies(T, rows, cols, q, qt), QLORA_EUNSUPPORTED,
+               "column sums need T 16-byte aligned, cols % 8 == 0, q 8-byte aligned and qt NULL or 16-byte "
+               "aligned with rows % 16 == 0");
+    QL_REQUIRE(workspace_bytes >= fp8_colsum_ws_bytes(rows, cols), QLORA_EINVAL, "workspace too small");
+    return cuda_status(launch_fp8_quantize(dtype == QLORA_BF16 ? kBF16 : kF32, T, rows, cols, scale_in,
+                                           scale_out, amax_history, history_len,
+                                           fmt == QLORA_FP8_E4M3 ? kFp8E4M3 : kFp8E5M2, q, qt, workspace,
+                                           colsum, static_cast<cudaStream_t>(stream)),
                        "float8 quantizer launch");
 }
 

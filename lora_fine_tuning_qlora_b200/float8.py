@@ -28,18 +28,27 @@ class Fp8State:
         self.history = torch.zeros(history_len, dtype=torch.float32, device=device)
         self.cur = 0
         self.ws = torch.empty(qlora.FP8_WORKSPACE_BYTES, dtype=torch.uint8, device=device)
+        self.cs_ws = None  # workspace of the quantization with column sums, grown on demand
 
     @property
     def scale(self) -> torch.Tensor:
         """The scale the next quantization uses (a one-element view)."""
         return self.scales[self.cur:self.cur + 1]
 
-    def quantize(self, T: torch.Tensor, fmt: int, q: torch.Tensor, qt: Optional[torch.Tensor]):
-        """Codes of T; returns the scale they were made with (a view that
-        stays valid until the state's second-next quantization)."""
+    def quantize(self, T: torch.Tensor, fmt: int, q: torch.Tensor, qt: Optional[torch.Tensor],
+                 colsum: Optional[torch.Tensor] = None):
+        """Codes of T (and, if colsum is given, T's column sums from the same
+        pass); returns the scale they were made with (a view that stays valid
+        until the state's second-next quantization)."""
         used = self.scales[self.cur:self.cur + 1]
         nxt = self.scales[1 - self.cur:2 - self.cur]
-        qlora.qlora_fp8_quantize(T, fmt, used, nxt, self.history, q, qt, self.ws)
+        if colsum is None:
+            qlora.qlora_fp8_quantize(T, fmt, used, nxt, self.history, q, qt, self.ws)
+        else:
+            need = qlora.qlora_fp8_colsum_workspace_bytes(*T.shape)
+            if self.cs_ws is None or self.cs_ws.numel() < need:
+                self.cs_ws = torch.empty(need, dtype=torch.uint8, device=T.device)
+            qlora.qlora_fp8_quantize_colsum(T, fmt, used, nxt, self.history, q, qt, colsum, self.cs_ws)
         self.cur = 1 - self.cur
         return used
 
@@ -78,7 +87,11 @@ class Float8Dense:
         dev = dY.device
         Gq = torch.empty((M, self.N), dtype=torch.uint8, device=dev)
         GqT = torch.empty((self.N, M), dtype=torch.uint8, device=dev)
-        s_g = self.sg.quantize(dY, qlora.FP8_E5M2, Gq, GqT)
+        # dbias = column sums of dY: from the quantizer's own pass where its
+        # layout allows, else by the library's column-sum pass below
+        fused = self.bias is not None and qlora.fp8_colsum_applies(dY, Gq, GqT)
+        dbias = torch.empty((self.N,), dtype=torch.float32, device=dev) if fused else None
+        s_g = self.sg.quantize(dY, qlora.FP8_E5M2, Gq, GqT, dbias)
         out = {"Gq": Gq, "s_g": s_g}
         if want_dx:
             dX = torch.empty((M, self.K), dtype=self.act, device=dev)
@@ -87,7 +100,9 @@ class Float8Dense:
         dW = torch.empty((self.K, self.N), dtype=torch.float32, device=dev)
         qlora.qlora_fp8_gemm(ctx["XqT"], qlora.FP8_E4M3, GqT, qlora.FP8_E5M2, ctx["s_x"], s_g, None, dW)
         out["dW"] = dW
-        if self.bias is not None:
+        if fused:
+            out["dbias"] = dbias
+        elif self.bias is not None:
             # column sums of dY by the library's pass (its dB output, for a
             # rank-1 factor of zeros, is discarded)
             d = qlora.desc(16, self.N, 1, 1.0, dY.dtype)

@@ -36,7 +36,8 @@ EXPORTED = ("qlora_quantize_weight", "qlora_workspace_bytes", "qlora_forward",
             "qlora_gemm_dx_int4", "qlora_merge_int4", "qlora_gemm_forward_int4",
             "qlora_outlier_cap", "qlora_outlier_workspace_bytes", "qlora_outlier_quantize",
             "qlora_outlier_forward", "qlora_outlier_backward", "qlora_permute",
-            "qlora_fp8_quantize", "qlora_fp8_gemm")
+            "qlora_fp8_quantize", "qlora_fp8_gemm", "qlora_fp8_colsum_workspace_bytes",
+            "qlora_fp8_quantize_colsum")
 
 
 class QLoraError(RuntimeError):
@@ -127,6 +128,10 @@ def _load():
         f.restype = I
     lib.qlora_fp8_quantize.argtypes = [P, I, I, I, I, P, P, P, I, P, P, P, Z, P]
     lib.qlora_fp8_quantize.restype = I
+    lib.qlora_fp8_colsum_workspace_bytes.argtypes = [I, I]
+    lib.qlora_fp8_colsum_workspace_bytes.restype = Z
+    lib.qlora_fp8_quantize_colsum.argtypes = [P, I, I, I, I, P, P, P, I, P, P, P, P, Z, P]
+    lib.qlora_fp8_quantize_colsum.restype = I
     lib.qlora_fp8_gemm.argtypes = [P, I, P, I, I, I, I, P, P, P, P, I, P]
     lib.qlora_fp8_gemm.restype = I
     lib.qlora_permute.argtypes = [P, P, I, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int), I, P]
@@ -445,6 +450,30 @@ def qlora_fp8_quantize(T: torch.Tensor, fmt: int, scale_in, scale_out, history, 
     _check(_lib.qlora_fp8_quantize(_ptr(T), rows, cols, act_code(T.dtype), int(fmt), _ptr(scale_in),
                                    _ptr(scale_out), _ptr(history), history.numel(), _ptr(q), _ptr(qt),
                                    _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def qlora_fp8_colsum_workspace_bytes(rows: int, cols: int) -> int:
+    return int(_lib.qlora_fp8_colsum_workspace_bytes(int(rows), int(cols)))
+
+
+def fp8_colsum_applies(T: torch.Tensor, q: torch.Tensor, qt=None) -> bool:
+    """Whether qlora_fp8_quantize_colsum takes these tensors (its layout
+    condition, checked here so a caller can choose another route)."""
+    rows, cols = T.shape
+    ok = T.data_ptr() % 16 == 0 and cols % 8 == 0 and q.data_ptr() % 8 == 0
+    if qt is not None:
+        ok = ok and qt.data_ptr() % 16 == 0 and rows % 16 == 0
+    return bool(ok)
+
+
+def qlora_fp8_quantize_colsum(T: torch.Tensor, fmt: int, scale_in, scale_out, history, q, qt, colsum, ws,
+                              stream=None):
+    """qlora_fp8_quantize plus colsum [cols] = column sums of T (fp32), in
+    the same pass; ws: qlora_fp8_colsum_workspace_bytes(rows, cols) bytes."""
+    rows, cols = T.shape
+    _check(_lib.qlora_fp8_quantize_colsum(_ptr(T), rows, cols, act_code(T.dtype), int(fmt), _ptr(scale_in),
+                                          _ptr(scale_out), _ptr(history), history.numel(), _ptr(q), _ptr(qt),
+                                          _ptr(colsum), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def qlora_fp8_gemm(A, fmt_a: int, B, fmt_b: int, scale_a, scale_b, bias, C, stream=None):

@@ -180,6 +180,19 @@ def test_new_entry_points_reject_bad_arguments(q):
                                        ctypes.c_int, P, P, P, ctypes.c_size_t, P]
     assert lib.qlora_fp8_quantize(fake, 4, 4, 1, 0, fake, fake, P(8192), 16, P(12288), None, P(16384), 256,
                                   None) == -1
+    # float8 quantizer with column sums: layout it cannot take, short workspace
+    lib.qlora_fp8_quantize_colsum.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P,
+                                              P, ctypes.c_int, P, P, P, P, ctypes.c_size_t, P]
+    need = q.qlora_fp8_colsum_workspace_bytes(300, 64)
+    assert need == 256 + 4 * 3 * 64 and q.qlora_fp8_colsum_workspace_bytes(0, 64) == 0
+    assert lib.qlora_fp8_quantize_colsum(fake, 300, 60, 1, 0, P(8192), P(8196), P(8448), 16, P(12288), None,
+                                         P(16384), P(32768), need, None) == -5   # cols % 8 != 0
+    assert lib.qlora_fp8_quantize_colsum(fake, 300, 64, 1, 0, P(8192), P(8196), P(8448), 16, P(12288),
+                                         P(65536), P(16384), P(32768), need, None) == -5  # rows % 16 != 0 with qt
+    assert lib.qlora_fp8_quantize_colsum(fake, 300, 64, 1, 0, P(8192), P(8196), P(8448), 16, P(12288), None,
+                                         P(16384), P(32768), need - 1, None) == -1
+    assert lib.qlora_fp8_quantize_colsum(fake, 300, 64, 1, 0, P(8192), P(8196), P(8448), 16, P(12288), None,
+                                         P(16384), P(32772), need, None) == -2   # workspace not 256-aligned
     # outlier kernel: capacity below the bound, NULL member
     cap = q.qlora_outlier_cap(256, 256)
     assert cap == (int((256 * 256 - 1) * 0.1 / 100) + 1) + (256 * 256 - 1 - int((256 * 256 - 1) * 99.9 / 100))

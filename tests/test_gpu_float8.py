@@ -66,6 +66,44 @@ def test_quantize_state_bit_exact(q, R, C, dtype, fmt, scale, L, with_qt):
     np.testing.assert_array_equal(to_np(h), new["history"])
 
 
+@pytest.mark.parametrize("R,C,dtype,fmt", [
+    (4096, 520, torch.bfloat16, f8.E5M2),   # 32 row tiles; ragged last column strip
+    (304, 1000, torch.float32, f8.E4M3),    # ragged row and column tiles
+    (16, 8, torch.bfloat16, f8.E5M2),       # one partial tile
+])
+def test_quantize_colsum(q, R, C, dtype, fmt):
+    """Codes, scale and history as without column sums; the sums within the
+    fp32 bound R u sum_r |T[r, c]| (u = 2^-24, 2u allowed) of the exact
+    column sums, and identical bits on a second call."""
+    rng = np.random.Generator(np.random.PCG64(R * C))
+    T = rng.normal(0, 1, (R, C)).astype(np.float32) + rng.normal(0, 3, C).astype(np.float32)[None, :]
+    Tt = torch.from_numpy(T).to(dtype).cuda()
+    Tv = to_np(Tt).astype(np.float64)
+    hist = (rng.random(8) * 5).astype(np.float32)
+    outs = []
+    for _ in range(2):
+        s_in = torch.tensor([0.05], device="cuda")
+        s_out = torch.zeros(1, device="cuda")
+        h = torch.from_numpy(hist).cuda()
+        qq = torch.empty((R, C), dtype=torch.uint8, device="cuda")
+        qt = torch.empty((C, R), dtype=torch.uint8, device="cuda")
+        cs = torch.full((C,), np.nan, dtype=torch.float32, device="cuda")
+        ws = torch.empty(q.qlora_fp8_colsum_workspace_bytes(R, C), dtype=torch.uint8, device="cuda")
+        q.qlora_fp8_quantize_colsum(Tt, _fmt(q, fmt), s_in, s_out, h, qq, qt, cs, ws)
+        torch.cuda.synchronize()
+        outs.append((qq.cpu().numpy(), qt.cpu().numpy(), to_np(s_out)[0], to_np(h), to_np(cs)))
+    codes, _, new = f8.step_tensor(Tv.astype(np.float32), {"scale": np.float32(0.05), "history": hist}, fmt)
+    qq, qt, s1, h1, cs = outs[0]
+    np.testing.assert_array_equal(qq, codes)
+    np.testing.assert_array_equal(qt, codes.T)
+    assert s1 == new["scale"]
+    np.testing.assert_array_equal(h1, new["history"])
+    ref = Tv.sum(axis=0)
+    bound = R * 2.0 ** -23 * np.abs(Tv).sum(axis=0) + 1e-30
+    assert np.all(np.abs(cs - ref) <= bound), np.abs(cs - ref).max()
+    np.testing.assert_array_equal(outs[1][4], cs)
+
+
 def test_zero_history_keeps_the_scale(q):
     T = torch.zeros((32, 32), dtype=torch.bfloat16, device="cuda")
     s_in = torch.tensor([0.5], device="cuda")
