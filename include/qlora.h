@@ -475,8 +475,8 @@ size_t qlora_fp8_colsum_workspace_bytes(int rows, int cols);
 
 /* qlora_fp8_quantize plus colsum[c] = sum_r T[r, c] in fp32 (the bias
  * gradient when T is the output gradient dY), read in the same pass as the
- * codes.  The sum's order is fixed (8-row runs, then 128-row tiles, then
- * the tiles in order), so repeated calls give the same bits.  Needs T
+ * codes.  The sum's order is fixed (within each 128-row tile, then over the
+ * tiles by a second, small kernel), so repeated calls give the same bits.  Needs T
  * 16-byte aligned, cols % 8 == 0, q 8-byte aligned and qt NULL or 16-byte
  * aligned with rows % 16 == 0 (else QLORA_EUNSUPPORTED); workspace: device
  * memory, 256-byte aligned, of at least

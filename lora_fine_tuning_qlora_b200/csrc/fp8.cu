@@ -145,36 +145,21 @@ __device__ __forceinline__ void transpose4x4(uint32_t w0, uint32_t w1, uint32_t 
 
 // Column sums (CS): each thread adds its 8 columns over its 8 rows, the 16
 // threads of a column chunk are added in a fixed order through shared
-// memory, and the tile's sums go to part[row tile][col].  The last block of
-// a column strip to finish (a counter per strip; it resets the counter)
-// adds the strip's partials over the row tiles in a fixed order, so the
-// result does not depend on which block finishes last.
-__device__ __forceinline__ float sum_strided_cg(const float* p, size_t stride, int n) {
-    float s = 0.f;
-    int b = 0;
-    for (; b + 8 <= n; b += 8) {
-        float v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = __ldcg(p + (b + u) * stride);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) s += v[u];
-    }
-    for (; b < n; ++b) s += __ldcg(p + b * stride);
-    return s;
-}
-
+// memory, and the tile's sums go to part[row tile][col]; a second kernel
+// (fp8_colsum_kernel) adds each column's partials over the row tiles in a
+// fixed order.  (Doing that last step in the last block of each column strip needs
+// a device-scope fence in every block, which measured slower than the extra
+// launch.)
 template <typename T, int FMT, bool CS>
 __global__ void __launch_bounds__(kFThreads) fp8_quantize_tiled_kernel(const T* __restrict__ src, int R, int Cc,
                                                                       const float* __restrict__ scale,
                                                                       uint8_t* __restrict__ q,
                                                                       uint8_t* __restrict__ qt,
                                                                       unsigned int* __restrict__ amax_bits,
-                                                                      float* part, unsigned int* cnt,
-                                                                      float* __restrict__ colsum) {
+                                                                      float* __restrict__ part) {
     __shared__ __align__(16) uint32_t tile[kFR * kFC / 4];
     __shared__ __align__(16) float csm[CS ? 16 * kFC : 1];
     __shared__ float wmax[kFThreads / 32];
-    __shared__ int last;
     pdl_trigger();
     pdl_wait();
     const int t = threadIdx.x;
@@ -236,24 +221,6 @@ __global__ void __launch_bounds__(kFThreads) fp8_quantize_tiled_kernel(const T* 
             for (int k = 0; k < 16; ++k) p += csm[k * kFC + t];
             if (c0 + t < Cc) part[static_cast<size_t>(blockIdx.x) * Cc + c0 + t] = p;
         }
-        __threadfence();
-        __syncthreads();
-        if (t == 0) last = atomicAdd(&cnt[blockIdx.y], 1u) == gridDim.x - 1;
-        __syncthreads();
-        if (last) {
-            __threadfence();
-            // two threads a column: row tiles h, h + 2, .. each, then h = 0 + h = 1
-            const int col = t % kFC, h = t / kFC;
-            const int nrt = static_cast<int>(gridDim.x);
-            float v = 0.f;
-            if (c0 + col < Cc && h < nrt)
-                v = sum_strided_cg(part + static_cast<size_t>(h) * Cc + c0 + col, 2 * static_cast<size_t>(Cc),
-                                   (nrt - h + 1) / 2);
-            csm[h * kFC + col] = v;
-            __syncthreads();
-            if (h == 0 && c0 + col < Cc) colsum[c0 + col] = csm[col] + csm[kFC + col];
-            if (t == 0) cnt[blockIdx.y] = 0u;
-        }
     }
     if (qt) {
         const int seg = t % 8, c4 = t / 8;
@@ -275,6 +242,42 @@ __global__ void __launch_bounds__(kFThreads) fp8_quantize_tiled_kernel(const T* 
                         make_uint4(col[jj][0], col[jj][1], col[jj][2], col[jj][3]);
             }
         }
+    }
+}
+
+// colsum[c] = sum over row tiles of part[t][c] in a fixed order: a block
+// takes 32 columns; its eight warps each add one eighth of the row tiles
+// (ascending, eight loads in flight), then one warp adds the eight sums in
+// warp order.
+constexpr int kCsCols = 32, kCsWarps = 8;
+__global__ void __launch_bounds__(32 * kCsWarps) fp8_colsum_kernel(const float* __restrict__ part, int nrt, int Cc,
+                                                                  float* __restrict__ colsum) {
+    __shared__ float sums[kCsWarps][kCsCols];
+    pdl_trigger();
+    pdl_wait();
+    const int lane = threadIdx.x % 32, w = threadIdx.x / 32;
+    const int c = blockIdx.x * kCsCols + lane;
+    const int per = (nrt + kCsWarps - 1) / kCsWarps;
+    const int t0 = w * per, t1 = min(nrt, t0 + per);
+    float v = 0.f;
+    if (c < Cc) {
+        int t = t0;
+        for (; t + 8 <= t1; t += 8) {
+            float x[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) x[u] = __ldg(part + static_cast<size_t>(t + u) * Cc + c);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v += x[u];
+        }
+        for (; t < t1; ++t) v += __ldg(part + static_cast<size_t>(t) * Cc + c);
+    }
+    sums[w][lane] = v;
+    __syncthreads();
+    if (w == 0 && c < Cc) {
+        float a = sums[0][lane];
+#pragma unroll
+        for (int k = 1; k < kCsWarps; ++k) a += sums[k][lane];
+        colsum[c] = a;
     }
 }
 
@@ -684,12 +687,9 @@ bool fp8_tiled_applies(const void* T, int R, int Cc, const uint8_t* q, const uin
            (Cc + kFC - 1) / kFC <= 65535;
 }
 
-// workspace: the amax word; with column sums, a counter per 128-column strip
-// and, from the next 256-byte boundary, the partial sums [row tiles][Cc]
-static size_t colsum_part_offset(int Cc) {
-    const size_t head = 4 + 4 * static_cast<size_t>((Cc + kFC - 1) / kFC);
-    return (head + 255) / 256 * 256;
-}
+// workspace: the amax word; with column sums, from byte 256 the partial sums
+// [row tiles][Cc]
+static size_t colsum_part_offset(int) { return 256; }
 
 size_t fp8_colsum_ws_bytes(int R, int Cc) {
     return colsum_part_offset(Cc) + 4 * static_cast<size_t>((R + kFR - 1) / kFR) * static_cast<size_t>(Cc);
@@ -699,18 +699,15 @@ cudaError_t launch_fp8_quantize(Act act, const void* T, int R, int Cc, const flo
                                 float* hist, int L, int fmt, uint8_t* q, uint8_t* qt, void* ws, float* colsum,
                                 cudaStream_t s) {
     unsigned int* amax_word = static_cast<unsigned int*>(ws);
-    unsigned int* cnt = amax_word + 1;
     float* part = colsum ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + colsum_part_offset(Cc)) : nullptr;
-    const size_t zero_bytes = colsum ? 4 + 4 * static_cast<size_t>((Cc + kFC - 1) / kFC) : 4;
-    cudaError_t e = cudaMemsetAsync(ws, 0, zero_bytes, s);
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(unsigned int), s);
     if (e != cudaSuccess) return e;
     const bool tiled = fp8_tiled_applies(T, R, Cc, q, qt);
     if (colsum && !tiled) return cudaErrorInvalidValue;
     if (tiled) {
         const dim3 grid((R + kFR - 1) / kFR, (Cc + kFC - 1) / kFC);
         auto go = [&](auto kern, auto src) {
-            return launch_k(kern, grid, dim3(kFThreads), 0, s, 1, src, R, Cc, scale_in, q, qt, amax_word, part, cnt,
-                            colsum);
+            return launch_k(kern, grid, dim3(kFThreads), 0, s, 1, src, R, Cc, scale_in, q, qt, amax_word, part);
         };
         const auto* sb = static_cast<const __nv_bfloat16*>(T);
         const auto* sf = static_cast<const float*>(T);
@@ -740,6 +737,11 @@ cudaError_t launch_fp8_quantize(Act act, const void* T, int R, int Cc, const flo
                            Cc, scale_in, fmt, q, qt, amax_word);
     }
     if (e != cudaSuccess) return e;
+    if (colsum) {
+        e = launch_k(fp8_colsum_kernel, dim3((Cc + kCsCols - 1) / kCsCols), dim3(32 * kCsWarps), 0, s, 1,
+                     static_cast<const float*>(part), (R + kFR - 1) / kFR, Cc, colsum);
+        if (e != cudaSuccess) return e;
+    }
     const float fmax = fmt == kFp8E4M3 ? 448.0f : 57344.0f;
     return launch_k(fp8_state_kernel, dim3(1), dim3(1024), 0, s, 1, static_cast<const unsigned int*>(amax_word),
                     scale_in, scale_out, hist, L, fmax);
