@@ -55,6 +55,7 @@ constexpr int kWorkers = 4;
 constexpr int kThreads = 64 + 32 * kWorkers;
 constexpr int kMaxCluster = 8;
 constexpr uint32_t kTabSbo = (kTileCols / 8) * 128;  // 8-row group stride of a 128-wide table
+constexpr int kMaxBulkR = 8;                         // rank limit of the bulk-copied V rows
 
 // What one launch computes.
 struct Parts {
@@ -73,14 +74,16 @@ struct RankTcArgs {
     int M, C, r;
     int tiles_per_cta;   // 128-row tiles per CTA
     float c;
+    int vbulk;           // column sums, one V slice, r % 4 == 0, r <= kMaxBulkR, V 16-byte aligned:
+                         // V's tile rows arrive by bulk copy, issued with the tile's
 };
 
 // Shared-memory and TMEM layout for rank r (same on host and device).
 struct RtLayout {
     int RP, NG, NV, JP;
-    uint32_t vtab, bcat, recv, bar, total;
+    uint32_t vtab, bcat, recv, bar, vraw, vslot, total;
     uint32_t tmem_cols, d_col, g_col;
-    __host__ __device__ RtLayout(Parts p, int r) {
+    __host__ __device__ RtLayout(Parts p, int r, bool vbulk) {
         RP = (r + 15) / 16 * 16;
         NG = p.g ? 2 * RP : 0;
         NV = p.d ? 2 * RP + (p.ones ? 16 : 0) : 0;
@@ -89,7 +92,9 @@ struct RtLayout {
         bcat = vtab + 2 * static_cast<uint32_t>(NV) * 256;
         recv = bcat + static_cast<uint32_t>(NG) * 256;
         bar = recv + (((kTileCols + kMaxCluster) * JP * 4 + 15) / 16) * 16;
-        total = bar + 128;
+        vraw = bar + 128;  // [2][128 rows][r] fp32 with vbulk
+        vslot = vbulk ? static_cast<uint32_t>(kTileRows * r * 4) : 0u;
+        total = vraw + 2 * vslot;
         d_col = 0;
         g_col = static_cast<uint32_t>(NV);
         const uint32_t need = static_cast<uint32_t>(NV + 2 * NG);
@@ -120,7 +125,7 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    const RtLayout L(Parts{kG, kD, kOnes}, a.r);
+    const RtLayout L(Parts{kG, kD, kOnes}, a.r, kD && a.vbulk);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar);
     uint64_t* full = bars;        // [2] tile landed
     uint64_t* vready = bars + 2;  // [2] Vcat table written
@@ -129,7 +134,8 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
     uint64_t* gempty = bars + 8;  // [2] G accumulator read out
     uint64_t* dfull = bars + 10;  // column accumulator final
     uint64_t* rbar = bars + 11;   // every CTA of the cluster delivered this CTA's column slice
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+    uint64_t* vfull = bars + 12;  // [2] vbulk: the tile's V rows landed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
     // recv[q][c][j]: partial of CTA q for column cbeg + c of this CTA's slice
     float* recv = reinterpret_cast<float*>(smem + L.recv);
 
@@ -158,6 +164,7 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
             mbar_init(&empty[s], 1);
             mbar_init(&gfull[s], 1);
             mbar_init(&gempty[s], kWorkers);
+            mbar_init(&vfull[s], 1);
         }
         mbar_init(dfull, 1);
         mbar_init(rbar, static_cast<uint32_t>(CL * (cend > cbeg ? cend - cbeg : 1)));
@@ -184,6 +191,13 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
                 if (i >= 2 && !mbar_wait(&empty[s], ((i >> 1) - 1) & 1, status)) break;
                 uint8_t* dst = smem + s * kTileBytes;
                 const int m0 = (t0 + i) * kTileRows;
+                // with vbulk, the tile's rows of V (16-byte multiples: r % 4 == 0) first, on a
+                // barrier of their own, so the V table is written while the tile is in flight
+                if (kD && a.vbulk) {
+                    const uint32_t vbytes = static_cast<uint32_t>(min(kTileRows, a.M - m0) * a.r * 4);
+                    mbar_arrive_expect_tx(&vfull[s], vbytes);
+                    bulk_load(smem + L.vraw + s * L.vslot, a.V + static_cast<size_t>(m0) * a.r, vbytes, &vfull[s]);
+                }
                 mbar_arrive_expect_tx(&full[s], kTileBytes);
                 if (t3d) {  // both 64-column blocks in one box
                     tma_load_3d(dst, &tmT, &full[s], 0, m0, col0 / kBoxCols);
@@ -309,6 +323,23 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
         if constexpr (kD) {
             // rows of V in whole 8-float groups at 16-byte alignment
             const bool vec4 = (a.r % 8) == 0 && (reinterpret_cast<uintptr_t>(a.V) & 15) == 0;
+            const int tw = threadIdx.x - 64;  // 0 .. 127
+            if (a.vbulk) {
+                // the parts of both V tables that no tile changes: zero rows
+                // beyond r in the head and remainder halves, and the ones block
+                // (a ones row, then zeros; the tile's rows past M are zero, so
+                // their ones add nothing), as 16-byte chunks of 8 tile rows
+                const int nconst = L.NV - 2 * a.r;
+                for (int idx = tw; idx < 2 * nconst * 16; idx += 32 * kWorkers) {
+                    const int b = idx / (nconst * 16), rem = idx % (nconst * 16);
+                    const int jj = rem / 16, kg = rem % 16;
+                    const int j = jj < L.RP - a.r ? a.r + jj : (jj < 2 * (L.RP - a.r) ? L.RP + a.r + jj - (L.RP - a.r)
+                                                                                      : 2 * L.RP + jj - 2 * (L.RP - a.r));
+                    const uint32_t w = (kOnes && j == 2 * L.RP) ? 0x3F803F80u : 0u;  // bf16 1.0 pairs
+                    *reinterpret_cast<uint4*>(smem + L.vtab + b * L.NV * 256 + ktab_off(j, 8 * kg)) =
+                        make_uint4(w, w, w, w);
+                }
+            }
             for (int i = 0; i < nt && ok; ++i) {
                 const int s = i & 1;
                 const int m = (t0 + i) * kTileRows + rr;
@@ -317,6 +348,37 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
                 if (!ok) break;
                 uint8_t* vt = smem + L.vtab + s * L.NV * 256;
                 const bool mok = m < a.M;
+                if (a.vbulk) {
+                    // the tile's V rows have landed: chunk (j, kg) of the head and
+                    // remainder tables from rows 8 kg .. 8 kg + 7
+                    ok = __all_sync(0xffffffffu, mbar_wait(&vfull[s], (i >> 1) & 1, status));
+                    if (!ok) break;
+                    const float* vr = reinterpret_cast<const float*>(smem + L.vraw + s * L.vslot);
+                    const int mt0 = (t0 + i) * kTileRows;
+                    for (int idx = tw; idx < a.r * 16; idx += 32 * kWorkers) {
+                        const int kg = idx / a.r, j = idx % a.r;
+                        uint32_t hi[4], lo[4];
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            float v2[2];
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                const int row = 8 * kg + 2 * e2 + h;
+                                v2[h] = mt0 + row < a.M ? vr[row * a.r + j] : 0.f;
+                            }
+                            const __nv_bfloat16 h0 = __float2bfloat16_rn(v2[0]), h1 = __float2bfloat16_rn(v2[1]);
+                            const __nv_bfloat16 l0 = __float2bfloat16_rn(v2[0] - __bfloat162float(h0));
+                            const __nv_bfloat16 l1 = __float2bfloat16_rn(v2[1] - __bfloat162float(h1));
+                            hi[e2] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+                                     (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+                            lo[e2] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) |
+                                     (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+                        }
+                        *reinterpret_cast<uint4*>(vt + ktab_off(j, 8 * kg)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                        *reinterpret_cast<uint4*>(vt + ktab_off(L.RP + j, 8 * kg)) =
+                            make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                    }
+                } else {
                 for (int j0 = 0; j0 < L.RP; j0 += 8) {
                     float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
                     bool vdone = false;
@@ -368,6 +430,7 @@ __global__ void __launch_bounds__(kThreads) k4_rank_tc_kernel(const __grid_const
                     *reinterpret_cast<__nv_bfloat16*>(vt + ktab_off(2 * L.RP, rr)) = one;
                     for (int j = 2 * L.RP + 1; j < L.NV; ++j)
                         *reinterpret_cast<__nv_bfloat16*>(vt + ktab_off(j, rr)) = zero;
+                }
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -463,7 +526,11 @@ cudaError_t launch_tc(const void* T, RankTcArgs a, int* status, cudaStream_t s) 
                            static_cast<uint64_t>(a.C) * 2, kTileRows, kBoxCols,
                            CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return cudaErrorInvalidValue;
-    const RtLayout L(Parts{kG, kD, kOnes}, a.r);
+    a.vbulk = (kD && a.nsl == 1 && a.r % 4 == 0 && a.r <= kMaxBulkR &&
+               (reinterpret_cast<uintptr_t>(a.V) & 15) == 0)
+                  ? 1
+                  : 0;
+    const RtLayout L(Parts{kG, kD, kOnes}, a.r, kD && a.vbulk);
     if (L.tmem_cols > 512) return cudaErrorInvalidValue;  // never reached for r <= 64
     const size_t smem = L.total + 1024;
     auto kern = k4_rank_tc_kernel<kG, kD, kOnes>;
