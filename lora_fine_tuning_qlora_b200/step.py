@@ -13,6 +13,12 @@ LoRA notebook, "LoRA equation"):
 five launch groups through the step-level C-ABI calls, so a step can be
 captured into a CUDA graph and replayed.  Optional CUDA events bracket each
 launch group for per-kernel timing.
+
+dX and dA both need only G (and the inputs), so after the dY pass the X pass
+runs on a second stream beside the dX GEMM (an event fork and join, which a
+CUDA graph captures as two branches): its CTAs take the SMs the GEMM leaves
+idle, in the GEMM's last partial wave of tiles or beside a GEMM too small to
+fill the GPU.
 """
 from __future__ import annotations
 
@@ -27,7 +33,7 @@ PARTS = ("quantize_input", "gemm_forward", "lora_grad_dy", "gemm_dx", "lora_grad
 
 
 class LayerStep:
-    def __init__(self, layer: qlora.Layer, M: int, device="cuda"):
+    def __init__(self, layer: qlora.Layer, M: int, device="cuda", overlap_x: Optional[bool] = None):
         dev = torch.device(device)
         self.layer = layer
         self.M = M
@@ -48,19 +54,27 @@ class LayerStep:
         self.dB = self.grad_flat[K * r:K * r + r * N].view(r, N)
         self.dbias = self.grad_flat[K * r + r * N:]
         self.graph: Optional[torch.cuda.CUDAGraph] = None
+        # the X pass's stream and the fork/join events (None: one stream).  By
+        # default from 512 tokens: below that the fork and join cost about as
+        # much as the overlap saves (measured on the configurations' layers)
+        if overlap_x is None:
+            overlap_x = M >= 512
+        self.side = torch.cuda.Stream(device=dev) if overlap_x else None
+        self.fork = torch.cuda.Event() if overlap_x else None
+        self.join = torch.cuda.Event() if overlap_x else None
 
     # ------------------------------------------------------------------
     def run(self, stream=None, events: Optional[Dict[str, Tuple[torch.cuda.Event, torch.cuda.Event]]] = None):
         L, D, M = self.layer, self.desc, self.M
         s = stream if stream is not None else torch.cuda.current_stream()
 
-        def timed(name, fn):
+        def timed(name, fn, st=s):
             ev = events.get(name) if events else None
             if ev:
-                ev[0].record(s)
+                ev[0].record(st)
             fn()
             if ev:
-                ev[1].record(s)
+                ev[1].record(st)
 
         timed("quantize_input",
               lambda: qlora.qlora_quantize_input(D, M, self.X, L.A, self.Xq, self.sx, self.xA, s))
@@ -70,9 +84,20 @@ class LayerStep:
         timed("lora_grad_dy",
               lambda: qlora.qlora_lora_grad_dy(D, M, self.dY, L.B, self.xA, self.dB, self.dbias,
                                                self.ws, None, s))
+        if self.side is None:
+            timed("gemm_dx",
+                  lambda: qlora.qlora_gemm_dx(D, M, self.dY, L.Wq, L.sw, L.A, self.dX, self.ws, s))
+            timed("lora_grad_x", lambda: qlora.qlora_lora_grad_x(D, M, self.X, self.dA, self.ws, s))
+            return
+        # G is final: the X pass on the side stream, the dX GEMM here, then join
+        x = self.side
+        self.fork.record(s)
+        x.wait_event(self.fork)
+        timed("lora_grad_x", lambda: qlora.qlora_lora_grad_x(D, M, self.X, self.dA, self.ws, x), x)
         timed("gemm_dx",
               lambda: qlora.qlora_gemm_dx(D, M, self.dY, L.Wq, L.sw, L.A, self.dX, self.ws, s))
-        timed("lora_grad_x", lambda: qlora.qlora_lora_grad_x(D, M, self.X, self.dA, self.ws, s))
+        self.join.record(x)
+        s.wait_event(self.join)
 
     def make_events(self, parts=PARTS):
         return {p: (torch.cuda.Event(enable_timing=True, external=True),
