@@ -255,6 +255,33 @@ cudaError_t launch_kx(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem
     return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
+// The device's greatest (most urgent) stream priority, looked up once.
+int greatest_priority();
+
+// launch_kx at the device's greatest priority: when kernels of several
+// streams are ready at once, this one's CTAs are placed first.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kx_urgent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                             int cluster_x, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[3];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster_x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    attr[2].id = cudaLaunchAttributePriority;
+    attr[2].val.priority = greatest_priority();
+    cfg.attrs = attr;
+    cfg.numAttrs = 3;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Sets the dynamic shared memory limit of `func` once per device.
 cudaError_t ensure_smem_attr(const void* func, int bytes);
 

@@ -16,8 +16,8 @@
 // quarter of the MMA instructions, with the same de-quantization per flop.
 //
 // Warps per CTA: 0 TMA producer; 1 TMEM owner (pair allocation) and, in
-// CTA 0, the MMA issuer; 2..9 de-quantize (four groups of two); 10..13
-// epilogue.
+// CTA 0, the MMA issuer; 2..11 de-quantize (five groups of two, one per
+// stage of the five-stage ring); 12..15 epilogue.
 // Barriers: full[s] (CTA 0) completes when both CTAs' dY boxes of stage s
 // have landed (the second CTA's box signals it across the pair); wready[s]
 // (CTA 0) takes an arrival from every warp of the de-quantize group that
@@ -42,8 +42,8 @@ namespace {
 constexpr int kPM = 128;             // dX rows per CTA (256 per pair)
 constexpr int kPN = 256;             // dX columns per pair tile (128 de-quantized per CTA)
 constexpr int kPK = 64;              // contraction (n) per stage: one 64-column dY block
-constexpr int kDqW = 8;              // de-quantize warps
-constexpr int kDqGroups = 4;         // stage groups of de-quantize warps (two warps each)
+constexpr int kDqW = 10;             // de-quantize warps
+constexpr int kDqGroups = 5;         // stage groups of de-quantize warps (two warps each)
 constexpr int kDqWPG = kDqW / kDqGroups;
 constexpr int kEpiW = 4;             // epilogue warps: one per TMEM lane quarter
 constexpr int kDqWarp0 = 2;
@@ -61,7 +61,12 @@ struct PairCfg {
     static constexpr int kATabBytes = kPN * (RP + 1) * 4;  // A rows (+ bias) of the tile's 256 columns
     static constexpr int kFixed = kStgBytes + kATabBytes + 512 + 1024;
     static constexpr int kStagesFit = (kPSmemLimit - kFixed) / kStageBytes;
-    static constexpr int STAGES = 4;  // a multiple of the stage groups (more measured no faster)
+    // a multiple of the stage groups.  A group may start stage g only when the
+    // MMAs of stage g - STAGES are done, so the other STAGES - 1 stages'
+    // MMAs are the window its load-convert-store-signal chain must fit in:
+    // five stages with five groups ran 462 us against 484 for four with
+    // four at 16384 x 4096 x 4096; six groups (576 threads) spill
+    static constexpr int STAGES = 5;
     static_assert(kStagesFit >= STAGES, "shared memory budget");
     static constexpr int kStgOff = STAGES * kStageBytes;
     static constexpr int kATabOff = kStgOff + kStgBytes;
@@ -435,7 +440,9 @@ cudaError_t launch_pair_t(const void* dY, const int8_t* Wq, const float* sw, int
         return cudaErrorInvalidValue;
     const int tiles = ((M + 2 * kPM - 1) / (2 * kPM)) * ((K + kPN - 1) / kPN);
     const int pairs = tiles < sm_count() / 2 ? tiles : sm_count() / 2;
-    return launch_kx(kern, dim3(2 * pairs), dim3(kPThreads), C::kTotal, s, 2, tdy, Wq, sw, M, N, K,
+    // at the greatest priority: a rank pass issued beside it on another stream
+    // takes only the SMs its pairs leave (its last partial wave of tiles)
+    return launch_kx_urgent(kern, dim3(2 * pairs), dim3(kPThreads), C::kTotal, s, 2, tdy, Wq, sw, M, N, K,
                      ep, status);
 }
 

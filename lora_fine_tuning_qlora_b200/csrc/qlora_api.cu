@@ -174,6 +174,20 @@ int sm_count() {
     return cache[dev];
 }
 
+int greatest_priority() {
+    static int cache[64];
+    static bool init[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (!init[dev]) {
+        int least = 0, greatest = 0;
+        if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) greatest = 0;
+        cache[dev] = greatest;
+        init[dev] = true;
+    }
+    return cache[dev];
+}
+
 cudaError_t ensure_smem_attr(const void* func, int bytes) {
     // largest dynamic shared memory size set so far, per (device, kernel):
     // some kernels size their shared memory by the rank at run time

@@ -90,12 +90,14 @@ class LayerStep:
             timed("lora_grad_x", lambda: qlora.qlora_lora_grad_x(D, M, self.X, self.dA, self.ws, s))
             return
         # G is final: the X pass on the side stream, the dX GEMM here, then join
+        # (the GEMM is issued first, at the library's greatest priority, so that
+        # its CTAs take the SMs and the X pass runs in what they leave)
         x = self.side
         self.fork.record(s)
-        x.wait_event(self.fork)
-        timed("lora_grad_x", lambda: qlora.qlora_lora_grad_x(D, M, self.X, self.dA, self.ws, x), x)
         timed("gemm_dx",
               lambda: qlora.qlora_gemm_dx(D, M, self.dY, L.Wq, L.sw, L.A, self.dX, self.ws, s))
+        x.wait_event(self.fork)
+        timed("lora_grad_x", lambda: qlora.qlora_lora_grad_x(D, M, self.X, self.dA, self.ws, x), x)
         self.join.record(x)
         s.wait_event(self.join)
 
