@@ -26,10 +26,14 @@
 //
 // W4 (packed int4 codes Wp [N, K/2]): each CTA's TMA brings its stage's
 // packed tile ([128 rows][64 bytes], no swizzle) onto a barrier of its own
-// (pfull), warps 6..9 expand it into the int8 tile the TMA would have written
-// (16-byte chunk c of row n at c ^ (n % 8)) and arrive on CTA 0's wready
-// (CTA-scope release: the tile stays in the writer's shared memory, published
-// to the tensor cores by a proxy fence); the MMA waits for both CTAs' tiles.
+// (pfull), and warps 6..15 expand it into the int8 tile the TMA would have
+// written (16-byte chunk c of row n at c ^ (n % 8)) and arrive on CTA 0's
+// wready (CTA-scope release: the tile stays in the writer's shared memory,
+// published to the tensor cores by a proxy fence); the MMA waits for both
+// CTAs' tiles.  The expansion warps form five groups of two, one per stage of
+// the five-stage ring (group q takes stages q, q + 5, ...), so a group's
+// wait-expand-signal chain has the other stages' MMAs to hide in (all warps
+// on every stage: 278 us at 16384 x 4096 x 4096; the groups: 231).
 #include "internal.h"
 #include "ptx.cuh"
 #include "tile_epilogue.cuh"
@@ -42,7 +46,9 @@ constexpr int kQM = 128;             // rows per CTA (256 per pair)
 constexpr int kQN = 256;             // output columns per pair tile (128 of Wq per CTA)
 constexpr int kQK = 128;             // int8 k per stage: one 128-byte swizzle row
 constexpr int kQEpi = 4;             // epilogue warps
-constexpr int kQUnpack = 4;          // W4: warps that expand the packed codes
+constexpr int kQUGroups = 5;         // W4: stage groups of expansion warps (one per stage of the ring)
+constexpr int kQUWPG = 2;            // W4: warps per stage group
+constexpr int kQUnpack = kQUGroups * kQUWPG;  // W4: warps that expand the packed codes
 template <bool W4>
 __host__ __device__ constexpr int q_threads() { return 32 * (2 + kQEpi + (W4 ? kQUnpack : 0)); }
 constexpr int kQSmemLimit = 232448;
@@ -59,6 +65,7 @@ struct PairFwdCfg {
     static constexpr int kStagesFit = (kQSmemLimit - kFixed) / kStageBytes;
     static constexpr int STAGES = kStagesFit > 6 ? 6 : kStagesFit;
     static_assert(STAGES >= 3, "shared memory budget");
+    static_assert(!W4 || STAGES % kQUGroups == 0, "W4: stages per expansion group");
     static constexpr int kStgOff = STAGES * kStageBytes;
     static constexpr int kTabOff = kStgOff + kStgBytes;
     static constexpr int kBarOff = kTabOff + kTabBytes;
@@ -111,7 +118,7 @@ __global__ void __launch_bounds__(q_threads<W4>(), 1)
         if constexpr (W4)
             for (int s = 0; s < S; ++s) {
                 mbar_init(&pfull[s], 1);
-                mbar_init(&wready[s], 2 * kQUnpack);
+                mbar_init(&wready[s], 2 * kQUWPG);
             }
         fence_mbar_init();
     }
@@ -205,28 +212,33 @@ __global__ void __launch_bounds__(q_threads<W4>(), 1)
         __syncwarp();
     } else if (W4 && warp >= 2 + kQEpi) {
         // ------------------------------------------------------ int4 expand (W4)
-        const int t = threadIdx.x - 32 * (2 + kQEpi);  // 0 .. 127
+        const int ew = warp - (2 + kQEpi);            // 0 .. kQUnpack - 1
+        const int grp = ew / kQUWPG;                   // this warp's stage group
+        const int tg = (ew % kQUWPG) * 32 + lane;      // 0 .. 32 kQUWPG - 1
         const uint32_t wready0 = dsmem_addr(wready, 0);
         int g = 0;
         bool ok = true;
         for (int tt = pair; tt < tiles && ok; tt += npairs) {
             for (int kb = 0; kb < nkb; ++kb, ++g) {
                 const int s = g % S;
+                if (g % kQUGroups != grp) continue;  // another group's stage
                 if (!__all_sync(0xffffffffu, mbar_wait(&pfull[s], (g / S) & 1, status))) {
                     ok = false;
                     break;
                 }
                 uint8_t* wb = smem + s * C::kStageBytes + C::kABytes;
                 const uint8_t* pk = wb + C::kBBytes;
-                uint4 raw[4];
+                // 512 chunks of 32 codes (128 rows x 4) over the group's threads
+                constexpr int kPer = 512 / (32 * kQUWPG);
+                uint4 raw[kPer];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int e = t + u * 128;
+                for (int u = 0; u < kPer; ++u) {
+                    const int e = tg + u * 32 * kQUWPG;
                     raw[u] = *reinterpret_cast<const uint4*>(pk + (e >> 2) * 64 + (e & 3) * 16);
                 }
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int e = t + u * 128;
+                for (int u = 0; u < kPer; ++u) {
+                    const int e = tg + u * 32 * kQUWPG;
                     const int n = e >> 2, p = e & 3;
                     uint4 lo, hi;
                     unpack_int4x32(raw[u], lo, hi);
