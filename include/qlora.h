@@ -134,6 +134,13 @@ int qlora_forward(const qlora_layer_desc* d, int M, const void* X, const int8_t*
  * dequantized kernel Wq * sw is rounded to bf16 before the tensor-core
  * product; accumulation is fp32.  dA, dB and dbias are deterministic
  * (fixed reduction order, no atomics).
+ * Streams: all work is ordered after earlier work on `stream`, and later
+ * work on `stream` is ordered after all of it.  From 512 tokens, with dX
+ * requested, the dA pass runs on a second stream of the library's (one per
+ * host thread and device, created on the first such call; make that call
+ * outside a global-mode stream capture) beside the dX GEMM, joined back to
+ * `stream` by events; stream capture records the two branches.  If the
+ * second stream cannot be created everything runs on `stream`.
  */
 int qlora_backward(const qlora_layer_desc* d, int M, const void* X, const void* dY,
                    const int8_t* Wq, const float* sw, const float* A, const float* B,

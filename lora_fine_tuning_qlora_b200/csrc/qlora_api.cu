@@ -539,6 +539,38 @@ int qlora_forward(const qlora_layer_desc* d, int M, const void* X, const int8_t*
                               stream);
 }
 
+// The backward's second stream: dX and dA both need only G and the inputs,
+// so from kSideStreamMinM tokens the X pass runs on it beside the dX GEMM
+// (an event fork and join, which stream capture records as two branches),
+// taking the SMs the GEMM's last partial wave of tiles leaves.  One stream
+// and two events per host thread and device, created on first use and kept
+// for the thread's life; if they cannot be created (for instance during a
+// global-mode stream capture) the backward stays on the caller's stream.
+namespace {
+constexpr int kSideStreamMinM = 512;
+struct SideStream {
+    bool tried = false;
+    cudaStream_t st = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+SideStream* side_stream() {
+    static thread_local SideStream per_dev[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    SideStream& ss = per_dev[dev];
+    if (!ss.tried) {
+        ss.tried = true;
+        if (cudaStreamCreateWithFlags(&ss.st, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
+            (void)cudaGetLastError();
+            ss.st = nullptr;
+        }
+    }
+    return ss.st ? &ss : nullptr;
+}
+}  // namespace
+
 int qlora_backward(const qlora_layer_desc* d, int M, const void* X, const void* dY,
                    const int8_t* Wq, const float* sw, const float* A, const float* B,
                    const float* xA, void* dX, float* dA, float* dB, float* dbias, void* workspace,
@@ -567,6 +599,27 @@ int qlora_backward(const qlora_layer_desc* d, int M, const void* X, const void* 
     QL_REQUIRE(workspace_bytes >= w.total, QLORA_EINVAL, "workspace too small");
     rc = qlora_lora_grad_dy(d, M, dY, B, xA, dB, dbias, nullptr, workspace, workspace_bytes, stream);
     if (rc != QLORA_OK) return rc;
+    SideStream* ss = (dX && M >= kSideStreamMinM) ? side_stream() : nullptr;
+    if (ss) {
+        // G is final: the dX GEMM here (issued first, at the greatest
+        // priority), the X pass on the second stream, then the join
+        rc = cuda_status(cudaEventRecord(ss->fork, s), "backward fork");
+        if (rc != QLORA_OK) return rc;
+        rc = qlora_gemm_dx(d, M, dY, Wq, sw, A, dX, workspace, workspace_bytes, stream);
+        const int rc_wait = cuda_status(cudaStreamWaitEvent(ss->st, ss->fork, 0), "backward fork");
+        const int rc_x = rc_wait == QLORA_OK
+                             ? qlora_lora_grad_x(d, M, X, dA, workspace, workspace_bytes, ss->st)
+                             : rc_wait;
+        // the join is recorded whatever happened, so the caller's stream never
+        // runs ahead of work issued on the second stream
+        const int rc_join = cuda_status(cudaEventRecord(ss->join, ss->st), "backward join");
+        const int rc_join2 = rc_join == QLORA_OK
+                                 ? cuda_status(cudaStreamWaitEvent(s, ss->join, 0), "backward join")
+                                 : rc_join;
+        if (rc != QLORA_OK) return rc;
+        if (rc_x != QLORA_OK) return rc_x;
+        return rc_join2;
+    }
     if (dX) {
         rc = qlora_gemm_dx(d, M, dY, Wq, sw, A, dX, workspace, workspace_bytes, stream);
         if (rc != QLORA_OK) return rc;

@@ -65,3 +65,30 @@ def test_step_matches_composite_calls(q, M, K, N, r, act):
                            ("dbias", st.dbias, dbias)):
             assert torch.equal(a, b), ("replay", overlap, name)
         assert np.isfinite(st.grad_flat.cpu().numpy()).all()
+
+
+def test_composite_backward_in_a_graph(q):
+    """qlora_backward with its second stream (from 512 tokens) captured into
+    a CUDA graph and replayed gives what the eager call gives."""
+    M, K, N, r, act = 1024, 1024, 1536, 4, torch.bfloat16
+    layer = _layer(q, K, N, r, act, 5)
+    g = torch.Generator(device="cpu").manual_seed(6)
+    X = torch.randn((M, K), generator=g).to(act).cuda()
+    dY = (torch.randn((M, N), generator=g) * 0.01).to(act).cuda()
+    ws = q.workspace(layer.desc(), M, torch.device("cuda"))
+    Y, xA = q.forward(layer, X, ws)
+    ref = q.backward(layer, X, dY, xA, ws)  # eager: also creates the second stream
+    torch.cuda.synchronize()
+    outs = [torch.empty_like(t) for t in ref]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        q.qlora_backward(layer.desc(), M, X, dY, layer.Wq, layer.sw, layer.A, layer.B, xA,
+                         outs[0], outs[1], outs[2], outs[3], ws, s)
+    for t in outs:
+        t.fill_(float("nan"))
+    graph.replay()
+    torch.cuda.synchronize()
+    for name, a, b in zip(("dX", "dA", "dB", "dbias"), outs, ref):
+        assert torch.equal(a, b), name
