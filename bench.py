@@ -355,6 +355,40 @@ def time_graph(replay, steps, warmup, flush, between=None):
     return [a.elapsed_time(b) for a, b in zip(s, e)]
 
 
+def x_pass_alone(st, steps, flush):
+    """Median us of the layer's X pass on its own (one call per replay, L2
+    flushed): inside the step it runs beside the dX GEMM, where its events
+    span the GEMM too.  G is the step's, left in the workspace."""
+    import torch
+    from lora_fine_tuning_qlora_b200 import qlora
+    L, D, M = st.layer, st.desc, st.M
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    fn = lambda: qlora.qlora_lora_grad_x(D, M, st.X, st.dA, st.ws, s)  # noqa: E731
+    with torch.cuda.stream(s):
+        fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        fn()
+    ms = time_graph(g.replay, steps, 1, flush)
+    del g
+    return 1e3 * statistics.median(ms)
+
+
+def overlapped_x(kern, st, steps, flush, M, K, N, r, e, roof):
+    """With the X pass beside the dX GEMM, its entry is its time alone, with
+    the span of its events inside the step beside it."""
+    if st.side is None:
+        return kern
+    span = kern["lora_grad_x"]["us"]
+    kern["lora_grad_x"] = roof.part("lora_grad_x", x_pass_alone(st, steps, flush), M, K, N, r, e)
+    kern["lora_grad_x"].update({"beside": "gemm_dx (second stream)", "span_in_step_us": span,
+                                "timed": "alone, L2 flushed"})
+    return kern
+
+
 def layer_entry(spec, dev, flush, roof, steps, warmup, data=None):
     """Step time and per-launch-group times of one layer workload."""
     import torch
@@ -380,8 +414,8 @@ def layer_entry(spec, dev, flush, roof, steps, warmup, data=None):
     ent = {"workload": spec.name, "M": M, "K": K, "N": N, "r": r, "act": spec.act,
            "step_us": step_us, "tflops": st.flops() / (step_us * 1e-6) / 1e12,
            "t_roof_us": t_roof, "roof_frac": t_roof / step_us,
-           "kernels": {p: roof.part(p, 1e3 * statistics.median(per[p]), M, K, N, r, e)
-                       for p in step_mod.PARTS}}
+           "kernels": overlapped_x({p: roof.part(p, 1e3 * statistics.median(per[p]), M, K, N, r, e)
+                                    for p in step_mod.PARTS}, st, steps, flush, M, K, N, r, e, roof)}
     st.graph = None
     del plain
     return ent, st
@@ -655,7 +689,10 @@ def run_ours(args):
     # ---------------- roofline of the dominant kernel and of the step
     M, K, N, r = spec.M, spec.K, spec.N, spec.r
     kern = {p: roof.part(p, 1e3 * statistics.mean(per[p]), M, K, N, r, 2) for p in step_mod.PARTS}
-    dom = max(kern, key=lambda p: kern[p]["us"])
+    kern = overlapped_x(kern, st, args.steps, flush, M, K, N, r, 2, roof)
+    # the dominant launch group by its own time (the X pass's events, beside
+    # the dX GEMM, are not its duration)
+    dom = max((p for p in kern if "span_in_step_us" not in kern[p]), key=lambda p: kern[p]["us"])
     kd = kern[dom]
     name, bound = PART_KERNELS[dom]
     if bound == "hbm":
