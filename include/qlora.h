@@ -502,6 +502,21 @@ int qlora_fp8_gemm(const uint8_t* A, qlora_fp8_format fmt_a, const uint8_t* B, q
                    int M, int N, int K, const float* scale_a, const float* scale_b, const float* bias,
                    void* C, qlora_dtype c_dtype, void* stream);
 
+/* Bytes of workspace qlora_fp8_gemm_ws uses at this shape on the current
+ * device (0: it would not split; then it is qlora_fp8_gemm). */
+size_t qlora_fp8_gemm_workspace_bytes(int M, int N, int K);
+
+/* qlora_fp8_gemm with a workspace (device memory, 256-byte aligned; NULL or
+ * too small: no split).  On CTA pairs, when the 256 x 256 output tiles leave
+ * the pairs a partial last wave, that wave's tiles are computed as two halves
+ * of the contraction each (one wave of half the length) and a second kernel
+ * adds the halves' fp32 accumulators (in either order the same sum), scales
+ * and adds the bias.  Results are deterministic; their fp32 sums are grouped
+ * differently from qlora_fp8_gemm's on those tiles. */
+int qlora_fp8_gemm_ws(const uint8_t* A, qlora_fp8_format fmt_a, const uint8_t* B, qlora_fp8_format fmt_b,
+                      int M, int N, int K, const float* scale_a, const float* scale_b, const float* bias,
+                      void* C, qlora_dtype c_dtype, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Message for the last non-OK status returned on the calling thread. */
 const char* qlora_last_error(void);
 

@@ -507,12 +507,35 @@ __device__ __forceinline__ void mma_f8_pair(uint32_t d_tmem, uint64_t a_desc, ui
         : "memory");
 }
 
+// The work of pair p: the whole tiles p, p + np, ... below t_full; then, when
+// the last wave of tiles is split (rem > 0), half of the contraction of
+// remainder tile t_full + p / 2 (pairs p < 2 rem), whose raw fp32
+// accumulator goes to part[tile - t_full][half] for fp8_combine_kernel.
+struct PairUnits {
+    int t_full, rem, nkb, p, np;
+    __device__ int whole() const { return p < t_full ? (t_full - 1 - p) / np + 1 : 0; }
+    __device__ int count() const { return whole() + (p < 2 * rem ? 1 : 0); }
+    __device__ void get(int u, int& t, int& kb0, int& kb1, int& half) const {
+        if (u < whole()) {
+            t = p + u * np;
+            kb0 = 0;
+            kb1 = nkb;
+            half = -1;
+        } else {
+            t = t_full + p / 2;
+            half = p % 2;
+            kb0 = half ? nkb / 2 : 0;
+            kb1 = half ? nkb : nkb / 2;
+        }
+    }
+};
+
 template <typename OutT>
 __global__ void __launch_bounds__(kGThreads, 1)
     fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          int M, int N, int K, uint32_t idesc, const float* __restrict__ sa,
                          const float* __restrict__ sb, const float* __restrict__ bias, OutT* __restrict__ C,
-                         int* status) {
+                         int t_full, int rem, float* __restrict__ part, int* status) {
     using P = PCfg<OutT>;
     constexpr int S = P::S;
     extern __shared__ uint8_t smem_raw[];
@@ -530,8 +553,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const int pair = static_cast<int>(blockIdx.x) / 2;
     const int npairs = static_cast<int>(gridDim.x) / 2;
     const int num_nt = (N + kPN - 1) / kPN;
-    const int tiles = ((M + 2 * kPM - 1) / (2 * kPM)) * num_nt;
     const int nkb = (K + kGK - 1) / kGK;
+    const PairUnits U{t_full, rem, nkb, pair, npairs};
+    const int nunits = U.count();
     pdl_trigger();
 
     if (threadIdx.x == 0) {
@@ -566,10 +590,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const uint32_t full0 = dsmem_addr(full, 0);  // CTA 0's full[0]
             int g = 0;
             bool ok = true;
-            for (int t = pair; t < tiles && ok; t += npairs) {
+            for (int u = 0; u < nunits && ok; ++u) {
+                int t, kb0, kb1, half;
+                U.get(u, t, kb0, kb1, half);
                 const int m0 = (t / num_nt) * 2 * kPM + static_cast<int>(rank) * kPM;
                 const int n0 = (t % num_nt) * kPN + static_cast<int>(rank) * (kPN / 2);
-                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                for (int kb = kb0; kb < kb1; ++kb, ++g) {
                     const int s = g % S;
                     if (g >= S && !mbar_wait(&empty[s], ((g / S) - 1) & 1, status)) {
                         ok = false;
@@ -594,13 +620,15 @@ __global__ void __launch_bounds__(kGThreads, 1)
         if (rank == 0 && lane == 0) {
             int g = 0, i = 0;
             bool ok = true;
-            for (int t = pair; t < tiles && ok; t += npairs, ++i) {
+            for (int u = 0; u < nunits && ok; ++u, ++i) {
+                int t, kb0, kb1, half;
+                U.get(u, t, kb0, kb1, half);
                 const int ab = i & 1;
                 const int use = i >> 1;
                 if (use > 0 && !mbar_wait(&tempty[ab], (use - 1) & 1, status)) break;
                 tc_fence_after();
                 const uint32_t dacc = tmem + ab * P::kAccCols;
-                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                for (int kb = kb0; kb < kb1; ++kb, ++g) {
                     const int s = g % S;
                     if (!mbar_wait(&full[s], (g / S) & 1, status)) {
                         ok = false;
@@ -613,7 +641,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     for (int kk = 0; kk < kGK / 32; ++kk) {
                         const uint64_t ad = smem_desc(a_base + kk * 32, 16, 1024, kLayoutSw128);
                         const uint64_t bd = smem_desc(b_base + kk * 32, 16, 1024, kLayoutSw128);
-                        mma_f8_pair(dacc, ad, bd, idesc, (kb != 0 || kk != 0) ? 1u : 0u);
+                        mma_f8_pair(dacc, ad, bd, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
                     }
                     mma_commit_pair(&empty[s], 0x3);
                 }
@@ -631,7 +659,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
         const uint32_t tempty0 = dsmem_addr(tempty, 0);
         const float sab = __fmul_rn(__ldg(sa), __ldg(sb));
         int i = 0;
-        for (int t = pair; t < tiles; t += npairs, ++i) {
+        for (int u = 0; u < nunits; ++u, ++i) {
+            int t, kb0, kb1, half;
+            U.get(u, t, kb0, kb1, half);
             const int ab = i & 1;
             const int use = i >> 1;
             const int m0 = (t / num_nt) * 2 * kPM + static_cast<int>(rank) * kPM;
@@ -648,7 +678,21 @@ __global__ void __launch_bounds__(kGThreads, 1)
             tc_fence_after();
             const int row0 = m0 + q * 32;
             const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * P::kAccCols;
-            if (nkb > 0) {
+            if (half >= 0) {
+                // half of a split tile: the raw accumulator, row-major over the
+                // pair's 256 rows, for fp8_combine_kernel
+                float* dst = part + (static_cast<size_t>(t - t_full) * 2 + half) * (2 * kPM * kPN) +
+                             static_cast<size_t>(static_cast<int>(rank) * kPM + q * 32 + lane) * kPN;
+#pragma unroll 1
+                for (int col = 0; col < kPN; col += kEpiCols) {
+                    uint32_t v[kEpiCols];
+                    tmem_ld16(tbase + col, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < kEpiCols; e += 4)
+                        *reinterpret_cast<uint4*>(dst + col + e) = make_uint4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                }
+            } else if (nkb > 0) {
 #pragma unroll 1
                 for (int col = 0; col < kPN; col += kEpiCols) {
                     uint32_t v[kEpiCols];
@@ -677,6 +721,42 @@ __global__ void __launch_bounds__(kGThreads, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc_pair(tmem, P::kTmemCols);
+    }
+}
+
+// The split tiles: C = (P0 + P1) sa sb + bias over each tile's 256 x 256
+// elements inside the matrix (the sum of the two halves' fp32 accumulators,
+// the same in either order).
+template <typename OutT>
+__global__ void __launch_bounds__(256) fp8_combine_kernel(const float* __restrict__ part, int rem, int t_full,
+                                                         int num_nt, int M, int N, const float* __restrict__ sa,
+                                                         const float* __restrict__ sb,
+                                                         const float* __restrict__ bias, OutT* __restrict__ C) {
+    pdl_trigger();
+    pdl_wait();
+    const float sab = __fmul_rn(__ldg(sa), __ldg(sb));
+    constexpr int kTileElems = 2 * kPM * kPN;
+    const size_t total = static_cast<size_t>(rem) * (kTileElems / 4);
+    for (size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+         idx += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        const size_t e = idx * 4;
+        const int tl = static_cast<int>(e / kTileElems);
+        const int w = static_cast<int>(e % kTileElems);
+        const int row = w / kPN, col = w % kPN;
+        const int t = t_full + tl;
+        const int m = (t / num_nt) * 2 * kPM + row;
+        const int n0 = (t % num_nt) * kPN + col;
+        if (m >= M || n0 >= N) continue;
+        const float4 a = __ldg(reinterpret_cast<const float4*>(part + static_cast<size_t>(tl) * 2 * kTileElems + w));
+        const float4 b =
+            __ldg(reinterpret_cast<const float4*>(part + (static_cast<size_t>(tl) * 2 + 1) * kTileElems + w));
+        const float acc[4] = {a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int n = n0 + j;
+            if (n < N)
+                C[static_cast<size_t>(m) * N + n] = ActIO<OutT>::from_f(fmaf(acc[j], sab, bias ? __ldg(bias + n) : 0.f));
+        }
     }
 }
 }  // namespace
@@ -747,9 +827,26 @@ cudaError_t launch_fp8_quantize(Act act, const void* T, int R, int Cc, const flo
                     scale_in, scale_out, hist, L, fmax);
 }
 
+// Split of the pairs' last wave of tiles: with T pair tiles on np pairs, rem =
+// T mod np tiles left for a partial last wave are computed as two halves of
+// the contraction each (2 rem <= np half-tiles, one wave of half the length)
+// when a workspace holds their partials.  Returns the rem used (0: none).
+static int fp8_split_rem(int M, int N, int K) {
+    const long long tiles =
+        static_cast<long long>((M + 2 * kPM - 1) / (2 * kPM)) * ((N + kPN - 1) / kPN);
+    const int np = sm_count() / 2;
+    if (tiles < np || (K + kGK - 1) / kGK < 2) return 0;
+    const int rem = static_cast<int>(tiles % np);
+    return (rem > 0 && 2 * rem <= np) ? rem : 0;
+}
+
+size_t fp8_gemm_ws_bytes(int M, int N, int K) {
+    return static_cast<size_t>(fp8_split_rem(M, N, K)) * 2 * (2 * kPM * kPN) * sizeof(float);
+}
+
 cudaError_t launch_fp8_gemm(const uint8_t* A, int afmt, const uint8_t* B, int bfmt, int M, int N, int K,
                             const float* sa, const float* sb, const float* bias, void* C, Act out, int* status,
-                            cudaStream_t s) {
+                            cudaStream_t s, void* ws, size_t ws_bytes) {
     CUtensorMap ta, tb;
     if (!make_tmap_2d(&ta, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, K, kGM, kGK, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tmap_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, 128, kGK, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -763,15 +860,34 @@ cudaError_t launch_fp8_gemm(const uint8_t* A, int afmt, const uint8_t* B, int bf
         // CTA pairs, persistent: one pair per two SMs; tb holds 128-row boxes of B
         const int pairs = pair_tiles < sm_count() / 2 ? pair_tiles : sm_count() / 2;
         const uint32_t idp = idesc_f8(2 * kPM, kPN, afmt, bfmt);
+        // the last wave split in halves where a workspace holds the partials
+        const size_t need = fp8_gemm_ws_bytes(M, N, K);
+        const int rem = (need > 0 && ws && ws_bytes >= need) ? fp8_split_rem(M, N, K) : 0;
+        const int t_full = rem ? pair_tiles - rem : pair_tiles;
+        float* part = rem ? static_cast<float*>(ws) : nullptr;
         auto runp = [&](auto kern, int total) -> cudaError_t {
             cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), total);
             if (e != cudaSuccess) return e;
             return launch_kx(kern, dim3(2 * pairs), dim3(kGThreads), static_cast<size_t>(total), s, 2, ta, tb, M,
-                             N, K, idp, sa, sb, bias, C, status);
+                             N, K, idp, sa, sb, bias, C, t_full, rem, part, status);
         };
-        if (out == kBF16)
-            return runp(fp8_gemm_pair_kernel<__nv_bfloat16>, PCfg<__nv_bfloat16>::kTotal);
-        return runp(fp8_gemm_pair_kernel<float>, PCfg<float>::kTotal);
+        const int num_nt = (N + kPN - 1) / kPN;
+        const int cgrid = rem * (2 * kPM * kPN / 4) / 256;
+        cudaError_t e;
+        if (out == kBF16) {
+            e = runp(fp8_gemm_pair_kernel<__nv_bfloat16>, PCfg<__nv_bfloat16>::kTotal);
+            if (e == cudaSuccess && rem)
+                e = launch_k(fp8_combine_kernel<__nv_bfloat16>, dim3(cgrid), dim3(256), 0, s, 1,
+                             static_cast<const float*>(part), rem, t_full, num_nt, M, N, sa, sb, bias,
+                             static_cast<__nv_bfloat16*>(C));
+        } else {
+            e = runp(fp8_gemm_pair_kernel<float>, PCfg<float>::kTotal);
+            if (e == cudaSuccess && rem)
+                e = launch_k(fp8_combine_kernel<float>, dim3(cgrid), dim3(256), 0, s, 1,
+                             static_cast<const float*>(part), rem, t_full, num_nt, M, N, sa, sb, bias,
+                             static_cast<float*>(C));
+        }
+        return e;
     }
     const uint32_t id = idesc_f8(kGM, bn, afmt, bfmt);
     const dim3 grid((N + bn - 1) / bn, (M + kGM - 1) / kGM);

@@ -135,7 +135,10 @@ size_t fp8_colsum_ws_bytes(int R, int Cc);
 // C [M,N] = (A [M,K] B [N,K]^T) * sa * sb (+ bias [N]); K-major fp8 codes.
 cudaError_t launch_fp8_gemm(const uint8_t* A, int afmt, const uint8_t* B, int bfmt, int M, int N, int K,
                             const float* sa, const float* sb, const float* bias, void* C, Act out, int* status,
-                            cudaStream_t s);
+                            cudaStream_t s, void* ws = nullptr, size_t ws_bytes = 0);
+// Workspace bytes that let launch_fp8_gemm split the CTA pairs' partial last
+// wave of tiles (0: no split at this shape on this device).
+size_t fp8_gemm_ws_bytes(int M, int N, int K);
 
 // ---------------------------------------------------------------- K4
 // The dY pass runs on the tensor cores for bf16 activations whose rows TMA

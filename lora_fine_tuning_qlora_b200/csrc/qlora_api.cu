@@ -929,9 +929,9 @@ int qlora_fp8_quantize_colsum(const void* T, int rows, int cols, qlora_dtype dty
                        "float8 quantizer launch");
 }
 
-int qlora_fp8_gemm(const uint8_t* A, qlora_fp8_format fmt_a, const uint8_t* B, qlora_fp8_format fmt_b,
-                   int M, int N, int K, const float* scale_a, const float* scale_b, const float* bias,
-                   void* C, qlora_dtype c_dtype, void* stream) {
+static int fp8_gemm_impl(const uint8_t* A, qlora_fp8_format fmt_a, const uint8_t* B, qlora_fp8_format fmt_b,
+                         int M, int N, int K, const float* scale_a, const float* scale_b, const float* bias,
+                         void* C, qlora_dtype c_dtype, void* workspace, size_t workspace_bytes, void* stream) {
     QL_REQUIRE(A && B && scale_a && scale_b && C, QLORA_EINVAL, "NULL pointer argument");
     QL_REQUIRE(M >= 1 && N >= 1 && K >= 1, QLORA_ESHAPE, "M, N and K must be >= 1");
     QL_REQUIRE(K % 16 == 0, QLORA_EUNSUPPORTED, "K must be a multiple of 16 (16-byte rows of codes)");
@@ -943,13 +943,32 @@ int qlora_fp8_gemm(const uint8_t* A, qlora_fp8_format fmt_a, const uint8_t* B, q
                "A, B and C must be 16-byte aligned");
     QL_REQUIRE(aligned(scale_a, 4) && aligned(scale_b, 4) && (!bias || aligned(bias, 4)), QLORA_EALIGN,
                "fp32 vectors must be 4-byte aligned");
+    QL_REQUIRE(!workspace || aligned(workspace, 256), QLORA_EALIGN, "workspace must be 256-byte aligned");
     int* status = status_ptr();
     QL_REQUIRE(status, QLORA_ECUDA, "no CUDA device");
     return cuda_status(launch_fp8_gemm(A, fmt_a == QLORA_FP8_E4M3 ? kFp8E4M3 : kFp8E5M2, B,
                                        fmt_b == QLORA_FP8_E4M3 ? kFp8E4M3 : kFp8E5M2, M, N, K, scale_a,
                                        scale_b, bias, C, c_dtype == QLORA_BF16 ? kBF16 : kF32, status,
-                                       static_cast<cudaStream_t>(stream)),
+                                       static_cast<cudaStream_t>(stream), workspace, workspace_bytes),
                        "float8 GEMM launch");
+}
+
+int qlora_fp8_gemm(const uint8_t* A, qlora_fp8_format fmt_a, const uint8_t* B, qlora_fp8_format fmt_b,
+                   int M, int N, int K, const float* scale_a, const float* scale_b, const float* bias,
+                   void* C, qlora_dtype c_dtype, void* stream) {
+    return fp8_gemm_impl(A, fmt_a, B, fmt_b, M, N, K, scale_a, scale_b, bias, C, c_dtype, nullptr, 0, stream);
+}
+
+size_t qlora_fp8_gemm_workspace_bytes(int M, int N, int K) {
+    if (M < 1 || N < 1 || K < 1) return 0;
+    return fp8_gemm_ws_bytes(M, N, K);
+}
+
+int qlora_fp8_gemm_ws(const uint8_t* A, qlora_fp8_format fmt_a, const uint8_t* B, qlora_fp8_format fmt_b,
+                      int M, int N, int K, const float* scale_a, const float* scale_b, const float* bias,
+                      void* C, qlora_dtype c_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+    return fp8_gemm_impl(A, fmt_a, B, fmt_b, M, N, K, scale_a, scale_b, bias, C, c_dtype, workspace,
+                         workspace_bytes, stream);
 }
 
 int qlora_selftest_wait_timeout(unsigned int limit_us, void* stream) {

@@ -3,8 +3,8 @@ Keras PR 19488): the input and the kernel quantized to E4M3 and the output
 gradient to E5M2 with per-tensor delayed scaling (a scale and an amax
 history per tensor, updated every step), the three GEMMs of a training step
 on float8 tensor cores.  The arithmetic runs in the library
-(qlora_fp8_quantize, qlora_fp8_gemm, qlora_lora_grad_b for the bias
-gradient); this module only holds the state and orders the calls.
+(qlora_fp8_quantize[_colsum], qlora_fp8_gemm_ws, qlora_lora_grad_b for the
+bias gradient where the quantizer cannot take it); this module only holds the state and orders the calls.
 
 State per tensor: two device scales used in turn (a step quantizes with
 one and writes the next into the other) and an amax history of
@@ -67,8 +67,16 @@ class Float8Dense:
         self.sx = Fp8State(history_len, dev)
         self.sw = Fp8State(history_len, dev)
         self.sg = Fp8State(history_len, dev)
+        self.gemm_ws = None  # the GEMMs' workspace (a split last wave of tiles), grown on demand
         self.Wq = torch.empty((self.K, self.N), dtype=torch.uint8, device=dev)   # for dX
         self.WqT = torch.empty((self.N, self.K), dtype=torch.uint8, device=dev)  # for Y
+
+    def _gemm(self, A, fa, B, fb, sa, sb, bias, C):
+        M, K = A.shape
+        need = qlora.qlora_fp8_gemm_workspace_bytes(M, B.shape[0], K)
+        if need and (self.gemm_ws is None or self.gemm_ws.numel() < need):
+            self.gemm_ws = torch.empty(need, dtype=torch.uint8, device=A.device)
+        qlora.qlora_fp8_gemm_ws(A, fa, B, fb, sa, sb, bias, C, self.gemm_ws if need else None)
 
     def forward(self, X: torch.Tensor) -> (torch.Tensor, Dict[str, torch.Tensor]):
         M = X.shape[0]
@@ -78,7 +86,7 @@ class Float8Dense:
         s_x = self.sx.quantize(X, qlora.FP8_E4M3, Xq, XqT)
         s_w = self.sw.quantize(self.W, qlora.FP8_E4M3, self.Wq, self.WqT)
         Y = torch.empty((M, self.N), dtype=self.act, device=dev)
-        qlora.qlora_fp8_gemm(Xq, qlora.FP8_E4M3, self.WqT, qlora.FP8_E4M3, s_x, s_w, self.bias, Y)
+        self._gemm(Xq, qlora.FP8_E4M3, self.WqT, qlora.FP8_E4M3, s_x, s_w, self.bias, Y)
         return Y, {"Xq": Xq, "XqT": XqT, "s_x": s_x, "s_w": s_w}
 
     def backward(self, ctx: Dict[str, torch.Tensor], dY: torch.Tensor, want_dx: bool = True):
@@ -95,10 +103,10 @@ class Float8Dense:
         out = {"Gq": Gq, "s_g": s_g}
         if want_dx:
             dX = torch.empty((M, self.K), dtype=self.act, device=dev)
-            qlora.qlora_fp8_gemm(Gq, qlora.FP8_E5M2, self.Wq, qlora.FP8_E4M3, s_g, ctx["s_w"], None, dX)
+            self._gemm(Gq, qlora.FP8_E5M2, self.Wq, qlora.FP8_E4M3, s_g, ctx["s_w"], None, dX)
             out["dX"] = dX
         dW = torch.empty((self.K, self.N), dtype=torch.float32, device=dev)
-        qlora.qlora_fp8_gemm(ctx["XqT"], qlora.FP8_E4M3, GqT, qlora.FP8_E5M2, ctx["s_x"], s_g, None, dW)
+        self._gemm(ctx["XqT"], qlora.FP8_E4M3, GqT, qlora.FP8_E5M2, ctx["s_x"], s_g, None, dW)
         out["dW"] = dW
         if fused:
             out["dbias"] = dbias

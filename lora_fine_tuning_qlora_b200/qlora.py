@@ -37,7 +37,7 @@ EXPORTED = ("qlora_quantize_weight", "qlora_workspace_bytes", "qlora_forward",
             "qlora_outlier_cap", "qlora_outlier_workspace_bytes", "qlora_outlier_quantize",
             "qlora_outlier_forward", "qlora_outlier_backward", "qlora_permute",
             "qlora_fp8_quantize", "qlora_fp8_gemm", "qlora_fp8_colsum_workspace_bytes",
-            "qlora_fp8_quantize_colsum")
+            "qlora_fp8_quantize_colsum", "qlora_fp8_gemm_workspace_bytes", "qlora_fp8_gemm_ws")
 
 
 class QLoraError(RuntimeError):
@@ -133,6 +133,10 @@ def _load():
     lib.qlora_fp8_quantize_colsum.argtypes = [P, I, I, I, I, P, P, P, I, P, P, P, P, Z, P]
     lib.qlora_fp8_quantize_colsum.restype = I
     lib.qlora_fp8_gemm.argtypes = [P, I, P, I, I, I, I, P, P, P, P, I, P]
+    lib.qlora_fp8_gemm_workspace_bytes.argtypes = [I, I, I]
+    lib.qlora_fp8_gemm_workspace_bytes.restype = Z
+    lib.qlora_fp8_gemm_ws.argtypes = [P, I, P, I, I, I, I, P, P, P, P, I, P, Z, P]
+    lib.qlora_fp8_gemm_ws.restype = I
     lib.qlora_fp8_gemm.restype = I
     lib.qlora_permute.argtypes = [P, P, I, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int), I, P]
     lib.qlora_permute.restype = I
@@ -474,6 +478,21 @@ def qlora_fp8_quantize_colsum(T: torch.Tensor, fmt: int, scale_in, scale_out, hi
     _check(_lib.qlora_fp8_quantize_colsum(_ptr(T), rows, cols, act_code(T.dtype), int(fmt), _ptr(scale_in),
                                           _ptr(scale_out), _ptr(history), history.numel(), _ptr(q), _ptr(qt),
                                           _ptr(colsum), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def qlora_fp8_gemm_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(_lib.qlora_fp8_gemm_workspace_bytes(int(M), int(N), int(K)))
+
+
+def qlora_fp8_gemm_ws(A, fmt_a: int, B, fmt_b: int, scale_a, scale_b, bias, C, ws, stream=None):
+    """qlora_fp8_gemm with a workspace for splitting a partial last wave of
+    CTA-pair tiles (ws may be None: no split)."""
+    M, K = A.shape
+    N = B.shape[0]
+    assert B.shape[1] == K and tuple(C.shape) == (M, N)
+    _check(_lib.qlora_fp8_gemm_ws(_ptr(A), int(fmt_a), _ptr(B), int(fmt_b), M, N, K, _ptr(scale_a),
+                                  _ptr(scale_b), _ptr(bias), _ptr(C), act_code(C.dtype), _ptr(ws),
+                                  ws.numel() if ws is not None else 0, _stream(stream)))
 
 
 def qlora_fp8_gemm(A, fmt_a: int, B, fmt_b: int, scale_a, scale_b, bias, C, stream=None):

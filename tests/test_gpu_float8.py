@@ -115,6 +115,7 @@ def test_zero_history_keeps_the_scale(q):
     assert float(s_out[0]) == 0.5 and float(h.abs().max()) == 0.0 and int(qq.max()) == 0
 
 
+@pytest.mark.parametrize("ws", [False, True])
 @pytest.mark.parametrize("M,N,K,fa,fb,out", [
     (128, 128, 128, f8.E4M3, f8.E4M3, torch.bfloat16),
     (300, 520, 784, f8.E4M3, f8.E4M3, torch.bfloat16),   # ragged tiles and k-block
@@ -128,7 +129,10 @@ def test_zero_history_keeps_the_scale(q):
     # stage ring wrap
     (4096, 4096, 256, f8.E4M3, f8.E5M2, torch.float32),
 ])
-def test_fp8_gemm(q, M, N, K, fa, fb, out):
+def test_fp8_gemm(q, M, N, K, fa, fb, out, ws):
+    """With ws, shapes that leave the CTA pairs a partial last wave (81 and
+    256 tiles on 74 pairs) take the split of that wave: both halves'
+    accumulators added by the second kernel."""
     rng = np.random.Generator(np.random.PCG64(M * N + K))
     A = rng.integers(0, 256, (M, K), dtype=np.uint8)
     B = rng.integers(0, 256, (N, K), dtype=np.uint8)
@@ -138,10 +142,16 @@ def test_fp8_gemm(q, M, N, K, fa, fb, out):
         X[bad] = 0x01
     sa, sb = np.float32(0.03125), np.float32(1.5)
     bias = rng.normal(0, 0.1, N).astype(np.float32)
-    C = torch.empty((M, N), dtype=out, device="cuda")
-    q.qlora_fp8_gemm(torch.from_numpy(A).cuda(), _fmt(q, fa), torch.from_numpy(B).cuda(), _fmt(q, fb),
-                     torch.tensor([sa], device="cuda"), torch.tensor([sb], device="cuda"),
-                     torch.from_numpy(bias).cuda(), C)
+    C = torch.full((M, N), float("nan"), dtype=out, device="cuda")
+    args = (torch.from_numpy(A).cuda(), _fmt(q, fa), torch.from_numpy(B).cuda(), _fmt(q, fb),
+            torch.tensor([sa], device="cuda"), torch.tensor([sb], device="cuda"),
+            torch.from_numpy(bias).cuda(), C)
+    if ws:
+        need = q.qlora_fp8_gemm_workspace_bytes(M, N, K)
+        w = torch.empty(max(need, 256), dtype=torch.uint8, device="cuda")
+        q.qlora_fp8_gemm_ws(*args, w)
+    else:
+        q.qlora_fp8_gemm(*args)
     torch.cuda.synchronize()
     da, db = f8.decode(A, fa), f8.decode(B, fb)
     sab = np.float64(sa) * np.float64(sb)
