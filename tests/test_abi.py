@@ -175,6 +175,15 @@ def test_new_entry_points_reject_bad_arguments(q):
                                    ctypes.c_int, P, P, P, P, ctypes.c_int, P]
     assert lib.qlora_fp8_gemm(fake, 0, fake, 0, 16, 16, 24, fake, fake, None, fake, 1, None) == -5
     assert lib.qlora_fp8_gemm(fake, 7, fake, 0, 16, 16, 32, fake, fake, None, fake, 1, None) == -1
+    # the workspace variant: a misaligned workspace, and the same shape checks
+    lib.qlora_fp8_gemm_ws.argtypes = [P, ctypes.c_int, P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_int, P, P, P, P, ctypes.c_int, P, ctypes.c_size_t, P]
+    assert lib.qlora_fp8_gemm_ws(fake, 0, fake, 0, 16, 16, 32, fake, fake, None, fake, 1, P(0x10010), 4096,
+                                 None) == -2
+    assert lib.qlora_fp8_gemm_ws(fake, 0, fake, 0, 16, 16, 24, fake, fake, None, fake, 1, None, 0, None) == -5
+    # no split below one wave of pair tiles; a split where the last wave is partial
+    assert q.qlora_fp8_gemm_workspace_bytes(256, 256, 1024) == 0
+    assert q.qlora_fp8_gemm_workspace_bytes(0, 256, 1024) == 0
     # float8 quantizer: the next scale must not overwrite the one in use
     lib.qlora_fp8_quantize.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P,
                                        ctypes.c_int, P, P, P, ctypes.c_size_t, P]
