@@ -504,19 +504,31 @@ __device__ __forceinline__ void bf16x8_to_f(const uint4 u, float (&f)[8]) {
     }
 }
 
-// Symmetric abs-max codes of 8 values: rne(fl(v * inv)).  The product is
-// rounded to fp32 (__fmul_rn, never contracted into a fused multiply-add),
-// then 1.5 * 2^23 is added (__fadd_rn): for |p| < 2^22 the sum rounds p to the
-// nearest integer, ties to even, and its low byte is the two's-complement
-// code.  |fl(v * inv)| <= 127 * (1 + 2^-24)^2 < 127.5, so no clamp is reached.
-// Both steps run on the FMA pipe (a float-to-int conversion would use the
-// narrow conversion pipe for every element).
+// Symmetric abs-max codes of 8 values: rne(fl(v * inv)).  The products are
+// rounded to fp32 lane by lane (mul.rn.f32x2: two per instruction, never
+// contracted), converted with round-to-nearest-even (cvt.rni.s32.f32, on the
+// conversion pipe beside the FMA pipe) and packed four to a word with
+// saturation (cvt.pack.sat.s8.s32: |fl(v * inv)| <= 127 * (1 + 2^-24)^2 <
+// 127.5, so saturation is never reached).  Against an fp32 multiply, a
+// 1.5 * 2^23 add and byte permutes on the FMA pipe this ran 72 against 76 us
+// at 16384 x 4096 with the same codes.
 __device__ __forceinline__ uint2 codes8(const float (&f)[8], float inv) {
-    uint32_t b[8];
+    const unsigned long long inv2 = pk2(inv, inv);
+    int c[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) b[i] = __float_as_uint(__fadd_rn(__fmul_rn(f[i], inv), 12582912.0f));
-    const uint32_t w0 = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
-    const uint32_t w1 = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
+    for (int p = 0; p < 4; ++p) {
+        unsigned long long prod;
+        asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(prod) : "l"(pk2(f[2 * p], f[2 * p + 1])), "l"(inv2));
+        float a, b;
+        unpk2(prod, a, b);
+        asm("cvt.rni.s32.f32 %0, %1;" : "=r"(c[2 * p]) : "f"(a));
+        asm("cvt.rni.s32.f32 %0, %1;" : "=r"(c[2 * p + 1]) : "f"(b));
+    }
+    uint32_t t0, w0, t1, w1;
+    asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(t0) : "r"(c[3]), "r"(c[2]), "r"(0));
+    asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(w0) : "r"(c[1]), "r"(c[0]), "r"(t0));
+    asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(t1) : "r"(c[7]), "r"(c[6]), "r"(0));
+    asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(w1) : "r"(c[5]), "r"(c[4]), "r"(t1));
     return make_uint2(w0, w1);
 }
 
