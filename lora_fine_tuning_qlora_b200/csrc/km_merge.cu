@@ -111,17 +111,15 @@ __global__ void __launch_bounds__(kThreads) km_merge_kernel(const uint8_t* __res
 constexpr int kNB = 8;
 constexpr int kKStep = kThreads * 16;
 
-// 16 int8 codes (k order) -> exact floats, by placing each code (offset by
-// 128) in the low mantissa byte of 2^23 and subtracting 2^23 + 128
-__device__ __forceinline__ void codes_to_f(const uint4 raw, float (&f)[16]) {
-    const uint32_t w[4] = {raw.x ^ 0x80808080u, raw.y ^ 0x80808080u, raw.z ^ 0x80808080u,
-                           raw.w ^ 0x80808080u};
+// codes 8h .. 8h + 7 of a 16-code chunk (k order) -> exact floats, by
+// placing each code (offset by 128) in the low mantissa byte of 2^23 and
+// subtracting 2^23 + 128
+__device__ __forceinline__ void codes_to_f8(const uint4 raw, int h, float (&f)[8]) {
+    const uint32_t w0 = (h ? raw.z : raw.x) ^ 0x80808080u, w1 = (h ? raw.w : raw.y) ^ 0x80808080u;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        f[4 * i + 0] = __fsub_rn(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7540)), 8388736.0f);
-        f[4 * i + 1] = __fsub_rn(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7541)), 8388736.0f);
-        f[4 * i + 2] = __fsub_rn(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7542)), 8388736.0f);
-        f[4 * i + 3] = __fsub_rn(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7543)), 8388736.0f);
+        f[i] = __fsub_rn(__uint_as_float(__byte_perm(w0, 0x4B000000u, 0x7540 + i)), 8388736.0f);
+        f[4 + i] = __fsub_rn(__uint_as_float(__byte_perm(w1, 0x4B000000u, 0x7540 + i)), 8388736.0f);
     }
 }
 
@@ -138,6 +136,7 @@ __global__ void __launch_bounds__(kThreads, RP <= 4 ? 2 : 1) km_merge_tiled_kern
     __shared__ float sS[kNB];
     __shared__ float red[kThreads / 32][kNB];
     __shared__ float s_amax[kNB];
+    __shared__ float s_inv[kNB];  // kLevels / amax (0 for a zero channel)
     pdl_trigger();
     pdl_wait();
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -199,9 +198,9 @@ __global__ void __launch_bounds__(kThreads, RP <= 4 ? 2 : 1) km_merge_tiled_kern
             load_a(k0 + 8 * h, a);
 #pragma unroll
             for (int nb = 0; nb < kNB; ++nb) {
-                float q[16], wp[8];
-                codes_to_f(raw[nb], q);
-                merged8(q + 8 * h, nb, a, wp);
+                float q[8], wp[8];
+                codes_to_f8(raw[nb], h, q);
+                merged8(q, nb, a, wp);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) amax[nb] = fmaxf(amax[nb], fabsf(wp[e]));
             }
@@ -217,6 +216,7 @@ __global__ void __launch_bounds__(kThreads, RP <= 4 ? 2 : 1) km_merge_tiled_kern
 #pragma unroll
         for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[w][t]);
         s_amax[t] = m;
+        s_inv[t] = m > 0.f ? __fdiv_rn(kLevels, m) : 0.f;
         if (n0 + t < N) sw_out[n0 + t] = __fdiv_rn(m, kLevels);
     }
     __syncthreads();
@@ -236,11 +236,10 @@ __global__ void __launch_bounds__(kThreads, RP <= 4 ? 2 : 1) km_merge_tiled_kern
             for (int nb = 0; nb < kNB; ++nb) {
                 const int n = n0 + nb;
                 if (n >= N) break;
-                float q[16], wp[8];
-                codes_to_f(raw[nb], q);
-                merged8(q + 8 * h, nb, a, wp);
-                const float m = s_amax[nb];
-                const float inv = m > 0.f ? __fdiv_rn(kLevels, m) : 0.f;
+                float q[8], wp[8];
+                codes_to_f8(raw[nb], h, q);
+                merged8(q, nb, a, wp);
+                const float inv = s_inv[nb];
                 uint8_t* orow = Wq_out + static_cast<size_t>(n) * row_bytes;
                 if constexpr (W4) {
                     uint32_t v = 0u;
