@@ -451,10 +451,12 @@ cudaError_t launch_pair_t(const void* dY, const int8_t* Wq, const float* sw, int
 bool gemm_dx_pair_applies(int M, int N, int K, int r) {
     if (N % kPK != 0 || K % 16 != 0 || r > 16) return false;
     const int tiles = ((M + 2 * kPM - 1) / (2 * kPM)) * ((K + kPN - 1) / kPN);
-    // from three quarters of a wave of pairs: at 1024 tokens of the 4096^2
-    // layer (64 pair tiles) the pairs ran 48.5 us against 58.7 for the
-    // single-CTA kernel's 1.7 waves of 128 x 128 tiles
-    return tiles >= sm_count() * 3 / 8;
+    // from half a wave of pairs: at 1024 tokens of the 4096^2 layer (64 pair
+    // tiles) the pairs ran 48.5 us against 58.7 for the single-CTA kernel's
+    // 1.7 waves of 128 x 128 tiles, and on the GPT-2 projections (48 tiles)
+    // 34 against 38 us (qkv), 40 against 47 (mlp up), the outlier-compensated
+    // layers' steps 4-11 us faster
+    return tiles >= sm_count() / 4;
 }
 
 template <int MODE>
