@@ -33,6 +33,7 @@ def _layer(q, K, N, r, act, seed):
     (16, 4096, 4096, 4, torch.bfloat16),    # few tokens: the GEMMs leave most SMs to the X pass
     (2304, 1024, 2048, 8, torch.bfloat16),  # CTA-pair GEMMs with a partial last wave
     (300, 784, 520, 4, torch.float32),      # fp32 activations, ragged tiles
+    (640, 256, 384, 4, torch.float32),      # fp32 with the second stream (from 512 tokens)
 ])
 def test_step_matches_composite_calls(q, M, K, N, r, act):
     from lora_fine_tuning_qlora_b200 import step
