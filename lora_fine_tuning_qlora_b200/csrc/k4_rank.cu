@@ -338,6 +338,38 @@ __global__ void k4_g_reduce_kernel(const float* __restrict__ Gp, int ncb, size_t
         G[i] = sum_slices(Gp + i, n, ncb);
 }
 
+// The same sums, four consecutive elements a thread (n % 4 == 0, 16-byte
+// aligned slices) with sixteen slices' 16-byte loads in flight; each
+// element's slices are still added in ascending order, so G is bit-identical.
+__global__ void k4_g_reduce4_kernel(const float4* __restrict__ Gp, int ncb, size_t n4,
+                                    float4* __restrict__ G) {
+    pdl_trigger();
+    pdl_wait();
+    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int b0 = 0; b0 < ncb; b0 += 16) {
+            float4 v[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+                if (b0 + u < ncb) v[u] = __ldg(Gp + static_cast<size_t>(b0 + u) * n4 + i);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                if (b0 + u >= ncb) break;
+                if (b0 + u == 0) {
+                    acc = v[u];
+                } else {
+                    acc.x += v[u].x;
+                    acc.y += v[u].y;
+                    acc.z += v[u].z;
+                    acc.w += v[u].w;
+                }
+            }
+        }
+        G[i] = acc;
+    }
+}
+
 // Cluster size along the rows.  The dY pass runs one CTA per SM (its
 // accumulators fill the register file), so it takes clusters of at most 4:
 // clusters of 8 such CTAs do not all fit in one wave of the GPCs.
@@ -378,6 +410,12 @@ cudaError_t launch_rank_dy(Act act, const void* dY, const float* B, const float*
 
 cudaError_t launch_g_reduce(const float* Gp, int ncb, int M, int r, float* G, cudaStream_t s) {
     const size_t n = static_cast<size_t>(M) * r;
+    if (n % 4 == 0 && (reinterpret_cast<uintptr_t>(Gp) & 15) == 0 && (reinterpret_cast<uintptr_t>(G) & 15) == 0) {
+        const size_t n4 = n / 4;
+        const int blocks = static_cast<int>((n4 + 127) / 128 < 2048 ? (n4 + 127) / 128 : 2048);
+        return launch_k(k4_g_reduce4_kernel, dim3(blocks < 1 ? 1 : blocks), dim3(128), 0, s, 1,
+                        reinterpret_cast<const float4*>(Gp), ncb, n4, reinterpret_cast<float4*>(G));
+    }
     const int blocks = static_cast<int>((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
     return launch_k(k4_g_reduce_kernel, dim3(blocks < 1 ? 1 : blocks), dim3(256), 0, s, 1, Gp, ncb,
                     n, G);
