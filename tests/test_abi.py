@@ -184,6 +184,13 @@ def test_new_entry_points_reject_bad_arguments(q):
     # no split below one wave of pair tiles; a split where the last wave is partial
     assert q.qlora_fp8_gemm_workspace_bytes(256, 256, 1024) == 0
     assert q.qlora_fp8_gemm_workspace_bytes(0, 256, 1024) == 0
+    # 4096 x 4096 outputs: 256 pair tiles on 74 pairs (148 SMs) leave 34 for a
+    # partial last wave, split in halves: 34 tiles x 2 halves x 256 x 256 fp32
+    assert q.qlora_fp8_gemm_workspace_bytes(4096, 4096, 16384) == 34 * 2 * 256 * 256 * 4
+    # 16384 x 4096: 1024 tiles leave 62, too many to split in one wave of halves
+    assert q.qlora_fp8_gemm_workspace_bytes(16384, 4096, 4096) == 0
+    # a single 128-deep k-block cannot be split
+    assert q.qlora_fp8_gemm_workspace_bytes(4096, 4096, 128) == 0
     # float8 quantizer: the next scale must not overwrite the one in use
     lib.qlora_fp8_quantize.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P,
                                        ctypes.c_int, P, P, P, ctypes.c_size_t, P]
