@@ -162,30 +162,33 @@ std::atomic<int> g_rank_pass_rows{0};
 int rank_pass_rows() { return g_rank_pass_rows.load(std::memory_order_relaxed); }
 
 int sm_count() {
-    static int cache[64] = {0};
+    // per device, looked up once (0: not yet); racing first lookups store the same value
+    static std::atomic<int> cache[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (cache[dev] == 0) {
-        int v = 0;
+    int v = cache[dev].load(std::memory_order_relaxed);
+    if (v == 0) {
         if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
             v = 148;
-        cache[dev] = v;
+        cache[dev].store(v, std::memory_order_relaxed);
     }
-    return cache[dev];
+    return v;
 }
 
 int greatest_priority() {
-    static int cache[64];
-    static bool init[64] = {false};
+    // per device, looked up once; threads that race on the first lookup
+    // store the same value
+    static std::atomic<int> cache[64] = {};
+    static std::atomic<bool> init[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    if (!init[dev]) {
+    if (!init[dev].load(std::memory_order_acquire)) {
         int least = 0, greatest = 0;
         if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) greatest = 0;
-        cache[dev] = greatest;
-        init[dev] = true;
+        cache[dev].store(greatest, std::memory_order_relaxed);
+        init[dev].store(true, std::memory_order_release);
     }
-    return cache[dev];
+    return cache[dev].load(std::memory_order_relaxed);
 }
 
 cudaError_t ensure_smem_attr(const void* func, int bytes) {
